@@ -1,0 +1,171 @@
+/*
+ * tq.h -- C ABI of the B200 (sm_100a) TurboQuant KV-cache library.
+ *
+ * TurboQuant stores each key/value head-vector x (dimension d) as its L2 norm,
+ * the per-coordinate codes of the randomly rotated unit vector under a
+ * Lloyd-Max scalar quantizer fitted to the Beta-shaped coordinate law, and,
+ * for keys, a 1-bit Johnson-Lindenstrauss sketch of the residual plus the
+ * residual norm. Attention logits and softmax-weighted values are computed
+ * directly on that packed cache.
+ *   - zubnet.ai news, "Google's TurboQuant quantizes LLM KV cache to 3.5 bits
+ *     per channel", paragraph 2 (two-stage pipeline; storage = indices, sign
+ *     bits, one L2-norm scalar);
+ *   - winningdata.io, "TurboQuant: Google comprime KV cache para 3 bits sem
+ *     perder acuracia", "Como o TurboQuant funciona" ("1. PolarQuant": random
+ *     orthogonal rotation; "2. QJL Residual": one extra bit per value removes
+ *     the inner-product bias);
+ *   - usedby.ai, "TurboQuant: Compresion de KV Cache a 3 bits y aceleracion de
+ *     inferencia en H100", "El Pitch" (logits computed on compressed keys).
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller unless the
+ *     comment says "host". The library never allocates device memory; scratch
+ *     space is a caller-provided workspace whose size a *_workspace_size call
+ *     returns.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and is asynchronous: no entry point synchronises the stream,
+ *     except tq_workspace_status, which says so.
+ *   - Arguments are checked on the host before anything is launched; a failed
+ *     check launches nothing and returns a status. Launch failures return
+ *     TQ_ERR_CUDA. tq_last_error() gives a thread-local message for the last
+ *     failure on the calling thread.
+ *   - Nothing aborts, asserts, traps or throws across the ABI.
+ *
+ * Cache record layout (one record per (sequence, kv head, token)):
+ *   R = index_words + sign_words little-endian uint32 words, with
+ *   index_words = ceil(idx_bits*d/32) and sign_words = ceil(d/32) for keys
+ *   (qjl = 1), 0 for values.
+ *   Index field: a bit stream (stream bit k = bit k%32 of word k/32); the
+ *   idx_bits-bit code of coordinate i sits at stream bits
+ *   [idx_bits*i, idx_bits*i + idx_bits), least significant bit first.
+ *   Sign field (keys): bit i = [ (S r)_i >= 0 ] at bit i%32 of word
+ *   index_words + i/32. Every unused bit is 0.
+ *   Records of one (sequence, head) are contiguous in token order; the array
+ *   is [n_seq][n_kv_heads][capacity][R]. Norms are separate float arrays
+ *   [n_seq][n_kv_heads][capacity].
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so that this header needs no CUDA include. */
+typedef struct CUstream_st *tq_stream;
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID = 1,     /* null or misaligned pointer, negative or inconsistent size   */
+  TQ_ERR_UNSUPPORTED = 2, /* d or idx_bits outside the supported range                    */
+  TQ_ERR_CAPACITY = 3,    /* pos + n_tokens exceeds the cache capacity                     */
+  TQ_ERR_WORKSPACE = 4,   /* workspace missing, misaligned or smaller than required        */
+  TQ_ERR_CUDA = 5,        /* a CUDA runtime call or a kernel launch failed                 */
+  TQ_ERR_DEVICE = 6       /* a kernel recorded a failure in the workspace status word     */
+} tq_status;
+
+typedef enum { TQ_BF16 = 0, TQ_FP16 = 1, TQ_FP32 = 2 } tq_dtype;
+
+/* Describes one packed K or V cache. All pointers are device memory owned by
+ * the caller; `records` must be 16-byte aligned, `norm`/`rnorm` 4-byte aligned. */
+typedef struct {
+  int32_t d;          /* head dimension: 8..256, multiple of 8                         */
+  int32_t idx_bits;   /* code bits per coordinate: 1..4 (keys use b-1, values use b)   */
+  int32_t qjl;        /* 1: key cache (sign field + rnorm), 0: value cache (MSE only)  */
+  int32_t n_seq;      /* sequences (batch)                                             */
+  int32_t n_kv_heads; /* KV heads per sequence                                         */
+  int32_t reserved;   /* must be 0                                                     */
+  int64_t capacity;   /* token slots per (sequence, head)                              */
+  uint32_t *records;  /* [n_seq][n_kv_heads][capacity][tq_record_words(d,idx_bits,qjl)] */
+  float *norm;        /* [n_seq][n_kv_heads][capacity]  ||x||                          */
+  float *rnorm;       /* same shape, ||r|| of the residual; NULL iff qjl == 0          */
+} tq_cache;
+
+/* Words per record for the layout above; -1 if (d, idx_bits) is unsupported. */
+int32_t tq_record_words(int32_t d, int32_t idx_bits, int32_t qjl);
+
+/* Lloyd-Max codebook for the coordinate law of a uniform point on the unit
+ * sphere S^{d-1}, density proportional to (1 - y^2)^((d-3)/2) on [-1, 1]
+ * (zubnet.ai, paragraph 2: "optimal scalar quantizer per coordinate" of the
+ * Beta-distributed rotated coordinates). Fitted in double precision on the
+ * HOST (setup, not the per-token path), made exactly symmetric and rounded to
+ * float. `centroids_host` receives 2^idx_bits ascending values (host memory).
+ * d: 3..4096; idx_bits: 1..8. */
+tq_status tq_codebook_fit(int32_t d, int32_t idx_bits, float *centroids_host);
+
+/* SPiT = S * Pi^T (d x d, row-major float). Pi: the d x d orthogonal rotation
+ * (row-major), S: the d x d Gaussian sketch matrix. The key quantizer projects
+ * the residual in the rotated domain, where S r = S Pi^T (y - yhat)
+ * (winningdata.io, "2. QJL Residual": the sketch acts on the residual).
+ * Accumulates in double on the device. d: 8..256. */
+tq_status tq_sketch_rotation(int32_t d, const float *Pi, const float *S, float *SPiT, tq_stream stream);
+
+/* Quantize n_tokens new vectors per (sequence, head) and write them into token
+ * slots [pos, pos + n_tokens) of `cache` (zubnet.ai, paragraph 2: rotate, MSE
+ * quantizer, 1-bit JL sketch of the residual, L2 norm).
+ *   x:        [n_seq][n_kv_heads][n_tokens][d] contiguous, dtype `dtype`.
+ *   Pi:       [d][d] float rotation, y = Pi x / ||x||.
+ *   SPiT:     [d][d] float, S Pi^T (see tq_sketch_rotation); ignored (may be NULL)
+ *             for a value cache.
+ *   codebook: 2^idx_bits ascending floats; code_i = #{j : y_i > (c_j + c_{j+1})/2}.
+ * For each vector: norm = ||x||; y = Pi x/||x||; codes; keys also store
+ * rnorm = ||y - c[code]|| and sign bits of SPiT (y - c[code]). A zero vector
+ * stores norm 0, rnorm 0, codes of y = 0 and all sign bits 1.
+ * Errors: TQ_ERR_CAPACITY if pos + n_tokens > capacity; n_tokens == 0 is a no-op. */
+tq_status tq_quantize_append(const tq_cache *cache, const void *x, tq_dtype dtype,
+                             int64_t pos, int64_t n_tokens,
+                             const float *Pi, const float *SPiT, const float *codebook,
+                             tq_stream stream);
+
+/* Workspace bytes tq_logits needs for this key cache and query-head count. */
+size_t tq_logits_workspace_size(const tq_cache *k, int32_t n_q_heads);
+
+/* Attention logits on the packed key cache, tokens [0, n_tokens) (usedby.ai,
+ * "El Pitch": logits computed directly on the compressed keys):
+ *   logits[s][h][t] = norm_t * ( <Pi q, c[code_t]> + rnorm_t * sqrt(pi/2)/d * <S q, 2 sign_t - 1> )
+ * where q = q[s][h] and the key cache head is h / (n_q_heads / n_kv_heads).
+ *   q:       [n_seq][n_q_heads][d] float.
+ *   logits:  [n_seq][n_q_heads][n_tokens] float.
+ *   Pi, S:   [d][d] float; codebook: 2^idx_bits floats (the key codebook).
+ * n_q_heads must be a positive multiple of k->n_kv_heads; k->qjl must be 1.
+ * workspace: >= tq_logits_workspace_size bytes, 256-byte aligned. */
+tq_status tq_logits(const tq_cache *k, const float *q, int32_t n_q_heads, int64_t n_tokens,
+                    const float *Pi, const float *S, const float *codebook,
+                    float *logits, void *workspace, size_t workspace_bytes, tq_stream stream);
+
+/* Workspace bytes tq_attend_v needs for this value cache, head count and length. */
+size_t tq_attend_workspace_size(const tq_cache *v, int32_t n_q_heads, int64_t n_tokens);
+
+/* Softmax-weighted sum of the packed values (zubnet.ai, paragraph 1: the cache
+ * holds keys and values):
+ *   p = softmax_t(scale * logits[s][h][t]),
+ *   out[s][h] = Pi^T sum_t p_t * norm_t * c[code_t]     (rotation undone once).
+ *   logits: [n_seq][n_q_heads][n_tokens] float; out: [n_seq][n_q_heads][d] float.
+ *   v->qjl must be 0. n_tokens == 0 writes zeros.
+ * workspace: >= tq_attend_workspace_size bytes, 256-byte aligned. */
+tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale,
+                      int32_t n_q_heads, int64_t n_tokens,
+                      const float *Pi, const float *codebook, float *out,
+                      void *workspace, size_t workspace_bytes, tq_stream stream);
+
+/* Synchronises `stream`, reads the status word that the kernels of the last
+ * tq_logits / tq_attend_v call on this workspace wrote, and clears it.
+ * TQ_OK if no kernel reported a failure, TQ_ERR_DEVICE otherwise (the message
+ * names the failure). */
+tq_status tq_workspace_status(void *workspace, tq_stream stream);
+
+/* Thread-local text of the last failure on this thread ("" if none). */
+const char *tq_last_error(void);
+
+/* Host-side fault injection for tests: the next `count` calls that would launch
+ * work return `status` instead, before any launch. count = 0 disarms. */
+void tq_debug_inject(tq_status status, int32_t count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

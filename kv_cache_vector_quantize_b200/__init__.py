@@ -1,0 +1,37 @@
+"""B200-native TurboQuant KV-cache quantization: Python binding of libtq.so.
+
+The package is a thin layer over the C ABI declared in ``include/tq.h``:
+``tq_quantize_append`` (online quantization of K/V head-vectors into a packed
+cache), ``tq_logits`` (attention logits on the packed keys) and
+``tq_attend_v`` (softmax-weighted packed values), plus the setup helpers
+``tq_codebook_fit`` and ``tq_sketch_rotation``. All compute runs in the CUDA
+kernels of ``csrc/`` built for sm_100a.
+"""
+
+from ._binding import (  # noqa: F401
+    LIB_PATH,
+    STATUS_NAMES,
+    TQ_ERR_CAPACITY,
+    TQ_ERR_CUDA,
+    TQ_ERR_DEVICE,
+    TQ_ERR_INVALID,
+    TQ_ERR_UNSUPPORTED,
+    TQ_ERR_WORKSPACE,
+    TQ_OK,
+    PackedCache,
+    TqCacheDesc,
+    TQError,
+    declared_symbols,
+    raw_lib,
+    tq_attend_v,
+    tq_attend_workspace_size,
+    tq_codebook_fit,
+    tq_debug_inject,
+    tq_last_error,
+    tq_logits,
+    tq_logits_workspace_size,
+    tq_quantize_append,
+    tq_record_words,
+    tq_sketch_rotation,
+    tq_workspace_status,
+)

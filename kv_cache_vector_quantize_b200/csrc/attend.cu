@@ -1,0 +1,171 @@
+// Softmax-weighted value accumulation on the packed value cache, split over
+// token chunks, and the log-sum-exp merge of the chunks.
+//
+// zubnet.ai news, "Google's TurboQuant quantizes LLM KV cache to 3.5 bits per
+// channel", paragraph 1: the cache holds keys and values; values are stored
+// MSE-only (norm + codes). With p = softmax(scale * logits):
+//   out = Pi^T sum_t p_t n_t c[code_t].
+// The sum runs in the rotated domain, so the d x d rotation is undone once per
+// query head (in the merge) instead of once per token.
+//
+// Chunk kernel: one CTA per (token chunk, sequence, KV head, query block).
+// It finds the chunk maximum m and sum l of exp(scale*logit - m) for each of
+// its query heads, keeps w_t = exp(scale*l_t - m) * n_t in shared memory, and
+// accumulates acc_i = sum_t w_t c[code_ti] with one thread per coordinate
+// (the codes of a token are read once and reused by every query head of the
+// group). Merge kernel: M = max_c m_c, L = sum_c l_c e^{m_c - M},
+// A = sum_c acc_c e^{m_c - M}, out = Pi^T A / L.
+#include "common.cuh"
+
+namespace tq {
+
+namespace {
+
+constexpr int kAThreads = 256;
+constexpr int kAMaxQ = 8;   // query heads per CTA (register accumulators)
+
+__device__ __forceinline__ float block_reduce(float v, float *red, bool is_max) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = is_max ? warp_max(v) : warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float r = red[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
+  return r;
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kAThreads) attend_chunk_kernel(const AttendParams p) {
+  constexpr int L = 1 << BITS;
+  extern __shared__ __align__(16) float sm[];
+  float *w = sm;                                   // [q_per_cta][chunk]
+  float *cbs = w + (size_t)p.q_per_cta * p.chunk;  // [16]
+  float *red = cbs + 16;                           // [32]
+  float *accs = red + 32;                          // [q_per_cta][d] split reduction
+  const int tid = threadIdx.x;
+  const int qb = blockIdx.y % p.qblocks;
+  const int sk = blockIdx.y / p.qblocks;
+  const int seq = sk / p.n_kv_heads, kvh = sk - seq * p.n_kv_heads;
+  const int h0 = kvh * p.group + qb * p.q_per_cta;
+  const int nq = min(p.q_per_cta, p.group - qb * p.q_per_cta);
+  const int c = blockIdx.x, d = p.d;
+  const int64_t t0 = (int64_t)c * p.chunk;
+  const int nt = (int)min((int64_t)p.chunk, p.n_tokens - t0);
+  const size_t slot0 = (size_t)sk * p.capacity + t0;
+
+  if (tid < L) cbs[tid] = p.codebook[tid];
+  for (int qq = 0; qq < nq; ++qq) {
+    const size_t hrow = (size_t)seq * p.n_q_heads + h0 + qq;
+    const float *lg = p.logits + hrow * p.n_tokens + t0;
+    float m = -INFINITY;
+    for (int t = tid; t < nt; t += kAThreads) m = fmaxf(m, p.scale * lg[t]);
+    m = block_reduce(m, red, true);
+    float s = 0.f;
+    for (int t = tid; t < nt; t += kAThreads) {
+      const float e = expf(p.scale * lg[t] - m);
+      s += e;
+      w[qq * p.chunk + t] = e * __ldg(p.norm + slot0 + t);
+    }
+    s = block_reduce(s, red, false);
+    if (tid == 0) {
+      float *part = p.partial + (hrow * p.n_chunks + c) * (size_t)(d + 2);
+      part[0] = m;
+      part[1] = s;
+    }
+  }
+  __syncthreads();
+
+  // one thread per coordinate; several token phases when d is small
+  const int dpad = (d + 31) & ~31;
+  const int nsplit = kAThreads / dpad;
+  const int i = tid % dpad, split = tid / dpad;
+  float acc[kAMaxQ];
+#pragma unroll
+  for (int qq = 0; qq < kAMaxQ; ++qq) acc[qq] = 0.f;
+  if (split < nsplit && i < d) {
+    for (int t = split; t < nt; t += nsplit) {
+      const uint32_t *rec = p.records + (slot0 + t) * p.rec_words;
+      const float cv = cbs[stream_bits(rec, BITS * i, BITS, p.rec_words)];
+#pragma unroll
+      for (int qq = 0; qq < kAMaxQ; ++qq)
+        if (qq < nq) acc[qq] = fmaf(w[qq * p.chunk + t], cv, acc[qq]);
+    }
+  }
+  // reduce the token phases through shared memory
+  for (int s = 0; s < nsplit; ++s) {
+    if (split == s && i < d) {
+      for (int qq = 0; qq < nq; ++qq) {
+        float *a = accs + qq * d + i;
+        *a = (s == 0) ? acc[qq] : *a + acc[qq];
+      }
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < nq * d; e += kAThreads) {
+    const int qq = e / d, ii = e - qq * d;
+    const size_t hrow = (size_t)seq * p.n_q_heads + h0 + qq;
+    p.partial[(hrow * p.n_chunks + c) * (size_t)(d + 2) + 2 + ii] = accs[e];
+  }
+}
+
+__global__ void attend_combine_kernel(const float *__restrict__ partial, int n_chunks, int d,
+                                      const float *__restrict__ Pi, float *__restrict__ out) {
+  __shared__ float a[kMaxD];
+  __shared__ float red[32];
+  const int row = blockIdx.x, tid = threadIdx.x;
+  const float *part = partial + (size_t)row * n_chunks * (d + 2);
+  float m = -INFINITY;
+  for (int c = tid; c < n_chunks; c += blockDim.x) m = fmaxf(m, part[(size_t)c * (d + 2)]);
+  m = block_reduce(m, red, true);
+  float l = 0.f;
+  for (int c = tid; c < n_chunks; c += blockDim.x) {
+    const float *pc = part + (size_t)c * (d + 2);
+    l += pc[1] * expf(pc[0] - m);
+  }
+  l = block_reduce(l, red, false);
+  for (int i = tid; i < d; i += blockDim.x) {
+    float s = 0.f;
+    for (int c = 0; c < n_chunks; ++c) {
+      const float *pc = part + (size_t)c * (d + 2);
+      s = fmaf(pc[2 + i], expf(pc[0] - m), s);
+    }
+    a[i] = s;
+  }
+  __syncthreads();
+  const float inv = 1.0f / l;
+  for (int j = tid; j < d; j += blockDim.x) {
+    float s = 0.f;
+    for (int i = 0; i < d; ++i) s = fmaf(__ldg(Pi + (size_t)i * d + j), a[i], s);
+    out[(size_t)row * d + j] = s * inv;
+  }
+}
+
+template <int BITS>
+cudaError_t launch_a(const AttendParams &p, int n_seq, size_t smem, cudaStream_t st) {
+  auto kern = attend_chunk_kernel<BITS>;
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.n_chunks, n_seq * p.n_kv_heads * p.qblocks);
+  kern<<<grid, kAThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attend(const AttendParams &p, int bits, int n_seq, size_t smem, cudaStream_t st) {
+  switch (bits) {
+    case 1: return launch_a<1>(p, n_seq, smem, st);
+    case 2: return launch_a<2>(p, n_seq, smem, st);
+    case 3: return launch_a<3>(p, n_seq, smem, st);
+    default: return launch_a<4>(p, n_seq, smem, st);
+  }
+}
+
+cudaError_t launch_combine(const float *partial, int rows, int n_chunks, int d, const float *Pi, float *out,
+                           cudaStream_t st) {
+  attend_combine_kernel<<<rows, 256, 0, st>>>(partial, n_chunks, d, Pi, out);
+  return cudaGetLastError();
+}
+
+}  // namespace tq

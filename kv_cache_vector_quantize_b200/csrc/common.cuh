@@ -1,0 +1,126 @@
+// Shared device helpers and launch parameter blocks for the TurboQuant kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tq.h"
+
+namespace tq {
+
+constexpr int kMaxBits = 4;           // code bits per coordinate handled by the kernels
+constexpr int kMaxD = 256;            // largest head dimension
+constexpr size_t kWsHeader = 256;     // bytes reserved at the start of every workspace
+
+// Status bits a kernel may set in the workspace status word.
+enum : uint32_t {
+  kDevBadShape = 1u << 0,   // a kernel met an argument its launch should have excluded
+};
+
+__device__ __forceinline__ float to_float(float v) { return v; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float to_float(__half v) { return __half2float(v); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Bits [pos, pos + nbits) of a little-endian word stream (nbits <= 25), read
+// through the read-only path. `words` is the number of valid words.
+__device__ __forceinline__ uint32_t stream_bits(const uint32_t *__restrict__ s, int pos, int nbits, int words) {
+  const int w = pos >> 5, sh = pos & 31;
+  uint32_t lo = __ldg(s + w);
+  uint32_t hi = (sh + nbits > 32 && w + 1 < words) ? __ldg(s + w + 1) : 0u;
+  return __funnelshift_r(lo, hi, sh) & ((1u << nbits) - 1u);
+}
+
+// ---------------------------------------------------------------------------
+// parameter blocks (plain structs passed by value to the kernels)
+// ---------------------------------------------------------------------------
+
+struct QuantParams {
+  const void *x;            // [rows][d]
+  uint32_t *records;        // cache records
+  float *norm;
+  float *rnorm;
+  const float *Pi;          // [d][d]
+  const float *SPiT;        // [d][d]
+  const float *codebook;    // [2^bits]
+  int64_t rows;             // n_seq * n_kv_heads * n_tokens
+  int64_t n_tokens;
+  int64_t capacity;
+  int64_t pos;
+  int d;
+  int rec_words;
+  int idx_words;
+};
+
+struct LogitsParams {
+  const uint32_t *records;
+  const float *norm;
+  const float *rnorm;
+  const float *qrot;        // [n_seq][n_q_heads][d]  Pi q
+  const float *qsk;         // [n_seq][n_q_heads][d]  S q
+  const float *codebook;
+  float *logits;            // [n_seq][n_q_heads][n_tokens]
+  uint32_t *status;
+  int64_t n_tokens;
+  int64_t capacity;
+  int64_t chunk;            // tokens per CTA
+  int d;
+  int rec_words;
+  int idx_words;
+  int n_kv_heads;
+  int n_q_heads;
+  int group;                // n_q_heads / n_kv_heads
+  int q_per_cta;            // query heads handled by one CTA
+  int qblocks;              // ceil(group / q_per_cta)
+};
+
+struct AttendParams {
+  const uint32_t *records;
+  const float *norm;
+  const float *logits;      // [n_seq][n_q_heads][n_tokens]
+  const float *codebook;
+  float *partial;           // [n_seq][n_q_heads][n_chunks][d + 2]
+  uint32_t *status;
+  int64_t n_tokens;
+  int64_t capacity;
+  int64_t chunk;
+  int n_chunks;
+  float scale;
+  int d;
+  int rec_words;
+  int n_kv_heads;
+  int n_q_heads;
+  int group;
+  int q_per_cta;
+  int qblocks;
+};
+
+// launchers (defined in the .cu files)
+cudaError_t launch_sketch_rotation(int d, const float *Pi, const float *S, float *SPiT, cudaStream_t st);
+cudaError_t launch_quantize(const QuantParams &p, int bits, bool qjl, tq_dtype dtype, cudaStream_t st);
+cudaError_t launch_qprep(const float *q, int rows, int d, const float *Pi, const float *S,
+                         float *qrot, float *qsk, uint32_t *status, cudaStream_t st);
+cudaError_t launch_logits(const LogitsParams &p, int bits, int n_seq, int n_chunks, size_t smem, cudaStream_t st);
+size_t logits_smem_per_query(int d, int bits);
+cudaError_t launch_attend(const AttendParams &p, int bits, int n_seq, size_t smem, cudaStream_t st);
+cudaError_t launch_combine(const float *partial, int rows, int n_chunks, int d, const float *Pi,
+                           float *out, cudaStream_t st);
+int device_sm_count();
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device).
+cudaError_t set_smem_once(const void *kernel, size_t bytes);
+size_t device_smem_optin();
+
+}  // namespace tq

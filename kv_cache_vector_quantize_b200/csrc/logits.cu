@@ -1,0 +1,147 @@
+// Query preparation and the attention-logit scan on the packed key cache.
+//
+// Estimator (usedby.ai, "TurboQuant: Compresion de KV Cache a 3 bits y
+// aceleracion de inferencia en H100", "El Pitch": logits on compressed keys;
+// winningdata.io, "TurboQuant: Google comprime KV cache para 3 bits sem perder
+// acuracia", "2. QJL Residual": the 1-bit sketch of the residual corrects the
+// inner-product bias):
+//   l_t = n_t ( <Pi q, c[code_t]> + rho_t sqrt(pi/2)/d <S q, 2 sign_t - 1> ).
+//
+// Both inner products are sums over small groups of coordinates, so each CTA
+// turns its queries into lookup tables in shared memory once and then reads
+// one table entry per group and key:
+//   index tables: one per group of g = 8/bits coordinates (2 for 3 bits); the
+//     entry for a group key (the g codes, as they sit in the code stream) is
+//     sum_c (Pi q)_c * c[code_c];
+//   sign tables: one per byte of the sign field; the entry for a byte is
+//     sqrt(pi/2)/d * sum_c (S q)_c * (+1 or -1).
+// A key then costs d/g + d/8 table reads and adds per query instead of 2d
+// multiply-adds on unpacked values.
+#include "common.cuh"
+
+namespace tq {
+
+namespace {
+
+constexpr int kLThreads = 256;
+
+__global__ void qprep_kernel(const float *__restrict__ q, int d, const float *__restrict__ Pi,
+                             const float *__restrict__ S, float *__restrict__ qrot, float *__restrict__ qsk,
+                             uint32_t *status) {
+  __shared__ float qs[kMaxD];
+  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (row == 0 && tid == 0) *status = 0u;   // this call's kernels report into a clean word
+  for (int k = tid; k < d; k += blockDim.x) qs[k] = q[(size_t)row * d + k];
+  __syncthreads();
+  for (int o = warp; o < 2 * d; o += blockDim.x / 32) {
+    const float *mrow = (o < d ? Pi : S) + (size_t)(o < d ? o : o - d) * d;
+    float s = 0.f;
+    for (int k = lane; k < d; k += 32) s = fmaf(__ldg(mrow + k), qs[k], s);
+    s = warp_sum(s);
+    if (lane == 0) (o < d ? qrot : qsk)[(size_t)row * d + (o < d ? o : o - d)] = s;
+  }
+}
+
+template <int BITS>
+struct Keys {
+  static constexpr int G = BITS == 1 ? 8 : BITS == 2 ? 4 : 2;   // coordinates per index key
+  static constexpr int KB = G * BITS;                           // key width in bits
+  static constexpr int E = 1 << KB;                             // entries per index table
+};
+
+template <int BITS>
+__global__ void __launch_bounds__(kLThreads) logits_kernel(const LogitsParams p) {
+  using K = Keys<BITS>;
+  constexpr int L = 1 << BITS;
+  extern __shared__ __align__(16) float tab[];
+  __shared__ float cbs[16];
+  const int tid = threadIdx.x;
+  const int qb = blockIdx.y % p.qblocks;
+  const int sk = blockIdx.y / p.qblocks;            // sequence * n_kv_heads + kv head
+  const int seq = sk / p.n_kv_heads, kvh = sk - seq * p.n_kv_heads;
+  const int h0 = kvh * p.group + qb * p.q_per_cta;
+  const int nq = min(p.q_per_cta, p.group - qb * p.q_per_cta);
+  const int d = p.d, nk = d / K::G, ns = d / 8;
+  const int per_q = nk * K::E + ns * 256;
+  const float kappa = 1.2533141373155003f / (float)d;   // sqrt(pi/2) / d
+
+  if (tid < L) cbs[tid] = p.codebook[tid];
+  __syncthreads();
+  for (int qq = 0; qq < nq; ++qq) {
+    const size_t qrow = ((size_t)seq * p.n_q_heads + h0 + qq) * d;
+    const float *qr = p.qrot + qrow;
+    const float *qs = p.qsk + qrow;
+    float *ti = tab + (size_t)qq * per_q;
+    for (int e = tid; e < nk * K::E; e += kLThreads) {
+      const int j = e / K::E, key = e - j * K::E;
+      float v = 0.f;
+#pragma unroll
+      for (int c = 0; c < K::G; ++c) v = fmaf(__ldg(qr + j * K::G + c), cbs[(key >> (BITS * c)) & (L - 1)], v);
+      ti[e] = v;
+    }
+    float *ts = ti + nk * K::E;
+    for (int e = tid; e < ns * 256; e += kLThreads) {
+      const int j = e >> 8, b = e & 255;
+      float v = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float s = __ldg(qs + 8 * j + c);
+        v += ((b >> c) & 1) ? s : -s;
+      }
+      ts[e] = kappa * v;
+    }
+  }
+  __syncthreads();
+
+  const int64_t t0 = (int64_t)blockIdx.x * p.chunk;
+  const int64_t t1 = min(p.n_tokens, t0 + p.chunk);
+  const int sw = (d + 31) / 32;
+  for (int64_t t = t0 + tid; t < t1; t += kLThreads) {
+    const size_t slot = (size_t)sk * p.capacity + t;
+    const uint32_t *rec = p.records + slot * p.rec_words;
+    const float n = __ldg(p.norm + slot), rho = __ldg(p.rnorm + slot);
+    for (int qq = 0; qq < nq; ++qq) {
+      const float *ti = tab + (size_t)qq * per_q;
+      const float *ts = ti + nk * K::E;
+      float ai = 0.f, as = 0.f;
+      for (int j = 0; j < nk; ++j) ai += ti[j * K::E + stream_bits(rec, K::KB * j, K::KB, p.idx_words)];
+      for (int j = 0; j < ns; ++j) as += ts[j * 256 + stream_bits(rec + p.idx_words, 8 * j, 8, sw)];
+      p.logits[((size_t)seq * p.n_q_heads + h0 + qq) * p.n_tokens + t] = n * fmaf(rho, as, ai);
+    }
+  }
+}
+
+template <int BITS>
+cudaError_t launch_l(const LogitsParams &p, int n_seq, int n_chunks, size_t smem, cudaStream_t st) {
+  auto kern = logits_kernel<BITS>;
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(n_chunks, n_seq * p.n_kv_heads * p.qblocks);
+  kern<<<grid, kLThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t logits_smem_per_query(int d, int bits) {
+  int g = bits == 1 ? 8 : bits == 2 ? 4 : 2;
+  int kb = g * bits;
+  return ((size_t)(d / g) * ((size_t)1 << kb) + (size_t)(d / 8) * 256) * sizeof(float);
+}
+
+cudaError_t launch_qprep(const float *q, int rows, int d, const float *Pi, const float *S, float *qrot, float *qsk,
+                         uint32_t *status, cudaStream_t st) {
+  qprep_kernel<<<rows, 256, 0, st>>>(q, d, Pi, S, qrot, qsk, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_logits(const LogitsParams &p, int bits, int n_seq, int n_chunks, size_t smem, cudaStream_t st) {
+  switch (bits) {
+    case 1: return launch_l<1>(p, n_seq, n_chunks, smem, st);
+    case 2: return launch_l<2>(p, n_seq, n_chunks, smem, st);
+    case 3: return launch_l<3>(p, n_seq, n_chunks, smem, st);
+    default: return launch_l<4>(p, n_seq, n_chunks, smem, st);
+  }
+}
+
+}  // namespace tq

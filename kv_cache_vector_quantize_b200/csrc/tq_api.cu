@@ -1,0 +1,358 @@
+// C ABI entry points (include/tq.h): host-side argument checks, workspace
+// carving, launch configuration and status reporting. Every compute step runs
+// in the kernels of quantize.cu, logits.cu and attend.cu.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+
+namespace tq {
+bool fit_lloyd_max(int d, int bits, float *out);
+
+namespace {
+
+thread_local char g_err[512] = "";
+std::atomic<int> g_inject_count{0};
+std::atomic<int> g_inject_status{0};
+
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices] = {0};
+int g_smem_optin[kMaxDevices] = {0};
+
+tq_status fail(tq_status s, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+tq_status cuda_fail(cudaError_t e, const char *where) {
+  return fail(TQ_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+// Host-side fault injection (tests): consume one armed failure, if any.
+bool injected(tq_status *s) {
+  int n = g_inject_count.load();
+  while (n > 0) {
+    if (g_inject_count.compare_exchange_weak(n, n - 1)) {
+      *s = fail((tq_status)g_inject_status.load(), "injected failure (tq_debug_inject)");
+      return true;
+    }
+  }
+  return false;
+}
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  return dev;
+}
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+tq_status check_cache(const tq_cache *c, const char *what) {
+  if (!c) return fail(TQ_ERR_INVALID, "%s: cache descriptor is NULL", what);
+  if (c->d < 8 || c->d > kMaxD || c->d % 8 != 0)
+    return fail(TQ_ERR_UNSUPPORTED, "%s: d=%d (need 8..%d, multiple of 8)", what, c->d, kMaxD);
+  if (c->idx_bits < 1 || c->idx_bits > kMaxBits)
+    return fail(TQ_ERR_UNSUPPORTED, "%s: idx_bits=%d (need 1..%d)", what, c->idx_bits, kMaxBits);
+  if (c->qjl != 0 && c->qjl != 1) return fail(TQ_ERR_INVALID, "%s: qjl=%d (need 0 or 1)", what, c->qjl);
+  if (c->n_seq <= 0 || c->n_kv_heads <= 0 || c->capacity < 0 || c->reserved != 0)
+    return fail(TQ_ERR_INVALID, "%s: n_seq=%d n_kv_heads=%d capacity=%lld reserved=%d", what, c->n_seq,
+                c->n_kv_heads, (long long)c->capacity, c->reserved);
+  if (!c->records || !aligned(c->records, 16)) return fail(TQ_ERR_INVALID, "%s: records NULL or not 16-byte aligned", what);
+  if (!c->norm || !aligned(c->norm, 4)) return fail(TQ_ERR_INVALID, "%s: norm NULL or misaligned", what);
+  if (c->qjl && (!c->rnorm || !aligned(c->rnorm, 4))) return fail(TQ_ERR_INVALID, "%s: key cache needs rnorm", what);
+  if (!c->qjl && c->rnorm) return fail(TQ_ERR_INVALID, "%s: value cache must have rnorm == NULL", what);
+  return TQ_OK;
+}
+
+int idx_words_of(int d, int bits) { return (bits * d + 31) / 32; }
+int rec_words_of(int d, int bits, int qjl) { return idx_words_of(d, bits) + (qjl ? (d + 31) / 32 : 0); }
+
+struct LogitsPlan {
+  int q_per_cta, qblocks, n_chunks;
+  int64_t chunk;
+  size_t smem;
+};
+
+LogitsPlan plan_logits(const tq_cache *k, int n_q_heads, int64_t n_tokens) {
+  LogitsPlan pl{};
+  const int group = n_q_heads / k->n_kv_heads;
+  const size_t per_q = logits_smem_per_query(k->d, k->idx_bits);
+  const size_t budget = device_smem_optin() - 1024;
+  int qpc = (int)(budget / per_q);
+  if (qpc > group) qpc = group;
+  pl.q_per_cta = qpc;
+  pl.qblocks = qpc > 0 ? (group + qpc - 1) / qpc : 0;
+  pl.smem = per_q * (size_t)(qpc > 0 ? qpc : 1);
+  const int64_t units = (int64_t)k->n_seq * k->n_kv_heads * (pl.qblocks > 0 ? pl.qblocks : 1);
+  const int64_t want = 4LL * device_sm_count();
+  int64_t chunks = (want + units - 1) / units;
+  const int64_t max_chunks = (n_tokens + 255) / 256;
+  if (chunks > max_chunks) chunks = max_chunks;
+  if (chunks < 1) chunks = 1;
+  int64_t chunk = (n_tokens + chunks - 1) / chunks;
+  chunk = (chunk + 127) / 128 * 128;
+  if (chunk < 128) chunk = 128;
+  pl.chunk = chunk;
+  pl.n_chunks = (int)((n_tokens + chunk - 1) / chunk);
+  return pl;
+}
+
+constexpr int64_t kAttendChunk = 512;
+constexpr int kAttendMaxQ = 8;
+
+}  // namespace
+
+int device_sm_count() {
+  const int dev = current_device();
+  if (g_sm_count[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 1;
+    g_sm_count[dev] = v;
+  }
+  return g_sm_count[dev];
+}
+
+size_t device_smem_optin() {
+  const int dev = current_device();
+  if (g_smem_optin[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess || v <= 0) v = 232448;  // sm_100 opt-in limit
+    g_smem_optin[dev] = v;
+  }
+  return (size_t)g_smem_optin[dev];
+}
+
+cudaError_t set_smem_once(const void *kernel, size_t bytes) {
+  // (kernel, device) pairs already raised; a small open table is enough for the
+  // few dozen kernel instantiations of this library.
+  struct Entry { const void *k; int dev; size_t bytes; };
+  static Entry table[512];
+  static std::atomic<int> used{0};
+  const int dev = current_device();
+  const int n = used.load();
+  for (int i = 0; i < n && i < 512; ++i)
+    if (table[i].k == kernel && table[i].dev == dev && table[i].bytes >= bytes) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  const int slot = used.fetch_add(1);
+  if (slot < 512) table[slot] = Entry{kernel, dev, bytes};
+  return cudaSuccess;
+}
+
+}  // namespace tq
+
+using namespace tq;
+
+extern "C" {
+
+int32_t tq_record_words(int32_t d, int32_t idx_bits, int32_t qjl) {
+  if (d < 8 || d > kMaxD || d % 8 != 0 || idx_bits < 1 || idx_bits > kMaxBits || (qjl != 0 && qjl != 1)) return -1;
+  return rec_words_of(d, idx_bits, qjl);
+}
+
+tq_status tq_codebook_fit(int32_t d, int32_t idx_bits, float *centroids_host) {
+  g_err[0] = 0;
+  if (d < 3 || d > 4096 || idx_bits < 1 || idx_bits > 8)
+    return fail(TQ_ERR_UNSUPPORTED, "tq_codebook_fit: d=%d idx_bits=%d (need d 3..4096, bits 1..8)", d, idx_bits);
+  if (!centroids_host) return fail(TQ_ERR_INVALID, "tq_codebook_fit: output is NULL");
+  if (!fit_lloyd_max(d, idx_bits, centroids_host)) return fail(TQ_ERR_INVALID, "tq_codebook_fit: iteration diverged");
+  return TQ_OK;
+}
+
+tq_status tq_sketch_rotation(int32_t d, const float *Pi, const float *S, float *SPiT, tq_stream stream) {
+  g_err[0] = 0;
+  if (d < 8 || d > kMaxD) return fail(TQ_ERR_UNSUPPORTED, "tq_sketch_rotation: d=%d", d);
+  if (!Pi || !S || !SPiT) return fail(TQ_ERR_INVALID, "tq_sketch_rotation: NULL matrix");
+  tq_status s;
+  if (injected(&s)) return s;
+  cudaError_t e = launch_sketch_rotation(d, Pi, S, SPiT, (cudaStream_t)stream);
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_sketch_rotation");
+}
+
+tq_status tq_quantize_append(const tq_cache *cache, const void *x, tq_dtype dtype, int64_t pos, int64_t n_tokens,
+                             const float *Pi, const float *SPiT, const float *codebook, tq_stream stream) {
+  g_err[0] = 0;
+  tq_status s = check_cache(cache, "tq_quantize_append");
+  if (s != TQ_OK) return s;
+  if (dtype != TQ_BF16 && dtype != TQ_FP16 && dtype != TQ_FP32)
+    return fail(TQ_ERR_INVALID, "tq_quantize_append: dtype=%d", (int)dtype);
+  if (pos < 0 || n_tokens < 0) return fail(TQ_ERR_INVALID, "tq_quantize_append: pos=%lld n_tokens=%lld",
+                                           (long long)pos, (long long)n_tokens);
+  if (pos + n_tokens > cache->capacity)
+    return fail(TQ_ERR_CAPACITY, "tq_quantize_append: pos %lld + n_tokens %lld > capacity %lld", (long long)pos,
+                (long long)n_tokens, (long long)cache->capacity);
+  if (n_tokens == 0) return TQ_OK;
+  const size_t esz = dtype == TQ_FP32 ? 4 : 2;
+  if (!x || !aligned(x, esz)) return fail(TQ_ERR_INVALID, "tq_quantize_append: x NULL or misaligned");
+  if (!Pi || !codebook) return fail(TQ_ERR_INVALID, "tq_quantize_append: Pi or codebook NULL");
+  if (cache->qjl && !SPiT) return fail(TQ_ERR_INVALID, "tq_quantize_append: key cache needs SPiT");
+  if (injected(&s)) return s;
+  QuantParams p{};
+  p.x = x;
+  p.records = cache->records;
+  p.norm = cache->norm;
+  p.rnorm = cache->rnorm;
+  p.Pi = Pi;
+  p.SPiT = SPiT;
+  p.codebook = codebook;
+  p.rows = (int64_t)cache->n_seq * cache->n_kv_heads * n_tokens;
+  p.n_tokens = n_tokens;
+  p.capacity = cache->capacity;
+  p.pos = pos;
+  p.d = cache->d;
+  p.rec_words = rec_words_of(cache->d, cache->idx_bits, cache->qjl);
+  p.idx_words = idx_words_of(cache->d, cache->idx_bits);
+  cudaError_t e = launch_quantize(p, cache->idx_bits, cache->qjl != 0, dtype, (cudaStream_t)stream);
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_quantize_append");
+}
+
+size_t tq_logits_workspace_size(const tq_cache *k, int32_t n_q_heads) {
+  if (!k || k->n_seq <= 0 || k->d <= 0 || n_q_heads <= 0) return 0;
+  return kWsHeader + 2 * sizeof(float) * (size_t)k->n_seq * n_q_heads * k->d;
+}
+
+tq_status tq_logits(const tq_cache *k, const float *q, int32_t n_q_heads, int64_t n_tokens, const float *Pi,
+                    const float *S, const float *codebook, float *logits, void *workspace, size_t workspace_bytes,
+                    tq_stream stream) {
+  g_err[0] = 0;
+  tq_status s = check_cache(k, "tq_logits");
+  if (s != TQ_OK) return s;
+  if (!k->qjl) return fail(TQ_ERR_INVALID, "tq_logits: the cache is a value cache (qjl == 0)");
+  if (n_q_heads <= 0 || n_q_heads % k->n_kv_heads != 0)
+    return fail(TQ_ERR_INVALID, "tq_logits: n_q_heads=%d is not a positive multiple of n_kv_heads=%d", n_q_heads,
+                k->n_kv_heads);
+  if (n_tokens < 0 || n_tokens > k->capacity)
+    return fail(TQ_ERR_CAPACITY, "tq_logits: n_tokens=%lld outside [0, capacity=%lld]", (long long)n_tokens,
+                (long long)k->capacity);
+  if (!q || !Pi || !S || !codebook || !logits) return fail(TQ_ERR_INVALID, "tq_logits: NULL tensor argument");
+  const size_t need = tq_logits_workspace_size(k, n_q_heads);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < need)
+    return fail(TQ_ERR_WORKSPACE, "tq_logits: workspace needs %zu bytes, 256-byte aligned (got %zu)", need,
+                workspace_bytes);
+  if (n_tokens == 0) return TQ_OK;
+  const LogitsPlan pl = plan_logits(k, n_q_heads, n_tokens);
+  if (pl.q_per_cta < 1)
+    return fail(TQ_ERR_UNSUPPORTED, "tq_logits: lookup tables for d=%d idx_bits=%d exceed shared memory", k->d,
+                k->idx_bits);
+  if (injected(&s)) return s;
+  uint32_t *status = static_cast<uint32_t *>(workspace);
+  float *qrot = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWsHeader);
+  float *qsk = qrot + (size_t)k->n_seq * n_q_heads * k->d;
+  cudaError_t e = launch_qprep(q, k->n_seq * n_q_heads, k->d, Pi, S, qrot, qsk, status, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_logits (query projection)");
+  LogitsParams p{};
+  p.records = k->records;
+  p.norm = k->norm;
+  p.rnorm = k->rnorm;
+  p.qrot = qrot;
+  p.qsk = qsk;
+  p.codebook = codebook;
+  p.logits = logits;
+  p.status = status;
+  p.n_tokens = n_tokens;
+  p.capacity = k->capacity;
+  p.chunk = pl.chunk;
+  p.d = k->d;
+  p.rec_words = rec_words_of(k->d, k->idx_bits, 1);
+  p.idx_words = idx_words_of(k->d, k->idx_bits);
+  p.n_kv_heads = k->n_kv_heads;
+  p.n_q_heads = n_q_heads;
+  p.group = n_q_heads / k->n_kv_heads;
+  p.q_per_cta = pl.q_per_cta;
+  p.qblocks = pl.qblocks;
+  e = launch_logits(p, k->idx_bits, k->n_seq, pl.n_chunks, pl.smem, (cudaStream_t)stream);
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_logits (scan)");
+}
+
+size_t tq_attend_workspace_size(const tq_cache *v, int32_t n_q_heads, int64_t n_tokens) {
+  if (!v || v->n_seq <= 0 || v->d <= 0 || n_q_heads <= 0 || n_tokens < 0) return 0;
+  const int64_t n_chunks = (n_tokens + kAttendChunk - 1) / kAttendChunk;
+  return kWsHeader + sizeof(float) * (size_t)v->n_seq * n_q_heads * (size_t)n_chunks * (v->d + 2);
+}
+
+tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale, int32_t n_q_heads, int64_t n_tokens,
+                      const float *Pi, const float *codebook, float *out, void *workspace, size_t workspace_bytes,
+                      tq_stream stream) {
+  g_err[0] = 0;
+  tq_status s = check_cache(v, "tq_attend_v");
+  if (s != TQ_OK) return s;
+  if (v->qjl) return fail(TQ_ERR_INVALID, "tq_attend_v: the cache is a key cache (qjl == 1)");
+  if (n_q_heads <= 0 || n_q_heads % v->n_kv_heads != 0)
+    return fail(TQ_ERR_INVALID, "tq_attend_v: n_q_heads=%d is not a positive multiple of n_kv_heads=%d", n_q_heads,
+                v->n_kv_heads);
+  if (n_tokens < 0 || n_tokens > v->capacity)
+    return fail(TQ_ERR_CAPACITY, "tq_attend_v: n_tokens=%lld outside [0, capacity=%lld]", (long long)n_tokens,
+                (long long)v->capacity);
+  if (!logits || !Pi || !codebook || !out) return fail(TQ_ERR_INVALID, "tq_attend_v: NULL tensor argument");
+  if (!(scale == scale) || scale == INFINITY || scale == -INFINITY) return fail(TQ_ERR_INVALID, "tq_attend_v: scale is not finite");
+  const size_t need = tq_attend_workspace_size(v, n_q_heads, n_tokens);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < need)
+    return fail(TQ_ERR_WORKSPACE, "tq_attend_v: workspace needs %zu bytes, 256-byte aligned (got %zu)", need,
+                workspace_bytes);
+  if (injected(&s)) return s;
+  const size_t out_bytes = sizeof(float) * (size_t)v->n_seq * n_q_heads * v->d;
+  if (n_tokens == 0) {
+    cudaError_t e = cudaMemsetAsync(out, 0, out_bytes, (cudaStream_t)stream);
+    return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_attend_v (empty)");
+  }
+  uint32_t *status = static_cast<uint32_t *>(workspace);
+  float *partial = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWsHeader);
+  const int group = n_q_heads / v->n_kv_heads;
+  AttendParams p{};
+  p.records = v->records;
+  p.norm = v->norm;
+  p.logits = logits;
+  p.codebook = codebook;
+  p.partial = partial;
+  p.status = status;
+  p.n_tokens = n_tokens;
+  p.capacity = v->capacity;
+  p.chunk = kAttendChunk;
+  p.n_chunks = (int)((n_tokens + kAttendChunk - 1) / kAttendChunk);
+  p.scale = scale;
+  p.d = v->d;
+  p.rec_words = rec_words_of(v->d, v->idx_bits, 0);
+  p.n_kv_heads = v->n_kv_heads;
+  p.n_q_heads = n_q_heads;
+  p.group = group;
+  p.q_per_cta = group < kAttendMaxQ ? group : kAttendMaxQ;
+  p.qblocks = (group + p.q_per_cta - 1) / p.q_per_cta;
+  const size_t smem = sizeof(float) * ((size_t)p.q_per_cta * kAttendChunk + 16 + 32 + (size_t)p.q_per_cta * v->d);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_attend_v (status)");
+  e = launch_attend(p, v->idx_bits, v->n_seq, smem, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_attend_v (chunks)");
+  e = launch_combine(partial, v->n_seq * n_q_heads, p.n_chunks, v->d, Pi, out, (cudaStream_t)stream);
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_attend_v (merge)");
+}
+
+tq_status tq_workspace_status(void *workspace, tq_stream stream) {
+  g_err[0] = 0;
+  if (!workspace || !aligned(workspace, 256)) return fail(TQ_ERR_WORKSPACE, "tq_workspace_status: bad workspace");
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_workspace_status (sync)");
+  uint32_t word = 0;
+  e = cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_workspace_status (read)");
+  if (word == 0) return TQ_OK;
+  const uint32_t zero = 0;
+  e = cudaMemcpy(workspace, &zero, sizeof zero, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_workspace_status (clear)");
+  return fail(TQ_ERR_DEVICE, "tq_workspace_status: kernel status 0x%08x%s", word,
+              (word & kDevBadShape) ? " (unexpected shape)" : "");
+}
+
+const char *tq_last_error(void) { return g_err; }
+
+void tq_debug_inject(tq_status status, int32_t count) {
+  g_inject_status.store((int)status);
+  g_inject_count.store(count > 0 ? count : 0);
+}
+
+}  // extern "C"

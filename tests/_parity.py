@@ -1,0 +1,96 @@
+"""Comparison of the CUDA path's packed cache, logits and outputs with the oracle.
+
+Tolerances (stated by the task for this method):
+  * codes and sign bits bit-exact, except a coordinate whose rotated value lies
+    within 1e-5 of a codebook threshold (|y_i - t_j| <= 1e-5 with ||u|| = 1 and
+    ||Pi_i|| = 1), or whose sketch value lies within 1e-5 ||S_i|| rho of zero;
+    such excused flips must be at most 1e-4 of all coordinates;
+  * norms (||x|| and rho) to 1e-5 relative;
+  * logits to 2e-3 * ||q|| * n_t, with the oracle evaluated on the GPU's cache;
+  * softmax.V to 2e-3 * max_t n_t (infinity norm), oracle on the GPU's cache and logits.
+Where the GPU moved a code across a threshold (excused), rho and the sign bits
+are checked against the oracle re-run on the GPU's codes.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from oracle import turboquant as otq
+
+FLIP_BAND = 1e-5
+FLIP_RATE_MAX = 1e-4
+NORM_RTOL = 1e-5
+LOGIT_TOL = 2e-3
+OUT_TOL = 2e-3
+
+
+def as_u32(records_i32) -> np.ndarray:
+    return np.ascontiguousarray(records_i32).view(np.uint32)
+
+
+def check_encoding(x, rec, norm, rnorm, Pi, S, codebook, d, bits, qjl):
+    """x: [n, d] float64 inputs (widened exactly), rec: [n, R] uint32, norm/rnorm [n].
+    Returns a dict of counts; raises AssertionError on any violation."""
+    x = np.asarray(x, dtype=np.float64)
+    Pi = np.asarray(Pi, dtype=np.float64)
+    c = np.asarray(codebook, dtype=np.float64)
+    n = x.shape[0]
+    assert rec.shape == (n, otq.record_words(d, bits, qjl)), rec.shape
+    assert otq.padding_is_zero(rec, d, bits, qjl), "non-zero padding bits"
+    enc = otq.quantize(x, Pi, codebook, S if qjl else None)
+    # ||x||
+    ref_n = enc["norm"]
+    bad = np.abs(norm - ref_n) > NORM_RTOL * np.maximum(ref_n, 1e-30)
+    assert not bad.any(), f"norm mismatch at rows {np.nonzero(bad)[0][:10]}: {norm[bad][:5]} vs {ref_n[bad][:5]}"
+    gi, gs = otq.unpack(rec, d, bits, qjl)
+    t = otq.thresholds_of(c)
+    dist = np.min(np.abs(enc["y"][:, :, None] - t[None, None, :]), axis=2)
+    idiff = gi != enc["idx"]
+    unexcused = idiff & (dist > FLIP_BAND)
+    assert not unexcused.any(), (
+        f"{unexcused.sum()} code mismatches outside the threshold band; first at "
+        f"{np.argwhere(unexcused)[:5].tolist()} y={enc['y'][unexcused][:5]} gpu={gi[unexcused][:5]} "
+        f"oracle={enc['idx'][unexcused][:5]}")
+    out = {"coords": n * d, "index_flips": int(idiff.sum()), "sign_flips": 0}
+    if qjl:
+        S64 = np.asarray(S, dtype=np.float64)
+        nz = ref_n > 0
+        u = np.zeros_like(x)
+        u[nz] = x[nz] / ref_n[nz, None]
+        r = u - c[gi] @ Pi
+        r[~nz] = 0.0
+        rho = np.sqrt(np.sum(r * r, axis=1))
+        bad = np.abs(rnorm - rho) > NORM_RTOL * np.maximum(rho, 1e-30) + 1e-7 * (rho == 0)
+        assert not bad.any(), f"rnorm mismatch at rows {np.nonzero(bad)[0][:10]}: {rnorm[bad][:5]} vs {rho[bad][:5]}"
+        s = r @ S64.T
+        want = (s >= 0).astype(np.int64)
+        sdiff = gs != want
+        band = FLIP_BAND * np.linalg.norm(S64, axis=1)[None, :] * rho[:, None]
+        unexcused = sdiff & (np.abs(s) > band)
+        assert not unexcused.any(), (
+            f"{unexcused.sum()} sign mismatches outside the zero band; first at {np.argwhere(unexcused)[:5].tolist()}")
+        out["sign_flips"] = int(sdiff.sum())
+    for field in ("index_flips", "sign_flips"):
+        assert out[field] <= FLIP_RATE_MAX * n * d, f"excused {field} {out[field]} exceed 1e-4 of {n * d} coordinates"
+    return out
+
+
+def check_logits(gpu, q, Pi, S, codebook, rec, norm, rnorm, d, bits):
+    """gpu: [nq, nt] logits; q: [nq, d] for ONE kv head; rec/norm/rnorm: that head's GPU cache."""
+    gi, gs = otq.unpack(rec, d, bits, True)
+    ref = otq.logits(q, Pi, S, codebook, norm, rnorm, gi, gs)
+    tol = LOGIT_TOL * np.linalg.norm(np.asarray(q, dtype=np.float64), axis=1)[:, None] * np.asarray(norm)[None, :]
+    err = np.abs(np.asarray(gpu, dtype=np.float64) - ref)
+    assert np.all(err <= tol + 1e-30), f"logit error {np.max(err / (tol + 1e-30)):.3g} x tolerance"
+    return float(np.max(err / (tol + 1e-30))) if err.size else 0.0
+
+
+def check_attend(gpu, lg, scale, Pi, codebook, rec, norm, d, bits):
+    """gpu: [nq, d] outputs; lg: [nq, nt] the logits fed to the GPU; rec/norm: one kv head's value cache."""
+    gi, _ = otq.unpack(rec, d, bits, False)
+    ref = otq.attend_v(lg, scale, norm, gi, Pi, codebook)
+    tol = OUT_TOL * (float(np.max(norm)) if len(norm) else 1.0)
+    err = np.abs(np.asarray(gpu, dtype=np.float64) - ref)
+    assert np.all(err <= tol), f"softmax.V error {np.max(err) / tol:.3g} x tolerance"
+    return float(np.max(err) / tol) if err.size else 0.0

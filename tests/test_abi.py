@@ -1,0 +1,124 @@
+"""C-ABI library on the host (no GPU needed): it loads, exports every symbol
+that include/tq.h declares, computes its record sizes and codebooks, and
+rejects bad arguments with the right status before launching anything.
+
+The argument-check tests pass placeholder device addresses; each such call
+must fail in the host checks. As a guard, a fault is armed with
+tq_debug_inject first, so a call that wrongly got past the checks returns the
+injected status instead of launching a kernel.
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+
+import kv_cache_vector_quantize_b200 as tqb
+from oracle import codebook as ocb
+from oracle import turboquant as otq
+
+lib = tqb.raw_lib()
+FAKE = 0x7F0000000000     # 256-byte aligned placeholder address (never dereferenced)
+
+
+def _desc(d=128, bits=2, qjl=1, n_seq=1, heads=2, cap=64, records=FAKE, norm=FAKE + 4096, rnorm=FAKE + 8192):
+    return tqb.TqCacheDesc(d, bits, qjl, n_seq, heads, 0, cap, records, norm, rnorm if qjl else None)
+
+
+@pytest.fixture(autouse=True)
+def _guard():
+    tqb.tq_debug_inject(tqb.TQ_ERR_CUDA, 1000)   # any call that passes the checks returns TQ_ERR_CUDA
+    yield
+    tqb.tq_debug_inject(tqb.TQ_OK, 0)
+
+
+def test_every_declared_symbol_is_exported():
+    names = tqb.declared_symbols()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+@pytest.mark.parametrize("d,bits,qjl", [(8, 1, 1), (128, 2, 1), (128, 3, 0), (200, 3, 1), (200, 4, 0), (256, 4, 1)])
+def test_record_words_match_layout(d, bits, qjl):
+    assert tqb.tq_record_words(d, bits, qjl) == otq.record_words(d, bits, bool(qjl))
+
+
+def test_record_words_rejects_unsupported():
+    for d, bits in ((7, 2), (12, 2), (264, 2), (128, 0), (128, 5)):
+        assert lib.tq_record_words(d, bits, 1) == -1
+
+
+@pytest.mark.parametrize("d", [8, 64, 128, 200, 256])
+def test_codebook_fit_matches_oracle_bit_exactly(d):
+    # The library integrates the law with the Wallis recurrence; the oracle with
+    # the regularized incomplete beta function. After rounding to float32 the two
+    # Lloyd-Max fixed points must be the same numbers.
+    for bits in (1, 2, 3, 4):
+        got = tqb.tq_codebook_fit(d, bits).numpy()
+        want = ocb.fit_codebook(d, bits)[0]
+        assert np.array_equal(got, want), (d, bits, got - want)
+
+
+def test_codebook_fit_more_levels_and_small_d():
+    for d, bits in ((128, 5), (128, 6), (3, 3), (5, 2)):
+        got = tqb.tq_codebook_fit(d, bits).numpy()
+        want = ocb.fit_codebook(d, bits)[0]
+        assert np.allclose(got, want, rtol=0, atol=2e-7 * np.abs(want).max()), (d, bits)
+    with pytest.raises(tqb.TQError) as e:
+        tqb.tq_codebook_fit(2, 2)
+    assert e.value.status == tqb.TQ_ERR_UNSUPPORTED
+
+
+def _q(desc, x=FAKE, pos=0, n=8, Pi=FAKE, SPiT=FAKE, cb=FAKE, dtype=0):
+    return lib.tq_quantize_append(ctypes.byref(desc) if desc is not None else None, x, dtype, pos, n, Pi, SPiT, cb, None)
+
+
+def test_quantize_argument_checks():
+    assert _q(None) == tqb.TQ_ERR_INVALID
+    assert _q(_desc(d=12)) == tqb.TQ_ERR_UNSUPPORTED
+    assert _q(_desc(bits=5)) == tqb.TQ_ERR_UNSUPPORTED
+    assert _q(_desc(cap=64), pos=60, n=5) == tqb.TQ_ERR_CAPACITY
+    assert "capacity" in tqb.tq_last_error()
+    assert _q(_desc(records=FAKE + 4)) == tqb.TQ_ERR_INVALID
+    assert _q(_desc(), dtype=7) == tqb.TQ_ERR_INVALID
+    assert _q(_desc(), SPiT=None) == tqb.TQ_ERR_INVALID
+    assert _q(_desc(qjl=0), SPiT=None) == tqb.TQ_ERR_CUDA          # passes the checks -> injected
+    assert _q(_desc(), n=0) == tqb.TQ_OK                           # nothing to do, nothing launched
+    d = _desc()
+    d.rnorm = None
+    assert _q(d) == tqb.TQ_ERR_INVALID
+
+
+def _lg(desc, hq=4, n=8, ws=FAKE, ws_bytes=1 << 20):
+    return lib.tq_logits(ctypes.byref(desc), FAKE, hq, n, FAKE, FAKE, FAKE, FAKE, ws, ws_bytes, None)
+
+
+def test_logits_argument_checks():
+    assert _lg(_desc(qjl=0)) == tqb.TQ_ERR_INVALID
+    assert _lg(_desc(heads=2), hq=3) == tqb.TQ_ERR_INVALID
+    assert _lg(_desc(cap=64), n=65) == tqb.TQ_ERR_CAPACITY
+    assert _lg(_desc(), ws=FAKE + 16) == tqb.TQ_ERR_WORKSPACE
+    assert _lg(_desc(), ws_bytes=16) == tqb.TQ_ERR_WORKSPACE
+    assert _lg(_desc(), n=0) == tqb.TQ_OK
+    assert _lg(_desc()) == tqb.TQ_ERR_CUDA                         # passes the checks -> injected
+    assert lib.tq_logits_workspace_size(ctypes.byref(_desc()), 4) == 256 + 2 * 4 * 4 * 128
+
+
+def test_attend_argument_checks():
+    def call(desc, hq=4, n=8, scale=0.1, ws_bytes=1 << 20):
+        return lib.tq_attend_v(ctypes.byref(desc), FAKE, ctypes.c_float(scale), hq, n, FAKE, FAKE, FAKE, FAKE,
+                               ws_bytes, None)
+    assert call(_desc(qjl=1)) == tqb.TQ_ERR_INVALID
+    assert call(_desc(qjl=0), hq=3) == tqb.TQ_ERR_INVALID
+    assert call(_desc(qjl=0), scale=float("nan")) == tqb.TQ_ERR_INVALID
+    assert call(_desc(qjl=0), ws_bytes=8) == tqb.TQ_ERR_WORKSPACE
+    assert call(_desc(qjl=0)) == tqb.TQ_ERR_CUDA                   # passes the checks -> injected
+
+
+def test_fault_injection_counts_down():
+    tqb.tq_debug_inject(tqb.TQ_ERR_DEVICE, 2)
+    assert _q(_desc(qjl=0)) == tqb.TQ_ERR_DEVICE
+    assert _q(_desc(qjl=0)) == tqb.TQ_ERR_DEVICE
+    assert "injected" in tqb.tq_last_error()
+    tqb.tq_debug_inject(tqb.TQ_ERR_CUDA, 1000)

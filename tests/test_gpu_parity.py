@@ -1,0 +1,268 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Small and ragged shapes are compared element by element; the full-size
+workloads (the Llama-3-8B-shaped decode that bench.py times, and the b-sweep
+caches) are compared on sampled rows and keys plus properties that hold at
+any size. Every call goes through kv_cache_vector_quantize_b200 -> libtq.so.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import tq_synth as syn
+from oracle import codebook as ocb
+from oracle import turboquant as otq
+from tests import _parity as par
+
+pytestmark = pytest.mark.gpu
+
+cuda_ok = torch.cuda.is_available()
+if cuda_ok:
+    import kv_cache_vector_quantize_b200 as tqb
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not cuda_ok:
+        pytest.skip("needs a CUDA device")
+
+
+def _codebook(d, bits):
+    return ocb.fit_codebook(d, bits)[0]          # float32 centroids the oracle also uses
+
+
+def _setup(d, k_idx_bits, v_bits):
+    Pi = syn.rotation(d)
+    S = syn.sketch(d)
+    ck = _codebook(d, k_idx_bits)
+    cv = _codebook(d, v_bits)
+    dev = torch.device("cuda")
+    g = dict(Pi=Pi.to(dev), S=S.to(dev), ck=torch.from_numpy(ck).to(dev), cv=torch.from_numpy(cv).to(dev))
+    g["SPiT"] = tqb.tq_sketch_rotation(g["Pi"], g["S"])
+    return Pi.numpy(), S.numpy(), ck, cv, g
+
+
+def _run_path(k, v, q, d, k_idx_bits, v_bits, g, capacity=None, scale=None):
+    """Quantize K and V, then logits and softmax.V. Returns GPU tensors."""
+    n_seq, hkv, T, _ = k.shape
+    cap = T if capacity is None else capacity
+    kc = tqb.PackedCache.empty(d, k_idx_bits, True, n_seq, hkv, cap)
+    vc = tqb.PackedCache.empty(d, v_bits, False, n_seq, hkv, cap)
+    tqb.tq_quantize_append(kc, k.cuda(), 0, g["Pi"], g["SPiT"], g["ck"])
+    tqb.tq_quantize_append(vc, v.cuda(), 0, g["Pi"], None, g["cv"])
+    lg = tqb.tq_logits(kc, q.cuda(), T, g["Pi"], g["S"], g["ck"])
+    sc = 1.0 / math.sqrt(d) if scale is None else scale
+    out = tqb.tq_attend_v(vc, lg, sc, T, g["Pi"], g["cv"])
+    torch.cuda.synchronize()
+    return kc, vc, lg, out, sc
+
+
+def _check_all(k, v, q, d, k_idx_bits, v_bits, Pi, S, ck, cv, kc, vc, lg, out, sc, rows=None):
+    n_seq, hkv, T, _ = k.shape
+    hq = q.shape[1]
+    G = hq // hkv
+    kx = k.float().numpy().astype(np.float64)
+    vx = v.float().numpy().astype(np.float64)
+    krec = par.as_u32(kc.records.cpu().numpy())
+    vrec = par.as_u32(vc.records.cpu().numpy())
+    kn, kr, vn = kc.norm.cpu().numpy(), kc.rnorm.cpu().numpy(), vc.norm.cpu().numpy()
+    lg_np, out_np, qn = lg.cpu().numpy(), out.cpu().numpy(), q.numpy().astype(np.float64)
+    stats = {"index_flips": 0, "sign_flips": 0, "coords": 0}
+    for s in range(n_seq):
+        for h in range(hkv):
+            sel = slice(None) if rows is None else rows
+            ek = par.check_encoding(kx[s, h, :T][sel], krec[s, h, :T][sel], kn[s, h, :T][sel], kr[s, h, :T][sel],
+                                    Pi, S, ck, d, k_idx_bits, True)
+            ev = par.check_encoding(vx[s, h, :T][sel], vrec[s, h, :T][sel], vn[s, h, :T][sel], None,
+                                    Pi, None, cv, d, v_bits, False)
+            for e in (ek, ev):
+                for key in stats:
+                    stats[key] += e[key]
+            qs = qn[s, h * G:(h + 1) * G]
+            par.check_logits(lg_np[s, h * G:(h + 1) * G], qs, Pi, S, ck, krec[s, h, :T], kn[s, h, :T],
+                             kr[s, h, :T], d, k_idx_bits)
+            par.check_attend(out_np[s, h * G:(h + 1) * G], lg_np[s, h * G:(h + 1) * G].astype(np.float64), sc, Pi,
+                             cv, vrec[s, h, :T], vn[s, h, :T], d, v_bits)
+    return stats
+
+
+def test_sketch_rotation_matches_float64_product():
+    d = 128
+    Pi, S = syn.rotation(d), syn.sketch(d)
+    got = tqb.tq_sketch_rotation(Pi.cuda(), S.cuda()).cpu().numpy()
+    want = S.double().numpy() @ Pi.double().numpy().T
+    assert np.allclose(got, want, rtol=0, atol=2e-6 * np.abs(want).max())
+
+
+def test_pr1_parity():
+    # d=128, 4096 keys fp32 N(0,1) seed 0, 16 queries; b=3 keys (2-bit codebook + QJL);
+    # values of the same law at 3 bits MSE-only.
+    k, v, q = syn.pr1_inputs()
+    Pi, S, ck, cv, g = _setup(128, 2, 3)
+    kc, vc, lg, out, sc = _run_path(k, v, q, 128, 2, 3, g)
+    stats = _check_all(k, v, q, 128, 2, 3, Pi, S, ck, cv, kc, vc, lg, out, sc)
+    assert stats["index_flips"] + stats["sign_flips"] <= 1e-4 * stats["coords"]
+
+
+SHAPES = [
+    # d, k index bits, v bits, n_seq, kv heads, group, tokens, dtype
+    (8, 1, 2, 2, 3, 2, 301, torch.float32),
+    (200, 2, 3, 1, 2, 4, 1037, torch.bfloat16),
+    (128, 3, 4, 2, 2, 1, 777, torch.float16),
+    (64, 2, 1, 1, 1, 8, 129, torch.bfloat16),
+    (256, 3, 4, 1, 1, 2, 300, torch.bfloat16),
+    (128, 1, 2, 1, 2, 4, 1, torch.float32),
+    (96, 2, 2, 3, 1, 3, 513, torch.float32),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"d{s[0]}-kb{s[1]}-vb{s[2]}-B{s[3]}-H{s[4]}-G{s[5]}-T{s[6]}")
+def test_shapes_parity(shape):
+    d, kb, vb, B, H, G, T, dt = shape
+    k = syn.gaussian((B, H, T, d), 10 + d).to(dt)
+    v = syn.lognormal_sphere((B, H, T, d), 20 + d, dtype=dt)
+    q = syn.gaussian((B, H * G, d), 30 + d)
+    Pi, S, ck, cv, g = _setup(d, kb, vb)
+    kc, vc, lg, out, sc = _run_path(k, v, q, d, kb, vb, g, capacity=T + 5)
+    _check_all(k, v, q, d, kb, vb, Pi, S, ck, cv, kc, vc, lg, out, sc)
+
+
+def test_append_in_parts_equals_one_call():
+    d, kb, T = 128, 2, 700
+    k = syn.gaussian((2, 2, T, d), 41).to(torch.bfloat16).cuda()
+    _, _, _, _, g = _setup(d, kb, 3)
+    one = tqb.PackedCache.empty(d, kb, True, 2, 2, T)
+    parts = tqb.PackedCache.empty(d, kb, True, 2, 2, T)
+    tqb.tq_quantize_append(one, k, 0, g["Pi"], g["SPiT"], g["ck"])
+    for a, b in ((0, 65), (65, 66), (66, 640), (640, 700)):
+        tqb.tq_quantize_append(parts, k[:, :, a:b].contiguous(), a, g["Pi"], g["SPiT"], g["ck"])
+    torch.cuda.synchronize()
+    assert torch.equal(one.records, parts.records)
+    assert torch.equal(one.norm, parts.norm) and torch.equal(one.rnorm, parts.rnorm)
+
+
+def test_special_vectors():
+    # zero vectors, codeword directions, tiny and huge norms
+    d, kb = 128, 2
+    Pi, S, ck, cv, g = _setup(d, kb, 3)
+    rng = np.random.default_rng(5)
+    rows = [np.zeros(d)]
+    c = ck.astype(np.float64)
+    for a in range(5):
+        w = c[rng.integers(0, 4, size=d)]
+        rows.append(3.0 * (w @ Pi.astype(np.float64)) / np.linalg.norm(w))
+    rows += [1e-20 * rng.standard_normal(d), 1e20 * rng.standard_normal(d), np.ones(d), -np.ones(d)]
+    x = torch.tensor(np.array(rows), dtype=torch.float32).reshape(1, 1, -1, d)
+    kc = tqb.PackedCache.empty(d, kb, True, 1, 1, x.shape[2])
+    tqb.tq_quantize_append(kc, x.cuda(), 0, g["Pi"], g["SPiT"], g["ck"])
+    torch.cuda.synchronize()
+    rec = par.as_u32(kc.records.cpu().numpy())[0, 0]
+    par.check_encoding(x[0, 0].double().numpy(), rec, kc.norm.cpu().numpy()[0, 0], kc.rnorm.cpu().numpy()[0, 0],
+                       Pi, S, ck, d, kb, True)
+    gi, gs = otq.unpack(rec, d, kb, True)
+    assert kc.norm[0, 0, 0].item() == 0 and kc.rnorm[0, 0, 0].item() == 0 and gs[0].all()
+
+
+def test_empty_inputs():
+    d = 64
+    _, _, _, _, g = _setup(d, 2, 2)
+    kc = tqb.PackedCache.empty(d, 2, True, 1, 2, 16)
+    vc = tqb.PackedCache.empty(d, 2, False, 1, 2, 16)
+    tqb.tq_quantize_append(kc, torch.empty((1, 2, 0, d), device="cuda"), 3, g["Pi"], g["SPiT"], g["ck"])
+    lg = tqb.tq_logits(kc, torch.randn(1, 4, d, device="cuda"), 0, g["Pi"], g["S"], g["ck"])
+    out = torch.full((1, 4, d), 7.0, device="cuda")
+    tqb.tq_attend_v(vc, lg, 0.125, 0, g["Pi"], g["cv"], out=out)
+    torch.cuda.synchronize()
+    assert lg.numel() == 0 and torch.all(out == 0)
+    assert torch.all(kc.records == 0)
+
+
+def test_errors_reported_without_launch():
+    d = 64
+    _, _, _, _, g = _setup(d, 2, 2)
+    kc = tqb.PackedCache.empty(d, 2, True, 1, 1, 8)
+    with pytest.raises(tqb.TQError) as e:
+        tqb.tq_quantize_append(kc, torch.zeros((1, 1, 9, d), device="cuda"), 0, g["Pi"], g["SPiT"], g["ck"])
+    assert e.value.status == tqb.TQ_ERR_CAPACITY
+    with pytest.raises(tqb.TQError) as e:
+        tqb.tq_logits(kc, torch.zeros((1, 1, d), device="cuda"), 9, g["Pi"], g["S"], g["ck"])
+    assert e.value.status == tqb.TQ_ERR_CAPACITY
+    ws = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    with pytest.raises(tqb.TQError) as e:
+        tqb.tq_logits(kc, torch.zeros((1, 1, d), device="cuda"), 4, g["Pi"], g["S"], g["ck"], workspace=ws)
+    assert e.value.status == tqb.TQ_ERR_WORKSPACE
+    assert torch.all(kc.records == 0)
+
+
+def test_workspace_status_clean_after_calls():
+    d = 128
+    _, _, _, _, g = _setup(d, 2, 3)
+    kc = tqb.PackedCache.empty(d, 2, True, 1, 1, 256)
+    tqb.tq_quantize_append(kc, torch.randn(1, 1, 256, d, device="cuda"), 0, g["Pi"], g["SPiT"], g["ck"])
+    ws = torch.empty(tqb.tq_logits_workspace_size(kc, 2), dtype=torch.uint8, device="cuda")
+    ws.fill_(0xFF)   # the call must clear the status word itself
+    tqb.tq_logits(kc, torch.randn(1, 2, d, device="cuda"), 256, g["Pi"], g["S"], g["ck"], workspace=ws)
+    tqb.tq_workspace_status(ws)
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, sampled
+# ---------------------------------------------------------------------------
+
+def test_llama_decode_full_size():
+    # 1 x 8 KV heads x 32768 tokens x 128, bf16 with outlier channels; 32 query heads;
+    # K at 3 bits (2-bit codes + QJL), V at 3 bits MSE-only; the bench's launch shapes.
+    k, v, q = syn.llama_inputs(device="cuda")
+    Pi, S, ck, cv, g = _setup(128, 2, 3)
+    kc, vc, lg, out, sc = _run_path(k, v, q, 128, 2, 3, g)
+    rng = np.random.default_rng(17)
+    rows = np.sort(rng.choice(32768, size=1024, replace=False))
+    kx = k[0].float().cpu().numpy()
+    vx = v[0].float().cpu().numpy()
+    krec = par.as_u32(kc.records.cpu().numpy())[0]
+    vrec = par.as_u32(vc.records.cpu().numpy())[0]
+    kn, kr, vn = kc.norm.cpu().numpy()[0], kc.rnorm.cpu().numpy()[0], vc.norm.cpu().numpy()[0]
+    lg_np, out_np, qn = lg.cpu().numpy()[0], out.cpu().numpy()[0], q.cpu().numpy()[0].astype(np.float64)
+    for h in range(8):
+        par.check_encoding(kx[h][rows], krec[h][rows], kn[h][rows], kr[h][rows], Pi, S, ck, 128, 2, True)
+        par.check_encoding(vx[h][rows], vrec[h][rows], vn[h][rows], None, Pi, None, cv, 128, 3, False)
+        # logits and outputs: every key and every query head of this KV head
+        par.check_logits(lg_np[4 * h:4 * h + 4], qn[4 * h:4 * h + 4], Pi, S, ck, krec[h], kn[h], kr[h], 128, 2)
+        par.check_attend(out_np[4 * h:4 * h + 4], lg_np[4 * h:4 * h + 4].astype(np.float64), sc, Pi, cv,
+                         vrec[h], vn[h], 128, 3)
+    assert np.isfinite(lg_np).all() and np.isfinite(out_np).all()
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_bsweep_full_size_sampled(bits):
+    # 8 x 8 KV heads x 131072 tokens x 128, bf16, lognormal norms; K at b bits (b-1 codes + QJL).
+    B, H, T, d = 8, 8, 131072, 128
+    k, v, q = syn.sweep_inputs(device="cuda")
+    Pi, S, ck, cv, g = _setup(d, bits - 1, bits)
+    kc = tqb.PackedCache.empty(d, bits - 1, True, B, H, T)
+    vc = tqb.PackedCache.empty(d, bits, False, B, H, T)
+    tqb.tq_quantize_append(kc, k, 0, g["Pi"], g["SPiT"], g["ck"])
+    tqb.tq_quantize_append(vc, v, 0, g["Pi"], None, g["cv"])
+    lg = tqb.tq_logits(kc, q, T, g["Pi"], g["S"], g["ck"])
+    torch.cuda.synchronize()
+    del v
+    rng = np.random.default_rng(100 + bits)
+    for _ in range(4):
+        s, h = int(rng.integers(B)), int(rng.integers(H))
+        rows = np.sort(rng.choice(T, size=512, replace=False))
+        idx = torch.from_numpy(rows).cuda()
+        kx = k[s, h].index_select(0, idx).float().cpu().numpy()
+        krec = par.as_u32(kc.records[s, h].index_select(0, idx).cpu().numpy())
+        kn = kc.norm[s, h].index_select(0, idx).cpu().numpy()
+        kr = kc.rnorm[s, h].index_select(0, idx).cpu().numpy()
+        par.check_encoding(kx, krec, kn, kr, Pi, S, ck, d, bits - 1, True)
+        par.check_logits(lg[s, h].index_select(0, idx).cpu().numpy()[None, :],
+                         q[s, h].cpu().numpy()[None, :].astype(np.float64), Pi, S, ck, krec, kn, kr, d, bits - 1)
+    # properties at full size: the packed norms are finite and positive, logits finite
+    assert torch.isfinite(lg).all()
+    assert bool((kc.norm > 0).all()) and bool(torch.isfinite(kc.rnorm).all())
