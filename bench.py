@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""Benchmark of the TurboQuant hot path on B200: one JSON line on stdout.
+
+A step is one pass of the whole path over one batch of synthetic input:
+  quantize-append of all keys and values into the packed caches
+  -> L2 flush (the decode reads a cache written long before, from HBM)
+  -> tq_logits (query projection + logit scan) -> tq_attend_v (softmax.V).
+
+Default workload (N = 1): the Llama-3-8B-shaped decode -- 1 sequence, 32 query
+heads on 8 KV heads, d = 128, 32768 cached tokens, bf16 K/V with outlier
+channels, keys at 3 bits (2-bit codes + 1 QJL bit), values at 3 bits MSE-only.
+`--workload sweep-b{2,3,4}` runs the b-sweep caches (8 x 8 x 131072 tokens).
+
+Metric: packed-KV logit-scan GB/s = packed key bytes (records + norms) read
+by one tq_logits call / its device time; quantize tokens/s is reported beside
+it. Times are CUDA events on the launching stream; with N ranks (torchrun)
+every rank runs its own copy of the workload (weak scaling, no collective on
+the data path) and the slowest rank's time is used.
+
+`--impl reference` times the float64 CPU oracle on a bounded sample of the
+same workload (the reference arm of this benchmark).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import tq_synth as syn  # noqa: E402
+
+METRIC = "packed-KV logit-scan GB/s (% of HBM peak); K/V quantize tokens/s at 1 B200"
+UNIT = "GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}
+SM_COUNT_B200 = 148
+FP32_LANES_PER_SM = 128
+
+# DRAM bytes per launch from ncu captures of the current kernels (None until
+# captured for the kernel as it stands). Keys: (kernel, workload).
+NCU_TRAFFIC = {}
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
+    ap.add_argument("--workload", default="llama", choices=["llama", "sweep-b2", "sweep-b3", "sweep-b4"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------
+# workloads
+# ----------------------------------------------------------------------------
+
+def workload(name: str):
+    if name == "llama":
+        return dict(name="llama3-8b-decode: B=1 Hq=32 Hkv=8 d=128 T=32768 bf16 K b=3 (2-bit codes+QJL) V b=3 MSE",
+                    n_seq=1, hq=32, hkv=8, d=128, T=32768, k_idx=2, v_idx=3, dtype=torch.bfloat16,
+                    gen=lambda dev, seed: syn.llama_inputs(device=dev, seed=seed))
+    b = int(name[-1])
+    return dict(name=f"bsweep-b{b}: B=8 Hq=8 Hkv=8 d=128 T=131072 bf16 lognormal norms, K b={b} V b={b}",
+                n_seq=8, hq=8, hkv=8, d=128, T=131072, k_idx=b - 1, v_idx=b, dtype=torch.bfloat16,
+                gen=lambda dev, seed: syn.sweep_inputs(device=dev, seed=seed))
+
+
+def key_bytes(w) -> int:
+    rec = 4 * ((w["k_idx"] * w["d"] + 31) // 32 + (w["d"] + 31) // 32)
+    return w["n_seq"] * w["hkv"] * w["T"] * (rec + 8)
+
+
+def value_bytes(w) -> int:
+    rec = 4 * ((w["v_idx"] * w["d"] + 31) // 32)
+    return w["n_seq"] * w["hkv"] * w["T"] * (rec + 4)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.t0 = self.t1 = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.strip()]
+        rows = [r for r in rows if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        # the whole sampling window brackets the timed region; prefer samples under load
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        loaded = [v for v in sm if v > 500] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows
+                                                                          if r[3].replace(".", "").isdigit())}
+
+
+# ----------------------------------------------------------------------------
+# the CUDA path
+# ----------------------------------------------------------------------------
+
+def run_tq(args, rank, world, local_rank):
+    import kv_cache_vector_quantize_b200 as tqb
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = workload(args.workload)
+    d = w["d"]
+    k, v, q = w["gen"](dev, syn.SEED_DATA + 7919 * rank)
+    Pi = syn.rotation(d).to(dev)
+    S = syn.sketch(d).to(dev)
+    ck = tqb.tq_codebook_fit(d, w["k_idx"]).to(dev)
+    cv = tqb.tq_codebook_fit(d, w["v_idx"]).to(dev)
+    SPiT = tqb.tq_sketch_rotation(Pi, S)
+    kc = tqb.PackedCache.empty(d, w["k_idx"], True, w["n_seq"], w["hkv"], w["T"], device=dev)
+    vc = tqb.PackedCache.empty(d, w["v_idx"], False, w["n_seq"], w["hkv"], w["T"], device=dev)
+    logits = torch.empty((w["n_seq"], w["hq"], w["T"]), dtype=torch.float32, device=dev)
+    out = torch.empty((w["n_seq"], w["hq"], d), dtype=torch.float32, device=dev)
+    ws_l = torch.empty(tqb.tq_logits_workspace_size(kc, w["hq"]), dtype=torch.uint8, device=dev)
+    ws_a = torch.empty(tqb.tq_attend_workspace_size(vc, w["hq"], w["T"]), dtype=torch.uint8, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
+    scale = 1.0 / math.sqrt(d)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        tqb.tq_quantize_append(kc, k, 0, Pi, SPiT, ck)
+        if ev is not None:
+            ev[1].record(stream)
+        tqb.tq_quantize_append(vc, v, 0, Pi, None, cv)
+        if ev is not None:
+            ev[2].record(stream)
+        flush.fill_(1.0)
+        if ev is not None:
+            ev[3].record(stream)
+        tqb.tq_logits(kc, q, w["T"], Pi, S, ck, logits=logits, workspace=ws_l)
+        if ev is not None:
+            ev[4].record(stream)
+        tqb.tq_attend_v(vc, logits, scale, w["T"], Pi, cv, out=out, workspace=ws_a)
+        if ev is not None:
+            ev[5].record(stream)
+
+    kernels_per_step = 6   # quantize K, quantize V, query projection, logit scan, V chunks, V merge
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    tqb.tq_workspace_status(ws_l)
+    tqb.tq_workspace_status(ws_a)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index)
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.mark_start()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.mark_end()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    per = {name: [] for name in ("quantize_k", "quantize_v", "l2_flush", "logits", "attend_v")}
+    for e in evs:
+        per["quantize_k"].append(e[0].elapsed_time(e[1]))
+        per["quantize_v"].append(e[1].elapsed_time(e[2]))
+        per["l2_flush"].append(e[2].elapsed_time(e[3]))
+        per["logits"].append(e[3].elapsed_time(e[4]))
+        per["attend_v"].append(e[4].elapsed_time(e[5]))
+    mean = {kk: sum(vv) / len(vv) for kk, vv in per.items()}
+
+    # slowest rank decides
+    t_max = torch.tensor([total_ms, mean["logits"], mean["quantize_k"] + mean["quantize_v"]], device=dev)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    total_ms, logits_ms, quant_ms = (float(x) for x in t_max.tolist())
+
+    kb, vb = key_bytes(w), value_bytes(w)
+    scan_gbs_rank = kb / (logits_ms * 1e-3) / 1e9
+    value = world * scan_gbs_rank
+    head_vectors = w["n_seq"] * w["hkv"] * w["T"]
+    quant_tps = world * w["n_seq"] * w["T"] / (quant_ms * 1e-3)
+
+    # ---- end to end: pinned host inputs in, result out, through the public API ----
+    e2e = None
+    if args.e2e_steps > 0:
+        hk = torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
+        hv = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+        hq_ = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        hk.copy_(k)
+        hv.copy_(v)
+        hq_.copy_(q)
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+
+        def step_e2e():
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            q.copy_(hq_, non_blocking=True)
+            step()
+            hout.copy_(out, non_blocking=True)
+
+        for _ in range(2):
+            step_e2e()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            step_e2e()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = torch.tensor([a.elapsed_time(b) / args.e2e_steps], device=dev)
+        if world > 1:
+            dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+        e2e_ms = float(e2e_ms.item())
+        h2d = (hk.numel() * hk.element_size() + hv.numel() * hv.element_size() + hq_.numel() * hq_.element_size())
+        e2e = {"value": world * kb / (e2e_ms * 1e-3) / 1e9, "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * hout.element_size(),
+               "note": "packed key bytes scanned per end-to-end step (pinned H2D of K, V, q; path; D2H of out)"}
+
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    sm_mhz_max = float(peaks.get("sm_max_mhz", 1965.0))
+    fp32_peak = SM_COUNT_B200 * FP32_LANES_PER_SM * 2 * sm_mhz_max * 1e6 / 1e12
+    qflops = head_vectors * (4 * d * d + 2 * d * d)
+    q_tflops = qflops / (quant_ms * 1e-3) / 1e12
+    roofline = {"kernel": "quantize_append (K and V launches)", "bound": "alu", "achieved": round(q_tflops, 3),
+                "peak": round(fp32_peak, 1), "unit": "TFLOP/s", "frac": round(q_tflops / fp32_peak, 4),
+                "traffic": NCU_TRAFFIC.get(("quantize", args.workload)),
+                "peak_source": f"FP32 FMA: {SM_COUNT_B200} SMs x {FP32_LANES_PER_SM} lanes x 2 flop x "
+                               f"{sm_mhz_max:.0f} MHz ({peak_src} max clock)",
+                "algorithmic": f"{4 * d * d} flop per key + {2 * d * d} per value (d x d projections)"}
+    roof_scan = {"kernel": "tq_logits (query projection + logit scan)", "bound": "hbm",
+                 "achieved": round(scan_gbs_rank, 1), "peak": hbm, "unit": "GB/s",
+                 "frac": round(scan_gbs_rank / hbm, 4), "traffic": NCU_TRAFFIC.get(("logits", args.workload)),
+                 "peak_source": f"hbm_gbs, {peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
+                 "algorithmic": f"{kb // (w['n_seq'] * w['hkv'] * w['T'])} B per key (record + norm + rnorm)"}
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w["name"], "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "flushed (2 x L2 write) between quantize and decode inside every step; the flush is in "
+                         "ms_per_step, not in the kernel times",
+                   "value_definition": "packed K bytes per tq_logits call / its mean device time (CUDA events), "
+                                       "summed over ranks"},
+        "quantize_tokens_per_s": round(quant_tps, 1),
+        "quantize_head_vectors_per_s": round(world * head_vectors / (quant_ms * 1e-3), 1),
+        "per_kernel_ms": {kk: round(vv, 5) for kk, vv in mean.items()},
+        "packed_bytes": {"keys": kb, "values": vb},
+        "roofline": roofline, "roofline_logit_scan": roof_scan,
+        "gpu_launches": kernels_per_step * args.steps,
+        "clocks": clk, "e2e": e2e,
+    }
+    return result, w
+
+
+# ----------------------------------------------------------------------------
+# the oracle on a bounded sample (cpu_baseline and the reference arm)
+# ----------------------------------------------------------------------------
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((p.get("num_threads", 1) for p in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return 1
+
+
+def oracle_sample_step(w, state):
+    """One bounded sample of the workload through the oracle: quantize 2048 keys and
+    2048 values of one KV head; unpack + logits of that head's query group over
+    all T keys of the head (pre-packed); softmax.V over the same head.
+    Returns (packed key bytes scanned, logit seconds, quantize seconds, head-vectors quantized)."""
+    from oracle import turboquant as otq
+
+    d = w["d"]
+    t0 = time.perf_counter()
+    ek = otq.quantize(state["k_rows"], state["Pi"], state["ck"], state["S"])
+    ev = otq.quantize(state["v_rows"], state["Pi"], state["cv"])
+    otq.pack(ek["idx"], ek["sign"], d, w["k_idx"], True)
+    otq.pack(ev["idx"], None, d, w["v_idx"], False)
+    t1 = time.perf_counter()
+    gi, gs = otq.unpack(state["krec"], d, w["k_idx"], True)
+    lg = otq.logits(state["q"], state["Pi"], state["S"], state["ck"], state["kn"], state["kr"], gi, gs)
+    t2 = time.perf_counter()
+    vi, _ = otq.unpack(state["vrec"], d, w["v_idx"], False)
+    otq.attend_v(lg, 1.0 / math.sqrt(d), state["vn"], vi, state["Pi"], state["cv"])
+    rec = 4 * ((w["k_idx"] * d + 31) // 32 + (d + 31) // 32)
+    return state["krec"].shape[0] * (rec + 8), t2 - t1, t1 - t0, state["k_rows"].shape[0]
+
+
+def oracle_state(w):
+    import numpy as np
+    from oracle import codebook as ocb
+    from oracle import turboquant as otq
+
+    d = w["d"]
+    T = w["T"]
+    G = w["hq"] // w["hkv"]
+    Pi = syn.rotation(d).double().numpy()
+    S = syn.sketch(d).double().numpy()
+    ck = ocb.fit_codebook(d, w["k_idx"])[0]
+    cv = ocb.fit_codebook(d, w["v_idx"])[0]
+    g = torch.Generator().manual_seed(5)
+    # one KV head of T keys/values of the workload's law, packed once by the oracle
+    kfull = torch.randn(T, d, generator=g).to(w["dtype"]).double().numpy()
+    vfull = torch.randn(T, d, generator=g).to(w["dtype"]).double().numpy()
+    ek = otq.quantize(kfull, Pi, ck, S)
+    ev = otq.quantize(vfull, Pi, cv)
+    return {"Pi": Pi, "S": S, "ck": ck, "cv": cv,
+            "k_rows": kfull[:2048], "v_rows": vfull[:2048],
+            "krec": otq.pack(ek["idx"], ek["sign"], d, w["k_idx"], True), "kn": ek["norm"], "kr": ek["rnorm"],
+            "vrec": otq.pack(ev["idx"], None, d, w["v_idx"], False), "vn": ev["norm"],
+            "q": torch.randn(G, d, generator=g).double().numpy()}
+
+
+def run_oracle(w, n_steps, n_warmup, budget_s=None):
+    """Returns (logit-scan GB/s, mean step seconds, steps, quantize head-vectors/s)."""
+    state = oracle_state(w)
+    for _ in range(n_warmup):
+        oracle_sample_step(w, state)
+    steps, lg_s, q_s, nbytes, nvec = [], 0.0, 0.0, 0, 0
+    t_all = time.perf_counter()
+    while True:
+        t0 = time.perf_counter()
+        b, tl, tq_, nv = oracle_sample_step(w, state)
+        steps.append(time.perf_counter() - t0)
+        lg_s += tl
+        q_s += tq_
+        nbytes += b
+        nvec += 2 * nv
+        if budget_s is None:
+            if len(steps) >= n_steps:
+                break
+        elif time.perf_counter() - t_all >= budget_s:
+            break
+    return nbytes / lg_s / 1e9, sum(steps) / len(steps), len(steps), nvec / q_s
+
+
+def sample_text(w):
+    G = w["hq"] // w["hkv"]
+    return (f"per step: oracle quantize of 2048 keys + 2048 values, unpack + logits of {G} query heads over one "
+            f"KV head's {w['T']} packed keys, softmax.V over that head (1/{w['n_seq'] * w['hkv']} of the "
+            f"workload's decode); value = that head's packed key bytes / oracle logit time (unpack + estimator)")
+
+
+# ----------------------------------------------------------------------------
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = workload(args.workload)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        val, step_s, n, qvps = run_oracle(w, args.steps, args.warmup)
+        cores = _threads()
+        line = {"metric": METRIC, "value": round(val, 6), "unit": UNIT, "n_gpus": args.gpus, "steps": n,
+                "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 2), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {"workload": w["name"], "parallelism": "single"},
+                "quantize_head_vectors_per_s": round(qvps, 1),
+                "cpu_baseline": {"value": round(val, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+                                 "sample": sample_text(w)},
+                "e2e": {"value": round(val, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    result, w = run_tq(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, step_s, n, qvps = run_oracle(w, 0, 1, budget_s=12.0)
+        result["cpu_baseline"] = {"value": round(val, 6), "unit": UNIT, "cores": _threads(), "kind": "oracle",
+                                  "quantize_head_vectors_per_s": round(qvps, 1),
+                                  "sample": sample_text(w) + f"; {n} steps of {step_s:.2f} s"}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -230,12 +230,12 @@ tq_status tq_logits(const tq_cache *k, const float *q, int32_t n_q_heads, int64_
   if (n_tokens < 0 || n_tokens > k->capacity)
     return fail(TQ_ERR_CAPACITY, "tq_logits: n_tokens=%lld outside [0, capacity=%lld]", (long long)n_tokens,
                 (long long)k->capacity);
+  if (n_tokens == 0) return TQ_OK;   // nothing to scan (logits may be an empty, NULL tensor)
   if (!q || !Pi || !S || !codebook || !logits) return fail(TQ_ERR_INVALID, "tq_logits: NULL tensor argument");
   const size_t need = tq_logits_workspace_size(k, n_q_heads);
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < need)
     return fail(TQ_ERR_WORKSPACE, "tq_logits: workspace needs %zu bytes, 256-byte aligned (got %zu)", need,
                 workspace_bytes);
-  if (n_tokens == 0) return TQ_OK;
   const LogitsPlan pl = plan_logits(k, n_q_heads, n_tokens);
   if (pl.q_per_cta < 1)
     return fail(TQ_ERR_UNSUPPORTED, "tq_logits: lookup tables for d=%d idx_bits=%d exceed shared memory", k->d,
@@ -289,7 +289,8 @@ tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale, int32
   if (n_tokens < 0 || n_tokens > v->capacity)
     return fail(TQ_ERR_CAPACITY, "tq_attend_v: n_tokens=%lld outside [0, capacity=%lld]", (long long)n_tokens,
                 (long long)v->capacity);
-  if (!logits || !Pi || !codebook || !out) return fail(TQ_ERR_INVALID, "tq_attend_v: NULL tensor argument");
+  if ((!logits && n_tokens > 0) || !Pi || !codebook || !out)
+    return fail(TQ_ERR_INVALID, "tq_attend_v: NULL tensor argument");
   if (!(scale == scale) || scale == INFINITY || scale == -INFINITY) return fail(TQ_ERR_INVALID, "tq_attend_v: scale is not finite");
   const size_t need = tq_attend_workspace_size(v, n_q_heads, n_tokens);
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < need)

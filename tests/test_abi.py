@@ -100,7 +100,7 @@ def test_logits_argument_checks():
     assert _lg(_desc(cap=64), n=65) == tqb.TQ_ERR_CAPACITY
     assert _lg(_desc(), ws=FAKE + 16) == tqb.TQ_ERR_WORKSPACE
     assert _lg(_desc(), ws_bytes=16) == tqb.TQ_ERR_WORKSPACE
-    assert _lg(_desc(), n=0) == tqb.TQ_OK
+    assert _lg(_desc(), n=0) == tqb.TQ_OK                           # nothing to scan
     assert _lg(_desc()) == tqb.TQ_ERR_CUDA                         # passes the checks -> injected
     assert lib.tq_logits_workspace_size(ctypes.byref(_desc()), 4) == 256 + 2 * 4 * 4 * 128
 

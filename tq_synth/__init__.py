@@ -34,7 +34,7 @@ def rotation(d: int, seed: int = SEED_PI) -> torch.Tensor:
     a = torch.randn(d, d, generator=_gen(seed), dtype=torch.float64)
     q, r = torch.linalg.qr(a)
     q = q * torch.sign(torch.diagonal(r))[None, :]
-    return q.to(torch.float32)
+    return q.to(torch.float32).contiguous()
 
 
 def sketch(d: int, seed: int = SEED_S) -> torch.Tensor:
