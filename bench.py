@@ -47,9 +47,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0
 SM_COUNT_B200 = 148
 FP32_LANES_PER_SM = 128
 
-# DRAM bytes per launch from ncu captures of the current kernels (None until
-# captured for the kernel as it stands). Keys: (kernel, workload).
-NCU_TRAFFIC = {}
+# DRAM bytes (read + write) per launch from one ncu --set full capture of the
+# kernels as they stand (profiles/*_llama3-8b-decode.md); a key is removed when
+# its kernel changes. Keys: (kernel, workload).
+NCU_TRAFFIC = {
+    ("quantize", "llama"): 67_361_536 + 3_891_456,   # key launch (quantize_kernel<128, 1, bf16>)
+    ("logits", "llama"): 14_728_448 + 0,             # logits_kernel<2>
+}
 
 
 def parse():
