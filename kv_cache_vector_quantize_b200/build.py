@@ -1,7 +1,7 @@
 """Build libtq.so (the C-ABI CUDA library) in-tree for sm_100a.
 
-Usage: ``python -m kv_cache_vector_quantize_b200.build`` (or ``build()`` from
-Python). Sources are compiled in parallel into ``_build/`` and linked into
+Usage: ``python kv_cache_vector_quantize_b200/build.py`` (run by path: the
+package itself loads the library this script builds). Sources are compiled in parallel into ``_build/`` and linked into
 ``kv_cache_vector_quantize_b200/libtq.so``; a source is recompiled only when it
 or a header is newer than its object file.
 """
