@@ -164,6 +164,35 @@ const char *tq_last_error(void);
  * work return `status` instead, before any launch. count = 0 disarms. */
 void tq_debug_inject(tq_status status, int32_t count);
 
+/* Size of the library's built-in scratch array used by tq_attend_v_noalloc:
+ * 4 MiB of device memory, held on every GPU that loads this library until the
+ * process exits. */
+#define TQ_ATTEND_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+
+/* tq_attend_v without a caller workspace (the pages have no counterpart: this
+ * is a deployment convenience of this library).
+ *
+ * For callers that cannot allocate device memory themselves: code that runs
+ * inside a host framework which owns every byte of device memory through its
+ * own pool and hands plugins no scratch buffer, or a latency-critical decode
+ * loop that must not call cudaMalloc (which can synchronise the device).
+ * Arguments and results are those of tq_attend_v; the scratch space comes from
+ * a fixed array compiled into the library (TQ_ATTEND_NOALLOC_SCRATCH_BYTES).
+ *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Returns TQ_ERR_WORKSPACE, before any launch, when
+ *     tq_attend_workspace_size(v, n_q_heads, n_tokens) exceeds the array.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents: two calls whose work can overlap on the GPU (different
+ *     streams, or different host threads) race and corrupt each other's
+ *     results. Serialise them on one stream. */
+tq_status tq_attend_v_noalloc(const tq_cache *v, const float *logits, float scale,
+                              int32_t n_q_heads, int64_t n_tokens,
+                              const float *Pi, const float *codebook, float *out,
+                              tq_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -42,7 +42,7 @@ class TqCacheDesc(ctypes.Structure):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m kv_cache_vector_quantize_b200.build` "
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python kv_cache_vector_quantize_b200/build.py` "
                           "(the CUDA library is the only implementation)")
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, I64, SZ, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -56,6 +56,7 @@ def _load() -> ctypes.CDLL:
         "tq_logits": (I32, [D, P, I32, I64, P, P, P, P, P, SZ, P]),
         "tq_attend_workspace_size": (SZ, [D, I32, I64]),
         "tq_attend_v": (I32, [D, P, F, I32, I64, P, P, P, P, SZ, P]),
+        "tq_attend_v_noalloc": (I32, [D, P, F, I32, I64, P, P, P, P]),
         "tq_workspace_status": (I32, [P, P]),
         "tq_last_error": (ctypes.c_char_p, []),
         "tq_debug_inject": (None, [I32, I32]),

@@ -15,6 +15,9 @@
 // (the codes of a token are read once and reused by every query head of the
 // group). Merge kernel: M = max_c m_c, L = sum_c l_c e^{m_c - M},
 // A = sum_c acc_c e^{m_c - M}, out = Pi^T A / L.
+#include <cstdio>
+#include <mutex>
+
 #include "common.cuh"
 
 namespace tq {
@@ -169,3 +172,70 @@ cudaError_t launch_combine(const float *partial, int rows, int n_chunks, int d, 
 }
 
 }  // namespace tq
+
+// ---------------------------------------------------------------------------
+// tq_attend_v_noalloc: softmax.V whose scratch lives in a fixed device array of
+// this library, for callers that cannot allocate device memory (see tq.h).
+// ---------------------------------------------------------------------------
+
+namespace tq {
+
+namespace {
+
+// Scratch for the chunk partials and the status word of tq_attend_v. Every
+// call on a device uses this one array; it is not cleared between calls (the
+// status word is reset by every call and every partial a call reads was
+// written by that same call).
+static __device__ __align__(256) unsigned char g_attend_scratch[TQ_ATTEND_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kScratchMaxDevices = 64;
+void *g_scratch_addr[kScratchMaxDevices] = {nullptr};
+std::mutex g_scratch_mutex;
+
+// Device address of g_attend_scratch on the current device (looked up once per
+// device; the host-side symbol is only a stand-in and must never reach a kernel).
+tq_status scratch_address(void **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    char msg[256];
+    snprintf(msg, sizeof msg, "tq_attend_v_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+    return report_error(TQ_ERR_CUDA, msg);
+  }
+  if (dev < 0 || dev >= kScratchMaxDevices) return report_error(TQ_ERR_UNSUPPORTED, "tq_attend_v_noalloc: device index too large");
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_attend_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      char msg[256];
+      snprintf(msg, sizeof msg, "tq_attend_v_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+      return report_error(TQ_ERR_CUDA, msg);
+    }
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return TQ_OK;
+}
+
+}  // namespace
+
+}  // namespace tq
+
+extern "C" tq_status tq_attend_v_noalloc(const tq_cache *v, const float *logits, float scale, int32_t n_q_heads,
+                                         int64_t n_tokens, const float *Pi, const float *codebook, float *out,
+                                         tq_stream stream) {
+  const size_t need = tq_attend_workspace_size(v, n_q_heads, n_tokens);
+  if (need > TQ_ATTEND_NOALLOC_SCRATCH_BYTES) {
+    char msg[256];
+    snprintf(msg, sizeof msg,
+             "tq_attend_v_noalloc: this shape needs %zu bytes of scratch but the built-in array holds %zu; "
+             "use tq_attend_v with a caller workspace", need, (size_t)TQ_ATTEND_NOALLOC_SCRATCH_BYTES);
+    return tq::report_error(TQ_ERR_WORKSPACE, msg);
+  }
+  void *scratch = nullptr;
+  tq_status s = tq::scratch_address(&scratch);
+  if (s != TQ_OK) return s;
+  return tq_attend_v(v, logits, scale, n_q_heads, n_tokens, Pi, codebook, out, scratch,
+                     TQ_ATTEND_NOALLOC_SCRATCH_BYTES, stream);
+}

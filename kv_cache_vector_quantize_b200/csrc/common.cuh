@@ -122,5 +122,6 @@ int device_sm_count();
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device).
 cudaError_t set_smem_once(const void *kernel, size_t bytes);
 size_t device_smem_optin();
+tq_status report_error(tq_status s, const char *msg);
 
 }  // namespace tq

@@ -145,6 +145,9 @@ cudaError_t set_smem_once(const void *kernel, size_t bytes) {
   return cudaSuccess;
 }
 
+// Record a failure message for tq_last_error() from another translation unit.
+tq_status report_error(tq_status s, const char *msg) { return fail(s, "%s", msg); }
+
 }  // namespace tq
 
 using namespace tq;
