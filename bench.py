@@ -62,7 +62,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
-    ap.add_argument("--workload", default="llama", choices=["llama", "sweep-b2", "sweep-b3", "sweep-b4"])
+    ap.add_argument("--workload", default="llama",
+                    choices=["llama"] + [f"sweep-b{b}{s}" for b in (2, 3, 4) for s in ("", "-s4")])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -77,10 +78,13 @@ def workload(name: str):
         return dict(name="llama3-8b-decode: B=1 Hq=32 Hkv=8 d=128 T=32768 bf16 K b=3 (2-bit codes+QJL) V b=3 MSE",
                     n_seq=1, hq=32, hkv=8, d=128, T=32768, k_idx=2, v_idx=3, dtype=torch.bfloat16,
                     gen=lambda dev, seed: syn.llama_inputs(device=dev, seed=seed))
-    b = int(name[-1])
-    return dict(name=f"bsweep-b{b}: B=8 Hq=8 Hkv=8 d=128 T=131072 bf16 lognormal norms, K b={b} V b={b}",
-                n_seq=8, hq=8, hkv=8, d=128, T=131072, k_idx=b - 1, v_idx=b, dtype=torch.bfloat16,
-                gen=lambda dev, seed: syn.sweep_inputs(device=dev, seed=seed))
+    # "sweep-b3" is the full b-sweep cache; "sweep-b3-s4" keeps 4 of its 8 sequences
+    # (a profiling size: still larger than L2, half the device memory)
+    b = int(name.split("-")[1][1:])
+    B = 4 if name.endswith("-s4") else 8
+    return dict(name=f"bsweep-b{b}: B={B} Hq=8 Hkv=8 d=128 T=131072 bf16 lognormal norms, K b={b} V b={b}",
+                n_seq=B, hq=8, hkv=8, d=128, T=131072, k_idx=b - 1, v_idx=b, dtype=torch.bfloat16,
+                gen=lambda dev, seed: syn.sweep_inputs(n_seq=B, device=dev, seed=seed))
 
 
 def key_bytes(w) -> int:
@@ -222,6 +226,8 @@ def run_tq(args, rank, world, local_rank):
     t_end.record(stream)
     torch.cuda.synchronize(dev)
     clocks.mark_end()
+    tqb.tq_workspace_status(ws_l)   # raises if a kernel of the timed region reported a failure
+    tqb.tq_workspace_status(ws_a)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()

@@ -103,6 +103,27 @@ LogitsPlan plan_logits(const tq_cache *k, int n_q_heads, int64_t n_tokens) {
   return pl;
 }
 
+// Launch shape of the d = 128 table scan: one CTA per SM; two query heads per
+// CTA when their tables leave room for at least three stages, else one.
+struct FastPlan {
+  bool use;
+  int q_per_cta;
+  size_t limit;
+};
+
+FastPlan plan_fast(const tq_cache *k, int n_q_heads) {
+  FastPlan f{false, 0, 0};
+  if (k->d != 128 || k->idx_bits > 3 || !k->qjl) return f;
+  const int group = n_q_heads / k->n_kv_heads;
+  const size_t limit = device_smem_optin() - 1024;
+  int q = 0;
+  if (group >= 2 && logits_fast_stages(k->idx_bits, 2, limit) >= 3) q = 2;
+  else if (logits_fast_stages(k->idx_bits, 1, limit) >= 2) q = 1;
+  if (q == 0) return f;
+  f = FastPlan{true, q, limit};
+  return f;
+}
+
 constexpr int64_t kAttendChunk = 512;
 constexpr int kAttendMaxQ = 8;
 
@@ -239,8 +260,9 @@ tq_status tq_logits(const tq_cache *k, const float *q, int32_t n_q_heads, int64_
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < need)
     return fail(TQ_ERR_WORKSPACE, "tq_logits: workspace needs %zu bytes, 256-byte aligned (got %zu)", need,
                 workspace_bytes);
+  const FastPlan fpl = plan_fast(k, n_q_heads);
   const LogitsPlan pl = plan_logits(k, n_q_heads, n_tokens);
-  if (pl.q_per_cta < 1)
+  if (!fpl.use && pl.q_per_cta < 1)
     return fail(TQ_ERR_UNSUPPORTED, "tq_logits: lookup tables for d=%d idx_bits=%d exceed shared memory", k->d,
                 k->idx_bits);
   if (injected(&s)) return s;
@@ -267,6 +289,12 @@ tq_status tq_logits(const tq_cache *k, const float *q, int32_t n_q_heads, int64_
   p.n_kv_heads = k->n_kv_heads;
   p.n_q_heads = n_q_heads;
   p.group = n_q_heads / k->n_kv_heads;
+  if (fpl.use) {
+    p.q_per_cta = fpl.q_per_cta;
+    p.qblocks = (p.group + fpl.q_per_cta - 1) / fpl.q_per_cta;
+    e = launch_logits_fast(p, k->idx_bits, k->n_seq, fpl.limit, (cudaStream_t)stream);
+    return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_logits (table scan)");
+  }
   p.q_per_cta = pl.q_per_cta;
   p.qblocks = pl.qblocks;
   e = launch_logits(p, k->idx_bits, k->n_seq, pl.n_chunks, pl.smem, (cudaStream_t)stream);

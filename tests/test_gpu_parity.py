@@ -55,10 +55,15 @@ def _run_path(k, v, q, d, k_idx_bits, v_bits, g, capacity=None, scale=None):
     vc = tqb.PackedCache.empty(d, v_bits, False, n_seq, hkv, cap)
     tqb.tq_quantize_append(kc, k.cuda(), 0, g["Pi"], g["SPiT"], g["ck"])
     tqb.tq_quantize_append(vc, v.cuda(), 0, g["Pi"], None, g["cv"])
-    lg = tqb.tq_logits(kc, q.cuda(), T, g["Pi"], g["S"], g["ck"])
+    ws_l = torch.empty(max(256, tqb.tq_logits_workspace_size(kc, q.shape[1])), dtype=torch.uint8, device="cuda")
+    ws_a = torch.empty(max(256, tqb.tq_attend_workspace_size(vc, q.shape[1], T)), dtype=torch.uint8, device="cuda")
+    lg = tqb.tq_logits(kc, q.cuda(), T, g["Pi"], g["S"], g["ck"], workspace=ws_l)
     sc = 1.0 / math.sqrt(d) if scale is None else scale
-    out = tqb.tq_attend_v(vc, lg, sc, T, g["Pi"], g["cv"])
+    out = tqb.tq_attend_v(vc, lg, sc, T, g["Pi"], g["cv"], workspace=ws_a)
     torch.cuda.synchronize()
+    if T > 0:
+        tqb.tq_workspace_status(ws_l)
+        tqb.tq_workspace_status(ws_a)
     return kc, vc, lg, out, sc
 
 
@@ -248,8 +253,10 @@ def test_bsweep_full_size_sampled(bits):
     vc = tqb.PackedCache.empty(d, bits, False, B, H, T)
     tqb.tq_quantize_append(kc, k, 0, g["Pi"], g["SPiT"], g["ck"])
     tqb.tq_quantize_append(vc, v, 0, g["Pi"], None, g["cv"])
-    lg = tqb.tq_logits(kc, q, T, g["Pi"], g["S"], g["ck"])
+    ws = torch.empty(tqb.tq_logits_workspace_size(kc, H), dtype=torch.uint8, device="cuda")
+    lg = tqb.tq_logits(kc, q, T, g["Pi"], g["S"], g["ck"], workspace=ws)
     torch.cuda.synchronize()
+    tqb.tq_workspace_status(ws)
     del v
     rng = np.random.default_rng(100 + bits)
     for _ in range(4):
