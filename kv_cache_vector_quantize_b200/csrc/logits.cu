@@ -25,20 +25,55 @@ namespace {
 
 constexpr int kLThreads = 256;
 
-__global__ void qprep_kernel(const float *__restrict__ q, int d, const float *__restrict__ Pi,
-                             const float *__restrict__ S, float *__restrict__ qrot, float *__restrict__ qsk,
-                             uint32_t *status) {
-  __shared__ float qs[kMaxD];
-  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (row == 0 && tid == 0) *status = 0u;   // this call's kernels report into a clean word
-  for (int k = tid; k < d; k += blockDim.x) qs[k] = q[(size_t)row * d + k];
-  __syncthreads();
-  for (int o = warp; o < 2 * d; o += blockDim.x / 32) {
-    const float *mrow = (o < d ? Pi : S) + (size_t)(o < d ? o : o - d) * d;
+// Pi q and S q for every query head: block (row, 32-output chunk); each warp
+// produces 8 outputs, each lane holding 4 consecutive q values and reading the
+// matching 4 matrix entries of a row with one vector load, so a warp's 8 rows
+// are in flight together.
+constexpr int kQpOut = 32;   // outputs per block
+__global__ void __launch_bounds__(128) qprep_kernel(const float *__restrict__ q, int d, const float *__restrict__ Pi,
+                                                    const float *__restrict__ S, float *__restrict__ qrot,
+                                                    float *__restrict__ qsk, uint32_t *status) {
+  const int row = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (row == 0 && chunk == 0 && tid == 0) *status = 0u;   // this call's kernels report into a clean word
+  const float *qr = q + (size_t)row * d;
+  // lane covers k in [4 lane, 4 lane + 4) and, for d > 128, [128 + 4 lane, ...)
+  float4 qv[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int k = 128 * h + 4 * lane;
+    qv[h] = make_float4(k < d ? qr[k] : 0.f, k + 1 < d ? qr[k + 1] : 0.f, k + 2 < d ? qr[k + 2] : 0.f,
+                        k + 3 < d ? qr[k + 3] : 0.f);
+  }
+  const bool vec = (d & 3) == 0 && ((reinterpret_cast<uintptr_t>(Pi) | reinterpret_cast<uintptr_t>(S)) & 15) == 0;
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int o = chunk * kQpOut + warp * 8 + j;   // output index in [0, 2d)
     float s = 0.f;
-    for (int k = lane; k < d; k += 32) s = fmaf(__ldg(mrow + k), qs[k], s);
-    s = warp_sum(s);
-    if (lane == 0) (o < d ? qrot : qsk)[(size_t)row * d + (o < d ? o : o - d)] = s;
+    if (o < 2 * d) {
+      const float *mrow = (o < d ? Pi : S) + (size_t)(o < d ? o : o - d) * d;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int k = 128 * h + 4 * lane;
+        if (vec && k + 3 < d) {
+          const float4 m = __ldg(reinterpret_cast<const float4 *>(mrow + k));
+          s = fmaf(m.x, qv[h].x, fmaf(m.y, qv[h].y, fmaf(m.z, qv[h].z, fmaf(m.w, qv[h].w, s))));
+        } else {
+          for (int c = 0; c < 4; ++c)
+            if (k + c < d) s = fmaf(__ldg(mrow + k + c), (&qv[h].x)[c], s);
+        }
+      }
+    }
+    acc[j] = s;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = warp_sum(acc[j]);
+  if (lane < 8) {
+    float v = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) if (j == lane) v = acc[j];
+    const int o = chunk * kQpOut + warp * 8 + lane;
+    if (o < 2 * d) (o < d ? qrot : qsk)[(size_t)row * d + (o < d ? o : o - d)] = v;
   }
 }
 
@@ -131,7 +166,8 @@ size_t logits_smem_per_query(int d, int bits) {
 
 cudaError_t launch_qprep(const float *q, int rows, int d, const float *Pi, const float *S, float *qrot, float *qsk,
                          uint32_t *status, cudaStream_t st) {
-  qprep_kernel<<<rows, 256, 0, st>>>(q, d, Pi, S, qrot, qsk, status);
+  dim3 grid((2 * d + kQpOut - 1) / kQpOut, rows);
+  qprep_kernel<<<grid, 128, 0, st>>>(q, d, Pi, S, qrot, qsk, status);
   return cudaGetLastError();
 }
 

@@ -133,17 +133,19 @@ __device__ __forceinline__ uint32_t key_addr7(const uint32_t (&r)[N], int pos, u
   return (shifted & mask) | bank;
 }
 
-// One query head's logit for a byte-key record (1 or 2 code bits), tables at T0 + QQ * 64 KB.
+// One query head's logit for a byte-key record (1 or 2 code bits), tables at
+// T0 + QQ * 64 KB. xi[m] / xs[m] hold, per lane, the table-base bytes 2..3 and
+// the row positions (l ^ s) * 4 of steps s = 2m and 2m + 1 in bytes 0 and 1, so
+// one byte-permute yields the whole address T0 | key << 8 | position.
 template <int BETA, int QQ>
 __device__ __forceinline__ float scan_bytes(const uint32_t (&wi)[BETA * 4], const uint32_t (&wsg)[4],
-                                            const uint32_t (&sel)[4], uint32_t T0, uint32_t lane4, float nrm,
-                                            float rho) {
+                                            const uint32_t (&sel)[4], const uint32_t (&xi)[BETA * 8],
+                                            const uint32_t (&xs)[8], float nrm, float rho) {
   constexpr int NI = BETA == 1 ? 16 : 32;
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, b0 = 0.f, b1 = 0.f;
 #pragma unroll
   for (int st = 0; st < NI; ++st) {
-    const uint32_t row = __byte_perm(wi[st >> 2], T0, sel[st & 3]);   // T0 | key << 8
-    const float v = lds_at<QQ * kTabStride>(row | (lane4 ^ (uint32_t)(st << 2)));
+    const float v = lds_at<QQ * kTabStride>(__byte_perm(wi[st >> 2], xi[st >> 1], sel[st & 3]));
     if ((st & 3) == 0) a0 += v;
     else if ((st & 3) == 1) a1 += v;
     else if ((st & 3) == 2) a2 += v;
@@ -151,8 +153,7 @@ __device__ __forceinline__ float scan_bytes(const uint32_t (&wi)[BETA * 4], cons
   }
 #pragma unroll
   for (int st = 0; st < 16; ++st) {
-    const uint32_t row = __byte_perm(wsg[st >> 2], T0, sel[st & 3]);
-    const float v = lds_at<QQ * kTabStride>(row | (lane4 ^ (uint32_t)(128 | (st << 2))));
+    const float v = lds_at<QQ * kTabStride>(__byte_perm(wsg[st >> 2], xs[st >> 1], sel[st & 3]));
     if (st & 1) b1 += v;
     else b0 += v;
   }
@@ -387,11 +388,20 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
 #pragma unroll
     for (int qq = 0; qq < QMAX; ++qq) out[qq] = 0.f;
     if constexpr (BETA != 3) {
-      // byte-permute selectors: byte (j ^ (l & 3)) of a record word into bits 8..15,
-      // table-base bytes 2..3 of T0 into bits 16..31, zero into bits 0..7
+      // byte-permute selectors for step s (j = s mod 4): result byte 0 = position byte
+      // (s mod 2) of the x register, byte 1 = key byte (j ^ (l & 3)) of the record
+      // word, bytes 2..3 = table-base bytes 2..3 of the x register
       uint32_t sel[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) sel[j] = 0x7604u | ((uint32_t)(j ^ (lane & 3)) << 4);
+      for (int j = 0; j < 4; ++j) sel[j] = 0x7600u | (uint32_t)(4 + (j & 1)) | ((uint32_t)(j ^ (lane & 3)) << 4);
+      uint32_t xi[BETA * 8], xs[8];
+#pragma unroll
+      for (int m = 0; m < BETA * 8; ++m)
+        xi[m] = (T0 & 0xFFFF0000u) | ((uint32_t)(lane ^ (2 * m)) << 2) | ((uint32_t)(lane ^ (2 * m + 1)) << 10);
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        xs[m] = (T0 & 0xFFFF0000u) | (128u | ((uint32_t)(lane ^ (2 * m)) << 2)) |
+                ((128u | ((uint32_t)(lane ^ (2 * m + 1)) << 2)) << 8);
       uint32_t wi[IW], wsg[4];
 #pragma unroll
       for (int j = 0; j < IW; ++j) wi[j] = w[j];
@@ -399,9 +409,9 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
       for (int j = 0; j < 4; ++j) wsg[j] = w[IW + j];
       xor_permute<IW>(wi, (lane >> 2) & (IW - 1));
       xor_permute<4>(wsg, (lane >> 2) & 3);
-      out[0] = scan_bytes<BETA, 0>(wi, wsg, sel, T0, lane4, nrm, rho);
+      out[0] = scan_bytes<BETA, 0>(wi, wsg, sel, xi, xs, nrm, rho);
       if constexpr (QMAX > 1)
-        if (nq > 1) out[1] = scan_bytes<BETA, 1>(wi, wsg, sel, T0, lane4, nrm, rho);
+        if (nq > 1) out[1] = scan_bytes<BETA, 1>(wi, wsg, sel, xi, xs, nrm, rho);
     } else {
       uint32_t bank[32];   // T0 | position offset ((s + l) mod 32, times 4)
 #pragma unroll
