@@ -262,6 +262,9 @@ __global__ void sketch_rotation_kernel(int d, const float *__restrict__ Pi, cons
 }  // namespace
 
 cudaError_t launch_quantize(const QuantParams &p, int bits, bool qjl, tq_dtype dtype, cudaStream_t st) {
+  // bf16 heads of 128 with 16-byte aligned rows take the tensor-core kernel (quantize_tc.cu)
+  if (p.d == 128 && dtype == TQ_BF16 && (reinterpret_cast<uintptr_t>(p.x) & 15) == 0)
+    return launch_quantize_tc(p, bits, qjl, st);
   if (p.d <= 32) return launch_q_dp<32>(p, bits, qjl, dtype, st);
   if (p.d <= 64) return launch_q_dp<64>(p, bits, qjl, dtype, st);
   if (p.d <= 128) return launch_q_dp<128>(p, bits, qjl, dtype, st);

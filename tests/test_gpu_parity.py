@@ -123,6 +123,10 @@ SHAPES = [
     (256, 3, 4, 1, 1, 2, 300, torch.bfloat16),
     (128, 1, 2, 1, 2, 4, 1, torch.float32),
     (96, 2, 2, 3, 1, 3, 513, torch.float32),
+    # bf16 heads of 128 take the tensor-core quantizer: ragged tails, all code widths
+    (128, 3, 4, 2, 2, 1, 901, torch.bfloat16),
+    (128, 1, 2, 1, 3, 2, 130, torch.bfloat16),
+    (128, 2, 1, 1, 1, 4, 257, torch.bfloat16),
 ]
 
 
@@ -151,8 +155,9 @@ def test_append_in_parts_equals_one_call():
     assert torch.equal(one.norm, parts.norm) and torch.equal(one.rnorm, parts.rnorm)
 
 
-def test_special_vectors():
-    # zero vectors, codeword directions, tiny and huge norms
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_special_vectors(dtype):
+    # zero vectors, codeword directions, tiny and huge norms (bf16: the tensor-core path)
     d, kb = 128, 2
     Pi, S, ck, cv, g = _setup(d, kb, 3)
     rng = np.random.default_rng(5)
@@ -162,7 +167,7 @@ def test_special_vectors():
         w = c[rng.integers(0, 4, size=d)]
         rows.append(3.0 * (w @ Pi.astype(np.float64)) / np.linalg.norm(w))
     rows += [1e-20 * rng.standard_normal(d), 1e20 * rng.standard_normal(d), np.ones(d), -np.ones(d)]
-    x = torch.tensor(np.array(rows), dtype=torch.float32).reshape(1, 1, -1, d)
+    x = torch.tensor(np.array(rows), dtype=torch.float32).reshape(1, 1, -1, d).to(dtype)
     kc = tqb.PackedCache.empty(d, kb, True, 1, 1, x.shape[2])
     tqb.tq_quantize_append(kc, x.cuda(), 0, g["Pi"], g["SPiT"], g["ck"])
     torch.cuda.synchronize()
