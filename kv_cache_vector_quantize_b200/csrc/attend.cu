@@ -25,7 +25,7 @@ namespace tq {
 namespace {
 
 constexpr int kAThreads = 256;
-constexpr int kAMaxQ = 8;   // query heads per CTA (register accumulators)
+constexpr int kAMaxQ = 4;   // query heads per CTA (one 16-byte weight load per token)
 
 __device__ __forceinline__ float block_reduce(float v, float *red, bool is_max) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -38,27 +38,52 @@ __device__ __forceinline__ float block_reduce(float v, float *red, bool is_max) 
   return r;
 }
 
+// Shared memory of the chunk kernel: the chunk's records, the weights w[t][4],
+// the codebook, a reduction scratch and the per-phase accumulators.
+size_t chunk_smem(int d, int bits, int64_t chunk) {
+  const int rw = (bits * d + 31) / 32;
+  const int phases = kAThreads / (d / 4);
+  return (size_t)chunk * rw * 4 + (size_t)chunk * 4 * 4 + (16 + 32) * 4 + (size_t)phases * 4 * d * 4;
+}
+
+// One CTA per (token chunk, sequence, KV head, query block of <= 4 heads).
+// Softmax statistics of the chunk, then each thread owns 4 consecutive
+// coordinates of one token phase: per token it reads the code bits of its 4
+// coordinates once, looks up their centroids and updates 4 x (query heads)
+// accumulators with one 16-byte weight load. Phases are summed in a fixed
+// order (deterministic).
 template <int BITS>
 __global__ void __launch_bounds__(kAThreads) attend_chunk_kernel(const AttendParams p) {
   constexpr int L = 1 << BITS;
   extern __shared__ __align__(16) float sm[];
-  float *w = sm;                                   // [q_per_cta][chunk]
-  float *cbs = w + (size_t)p.q_per_cta * p.chunk;  // [16]
-  float *red = cbs + 16;                           // [32]
-  float *accs = red + 32;                          // [q_per_cta][d] split reduction
+  const int d = p.d, rw = p.rec_words;
+  uint32_t *rec_s = reinterpret_cast<uint32_t *>(sm);          // [chunk][rw]
+  float4 *w_s = reinterpret_cast<float4 *>(sm + p.chunk * rw);  // [chunk] (one lane per query head)
+  float *cbs = reinterpret_cast<float *>(w_s + p.chunk);         // [16]
+  float *red = cbs + 16;                                         // [32]
+  float *accs = red + 32;                                        // [phases][4][d]
   const int tid = threadIdx.x;
   const int qb = blockIdx.y % p.qblocks;
   const int sk = blockIdx.y / p.qblocks;
   const int seq = sk / p.n_kv_heads, kvh = sk - seq * p.n_kv_heads;
   const int h0 = kvh * p.group + qb * p.q_per_cta;
   const int nq = min(p.q_per_cta, p.group - qb * p.q_per_cta);
-  const int c = blockIdx.x, d = p.d;
+  const int c = blockIdx.x;
   const int64_t t0 = (int64_t)c * p.chunk;
   const int nt = (int)min((int64_t)p.chunk, p.n_tokens - t0);
   const size_t slot0 = (size_t)sk * p.capacity + t0;
 
   if (tid < L) cbs[tid] = p.codebook[tid];
-  for (int qq = 0; qq < nq; ++qq) {
+  // the chunk's records (contiguous in the cache) into shared memory
+  const uint32_t *src = p.records + slot0 * rw;
+  for (int e = tid; e < nt * rw; e += kAThreads) rec_s[e] = __ldg(src + e);
+  // softmax statistics per query head, weights w_t = exp(scale l_t - m) n_t
+  for (int qq = 0; qq < 4; ++qq) {
+    float *wq = reinterpret_cast<float *>(w_s) + qq;
+    if (qq >= nq) {
+      for (int t = tid; t < nt; t += kAThreads) wq[4 * t] = 0.f;
+      continue;
+    }
     const size_t hrow = (size_t)seq * p.n_q_heads + h0 + qq;
     const float *lg = p.logits + hrow * p.n_tokens + t0;
     float m = -INFINITY;
@@ -68,7 +93,7 @@ __global__ void __launch_bounds__(kAThreads) attend_chunk_kernel(const AttendPar
     for (int t = tid; t < nt; t += kAThreads) {
       const float e = expf(p.scale * lg[t] - m);
       s += e;
-      w[qq * p.chunk + t] = e * __ldg(p.norm + slot0 + t);
+      wq[4 * t] = e * __ldg(p.norm + slot0 + t);
     }
     s = block_reduce(s, red, false);
     if (tid == 0) {
@@ -79,41 +104,52 @@ __global__ void __launch_bounds__(kAThreads) attend_chunk_kernel(const AttendPar
   }
   __syncthreads();
 
-  // one thread per coordinate; several token phases when d is small
-  const int dpad = (d + 31) & ~31;
-  const int nsplit = kAThreads / dpad;
-  const int i = tid % dpad, split = tid / dpad;
-  float acc[kAMaxQ];
+  // accumulate: thread = (token phase, group of 4 coordinates)
+  const int npt = d / 4, phases = kAThreads / npt;
+  const int ph = tid / npt, i0 = 4 * (tid - ph * npt);
+  float acc[4][4];
 #pragma unroll
-  for (int qq = 0; qq < kAMaxQ; ++qq) acc[qq] = 0.f;
-  if (split < nsplit && i < d) {
-    for (int t = split; t < nt; t += nsplit) {
-      const uint32_t *rec = p.records + (slot0 + t) * p.rec_words;
-      const float cv = cbs[stream_bits(rec, BITS * i, BITS, p.rec_words)];
+  for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int qq = 0; qq < kAMaxQ; ++qq)
-        if (qq < nq) acc[qq] = fmaf(w[qq * p.chunk + t], cv, acc[qq]);
-    }
-  }
-  // reduce the token phases through shared memory
-  for (int s = 0; s < nsplit; ++s) {
-    if (split == s && i < d) {
-      for (int qq = 0; qq < nq; ++qq) {
-        float *a = accs + qq * d + i;
-        *a = (s == 0) ? acc[qq] : *a + acc[qq];
+    for (int qq = 0; qq < 4; ++qq) acc[a][qq] = 0.f;
+  if (ph < phases) {
+    const int bit0 = BITS * i0, wd = bit0 >> 5, sh = bit0 & 31;
+    const bool two = sh + 4 * BITS > 32 && wd + 1 < rw;
+    for (int t = ph; t < nt; t += phases) {
+      const uint32_t *rec = rec_s + t * rw;
+      const uint32_t lo = rec[wd], hi = two ? rec[wd + 1] : 0u;
+      const uint32_t bits = __funnelshift_r(lo, hi, sh);      // codes of the 4 coordinates
+      const float4 wt = w_s[t];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const float cv = cbs[(bits >> (BITS * a)) & (L - 1)];
+        acc[a][0] = fmaf(wt.x, cv, acc[a][0]);
+        acc[a][1] = fmaf(wt.y, cv, acc[a][1]);
+        acc[a][2] = fmaf(wt.z, cv, acc[a][2]);
+        acc[a][3] = fmaf(wt.w, cv, acc[a][3]);
       }
     }
-    __syncthreads();
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+      for (int a = 0; a < 4; ++a) accs[(ph * 4 + qq) * d + i0 + a] = acc[a][qq];
   }
+  __syncthreads();
   for (int e = tid; e < nq * d; e += kAThreads) {
     const int qq = e / d, ii = e - qq * d;
+    float v = 0.f;
+    for (int q2 = 0; q2 < phases; ++q2) v += accs[(q2 * 4 + qq) * d + ii];
     const size_t hrow = (size_t)seq * p.n_q_heads + h0 + qq;
-    p.partial[(hrow * p.n_chunks + c) * (size_t)(d + 2) + 2 + ii] = accs[e];
+    p.partial[(hrow * p.n_chunks + c) * (size_t)(d + 2) + 2 + ii] = v;
   }
 }
 
-__global__ void attend_combine_kernel(const float *__restrict__ partial, int n_chunks, int d,
-                                      const float *__restrict__ Pi, float *__restrict__ out) {
+// Merge of the chunks of one query head: scale factors e^{m_c - M} once, the
+// chunk sums split over all threads, then out = Pi^T A / L with the column
+// loop unrolled (independent loads in flight).
+__global__ void __launch_bounds__(256) attend_combine_kernel(const float *__restrict__ partial, int n_chunks, int d,
+                                                             const float *__restrict__ Pi, float *__restrict__ out) {
+  extern __shared__ __align__(16) float cs[];          // [n_chunks] scale factors
   __shared__ float a[kMaxD];
   __shared__ float red[32];
   const int row = blockIdx.x, tid = threadIdx.x;
@@ -123,24 +159,36 @@ __global__ void attend_combine_kernel(const float *__restrict__ partial, int n_c
   m = block_reduce(m, red, true);
   float l = 0.f;
   for (int c = tid; c < n_chunks; c += blockDim.x) {
-    const float *pc = part + (size_t)c * (d + 2);
-    l += pc[1] * expf(pc[0] - m);
+    const float f = expf(part[(size_t)c * (d + 2)] - m);
+    cs[c] = f;
+    l = fmaf(part[(size_t)c * (d + 2) + 1], f, l);
   }
-  l = block_reduce(l, red, false);
+  l = block_reduce(l, red, false);   // also orders the cs[] writes before their reads
   for (int i = tid; i < d; i += blockDim.x) {
-    float s = 0.f;
-    for (int c = 0; c < n_chunks; ++c) {
-      const float *pc = part + (size_t)c * (d + 2);
-      s = fmaf(pc[2 + i], expf(pc[0] - m), s);
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    int c = 0;
+    for (; c + 4 <= n_chunks; c += 4) {
+      s0 = fmaf(part[(size_t)c * (d + 2) + 2 + i], cs[c], s0);
+      s1 = fmaf(part[(size_t)(c + 1) * (d + 2) + 2 + i], cs[c + 1], s1);
+      s2 = fmaf(part[(size_t)(c + 2) * (d + 2) + 2 + i], cs[c + 2], s2);
+      s3 = fmaf(part[(size_t)(c + 3) * (d + 2) + 2 + i], cs[c + 3], s3);
     }
-    a[i] = s;
+    for (; c < n_chunks; ++c) s0 = fmaf(part[(size_t)c * (d + 2) + 2 + i], cs[c], s0);
+    a[i] = (s0 + s1) + (s2 + s3);
   }
   __syncthreads();
   const float inv = 1.0f / l;
   for (int j = tid; j < d; j += blockDim.x) {
-    float s = 0.f;
-    for (int i = 0; i < d; ++i) s = fmaf(__ldg(Pi + (size_t)i * d + j), a[i], s);
-    out[(size_t)row * d + j] = s * inv;
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    int i = 0;
+    for (; i + 4 <= d; i += 4) {
+      s0 = fmaf(__ldg(Pi + (size_t)i * d + j), a[i], s0);
+      s1 = fmaf(__ldg(Pi + (size_t)(i + 1) * d + j), a[i + 1], s1);
+      s2 = fmaf(__ldg(Pi + (size_t)(i + 2) * d + j), a[i + 2], s2);
+      s3 = fmaf(__ldg(Pi + (size_t)(i + 3) * d + j), a[i + 3], s3);
+    }
+    for (; i < d; ++i) s0 = fmaf(__ldg(Pi + (size_t)i * d + j), a[i], s0);
+    out[(size_t)row * d + j] = ((s0 + s1) + (s2 + s3)) * inv;
   }
 }
 
@@ -167,9 +215,14 @@ cudaError_t launch_attend(const AttendParams &p, int bits, int n_seq, size_t sme
 
 cudaError_t launch_combine(const float *partial, int rows, int n_chunks, int d, const float *Pi, float *out,
                            cudaStream_t st) {
-  attend_combine_kernel<<<rows, 256, 0, st>>>(partial, n_chunks, d, Pi, out);
+  const size_t smem = (size_t)n_chunks * sizeof(float);
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(attend_combine_kernel), smem);
+  if (e != cudaSuccess) return e;
+  attend_combine_kernel<<<rows, 256, smem, st>>>(partial, n_chunks, d, Pi, out);
   return cudaGetLastError();
 }
+
+size_t attend_chunk_smem(int d, int bits, int64_t chunk) { return chunk_smem(d, bits, chunk); }
 
 }  // namespace tq
 

@@ -119,6 +119,7 @@ size_t logits_smem_per_query(int d, int bits);
 int logits_fast_stages(int bits, int q, size_t limit);
 cudaError_t launch_logits_fast(const LogitsParams &p, int bits, int n_seq, size_t limit, cudaStream_t st);
 cudaError_t launch_attend(const AttendParams &p, int bits, int n_seq, size_t smem, cudaStream_t st);
+size_t attend_chunk_smem(int d, int bits, int64_t chunk);
 cudaError_t launch_combine(const float *partial, int rows, int n_chunks, int d, const float *Pi,
                            float *out, cudaStream_t st);
 int device_sm_count();

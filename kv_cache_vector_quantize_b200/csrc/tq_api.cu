@@ -125,7 +125,7 @@ FastPlan plan_fast(const tq_cache *k, int n_q_heads) {
 }
 
 constexpr int64_t kAttendChunk = 512;
-constexpr int kAttendMaxQ = 8;
+constexpr int kAttendMaxQ = 4;
 
 }  // namespace
 
@@ -333,6 +333,9 @@ tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale, int32
     cudaError_t e = cudaMemsetAsync(out, 0, out_bytes, (cudaStream_t)stream);
     return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_attend_v (empty)");
   }
+  if ((n_tokens + kAttendChunk - 1) / kAttendChunk > 50000)
+    return fail(TQ_ERR_UNSUPPORTED, "tq_attend_v: n_tokens=%lld exceeds the merge limit of %lld tokens",
+                (long long)n_tokens, 50000LL * kAttendChunk);
   uint32_t *status = static_cast<uint32_t *>(workspace);
   float *partial = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWsHeader);
   const int group = n_q_heads / v->n_kv_heads;
@@ -355,7 +358,7 @@ tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale, int32
   p.group = group;
   p.q_per_cta = group < kAttendMaxQ ? group : kAttendMaxQ;
   p.qblocks = (group + p.q_per_cta - 1) / p.q_per_cta;
-  const size_t smem = sizeof(float) * ((size_t)p.q_per_cta * kAttendChunk + 16 + 32 + (size_t)p.q_per_cta * v->d);
+  const size_t smem = attend_chunk_smem(v->d, v->idx_bits, kAttendChunk);
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "tq_attend_v (status)");
   e = launch_attend(p, v->idx_bits, v->n_seq, smem, (cudaStream_t)stream);
