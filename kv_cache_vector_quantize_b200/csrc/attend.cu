@@ -145,50 +145,86 @@ __global__ void __launch_bounds__(kAThreads) attend_chunk_kernel(const AttendPar
 }
 
 // Merge of the chunks of one query head: scale factors e^{m_c - M} once, the
-// chunk sums split over all threads, then out = Pi^T A / L with the column
-// loop unrolled (independent loads in flight).
-__global__ void __launch_bounds__(256) attend_combine_kernel(const float *__restrict__ partial, int n_chunks, int d,
-                                                             const float *__restrict__ Pi, float *__restrict__ out) {
-  extern __shared__ __align__(16) float cs[];          // [n_chunks] scale factors
+// chunk sums split over all threads with independent loads in flight, then
+// out = Pi^T A / L, with Pi staged in shared memory when it fits.
+constexpr int kCThreads = 512;
+__global__ void __launch_bounds__(kCThreads) attend_combine_kernel(const float *__restrict__ partial, int n_chunks,
+                                                                   int d, const float *__restrict__ Pi,
+                                                                   float *__restrict__ out, int pi_in_smem) {
+  extern __shared__ __align__(16) float cs[];          // [n_chunks] scale factors, then Pi (d x d) if staged
   __shared__ float a[kMaxD];
+  __shared__ float part_sum[kCThreads];
   __shared__ float red[32];
   const int row = blockIdx.x, tid = threadIdx.x;
   const float *part = partial + (size_t)row * n_chunks * (d + 2);
+  float *pis = cs + ((n_chunks + 3) & ~3);
+  if (pi_in_smem) {
+    const float4 *src = reinterpret_cast<const float4 *>(Pi);
+    for (int e = tid; e < d * d / 4; e += kCThreads) reinterpret_cast<float4 *>(pis)[e] = __ldg(src + e);
+  }
   float m = -INFINITY;
-  for (int c = tid; c < n_chunks; c += blockDim.x) m = fmaxf(m, part[(size_t)c * (d + 2)]);
+  for (int c = tid; c < n_chunks; c += kCThreads) m = fmaxf(m, part[(size_t)c * (d + 2)]);
   m = block_reduce(m, red, true);
   float l = 0.f;
-  for (int c = tid; c < n_chunks; c += blockDim.x) {
+  for (int c = tid; c < n_chunks; c += kCThreads) {
     const float f = expf(part[(size_t)c * (d + 2)] - m);
     cs[c] = f;
     l = fmaf(part[(size_t)c * (d + 2) + 1], f, l);
   }
-  l = block_reduce(l, red, false);   // also orders the cs[] writes before their reads
-  for (int i = tid; i < d; i += blockDim.x) {
-    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-    int c = 0;
-    for (; c + 4 <= n_chunks; c += 4) {
-      s0 = fmaf(part[(size_t)c * (d + 2) + 2 + i], cs[c], s0);
-      s1 = fmaf(part[(size_t)(c + 1) * (d + 2) + 2 + i], cs[c + 1], s1);
-      s2 = fmaf(part[(size_t)(c + 2) * (d + 2) + 2 + i], cs[c + 2], s2);
-      s3 = fmaf(part[(size_t)(c + 3) * (d + 2) + 2 + i], cs[c + 3], s3);
+  l = block_reduce(l, red, false);   // also orders the cs[] and Pi writes before their reads
+  // chunk sums: thread = (coordinate i, chunk phase)
+  const int nsplit = kCThreads / d;
+  const int i = tid % d, ph = tid / d;
+  if (ph < nsplit) {
+    float s[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) s[u] = 0.f;
+    int c = ph;
+    for (; c + 7 * nsplit < n_chunks; c += 8 * nsplit) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) s[u] = fmaf(part[(size_t)(c + u * nsplit) * (d + 2) + 2 + i], cs[c + u * nsplit], s[u]);
     }
-    for (; c < n_chunks; ++c) s0 = fmaf(part[(size_t)c * (d + 2) + 2 + i], cs[c], s0);
-    a[i] = (s0 + s1) + (s2 + s3);
+    for (; c < n_chunks; c += nsplit) s[0] = fmaf(part[(size_t)c * (d + 2) + 2 + i], cs[c], s[0]);
+    part_sum[tid] = ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
   }
   __syncthreads();
+  if (tid < d) {
+    float v = 0.f;
+    for (int q = 0; q < nsplit; ++q) v += part_sum[q * d + tid];
+    a[tid] = v;
+  }
+  __syncthreads();
+  // out_j = sum_i Pi[i][j] a_i / L, the i range split over the threads of column j
   const float inv = 1.0f / l;
-  for (int j = tid; j < d; j += blockDim.x) {
+  const int j = tid % d, seg = tid / d, nseg = kCThreads / d;
+  if (seg < nseg) {
+    const int i0 = seg * ((d + nseg - 1) / nseg), i1 = min(d, i0 + (d + nseg - 1) / nseg);
     float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-    int i = 0;
-    for (; i + 4 <= d; i += 4) {
-      s0 = fmaf(__ldg(Pi + (size_t)i * d + j), a[i], s0);
-      s1 = fmaf(__ldg(Pi + (size_t)(i + 1) * d + j), a[i + 1], s1);
-      s2 = fmaf(__ldg(Pi + (size_t)(i + 2) * d + j), a[i + 2], s2);
-      s3 = fmaf(__ldg(Pi + (size_t)(i + 3) * d + j), a[i + 3], s3);
+    int ii = i0;
+    if (pi_in_smem) {
+      for (; ii + 4 <= i1; ii += 4) {
+        s0 = fmaf(pis[ii * d + j], a[ii], s0);
+        s1 = fmaf(pis[(ii + 1) * d + j], a[ii + 1], s1);
+        s2 = fmaf(pis[(ii + 2) * d + j], a[ii + 2], s2);
+        s3 = fmaf(pis[(ii + 3) * d + j], a[ii + 3], s3);
+      }
+      for (; ii < i1; ++ii) s0 = fmaf(pis[ii * d + j], a[ii], s0);
+    } else {
+      for (; ii + 4 <= i1; ii += 4) {
+        s0 = fmaf(__ldg(Pi + (size_t)ii * d + j), a[ii], s0);
+        s1 = fmaf(__ldg(Pi + (size_t)(ii + 1) * d + j), a[ii + 1], s1);
+        s2 = fmaf(__ldg(Pi + (size_t)(ii + 2) * d + j), a[ii + 2], s2);
+        s3 = fmaf(__ldg(Pi + (size_t)(ii + 3) * d + j), a[ii + 3], s3);
+      }
+      for (; ii < i1; ++ii) s0 = fmaf(__ldg(Pi + (size_t)ii * d + j), a[ii], s0);
     }
-    for (; i < d; ++i) s0 = fmaf(__ldg(Pi + (size_t)i * d + j), a[i], s0);
-    out[(size_t)row * d + j] = ((s0 + s1) + (s2 + s3)) * inv;
+    part_sum[tid] = (s0 + s1) + (s2 + s3);
+  }
+  __syncthreads();
+  if (tid < d) {
+    float v = 0.f;
+    for (int q = 0; q < nseg; ++q) v += part_sum[q * d + tid];
+    out[(size_t)row * d + tid] = v * inv;
   }
 }
 
@@ -215,10 +251,14 @@ cudaError_t launch_attend(const AttendParams &p, int bits, int n_seq, size_t sme
 
 cudaError_t launch_combine(const float *partial, int rows, int n_chunks, int d, const float *Pi, float *out,
                            cudaStream_t st) {
-  const size_t smem = (size_t)n_chunks * sizeof(float);
+  const size_t cs_bytes = (size_t)((n_chunks + 3) & ~3) * sizeof(float);
+  const size_t pi_bytes = (size_t)d * d * sizeof(float);
+  const int pi_in_smem = (cs_bytes + pi_bytes <= 160 * 1024 && (reinterpret_cast<uintptr_t>(Pi) & 15) == 0 &&
+                          (d * d) % 4 == 0) ? 1 : 0;
+  const size_t smem = cs_bytes + (pi_in_smem ? pi_bytes : 0);
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(attend_combine_kernel), smem);
   if (e != cudaSuccess) return e;
-  attend_combine_kernel<<<rows, 256, smem, st>>>(partial, n_chunks, d, Pi, out);
+  attend_combine_kernel<<<rows, kCThreads, smem, st>>>(partial, n_chunks, d, Pi, out, pi_in_smem);
   return cudaGetLastError();
 }
 

@@ -54,6 +54,7 @@ constexpr int kFTile = 32 * kFConsumers;       // keys per stage
 constexpr int kFMaxStages = 8;
 constexpr uint32_t kTabStride = 0x10000;       // shared bytes per query head's tables (64 KB)
 constexpr uint32_t kBarBytes = 2 * kFMaxStages * 8;
+constexpr uint32_t kQStage = 2048;                     // shared bytes for the staged Pi q and S q of 2 query heads
 
 template <int BETA>
 struct FastKeys {
@@ -200,7 +201,8 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
   const uint32_t dyn_end = dyn0 + fp.dyn_bytes;
   const uint32_t T0 = (dyn0 + kBarBytes + kTabStride - 1) & ~(kTabStride - 1);
   const uint32_t a0 = dyn0 + kBarBytes;                  // first stage slot below the tables
-  const int n_a = (int)((T0 - a0) / SB);
+  const uint32_t qst = T0 - kQStage;                     // staged query projections, just below the tables
+  const int n_a = (int)((qst - a0) / SB);
   const uint32_t b0 = T0 + QMAX * kTabStride;            // slots after the tables
   const int n_b = b0 < dyn_end ? (int)((dyn_end - b0) / SB) : 0;
   const int stages = min(kFMaxStages, n_a + n_b);
@@ -296,9 +298,15 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
       const int kvh = sk - seq * p.n_kv_heads;
       h0 = kvh * p.group + qb * p.q_per_cta;
       nq = min(p.q_per_cta, p.group - qb * p.q_per_cta);
-      for (int qq = 0; qq < nq; ++qq) {
+      float *qv = reinterpret_cast<float *>(smem + (qst - dyn0));   // [qq][Pi q | S q][128]
+      for (int e = tid; e < nq * 2 * kFD; e += 32 * kFConsumers) {
+        const int qq = e / (2 * kFD), r = e - qq * 2 * kFD;
         const size_t qrow = ((size_t)seq * p.n_q_heads + h0 + qq) * kFD;
-        const float *qr = p.qrot + qrow, *qs = p.qsk + qrow;
+        qv[e] = r < kFD ? p.qrot[qrow + r] : p.qsk[qrow + r - kFD];
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * kFConsumers) : "memory");
+      for (int qq = 0; qq < nq; ++qq) {
+        const float *qr = qv + qq * 2 * kFD, *qs = qr + kFD;
         float *tq_ = tables + (size_t)qq * (kTabStride / 4);
         if constexpr (BETA != 3) {
           // 256 rows of 64 words: [0, 32) index positions, [32, 64) sign positions
@@ -309,12 +317,12 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
               const int t = pos & (K::NI - 1);
 #pragma unroll
               for (int c = 0; c < K::G; ++c)
-                v = fmaf(__ldg(qr + t * K::G + c), cbs[(key >> (BETA * c)) & ((1 << BETA) - 1)], v);
+                v = fmaf(qr[t * K::G + c], cbs[(key >> (BETA * c)) & ((1 << BETA) - 1)], v);
             } else {
               const int t = pos & 15;
 #pragma unroll
               for (int c = 0; c < 8; ++c) {
-                const float sv = __ldg(qs + 8 * t + c);
+                const float sv = qs[8 * t + c];
                 v += ((key >> c) & 1) ? sv : -sv;
               }
               v *= kappa;
@@ -327,7 +335,7 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
             const int t = e & 63, key = e >> 6;
             float v = 0.f;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) v = fmaf(__ldg(qr + 2 * t + c), cbs[(key >> (3 * c)) & 7], v);
+            for (int c = 0; c < 2; ++c) v = fmaf(qr[2 * t + c], cbs[(key >> (3 * c)) & 7], v);
             tq_[((t >> 5) * 64 + key) * 32 + (t & 31)] = v;
           }
           float *ts = tq_ + 8192;
@@ -336,7 +344,7 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
             float v = 0.f;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-              const float sv = __ldg(qs + 8 * t + c);
+              const float sv = qs[8 * t + c];
               v += ((key >> c) & 1) ? sv : -sv;
             }
             ts[e] = v * kappa;
@@ -448,7 +456,7 @@ uint32_t fast_dyn_bytes(int qmax, uint32_t limit, int *stages_out) {
   using K = FastKeys<BETA>;
   const uint32_t dyn0 = 1024;   // reserved shared memory below the dynamic window on sm_100
   const uint32_t T0 = (dyn0 + kBarBytes + kTabStride - 1) & ~(kTabStride - 1);
-  const uint32_t n_a = (T0 - dyn0 - kBarBytes) / K::kStageBytes;
+  const uint32_t n_a = (T0 - kQStage - dyn0 - kBarBytes) / K::kStageBytes;
   const uint32_t b0 = T0 + qmax * kTabStride;
   const uint32_t dyn_end = dyn0 + limit;
   const uint32_t n_b = b0 < dyn_end ? (dyn_end - b0) / K::kStageBytes : 0;
