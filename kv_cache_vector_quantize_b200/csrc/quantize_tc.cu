@@ -43,18 +43,62 @@ struct TcLayout {
   static constexpr uint32_t kMhi = 2 * kTile, kMlo = 3 * kTile;              // keys only
   static constexpr uint32_t kX = QJL ? 4 * kTile : 2 * kTile;
   static constexpr uint32_t kEhi = kX + kTile, kElo = kX + 2 * kTile;        // keys only
-  static constexpr uint32_t kSmall = QJL ? kX + 3 * kTile : kX + kTile;
-  static constexpr uint32_t kNrm = kSmall;                                   // float[128]
-  static constexpr uint32_t kCb = kNrm + 512;                                // float[16] centroids, [16] thresholds
+  // record staging: inside the E tiles for keys (free once the sketch product is done),
+  // a buffer of its own for values
+  static constexpr uint32_t kRec = QJL ? kEhi : kX + kTile;                  // uint32[128][<= 21] records
+  static constexpr uint32_t kRho = kRec + 11264;                             // float[2][128] residual partials
+  static constexpr uint32_t kSlot = kRec + 12288;                            // int64[128] cache slots
+  static constexpr uint32_t kSmall = QJL ? kX + 3 * kTile : kRec + 13312;
+  static constexpr uint32_t kNrm = kSmall;                                   // float[2][128] (two tiles in flight)
+  static constexpr uint32_t kCb = kNrm + 1024;                               // float[16] centroids, [16] thresholds
   static constexpr uint32_t kBar = kCb + 128;                                // 2 mbarriers
   static constexpr uint32_t kTslot = kBar + 16;                              // tensor-memory base address
   static constexpr uint32_t kBytes = kTslot + 16;
-  // inside the X tile once the first product is done
-  static constexpr uint32_t kRec = kX;                                       // uint32[128][<= 21] records
-  static constexpr uint32_t kRho = kX + 11264;                               // float[2][128] residual partials
-  static constexpr uint32_t kSlot = kX + 12288;                              // int64[128] cache slots
   static constexpr uint32_t kTmemCols = QJL ? 256 : 128;
 };
+
+// The x rows of one tile as this thread loads them: rows 16 w + 8 g + (lane & 7),
+// 16-byte chunks 4 i + (lane >> 3), for g = 0..1, i = 0..3.
+struct XRegs {
+  uint4 v[2][4];
+};
+
+__device__ __forceinline__ void load_x(XRegs &xr, const __nv_bfloat16 *__restrict__ x, int64_t row0, int64_t rows,
+                                       int warp, int lane) {
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    const int64_t row = row0 + 16 * warp + 8 * g + (lane & 7);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int kc = 4 * i + (lane >> 3);
+      xr.v[g][i] = row < rows ? __ldg(reinterpret_cast<const uint4 *>(x + row * kTD + 8 * kc)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+}
+
+// Registers -> A tile, and ||x|| (double accumulation) -> nrm[row].
+__device__ __forceinline__ void store_x(const XRegs &xr, unsigned char *xtile, float *nrm, int warp, int lane) {
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    const int t = 16 * warp + 8 * g + (lane & 7);
+    double ss = 0.0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int kc = 4 * i + (lane >> 3);
+      const uint4 v = xr.v[g][i];
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const double a = (double)__uint_as_float(wv[q] << 16), b = (double)__uint_as_float(wv[q] & 0xFFFF0000u);
+        ss = fma(a, a, fma(b, b, ss));
+      }
+      *reinterpret_cast<uint4 *>(xtile + tc::tile_off(kTT, t, 8 * kc)) = v;
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 16);
+    if ((lane >> 3) == 0) nrm[t] = (float)sqrt(ss);
+  }
+}
 
 // Split float32 matrix rows into hi/lo bf16 operand tiles (rows = output coordinates).
 __device__ __forceinline__ void load_split(unsigned char *hi, unsigned char *lo, const float *__restrict__ src) {
@@ -80,7 +124,7 @@ __device__ __forceinline__ uint4 pack8(const __nv_bfloat16 (&v)[8]) {
 }
 
 template <bool QJL, int BITS>
-__global__ void __launch_bounds__(kTThreads, 1) quantize_tc_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(kTThreads, QJL ? 1 : 2) quantize_tc_kernel(const QuantParams p) {
   using Lay = TcLayout<QJL>;
   constexpr int IW = BITS * kTD / 32;                 // code-stream words
   constexpr int RW = IW + (QJL ? kTD / 32 : 0);       // record words
@@ -94,9 +138,16 @@ __global__ void __launch_bounds__(kTThreads, 1) quantize_tc_kernel(const QuantPa
   uint32_t *rec_s = reinterpret_cast<uint32_t *>(smem + Lay::kRec);
   float *rho_s = reinterpret_cast<float *>(smem + Lay::kRho);
   int64_t *slot_s = reinterpret_cast<int64_t *>(smem + Lay::kSlot);
+  unsigned char *xtile = smem + Lay::kX;
   const uint32_t bar1 = sbase + Lay::kBar, bar2 = sbase + Lay::kBar + 8;
+  const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(p.x);
+  const int64_t n_tiles = (p.rows + kTT - 1) / kTT;
+  const int n_my = n_tiles > blockIdx.x ? (int)((n_tiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+  auto row0_of = [&](int i) -> int64_t { return ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * kTT; };
 
-  // ---- one-time set-up: split matrices, codebook, barriers, tensor memory ----
+  // ---- set-up: split matrices, codebook, barriers, tensor memory, first tile ----
+  XRegs xr;
+  if (n_my > 0) load_x(xr, x, row0_of(0), p.rows, warp, lane);
   load_split(smem + Lay::kPhi, smem + Lay::kPlo, p.Pi);
   if constexpr (QJL) load_split(smem + Lay::kMhi, smem + Lay::kMlo, p.SPiT);
   if (tid < L) cb[tid] = p.codebook[tid];
@@ -109,6 +160,7 @@ __global__ void __launch_bounds__(kTThreads, 1) quantize_tc_kernel(const QuantPa
     tc::alloc(sbase + Lay::kTslot, Lay::kTmemCols);
     tc::relinquish();
   }
+  if (n_my > 0) store_x(xr, xtile, nrm_s, warp, lane);
   tc::fence_proxy_async();
   tc::fence_before();
   __syncthreads();
@@ -116,125 +168,98 @@ __global__ void __launch_bounds__(kTThreads, 1) quantize_tc_kernel(const QuantPa
   if (tid < L - 1) cb[16 + tid] = 0.5f * (cb[tid] + cb[tid + 1]);
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + Lay::kTslot);
   const uint32_t d1 = tmem, d2 = tmem + 128;           // accumulator columns
+  const uint32_t idesc = tc::idesc_bf16(kTT, kTD);
+  auto issue_pi = [&]() {     // D1 = x Pi_hi^T + x Pi_lo^T
+    tc::fence_after();
+#pragma unroll 1
+    for (int part = 0; part < 2; ++part) {
+      const uint32_t b = sbase + (part == 0 ? Lay::kPhi : Lay::kPlo);
+#pragma unroll 1
+      for (int s = 0; s < 8; ++s)
+        tc::mma_bf16(d1, tc::smem_desc(sbase + Lay::kX + s * 2 * kLBO, kLBO, kSBO),
+                     tc::smem_desc(b + s * 2 * kLBO, kLBO, kSBO), idesc, (part | s) ? 1u : 0u);
+    }
+    tc::commit(bar1);
+  };
+  if (tid == 0 && n_my > 0) issue_pi();
+  if (n_my > 1) load_x(xr, x, row0_of(1), p.rows, warp, lane);   // prefetch the next tile
   __syncthreads();
   float th[L - 1];
 #pragma unroll
   for (int j = 0; j < L - 1; ++j) th[j] = cb[16 + j];
 
-  const uint32_t idesc = tc::idesc_bf16(kTT, kTD);
-  const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(p.x);
-  const int64_t n_tiles = (p.rows + kTT - 1) / kTT;
   // epilogue role: token t = tensor-memory lane, column half h
   const int t_ep = 32 * (warp & 3) + lane, h = warp >> 2;
   const uint32_t lane_ofs = (uint32_t)(32 * (warp & 3)) << 16;
   bool ok = true;
   int it = 0;
+  int last_pi = n_my > 0 ? 0 : -1;   // index of the last tile whose first product was issued
 
-  for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++it) {
-    const int64_t row0 = tile * kTT;
-    // ---- x rows into the A tile; ||x|| in double ----
-    {
-      const int r = lane & 7, cg = lane >> 3;
-#pragma unroll
-      for (int rg = 0; rg < 2; ++rg) {
-        const int t = 16 * warp + 8 * rg + r;
-        const int64_t row = row0 + t;
-        double ss = 0.0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int kc = 4 * i + cg;
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (row < p.rows) v = __ldg(reinterpret_cast<const uint4 *>(x + row * kTD + 8 * kc));
-          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const double a = (double)__uint_as_float(wv[q] << 16), b = (double)__uint_as_float(wv[q] & 0xFFFF0000u);
-            ss = fma(a, a, fma(b, b, ss));
-          }
-          *reinterpret_cast<uint4 *>(smem + Lay::kX + tc::tile_off(kTT, t, 8 * kc)) = v;
-        }
-        ss += __shfl_xor_sync(0xffffffffu, ss, 8);
-        ss += __shfl_xor_sync(0xffffffffu, ss, 16);
-        if (cg == 0) nrm_s[t] = (float)sqrt(ss);
-      }
-    }
-    tc::fence_proxy_async();
-    tc::fence_before();
-    __syncthreads();
-    // ---- Pi x: 2 split parts x 8 K-steps ----
-    if (tid == 0) {
-      tc::fence_after();
-#pragma unroll 1
-      for (int part = 0; part < 2; ++part) {
-        const uint32_t b = sbase + (part == 0 ? Lay::kPhi : Lay::kPlo);
-#pragma unroll 1
-        for (int s = 0; s < 8; ++s)
-          tc::mma_bf16(d1, tc::smem_desc(sbase + Lay::kX + s * 2 * kLBO, kLBO, kSBO),
-                       tc::smem_desc(b + s * 2 * kLBO, kLBO, kSBO), idesc, (part | s) ? 1u : 0u);
-      }
-      tc::commit(bar1);
-    }
+  for (; it < n_my; ++it) {
+    const int64_t row0 = row0_of(it);
+    const float *nrm_cur = nrm_s + 128 * (it & 1);
+    // (A) the first product of this tile is done: D1 full, the A tile free
     if (__syncthreads_or(!mbar_wait(bar1, it & 1))) { ok = false; break; }
     tc::fence_after();
-
-    // ---- epilogue 1: codes, code-stream words, residual parts ----
-    const float n = nrm_s[t_ep];
+    // (B) next tile's rows into the A tile (prefetched into registers one step ago)
+    if (it + 1 < n_my) store_x(xr, xtile, nrm_s + 128 * ((it + 1) & 1), warp, lane);
+    // (C) epilogue 1: codes, code-stream words (kept in registers), residual parts
+    const float n = nrm_cur[t_ep];
     const float inv = n > 0.f ? 1.0f / n : 0.f;
-    {
-      uint32_t words[2 * BITS];
+    uint32_t words[2 * BITS];
 #pragma unroll
-      for (int w = 0; w < 2 * BITS; ++w) words[w] = 0u;
-      float e2 = 0.f;
+    for (int w = 0; w < 2 * BITS; ++w) words[w] = 0u;
+    float e2 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
-        tc::ld32(d1 + lane_ofs + 64 * h + 32 * c, r);
-        tc::wait_ld();
+    for (int c = 0; c < 2; ++c) {
+      uint32_t r[32];
+      tc::ld32(d1 + lane_ofs + 64 * h + 32 * c, r);
+      tc::wait_ld();
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          __nv_bfloat16 eh[8], el[8];
+      for (int g = 0; g < 4; ++g) {
+        __nv_bfloat16 eh[8], el[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int j = 32 * c + 8 * g + q;            // column within this half
-            const float y = __uint_as_float(r[8 * g + q]) * inv;
-            uint32_t code = 0;
+        for (int q = 0; q < 8; ++q) {
+          const int j = 32 * c + 8 * g + q;            // column within this half
+          const float y = __uint_as_float(r[8 * g + q]) * inv;
+          uint32_t code = 0;
 #pragma unroll
-            for (int k = 0; k < L - 1; ++k) code += (y > th[k]) ? 1u : 0u;
-            const int bit = BITS * j, wd = bit >> 5, off = bit & 31;
-            words[wd] |= code << off;
-            if (off + BITS > 32) words[wd + 1] |= code >> (32 - off);
-            if constexpr (QJL) {
-              const float e = n > 0.f ? y - cb[code] : 0.f;
-              e2 = fmaf(e, e, e2);
-              eh[q] = __float2bfloat16_rn(e);
-              el[q] = __float2bfloat16_rn(e - __bfloat162float(eh[q]));
-            }
-          }
+          for (int k = 0; k < L - 1; ++k) code += (y > th[k]) ? 1u : 0u;
+          const int bit = BITS * j, wd = bit >> 5, off = bit & 31;
+          words[wd] |= code << off;
+          if (off + BITS > 32) words[wd + 1] |= code >> (32 - off);
           if constexpr (QJL) {
-            const uint32_t off = tc::tile_off(kTT, t_ep, 64 * h + 32 * c + 8 * g);
-            *reinterpret_cast<uint4 *>(smem + Lay::kEhi + off) = pack8(eh);
-            *reinterpret_cast<uint4 *>(smem + Lay::kElo + off) = pack8(el);
+            const float e = n > 0.f ? y - cb[code] : 0.f;
+            e2 = fmaf(e, e, e2);
+            eh[q] = __float2bfloat16_rn(e);
+            el[q] = __float2bfloat16_rn(e - __bfloat162float(eh[q]));
           }
         }
-      }
-#pragma unroll
-      for (int w = 0; w < 2 * BITS; ++w) rec_s[t_ep * RS + 2 * BITS * h + w] = words[w];
-      if constexpr (QJL) rho_s[128 * h + t_ep] = e2;
-      if (h == 0) {
-        const int64_t row = row0 + t_ep;
-        if (row < p.rows) {
-          const int64_t sh = row / p.n_tokens, tt = row - sh * p.n_tokens;
-          slot_s[t_ep] = sh * p.capacity + p.pos + tt;
+        if constexpr (QJL) {
+          const uint32_t off = tc::tile_off(kTT, t_ep, 64 * h + 32 * c + 8 * g);
+          *reinterpret_cast<uint4 *>(smem + Lay::kEhi + off) = pack8(eh);
+          *reinterpret_cast<uint4 *>(smem + Lay::kElo + off) = pack8(el);
         }
       }
     }
+    if constexpr (!QJL) {
+#pragma unroll
+      for (int w = 0; w < 2 * BITS; ++w) rec_s[t_ep * RS + 2 * BITS * h + w] = words[w];
+    }
+    if (h == 0) {
+      const int64_t row = row0 + t_ep;
+      if (row < p.rows && !QJL) {
+        const int64_t sh = row / p.n_tokens, tt = row - sh * p.n_tokens;
+        slot_s[t_ep] = sh * p.capacity + p.pos + tt;
+      }
+    }
+    // (D) residual tiles and the next A tile visible to the tensor core; D1 read out
     tc::fence_proxy_async();
     tc::fence_before();
     __syncthreads();
-
-    if constexpr (QJL) {
-      // ---- (S Pi^T) e: 4 split products x 8 K-steps ----
-      if (tid == 0) {
+    // (E) sketch product of this tile, then the first product of the next tile
+    if (tid == 0) {
+      if constexpr (QJL) {
         tc::fence_after();
 #pragma unroll 1
         for (int part = 0; part < 4; ++part) {
@@ -247,24 +272,42 @@ __global__ void __launch_bounds__(kTThreads, 1) quantize_tc_kernel(const QuantPa
         }
         tc::commit(bar2);
       }
+      if (it + 1 < n_my) issue_pi();
+    }
+    if (it + 1 < n_my) last_pi = it + 1;
+    // (F) prefetch the tile after next
+    if (it + 2 < n_my) load_x(xr, x, row0_of(it + 2), p.rows, warp, lane);
+    if constexpr (QJL) {
+      // (G) epilogue 2: sign words; records staged in the (now free) E tiles
       if (__syncthreads_or(!mbar_wait(bar2, it & 1))) { ok = false; break; }
       tc::fence_after();
-      // ---- epilogue 2: sign words ----
+      uint32_t sw[2];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
         tc::ld32(d2 + lane_ofs + 64 * h + 32 * c, r);
         tc::wait_ld();
-        uint32_t sw = 0u;
+        uint32_t wsum = 0u;
 #pragma unroll
-        for (int q = 0; q < 32; ++q) sw |= (__uint_as_float(r[q]) >= 0.f ? 1u : 0u) << q;
-        rec_s[t_ep * RS + IW + 2 * h + c] = sw;
+        for (int q = 0; q < 32; ++q) wsum |= (__uint_as_float(r[q]) >= 0.f ? 1u : 0u) << q;
+        sw[c] = wsum;
+      }
+#pragma unroll
+      for (int w = 0; w < 2 * BITS; ++w) rec_s[t_ep * RS + 2 * BITS * h + w] = words[w];
+      rec_s[t_ep * RS + IW + 2 * h] = sw[0];
+      rec_s[t_ep * RS + IW + 2 * h + 1] = sw[1];
+      rho_s[128 * h + t_ep] = e2;
+      if (h == 0) {
+        const int64_t row = row0 + t_ep;
+        if (row < p.rows) {
+          const int64_t sh = row / p.n_tokens, tt = row - sh * p.n_tokens;
+          slot_s[t_ep] = sh * p.capacity + p.pos + tt;
+        }
       }
       tc::fence_before();
-      __syncthreads();
     }
-
-    // ---- records and norms to the cache ----
+    __syncthreads();
+    // (H) records and norms to the cache
     for (int e = tid; e < kTT * RW; e += kTThreads) {
       const int t = e / RW, w = e - t * RW;
       if (row0 + t < p.rows) p.records[slot_s[t] * RW + w] = rec_s[t * RS + w];
@@ -278,7 +321,7 @@ __global__ void __launch_bounds__(kTThreads, 1) quantize_tc_kernel(const QuantPa
 
   // ---- tear-down: no MMA may still write tensor memory when it is freed ----
   if (!ok) {
-    mbar_wait(bar1, it & 1);
+    if (last_pi >= 0) mbar_wait(bar1, last_pi & 1);
     if constexpr (QJL) mbar_wait(bar2, it & 1);
   }
   tc::fence_before();
@@ -293,7 +336,8 @@ cudaError_t launch_tc(const QuantParams &p, cudaStream_t st) {
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
   const int64_t tiles = (p.rows + kTT - 1) / kTT;
-  const int grid = (int)(tiles < (int64_t)device_sm_count() ? tiles : device_sm_count());
+  const int64_t slots = (int64_t)device_sm_count() * (QJL ? 1 : 2);   // values: two CTAs per SM
+  const int grid = (int)(tiles < slots ? tiles : slots);
   kern<<<grid, kTThreads, smem, st>>>(p);
   return cudaGetLastError();
 }
