@@ -31,7 +31,9 @@ namespace {
 
 constexpr int kTD = 128;                   // head dimension
 constexpr int kTT = 128;                   // tokens per tile (MMA M)
-constexpr int kTThreads = 256;
+// keys: 16 warps (4 threads per token, 32 columns each); values: 8 warps, two CTAs per SM
+template <bool QJL>
+__host__ __device__ constexpr int tc_threads() { return QJL ? 512 : 256; }
 constexpr uint32_t kTile = kTT * kTD * 2;  // bytes of one bf16 operand tile (32 KB)
 constexpr uint32_t kLBO = kTT * 16;        // K-direction core-matrix stride (2048 B)
 constexpr uint32_t kSBO = 128;             // row-direction core-matrix stride
@@ -46,9 +48,9 @@ struct TcLayout {
   // record staging: inside the E tiles for keys (free once the sketch product is done),
   // a buffer of its own for values
   static constexpr uint32_t kRec = QJL ? kEhi : kX + kTile;                  // uint32[128][<= 21] records
-  static constexpr uint32_t kRho = kRec + 11264;                             // float[2][128] residual partials
-  static constexpr uint32_t kSlot = kRec + 12288;                            // int64[128] cache slots
-  static constexpr uint32_t kSmall = QJL ? kX + 3 * kTile : kRec + 13312;
+  static constexpr uint32_t kRho = kRec + 11264;                             // float[4][128] residual partials
+  static constexpr uint32_t kSlot = kRec + 13312;                            // int64[128] cache slots
+  static constexpr uint32_t kSmall = QJL ? kX + 3 * kTile : kRec + 14336;
   static constexpr uint32_t kNrm = kSmall;                                   // float[2][128] (two tiles in flight)
   static constexpr uint32_t kCb = kNrm + 1024;                               // float[16] centroids, [16] thresholds
   static constexpr uint32_t kBar = kCb + 128;                                // 2 mbarriers
@@ -57,17 +59,21 @@ struct TcLayout {
   static constexpr uint32_t kTmemCols = QJL ? 256 : 128;
 };
 
-// The x rows of one tile as this thread loads them: rows 16 w + 8 g + (lane & 7),
-// 16-byte chunks 4 i + (lane >> 3), for g = 0..1, i = 0..3.
+// The x rows of one tile as this thread loads them: with NW warps, warp w owns
+// rows [w R, w R + R) (R = 128 / NW, a multiple of 8), lane l row 8 g + (l & 7)
+// and 16-byte chunks 4 i + (l >> 3), for g < R / 8, i < 4.
+template <int NW>
 struct XRegs {
-  uint4 v[2][4];
+  uint4 v[128 / NW / 8][4];
 };
 
-__device__ __forceinline__ void load_x(XRegs &xr, const __nv_bfloat16 *__restrict__ x, int64_t row0, int64_t rows,
-                                       int warp, int lane) {
+template <int NW>
+__device__ __forceinline__ void load_x(XRegs<NW> &xr, const __nv_bfloat16 *__restrict__ x, int64_t row0,
+                                       int64_t rows, int warp, int lane) {
+  constexpr int R = 128 / NW;
 #pragma unroll
-  for (int g = 0; g < 2; ++g) {
-    const int64_t row = row0 + 16 * warp + 8 * g + (lane & 7);
+  for (int g = 0; g < R / 8; ++g) {
+    const int64_t row = row0 + R * warp + 8 * g + (lane & 7);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int kc = 4 * i + (lane >> 3);
@@ -77,10 +83,12 @@ __device__ __forceinline__ void load_x(XRegs &xr, const __nv_bfloat16 *__restric
 }
 
 // Registers -> A tile, and ||x|| (double accumulation) -> nrm[row].
-__device__ __forceinline__ void store_x(const XRegs &xr, unsigned char *xtile, float *nrm, int warp, int lane) {
+template <int NW>
+__device__ __forceinline__ void store_x(const XRegs<NW> &xr, unsigned char *xtile, float *nrm, int warp, int lane) {
+  constexpr int R = 128 / NW;
 #pragma unroll
-  for (int g = 0; g < 2; ++g) {
-    const int t = 16 * warp + 8 * g + (lane & 7);
+  for (int g = 0; g < R / 8; ++g) {
+    const int t = R * warp + 8 * g + (lane & 7);
     double ss = 0.0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -102,7 +110,7 @@ __device__ __forceinline__ void store_x(const XRegs &xr, unsigned char *xtile, f
 
 // Split float32 matrix rows into hi/lo bf16 operand tiles (rows = output coordinates).
 __device__ __forceinline__ void load_split(unsigned char *hi, unsigned char *lo, const float *__restrict__ src) {
-  for (int e = threadIdx.x; e < kTD * kTD; e += kTThreads) {
+  for (int e = threadIdx.x; e < kTD * kTD; e += blockDim.x) {
     const int n = e >> 7, k = e & 127;
     const float v = __ldg(src + e);
     const __nv_bfloat16 h = __float2bfloat16_rn(v);
@@ -124,8 +132,12 @@ __device__ __forceinline__ uint4 pack8(const __nv_bfloat16 (&v)[8]) {
 }
 
 template <bool QJL, int BITS>
-__global__ void __launch_bounds__(kTThreads, QJL ? 1 : 2) quantize_tc_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(tc_threads<QJL>(), QJL ? 1 : 2) quantize_tc_kernel(const QuantParams p) {
   using Lay = TcLayout<QJL>;
+  constexpr int NT = tc_threads<QJL>(), NW = NT / 32;
+  constexpr int NSPLIT = NT / 128;                    // threads per token in the epilogues
+  constexpr int CPT = 128 / NSPLIT;                   // columns per thread (32 or 64)
+  constexpr int WPT = CPT * BITS / 32;                // code-stream words per thread
   constexpr int IW = BITS * kTD / 32;                 // code-stream words
   constexpr int RW = IW + (QJL ? kTD / 32 : 0);       // record words
   constexpr int RS = RW | 1;                          // record row stride in shared memory (odd: no bank conflicts)
@@ -146,8 +158,8 @@ __global__ void __launch_bounds__(kTThreads, QJL ? 1 : 2) quantize_tc_kernel(con
   auto row0_of = [&](int i) -> int64_t { return ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * kTT; };
 
   // ---- set-up: split matrices, codebook, barriers, tensor memory, first tile ----
-  XRegs xr;
-  if (n_my > 0) load_x(xr, x, row0_of(0), p.rows, warp, lane);
+  XRegs<NW> xr;
+  if (n_my > 0) load_x<NW>(xr, x, row0_of(0), p.rows, warp, lane);
   load_split(smem + Lay::kPhi, smem + Lay::kPlo, p.Pi);
   if constexpr (QJL) load_split(smem + Lay::kMhi, smem + Lay::kMlo, p.SPiT);
   if (tid < L) cb[tid] = p.codebook[tid];
@@ -160,7 +172,7 @@ __global__ void __launch_bounds__(kTThreads, QJL ? 1 : 2) quantize_tc_kernel(con
     tc::alloc(sbase + Lay::kTslot, Lay::kTmemCols);
     tc::relinquish();
   }
-  if (n_my > 0) store_x(xr, xtile, nrm_s, warp, lane);
+  if (n_my > 0) store_x<NW>(xr, xtile, nrm_s, warp, lane);
   tc::fence_proxy_async();
   tc::fence_before();
   __syncthreads();
@@ -182,13 +194,15 @@ __global__ void __launch_bounds__(kTThreads, QJL ? 1 : 2) quantize_tc_kernel(con
     tc::commit(bar1);
   };
   if (tid == 0 && n_my > 0) issue_pi();
-  if (n_my > 1) load_x(xr, x, row0_of(1), p.rows, warp, lane);   // prefetch the next tile
+  if (n_my > 1) load_x<NW>(xr, x, row0_of(1), p.rows, warp, lane);   // prefetch the next tile
   __syncthreads();
-  float th[L - 1];
+  float th[L - 1], cv[L];
 #pragma unroll
   for (int j = 0; j < L - 1; ++j) th[j] = cb[16 + j];
+#pragma unroll
+  for (int j = 0; j < L; ++j) cv[j] = cb[j];
 
-  // epilogue role: token t = tensor-memory lane, column half h
+  // epilogue role: token t = tensor-memory lane, column block h of CPT columns
   const int t_ep = 32 * (warp & 3) + lane, h = warp >> 2;
   const uint32_t lane_ofs = (uint32_t)(32 * (warp & 3)) << 16;
   bool ok = true;
@@ -202,55 +216,64 @@ __global__ void __launch_bounds__(kTThreads, QJL ? 1 : 2) quantize_tc_kernel(con
     if (__syncthreads_or(!mbar_wait(bar1, it & 1))) { ok = false; break; }
     tc::fence_after();
     // (B) next tile's rows into the A tile (prefetched into registers one step ago)
-    if (it + 1 < n_my) store_x(xr, xtile, nrm_s + 128 * ((it + 1) & 1), warp, lane);
+    if (it + 1 < n_my) store_x<NW>(xr, xtile, nrm_s + 128 * ((it + 1) & 1), warp, lane);
     // (C) epilogue 1: codes, code-stream words (kept in registers), residual parts
     const float n = nrm_cur[t_ep];
     const float inv = n > 0.f ? 1.0f / n : 0.f;
-    uint32_t words[2 * BITS];
+    uint32_t words[WPT];
 #pragma unroll
-    for (int w = 0; w < 2 * BITS; ++w) words[w] = 0u;
+    for (int w = 0; w < WPT; ++w) words[w] = 0u;
     float e2 = 0.f;
+    uint32_t r[CPT];
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      uint32_t r[32];
-      tc::ld32(d1 + lane_ofs + 64 * h + 32 * c, r);
-      tc::wait_ld();
+    for (int c = 0; c < CPT / 32; ++c) tc::ld32(d1 + lane_ofs + CPT * h + 32 * c, *reinterpret_cast<uint32_t (*)[32]>(r + 32 * c));
+    tc::wait_ld();
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        __nv_bfloat16 eh[8], el[8];
+    for (int g = 0; g < CPT / 8; ++g) {
+      float ev[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int j = 32 * c + 8 * g + q;            // column within this half
-          const float y = __uint_as_float(r[8 * g + q]) * inv;
-          uint32_t code = 0;
+      for (int q = 0; q < 8; ++q) {
+        const int j = 8 * g + q;                      // column within this block
+        const float y = __uint_as_float(r[j]) * inv;
+        uint32_t code = 0;
+        float c_sel = cv[0];
 #pragma unroll
-          for (int k = 0; k < L - 1; ++k) code += (y > th[k]) ? 1u : 0u;
-          const int bit = BITS * j, wd = bit >> 5, off = bit & 31;
-          words[wd] |= code << off;
-          if (off + BITS > 32) words[wd + 1] |= code >> (32 - off);
-          if constexpr (QJL) {
-            const float e = n > 0.f ? y - cb[code] : 0.f;
-            e2 = fmaf(e, e, e2);
-            eh[q] = __float2bfloat16_rn(e);
-            el[q] = __float2bfloat16_rn(e - __bfloat162float(eh[q]));
-          }
+        for (int k = 0; k < L - 1; ++k) {
+          const bool above = y > th[k];
+          code += above ? 1u : 0u;
+          c_sel = above ? cv[k + 1] : c_sel;
         }
-        if constexpr (QJL) {
-          const uint32_t off = tc::tile_off(kTT, t_ep, 64 * h + 32 * c + 8 * g);
-          *reinterpret_cast<uint4 *>(smem + Lay::kEhi + off) = pack8(eh);
-          *reinterpret_cast<uint4 *>(smem + Lay::kElo + off) = pack8(el);
+        const int bit = BITS * j, wd = bit >> 5, off = bit & 31;
+        words[wd] |= code << off;
+        if (off + BITS > 32) words[wd + 1] |= code >> (32 - off);
+        ev[q] = n > 0.f ? y - c_sel : 0.f;
+        e2 = fmaf(ev[q], ev[q], e2);
+      }
+      if constexpr (QJL) {
+        // e = e_hi + e_lo (bf16 pairs)
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const __nv_bfloat162 hb = __floats2bfloat162_rn(ev[2 * q], ev[2 * q + 1]);
+          const float2 hf = __bfloat1622float2(hb);
+          const __nv_bfloat162 lb = __floats2bfloat162_rn(ev[2 * q] - hf.x, ev[2 * q + 1] - hf.y);
+          hi[q] = *reinterpret_cast<const uint32_t *>(&hb);
+          lo[q] = *reinterpret_cast<const uint32_t *>(&lb);
         }
+        const uint32_t off = tc::tile_off(kTT, t_ep, CPT * h + 8 * g);
+        *reinterpret_cast<uint4 *>(smem + Lay::kEhi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(smem + Lay::kElo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
     }
     if constexpr (!QJL) {
 #pragma unroll
-      for (int w = 0; w < 2 * BITS; ++w) rec_s[t_ep * RS + 2 * BITS * h + w] = words[w];
-    }
-    if (h == 0) {
-      const int64_t row = row0 + t_ep;
-      if (row < p.rows && !QJL) {
-        const int64_t sh = row / p.n_tokens, tt = row - sh * p.n_tokens;
-        slot_s[t_ep] = sh * p.capacity + p.pos + tt;
+      for (int w = 0; w < WPT; ++w) rec_s[t_ep * RS + WPT * h + w] = words[w];
+      if (h == 0) {
+        const int64_t row = row0 + t_ep;
+        if (row < p.rows) {
+          const int64_t sh = row / p.n_tokens, tt = row - sh * p.n_tokens;
+          slot_s[t_ep] = sh * p.capacity + p.pos + tt;
+        }
       }
     }
     // (D) residual tiles and the next A tile visible to the tensor core; D1 read out
@@ -276,26 +299,23 @@ __global__ void __launch_bounds__(kTThreads, QJL ? 1 : 2) quantize_tc_kernel(con
     }
     if (it + 1 < n_my) last_pi = it + 1;
     // (F) prefetch the tile after next
-    if (it + 2 < n_my) load_x(xr, x, row0_of(it + 2), p.rows, warp, lane);
+    if (it + 2 < n_my) load_x<NW>(xr, x, row0_of(it + 2), p.rows, warp, lane);
     if constexpr (QJL) {
       // (G) epilogue 2: sign words; records staged in the (now free) E tiles
       if (__syncthreads_or(!mbar_wait(bar2, it & 1))) { ok = false; break; }
       tc::fence_after();
-      uint32_t sw[2];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
-        tc::ld32(d2 + lane_ofs + 64 * h + 32 * c, r);
-        tc::wait_ld();
+      for (int c = 0; c < CPT / 32; ++c) tc::ld32(d2 + lane_ofs + CPT * h + 32 * c, *reinterpret_cast<uint32_t (*)[32]>(r + 32 * c));
+      tc::wait_ld();
+#pragma unroll
+      for (int w = 0; w < WPT; ++w) rec_s[t_ep * RS + WPT * h + w] = words[w];
+#pragma unroll
+      for (int c = 0; c < CPT / 32; ++c) {
         uint32_t wsum = 0u;
 #pragma unroll
-        for (int q = 0; q < 32; ++q) wsum |= (__uint_as_float(r[q]) >= 0.f ? 1u : 0u) << q;
-        sw[c] = wsum;
+        for (int q = 0; q < 32; ++q) wsum |= (__uint_as_float(r[32 * c + q]) >= 0.f ? 1u : 0u) << q;
+        rec_s[t_ep * RS + IW + (CPT / 32) * h + c] = wsum;
       }
-#pragma unroll
-      for (int w = 0; w < 2 * BITS; ++w) rec_s[t_ep * RS + 2 * BITS * h + w] = words[w];
-      rec_s[t_ep * RS + IW + 2 * h] = sw[0];
-      rec_s[t_ep * RS + IW + 2 * h + 1] = sw[1];
       rho_s[128 * h + t_ep] = e2;
       if (h == 0) {
         const int64_t row = row0 + t_ep;
@@ -308,13 +328,18 @@ __global__ void __launch_bounds__(kTThreads, QJL ? 1 : 2) quantize_tc_kernel(con
     }
     __syncthreads();
     // (H) records and norms to the cache
-    for (int e = tid; e < kTT * RW; e += kTThreads) {
+    for (int e = tid; e < kTT * RW; e += NT) {
       const int t = e / RW, w = e - t * RW;
       if (row0 + t < p.rows) p.records[slot_s[t] * RW + w] = rec_s[t * RS + w];
     }
     if (h == 0 && row0 + t_ep < p.rows) {
       p.norm[slot_s[t_ep]] = n;
-      if constexpr (QJL) p.rnorm[slot_s[t_ep]] = sqrtf(rho_s[t_ep] + rho_s[128 + t_ep]);
+      if constexpr (QJL) {
+        float rr = 0.f;
+#pragma unroll
+        for (int q = 0; q < NSPLIT; ++q) rr += rho_s[128 * q + t_ep];
+        p.rnorm[slot_s[t_ep]] = sqrtf(rr);
+      }
     }
     __syncthreads();
   }
@@ -338,7 +363,7 @@ cudaError_t launch_tc(const QuantParams &p, cudaStream_t st) {
   const int64_t tiles = (p.rows + kTT - 1) / kTT;
   const int64_t slots = (int64_t)device_sm_count() * (QJL ? 1 : 2);   // values: two CTAs per SM
   const int grid = (int)(tiles < slots ? tiles : slots);
-  kern<<<grid, kTThreads, smem, st>>>(p);
+  kern<<<grid, tc_threads<QJL>(), smem, st>>>(p);
   return cudaGetLastError();
 }
 
