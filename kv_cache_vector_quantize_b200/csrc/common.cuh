@@ -136,6 +136,14 @@ tq_status report_error(tq_status s, const char *msg);
 namespace tq {
 
 enum : uint32_t { kDevTimeout = 1u << 1 };   // an mbarrier wait gave up (status word bit)
+// Programmatic dependent launch (sm_90 and later). A grid launched with the
+// programmatic-serialization attribute may start while the previous grid in
+// the stream still runs; it must call pdl_wait() before it reads that grid's
+// results or writes anything that grid writes. Both are no-ops for a grid
+// launched without the attribute.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 constexpr uint32_t kSpinLimit = 1u << 24;    // try_wait attempts before a wait gives up
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

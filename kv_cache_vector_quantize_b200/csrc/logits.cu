@@ -34,6 +34,7 @@ __global__ void __launch_bounds__(128) qprep_kernel(const float *__restrict__ q,
                                                     const float *__restrict__ S, float *__restrict__ qrot,
                                                     float *__restrict__ qsk, uint32_t *status) {
   const int row = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_launch_dependents();   // the scan may start staging keys now; it waits for this grid before reading
   if (row == 0 && chunk == 0 && tid == 0) *status = 0u;   // this call's kernels report into a clean word
   const float *qr = q + (size_t)row * d;
   // lane covers k in [4 lane, 4 lane + 4) and, for d > 128, [128 + 4 lane, ...)

@@ -8,8 +8,10 @@
 //   l_t = n_t ( <Pi q, c[code_t]> + rho_t sqrt(pi/2)/d <S q, 2 sign_t - 1> ).
 //
 // Work split. The key tiles of all (sequence, KV head, query block) units form
-// one list; each CTA (one per SM) takes a contiguous slice of it, so it
-// rebuilds its tables only when its slice crosses into the next unit. One
+// one list. With at least as many units as SMs each CTA (one per SM) takes a
+// contiguous slice of it and rebuilds its tables only when its slice crosses
+// into the next unit; with fewer, every unit gets the same number of CTAs and
+// each CTA a slice of one unit, so it builds its tables once. One
 // producer thread streams 512-key tiles of records (and, when aligned, norms)
 // with cp.async.bulk into a ring of shared-memory stages guarded by mbarriers;
 // 16 consumer warps take 32 keys each per tile (one key per lane). Every wait
@@ -55,6 +57,7 @@ constexpr int kFMaxStages = 8;
 constexpr uint32_t kTabStride = 0x10000;       // shared bytes per query head's tables (64 KB)
 constexpr uint32_t kBarBytes = 2 * kFMaxStages * 8;
 constexpr uint32_t kQStage = 2048;                     // shared bytes for the staged Pi q and S q of 2 query heads
+static_assert(kFTile % 64 == 0, "table builds walk key values with a stride of kFTile / 64");
 
 template <int BETA>
 struct FastKeys {
@@ -68,6 +71,7 @@ struct FastKeys {
 struct FastParams {
   LogitsParams p;
   int tiles_per_unit;
+  int ctas_per_unit;       // > 0: CTA b scans part b % ctas_per_unit of unit b / ctas_per_unit
   int64_t total_tiles;
   uint32_t dyn_bytes;      // dynamic shared memory of the launch
 };
@@ -213,12 +217,23 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (stages < 2 || T0 + QMAX * kTabStride > dyn_end) {
-    if (tid == 0) atomicOr(p.status, kDevBadShape);   // the launch's shared memory cannot hold this layout
+    if (tid == 0) {
+      pdl_wait();   // the query projection clears the status word first
+      atomicOr(p.status, kDevBadShape);   // the launch's shared memory cannot hold this layout
+    }
     return;
   }
-  const int64_t per_cta = (fp.total_tiles + gridDim.x - 1) / gridDim.x;
-  const int64_t g0 = (int64_t)blockIdx.x * per_cta;
-  const int64_t g1 = min(fp.total_tiles, g0 + per_cta);
+  int64_t g0, g1;
+  if (fp.ctas_per_unit > 0) {
+    const int unit = blockIdx.x / fp.ctas_per_unit, part = blockIdx.x - unit * fp.ctas_per_unit;
+    const int64_t base = (int64_t)unit * fp.tiles_per_unit;
+    g0 = base + (int64_t)part * fp.tiles_per_unit / fp.ctas_per_unit;
+    g1 = base + (int64_t)(part + 1) * fp.tiles_per_unit / fp.ctas_per_unit;
+  } else {
+    const int64_t per_cta = (fp.total_tiles + gridDim.x - 1) / gridDim.x;
+    g0 = (int64_t)blockIdx.x * per_cta;
+    g1 = min(fp.total_tiles, g0 + per_cta);
+  }
   if (g0 >= g1) return;
   const int n_my = (int)(g1 - g0);
   const int unit0 = (int)(g0 / fp.tiles_per_unit);
@@ -246,6 +261,7 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
       for (int i = 0; i < n_my; ++i) {
         const int s = i % stages;
         if (i >= stages && !mbar_wait(empty_bar(s), ((i / stages) - 1) & 1)) {
+          pdl_wait();
           atomicOr(p.status, kDevTimeout);
           break;
         }
@@ -271,6 +287,7 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
       // drain: every issued copy must land before the CTA exits
       for (int i = max(0, issued - stages); i < issued; ++i)
         if (!mbar_wait(full_bar(i % stages), (i / stages) & 1)) {
+          pdl_wait();
           atomicOr(p.status, kDevTimeout);
           break;
         }
@@ -279,6 +296,7 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
   }
 
   // -------------------------------- consumers --------------------------------
+  pdl_wait();   // the query projections (and a clean status word) come from the previous grid
   const float kappa = 1.2533141373155003f / (float)kFD;   // sqrt(pi/2)/d
   const uint32_t lane4 = (uint32_t)lane << 2;
   int vunit = unit0, tile = tile0, cur_unit = -1;
@@ -305,49 +323,59 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
         qv[e] = r < kFD ? p.qrot[qrow + r] : p.qsk[qrow + r - kFD];
       }
       asm volatile("bar.sync 1, %0;" ::"n"(32 * kFConsumers) : "memory");
+      // Each thread keeps one table position (and so its few query values) in
+      // registers and walks the key values with a stride of kFTile / width, so a
+      // warp shares one key: codebook reads broadcast and stores hit 32 banks.
       for (int qq = 0; qq < nq; ++qq) {
         const float *qr = qv + qq * 2 * kFD, *qs = qr + kFD;
         float *tq_ = tables + (size_t)qq * (kTabStride / 4);
         if constexpr (BETA != 3) {
           // 256 rows of 64 words: [0, 32) index positions, [32, 64) sign positions
-          for (int e = tid; e < 256 * 64; e += 32 * kFConsumers) {
-            const int pos = e & 63, key = e >> 6;
-            float v = 0.f;
-            if (pos < 32) {
-              const int t = pos & (K::NI - 1);
+          const int pos = tid & 63;
+          if (pos < 32) {
+            const int t = pos & (K::NI - 1);
+            float qc[K::G];
 #pragma unroll
-              for (int c = 0; c < K::G; ++c)
-                v = fmaf(qr[t * K::G + c], cbs[(key >> (BETA * c)) & ((1 << BETA) - 1)], v);
-            } else {
-              const int t = pos & 15;
+            for (int c = 0; c < K::G; ++c) qc[c] = qr[t * K::G + c];
+            for (int key = tid >> 6; key < 256; key += kFTile / 64) {
+              float v = 0.f;
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                const float sv = qs[8 * t + c];
-                v += ((key >> c) & 1) ? sv : -sv;
-              }
-              v *= kappa;
+              for (int c = 0; c < K::G; ++c) v = fmaf(qc[c], cbs[(key >> (BETA * c)) & ((1 << BETA) - 1)], v);
+              tq_[key * 64 + pos] = v;
             }
-            tq_[e] = v;
+          } else {
+            const int t = pos & 15;
+            float sv[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) sv[c] = kappa * qs[8 * t + c];
+            for (int key = tid >> 6; key < 256; key += kFTile / 64) {
+              float v = 0.f;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) v += ((key >> c) & 1) ? sv[c] : -sv[c];
+              tq_[key * 64 + pos] = v;
+            }
           }
         } else {
           // index: 2 groups x 64 rows x 32 words at +0; sign: 256 rows x 32 words at +32 KB
-          for (int e = tid; e < 64 * 64; e += 32 * kFConsumers) {
-            const int t = e & 63, key = e >> 6;
-            float v = 0.f;
-#pragma unroll
-            for (int c = 0; c < 2; ++c) v = fmaf(qr[2 * t + c], cbs[(key >> (3 * c)) & 7], v);
-            tq_[((t >> 5) * 64 + key) * 32 + (t & 31)] = v;
+          {
+            const int t = tid & 63;
+            const float q0 = qr[2 * t], q1 = qr[2 * t + 1];
+            float *row = tq_ + (t >> 5) * 64 * 32 + (t & 31);
+            for (int key = tid >> 6; key < 64; key += kFTile / 64)
+              row[key * 32] = fmaf(q1, cbs[(key >> 3) & 7], q0 * cbs[key & 7]);
           }
-          float *ts = tq_ + 8192;
-          for (int e = tid; e < 256 * 32; e += 32 * kFConsumers) {
-            const int pos = e & 31, key = e >> 5, t = pos & 15;
-            float v = 0.f;
+          {
+            const int pos = tid & 31, t = pos & 15;
+            float sv[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const float sv = qs[8 * t + c];
-              v += ((key >> c) & 1) ? sv : -sv;
+            for (int c = 0; c < 8; ++c) sv[c] = kappa * qs[8 * t + c];
+            float *ts = tq_ + 8192;
+            for (int key = tid >> 5; key < 256; key += kFTile / 32) {
+              float v = 0.f;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) v += ((key >> c) & 1) ? sv[c] : -sv[c];
+              ts[key * 32 + pos] = v;
             }
-            ts[e] = v * kappa;
           }
         }
       }
@@ -480,10 +508,41 @@ cudaError_t launch_fast(const LogitsParams &p, int n_seq, uint32_t limit, cudaSt
   auto kern = logits_fast_kernel<BETA, QMAX>;
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), fp.dyn_bytes);
   if (e != cudaSuccess) return e;
+  // Two splits over one CTA per SM, costed in tiles of the busiest CTA, a table
+  // build counting as kTableTiles: contiguous slices of the tile list (a slice
+  // may cross into a second unit and build twice), or, with fewer units than
+  // SMs, the same whole number of CTAs per unit (one build each, but some SMs
+  // may idle).
+  constexpr int64_t kTableTiles = 3;
+  if (fp.total_tiles <= 0) return cudaSuccess;
   const int64_t slots = device_sm_count();
-  const int64_t grid = fp.total_tiles < slots ? fp.total_tiles : slots;
-  kern<<<(int)grid, kFThreads, fp.dyn_bytes, st>>>(fp);
-  return cudaGetLastError();
+  const int64_t units = fp.tiles_per_unit > 0 ? fp.total_tiles / fp.tiles_per_unit : 0;
+  const int64_t cpu = units > 0 ? (slots / units < fp.tiles_per_unit ? slots / units : fp.tiles_per_unit) : 0;
+  const int64_t cost_aligned = cpu > 0 ? (fp.tiles_per_unit + cpu - 1) / cpu + kTableTiles : INT64_MAX;
+  const int64_t per_slice = (fp.total_tiles + slots - 1) / slots;
+  const int64_t cost_slices = per_slice + (per_slice < fp.tiles_per_unit ? 2 : 1 + per_slice / fp.tiles_per_unit) * kTableTiles;
+  int64_t grid;
+  if (units > 0 && units < slots && cost_aligned < cost_slices) {
+    fp.ctas_per_unit = (int)cpu;
+    grid = units * cpu;
+  } else {
+    fp.ctas_per_unit = 0;
+    grid = fp.total_tiles < slots ? fp.total_tiles : slots;
+  }
+  // Launched as a programmatic dependent of the query projection: the producer
+  // starts streaming keys (written by earlier grids, not by that one) while the
+  // projection runs; consumers wait for it before building tables.
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kFThreads);
+  cfg.dynamicSmemBytes = fp.dyn_bytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, fp);
 }
 
 }  // namespace
