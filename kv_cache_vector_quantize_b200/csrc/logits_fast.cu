@@ -298,7 +298,6 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
   // -------------------------------- consumers --------------------------------
   pdl_wait();   // the query projections (and a clean status word) come from the previous grid
   const float kappa = 1.2533141373155003f / (float)kFD;   // sqrt(pi/2)/d
-  const uint32_t lane4 = (uint32_t)lane << 2;
   int vunit = unit0, tile = tile0, cur_unit = -1;
   int nq = 0, seq = 0, h0 = 0;
   size_t unit_first = 0;
@@ -428,16 +427,16 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
       // (s mod 2) of the x register, byte 1 = key byte (j ^ (l & 3)) of the record
       // word, bytes 2..3 = table-base bytes 2..3 of the x register
       uint32_t sel[4];
+      const uint32_t sel0 = 0x7604u | ((uint32_t)(lane & 3) << 4);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) sel[j] = 0x7600u | (uint32_t)(4 + (j & 1)) | ((uint32_t)(j ^ (lane & 3)) << 4);
+      for (int j = 0; j < 4; ++j) sel[j] = sel0 ^ ((uint32_t)(j & 1) | ((uint32_t)j << 4));
+      const uint32_t xi0 = (T0 & 0xFFFF0000u) | ((uint32_t)lane << 2) | ((uint32_t)(lane ^ 1) << 10);
+      const uint32_t xs0 = xi0 | 0x8080u;
       uint32_t xi[BETA * 8], xs[8];
 #pragma unroll
-      for (int m = 0; m < BETA * 8; ++m)
-        xi[m] = (T0 & 0xFFFF0000u) | ((uint32_t)(lane ^ (2 * m)) << 2) | ((uint32_t)(lane ^ (2 * m + 1)) << 10);
+      for (int m = 0; m < BETA * 8; ++m) xi[m] = xi0 ^ ((uint32_t)m * 0x808u);
 #pragma unroll
-      for (int m = 0; m < 8; ++m)
-        xs[m] = (T0 & 0xFFFF0000u) | (128u | ((uint32_t)(lane ^ (2 * m)) << 2)) |
-                ((128u | ((uint32_t)(lane ^ (2 * m + 1)) << 2)) << 8);
+      for (int m = 0; m < 8; ++m) xs[m] = xs0 ^ ((uint32_t)m * 0x808u);
       uint32_t wi[IW], wsg[4];
 #pragma unroll
       for (int j = 0; j < IW; ++j) wi[j] = w[j];
