@@ -44,16 +44,11 @@ import tq_synth as syn  # noqa: E402
 METRIC = "packed-KV logit-scan GB/s (% of HBM peak); K/V quantize tokens/s at 1 B200"
 UNIT = "GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}
-SM_COUNT_B200 = 148
-FP32_LANES_PER_SM = 128
 
-# DRAM bytes (read + write) per launch from one ncu --set full capture of the
-# kernels as they stand (profiles/*_llama3-8b-decode.md); a key is removed when
-# its kernel changes. Keys: (kernel, workload).
-NCU_TRAFFIC = {
-    ("quantize", "llama"): 67_361_536 + 3_891_456,   # key launch (quantize_kernel<128, 1, bf16>)
-    ("logits", "llama"): 14_728_448 + 0,             # logits_kernel<2>
-}
+# DRAM bytes (read + write) per launch from one ncu capture of the kernel as it
+# stands (profiles/), keyed by (kernel, workload); a key is removed when its
+# kernel changes, and the bench then reports traffic as null.
+NCU_TRAFFIC = {}
 
 
 def parse():
@@ -293,21 +288,37 @@ def run_tq(args, rank, world, local_rank):
 
     peaks, peak_src = load_peaks()
     hbm = float(peaks["hbm_gbs"])
-    sm_mhz_max = float(peaks.get("sm_max_mhz", 1965.0))
-    fp32_peak = SM_COUNT_B200 * FP32_LANES_PER_SM * 2 * sm_mhz_max * 1e6 / 1e12
-    qflops = head_vectors * (4 * d * d + 2 * d * d)
-    q_tflops = qflops / (quant_ms * 1e-3) / 1e12
-    roofline = {"kernel": "quantize_append (K and V launches)", "bound": "alu", "achieved": round(q_tflops, 3),
-                "peak": round(fp32_peak, 1), "unit": "TFLOP/s", "frac": round(q_tflops / fp32_peak, 4),
-                "traffic": NCU_TRAFFIC.get(("quantize", args.workload)),
-                "peak_source": f"FP32 FMA: {SM_COUNT_B200} SMs x {FP32_LANES_PER_SM} lanes x 2 flop x "
-                               f"{sm_mhz_max:.0f} MHz ({peak_src} max clock)",
-                "algorithmic": f"{4 * d * d} flop per key + {2 * d * d} per value (d x d projections)"}
+    bf16 = float(peaks["bf16_tflops"])
+    src_txt = f"hbm_gbs / bf16_tflops, {peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    # quantize: algorithmic bytes = bf16 input + record + norms; algorithmic flops = the d x d projections
+    qk_bytes = head_vectors * (2 * d + kb // head_vectors)
+    qv_bytes = head_vectors * (2 * d + vb // head_vectors)
+    qk_flops, qv_flops = head_vectors * 4 * d * d, head_vectors * 2 * d * d
+
+    def quant_roof(kernel, nbytes, nflops, ms, traffic):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        tfs = nflops / (ms * 1e-3) / 1e12
+        # the roofline bound is the slower of bytes at HBM peak and flops at dense bf16 peak
+        bound = "hbm" if nbytes / hbm > nflops / (bf16 * 1e3) else "tensor"
+        ach, peak, unit = (gbs, hbm, "GB/s") if bound == "hbm" else (tfs, bf16, "TFLOP/s")
+        return {"kernel": kernel, "bound": bound, "achieved": round(ach, 1), "peak": peak, "unit": unit,
+                "frac": round(ach / peak, 4), "traffic": traffic, "peak_source": src_txt,
+                "tensor_tflops": round(tfs, 1), "tensor_frac": round(tfs / bf16, 4),
+                "algorithmic": f"{nbytes // head_vectors} B and {nflops // head_vectors} flop per head-vector"}
+
+    roofline = quant_roof("quantize_tc_kernel, key launch (tq_quantize_append on the K cache)", qk_bytes, qk_flops,
+                          mean["quantize_k"], NCU_TRAFFIC.get(("quantize_k", args.workload)))
+    roof_qv = quant_roof("quantize_tc_kernel, value launch (tq_quantize_append on the V cache)", qv_bytes, qv_flops,
+                         mean["quantize_v"], NCU_TRAFFIC.get(("quantize_v", args.workload)))
     roof_scan = {"kernel": "tq_logits (query projection + logit scan)", "bound": "hbm",
                  "achieved": round(scan_gbs_rank, 1), "peak": hbm, "unit": "GB/s",
                  "frac": round(scan_gbs_rank / hbm, 4), "traffic": NCU_TRAFFIC.get(("logits", args.workload)),
-                 "peak_source": f"hbm_gbs, {peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
-                 "algorithmic": f"{kb // (w['n_seq'] * w['hkv'] * w['T'])} B per key (record + norm + rnorm)"}
+                 "peak_source": src_txt,
+                 "algorithmic": f"{kb // head_vectors} B per key (record + norm + rnorm)"}
+    att_gbs = vb / (mean["attend_v"] * 1e-3) / 1e9
+    roof_att = {"kernel": "tq_attend_v (chunk softmax.V + merge)", "bound": "hbm", "achieved": round(att_gbs, 1),
+                "peak": hbm, "unit": "GB/s", "frac": round(att_gbs / hbm, 4), "traffic": None, "peak_source": src_txt,
+                "algorithmic": f"{vb // head_vectors} B per value (record + norm)"}
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
@@ -321,7 +332,8 @@ def run_tq(args, rank, world, local_rank):
         "quantize_head_vectors_per_s": round(world * head_vectors / (quant_ms * 1e-3), 1),
         "per_kernel_ms": {kk: round(vv, 5) for kk, vv in mean.items()},
         "packed_bytes": {"keys": kb, "values": vb},
-        "roofline": roofline, "roofline_logit_scan": roof_scan,
+        "roofline": roofline, "roofline_logit_scan": roof_scan, "roofline_quantize_v": roof_qv,
+        "roofline_attend_v": roof_att,
         "gpu_launches": kernels_per_step * args.steps,
         "clocks": clk, "e2e": e2e,
     }
