@@ -87,6 +87,17 @@ struct LogitsParams {
   int qblocks;              // ceil(group / q_per_cta)
 };
 
+// Lookup tables of the grouped-query scan (logits_gqa.cu).
+struct GqaParams {
+  const float *q;           // [n_seq][n_q_heads][d]
+  const float *Pi, *S;      // [d][d]
+  const float *codebook;
+  unsigned char *tables;    // units x 128 KB
+  float *sigma;             // [n_seq][n_q_heads] table scale of each head
+  uint32_t *status;
+  int n_kv_heads, n_q_heads, group, qblocks;
+};
+
 struct AttendParams {
   const uint32_t *records;
   const float *norm;
@@ -118,6 +129,10 @@ cudaError_t launch_logits(const LogitsParams &p, int bits, int n_seq, int n_chun
 size_t logits_smem_per_query(int d, int bits);
 int logits_fast_stages(int bits, int q, size_t limit);
 cudaError_t launch_logits_fast(const LogitsParams &p, int bits, int n_seq, size_t limit, cudaStream_t st);
+bool gqa_supported(int d, int bits, int group);
+size_t gqa_table_bytes(int units);
+cudaError_t launch_logits_gqa(const LogitsParams &p, const GqaParams &g, int bits, int n_seq, size_t limit,
+                              cudaStream_t st);
 cudaError_t launch_attend(const AttendParams &p, int bits, int n_seq, size_t smem, cudaStream_t st);
 size_t attend_chunk_smem(int d, int bits, int64_t chunk);
 cudaError_t launch_combine(const float *partial, int rows, int n_chunks, int d, const float *Pi,

@@ -236,9 +236,33 @@ tq_status tq_quantize_append(const tq_cache *cache, const void *x, tq_dtype dtyp
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_quantize_append");
 }
 
+// Workspace of tq_logits: status word | Pi q | S q, and for the grouped-query
+// path a 256-byte aligned table block per unit and one scale per query head.
+namespace {
+struct LogitsWs {
+  size_t proj, tables, sigma, total;
+  int qh, units;
+};
+LogitsWs logits_ws(const tq_cache *k, int32_t n_q_heads) {
+  LogitsWs w{};
+  w.proj = kWsHeader;
+  w.tables = w.proj + ((2 * sizeof(float) * (size_t)k->n_seq * n_q_heads * k->d + 255) & ~(size_t)255);
+  w.sigma = w.tables;
+  w.total = w.tables;
+  const int group = k->n_kv_heads > 0 ? n_q_heads / k->n_kv_heads : 0;
+  if (k->qjl && group * k->n_kv_heads == n_q_heads && gqa_supported(k->d, k->idx_bits, group)) {
+    w.qh = group >= 4 ? 4 : 2;
+    w.units = k->n_seq * k->n_kv_heads * (group / w.qh);
+    w.sigma = w.tables + gqa_table_bytes(w.units);
+    w.total = w.sigma + ((sizeof(float) * (size_t)k->n_seq * n_q_heads + 255) & ~(size_t)255);
+  }
+  return w;
+}
+}  // namespace
+
 size_t tq_logits_workspace_size(const tq_cache *k, int32_t n_q_heads) {
-  if (!k || k->n_seq <= 0 || k->d <= 0 || n_q_heads <= 0) return 0;
-  return kWsHeader + 2 * sizeof(float) * (size_t)k->n_seq * n_q_heads * k->d;
+  if (!k || k->n_seq <= 0 || k->d <= 0 || n_q_heads <= 0 || k->n_kv_heads <= 0) return 0;
+  return logits_ws(k, n_q_heads).total;
 }
 
 tq_status tq_logits(const tq_cache *k, const float *q, int32_t n_q_heads, int64_t n_tokens, const float *Pi,
@@ -269,8 +293,13 @@ tq_status tq_logits(const tq_cache *k, const float *q, int32_t n_q_heads, int64_
   uint32_t *status = static_cast<uint32_t *>(workspace);
   float *qrot = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWsHeader);
   float *qsk = qrot + (size_t)k->n_seq * n_q_heads * k->d;
-  cudaError_t e = launch_qprep(q, k->n_seq * n_q_heads, k->d, Pi, S, qrot, qsk, status, (cudaStream_t)stream);
-  if (e != cudaSuccess) return cuda_fail(e, "tq_logits (query projection)");
+  LogitsWs lw = logits_ws(k, n_q_heads);
+  if (!aligned(Pi, 16) || !aligned(S, 16)) lw.qh = 0;   // the table builder reads matrix rows as float4
+  cudaError_t e = cudaSuccess;
+  if (lw.qh == 0) {
+    e = launch_qprep(q, k->n_seq * n_q_heads, k->d, Pi, S, qrot, qsk, status, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "tq_logits (query projection)");
+  }
   LogitsParams p{};
   p.records = k->records;
   p.norm = k->norm;
@@ -289,6 +318,25 @@ tq_status tq_logits(const tq_cache *k, const float *q, int32_t n_q_heads, int64_
   p.n_kv_heads = k->n_kv_heads;
   p.n_q_heads = n_q_heads;
   p.group = n_q_heads / k->n_kv_heads;
+  if (lw.qh > 0) {
+    // grouped queries: fp16 tables built once per call, one CTA group per KV head block
+    p.q_per_cta = lw.qh;
+    p.qblocks = p.group / lw.qh;
+    GqaParams g{};
+    g.q = q;
+    g.Pi = Pi;
+    g.S = S;
+    g.codebook = codebook;
+    g.tables = static_cast<unsigned char *>(workspace) + lw.tables;
+    g.sigma = reinterpret_cast<float *>(static_cast<char *>(workspace) + lw.sigma);
+    g.status = status;
+    g.n_kv_heads = k->n_kv_heads;
+    g.n_q_heads = n_q_heads;
+    g.group = p.group;
+    g.qblocks = p.qblocks;
+    e = launch_logits_gqa(p, g, k->idx_bits, k->n_seq, device_smem_optin() - 1024, (cudaStream_t)stream);
+    return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_logits (grouped-query scan)");
+  }
   if (fpl.use) {
     p.q_per_cta = fpl.q_per_cta;
     p.qblocks = (p.group + fpl.q_per_cta - 1) / fpl.q_per_cta;

@@ -102,7 +102,14 @@ def test_logits_argument_checks():
     assert _lg(_desc(), ws_bytes=16) == tqb.TQ_ERR_WORKSPACE
     assert _lg(_desc(), n=0) == tqb.TQ_OK                           # nothing to scan
     assert _lg(_desc()) == tqb.TQ_ERR_CUDA                         # passes the checks -> injected
-    assert lib.tq_logits_workspace_size(ctypes.byref(_desc()), 4) == 256 + 2 * 4 * 4 * 128
+    # status header + Pi q and S q (4 query heads) ...
+    proj = 256 + 2 * 4 * 4 * 128
+    assert lib.tq_logits_workspace_size(ctypes.byref(_desc(bits=3)), 4) == proj
+    # ... and, for grouped queries on 1- or 2-bit codes, a 128 KB table block per
+    # (KV head, block of up to 4 query heads) plus one float scale per query head (256-byte aligned)
+    assert lib.tq_logits_workspace_size(ctypes.byref(_desc()), 4) == proj + 2 * 131072 + 256
+    assert lib.tq_logits_workspace_size(ctypes.byref(_desc(heads=1)), 4) == 256 + 2 * 4 * 4 * 128 + 131072 + 256
+    assert lib.tq_logits_workspace_size(ctypes.byref(_desc(heads=4)), 4) == proj   # one query head per KV head
 
 
 def test_attend_argument_checks():

@@ -127,6 +127,11 @@ SHAPES = [
     (128, 3, 4, 2, 2, 1, 901, torch.bfloat16),
     (128, 1, 2, 1, 3, 2, 130, torch.bfloat16),
     (128, 2, 1, 1, 1, 4, 257, torch.bfloat16),
+    # grouped queries on 1-/2-bit codes take the float16-table scan: 2, 4 and 8 heads per KV head,
+    # several 512-key tiles with a ragged tail, more units than one CTA each
+    (128, 2, 3, 2, 1, 8, 1100, torch.bfloat16),
+    (128, 2, 2, 3, 2, 2, 1537, torch.bfloat16),
+    (128, 1, 3, 1, 4, 4, 2049, torch.float16),
 ]
 
 
