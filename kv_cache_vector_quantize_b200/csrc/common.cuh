@@ -122,7 +122,7 @@ struct AttendParams {
 // launchers (defined in the .cu files)
 cudaError_t launch_sketch_rotation(int d, const float *Pi, const float *S, float *SPiT, cudaStream_t st);
 cudaError_t launch_quantize(const QuantParams &p, int bits, bool qjl, tq_dtype dtype, cudaStream_t st);
-cudaError_t launch_quantize_tc(const QuantParams &p, int bits, bool qjl, cudaStream_t st);
+cudaError_t launch_quantize_tc(const QuantParams &p, int bits, bool qjl, bool f16, cudaStream_t st);
 cudaError_t launch_qprep(const float *q, int rows, int d, const float *Pi, const float *S,
                          float *qrot, float *qsk, uint32_t *status, cudaStream_t st);
 cudaError_t launch_logits(const LogitsParams &p, int bits, int n_seq, int n_chunks, size_t smem, cudaStream_t st);

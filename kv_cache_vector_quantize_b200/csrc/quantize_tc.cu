@@ -1,4 +1,4 @@
-// Quantize-append on the tcgen05 tensor cores, for bf16 inputs with d = 128.
+// Quantize-append on the tcgen05 tensor cores, for bf16 or fp16 inputs with d = 128.
 //
 // The method is the encoder of zubnet.ai news, "Google's TurboQuant quantizes
 // LLM KV cache to 3.5 bits per channel", paragraph 2, and winningdata.io,
@@ -8,9 +8,10 @@
 //
 // Precision. The codes must agree with a float64 encoder except within 1e-5
 // of a threshold, so the projections need about 1e-6 of the vectors' scale:
-// more than one bf16 product gives. A bf16 input x is exact in bf16; each
-// float32 matrix is split into two bf16 parts, P = P_hi + P_lo with
-// |P - P_hi - P_lo| <= 2^-16 |P| elementwise, and Pi x = x Pi_hi^T + x Pi_lo^T
+// more than one bf16 product gives. A 16-bit input x is exact in its own type
+// (bf16 or fp16; both MMA operands then use that type); each float32 matrix is
+// split into two parts of that type, P = P_hi + P_lo with
+// |P - P_hi - P_lo| <= 2^-16 |P| elementwise (bf16; fp16 is finer), and Pi x = x Pi_hi^T + x Pi_lo^T
 // accumulates in float32 in tensor memory. The residual e (float32) is split
 // the same way, and (S Pi^T) e = E_hi M_hi^T + E_hi M_lo^T + E_lo M_hi^T
 // (three products; the dropped E_lo M_lo^T is below 2^-16 of the scale).
@@ -48,6 +49,45 @@ constexpr uint32_t kLBO = kTT * 16;        // K-direction core-matrix stride (20
 constexpr uint32_t kSBO = 128;             // row-direction core-matrix stride
 constexpr int kEpiWarps = 8;               // epilogue warps: 2 per lane quarter, 64 columns each
 constexpr int kNormRing = 4;               // n_full barriers (the loaders run at most 3 tiles ahead)
+
+// The 16-bit operand type: bf16 (inputs in bf16) or f16 (inputs in fp16). A split
+// P = P_hi + P_lo rounds to nearest twice; RN pairs pack two values (lower index
+// in the low half).
+template <bool F16>
+struct H16 {
+  static __device__ __forceinline__ uint32_t pack(float a, float b) {
+    if constexpr (F16) {
+      const __half2 h = __floats2half2_rn(a, b);
+      return *reinterpret_cast<const uint32_t *>(&h);
+    } else {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+      return *reinterpret_cast<const uint32_t *>(&h);
+    }
+  }
+  static __device__ __forceinline__ float lo(uint32_t w) {
+    if constexpr (F16) {
+      float f;
+      asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n cvt.f32.f16 %0, l;\n}" : "=f"(f) : "r"(w));
+      return f;
+    } else {
+      return __uint_as_float(w << 16);
+    }
+  }
+  static __device__ __forceinline__ float hi(uint32_t w) {
+    if constexpr (F16) {
+      float f;
+      asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n cvt.f32.f16 %0, h;\n}" : "=f"(f) : "r"(w));
+      return f;
+    } else {
+      return __uint_as_float(w & 0xFFFF0000u);
+    }
+  }
+  // pair of (hi, lo) words for two floats: hi = RN(v), lo = RN(v - hi)
+  static __device__ __forceinline__ void split2(float a, float b, uint32_t &hw, uint32_t &lw) {
+    hw = pack(a, b);
+    lw = pack(a - lo(hw), b - hi(hw));
+  }
+};
 
 template <bool QJL>
 struct Ws {
@@ -122,7 +162,7 @@ struct TileCursor {
 // contiguous 128-byte block); every thread issues all of its loads before
 // converting, so the L2 round trips overlap instead of serialising.
 // src must be 16-byte aligned.
-template <int NTHREADS>
+template <int NTHREADS, bool F16>
 __device__ __forceinline__ void load_split(unsigned char *hi, unsigned char *lo, const float *__restrict__ src) {
   constexpr int kChunks = kTD * kTD / 8;                       // 2048
   constexpr int kPer = (kChunks + NTHREADS - 1) / NTHREADS;
@@ -143,13 +183,7 @@ __device__ __forceinline__ void load_split(unsigned char *hi, unsigned char *lo,
       const float f[8] = {v[c][0].x, v[c][0].y, v[c][0].z, v[c][0].w, v[c][1].x, v[c][1].y, v[c][1].z, v[c][1].w};
       uint32_t hw[4], lw[4];
 #pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
-        const __nv_bfloat162 hb = __floats2bfloat162_rn(f[2 * qq], f[2 * qq + 1]);
-        const float2 hf = __bfloat1622float2(hb);
-        const __nv_bfloat162 lb = __floats2bfloat162_rn(f[2 * qq] - hf.x, f[2 * qq + 1] - hf.y);
-        hw[qq] = *reinterpret_cast<const uint32_t *>(&hb);
-        lw[qq] = *reinterpret_cast<const uint32_t *>(&lb);
-      }
+      for (int qq = 0; qq < 4; ++qq) H16<F16>::split2(f[2 * qq], f[2 * qq + 1], hw[qq], lw[qq]);
       const int n = e & 127, k = 8 * (e >> 7);
       const uint32_t off = tc::tile_off(kTT, n, k);
       *reinterpret_cast<uint4 *>(hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
@@ -244,7 +278,7 @@ struct XRegs {
   uint4 v[4][4];
 };
 
-__device__ __forceinline__ void load_tile(XRegs &xr, const __nv_bfloat16 *__restrict__ x, int64_t row0, int64_t rows,
+__device__ __forceinline__ void load_tile(XRegs &xr, const uint16_t *__restrict__ x, int64_t row0, int64_t rows,
                                           int w, int lane) {
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
@@ -259,11 +293,12 @@ __device__ __forceinline__ void load_tile(XRegs &xr, const __nv_bfloat16 *__rest
 }
 
 // ||x|| of the four rows this lane holds; every lane of a row's quartet ends
-// with the full value. bf16 squares are exact in float32, and a float32 sum of
+// with the full value. bf16 and fp16 squares are exact in float32, and a float32 sum of
 // 128 of them is within 128 * 2^-24 of ||x||^2 (half that on ||x||, inside the
 // 1e-5 tolerance); a row whose sum is outside [2^-100, 2^126) (an overflowed
-// or underflowed square, or a zero vector) is redone in double, which is exact
-// for any finite bf16 input. Each row's result depends on that row alone.
+// or underflowed square, or a zero vector) is redone with rescaled values.
+// Each row's result depends on that row alone.
+template <bool F16>
 __device__ __forceinline__ void tile_norms(const XRegs &xr, float (&nrm)[4]) {
   float sf[4];
 #pragma unroll
@@ -274,7 +309,7 @@ __device__ __forceinline__ void tile_norms(const XRegs &xr, float (&nrm)[4]) {
       const uint32_t wv[4] = {xr.v[g][i].x, xr.v[g][i].y, xr.v[g][i].z, xr.v[g][i].w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float a = __uint_as_float(wv[q] << 16), b = __uint_as_float(wv[q] & 0xFFFF0000u);
+        const float a = H16<F16>::lo(wv[q]), b = H16<F16>::hi(wv[q]);
         s = fmaf(a, a, fmaf(b, b, s));
       }
     }
@@ -289,22 +324,37 @@ __device__ __forceinline__ void tile_norms(const XRegs &xr, float (&nrm)[4]) {
     any |= bad[g];
     nrm[g] = sqrtf(sf[g]);
   }
-  if (__any_sync(0xffffffffu, any)) {   // the whole warp takes part in the shuffles
+  // fp16 values are below 2^16 and at least 2^-24, so their sums of squares never leave float32's
+  // range (a zero vector sums to exactly 0); for bf16 a row out of range is summed again with its
+  // values scaled by a power of two taken from its largest magnitude (exact scaling; squares more
+  // than 2^-100 below the largest one are negligible)
+  if (!F16 && __any_sync(0xffffffffu, any)) {   // the whole warp takes part in the shuffles
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
-      double s = 0.0;
+      uint32_t mx = 0;   // largest |x| as a bit pattern (ordered like the magnitudes)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t wv[4] = {xr.v[g][i].x, xr.v[g][i].y, xr.v[g][i].z, xr.v[g][i].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) mx = max(mx, max((wv[q] << 16) & 0x7FFFFFFFu, wv[q] & 0x7FFF0000u));
+      }
+      mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const int e = (int)(mx >> 23) - 127;            // exponent of the largest magnitude
+      const float sc = __uint_as_float((uint32_t)(127 - e) << 23);   // 2^-e (e in [-127, 127])
+      float s = 0.f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint32_t wv[4] = {xr.v[g][i].x, xr.v[g][i].y, xr.v[g][i].z, xr.v[g][i].w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const double a = (double)__uint_as_float(wv[q] << 16), b = (double)__uint_as_float(wv[q] & 0xFFFF0000u);
-          s = fma(a, a, fma(b, b, s));
+          const float a = H16<F16>::lo(wv[q]) * sc, b = H16<F16>::hi(wv[q]) * sc;
+          s = fmaf(a, a, fmaf(b, b, s));
         }
       }
       s += __shfl_xor_sync(0xffffffffu, s, 8);
       s += __shfl_xor_sync(0xffffffffu, s, 16);
-      if (bad[g]) nrm[g] = (float)sqrt(s);
+      if (bad[g]) nrm[g] = mx == 0 ? 0.f : ldexpf(sqrtf(s), e);
     }
   }
 }
@@ -355,7 +405,7 @@ __device__ __forceinline__ void mma_tile(uint32_t d, uint32_t a, uint32_t b, uin
                  (accumulate_first || s) ? 1u : 0u);
 }
 
-template <bool QJL, int BITS>
+template <bool QJL, int BITS, bool F16>
 __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const QuantParams p) {
   using L = Ws<QJL>;
   constexpr int CPT = 64;                         // columns per epilogue thread
@@ -368,14 +418,14 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const
   const uint32_t sbase = smem_u32(smem);
   const Bars<QJL> bar{sbase + L::kBar};
   float *cb = reinterpret_cast<float *>(smem + L::kCb);
-  const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(p.x);
+  const uint16_t *x = static_cast<const uint16_t *>(p.x);
   const int64_t n_tiles = (p.rows + kTT - 1) / kTT;
   const int n_my = n_tiles > blockIdx.x ? (int)((n_tiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
   auto row0_of = [&](int i) -> int64_t { return ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * kTT; };
 
   // ---- set-up: split matrices, codebook, barriers, tensor memory ----
-  load_split<L::kThreads>(smem + L::kPhi, smem + L::kPlo, p.Pi);
-  if constexpr (QJL) load_split<L::kThreads>(smem + L::kMhi, smem + L::kMlo, p.SPiT);
+  load_split<L::kThreads, F16>(smem + L::kPhi, smem + L::kPlo, p.Pi);
+  if constexpr (QJL) load_split<L::kThreads, F16>(smem + L::kMhi, smem + L::kMlo, p.SPiT);
   if (tid < NL) cb[tid] = p.codebook[tid];
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -411,7 +461,7 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const
     for (int i = 0; i < n_my; ++i) {
       const int64_t row0 = row0_of(i);
       float nrm[4];
-      tile_norms(xr, nrm);
+      tile_norms<F16>(xr, nrm);
       if ((lane >> 3) == 0) {
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
@@ -434,7 +484,7 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const
   } else if (warp == L::kMmaWarp) {
     // ----------------------------- MMA issuer ------------------------------
     if (lane == 0) {
-      const uint32_t idesc = tc::idesc_bf16(kTT, kTD);
+      const uint32_t idesc = tc::idesc_bf16(kTT, kTD, !F16);
       int last_pi = -1, last_sk = -1;
       auto sketch = [&](int j) -> bool {   // D2 = E_hi M_hi^T + E_hi M_lo^T + E_lo M_hi^T
         if (!mbar_wait(bar.e_full(), j & 1)) return false;
@@ -548,13 +598,7 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const
               }
               uint32_t hp[4], lp[4];
 #pragma unroll
-              for (int qq = 0; qq < 4; ++qq) {
-                const __nv_bfloat162 hb = __floats2bfloat162_rn(ev[2 * qq], ev[2 * qq + 1]);
-                const float2 hf = __bfloat1622float2(hb);
-                const __nv_bfloat162 lb = __floats2bfloat162_rn(ev[2 * qq] - hf.x, ev[2 * qq + 1] - hf.y);
-                hp[qq] = *reinterpret_cast<const uint32_t *>(&hb);
-                lp[qq] = *reinterpret_cast<const uint32_t *>(&lb);
-              }
+              for (int qq = 0; qq < 4; ++qq) H16<F16>::split2(ev[2 * qq], ev[2 * qq + 1], hp[qq], lp[qq]);
               tmem_st4(e_hi + 4 * g, hp[0], hp[1], hp[2], hp[3]);
               tmem_st4(e_hi + 64 + 4 * g, lp[0], lp[1], lp[2], lp[3]);
             }
@@ -626,9 +670,9 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const
   if (warp == 0) tc::dealloc(tmem, L::kTmemCols);
 }
 
-template <bool QJL, int BITS>
+template <bool QJL, int BITS, bool F16>
 cudaError_t launch_tc(const QuantParams &p, cudaStream_t st) {
-  auto kern = quantize_tc_kernel<QJL, BITS>;
+  auto kern = quantize_tc_kernel<QJL, BITS, F16>;
   constexpr size_t smem = Ws<QJL>::kBytes;
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
@@ -639,17 +683,22 @@ cudaError_t launch_tc(const QuantParams &p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <bool F16>
+cudaError_t launch_tc_t(const QuantParams &p, int bits, bool qjl, cudaStream_t st) {
+  switch (bits) {
+    case 1: return qjl ? launch_tc<true, 1, F16>(p, st) : launch_tc<false, 1, F16>(p, st);
+    case 2: return qjl ? launch_tc<true, 2, F16>(p, st) : launch_tc<false, 2, F16>(p, st);
+    case 3: return qjl ? launch_tc<true, 3, F16>(p, st) : launch_tc<false, 3, F16>(p, st);
+    default: return qjl ? launch_tc<true, 4, F16>(p, st) : launch_tc<false, 4, F16>(p, st);
+  }
+}
+
 }  // namespace
 
-// Tensor-core quantize for d = 128 bf16 inputs; returns cudaErrorNotSupported for other shapes.
-cudaError_t launch_quantize_tc(const QuantParams &p, int bits, bool qjl, cudaStream_t st) {
+// Tensor-core quantize for d = 128 bf16 or fp16 inputs; returns cudaErrorNotSupported for other shapes.
+cudaError_t launch_quantize_tc(const QuantParams &p, int bits, bool qjl, bool f16, cudaStream_t st) {
   if (p.d != 128) return cudaErrorNotSupported;
-  switch (bits) {
-    case 1: return qjl ? launch_tc<true, 1>(p, st) : launch_tc<false, 1>(p, st);
-    case 2: return qjl ? launch_tc<true, 2>(p, st) : launch_tc<false, 2>(p, st);
-    case 3: return qjl ? launch_tc<true, 3>(p, st) : launch_tc<false, 3>(p, st);
-    default: return qjl ? launch_tc<true, 4>(p, st) : launch_tc<false, 4>(p, st);
-  }
+  return f16 ? launch_tc_t<true>(p, bits, qjl, st) : launch_tc_t<false>(p, bits, qjl, st);
 }
 
 }  // namespace tq

@@ -160,10 +160,12 @@ def test_append_in_parts_equals_one_call():
     assert torch.equal(one.norm, parts.norm) and torch.equal(one.rnorm, parts.rnorm)
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
 def test_special_vectors(dtype):
-    # zero vectors, codeword directions, tiny and huge norms (bf16: the tensor-core path)
+    # zero vectors, codeword directions, tiny and huge norms (bf16 and fp16: the tensor-core path;
+    # fp16 keeps its tiny and huge rows inside its own range)
     d, kb = 128, 2
+    tiny, huge = (1e-3, 1e3) if dtype == torch.float16 else (1e-20, 1e20)
     Pi, S, ck, cv, g = _setup(d, kb, 3)
     rng = np.random.default_rng(5)
     rows = [np.zeros(d)]
@@ -171,7 +173,7 @@ def test_special_vectors(dtype):
     for a in range(5):
         w = c[rng.integers(0, 4, size=d)]
         rows.append(3.0 * (w @ Pi.astype(np.float64)) / np.linalg.norm(w))
-    rows += [1e-20 * rng.standard_normal(d), 1e20 * rng.standard_normal(d), np.ones(d), -np.ones(d)]
+    rows += [tiny * rng.standard_normal(d), huge * rng.standard_normal(d), np.ones(d), -np.ones(d)]
     x = torch.tensor(np.array(rows), dtype=torch.float32).reshape(1, 1, -1, d).to(dtype)
     kc = tqb.PackedCache.empty(d, kb, True, 1, 1, x.shape[2])
     tqb.tq_quantize_append(kc, x.cuda(), 0, g["Pi"], g["SPiT"], g["ck"])
