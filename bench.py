@@ -58,7 +58,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--workload", default="llama",
-                    choices=["llama"] + [f"sweep-b{b}{s}" for b in (2, 3, 4) for s in ("", "-s4")])
+                    choices=["llama"] + [f"sweep-b{b}{s}" for b in (2, 3, 4) for s in ("", "-s4")]
+                    + ["large-b3", "large-b4"])
+    ap.add_argument("--layers", type=int, default=80, help="layers streamed by the large-model workload")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -73,6 +75,12 @@ def workload(name: str):
         return dict(name="llama3-8b-decode: B=1 Hq=32 Hkv=8 d=128 T=32768 bf16 K b=3 (2-bit codes+QJL) V b=3 MSE",
                     n_seq=1, hq=32, hkv=8, d=128, T=32768, k_idx=2, v_idx=3, dtype=torch.bfloat16,
                     gen=lambda dev, seed: syn.llama_inputs(device=dev, seed=seed))
+    if name.startswith("large"):
+        b = int(name.split("-")[1][1:])
+        return dict(name=f"large-model-b{b}: L layers x 128 KV heads x d=128 x 131072 tokens fp16 N(0,1) with outlier "
+                         f"channels, streamed layer by layer, K b={b} V b={b}, one query head per KV head",
+                    n_seq=1, hq=128, hkv=128, d=128, T=131072, k_idx=b - 1, v_idx=b, dtype=torch.float16,
+                    gen=lambda dev, seed: syn.large_layer_inputs(seed, device=dev))
     # "sweep-b3" is the full b-sweep cache; "sweep-b3-s4" keeps 4 of its 8 sequences
     # (a profiling size: still larger than L2, half the device memory)
     b = int(name.split("-")[1][1:])
@@ -340,6 +348,108 @@ def run_tq(args, rank, world, local_rank):
     return result, w
 
 
+def run_large(args, rank, world, local_rank):
+    """Large-model cache streamed layer by layer: per layer, generate K and V on the device
+    (untimed), quantize both into the packed caches, flush L2, one decode step (logits and
+    softmax.V); the packed buffers are reused by every layer."""
+    import kv_cache_vector_quantize_b200 as tqb
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = workload(args.workload)
+    d, H, T = w["d"], w["hkv"], w["T"]
+    Pi = syn.rotation(d).to(dev)
+    S = syn.sketch(d).to(dev)
+    ck = tqb.tq_codebook_fit(d, w["k_idx"]).to(dev)
+    cv = tqb.tq_codebook_fit(d, w["v_idx"]).to(dev)
+    SPiT = tqb.tq_sketch_rotation(Pi, S)
+    kc = tqb.PackedCache.empty(d, w["k_idx"], True, 1, H, T, device=dev)
+    vc = tqb.PackedCache.empty(d, w["v_idx"], False, 1, H, T, device=dev)
+    logits = torch.empty((1, w["hq"], T), dtype=torch.float32, device=dev)
+    out = torch.empty((1, w["hq"], d), dtype=torch.float32, device=dev)
+    ws_l = torch.empty(tqb.tq_logits_workspace_size(kc, w["hq"]), dtype=torch.uint8, device=dev)
+    ws_a = torch.empty(tqb.tq_attend_workspace_size(vc, w["hq"], T), dtype=torch.uint8, device=dev)
+    flush = torch.empty((2 * torch.cuda.get_device_properties(dev).L2_cache_size) // 4, dtype=torch.float32,
+                        device=dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = 1.0 / math.sqrt(d)
+
+    def path(k, v, q, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        tqb.tq_quantize_append(kc, k, 0, Pi, SPiT, ck)
+        if ev is not None:
+            ev[1].record(stream)
+        tqb.tq_quantize_append(vc, v, 0, Pi, None, cv)
+        if ev is not None:
+            ev[2].record(stream)
+        flush.fill_(1.0)
+        if ev is not None:
+            ev[3].record(stream)
+        tqb.tq_logits(kc, q, T, Pi, S, ck, logits=logits, workspace=ws_l)
+        if ev is not None:
+            ev[4].record(stream)
+        tqb.tq_attend_v(vc, logits, scale, T, Pi, cv, out=out, workspace=ws_a)
+        if ev is not None:
+            ev[5].record(stream)
+
+    k, v, q = w["gen"](dev, 7919 * rank)
+    for _ in range(args.warmup):
+        path(k, v, q)
+    torch.cuda.synchronize(dev)
+    per = {n: 0.0 for n in ("quantize_k", "quantize_v", "l2_flush", "logits", "attend_v")}
+    clocks = ClockSampler(dev.index)
+    if world > 1:
+        dist.barrier()
+    clocks.mark_start()
+    for layer in range(args.layers):
+        if layer > 0:
+            del k, v
+            k, v, q = w["gen"](dev, layer + 7919 * rank)   # untimed input generation
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        torch.cuda.synchronize(dev)
+        path(k, v, q, ev)
+        torch.cuda.synchronize(dev)
+        for i, n in enumerate(per):
+            per[n] += ev[i].elapsed_time(ev[i + 1])
+    clocks.mark_end()
+    tqb.tq_workspace_status(ws_l)
+    tqb.tq_workspace_status(ws_a)
+    clk = clocks.stop()
+    t = torch.tensor([per["logits"], per["quantize_k"] + per["quantize_v"], sum(per.values())], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    logits_ms, quant_ms, total_ms = (float(x) for x in t.tolist())
+    L = args.layers
+    kb, vb = key_bytes(w), value_bytes(w)
+    fp16_bytes = 2 * H * T * d * 2
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    scan_gbs = L * kb / (logits_ms * 1e-3) / 1e9
+    qk_bytes = H * T * (2 * d) + kb
+    result = {
+        "metric": METRIC, "value": round(world * scan_gbs, 2), "unit": UNIT, "n_gpus": world, "steps": L,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / L, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w["name"].replace("L layers", f"{L} layers"), "parallelism": "single" if world == 1
+                   else f"replicas{world}", "step": "one layer (inputs generated on the device outside the timed "
+                   "calls)", "l2": "flushed (2 x L2 write) between quantize and decode in every layer"},
+        "quantize_tokens_per_s": round(world * L * T / (quant_ms * 1e-3), 1),
+        "quantize_head_vectors_per_s": round(world * L * H * T / (quant_ms * 1e-3), 1),
+        "per_kernel_ms_per_layer": {n: round(x / L, 5) for n, x in per.items()},
+        "compressed_bytes_total": L * (kb + vb), "uncompressed_fp16_bytes_total": L * fp16_bytes,
+        "compression_ratio_vs_fp16": round(fp16_bytes / (kb + vb), 4),
+        "roofline_logit_scan": {"kernel": "tq_logits", "bound": "hbm", "achieved": round(scan_gbs, 1), "peak": hbm,
+                                "unit": "GB/s", "frac": round(scan_gbs / hbm, 4), "traffic": None,
+                                "peak_source": peak_src},
+        "roofline_quantize_k": {"kernel": "quantize_tc_kernel (fp16 keys)", "bound": "hbm",
+                                "achieved": round(L * qk_bytes / (per["quantize_k"] * 1e-3) / 1e9, 1), "peak": hbm,
+                                "unit": "GB/s"},
+        "gpu_launches": 6 * L, "clocks": clk, "e2e": None,
+    }
+    return result, w
+
+
 # ----------------------------------------------------------------------------
 # the oracle on a bounded sample (cpu_baseline and the reference arm)
 # ----------------------------------------------------------------------------
@@ -459,7 +569,10 @@ def main():
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    result, w = run_tq(args, rank, world, local_rank)
+    if args.workload.startswith("large"):
+        result, w = run_large(args, rank, world, local_rank)
+    else:
+        result, w = run_tq(args, rank, world, local_rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         val, step_s, n, qvps = run_oracle(w, 0, 1, budget_s=12.0)
         result["cpu_baseline"] = {"value": round(val, 6), "unit": UNIT, "cores": _threads(), "kind": "oracle",

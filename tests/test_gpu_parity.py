@@ -285,3 +285,43 @@ def test_bsweep_full_size_sampled(bits):
     # properties at full size: the packed norms are finite and positive, logits finite
     assert torch.isfinite(lg).all()
     assert bool((kc.norm > 0).all()) and bool(torch.isfinite(kc.rnorm).all())
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_large_model_layer_sampled(bits):
+    # one layer of the large-model cache: 128 KV heads x 131072 tokens x 128, fp16 N(0,1) with
+    # outlier channels, one query head per KV head; K at b bits (b-1 codes + QJL), V at b bits.
+    H, T, d = 128, 131072, 128
+    k, v, q = syn.large_layer_inputs(0, device="cuda")
+    Pi, S, ck, cv, g = _setup(d, bits - 1, bits)
+    kc = tqb.PackedCache.empty(d, bits - 1, True, 1, H, T)
+    vc = tqb.PackedCache.empty(d, bits, False, 1, H, T)
+    tqb.tq_quantize_append(kc, k, 0, g["Pi"], g["SPiT"], g["ck"])
+    tqb.tq_quantize_append(vc, v, 0, g["Pi"], None, g["cv"])
+    ws_l = torch.empty(tqb.tq_logits_workspace_size(kc, H), dtype=torch.uint8, device="cuda")
+    ws_a = torch.empty(tqb.tq_attend_workspace_size(vc, H, T), dtype=torch.uint8, device="cuda")
+    lg = tqb.tq_logits(kc, q, T, g["Pi"], g["S"], g["ck"], workspace=ws_l)
+    sc = 1.0 / math.sqrt(d)
+    out = tqb.tq_attend_v(vc, lg, sc, T, g["Pi"], g["cv"], workspace=ws_a)
+    torch.cuda.synchronize()
+    tqb.tq_workspace_status(ws_l)
+    tqb.tq_workspace_status(ws_a)
+    rng = np.random.default_rng(300 + bits)
+    for h in [int(x) for x in rng.choice(H, size=3, replace=False)]:
+        rows = np.sort(rng.choice(T, size=512, replace=False))
+        idx = torch.from_numpy(rows).cuda()
+        kx = k[0, h].index_select(0, idx).float().cpu().numpy()
+        vx = v[0, h].index_select(0, idx).float().cpu().numpy()
+        krec = par.as_u32(kc.records[0, h].index_select(0, idx).cpu().numpy())
+        kn = kc.norm[0, h].index_select(0, idx).cpu().numpy()
+        kr = kc.rnorm[0, h].index_select(0, idx).cpu().numpy()
+        par.check_encoding(kx, krec, kn, kr, Pi, S, ck, d, bits - 1, True)
+        par.check_encoding(vx, par.as_u32(vc.records[0, h].index_select(0, idx).cpu().numpy()),
+                           vc.norm[0, h].index_select(0, idx).cpu().numpy(), None, Pi, None, cv, d, bits, False)
+        par.check_logits(lg[0, h].index_select(0, idx).cpu().numpy()[None, :],
+                         q[0, h].cpu().numpy()[None, :].astype(np.float64), Pi, S, ck, krec, kn, kr, d, bits - 1)
+        # softmax.V over all of this head's tokens, oracle on the GPU's cache and logits
+        par.check_attend(out[0, h:h + 1].cpu().numpy(), lg[0, h:h + 1].cpu().numpy().astype(np.float64), sc, Pi, cv,
+                         par.as_u32(vc.records[0, h].cpu().numpy()), vc.norm[0, h].cpu().numpy(), d, bits)
+    assert torch.isfinite(lg).all() and torch.isfinite(out).all()
+    assert bool((kc.norm > 0).all()) and bool(torch.isfinite(kc.rnorm).all())
