@@ -48,7 +48,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0
 # DRAM bytes (read + write) per launch from one ncu capture of the kernel as it
 # stands (profiles/), keyed by (kernel, workload); a key is removed when its
 # kernel changes, and the bench then reports traffic as null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    ("quantize_k", "llama"): 67_335_680 + 2_341_632,   # quantize_tc_kernel<1, 2, 0>
+    ("quantize_v", "llama"): 67_250_944 + 1_929_728,   # quantize_tc_kernel<0, 3, 0>
+    ("logits", "llama"): 15_757_312 + 0,               # logits_gqa_kernel<2, 4> (the scan; tables read from L2)
+    ("logits", "sweep-b3"): 2 * (234_968_320 + 14_149_632),   # logits_fast_kernel<2, 1>, 4-sequence capture x 2
+}
 
 
 def parse():
@@ -98,6 +103,19 @@ def key_bytes(w) -> int:
 def value_bytes(w) -> int:
     rec = 4 * ((w["v_idx"] * w["d"] + 31) // 32)
     return w["n_seq"] * w["hkv"] * w["T"] * (rec + 4)
+
+
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's replica of the workload (ranks draw different data)."""
+    return syn.SEED_DATA + 7919 * rank
+
+
+def max_over_ranks(values, device, world: int):
+    """Element-wise maximum of per-rank timings (the slowest rank decides)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
 
 
 def load_peaks():
@@ -172,7 +190,7 @@ def run_tq(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     w = workload(args.workload)
     d = w["d"]
-    k, v, q = w["gen"](dev, syn.SEED_DATA + 7919 * rank)
+    k, v, q = w["gen"](dev, rank_seed(rank))
     Pi = syn.rotation(d).to(dev)
     S = syn.sketch(d).to(dev)
     ck = tqb.tq_codebook_fit(d, w["k_idx"]).to(dev)
@@ -245,10 +263,8 @@ def run_tq(args, rank, world, local_rank):
     mean = {kk: sum(vv) / len(vv) for kk, vv in per.items()}
 
     # slowest rank decides
-    t_max = torch.tensor([total_ms, mean["logits"], mean["quantize_k"] + mean["quantize_v"]], device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    total_ms, logits_ms, quant_ms = (float(x) for x in t_max.tolist())
+    total_ms, logits_ms, quant_ms = max_over_ranks(
+        [total_ms, mean["logits"], mean["quantize_k"] + mean["quantize_v"]], dev, world)
 
     kb, vb = key_bytes(w), value_bytes(w)
     scan_gbs_rank = kb / (logits_ms * 1e-3) / 1e9
@@ -285,10 +301,7 @@ def run_tq(args, rank, world, local_rank):
             step_e2e()
         b.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = torch.tensor([a.elapsed_time(b) / args.e2e_steps], device=dev)
-        if world > 1:
-            dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-        e2e_ms = float(e2e_ms.item())
+        e2e_ms = max_over_ranks([a.elapsed_time(b) / args.e2e_steps], dev, world)[0]
         h2d = (hk.numel() * hk.element_size() + hv.numel() * hv.element_size() + hq_.numel() * hq_.element_size())
         e2e = {"value": world * kb / (e2e_ms * 1e-3) / 1e9, "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * hout.element_size(),
@@ -393,7 +406,7 @@ def run_large(args, rank, world, local_rank):
         if ev is not None:
             ev[5].record(stream)
 
-    k, v, q = w["gen"](dev, 7919 * rank)
+    k, v, q = w["gen"](dev, rank_seed(rank))
     for _ in range(args.warmup):
         path(k, v, q)
     torch.cuda.synchronize(dev)
@@ -405,7 +418,7 @@ def run_large(args, rank, world, local_rank):
     for layer in range(args.layers):
         if layer > 0:
             del k, v
-            k, v, q = w["gen"](dev, layer + 7919 * rank)   # untimed input generation
+            k, v, q = w["gen"](dev, layer + rank_seed(rank))   # untimed input generation
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
         torch.cuda.synchronize(dev)
         path(k, v, q, ev)
@@ -416,10 +429,8 @@ def run_large(args, rank, world, local_rank):
     tqb.tq_workspace_status(ws_l)
     tqb.tq_workspace_status(ws_a)
     clk = clocks.stop()
-    t = torch.tensor([per["logits"], per["quantize_k"] + per["quantize_v"], sum(per.values())], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    logits_ms, quant_ms, total_ms = (float(x) for x in t.tolist())
+    logits_ms, quant_ms, total_ms = max_over_ranks(
+        [per["logits"], per["quantize_k"] + per["quantize_v"], sum(per.values())], dev, world)
     L = args.layers
     kb, vb = key_bytes(w), value_bytes(w)
     fp16_bytes = 2 * H * T * d * 2
