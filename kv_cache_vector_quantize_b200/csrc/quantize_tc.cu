@@ -17,9 +17,9 @@
 // (three products; the dropped E_lo M_lo^T is below 2^-16 of the scale).
 //
 // Warp roles (one persistent CTA per SM, 128-token tiles):
-//   - 4 loader warps: global -> registers one tile ahead, ||x|| (written to
-//     the cache), registers -> one of two A tiles in shared memory
-//     once the tensor core has finished reading it;
+//   - one copy thread: tensor-map copies of x straight into a ring of A tiles
+//     in shared memory (2 for keys, 4 for values), in the 128-byte swizzle layout;
+//   - 4 norm warps: ||x|| from each landed tile, written to the cache;
 //   - one MMA thread: for tile i, D1 = x Pi^T (two products); then, keys, the
 //     sketch product of tile i - 1, D2 = E M^T, with E (the split residual) read
 //     from tensor memory;
@@ -34,7 +34,10 @@
 // Every stage hand-off is an mbarrier; every wait is bounded (a timed-out
 // role stops and the others time out behind it; no MMA is in flight when
 // tensor memory is freed).
-// Shared-memory operand tiles use the no-swizzle K-major core-matrix layout of tc.cuh.
+// Shared-memory operand tiles use the 128-byte swizzle K-major layout of tc.cuh (sw128_off).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -45,10 +48,8 @@ namespace {
 constexpr int kTD = 128;                   // head dimension
 constexpr int kTT = 128;                   // tokens per tile (MMA M)
 constexpr uint32_t kTile = kTT * kTD * 2;  // bytes of one bf16 operand tile (32 KB)
-constexpr uint32_t kLBO = kTT * 16;        // K-direction core-matrix stride (2048 B)
-constexpr uint32_t kSBO = 128;             // row-direction core-matrix stride
 constexpr int kEpiWarps = 8;               // epilogue warps: 2 per lane quarter, 64 columns each
-constexpr int kNormRing = 4;               // n_full barriers (the loaders run at most 3 tiles ahead)
+constexpr int kNormRing = 8;               // ||x|| ring in shared memory (the norm warps run at most kNX + 1 tiles ahead)
 
 // The 16-bit operand type: bf16 (inputs in bf16) or f16 (inputs in fp16). A split
 // P = P_hi + P_lo rounds to nearest twice; RN pairs pack two values (lower index
@@ -91,21 +92,28 @@ struct H16 {
 
 template <bool QJL>
 struct Ws {
-  static constexpr int kLoadWarps = 4;
-  static constexpr int kMmaWarp = kEpiWarps + kLoadWarps;
-  static constexpr int kThreads = 32 * (kMmaWarp + 1);   // 416: at most 4 warps per SM sub-partition (128 registers)
+  static constexpr int kNormWarps = 4;                  // ||x|| from the landed A tiles
+  static constexpr int kTmaWarp = kEpiWarps + kNormWarps;
+  static constexpr int kMmaWarp = kTmaWarp + 1;
+  static constexpr int kThreads = 32 * (kMmaWarp + 1);   // 448: at most 4 warps per SM sub-partition (128 registers)
+  static constexpr int kNX = QJL ? 2 : 4;                // A-tile stages (tensor-map copies in flight)
+  // values: Pi_hi and Pi_lo stacked as one 256-row B tile, so one N = 256 product per K step gives
+  // both parts (summed by the epilogue), with two D1 buffers; keys: two N = 128 products into one D1
+  static constexpr int kND1 = QJL ? 1 : 2;
+  static constexpr int kPW = QJL ? 128 : 256;
   // dynamic shared memory, byte offsets
   static constexpr uint32_t kPhi = 0, kPlo = kTile;
   static constexpr uint32_t kMhi = 2 * kTile, kMlo = 3 * kTile;              // keys only
-  static constexpr uint32_t kX = QJL ? 4 * kTile : 2 * kTile;                // two A tiles
-  static constexpr uint32_t kRho = kX + 2 * kTile;                           // float[3][128] (keys)
-  static constexpr uint32_t kCb = kRho + (QJL ? 3 * 128 * 4 : 0);            // float[16] centroids
+  static constexpr uint32_t kX = QJL ? 4 * kTile : 2 * kTile;                // kNX A tiles
+  static constexpr uint32_t kRho = kX + kNX * kTile;                         // float[3][128] (keys)
+  static constexpr uint32_t kNrm = kRho + (QJL ? 3 * 128 * 4 : 0);           // float[kNormRing][128] ||x||
+  static constexpr uint32_t kCb = kNrm + kNormRing * 128 * 4;                // float[16] centroids
   static constexpr uint32_t kBar = kCb + 64;
-  // barriers: x_full[2], x_empty[2], d1_full, d1_empty, e_full, d2_full, d2_empty, n_full[4]
-  static constexpr int kBars = 2 + 2 + 1 + 1 + 1 + 1 + 1 + kNormRing;
+  // barriers: x_full[4], x_empty[4], d1_full[2], d1_empty[2], e_full, d2_full, d2_empty, n_full[kNormRing]
+  static constexpr int kBars = 4 + 4 + 2 + 2 + 1 + 1 + 1 + kNormRing;
   static constexpr uint32_t kTslot = kBar + 8 * kBars;
   static constexpr uint32_t kBytes = kTslot + 16;
-  static constexpr uint32_t kTmemCols = QJL ? 512 : 128;
+  static constexpr uint32_t kTmemCols = 512;   // keys: D1, D2, E[0], E[1]; values: D1[0], D1[1] (256 each)
   static constexpr uint32_t kD2 = 128, kE = 256;   // tensor-memory column offsets (keys)
   static_assert(kBytes <= 232448, "shared memory over the per-CTA limit");
 };
@@ -115,13 +123,13 @@ template <bool QJL>
 struct Bars {
   uint32_t base;
   __device__ uint32_t x_full(int s) const { return base + 8u * s; }
-  __device__ uint32_t x_empty(int s) const { return base + 8u * (2 + s); }
-  __device__ uint32_t d1_full() const { return base + 8u * 4; }
-  __device__ uint32_t d1_empty() const { return base + 8u * 5; }
-  __device__ uint32_t e_full() const { return base + 8u * 6; }
-  __device__ uint32_t d2_full() const { return base + 8u * 7; }
-  __device__ uint32_t d2_empty() const { return base + 8u * 8; }
-  __device__ uint32_t n_full(int k) const { return base + 8u * (9 + k); }
+  __device__ uint32_t x_empty(int s) const { return base + 8u * (4 + s); }
+  __device__ uint32_t d1_full(int b) const { return base + 8u * (8 + b); }
+  __device__ uint32_t d1_empty(int b) const { return base + 8u * (10 + b); }
+  __device__ uint32_t e_full() const { return base + 8u * 12; }
+  __device__ uint32_t d2_full() const { return base + 8u * 13; }
+  __device__ uint32_t d2_empty() const { return base + 8u * 14; }
+  __device__ uint32_t n_full(int k) const { return base + 8u * (15 + k); }
 };
 
 // Position of a CTA's current tile in the (sequence x head, token) grid, kept
@@ -129,13 +137,14 @@ struct Bars {
 // sh * n_tokens + tt with 0 <= tt < n_tokens; the persistent CTA advances by
 // gridDim.x tiles = step_q * n_tokens + step_r rows.
 struct TileCursor {
-  int64_t sh, tt, step_q, step_r;
+  int64_t sh, tt, step_q, step_r, base;   // base = slot of the tile's first row
   __device__ void init(const QuantParams &p) {
     const int64_t row0 = (int64_t)blockIdx.x * 128, step = (int64_t)gridDim.x * 128;
     sh = row0 / p.n_tokens;
     tt = row0 - sh * p.n_tokens;
     step_q = step / p.n_tokens;
     step_r = step - step_q * p.n_tokens;
+    base = sh * p.capacity + p.pos + tt;
   }
   __device__ void advance(const QuantParams &p) {
     tt += step_r;
@@ -144,9 +153,11 @@ struct TileCursor {
       tt -= p.n_tokens;
       ++sh;
     }
+    base = sh * p.capacity + p.pos + tt;
   }
   // cache slot of tile row r
   __device__ int64_t slot(const QuantParams &p, int r) const {
+    if (tt + r < p.n_tokens) return base + r;   // the row is in the tile's first (sequence, head)
     int64_t t2 = tt + r, s2 = sh;
     while (t2 >= p.n_tokens) {
       t2 -= p.n_tokens;
@@ -157,12 +168,12 @@ struct TileCursor {
 };
 
 // Split float32 matrix rows into hi/lo bf16 operand tiles (rows = output coordinates).
-// A work item is one 16-byte core-matrix row chunk (8 consecutive k of one row;
+// A work item is one 16-byte row chunk (8 consecutive k of one row;
 // consecutive threads take consecutive rows, so each quarter-warp stores one
 // contiguous 128-byte block); every thread issues all of its loads before
 // converting, so the L2 round trips overlap instead of serialising.
 // src must be 16-byte aligned.
-template <int NTHREADS, bool F16>
+template <int NTHREADS, bool F16, bool STACKED = false>
 __device__ __forceinline__ void load_split(unsigned char *hi, unsigned char *lo, const float *__restrict__ src) {
   constexpr int kChunks = kTD * kTD / 8;                       // 2048
   constexpr int kPer = (kChunks + NTHREADS - 1) / NTHREADS;
@@ -185,9 +196,11 @@ __device__ __forceinline__ void load_split(unsigned char *hi, unsigned char *lo,
 #pragma unroll
       for (int qq = 0; qq < 4; ++qq) H16<F16>::split2(f[2 * qq], f[2 * qq + 1], hw[qq], lw[qq]);
       const int n = e & 127, k = 8 * (e >> 7);
-      const uint32_t off = tc::tile_off(kTT, n, k);
-      *reinterpret_cast<uint4 *>(hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4 *>(lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      // STACKED: one 256-row tile at `hi`, rows [0, 128) the hi parts, [128, 256) the lo parts
+      const uint32_t oh = STACKED ? tc::sw128_off(2 * kTT, n, k) : tc::sw128_off(kTT, n, k);
+      const uint32_t ol = STACKED ? tc::sw128_off(2 * kTT, n + kTT, k) : tc::sw128_off(kTT, n, k);
+      *reinterpret_cast<uint4 *>(hi + oh) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4 *>((STACKED ? hi : lo) + ol) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
   }
 }
@@ -258,6 +271,92 @@ __device__ __forceinline__ float centroid_of(const uint32_t (&m)[BITS], const fl
   }
 }
 
+// Code search on the FMA pipe. With B = 2^126, sat(y B - t B) is 1.0 when y > t and 0.0 when
+// y <= t for the coordinates of a unit vector (|y - t| is either 0 or at least one float32 ulp of
+// t, times 2^126 >= 1; the middle threshold 0 is passed by any normal y > 0). The code is built as
+// a float (sum of its bit flags times their weights) plus 2^23, whose bit pattern is 0x4B000000 +
+// code, and added into the words by integer multiply-add; the 0x4B000000 parts are subtracted per
+// word once (kMagicSum). Threshold choices of the binary search are multiply-adds of the flags.
+__device__ __forceinline__ float sat_gt(float y, float tb) {   // 1.0 if y > t else 0.0 (tb = t B)
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, 0f7E800000, %2;" : "=f"(r) : "f"(y), "f"(-tb));
+  return r;
+}
+
+// bit flags f[k] (0.0 or 1.0) of code = #{j : y > th[j]}; tb[] = th[] * 2^126, dt[] precomputed differences
+template <int BITS>
+struct FmaSearch {
+  float tb[(1 << BITS) - 1];
+  __device__ void init(const float (&th)[(1 << BITS) - 1]) {
+#pragma unroll
+    for (int k = 0; k < (1 << BITS) - 1; ++k) tb[k] = th[k] * 0x1p126f;
+  }
+  __device__ __forceinline__ void flags(float y, float (&f)[BITS]) const {
+    if constexpr (BITS == 1) {
+      f[0] = sat_gt(y, tb[0]);
+    } else if constexpr (BITS == 2) {
+      f[1] = sat_gt(y, tb[1]);
+      f[0] = sat_gt(y, fmaf(f[1], tb[2] - tb[0], tb[0]));
+    } else if constexpr (BITS == 3) {
+      f[2] = sat_gt(y, tb[3]);
+      f[1] = sat_gt(y, fmaf(f[2], tb[5] - tb[1], tb[1]));
+      const float lo = fmaf(f[1], tb[2] - tb[0], tb[0]), hi = fmaf(f[1], tb[6] - tb[4], tb[4]);
+      f[0] = sat_gt(y, fmaf(f[2], hi - lo, lo));
+    } else {
+      f[3] = sat_gt(y, tb[7]);
+      f[2] = sat_gt(y, fmaf(f[3], tb[11] - tb[3], tb[3]));
+      const float l1 = fmaf(f[2], tb[5] - tb[1], tb[1]), h1 = fmaf(f[2], tb[13] - tb[9], tb[9]);
+      f[1] = sat_gt(y, fmaf(f[3], h1 - l1, l1));
+      const float a = fmaf(f[1], tb[2] - tb[0], tb[0]), b = fmaf(f[1], tb[6] - tb[4], tb[4]);
+      const float c = fmaf(f[1], tb[10] - tb[8], tb[8]), d = fmaf(f[1], tb[14] - tb[12], tb[12]);
+      const float lo = fmaf(f[2], b - a, a), hi = fmaf(f[2], d - c, c);
+      f[0] = sat_gt(y, fmaf(f[3], hi - lo, lo));
+    }
+  }
+};
+
+// 0x4B000000 + v for a small integer-valued float v >= 0
+__device__ __forceinline__ uint32_t magic(float v) { return __float_as_uint(v + 8388608.0f); }
+
+// Adds the code of coordinate j (flags f) into this thread's words; the words carry
+// 0x4B000000-multiples that fix_words removes.
+template <int BITS, int NW>
+__device__ __forceinline__ void put_code_f(uint32_t (&w)[NW], const float (&f)[BITS], int j) {
+  const int bit = BITS * j, wd = bit >> 5, off = bit & 31;
+  if (off + BITS <= 32) {
+    float v = f[0];
+#pragma unroll
+    for (int k = 1; k < BITS; ++k) v = fmaf(f[k], (float)(1 << k), v);
+    w[wd] += magic(v) * (1u << off);
+  } else {
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) {
+      const int b = bit + k;
+      w[b >> 5] += magic(f[k]) * (1u << (b & 31));
+    }
+  }
+}
+
+// Subtracts the 0x4B000000 terms put_code_f added for coordinates [0, n) of this thread.
+template <int BITS, int NW>
+__device__ __forceinline__ void fix_words(uint32_t (&w)[NW], int n) {
+  uint32_t corr[NW];
+#pragma unroll
+  for (int k = 0; k < NW; ++k) corr[k] = 0u;
+#pragma unroll
+  for (int j = 0; j < n; ++j) {
+    const int bit = BITS * j, off = bit & 31;
+    if (off + BITS <= 32) {
+      corr[bit >> 5] += 0x4B000000u * (1u << off);
+    } else {
+#pragma unroll
+      for (int k = 0; k < BITS; ++k) corr[(bit + k) >> 5] += 0x4B000000u * (1u << ((bit + k) & 31));
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < NW; ++k) w[k] -= corr[k];
+}
+
 // Code of coordinate j (BITS bits at stream bit BITS * j) into this thread's words.
 template <int BITS, int NW>
 __device__ __forceinline__ void put_code(uint32_t (&w)[NW], const uint32_t (&m)[BITS], int j) {
@@ -269,27 +368,18 @@ __device__ __forceinline__ void put_code(uint32_t (&w)[NW], const uint32_t (&m)[
 }
 
 // --------------------------------------------------------------------------
-// loader: a group of 4 warps moves whole 128-token tiles. Warp w of the group
-// owns tile rows [32 w, 32 w + 32); lane l loads row 32 w + 8 g + (l & 7),
-// 16-byte chunks 4 i + (l >> 3) (g, i < 4), so each quarter-warp stores one
-// contiguous 128-byte core matrix row block.
+// A tiles arrive by tensor-map copies (16 per tile, one per K chunk). The 4
+// norm warps then read them back: warp w owns tile rows [32 w, 32 w + 32);
+// lane l reads row 32 w + 8 g + (l & 7), 16-byte chunks 4 i + (l >> 3)
+// (g, i < 4), so each quarter-warp reads one contiguous 128-byte block.
 // --------------------------------------------------------------------------
-struct XRegs {
-  uint4 v[4][4];
-};
-
-__device__ __forceinline__ void load_tile(XRegs &xr, const uint16_t *__restrict__ x, int64_t row0, int64_t rows,
-                                          int w, int lane) {
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    const int64_t row = row0 + 32 * w + 8 * g + (lane & 7);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int kc = 4 * i + (lane >> 3);
-      xr.v[g][i] = row < rows ? __ldg(reinterpret_cast<const uint4 *>(x + row * kTD + 8 * kc))
-                              : make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
+// One 2-D tensor-map copy: 64 columns (128 bytes) x 128 rows, landing as one K block of the
+// 128-byte swizzle layout (16 KB); completion counted on `bar`.
+__device__ __forceinline__ void tma_x_chunk(uint32_t dst, const CUtensorMap *map, int col, int row, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(row), "r"(bar)
+      : "memory");
 }
 
 // ||x|| of the four rows this lane holds; every lane of a row's quartet ends
@@ -299,42 +389,51 @@ __device__ __forceinline__ void load_tile(XRegs &xr, const uint16_t *__restrict_
 // or underflowed square, or a zero vector) is redone with rescaled values.
 // Each row's result depends on that row alone.
 template <bool F16>
-__device__ __forceinline__ void tile_norms(const XRegs &xr, float (&nrm)[4]) {
+__device__ __forceinline__ void tile_norms(const unsigned char *xt, int w, int lane, float (&nrm)[4]) {
+  auto chunk = [&](int g, int i) {
+    return *reinterpret_cast<const uint4 *>(xt + tc::sw128_off(kTT, 32 * w + 8 * g + (lane & 7), 8 * (4 * i + (lane >> 3))));
+  };
+  uint4 v[4][4];   // all 16 chunks in flight before any arithmetic
+#pragma unroll
+  for (int g = 0; g < 4; ++g)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[g][i] = chunk(g, i);
   float sf[4];
+  bool bad[4], any = false;
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
-    float s = 0.f;
+    float part[4];   // one accumulator per chunk: four short chains instead of one long one
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t wv[4] = {xr.v[g][i].x, xr.v[g][i].y, xr.v[g][i].z, xr.v[g][i].w};
+      const uint32_t wv[4] = {v[g][i].x, v[g][i].y, v[g][i].z, v[g][i].w};
+      float s = 0.f;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float a = H16<F16>::lo(wv[q]), b = H16<F16>::hi(wv[q]);
         s = fmaf(a, a, fmaf(b, b, s));
       }
+      part[i] = s;
     }
+    float s = (part[0] + part[1]) + (part[2] + part[3]);
     s += __shfl_xor_sync(0xffffffffu, s, 8);
     s += __shfl_xor_sync(0xffffffffu, s, 16);
     sf[g] = s;
-  }
-  bool bad[4], any = false;
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    bad[g] = !(sf[g] >= 0x1p-100f && sf[g] < 0x1p126f);
+    bad[g] = !(s >= 0x1p-100f && s < 0x1p126f);
     any |= bad[g];
-    nrm[g] = sqrtf(sf[g]);
+    nrm[g] = sqrtf(s);
   }
   // fp16 values are below 2^16 and at least 2^-24, so their sums of squares never leave float32's
   // range (a zero vector sums to exactly 0); for bf16 a row out of range is summed again with its
   // values scaled by a power of two taken from its largest magnitude (exact scaling; squares more
   // than 2^-100 below the largest one are negligible)
   if (!F16 && __any_sync(0xffffffffu, any)) {   // the whole warp takes part in the shuffles
-#pragma unroll
+#pragma unroll 1
     for (int g = 0; g < 4; ++g) {
       uint32_t mx = 0;   // largest |x| as a bit pattern (ordered like the magnitudes)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint32_t wv[4] = {xr.v[g][i].x, xr.v[g][i].y, xr.v[g][i].z, xr.v[g][i].w};
+        const uint4 v = chunk(g, i);
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) mx = max(mx, max((wv[q] << 16) & 0x7FFFFFFFu, wv[q] & 0x7FFF0000u));
       }
@@ -345,7 +444,8 @@ __device__ __forceinline__ void tile_norms(const XRegs &xr, float (&nrm)[4]) {
       float s = 0.f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint32_t wv[4] = {xr.v[g][i].x, xr.v[g][i].y, xr.v[g][i].z, xr.v[g][i].w};
+        const uint4 v = chunk(g, i);
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float a = H16<F16>::lo(wv[q]) * sc, b = H16<F16>::hi(wv[q]) * sc;
@@ -356,16 +456,6 @@ __device__ __forceinline__ void tile_norms(const XRegs &xr, float (&nrm)[4]) {
       s += __shfl_xor_sync(0xffffffffu, s, 16);
       if (bad[g]) nrm[g] = mx == 0 ? 0.f : ldexpf(sqrtf(s), e);
     }
-  }
-}
-
-__device__ __forceinline__ void store_tile(const XRegs &xr, unsigned char *xtile, int w, int lane) {
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    const int t = 32 * w + 8 * g + (lane & 7);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      *reinterpret_cast<uint4 *>(xtile + tc::tile_off(kTT, t, 8 * (4 * i + (lane >> 3)))) = xr.v[g][i];
   }
 }
 
@@ -393,20 +483,22 @@ __device__ __forceinline__ void mma_tile_ts(uint32_t d, uint32_t a_tmem, uint32_
                                             bool accumulate_first) {
 #pragma unroll 1
   for (int s = 0; s < 8; ++s)
-    mma_bf16_ts(d, a_tmem + 8 * s, tc::smem_desc(b + s * 2 * kLBO, kLBO, kSBO), idesc,
+    mma_bf16_ts(d, a_tmem + 8 * s, tc::smem_desc_sw128(tc::sw128_kstep(b, kTT, s)), idesc,
                 (accumulate_first || s) ? 1u : 0u);
 }
 
 // Issue the 8 K-steps of one split product D (+)= A B^T (A, B: 128 x 128 bf16 tiles).
-__device__ __forceinline__ void mma_tile(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc, bool accumulate_first) {
+__device__ __forceinline__ void mma_tile(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc, bool accumulate_first,
+                                         int rows_b = kTT) {
 #pragma unroll 1
   for (int s = 0; s < 8; ++s)
-    tc::mma_bf16(d, tc::smem_desc(a + s * 2 * kLBO, kLBO, kSBO), tc::smem_desc(b + s * 2 * kLBO, kLBO, kSBO), idesc,
-                 (accumulate_first || s) ? 1u : 0u);
+    tc::mma_bf16(d, tc::smem_desc_sw128(tc::sw128_kstep(a, kTT, s)), tc::smem_desc_sw128(tc::sw128_kstep(b, rows_b, s)),
+                 idesc, (accumulate_first || s) ? 1u : 0u);
 }
 
 template <bool QJL, int BITS, bool F16>
-__global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
+    quantize_tc_kernel(const QuantParams p, const __grid_constant__ CUtensorMap xmap) {
   using L = Ws<QJL>;
   constexpr int CPT = 64;                         // columns per epilogue thread
   constexpr int WPT = CPT * BITS / 32;            // code-stream words per epilogue thread
@@ -418,26 +510,27 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const
   const uint32_t sbase = smem_u32(smem);
   const Bars<QJL> bar{sbase + L::kBar};
   float *cb = reinterpret_cast<float *>(smem + L::kCb);
-  const uint16_t *x = static_cast<const uint16_t *>(p.x);
   const int64_t n_tiles = (p.rows + kTT - 1) / kTT;
   const int n_my = n_tiles > blockIdx.x ? (int)((n_tiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
   auto row0_of = [&](int i) -> int64_t { return ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * kTT; };
 
   // ---- set-up: split matrices, codebook, barriers, tensor memory ----
-  load_split<L::kThreads, F16>(smem + L::kPhi, smem + L::kPlo, p.Pi);
+  load_split<L::kThreads, F16, !QJL>(smem + L::kPhi, smem + L::kPlo, p.Pi);
   if constexpr (QJL) load_split<L::kThreads, F16>(smem + L::kMhi, smem + L::kMlo, p.SPiT);
   if (tid < NL) cb[tid] = p.codebook[tid];
   if (tid == 0) {
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar.x_full(s), 128);
-      mbar_init(bar.x_empty(s), 1);
+    for (int s = 0; s < L::kNX; ++s) {
+      mbar_init(bar.x_full(s), 1);                         // the copy thread's expect_tx
+      mbar_init(bar.x_empty(s), 1 + 32 * L::kNormWarps);   // the first product's commit + the norm threads
     }
-    mbar_init(bar.d1_full(), 1);
-    mbar_init(bar.d1_empty(), kEpiWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar.d1_full(b), 1);
+      mbar_init(bar.d1_empty(b), kEpiWarps);
+    }
     mbar_init(bar.e_full(), kEpiWarps);
     mbar_init(bar.d2_full(), 1);
     mbar_init(bar.d2_empty(), kEpiWarps);
-    for (int k = 0; k < kNormRing; ++k) mbar_init(bar.n_full(k), 128);
+    for (int k = 0; k < kNormRing; ++k) mbar_init(bar.n_full(k), 32 * L::kNormWarps);
     mbar_fence_init();
   }
   if (warp == 0) {
@@ -451,40 +544,57 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + L::kTslot);
   bool ok = true;
 
-  if (warp >= kEpiWarps && warp < L::kMmaWarp) {
-    // ------------------------------- loaders -------------------------------
+  if (warp == L::kTmaWarp) {
+    // --------------------------- tensor-map copies ---------------------------
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
+      int issued = 0;
+      for (int i = 0; i < n_my; ++i) {
+        const int s = i % L::kNX;
+        // A tile s is free once tile i - kNX's first product is done and its norms are read
+        if (i >= L::kNX && !mbar_wait(bar.x_empty(s), ((i / L::kNX) - 1) & 1)) break;
+        mbar_arrive_expect_tx(bar.x_full(s), kTile);
+        const uint32_t dst = sbase + L::kX + s * kTile;
+        const int row0 = (int)row0_of(i);
+#pragma unroll 1
+        for (int kb = 0; kb < 2; ++kb) tma_x_chunk(dst + kb * (kTile / 2), &xmap, 64 * kb, row0, bar.x_full(s));
+        ++issued;
+      }
+      // no copy may still be landing when the CTA exits
+      for (int i = max(0, issued - L::kNX); i < issued; ++i) mbar_wait(bar.x_full(i % L::kNX), (i / L::kNX) & 1);
+    }
+  } else if (warp >= kEpiWarps && warp < L::kTmaWarp) {
+    // ------------------------------- norms -------------------------------
     const int w = warp - kEpiWarps;
-    XRegs xr;
     TileCursor cur;
     cur.init(p);
-    if (n_my > 0) load_tile(xr, x, row0_of(0), p.rows, w, lane);
     for (int i = 0; i < n_my; ++i) {
+      const int s = i % L::kNX;
+      if (!mbar_wait(bar.x_full(s), (i / L::kNX) & 1)) {
+        ok = false;
+        break;
+      }
       const int64_t row0 = row0_of(i);
       float nrm[4];
-      tile_norms<F16>(xr, nrm);
+      tile_norms<F16>(smem + L::kX + s * kTile, w, lane, nrm);
+      mbar_arrive(bar.x_empty(s));   // this thread is done reading the tile
       if ((lane >> 3) == 0) {
+        float *ring = reinterpret_cast<float *>(smem + L::kNrm) + (i & (kNormRing - 1)) * 128;
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const int r = 32 * w + 8 * g + lane;
+          ring[r] = nrm[g];
           if (row0 + r < p.rows) p.norm[cur.slot(p, r)] = nrm[g];
         }
       }
       cur.advance(p);
-      mbar_arrive(bar.n_full(i & (kNormRing - 1)));   // releases this lane's norm stores
-      // A tile i & 1 is free once the first product of tile i - 2 is done
-      if (i >= 2 && !mbar_wait(bar.x_empty(i & 1), ((i >> 1) - 1) & 1)) {
-        ok = false;
-        break;
-      }
-      store_tile(xr, smem + L::kX + (i & 1) * kTile, w, lane);
-      tc::fence_proxy_async();
-      mbar_arrive(bar.x_full(i & 1));
-      if (i + 1 < n_my) load_tile(xr, x, row0_of(i + 1), p.rows, w, lane);
+      mbar_arrive(bar.n_full(i & (kNormRing - 1)));   // releases this lane's ring entries
     }
   } else if (warp == L::kMmaWarp) {
     // ----------------------------- MMA issuer ------------------------------
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16(kTT, kTD, !F16);
+      const uint32_t idesc_w = tc::idesc_bf16(kTT, L::kPW, !F16);
       int last_pi = -1, last_sk = -1;
       auto sketch = [&](int j) -> bool {   // D2 = E_hi M_hi^T + E_hi M_lo^T + E_lo M_hi^T
         if (!mbar_wait(bar.e_full(), j & 1)) return false;
@@ -499,16 +609,23 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const
         return true;
       };
       for (int i = 0; i < n_my && ok; ++i) {
-        if (!mbar_wait(bar.x_full(i & 1), (i >> 1) & 1) || (i >= 1 && !mbar_wait(bar.d1_empty(), (i - 1) & 1))) {
+        const int xs = i % L::kNX;
+        const int db = i % L::kND1;
+        if (!mbar_wait(bar.x_full(xs), (i / L::kNX) & 1) ||
+            (i >= L::kND1 && !mbar_wait(bar.d1_empty(db), ((i / L::kND1) - 1) & 1))) {
           ok = false;
           break;
         }
         tc::fence_after();
-        const uint32_t xa = sbase + L::kX + (i & 1) * kTile;
-        mma_tile(tmem, xa, sbase + L::kPhi, idesc, false);
-        mma_tile(tmem, xa, sbase + L::kPlo, idesc, true);
-        tc::commit(bar.x_empty(i & 1));
-        tc::commit(bar.d1_full());
+        const uint32_t xa = sbase + L::kX + xs * kTile;
+        if constexpr (L::kPW == 256) {
+          mma_tile(tmem + 256 * db, xa, sbase + L::kPhi, idesc_w, false, 2 * kTT);
+        } else {
+          mma_tile(tmem, xa, sbase + L::kPhi, idesc, false);
+          mma_tile(tmem, xa, sbase + L::kPlo, idesc, true);
+        }
+        tc::commit(bar.x_empty(xs));
+        tc::commit(bar.d1_full(db));
         last_pi = i;
         if constexpr (QJL)
           if (i >= 1) ok = sketch(i - 1);
@@ -516,7 +633,7 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const
       if constexpr (QJL)
         if (ok && n_my > 0) ok = sketch(n_my - 1);
       // nothing may still write tensor memory when it is freed
-      if (last_pi >= 0) mbar_wait(bar.d1_full(), last_pi & 1);
+      if (last_pi >= 0) mbar_wait(bar.d1_full(last_pi % L::kND1), (last_pi / L::kND1) & 1);
       if (last_sk >= 0) mbar_wait(bar.d2_full(), last_sk & 1);
     }
   } else {
@@ -531,26 +648,15 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const
     for (int j = 0; j < NL - 1; ++j) th[j] = 0.5f * (cb[j] + cb[j + 1]);
 #pragma unroll
     for (int j = 0; j < NC; ++j) cvk[j] = QJL && j < NL ? cb[j] : 0.f;
+    FmaSearch<BITS> fs;
+    fs.init(th);
     float *rho = reinterpret_cast<float *>(smem + L::kRho);   // [3][128]: the h = 1 half's sum of e^2
     float e2prev = 0.f;
     int64_t slot_prev = 0;
     bool vprev = false;
-    // slot and ||x|| of the next tile, fetched one tile ahead so that the L2
-    // round trip of the loader's norm store overlaps the current tile's work
-    float n_next = 0.f;
-    int64_t slot_next = 0;
-    bool valid_next = false;
+    const float *nrm_ring = reinterpret_cast<const float *>(smem + L::kNrm);
     TileCursor cur;
     cur.init(p);
-    auto fetch_norm = [&](int i) -> bool {   // tiles are fetched in order 0, 1, 2, ...
-      if (!mbar_wait(bar.n_full(i & (kNormRing - 1)), (i / kNormRing) & 1)) return false;
-      valid_next = row0_of(i) + t < p.rows;
-      slot_next = valid_next ? cur.slot(p, t) : 0;
-      n_next = valid_next ? __ldcg(p.norm + slot_next) : 0.f;
-      cur.advance(p);
-      return true;
-    };
-    if (n_my > 0) ok = fetch_norm(0);
 
     // Every epilogue thread runs all n_my + 1 iterations (after a failed wait it
     // skips the work but still meets the pair barrier of each iteration).
@@ -560,20 +666,41 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const
       bool valid = false;
       if (i < n_my && ok) {
         // ---- first epilogue of tile i: codes (and, keys, the residual into E[i & 1]) ----
-        if (!mbar_wait(bar.d1_full(), i & 1)) {
+        // ||x|| of this token from the norm warps' ring (read before D1 is released, which keeps
+        // the ring slot from being overwritten: see kNormRing)
+        float n = 0.f;
+        if (!mbar_wait(bar.n_full(i & (kNormRing - 1)), (i / kNormRing) & 1)) {
+          ok = false;
+        } else {
+          n = nrm_ring[(i & (kNormRing - 1)) * 128 + t];
+          valid = row0_of(i) + t < p.rows;
+          slot = valid ? cur.slot(p, t) : 0;
+          cur.advance(p);
+        }
+        const int db = i % L::kND1;
+        if (!ok || !mbar_wait(bar.d1_full(db), (i / L::kND1) & 1)) {
           ok = false;
         } else {
           tc::fence_after();
           uint32_t r[CPT];
-          tc::ld32(tmem + lane_ofs + CPT * h, *reinterpret_cast<uint32_t (*)[32]>(r));
-          tc::ld32(tmem + lane_ofs + CPT * h + 32, *reinterpret_cast<uint32_t (*)[32]>(r + 32));
+          const uint32_t d1 = tmem + lane_ofs + 256 * db + CPT * h;
+          tc::ld32(d1, *reinterpret_cast<uint32_t (*)[32]>(r));
+          tc::ld32(d1 + 32, *reinterpret_cast<uint32_t (*)[32]>(r + 32));
           tc::wait_ld();
+          if constexpr (L::kPW == 256) {
+            // the lo-part product sits 128 columns to the right: D1 = x Pi_hi^T + x Pi_lo^T
+#pragma unroll
+            for (int c = 0; c < CPT / 32; ++c) {
+              uint32_t lo[32];
+              tc::ld32(d1 + 128 + 32 * c, lo);
+              tc::wait_ld();
+#pragma unroll
+              for (int q = 0; q < 32; ++q) r[32 * c + q] = __float_as_uint(__uint_as_float(r[32 * c + q]) + __uint_as_float(lo[q]));
+            }
+          }
           tc::fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar.d1_empty());   // D1 may take the next tile's product
-          valid = valid_next;
-          slot = slot_next;
-          const float n = n_next;
+          if (lane == 0) mbar_arrive(bar.d1_empty(db));   // D1 may take the next tile's product
           uint32_t wcur[WPT];
 #pragma unroll
           for (int w = 0; w < WPT; ++w) wcur[w] = 0u;
@@ -608,18 +735,15 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const
             __syncwarp();
             if (lane == 0) mbar_arrive(bar.e_full());
           } else {
-            // values need only the codes: compare D1 = n y against n th (th itself for a zero vector,
-            // whose D1 row is 0), which equals y > th up to one rounding
-            const float sc = n > 0.f ? n : 1.f;
-            float ths[NL - 1];
-#pragma unroll
-            for (int k = 0; k < NL - 1; ++k) ths[k] = th[k] * sc;
+            // values need only the codes (FMA-pipe search on y = D1 / n, 0 for a zero vector)
+            const float inv = n > 0.f ? 1.0f / n : 0.f;
 #pragma unroll
             for (int j = 0; j < CPT; ++j) {
-              uint32_t m[BITS];
-              code_masks<BITS>(__uint_as_float(r[j]), ths, m);
-              put_code<BITS>(wcur, m, j);
+              float f[BITS];
+              fs.flags(__uint_as_float(r[j]) * inv, f);
+              put_code_f<BITS>(wcur, f, j);
             }
+            fix_words<BITS>(wcur, CPT);
           }
           if (valid) {
             uint32_t *rec = p.records + slot * RW + WPT * h;
@@ -628,7 +752,6 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const
           }
         }
       }
-      if (i + 1 < n_my && ok) ok = fetch_norm(i + 1);
       if constexpr (QJL) {
         if (i >= 1) {
           // ---- second epilogue of tile i - 1: sign words and ||e|| ----
@@ -670,8 +793,32 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1) quantize_tc_kernel(const
   if (warp == 0) tc::dealloc(tmem, L::kTmemCols);
 }
 
+// The x rows as a 2-D tensor map: 128 16-bit elements per row, `rows` rows of 256 bytes; a
+// box of 64 elements x 128 rows with 128-byte swizzle is one K block of an A tile. Rows past the
+// end read 0.
+bool make_x_map(CUtensorMap *map, const QuantParams &p, bool f16) {
+  static PFN_cuTensorMapEncodeTiled encode = nullptr;
+  if (!encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess || !fn)
+      return false;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(fn);
+  }
+  const cuuint64_t dims[2] = {(cuuint64_t)kTD, (cuuint64_t)p.rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kTD * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kTT};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                const_cast<void *>(p.x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool QJL, int BITS, bool F16>
 cudaError_t launch_tc(const QuantParams &p, cudaStream_t st) {
+  CUtensorMap xmap;
+  if (p.rows >= (int64_t)1 << 31 || !make_x_map(&xmap, p, F16)) return cudaErrorNotSupported;
   auto kern = quantize_tc_kernel<QJL, BITS, F16>;
   constexpr size_t smem = Ws<QJL>::kBytes;
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
@@ -679,7 +826,7 @@ cudaError_t launch_tc(const QuantParams &p, cudaStream_t st) {
   const int64_t tiles = (p.rows + kTT - 1) / kTT;
   const int64_t slots = (int64_t)device_sm_count();
   const int grid = (int)(tiles < slots ? tiles : slots);
-  kern<<<grid, Ws<QJL>::kThreads, smem, st>>>(p);
+  kern<<<grid, Ws<QJL>::kThreads, smem, st>>>(p, xmap);
   return cudaGetLastError();
 }
 

@@ -20,6 +20,27 @@ __host__ __device__ constexpr uint32_t tile_off(int rows, int row, int k) {
   return (uint32_t)((((k >> 3) * (rows >> 3) + (row >> 3)) << 7) + ((row & 7) << 4) + ((k & 7) << 1));
 }
 
+// Byte offset of element (row, k) in a [rows x 128] K-major 16-bit tile in the 128-byte swizzle
+// layout: two K blocks of 64 elements (each rows x 128 bytes, the second at rows * 128), rows
+// 128 bytes apart, and the 16-byte chunk index of a row XOR (row & 7), in 1024-byte aligned
+// 8-row atoms. This is the layout a tensor-map copy with 128-byte swizzle writes.
+__host__ __device__ constexpr uint32_t sw128_off(int rows, int row, int k) {
+  return (uint32_t)((k >> 6) * rows * 128 + row * 128 + ((((k >> 3) & 7) ^ (row & 7)) << 4) + ((k & 7) << 1));
+}
+
+// Descriptor of a 128-byte-swizzle K-major operand: 8-row groups 1024 bytes apart (stride byte
+// offset), leading byte offset unused for this layout (1), descriptor version 1, layout type 2.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+
+// Start address of K step s (16 elements) of a [rows x 128] 128-byte-swizzle tile at `base`:
+// the K block, then 32 bytes per step inside the block's 128-byte rows.
+__host__ __device__ constexpr uint32_t sw128_kstep(uint32_t base, int rows, int s) {
+  return base + (uint32_t)((s >> 2) * rows * 128 + (s & 3) * 32);
+}
+
 // Shared-memory matrix descriptor: start address, leading (K-direction) and
 // stride (row-direction) byte offsets, descriptor version 1, no swizzle.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
