@@ -227,6 +227,41 @@ def test_workspace_status_clean_after_calls():
     tqb.tq_workspace_status(ws)
 
 
+@pytest.mark.parametrize("kb,G", [(3, 1), (2, 1), (3, 2), (2, 2), (1, 4)])
+def test_logits_unaligned_query_and_matrices(kb, G):
+    # q, Pi and S 4 bytes off a 16-byte boundary: the scans that read them as float4 (the
+    # single-head scan projecting its own queries, the float16-table scan) leave the projection
+    # to a kernel of its own; both layouts must give the oracle's logits
+    d, T, H = 128, 1100, 2
+    Pi, S, ck, cv, g = _setup(d, kb, 3)
+    k = syn.gaussian((1, H, T, d), 51).to(torch.bfloat16)
+    q = syn.gaussian((1, H * G, d), 52)
+    kc = tqb.PackedCache.empty(d, kb, True, 1, H, T)
+    tqb.tq_quantize_append(kc, k.cuda(), 0, g["Pi"], g["SPiT"], g["ck"])
+
+    def shifted(t):
+        buf = torch.empty(t.numel() + 1, dtype=t.dtype, device="cuda")
+        buf[1:] = t.reshape(-1)
+        return buf[1:].view(t.shape)
+
+    qd = q.cuda()
+    runs = [(qd, g["Pi"], g["S"]), (shifted(qd), shifted(g["Pi"]), shifted(g["S"]))]
+    assert runs[1][0].data_ptr() % 16 == 4
+    krec = par.as_u32(kc.records.cpu().numpy())
+    kn, kr = kc.norm.cpu().numpy(), kc.rnorm.cpu().numpy()
+    qn = q.numpy().astype(np.float64)
+    for qq, pi, sk in runs:
+        ws = torch.empty(max(256, tqb.tq_logits_workspace_size(kc, H * G)), dtype=torch.uint8, device="cuda")
+        ws.fill_(0xFF)
+        lg = tqb.tq_logits(kc, qq, T, pi, sk, g["ck"], workspace=ws)
+        torch.cuda.synchronize()
+        tqb.tq_workspace_status(ws)
+        lg_np = lg.cpu().numpy()
+        for h in range(H):
+            par.check_logits(lg_np[0, h * G:(h + 1) * G], qn[0, h * G:(h + 1) * G], Pi, S, ck, krec[0, h],
+                             kn[0, h], kr[0, h], d, kb)
+
+
 # ---------------------------------------------------------------------------
 # full-size workloads, sampled
 # ---------------------------------------------------------------------------
