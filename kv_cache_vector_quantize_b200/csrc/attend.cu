@@ -146,7 +146,9 @@ __global__ void __launch_bounds__(kAThreads) attend_chunk_kernel(const AttendPar
 
 // Merge of the chunks of one query head: scale factors e^{m_c - M} once, the
 // chunk sums split over all threads with independent loads in flight, then
-// out = Pi^T A / L, with Pi staged in shared memory when it fits.
+// out = Pi^T A / L, with Pi staged in shared memory when it fits. Launched as a
+// programmatic dependent of the chunk grid: it stages Pi while that grid's last
+// CTAs run and waits for the grid before reading any partial.
 constexpr int kCThreads = 512;
 __global__ void __launch_bounds__(kCThreads) attend_combine_kernel(const float *__restrict__ partial, int n_chunks,
                                                                    int d, const float *__restrict__ Pi,
@@ -162,6 +164,7 @@ __global__ void __launch_bounds__(kCThreads) attend_combine_kernel(const float *
     const float4 *src = reinterpret_cast<const float4 *>(Pi);
     for (int e = tid; e < d * d / 4; e += kCThreads) reinterpret_cast<float4 *>(pis)[e] = __ldg(src + e);
   }
+  pdl_wait();   // the partials come from the chunk grid (a programmatic primary, or plainly finished)
   float m = -INFINITY;
   for (int c = tid; c < n_chunks; c += kCThreads) m = fmaxf(m, part[(size_t)c * (d + 2)]);
   m = block_reduce(m, red, true);
@@ -258,8 +261,17 @@ cudaError_t launch_combine(const float *partial, int rows, int n_chunks, int d, 
   const size_t smem = cs_bytes + (pi_in_smem ? pi_bytes : 0);
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(attend_combine_kernel), smem);
   if (e != cudaSuccess) return e;
-  attend_combine_kernel<<<rows, kCThreads, smem, st>>>(partial, n_chunks, d, Pi, out, pi_in_smem);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)rows);
+  cfg.blockDim = dim3(kCThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attend_combine_kernel, partial, n_chunks, d, Pi, out, pi_in_smem);
 }
 
 size_t attend_chunk_smem(int d, int bits, int64_t chunk) { return chunk_smem(d, bits, chunk); }

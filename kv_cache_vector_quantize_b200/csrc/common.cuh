@@ -134,6 +134,10 @@ size_t gqa_table_bytes(int units);
 cudaError_t launch_logits_gqa(const LogitsParams &p, const GqaParams &g, int bits, int n_seq, size_t limit,
                               cudaStream_t st);
 cudaError_t launch_attend(const AttendParams &p, int bits, int n_seq, size_t smem, cudaStream_t st);
+// d = 128 softmax.V streamed by bulk copies (attend_fast.cu); p.chunk from attend_fast_chunk.
+bool attend_fast_supported(int d, int bits, int q_per_cta, const void *records);
+int64_t attend_fast_chunk(int64_t n_tokens, int units);
+cudaError_t launch_attend_fast(const AttendParams &p, int bits, int n_seq, cudaStream_t st);
 size_t attend_chunk_smem(int d, int bits, int64_t chunk);
 cudaError_t launch_combine(const float *partial, int rows, int n_chunks, int d, const float *Pi,
                            float *out, cudaStream_t st);

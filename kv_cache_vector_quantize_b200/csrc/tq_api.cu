@@ -406,10 +406,18 @@ tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale, int32
   p.group = group;
   p.q_per_cta = group < kAttendMaxQ ? group : kAttendMaxQ;
   p.qblocks = (group + p.q_per_cta - 1) / p.q_per_cta;
-  const size_t smem = attend_chunk_smem(v->d, v->idx_bits, kAttendChunk);
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "tq_attend_v (status)");
-  e = launch_attend(p, v->idx_bits, v->n_seq, smem, (cudaStream_t)stream);
+  if (attend_fast_supported(v->d, v->idx_bits, p.q_per_cta, v->records)) {
+    // d = 128: tiles streamed by bulk copies, chunks sized to whole waves (never more chunks than
+    // the 512-token split the workspace is sized for)
+    p.chunk = attend_fast_chunk(n_tokens, v->n_seq * v->n_kv_heads * p.qblocks);
+    p.n_chunks = (int)((n_tokens + p.chunk - 1) / p.chunk);
+    e = launch_attend_fast(p, v->idx_bits, v->n_seq, (cudaStream_t)stream);
+  } else {
+    e = launch_attend(p, v->idx_bits, v->n_seq, attend_chunk_smem(v->d, v->idx_bits, kAttendChunk),
+                      (cudaStream_t)stream);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "tq_attend_v (chunks)");
   e = launch_combine(partial, v->n_seq * n_q_heads, p.n_chunks, v->d, Pi, out, (cudaStream_t)stream);
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_attend_v (merge)");
