@@ -302,9 +302,16 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
   int nq = 0, seq = 0, h0 = 0;
   size_t unit_first = 0;
   float *tables = reinterpret_cast<float *>(smem + (T0 - dyn0));
+  // per-unit values, set at each table build: this unit's logits row, norm and rnorm
+  // pointers, and whether its norms come with the tiles (tiles start 512 keys apart)
+  float *lg_row = nullptr;
+  const float *nrm_p = nullptr, *rho_p = nullptr;
+  bool unit_nc = false;
+  const int k = warp * 32 + lane;   // this lane's key in a tile
+  int s = 0;                        // stage of key tile i, and its phase parity
+  uint32_t phase = 0;
 
   for (int i = 0; i < n_my; ++i) {
-    const int s = i % stages;
     if (vunit != cur_unit) {
       // (re)build this unit's tables; all consumer warps take part
       asm volatile("bar.sync 1, %0;" ::"n"(32 * kFConsumers) : "memory");
@@ -315,6 +322,10 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
       const int kvh = sk - seq * p.n_kv_heads;
       h0 = kvh * p.group + qb * p.q_per_cta;
       nq = min(p.q_per_cta, p.group - qb * p.q_per_cta);
+      lg_row = p.logits + ((size_t)seq * p.n_q_heads + h0) * p.n_tokens;
+      nrm_p = p.norm + unit_first;
+      rho_p = p.rnorm + unit_first;
+      unit_nc = (reinterpret_cast<uintptr_t>(nrm_p) % 16 == 0) && (reinterpret_cast<uintptr_t>(rho_p) % 16 == 0);
       float *qv = reinterpret_cast<float *>(smem + (qst - dyn0));   // [qq][Pi q | S q][128]
       for (int e = tid; e < nq * 2 * kFD; e += 32 * kFConsumers) {
         const int qq = e / (2 * kFD), r = e - qq * 2 * kFD;
@@ -381,15 +392,13 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
       asm volatile("bar.sync 1, %0;" ::"n"(32 * kFConsumers) : "memory");
     }
 
-    if (!mbar_wait(full_bar(s), (i / stages) & 1)) {
+    if (!mbar_wait(full_bar(s), phase)) {
       atomicOr(p.status, kDevTimeout);
       return;
     }
     const int64_t t0 = (int64_t)tile * kFTile;
     const int n = (int)min((int64_t)kFTile, p.n_tokens - t0);
-    const int k = warp * 32 + lane;
     const bool valid = k < n;
-    const size_t first = unit_first + t0;
     const unsigned char *st = smem + (slot(s) - dyn0);
     uint32_t w[RW];
     if (valid) {
@@ -408,16 +417,20 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
     }
     float nrm = 0.f, rho = 0.f;
     if (valid) {
-      if (norms_by_copy(first, n)) {
+      if (unit_nc && (n & 3) == 0) {   // the producer's condition (norms_by_copy) for this tile
         nrm = reinterpret_cast<const float *>(st + kFTile * RW * 4)[k];
         rho = reinterpret_cast<const float *>(st + kFTile * RW * 4 + kFTile * 4)[k];
       } else {
-        nrm = __ldg(p.norm + first + k);
-        rho = __ldg(p.rnorm + first + k);
+        nrm = __ldg(nrm_p + t0 + k);
+        rho = __ldg(rho_p + t0 + k);
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_bar(s));   // this warp is done with the stage
+    if (++s == stages) {
+      s = 0;
+      phase ^= 1u;
+    }
 
     float out[QMAX];
 #pragma unroll
@@ -466,7 +479,7 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
     if (valid) {
 #pragma unroll
       for (int qq = 0; qq < QMAX; ++qq)
-        if (qq < nq) p.logits[((size_t)seq * p.n_q_heads + h0 + qq) * p.n_tokens + t0 + k] = out[qq];
+        if (qq < nq) lg_row[qq * p.n_tokens + t0 + k] = out[qq];
     }
     if (++tile == fp.tiles_per_unit) {
       tile = 0;
