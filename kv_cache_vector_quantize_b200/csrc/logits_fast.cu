@@ -256,11 +256,11 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
   if (warp == kFConsumers) {
     // ------------------------------ producer ------------------------------
     if (lane == 0) {
-      int issued = 0, vunit = unit0, tile = tile0;
+      int issued = 0, vunit = unit0, tile = tile0, s = 0;
+      uint32_t phase = 1u;   // parity of the empty-barrier phase a stage's reuse waits for
       size_t unit_first = (size_t)(vunit / p.qblocks) * p.capacity;
       for (int i = 0; i < n_my; ++i) {
-        const int s = i % stages;
-        if (i >= stages && !mbar_wait(empty_bar(s), ((i / stages) - 1) & 1)) {
+        if (i >= stages && !mbar_wait(empty_bar(s), phase)) {
           pdl_wait();
           atomicOr(p.status, kDevTimeout);
           break;
@@ -278,6 +278,10 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
           bulk_g2s(st + kFTile * RW * 4 + kFTile * 4, p.rnorm + first, 4u * n, full_bar(s));
         }
         ++issued;
+        if (++s == stages) {
+          s = 0;
+          phase ^= 1u;
+        }
         if (++tile == fp.tiles_per_unit) {
           tile = 0;
           ++vunit;

@@ -307,10 +307,10 @@ __global__ void __launch_bounds__(kGThreads, 1) logits_gqa_kernel(const GScan gs
   if (warp == kGConsumers) {
     // ------------------------------ producer ------------------------------
     if (lane == 0) {
-      int issued = 0;
+      int issued = 0, s = 0;
+      uint32_t phase = 1u;   // parity of the empty-barrier phase a stage's reuse waits for
       for (int i = 0; i < n_my; ++i) {
-        const int s = i % stages;
-        if (i >= stages && !mbar_wait(empty_bar(s), ((i / stages) - 1) & 1)) {
+        if (i >= stages && !mbar_wait(empty_bar(s), phase)) {
           pdl_wait();
           atomicOr(p.status, kDevTimeout);
           break;
@@ -328,6 +328,10 @@ __global__ void __launch_bounds__(kGThreads, 1) logits_gqa_kernel(const GScan gs
           bulk_g2s(st + kGTile * RW * 4 + kGTile * 4, p.rnorm + first, 4u * n, full_bar(s));
         }
         ++issued;
+        if (++s == stages) {
+          s = 0;
+          phase ^= 1u;
+        }
       }
       for (int i = max(0, issued - stages); i < issued; ++i)
         if (!mbar_wait(full_bar(i % stages), (i / stages) & 1)) {
@@ -370,18 +374,23 @@ __global__ void __launch_bounds__(kGThreads, 1) logits_gqa_kernel(const GScan gs
   uint32_t xv[16];
 #pragma unroll
   for (int m = 0; m < 16; ++m) xv[m] = x0 ^ ((uint32_t)m * (0x202u << PSH));
+  // the unit's logits rows and norm pointers; its norms come with the tiles when aligned (tiles
+  // start 512 keys apart, so one check per unit decides it with the tile's length)
+  float *lg_row = p.logits + ((size_t)seq * p.n_q_heads + h0) * p.n_tokens;
+  const float *nrm_p = p.norm + unit_first, *rho_p = p.rnorm + unit_first;
+  const bool unit_nc = (reinterpret_cast<uintptr_t>(nrm_p) % 16 == 0) && (reinterpret_cast<uintptr_t>(rho_p) % 16 == 0);
+  const int k = warp * 32 + lane;
+  int s = 0;
+  uint32_t phase = 0;
 
   for (int i = 0; i < n_my; ++i) {
-    const int s = i % stages;
-    if (!mbar_wait(full_bar(s), (i / stages) & 1)) {
+    if (!mbar_wait(full_bar(s), phase)) {
       atomicOr(p.status, kDevTimeout);
       return;
     }
     const int64_t t0 = (int64_t)(g0 + i) * kGTile;
     const int n = (int)min((int64_t)kGTile, p.n_tokens - t0);
-    const int k = warp * 32 + lane;
     const bool valid = k < n;
-    const size_t first = unit_first + t0;
     const unsigned char *st = smem + (slot(s) - dyn0);
     uint32_t w[RW];
     if (valid) {
@@ -400,16 +409,20 @@ __global__ void __launch_bounds__(kGThreads, 1) logits_gqa_kernel(const GScan gs
     }
     float nrm = 0.f, rho = 0.f;
     if (valid) {
-      if (norms_by_copy(first, n)) {
+      if (unit_nc && (n & 3) == 0) {   // the producer's condition (norms_by_copy) for this tile
         nrm = reinterpret_cast<const float *>(st + kGTile * RW * 4)[k];
         rho = reinterpret_cast<const float *>(st + kGTile * RW * 4 + kGTile * 4)[k];
       } else {
-        nrm = __ldg(p.norm + first + k);
-        rho = __ldg(p.rnorm + first + k);
+        nrm = __ldg(nrm_p + t0 + k);
+        rho = __ldg(rho_p + t0 + k);
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_bar(s));   // this warp is done with the stage
+    if (++s == stages) {
+      s = 0;
+      phase ^= 1u;
+    }
 
     uint32_t wi[IW], wsg[4];
 #pragma unroll
@@ -426,7 +439,7 @@ __global__ void __launch_bounds__(kGThreads, 1) logits_gqa_kernel(const GScan gs
     if (valid) {
 #pragma unroll
       for (int h = 0; h < QH; ++h)
-        p.logits[((size_t)seq * p.n_q_heads + h0 + h) * p.n_tokens + t0 + k] = nrm * sg[h] * fmaf(rho, fs[h], fi[h]);
+        lg_row[h * p.n_tokens + t0 + k] = nrm * sg[h] * fmaf(rho, fs[h], fi[h]);
     }
   }
 }
