@@ -49,10 +49,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0
 # stands (profiles/), keyed by (kernel, workload); a key is removed when its
 # kernel changes, and the bench then reports traffic as null.
 NCU_TRAFFIC = {
-    ("quantize_k", "llama"): 67_335_680 + 2_341_632,   # quantize_tc_kernel<1, 2, 0>
-    ("quantize_v", "llama"): 67_250_944 + 1_929_728,   # quantize_tc_kernel<0, 3, 0>
-    ("logits", "llama"): 15_757_312 + 0,               # logits_gqa_kernel<2, 4> (the scan; tables read from L2)
-    ("logits", "sweep-b3"): 2 * (234_968_320 + 14_149_632),   # logits_fast_kernel<2, 1>, 4-sequence capture x 2
+    ("quantize_k", "llama"): 67_326_976 + 2_125_824,   # quantize_tc_kernel<1, 2, 0>
+    ("quantize_v", "llama"): 67_240_704 + 2_118_144,   # quantize_tc_kernel<0, 3, 0>
+    ("logits", "sweep-b3"): 2 * (234_978_304 + 16_730_368),   # logits_fast_kernel<2, 1>, 4-sequence capture x 2
+    ("attend_v", "sweep-b3"): 2 * (234_927_616 + 3_965_184),  # attend_fast_kernel<3, 1>, 4-sequence capture x 2
+    ("logits", "llama"): 15_756_288 + 0,               # logits_gqa_kernel<2, 4> (the scan; tables read from L2)
+    ("attend_v", "llama"): 17_871_872 + 0,             # attend_fast_kernel<3, 4> (records, norms and logits)
 }
 
 
@@ -338,7 +340,8 @@ def run_tq(args, rank, world, local_rank):
                  "algorithmic": f"{kb // head_vectors} B per key (record + norm + rnorm)"}
     att_gbs = vb / (mean["attend_v"] * 1e-3) / 1e9
     roof_att = {"kernel": "tq_attend_v (chunk softmax.V + merge)", "bound": "hbm", "achieved": round(att_gbs, 1),
-                "peak": hbm, "unit": "GB/s", "frac": round(att_gbs / hbm, 4), "traffic": None, "peak_source": src_txt,
+                "peak": hbm, "unit": "GB/s", "frac": round(att_gbs / hbm, 4),
+                "traffic": NCU_TRAFFIC.get(("attend_v", args.workload)), "peak_source": src_txt,
                 "algorithmic": f"{vb // head_vectors} B per value (record + norm)"}
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
