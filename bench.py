@@ -274,6 +274,27 @@ def run_tq(args, rank, world, local_rank):
     head_vectors = w["n_seq"] * w["hkv"] * w["T"]
     quant_tps = world * w["n_seq"] * w["T"] / (quant_ms * 1e-3)
 
+    # ---- the one-call decode step (tq_decode_attend) on the same caches, L2 flushed before each ----
+    ws_d = torch.empty(max(256, tqb.tq_decode_workspace_size(kc, vc, w["hq"], w["T"])), dtype=torch.uint8, device=dev)
+    out_d = torch.empty_like(out)
+
+    def decode_step():
+        tqb.tq_decode_attend(kc, vc, q, w["T"], scale, Pi, S, ck, cv, out=out_d, workspace=ws_d)
+
+    for _ in range(3):
+        flush.fill_(1.0)
+        decode_step()
+    torch.cuda.synchronize(dev)
+    dec_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in dec_evs:
+        flush.fill_(1.0)
+        a.record(stream)
+        decode_step()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    tqb.tq_workspace_status(ws_d)
+    dec_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in dec_evs) / len(dec_evs)], dev, world)[0]
+
     # ---- end to end: pinned host inputs in, result out, through the public API ----
     e2e = None
     if args.e2e_steps > 0:
@@ -358,10 +379,22 @@ def run_tq(args, rank, world, local_rank):
         "packed_bytes": {"keys": kb, "values": vb},
         "roofline": roofline, "roofline_logit_scan": roof_scan, "roofline_quantize_v": roof_qv,
         "roofline_attend_v": roof_att,
+        "roofline_decode_attend": decode_roof(dec_ms, mean["logits"] + mean["attend_v"], kb + vb, w, hbm, src_txt),
         "gpu_launches": kernels_per_step * args.steps,
         "clocks": clk, "e2e": e2e,
     }
     return result, w
+
+
+def decode_roof(ms, two_call_ms, nbytes, w, hbm, src_txt):
+    """The one-call decode step against HBM: packed key + value bytes per call / its time."""
+    one_pass = w["hq"] == w["hkv"] and w["d"] == 128 and w["k_idx"] in (1, 2)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"kernel": "tq_decode_attend (" + ("query projection + fused logits/softmax.V pass + merge" if one_pass
+                                              else "tq_logits + tq_attend_v") + ")",
+            "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+            "traffic": None, "peak_source": src_txt, "ms": round(ms, 5),
+            "two_calls_ms": round(two_call_ms, 5), "algorithmic": "packed key and value records + norms per call"}
 
 
 def run_large(args, rank, world, local_rank):
@@ -385,6 +418,8 @@ def run_large(args, rank, world, local_rank):
     out = torch.empty((1, w["hq"], d), dtype=torch.float32, device=dev)
     ws_l = torch.empty(tqb.tq_logits_workspace_size(kc, w["hq"]), dtype=torch.uint8, device=dev)
     ws_a = torch.empty(tqb.tq_attend_workspace_size(vc, w["hq"], T), dtype=torch.uint8, device=dev)
+    ws_d = torch.empty(max(256, tqb.tq_decode_workspace_size(kc, vc, w["hq"], T)), dtype=torch.uint8, device=dev)
+    out_d = torch.empty_like(out)
     flush = torch.empty((2 * torch.cuda.get_device_properties(dev).L2_cache_size) // 4, dtype=torch.float32,
                         device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -408,12 +443,19 @@ def run_large(args, rank, world, local_rank):
         tqb.tq_attend_v(vc, logits, scale, T, Pi, cv, out=out, workspace=ws_a)
         if ev is not None:
             ev[5].record(stream)
+        flush.fill_(1.0)   # the one-call decode step on the same caches, from HBM
+        if ev is not None:
+            ev[6].record(stream)
+        tqb.tq_decode_attend(kc, vc, q, T, scale, Pi, S, ck, cv, out=out_d, workspace=ws_d)
+        if ev is not None:
+            ev[7].record(stream)
 
     k, v, q = w["gen"](dev, rank_seed(rank))
     for _ in range(args.warmup):
         path(k, v, q)
     torch.cuda.synchronize(dev)
-    per = {n: 0.0 for n in ("quantize_k", "quantize_v", "l2_flush", "logits", "attend_v")}
+    per = {n: 0.0 for n in ("quantize_k", "quantize_v", "l2_flush", "logits", "attend_v", "l2_flush_2",
+                            "decode_attend")}
     clocks = ClockSampler(dev.index)
     if world > 1:
         dist.barrier()
@@ -422,7 +464,7 @@ def run_large(args, rank, world, local_rank):
         if layer > 0:
             del k, v
             k, v, q = w["gen"](dev, layer + rank_seed(rank))   # untimed input generation
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
         torch.cuda.synchronize(dev)
         path(k, v, q, ev)
         torch.cuda.synchronize(dev)
@@ -431,9 +473,10 @@ def run_large(args, rank, world, local_rank):
     clocks.mark_end()
     tqb.tq_workspace_status(ws_l)
     tqb.tq_workspace_status(ws_a)
+    tqb.tq_workspace_status(ws_d)
     clk = clocks.stop()
-    logits_ms, quant_ms, total_ms = max_over_ranks(
-        [per["logits"], per["quantize_k"] + per["quantize_v"], sum(per.values())], dev, world)
+    logits_ms, quant_ms, total_ms, dec_ms = max_over_ranks(
+        [per["logits"], per["quantize_k"] + per["quantize_v"], sum(per.values()), per["decode_attend"]], dev, world)
     L = args.layers
     kb, vb = key_bytes(w), value_bytes(w)
     fp16_bytes = 2 * H * T * d * 2
@@ -459,7 +502,11 @@ def run_large(args, rank, world, local_rank):
         "roofline_quantize_k": {"kernel": "quantize_tc_kernel (fp16 keys)", "bound": "hbm",
                                 "achieved": round(L * qk_bytes / (per["quantize_k"] * 1e-3) / 1e9, 1), "peak": hbm,
                                 "unit": "GB/s"},
-        "gpu_launches": 6 * L, "clocks": clk, "e2e": None,
+        "roofline_decode_attend": decode_roof(dec_ms / L, (per["logits"] + per["attend_v"]) / L, kb + vb, w, hbm,
+                                              peak_src),
+        # per layer: quantize K, V; projection + scan; V chunks + merge; and the one-call decode step
+        # (projection, fused pass, merge; or the two calls' four kernels and the status merge)
+        "gpu_launches": (6 + (3 if w["k_idx"] in (1, 2) else 5)) * L, "clocks": clk, "e2e": None,
     }
     return result, w
 

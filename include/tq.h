@@ -151,8 +151,32 @@ tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale,
                       const float *Pi, const float *codebook, float *out,
                       void *workspace, size_t workspace_bytes, tq_stream stream);
 
+/* Workspace bytes tq_decode_attend needs for these caches, head count and length
+ * (0 if the caches differ in d, n_seq or n_kv_heads). */
+size_t tq_decode_workspace_size(const tq_cache *k, const tq_cache *v, int32_t n_q_heads, int64_t n_tokens);
+
+/* One decode step on the packed caches: the logits of tq_logits, the softmax
+ * and the value sum of tq_attend_v (usedby.ai, "El Pitch": attention computed
+ * on the compressed cache; zubnet.ai, paragraph 1: keys and values):
+ *   out[s][h] = Pi^T sum_t softmax_t(scale * l_t) * vnorm_t * cV[vcode_t],
+ *   l_t = knorm_t * ( <Pi q, cK[kcode_t]> + krnorm_t * sqrt(pi/2)/d * <S q, 2 sign_t - 1> ).
+ * With one query head per KV head, d = 128 and 1- or 2-bit key codes the whole
+ * step is one pass over the tokens (the logits stay on chip); other shapes run
+ * tq_logits and tq_attend_v inside the workspace and give the same results.
+ *   k: key cache (qjl = 1); v: value cache (qjl = 0), same d, n_seq, n_kv_heads.
+ *   q: [n_seq][n_q_heads][d] float; out: [n_seq][n_q_heads][d] float.
+ *   Pi, S: [d][d] float; codebook_k / codebook_v: 2^idx_bits floats of each cache.
+ * n_q_heads must be a positive multiple of n_kv_heads; n_tokens <= both
+ * capacities (n_tokens == 0 writes zeros); scale finite.
+ * workspace: >= tq_decode_workspace_size bytes, 256-byte aligned; its status
+ * word is read by tq_workspace_status. */
+tq_status tq_decode_attend(const tq_cache *k, const tq_cache *v, const float *q, int32_t n_q_heads,
+                           int64_t n_tokens, float scale, const float *Pi, const float *S,
+                           const float *codebook_k, const float *codebook_v, float *out,
+                           void *workspace, size_t workspace_bytes, tq_stream stream);
+
 /* Synchronises `stream`, reads the status word that the kernels of the last
- * tq_logits / tq_attend_v call on this workspace wrote, and clears it.
+ * tq_logits / tq_attend_v / tq_decode_attend call on this workspace wrote, and clears it.
  * TQ_OK if no kernel reported a failure, TQ_ERR_DEVICE otherwise (the message
  * names the failure). */
 tq_status tq_workspace_status(void *workspace, tq_stream stream);

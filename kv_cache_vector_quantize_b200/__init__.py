@@ -3,7 +3,9 @@
 The package is a thin layer over the C ABI declared in ``include/tq.h``:
 ``tq_quantize_append`` (online quantization of K/V head-vectors into a packed
 cache), ``tq_logits`` (attention logits on the packed keys) and
-``tq_attend_v`` (softmax-weighted packed values), plus the setup helpers
+``tq_attend_v`` (softmax-weighted packed values), ``tq_decode_attend`` (the
+three decode steps in one call, one pass over the tokens where the shapes allow),
+plus the setup helpers
 ``tq_codebook_fit`` and ``tq_sketch_rotation``. All compute runs in the CUDA
 kernels of ``csrc/`` built for sm_100a.
 """
@@ -27,6 +29,8 @@ from ._binding import (  # noqa: F401
     tq_attend_workspace_size,
     tq_codebook_fit,
     tq_debug_inject,
+    tq_decode_attend,
+    tq_decode_workspace_size,
     tq_last_error,
     tq_logits,
     tq_logits_workspace_size,

@@ -57,6 +57,8 @@ def _load() -> ctypes.CDLL:
         "tq_attend_workspace_size": (SZ, [D, I32, I64]),
         "tq_attend_v": (I32, [D, P, F, I32, I64, P, P, P, P, SZ, P]),
         "tq_attend_v_noalloc": (I32, [D, P, F, I32, I64, P, P, P, P]),
+        "tq_decode_workspace_size": (SZ, [D, D, I32, I64]),
+        "tq_decode_attend": (I32, [D, D, P, I32, I64, F, P, P, P, P, P, P, SZ, P]),
         "tq_workspace_status": (I32, [P, P]),
         "tq_last_error": (ctypes.c_char_p, []),
         "tq_debug_inject": (None, [I32, I32]),
@@ -246,6 +248,37 @@ def tq_attend_v(cache: PackedCache, logits: torch.Tensor, scale: float, n_tokens
     _check(_lib.tq_attend_v(ctypes.byref(desc), _ptr(logits), float(scale), hq, int(n_tokens), _ptr(Pi),
                             _ptr(codebook), _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
                             _stream(stream)))
+    return out
+
+
+def tq_decode_workspace_size(kcache: PackedCache, vcache: PackedCache, n_q_heads: int, n_tokens: int) -> int:
+    kd, vd = kcache.desc(), vcache.desc()
+    return int(_lib.tq_decode_workspace_size(ctypes.byref(kd), ctypes.byref(vd), n_q_heads, int(n_tokens)))
+
+
+def tq_decode_attend(kcache: PackedCache, vcache: PackedCache, q: torch.Tensor, n_tokens: int, scale: float,
+                     Pi: torch.Tensor, S: torch.Tensor, codebook_k: torch.Tensor, codebook_v: torch.Tensor,
+                     out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """q [n_seq, H_q, d] float32 -> out [n_seq, H_q, d] float32 (logits, softmax and values in one call)."""
+    if q.dim() != 3 or q.shape[0] != kcache.n_seq or q.shape[2] != kcache.d:
+        raise ValueError(f"q must be [{kcache.n_seq}, H_q, {kcache.d}], got {tuple(q.shape)}")
+    hq = q.shape[1]
+    _need(q, "q", torch.float32, device=kcache.device)
+    _need(Pi, "Pi", torch.float32, (kcache.d, kcache.d), kcache.device)
+    _need(S, "S", torch.float32, (kcache.d, kcache.d), kcache.device)
+    _need(codebook_k, "codebook_k", torch.float32, (1 << kcache.idx_bits,), kcache.device)
+    _need(codebook_v, "codebook_v", torch.float32, (1 << vcache.idx_bits,), kcache.device)
+    if out is None:
+        out = torch.empty((kcache.n_seq, hq, kcache.d), dtype=torch.float32, device=kcache.device)
+    _need(out, "out", torch.float32, (kcache.n_seq, hq, kcache.d), kcache.device)
+    if workspace is None:
+        workspace = torch.empty(max(tq_decode_workspace_size(kcache, vcache, hq, n_tokens), 256), dtype=torch.uint8,
+                                device=kcache.device)
+    kd, vd = kcache.desc(), vcache.desc()
+    _check(_lib.tq_decode_attend(ctypes.byref(kd), ctypes.byref(vd), _ptr(q), hq, int(n_tokens), float(scale),
+                                 _ptr(Pi), _ptr(S), _ptr(codebook_k), _ptr(codebook_v), _ptr(out), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
 
 

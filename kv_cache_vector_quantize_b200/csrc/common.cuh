@@ -134,6 +134,26 @@ size_t gqa_table_bytes(int units);
 cudaError_t launch_logits_gqa(const LogitsParams &p, const GqaParams &g, int bits, int n_seq, size_t limit,
                               cudaStream_t st);
 cudaError_t launch_attend(const AttendParams &p, int bits, int n_seq, size_t smem, cudaStream_t st);
+// Fused decode attention (decode_fused.cu): one query head per KV head, d = 128, 1- or 2-bit key
+// codes; writes the chunk partials of the softmax.V merge.
+struct DecodeFusedArgs {
+  const uint32_t *krec;
+  const float *knorm, *krnorm;
+  const uint32_t *vrec;
+  const float *vnorm;
+  const float *qrot, *qsk;    // [n_seq][n_heads][128]
+  const float *cbk, *cbv;
+  float *partial;             // [n_seq][n_heads][n_chunks][130]
+  uint32_t *status;
+  int64_t n_tokens, cap_k, cap_v, chunk;
+  int n_seq, n_heads, n_chunks, kbits, vbits;
+  float scale;
+  size_t smem_limit;
+};
+bool decode_fused_supported(int d, int kbits, int vbits, int n_q_heads, int n_kv_heads, const void *krec,
+                            const void *vrec, size_t limit);
+cudaError_t launch_decode_fused(const DecodeFusedArgs &a, cudaStream_t st);
+cudaError_t launch_status_or(uint32_t *dst, const uint32_t *a, const uint32_t *b, cudaStream_t st);
 // d = 128 softmax.V streamed by bulk copies (attend_fast.cu); p.chunk from attend_fast_chunk.
 bool attend_fast_supported(int d, int bits, int q_per_cta, const void *records);
 int64_t attend_fast_chunk(int64_t n_tokens, int units);

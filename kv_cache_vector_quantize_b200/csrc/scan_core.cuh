@@ -1,0 +1,279 @@
+// Lookup-table logit machinery for d = 128 key records (1..3 code bits + the
+// QJL sign field), shared by the logit scan (logits_fast.cu) and the fused
+// decode attention (decode_fused.cu).
+//
+// Estimator (usedby.ai, "TurboQuant: Compresion de KV Cache a 3 bits y
+// aceleracion de inferencia en H100", "El Pitch"; winningdata.io, "TurboQuant:
+// Google comprime KV cache para 3 bits sem perder acuracia", "2. QJL
+// Residual"):
+//   l_t = n_t ( <Pi q, c[code_t]> + rho_t sqrt(pi/2)/d <S q, 2 sign_t - 1> ).
+//
+// Tables. The tables of query head q start at a 64 KB-aligned shared address
+// T0 + q * 64 KB, so a lookup address is formed by bit operations alone and the
+// per-query offset is the load's immediate. An index key is the codes of g
+// consecutive coordinates as they sit in the code stream (g = 8, 4, 2 for 1, 2,
+// 3 code bits: 8, 8 and 6 key bits); a d = 128 key has 16, 32 or 64 of them plus
+// 16 sign bytes. Each table entry is the partial dot product of the query with
+// that group.
+//
+// Byte keys (1 and 2 code bits): one table row per key value holds 64 words,
+// positions 0..31 for the index tables and 32..63 for the sign tables (a
+// 16-table set sits twice, at p and p + 16). At step s lane l reads position
+// p = s XOR l, so the 32 lanes hit 32 different banks whatever the key values.
+// The lane first permutes its record words by XOR with l/4 (a few selects,
+// shared by every query head of the group); the byte of key p is then picked
+// by one byte-permute whose selector depends only on l mod 4 and s mod 4, and
+// lands already shifted into the row field, merged with the table base's high
+// bytes. A lookup is one byte-permute, one shared load and one add.
+//
+// 6-bit keys (3 code bits): 64 tables of 64 entries in two groups of 32 (row
+// stride 32 words), and the 16 sign tables in their own rows (twice, rows of
+// 32 words). At step s lane l reads position (s + l) mod 32 after rotating its
+// record so that key (s + l) sits at static position s.
+#pragma once
+
+#include "common.cuh"
+
+namespace tq {
+namespace scan {
+
+constexpr int kFD = 128;                       // head dimension
+constexpr uint32_t kTabStride = 0x10000;       // shared bytes per query head's tables (64 KB)
+
+template <int BETA>
+struct FastKeys {
+  static constexpr int IW = BETA * kFD / 32;               // code-stream words
+  static constexpr int RW = IW + kFD / 32;                 // record words
+  static constexpr int NI = BETA == 1 ? 16 : BETA == 2 ? 32 : 64;   // index keys per record
+  static constexpr int G = BETA == 3 ? 2 : 8 / BETA;       // coordinates per index key
+};
+
+template <uint32_t OFF>
+__device__ __forceinline__ float lds_at(uint32_t addr) {
+  float v;
+  asm("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(OFF));
+  return v;
+}
+
+// Rotate an n-word cyclic bit stream right by `rb` bits (0 <= rb < 32 n):
+// out bit k = in bit (k + rb) mod 32n.
+template <int N>
+__device__ __forceinline__ void rotate_stream(uint32_t (&w)[N], int rb) {
+  const int wofs = rb >> 5, boff = rb & 31;
+#pragma unroll
+  for (int bit = 1; bit < N; bit <<= 1) {
+    uint32_t t[N];
+    const bool take = (wofs & bit) != 0;
+#pragma unroll
+    for (int j = 0; j < N; ++j) t[j] = take ? w[(j + bit) % N] : w[j];
+#pragma unroll
+    for (int j = 0; j < N; ++j) w[j] = t[j];
+  }
+  uint32_t t[N];
+#pragma unroll
+  for (int j = 0; j < N; ++j) t[j] = __funnelshift_r(w[j], w[(j + 1) % N], boff);
+#pragma unroll
+  for (int j = 0; j < N; ++j) w[j] = t[j];
+}
+
+// Permute N words by XOR of their index with c (N a power of two, c < N).
+template <int N>
+__device__ __forceinline__ void xor_permute(uint32_t (&w)[N], int c) {
+#pragma unroll
+  for (int bit = 1; bit < N; bit <<= 1) {
+    uint32_t t[N];
+    const bool take = (c & bit) != 0;
+#pragma unroll
+    for (int j = 0; j < N; ++j) t[j] = take ? w[j ^ bit] : w[j];
+#pragma unroll
+    for (int j = 0; j < N; ++j) w[j] = t[j];
+  }
+}
+
+// Key of KB bits at bit `pos` of a rotated stream, shifted to bit 7 (rows of 32
+// words) and merged with `bank` (table base | position offset).
+template <int KB, int N>
+__device__ __forceinline__ uint32_t key_addr7(const uint32_t (&r)[N], int pos, uint32_t bank) {
+  const int w = pos >> 5, b = pos & 31;
+  uint32_t v;
+  int at;
+  if (b + KB <= 32) {
+    v = r[w];
+    at = b;
+  } else {
+    v = __funnelshift_r(r[w], r[(w + 1) % N], b);
+    at = 0;
+  }
+  const uint32_t shifted = at >= 7 ? (v >> (at - 7)) : (v << (7 - at));
+  constexpr uint32_t mask = ((1u << KB) - 1u) << 7;
+  return (shifted & mask) | bank;
+}
+
+// One query head's logit for a byte-key record (1 or 2 code bits), tables at
+// T0 + QQ * 64 KB. xi[m] / xs[m] hold, per lane, the table-base bytes 2..3 and
+// the row positions (l ^ s) * 4 of steps s = 2m and 2m + 1 in bytes 0 and 1, so
+// one byte-permute yields the whole address T0 | key << 8 | position.
+template <int BETA, int QQ>
+__device__ __forceinline__ float scan_bytes(const uint32_t (&wi)[BETA * 4], const uint32_t (&wsg)[4],
+                                            const uint32_t (&sel)[4], const uint32_t (&xi)[BETA * 8],
+                                            const uint32_t (&xs)[8], float nrm, float rho) {
+  constexpr int NI = BETA == 1 ? 16 : 32;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+  for (int st = 0; st < NI; ++st) {
+    const float v = lds_at<QQ * kTabStride>(__byte_perm(wi[st >> 2], xi[st >> 1], sel[st & 3]));
+    if ((st & 3) == 0) a0 += v;
+    else if ((st & 3) == 1) a1 += v;
+    else if ((st & 3) == 2) a2 += v;
+    else a3 += v;
+  }
+#pragma unroll
+  for (int st = 0; st < 16; ++st) {
+    const float v = lds_at<QQ * kTabStride>(__byte_perm(wsg[st >> 2], xs[st >> 1], sel[st & 3]));
+    if (st & 1) b1 += v;
+    else b0 += v;
+  }
+  return nrm * fmaf(rho, b0 + b1, (a0 + a1) + (a2 + a3));
+}
+
+// One query head's logit for a 3-bit-code record (rotated halves lo/hi and sign stream rs).
+template <int QQ>
+__device__ __forceinline__ float scan_six(const uint32_t (&lo)[6], const uint32_t (&hi)[6], const uint32_t (&rs)[4],
+                                          const uint32_t (&bank)[32], float nrm, float rho) {
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+  for (int st = 0; st < 32; ++st) {
+    const float v = lds_at<QQ * kTabStride>(key_addr7<6>(lo, 6 * st, bank[st]));
+    if (st & 1) a1 += v;
+    else a0 += v;
+  }
+#pragma unroll
+  for (int st = 0; st < 32; ++st) {
+    const float v = lds_at<QQ * kTabStride + 8192>(key_addr7<6>(hi, 6 * st, bank[st]));
+    if (st & 1) a3 += v;
+    else a2 += v;
+  }
+#pragma unroll
+  for (int st = 0; st < 16; ++st) {
+    const float v = lds_at<QQ * kTabStride + 32768>(key_addr7<8>(rs, 8 * st, bank[st]));
+    if (st & 1) b1 += v;
+    else b0 += v;
+  }
+  return nrm * fmaf(rho, b0 + b1, (a0 + a1) + (a2 + a3));
+}
+
+// The logits of one key record for QMAX query heads (tables at T0 + qq * 64 KB;
+// heads past nq are left at 0). w: the record words of this lane's key.
+template <int BETA, int QMAX>
+__device__ __forceinline__ void key_logits(const uint32_t (&w)[FastKeys<BETA>::RW], int lane, uint32_t T0, int nq,
+                                           float nrm, float rho, float (&out)[QMAX]) {
+  constexpr int IW = FastKeys<BETA>::IW;
+#pragma unroll
+  for (int qq = 0; qq < QMAX; ++qq) out[qq] = 0.f;
+  if constexpr (BETA != 3) {
+    // byte-permute selectors for step s (j = s mod 4): result byte 0 = position byte
+    // (s mod 2) of the x register, byte 1 = key byte (j ^ (l & 3)) of the record
+    // word, bytes 2..3 = table-base bytes 2..3 of the x register
+    uint32_t sel[4];
+    const uint32_t sel0 = 0x7604u | ((uint32_t)(lane & 3) << 4);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sel[j] = sel0 ^ ((uint32_t)(j & 1) | ((uint32_t)j << 4));
+    const uint32_t xi0 = (T0 & 0xFFFF0000u) | ((uint32_t)lane << 2) | ((uint32_t)(lane ^ 1) << 10);
+    const uint32_t xs0 = xi0 | 0x8080u;
+    uint32_t xi[BETA * 8], xs[8];
+#pragma unroll
+    for (int m = 0; m < BETA * 8; ++m) xi[m] = xi0 ^ ((uint32_t)m * 0x808u);
+#pragma unroll
+    for (int m = 0; m < 8; ++m) xs[m] = xs0 ^ ((uint32_t)m * 0x808u);
+    uint32_t wi[IW], wsg[4];
+#pragma unroll
+    for (int j = 0; j < IW; ++j) wi[j] = w[j];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) wsg[j] = w[IW + j];
+    xor_permute<IW>(wi, (lane >> 2) & (IW - 1));
+    xor_permute<4>(wsg, (lane >> 2) & 3);
+    out[0] = scan_bytes<BETA, 0>(wi, wsg, sel, xi, xs, nrm, rho);
+    if constexpr (QMAX > 1)
+      if (nq > 1) out[1] = scan_bytes<BETA, 1>(wi, wsg, sel, xi, xs, nrm, rho);
+  } else {
+    uint32_t bank[32];   // T0 | position offset ((s + l) mod 32, times 4)
+#pragma unroll
+    for (int s2 = 0; s2 < 32; ++s2) bank[s2] = T0 | (uint32_t)(((s2 + lane) & 31) << 2);
+    uint32_t lo[6], hi[6], rs[4];
+#pragma unroll
+    for (int j = 0; j < 6; ++j) { lo[j] = w[j]; hi[j] = w[6 + j]; }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) rs[j] = w[12 + j];
+    rotate_stream<6>(lo, 6 * lane);
+    rotate_stream<6>(hi, 6 * lane);
+    rotate_stream<4>(rs, 8 * (lane & 15));
+    out[0] = scan_six<0>(lo, hi, rs, bank, nrm, rho);
+    if constexpr (QMAX > 1)
+      if (nq > 1) out[1] = scan_six<1>(lo, hi, rs, bank, nrm, rho);
+  }
+}
+
+// The lookup tables of one query head at tq_ (its 64 KB block), from qr = Pi q
+// and qs = S q, with kappa = sqrt(pi/2)/d folded into the sign tables. Called
+// by NTHR threads (tid < NTHR), a multiple of 64. Each thread keeps one table
+// position (and so its few query values) in registers and walks the key values
+// with a stride of NTHR / width, so a warp shares one key: codebook reads
+// broadcast and stores hit 32 banks.
+template <int BETA, int NTHR>
+__device__ __forceinline__ void build_tables(const float *qr, const float *qs, float *tq_, const float *cbs, int tid,
+                                             float kappa) {
+  using K = FastKeys<BETA>;
+  static_assert(NTHR % 64 == 0, "table builds walk key values with a stride of NTHR / 64");
+  if constexpr (BETA != 3) {
+    // 256 rows of 64 words: [0, 32) index positions, [32, 64) sign positions
+    const int pos = tid & 63;
+    if (pos < 32) {
+      const int t = pos & (K::NI - 1);
+      float qc[K::G];
+#pragma unroll
+      for (int c = 0; c < K::G; ++c) qc[c] = qr[t * K::G + c];
+      for (int key = tid >> 6; key < 256; key += NTHR / 64) {
+        float v = 0.f;
+#pragma unroll
+        for (int c = 0; c < K::G; ++c) v = fmaf(qc[c], cbs[(key >> (BETA * c)) & ((1 << BETA) - 1)], v);
+        tq_[key * 64 + pos] = v;
+      }
+    } else {
+      const int t = pos & 15;
+      float sv[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) sv[c] = kappa * qs[8 * t + c];
+      for (int key = tid >> 6; key < 256; key += NTHR / 64) {
+        float v = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) v += ((key >> c) & 1) ? sv[c] : -sv[c];
+        tq_[key * 64 + pos] = v;
+      }
+    }
+  } else {
+    // index: 2 groups x 64 rows x 32 words at +0; sign: 256 rows x 32 words at +32 KB
+    {
+      const int t = tid & 63;
+      const float q0 = qr[2 * t], q1 = qr[2 * t + 1];
+      float *row = tq_ + (t >> 5) * 64 * 32 + (t & 31);
+      for (int key = tid >> 6; key < 64; key += NTHR / 64)
+        row[key * 32] = fmaf(q1, cbs[(key >> 3) & 7], q0 * cbs[key & 7]);
+    }
+    {
+      const int pos = tid & 31, t = pos & 15;
+      float sv[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) sv[c] = kappa * qs[8 * t + c];
+      float *ts = tq_ + 8192;
+      for (int key = tid >> 5; key < 256; key += NTHR / 32) {
+        float v = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) v += ((key >> c) & 1) ? sv[c] : -sv[c];
+        ts[key * 32 + pos] = v;
+      }
+    }
+  }
+}
+
+}  // namespace scan
+}  // namespace tq

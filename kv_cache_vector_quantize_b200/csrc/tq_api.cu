@@ -423,6 +423,138 @@ tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale, int32
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_attend_v (merge)");
 }
 
+// Workspace of tq_decode_attend. Fused path: status word | Pi q | S q | chunk partials.
+// Otherwise: status word | logits | tq_logits workspace | tq_attend_v workspace.
+namespace {
+
+size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+struct DecodeWs {
+  bool fused;
+  size_t qrot, qsk, partial;                  // fused
+  size_t logits, ws_l, ws_l_bytes, ws_a, ws_a_bytes;   // two calls
+  size_t total;
+};
+
+bool same_heads(const tq_cache *k, const tq_cache *v) {
+  return k->d == v->d && k->n_seq == v->n_seq && k->n_kv_heads == v->n_kv_heads;
+}
+
+DecodeWs decode_ws(const tq_cache *k, const tq_cache *v, int n_q_heads, int64_t n_tokens) {
+  DecodeWs w{};
+  w.fused = decode_fused_supported(k->d, k->idx_bits, v->idx_bits, n_q_heads, k->n_kv_heads, k->records,
+                                   v->records, device_smem_optin() - 1024);
+  const size_t rows = (size_t)k->n_seq * n_q_heads;
+  if (w.fused) {
+    const int64_t n_chunks = (n_tokens + kAttendChunk - 1) / kAttendChunk;   // at least as many as the split uses
+    w.qrot = kWsHeader;
+    w.qsk = w.qrot + align256(sizeof(float) * rows * k->d);
+    w.partial = w.qsk + align256(sizeof(float) * rows * k->d);
+    w.total = w.partial + sizeof(float) * rows * (size_t)n_chunks * (k->d + 2);
+  } else {
+    w.logits = kWsHeader;
+    w.ws_l = w.logits + align256(sizeof(float) * rows * (size_t)n_tokens);
+    w.ws_l_bytes = align256(tq_logits_workspace_size(k, n_q_heads));
+    w.ws_a = w.ws_l + w.ws_l_bytes;
+    w.ws_a_bytes = tq_attend_workspace_size(v, n_q_heads, n_tokens);
+    w.total = w.ws_a + w.ws_a_bytes;
+  }
+  return w;
+}
+
+}  // namespace
+
+size_t tq_decode_workspace_size(const tq_cache *k, const tq_cache *v, int32_t n_q_heads, int64_t n_tokens) {
+  if (!k || !v || k->n_seq <= 0 || k->d <= 0 || k->n_kv_heads <= 0 || n_q_heads <= 0 || n_tokens < 0 ||
+      !same_heads(k, v))
+    return 0;
+  return decode_ws(k, v, n_q_heads, n_tokens).total;
+}
+
+tq_status tq_decode_attend(const tq_cache *k, const tq_cache *v, const float *q, int32_t n_q_heads,
+                           int64_t n_tokens, float scale, const float *Pi, const float *S,
+                           const float *codebook_k, const float *codebook_v, float *out, void *workspace,
+                           size_t workspace_bytes, tq_stream stream) {
+  g_err[0] = 0;
+  tq_status s = check_cache(k, "tq_decode_attend (keys)");
+  if (s != TQ_OK) return s;
+  s = check_cache(v, "tq_decode_attend (values)");
+  if (s != TQ_OK) return s;
+  if (!k->qjl || v->qjl) return fail(TQ_ERR_INVALID, "tq_decode_attend: k must be a key cache (qjl 1), v a value cache (qjl 0)");
+  if (!same_heads(k, v))
+    return fail(TQ_ERR_INVALID, "tq_decode_attend: key and value caches differ in d, n_seq or n_kv_heads");
+  if (n_q_heads <= 0 || n_q_heads % k->n_kv_heads != 0)
+    return fail(TQ_ERR_INVALID, "tq_decode_attend: n_q_heads=%d is not a positive multiple of n_kv_heads=%d",
+                n_q_heads, k->n_kv_heads);
+  if (n_tokens < 0 || n_tokens > k->capacity || n_tokens > v->capacity)
+    return fail(TQ_ERR_CAPACITY, "tq_decode_attend: n_tokens=%lld outside [0, capacity]", (long long)n_tokens);
+  if (!q || !Pi || !S || !codebook_k || !codebook_v || !out)
+    return fail(TQ_ERR_INVALID, "tq_decode_attend: NULL tensor argument");
+  if (!(scale == scale) || scale == INFINITY || scale == -INFINITY)
+    return fail(TQ_ERR_INVALID, "tq_decode_attend: scale is not finite");
+  const DecodeWs w = decode_ws(k, v, n_q_heads, n_tokens);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.total)
+    return fail(TQ_ERR_WORKSPACE, "tq_decode_attend: workspace needs %zu bytes, 256-byte aligned (got %zu)", w.total,
+                workspace_bytes);
+  if (injected(&s)) return s;
+  if ((n_tokens + kAttendChunk - 1) / kAttendChunk > 50000)
+    return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attend: n_tokens=%lld exceeds the merge limit of %lld tokens",
+                (long long)n_tokens, 50000LL * kAttendChunk);
+  char *ws = static_cast<char *>(workspace);
+  uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+  const size_t out_bytes = sizeof(float) * (size_t)k->n_seq * n_q_heads * k->d;
+  cudaError_t e = cudaSuccess;
+  if (n_tokens == 0) {
+    e = cudaMemsetAsync(out, 0, out_bytes, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, sizeof(uint32_t), (cudaStream_t)stream);
+    return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_decode_attend (empty)");
+  }
+  if (!w.fused) {
+    // other head groupings and code widths: the two calls, their status words merged into this one
+    s = tq_logits(k, q, n_q_heads, n_tokens, Pi, S, codebook_k, reinterpret_cast<float *>(ws + w.logits), ws + w.ws_l,
+                  w.ws_l_bytes, stream);
+    if (s != TQ_OK) return s;
+    s = tq_attend_v(v, reinterpret_cast<const float *>(ws + w.logits), scale, n_q_heads, n_tokens, Pi, codebook_v, out,
+                    ws + w.ws_a, w.ws_a_bytes, stream);
+    if (s != TQ_OK) return s;
+    e = launch_status_or(status, reinterpret_cast<const uint32_t *>(ws + w.ws_l),
+                         reinterpret_cast<const uint32_t *>(ws + w.ws_a), (cudaStream_t)stream);
+    return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_decode_attend (status)");
+  }
+  float *qrot = reinterpret_cast<float *>(ws + w.qrot), *qsk = reinterpret_cast<float *>(ws + w.qsk);
+  float *partial = reinterpret_cast<float *>(ws + w.partial);
+  // the projection clears the status word and lets the fused grid start streaming tiles
+  e = launch_qprep(q, k->n_seq * n_q_heads, k->d, Pi, S, qrot, qsk, status, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_decode_attend (query projection)");
+  DecodeFusedArgs a{};
+  a.krec = k->records;
+  a.knorm = k->norm;
+  a.krnorm = k->rnorm;
+  a.vrec = v->records;
+  a.vnorm = v->norm;
+  a.qrot = qrot;
+  a.qsk = qsk;
+  a.cbk = codebook_k;
+  a.cbv = codebook_v;
+  a.partial = partial;
+  a.status = status;
+  a.n_tokens = n_tokens;
+  a.cap_k = k->capacity;
+  a.cap_v = v->capacity;
+  a.chunk = attend_fast_chunk(n_tokens, k->n_seq * k->n_kv_heads);
+  a.n_seq = k->n_seq;
+  a.n_heads = n_q_heads;
+  a.n_chunks = (int)((n_tokens + a.chunk - 1) / a.chunk);
+  a.kbits = k->idx_bits;
+  a.vbits = v->idx_bits;
+  a.scale = scale;
+  a.smem_limit = device_smem_optin() - 1024;
+  e = launch_decode_fused(a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_decode_attend (fused scan)");
+  e = launch_combine(partial, k->n_seq * n_q_heads, a.n_chunks, k->d, Pi, out, (cudaStream_t)stream);
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_decode_attend (merge)");
+}
+
 tq_status tq_workspace_status(void *workspace, tq_stream stream) {
   g_err[0] = 0;
   if (!workspace || !aligned(workspace, 256)) return fail(TQ_ERR_WORKSPACE, "tq_workspace_status: bad workspace");

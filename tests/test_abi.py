@@ -123,6 +123,33 @@ def test_attend_argument_checks():
     assert call(_desc(qjl=0)) == tqb.TQ_ERR_CUDA                   # passes the checks -> injected
 
 
+def test_decode_attend_argument_checks():
+    def call(kd, vd, hq=2, n=8, scale=0.1, ws_bytes=1 << 24, q=FAKE):
+        return lib.tq_decode_attend(ctypes.byref(kd), ctypes.byref(vd), q, hq, n, ctypes.c_float(scale), FAKE, FAKE,
+                                    FAKE, FAKE, FAKE, FAKE, ws_bytes, None)
+    k, v = _desc(qjl=1), _desc(qjl=0, records=FAKE + (1 << 20), norm=FAKE + (2 << 20))
+    assert call(v, v) == tqb.TQ_ERR_INVALID                        # keys must carry the sign field
+    assert call(k, k) == tqb.TQ_ERR_INVALID                        # values must not
+    assert call(k, _desc(qjl=0, heads=4)) == tqb.TQ_ERR_INVALID    # different KV head counts
+    assert call(k, _desc(qjl=0, d=64)) == tqb.TQ_ERR_INVALID       # different head dimensions
+    assert call(k, v, hq=3) == tqb.TQ_ERR_INVALID
+    assert call(k, _desc(qjl=0, cap=16), n=17) == tqb.TQ_ERR_CAPACITY
+    assert call(k, v, scale=float("inf")) == tqb.TQ_ERR_INVALID
+    assert call(k, v, q=None) == tqb.TQ_ERR_INVALID
+    assert call(k, v, ws_bytes=64) == tqb.TQ_ERR_WORKSPACE
+    assert call(k, v) == tqb.TQ_ERR_CUDA                           # passes the checks -> injected
+    # one query head per KV head, d = 128, 2-bit key codes: status | Pi q | S q | partials of 512-token chunks
+    rows, nt = 2, 1000
+    fused = 256 + 2 * rows * 128 * 4 + rows * 2 * 130 * 4
+    assert lib.tq_decode_workspace_size(ctypes.byref(k), ctypes.byref(v), 2, nt) == fused
+    # grouped queries: status | logits | the tq_logits and tq_attend_v workspaces
+    lg = (4 * nt * 4 + 255) // 256 * 256
+    ws_l = (lib.tq_logits_workspace_size(ctypes.byref(k), 4) + 255) // 256 * 256
+    ws_a = lib.tq_attend_workspace_size(ctypes.byref(v), 4, nt)
+    assert lib.tq_decode_workspace_size(ctypes.byref(k), ctypes.byref(v), 4, nt) == 256 + lg + ws_l + ws_a
+    assert lib.tq_decode_workspace_size(ctypes.byref(k), ctypes.byref(_desc(qjl=0, heads=4)), 2, nt) == 0
+
+
 def test_fault_injection_counts_down():
     tqb.tq_debug_inject(tqb.TQ_ERR_DEVICE, 2)
     assert _q(_desc(qjl=0)) == tqb.TQ_ERR_DEVICE

@@ -262,6 +262,56 @@ def test_logits_unaligned_query_and_matrices(kb, G):
                              kn[0, h], kr[0, h], d, kb)
 
 
+DECODE_SHAPES = [
+    # k index bits, v bits, n_seq, kv heads, group, tokens: one query head per KV head takes the fused
+    # pass (1- or 2-bit key codes), every other shape the two calls inside the same entry point
+    (2, 3, 2, 3, 1, 1537),
+    (1, 2, 1, 2, 1, 777),
+    (2, 4, 1, 1, 1, 4096),
+    (2, 1, 3, 1, 1, 130),
+    (3, 3, 1, 2, 1, 901),
+    (2, 3, 1, 2, 4, 1100),
+]
+
+
+@pytest.mark.parametrize("shape", DECODE_SHAPES, ids=lambda s: f"kb{s[0]}-vb{s[1]}-B{s[2]}-H{s[3]}-G{s[4]}-T{s[5]}")
+def test_decode_attend_parity(shape):
+    # the one-call decode step equals tq_logits followed by tq_attend_v bit for bit (same tables,
+    # chunks and accumulation order), and that output matches the oracle's softmax.V of those logits
+    kb, vb, B, H, G, T = shape
+    d = 128
+    k = syn.gaussian((B, H, T, d), 61).to(torch.bfloat16)
+    v = syn.lognormal_sphere((B, H, T, d), 62, dtype=torch.bfloat16)
+    q = syn.gaussian((B, H * G, d), 63)
+    Pi, S, ck, cv, g = _setup(d, kb, vb)
+    kc, vc, lg, out2, sc = _run_path(k, v, q, d, kb, vb, g, capacity=T + 3)
+    ws = torch.empty(max(256, tqb.tq_decode_workspace_size(kc, vc, H * G, T)), dtype=torch.uint8, device="cuda")
+    ws.fill_(0xFF)   # the call must clear the status word itself
+    out1 = tqb.tq_decode_attend(kc, vc, q.cuda(), T, sc, g["Pi"], g["S"], g["ck"], g["cv"], workspace=ws)
+    torch.cuda.synchronize()
+    tqb.tq_workspace_status(ws)
+    assert torch.equal(out1, out2)
+    vrec = par.as_u32(vc.records.cpu().numpy())
+    vn = vc.norm.cpu().numpy()
+    lg_np, o1 = lg.cpu().numpy().astype(np.float64), out1.cpu().numpy()
+    for s_ in range(B):
+        for h in range(H):
+            par.check_attend(o1[s_, h * G:(h + 1) * G], lg_np[s_, h * G:(h + 1) * G], sc, Pi, cv, vrec[s_, h, :T],
+                             vn[s_, h, :T], d, vb)
+
+
+def test_decode_attend_empty():
+    d = 128
+    _, _, _, _, g = _setup(d, 2, 3)
+    kc = tqb.PackedCache.empty(d, 2, True, 1, 2, 16)
+    vc = tqb.PackedCache.empty(d, 3, False, 1, 2, 16)
+    out = torch.full((1, 2, d), 7.0, device="cuda")
+    tqb.tq_decode_attend(kc, vc, torch.randn(1, 2, d, device="cuda"), 0, 0.1, g["Pi"], g["S"], g["ck"], g["cv"],
+                         out=out)
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)
+
+
 # ---------------------------------------------------------------------------
 # full-size workloads, sampled
 # ---------------------------------------------------------------------------
