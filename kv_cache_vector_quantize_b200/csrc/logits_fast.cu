@@ -211,8 +211,10 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
     const int n = (int)min((int64_t)kFTile, p.n_tokens - t0);
     const bool valid = k < n;
     const unsigned char *st = smem + (slot(s) - dyn0);
+    // this lane's record, read whether or not the key exists: slots past n hold stale words whose
+    // logits are never stored, so the load needs no branch
     uint32_t w[RW];
-    if (valid) {
+    {
       const uint4 *src = reinterpret_cast<const uint4 *>(st + (size_t)k * RW * 4);
 #pragma unroll
       for (int j = 0; j < RW / 4; ++j) {
@@ -222,19 +224,14 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
         w[4 * j + 2] = v.z;
         w[4 * j + 3] = v.w;
       }
-    } else {
-#pragma unroll
-      for (int j = 0; j < RW; ++j) w[j] = 0u;
     }
-    float nrm = 0.f, rho = 0.f;
-    if (valid) {
-      if (unit_nc && (n & 3) == 0) {   // the producer's condition (norms_by_copy) for this tile
-        nrm = reinterpret_cast<const float *>(st + kFTile * RW * 4)[k];
-        rho = reinterpret_cast<const float *>(st + kFTile * RW * 4 + kFTile * 4)[k];
-      } else {
-        nrm = __ldg(nrm_p + t0 + k);
-        rho = __ldg(rho_p + t0 + k);
-      }
+    float nrm, rho;
+    if (unit_nc && (n & 3) == 0) {   // the producer's condition (norms_by_copy) for this tile
+      nrm = reinterpret_cast<const float *>(st + kFTile * RW * 4)[k];
+      rho = reinterpret_cast<const float *>(st + kFTile * RW * 4 + kFTile * 4)[k];
+    } else {
+      nrm = valid ? __ldg(nrm_p + t0 + k) : 0.f;
+      rho = valid ? __ldg(rho_p + t0 + k) : 0.f;
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_bar(s));   // this warp is done with the stage

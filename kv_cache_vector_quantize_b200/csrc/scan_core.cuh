@@ -118,21 +118,18 @@ __device__ __forceinline__ float scan_bytes(const uint32_t (&wi)[BETA * 4], cons
                                             const uint32_t (&sel)[4], const uint32_t (&xi)[BETA * 8],
                                             const uint32_t (&xs)[8], float nrm, float rho) {
   constexpr int NI = BETA == 1 ? 16 : 32;
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, b0 = 0.f, b1 = 0.f;
+  float a[4], b[2];   // each chain starts at its first lookup (no zeroing, no add to zero)
 #pragma unroll
   for (int st = 0; st < NI; ++st) {
     const float v = lds_at<QQ * kTabStride>(__byte_perm(wi[st >> 2], xi[st >> 1], sel[st & 3]));
-    if ((st & 3) == 0) a0 += v;
-    else if ((st & 3) == 1) a1 += v;
-    else if ((st & 3) == 2) a2 += v;
-    else a3 += v;
+    a[st & 3] = st < 4 ? v : a[st & 3] + v;
   }
 #pragma unroll
   for (int st = 0; st < 16; ++st) {
     const float v = lds_at<QQ * kTabStride>(__byte_perm(wsg[st >> 2], xs[st >> 1], sel[st & 3]));
-    if (st & 1) b1 += v;
-    else b0 += v;
+    b[st & 1] = st < 2 ? v : b[st & 1] + v;
   }
+  const float a0 = a[0], a1 = a[1], a2 = a[2], a3 = a[3], b0 = b[0], b1 = b[1];
   return nrm * fmaf(rho, b0 + b1, (a0 + a1) + (a2 + a3));
 }
 
@@ -140,25 +137,23 @@ __device__ __forceinline__ float scan_bytes(const uint32_t (&wi)[BETA * 4], cons
 template <int QQ>
 __device__ __forceinline__ float scan_six(const uint32_t (&lo)[6], const uint32_t (&hi)[6], const uint32_t (&rs)[4],
                                           const uint32_t (&bank)[32], float nrm, float rho) {
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, b0 = 0.f, b1 = 0.f;
+  float a[4], b[2];   // each chain starts at its first lookup (no zeroing, no add to zero)
 #pragma unroll
   for (int st = 0; st < 32; ++st) {
     const float v = lds_at<QQ * kTabStride>(key_addr7<6>(lo, 6 * st, bank[st]));
-    if (st & 1) a1 += v;
-    else a0 += v;
+    a[st & 1] = st < 2 ? v : a[st & 1] + v;
   }
 #pragma unroll
   for (int st = 0; st < 32; ++st) {
     const float v = lds_at<QQ * kTabStride + 8192>(key_addr7<6>(hi, 6 * st, bank[st]));
-    if (st & 1) a3 += v;
-    else a2 += v;
+    a[2 + (st & 1)] = st < 2 ? v : a[2 + (st & 1)] + v;
   }
 #pragma unroll
   for (int st = 0; st < 16; ++st) {
     const float v = lds_at<QQ * kTabStride + 32768>(key_addr7<8>(rs, 8 * st, bank[st]));
-    if (st & 1) b1 += v;
-    else b0 += v;
+    b[st & 1] = st < 2 ? v : b[st & 1] + v;
   }
+  const float a0 = a[0], a1 = a[1], a2 = a[2], a3 = a[3], b0 = b[0], b1 = b[1];
   return nrm * fmaf(rho, b0 + b1, (a0 + a1) + (a2 + a3));
 }
 
