@@ -183,6 +183,25 @@ enum : uint32_t { kDevTimeout = 1u << 1 };   // an mbarrier wait gave up (status
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Launch a grid as a programmatic dependent of the work before it in the stream,
+// so that its launch is processed while that work finishes. The kernel must
+// call pdl_wait() before it reads or writes global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                         Args &&...args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
 constexpr uint32_t kSpinLimit = 1u << 24;    // try_wait attempts before a wait gives up
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

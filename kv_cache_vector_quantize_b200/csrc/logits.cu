@@ -34,6 +34,7 @@ __global__ void __launch_bounds__(128) qprep_kernel(const float *__restrict__ q,
                                                     const float *__restrict__ S, float *__restrict__ qrot,
                                                     float *__restrict__ qsk, uint32_t *status) {
   const int row = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();                // launched as a dependent of the previous work: it must be finished first
   pdl_launch_dependents();   // the scan may start staging keys now; it waits for this grid before reading
   if (row == 0 && chunk == 0 && tid == 0) *status = 0u;   // this call's kernels report into a clean word
   const float *qr = q + (size_t)row * d;
@@ -168,8 +169,7 @@ size_t logits_smem_per_query(int d, int bits) {
 cudaError_t launch_qprep(const float *q, int rows, int d, const float *Pi, const float *S, float *qrot, float *qsk,
                          uint32_t *status, cudaStream_t st) {
   dim3 grid((2 * d + kQpOut - 1) / kQpOut, rows);
-  qprep_kernel<<<grid, 128, 0, st>>>(q, d, Pi, S, qrot, qsk, status);
-  return cudaGetLastError();
+  return launch_after(qprep_kernel, grid, dim3(128), 0, st, q, d, Pi, S, qrot, qsk, status);
 }
 
 cudaError_t launch_logits(const LogitsParams &p, int bits, int n_seq, int n_chunks, size_t smem, cudaStream_t st) {

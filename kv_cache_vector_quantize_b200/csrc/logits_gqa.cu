@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(256) gqa_tables_kernel(GqaParams g) {
   const int qb = unit % g.qblocks, sk = unit / g.qblocks;
   const int seq = sk / g.n_kv_heads, kvh = sk - seq * g.n_kv_heads;
   const int h0 = kvh * g.group + qb * QH;
+  pdl_wait();   // launched as a dependent of the previous work: it must be finished first
   if (unit == 0 && half == 0 && part == 0 && tid == 0) *g.status = 0u;   // this call reports into a clean word
   pdl_launch_dependents();   // the scan may start streaming keys; it waits for this grid before its tables
   // coordinates of byte positions [8 part, 8 part + 8): index bytes of 1-bit codes and sign bytes
@@ -449,8 +450,7 @@ cudaError_t launch_gqa_t(const LogitsParams &p, const GqaParams &g, int n_seq, s
   using K = GKeys<BETA>;
   const int units = n_seq * p.n_kv_heads * p.qblocks;
   // tables: one small grid, then the scan as its programmatic dependent
-  gqa_tables_kernel<BETA, QH><<<dim3(units, 2, 4), 256, 0, st>>>(g);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_after(gqa_tables_kernel<BETA, QH>, dim3(units, 2, 4), dim3(256), 0, st, g);
   if (e != cudaSuccess) return e;
   GScan gs{};
   gs.p = p;

@@ -507,6 +507,7 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
   constexpr int NL = 1 << BITS;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_wait();   // launched as a dependent of the previous work: it must be finished first
   const uint32_t sbase = smem_u32(smem);
   const Bars<QJL> bar{sbase + L::kBar};
   float *cb = reinterpret_cast<float *>(smem + L::kCb);
@@ -826,8 +827,7 @@ cudaError_t launch_tc(const QuantParams &p, cudaStream_t st) {
   const int64_t tiles = (p.rows + kTT - 1) / kTT;
   const int64_t slots = (int64_t)device_sm_count();
   const int grid = (int)(tiles < slots ? tiles : slots);
-  kern<<<grid, Ws<QJL>::kThreads, smem, st>>>(p, xmap);
-  return cudaGetLastError();
+  return launch_after(kern, dim3(grid), dim3(Ws<QJL>::kThreads), smem, st, p, xmap);
 }
 
 template <bool F16>
