@@ -210,41 +210,80 @@ __device__ __forceinline__ void key_logits(const uint32_t (&w)[FastKeys<BETA>::R
 
 // The lookup tables of one query head at tq_ (its 64 KB block), from qr = Pi q
 // and qs = S q, with kappa = sqrt(pi/2)/d folded into the sign tables. Called
-// by NTHR threads (tid < NTHR), a multiple of 64. Each thread keeps one table
-// position (and so its few query values) in registers and walks the key values
-// with a stride of NTHR / width, so a warp shares one key: codebook reads
-// broadcast and stores hit 32 banks.
+// by NTHR threads (tid < NTHR).
+//
+// Byte keys (1 and 2 code bits; NTHR = 512, 16 warps): an entry is the sum of a
+// part over its low nibble and a part over its high nibble. Lane l of warp w
+// owns table column l (warps 0-7: index positions) or 32 + l (warps 8-15: sign
+// positions) and the 32 keys whose high nibble is 2 (w mod 8) or 2 (w mod 8) + 1:
+// it forms the 16 low-nibble parts and its 2 high-nibble parts in registers,
+// and then each entry is one add and one store, a warp storing 32 consecutive
+// words of one row.
+//
+// 6-bit keys (3 code bits): each thread keeps one table position (and so its
+// few query values) in registers and walks the key values with a stride of
+// NTHR / width, so a warp shares one key: codebook reads broadcast and stores
+// hit 32 banks.
 template <int BETA, int NTHR>
 __device__ __forceinline__ void build_tables(const float *qr, const float *qs, float *tq_, const float *cbs, int tid,
                                              float kappa) {
   using K = FastKeys<BETA>;
-  static_assert(NTHR % 64 == 0, "table builds walk key values with a stride of NTHR / 64");
   if constexpr (BETA != 3) {
-    // 256 rows of 64 words: [0, 32) index positions, [32, 64) sign positions
-    const int pos = tid & 63;
-    if (pos < 32) {
-      const int t = pos & (K::NI - 1);
-      float qc[K::G];
+    static_assert(NTHR == 512, "byte-key tables: 16 warps, 2 high nibbles each");
+    constexpr int L = 1 << BETA, GH = K::G / 2;   // codes per nibble
+    const int warp = tid >> 5, lane = tid & 31, hn0 = 2 * (warp & 7);
+    const bool sign = warp >= 8;
+    float lo[16], hi[2];
+    if (!sign) {
+      // index position t: the G codes of one byte of the code stream
+      const int t = lane & (K::NI - 1);
+      float qc[K::G], cv[L];
 #pragma unroll
       for (int c = 0; c < K::G; ++c) qc[c] = qr[t * K::G + c];
-      for (int key = tid >> 6; key < 256; key += NTHR / 64) {
-        float v = 0.f;
 #pragma unroll
-        for (int c = 0; c < K::G; ++c) v = fmaf(qc[c], cbs[(key >> (BETA * c)) & ((1 << BETA) - 1)], v);
-        tq_[key * 64 + pos] = v;
+      for (int c = 0; c < L; ++c) cv[c] = cbs[c];
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {
+        float v = qc[0] * cv[n & (L - 1)];
+#pragma unroll
+        for (int c = 1; c < GH; ++c) v = fmaf(qc[c], cv[(n >> (BETA * c)) & (L - 1)], v);
+        lo[n] = v;
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int n = hn0 + j;
+        float v = qc[GH] * cv[n & (L - 1)];
+#pragma unroll
+        for (int c = 1; c < GH; ++c) v = fmaf(qc[GH + c], cv[(n >> (BETA * c)) & (L - 1)], v);
+        hi[j] = v;
       }
     } else {
-      const int t = pos & 15;
+      // sign position t: 8 sign bits, +-kappa (S q)_i
+      const int t = lane & 15;
       float sv[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) sv[c] = kappa * qs[8 * t + c];
-      for (int key = tid >> 6; key < 256; key += NTHR / 64) {
-        float v = 0.f;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) v += ((key >> c) & 1) ? sv[c] : -sv[c];
-        tq_[key * 64 + pos] = v;
+      for (int n = 0; n < 16; ++n) {
+        float v = (n & 1) ? sv[0] : -sv[0];
+#pragma unroll
+        for (int c = 1; c < 4; ++c) v += ((n >> c) & 1) ? sv[c] : -sv[c];
+        lo[n] = v;
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int n = hn0 + j;
+        float v = (n & 1) ? sv[4] : -sv[4];
+#pragma unroll
+        for (int c = 1; c < 4; ++c) v += ((n >> c) & 1) ? sv[4 + c] : -sv[4 + c];
+        hi[j] = v;
       }
     }
+    float *col = tq_ + (sign ? 32 : 0) + lane;   // 256 rows of 64 words: [0, 32) index, [32, 64) sign positions
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int n = 0; n < 16; ++n) col[((hn0 + j) * 16 + n) * 64] = lo[n] + hi[j];
   } else {
     // index: 2 groups x 64 rows x 32 words at +0; sign: 256 rows x 32 words at +32 KB
     {
