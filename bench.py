@@ -51,10 +51,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0
 NCU_TRAFFIC = {
     ("quantize_k", "llama"): 67_326_976 + 2_125_824,   # quantize_tc_kernel<1, 2, 0>
     ("quantize_v", "llama"): 67_240_704 + 2_118_144,   # quantize_tc_kernel<0, 3, 0>
-    ("logits", "sweep-b3"): 2 * (234_978_304 + 16_730_368),   # logits_fast_kernel<2, 1>, 4-sequence capture x 2
+    ("logits", "sweep-b3"): 2 * (234_967_296 + 16_118_528),   # logits_fast_kernel<2, 1>, 4-sequence capture x 2
     ("attend_v", "sweep-b3"): 2 * (234_927_616 + 3_965_184),  # attend_fast_kernel<3, 1>, 4-sequence capture x 2
     ("logits", "llama"): 15_756_288 + 0,               # logits_gqa_kernel<2, 4> (the scan; tables read from L2)
     ("attend_v", "llama"): 17_871_872 + 0,             # attend_fast_kernel<3, 4> (records, norms and logits)
+    ("decode_attend", "sweep-b3"): 2 * (453_061_376 + 5_822_720),   # decode_fused_kernel<2, 3>, 4-sequence capture x 2
 }
 
 
@@ -379,21 +380,22 @@ def run_tq(args, rank, world, local_rank):
         "packed_bytes": {"keys": kb, "values": vb},
         "roofline": roofline, "roofline_logit_scan": roof_scan, "roofline_quantize_v": roof_qv,
         "roofline_attend_v": roof_att,
-        "roofline_decode_attend": decode_roof(dec_ms, mean["logits"] + mean["attend_v"], kb + vb, w, hbm, src_txt),
+        "roofline_decode_attend": decode_roof(dec_ms, mean["logits"] + mean["attend_v"], kb + vb, w, hbm, src_txt,
+                                              NCU_TRAFFIC.get(("decode_attend", args.workload))),
         "gpu_launches": kernels_per_step * args.steps,
         "clocks": clk, "e2e": e2e,
     }
     return result, w
 
 
-def decode_roof(ms, two_call_ms, nbytes, w, hbm, src_txt):
+def decode_roof(ms, two_call_ms, nbytes, w, hbm, src_txt, traffic=None):
     """The one-call decode step against HBM: packed key + value bytes per call / its time."""
     one_pass = w["hq"] == w["hkv"] and w["d"] == 128 and w["k_idx"] in (1, 2)
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"kernel": "tq_decode_attend (" + ("query projection + fused logits/softmax.V pass + merge" if one_pass
                                               else "tq_logits + tq_attend_v") + ")",
             "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
-            "traffic": None, "peak_source": src_txt, "ms": round(ms, 5),
+            "traffic": traffic, "peak_source": src_txt, "ms": round(ms, 5),
             "two_calls_ms": round(two_call_ms, 5), "algorithmic": "packed key and value records + norms per call"}
 
 
