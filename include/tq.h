@@ -175,8 +175,39 @@ tq_status tq_decode_attend(const tq_cache *k, const tq_cache *v, const float *q,
                            const float *codebook_k, const float *codebook_v, float *out,
                            void *workspace, size_t workspace_bytes, tq_stream stream);
 
+/* Workspace bytes tq_nn_search needs for a database of n_db vectors and n_queries
+ * queries (independent of k and of the device). */
+size_t tq_nn_workspace_size(const tq_cache *db, int32_t n_queries, int64_t n_db);
+
+/* Nearest-neighbour search on a packed key stream (zubnet.ai, paragraph 3, and
+ * winningdata.io, "Os numeros que importam": the quantizer also serves
+ * inner-product vector search). For every query a, the k database vectors j in
+ * [0, n_db) with the largest estimated inner product
+ *   score(a, j) = norm_j * ( <Pi q_a, c[code_j]> + rnorm_j * sqrt(pi/2)/d * <S q_a, 2 sign_j - 1> ),
+ * the key estimator of tq_logits, in order of decreasing score (equal scores:
+ * lower j first).
+ *   db: key cache (qjl = 1) with n_seq = n_kv_heads = 1, d 128 or 200,
+ *       idx_bits 1..3; its norm array 16-byte aligned. Fill it with
+ *       tq_quantize_append.
+ *   queries: [n_queries][d] float; Pi, S: [d][d] float, 16-byte aligned;
+ *   codebook: 2^idx_bits floats.
+ *   top_scores: [n_queries][k] float; top_ids: [n_queries][k] int64. A query
+ *   with fewer than k candidates (n_db < k) gets score -inf and id -1 in the
+ *   missing places.
+ * k: 1..16; n_db <= capacity and < 2^31; n_queries == 0 does nothing.
+ * Precision: the products run on the tensor core in fp16 with float32
+ * accumulation (Pi q and S q scaled per query by a power of two; centroids and
+ * rnorm_j sqrt(pi/2)/d rounded to fp16), so a score differs from the float64
+ * value of the estimator by about 1e-4 ||q|| norm_j.
+ * workspace: >= tq_nn_workspace_size bytes, 256-byte aligned; its status word
+ * is read by tq_workspace_status. */
+tq_status tq_nn_search(const tq_cache *db, const float *queries, int32_t n_queries, int64_t n_db,
+                       const float *Pi, const float *S, const float *codebook, int32_t k,
+                       float *top_scores, int64_t *top_ids,
+                       void *workspace, size_t workspace_bytes, tq_stream stream);
+
 /* Synchronises `stream`, reads the status word that the kernels of the last
- * tq_logits / tq_attend_v / tq_decode_attend call on this workspace wrote, and clears it.
+ * tq_logits / tq_attend_v / tq_decode_attend / tq_nn_search call on this workspace wrote, and clears it.
  * TQ_OK if no kernel reported a failure, TQ_ERR_DEVICE otherwise (the message
  * names the failure). */
 tq_status tq_workspace_status(void *workspace, tq_stream stream);

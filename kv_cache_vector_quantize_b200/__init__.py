@@ -5,6 +5,7 @@ The package is a thin layer over the C ABI declared in ``include/tq.h``:
 cache), ``tq_logits`` (attention logits on the packed keys) and
 ``tq_attend_v`` (softmax-weighted packed values), ``tq_decode_attend`` (the
 three decode steps in one call, one pass over the tokens where the shapes allow),
+``tq_nn_search`` (top-k inner-product search over a packed key stream),
 plus the setup helpers
 ``tq_codebook_fit`` and ``tq_sketch_rotation``. All compute runs in the CUDA
 kernels of ``csrc/`` built for sm_100a.
@@ -34,6 +35,8 @@ from ._binding import (  # noqa: F401
     tq_last_error,
     tq_logits,
     tq_logits_workspace_size,
+    tq_nn_search,
+    tq_nn_workspace_size,
     tq_quantize_append,
     tq_record_words,
     tq_sketch_rotation,

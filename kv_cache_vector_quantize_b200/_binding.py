@@ -59,6 +59,8 @@ def _load() -> ctypes.CDLL:
         "tq_attend_v_noalloc": (I32, [D, P, F, I32, I64, P, P, P, P]),
         "tq_decode_workspace_size": (SZ, [D, D, I32, I64]),
         "tq_decode_attend": (I32, [D, D, P, I32, I64, F, P, P, P, P, P, P, SZ, P]),
+        "tq_nn_workspace_size": (SZ, [D, I32, I64]),
+        "tq_nn_search": (I32, [D, P, I32, I64, P, P, P, I32, P, P, P, SZ, P]),
         "tq_workspace_status": (I32, [P, P]),
         "tq_last_error": (ctypes.c_char_p, []),
         "tq_debug_inject": (None, [I32, I32]),
@@ -280,6 +282,38 @@ def tq_decode_attend(kcache: PackedCache, vcache: PackedCache, q: torch.Tensor, 
                                  _ptr(Pi), _ptr(S), _ptr(codebook_k), _ptr(codebook_v), _ptr(out), _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
+
+
+def tq_nn_workspace_size(db: PackedCache, n_queries: int, n_db: int) -> int:
+    d = db.desc()
+    return int(_lib.tq_nn_workspace_size(ctypes.byref(d), int(n_queries), int(n_db)))
+
+
+def tq_nn_search(db: PackedCache, queries: torch.Tensor, n_db: int, Pi: torch.Tensor, S: torch.Tensor,
+                 codebook: torch.Tensor, k: int, scores: torch.Tensor | None = None, ids: torch.Tensor | None = None,
+                 workspace: torch.Tensor | None = None, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """queries [n_q, d] float32 -> (scores [n_q, k] float32, ids [n_q, k] int64): the k database
+    vectors of db[0, 0, :n_db] with the largest estimated inner product per query."""
+    if queries.dim() != 2 or queries.shape[1] != db.d:
+        raise ValueError(f"queries must be [n_q, {db.d}], got {tuple(queries.shape)}")
+    nq = queries.shape[0]
+    _need(queries, "queries", torch.float32, device=db.device)
+    _need(Pi, "Pi", torch.float32, (db.d, db.d), db.device)
+    _need(S, "S", torch.float32, (db.d, db.d), db.device)
+    _need(codebook, "codebook", torch.float32, (1 << db.idx_bits,), db.device)
+    if scores is None:
+        scores = torch.empty((nq, k), dtype=torch.float32, device=db.device)
+    if ids is None:
+        ids = torch.empty((nq, k), dtype=torch.int64, device=db.device)
+    _need(scores, "scores", torch.float32, (nq, k), db.device)
+    _need(ids, "ids", torch.int64, (nq, k), db.device)
+    if workspace is None:
+        workspace = torch.empty(max(tq_nn_workspace_size(db, nq, n_db), 256), dtype=torch.uint8, device=db.device)
+    d = db.desc()
+    _check(_lib.tq_nn_search(ctypes.byref(d), _ptr(queries), nq, int(n_db), _ptr(Pi), _ptr(S), _ptr(codebook),
+                             int(k), _ptr(scores), _ptr(ids), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream)))
+    return scores, ids
 
 
 def tq_workspace_status(workspace: torch.Tensor, stream=None) -> None:

@@ -161,6 +161,28 @@ cudaError_t launch_attend_fast(const AttendParams &p, int bits, int n_seq, cudaS
 size_t attend_chunk_smem(int d, int bits, int64_t chunk);
 cudaError_t launch_combine(const float *partial, int rows, int n_chunks, int d, const float *Pi,
                            float *out, cudaStream_t st);
+// Nearest-neighbour search (nn_search.cu): running top-k of the key estimator over one packed
+// database stream for a batch of queries.
+struct NnArgs {
+  const uint32_t *records;
+  const float *norm, *rnorm;
+  const float *q;             // [n_q][d]
+  const float *Pi, *S, *codebook;
+  float *top_s;               // [n_q][k]
+  int64_t *top_i;             // [n_q][k]
+  unsigned char *qimg;        // workspace: fp16 query rows
+  float *sigma;               // workspace: per-query scale
+  float *part_s;              // workspace: per-CTA top-k lists
+  int *part_i;
+  uint32_t *status;
+  int64_t n_db;
+  int n_q, d, bits, k, grid;
+};
+constexpr int kNnMaxGrid = 256;     // upper bound on the search grid (sizes the workspace)
+constexpr int kNnMaxK = 16;
+bool nn_supported(int d, int bits);
+int nn_kp(int d);                   // padded K of a query row (fp16 elements)
+cudaError_t launch_nn_search(const NnArgs &a, cudaStream_t st);
 int device_sm_count();
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device).
 cudaError_t set_smem_once(const void *kernel, size_t bytes);

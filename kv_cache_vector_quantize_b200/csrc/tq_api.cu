@@ -555,6 +555,95 @@ tq_status tq_decode_attend(const tq_cache *k, const tq_cache *v, const float *q,
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_decode_attend (merge)");
 }
 
+// Workspace of tq_nn_search: header | fp16 query rows | per-query scale | partial top-k lists
+// (one per (CTA, query block) pair a CTA's contiguous unit range touches: grid + blocks - 1).
+struct NnWs {
+  size_t qimg, sigma, part_s, part_i, total;
+};
+
+NnWs nn_ws(int d, int n_queries, int64_t n_db) {
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  const int64_t n_qb = (n_queries + 127) / 128, n_tiles = (n_db + 127) / 128, units = n_qb * n_tiles;
+  const int64_t grid = units < kNnMaxGrid ? units : kNnMaxGrid;
+  const int64_t slots = grid > 0 ? grid + n_qb - 1 : 0;
+  NnWs w{};
+  w.qimg = kWsHeader;
+  w.sigma = w.qimg + up((size_t)n_qb * 128 * nn_kp(d) * 2);
+  w.part_s = w.sigma + up((size_t)n_qb * 128 * sizeof(float));
+  w.part_i = w.part_s + up((size_t)slots * 128 * kNnMaxK * sizeof(float));
+  w.total = w.part_i + up((size_t)slots * 128 * kNnMaxK * sizeof(int));
+  return w;
+}
+
+size_t tq_nn_workspace_size(const tq_cache *db, int32_t n_queries, int64_t n_db) {
+  if (!db || db->d <= 0 || n_queries < 0 || n_db < 0) return 0;
+  return nn_ws(db->d, n_queries, n_db).total;
+}
+
+tq_status tq_nn_search(const tq_cache *db, const float *queries, int32_t n_queries, int64_t n_db, const float *Pi,
+                       const float *S, const float *codebook, int32_t k, float *top_scores, int64_t *top_ids,
+                       void *workspace, size_t workspace_bytes, tq_stream stream) {
+  g_err[0] = 0;
+  tq_status s = check_cache(db, "tq_nn_search");
+  if (s != TQ_OK) return s;
+  if (!db->qjl) return fail(TQ_ERR_INVALID, "tq_nn_search: the database must be a key cache (qjl = 1)");
+  if (db->n_seq != 1 || db->n_kv_heads != 1)
+    return fail(TQ_ERR_INVALID, "tq_nn_search: the database is one stream (n_seq = n_kv_heads = 1), got %d x %d",
+                db->n_seq, db->n_kv_heads);
+  if (!nn_supported(db->d, db->idx_bits))
+    return fail(TQ_ERR_UNSUPPORTED, "tq_nn_search: d=%d idx_bits=%d (need d 128 or 200, idx_bits 1..3)", db->d,
+                db->idx_bits);
+  if (k < 1 || k > kNnMaxK) return fail(TQ_ERR_INVALID, "tq_nn_search: k=%d (need 1..%d)", k, kNnMaxK);
+  if (n_queries < 0) return fail(TQ_ERR_INVALID, "tq_nn_search: n_queries=%d", n_queries);
+  if (n_db < 0 || n_db > db->capacity)
+    return fail(TQ_ERR_CAPACITY, "tq_nn_search: n_db=%lld outside [0, capacity=%lld]", (long long)n_db,
+                (long long)db->capacity);
+  if (n_db > 0x7fffffffLL) return fail(TQ_ERR_UNSUPPORTED, "tq_nn_search: n_db=%lld above 2^31 - 1", (long long)n_db);
+  if (n_queries == 0) return TQ_OK;
+  if (!queries || !Pi || !S || !codebook || !top_scores || !top_ids)
+    return fail(TQ_ERR_INVALID, "tq_nn_search: NULL tensor argument");
+  if (!aligned(Pi, 16) || !aligned(S, 16) || !aligned(db->norm, 16))
+    return fail(TQ_ERR_INVALID, "tq_nn_search: Pi, S and the database norms must be 16-byte aligned");
+  const NnWs w = nn_ws(db->d, n_queries, n_db);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.total)
+    return fail(TQ_ERR_WORKSPACE, "tq_nn_search: workspace needs %zu bytes, 256-byte aligned (got %zu)", w.total,
+                workspace_bytes);
+  if (injected(&s)) return s;
+  unsigned char *ws = static_cast<unsigned char *>(workspace);
+  NnArgs a{};
+  a.records = db->records;
+  a.norm = db->norm;
+  a.rnorm = db->rnorm;
+  a.q = queries;
+  a.Pi = Pi;
+  a.S = S;
+  a.codebook = codebook;
+  a.top_s = top_scores;
+  a.top_i = top_ids;
+  a.qimg = ws + w.qimg;
+  a.sigma = reinterpret_cast<float *>(ws + w.sigma);
+  a.part_s = reinterpret_cast<float *>(ws + w.part_s);
+  a.part_i = reinterpret_cast<int *>(ws + w.part_i);
+  a.status = static_cast<uint32_t *>(workspace);
+  a.n_db = n_db;
+  a.n_q = n_queries;
+  a.d = db->d;
+  a.bits = db->idx_bits;
+  a.k = k;
+  const int64_t units = (int64_t)((n_queries + 127) / 128) * ((n_db + 127) / 128);
+  int64_t grid = device_sm_count();
+  if (grid > kNnMaxGrid) grid = kNnMaxGrid;
+  if (grid > units) grid = units;
+  a.grid = (int)grid;
+  cudaError_t e = cudaSuccess;
+  if (n_db == 0) {   // no scan: the status word is cleared here, the merge writes empty lists
+    e = cudaMemsetAsync(workspace, 0, sizeof(uint32_t), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "tq_nn_search (status)");
+  }
+  e = launch_nn_search(a, (cudaStream_t)stream);
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_nn_search");
+}
+
 tq_status tq_workspace_status(void *workspace, tq_stream stream) {
   g_err[0] = 0;
   if (!workspace || !aligned(workspace, 256)) return fail(TQ_ERR_WORKSPACE, "tq_workspace_status: bad workspace");

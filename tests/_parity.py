@@ -7,7 +7,12 @@ Tolerances (stated by the task for this method):
     such excused flips must be at most 1e-4 of all coordinates;
   * norms (||x|| and rho) to 1e-5 relative;
   * logits to 2e-3 * ||q|| * n_t, with the oracle evaluated on the GPU's cache;
-  * softmax.V to 2e-3 * max_t n_t (infinity norm), oracle on the GPU's cache and logits.
+  * softmax.V to 2e-3 * max_t n_t (infinity norm), oracle on the GPU's cache and logits;
+  * nearest-neighbour top-k: each returned score within the logit tolerance of the
+    oracle's score of that database vector, the r-th returned score within the
+    tolerance of the oracle's r-th largest score (order statistics move by at most
+    the largest score error), indices distinct, scores non-increasing, equal scores
+    in index order, and (-inf, -1) exactly where the database has fewer than k vectors.
 Where the GPU moved a code across a threshold (excused), rho and the sign bits
 are checked against the oracle re-run on the GPU's codes.
 """
@@ -94,3 +99,34 @@ def check_attend(gpu, lg, scale, Pi, codebook, rec, norm, d, bits):
     err = np.abs(np.asarray(gpu, dtype=np.float64) - ref)
     assert np.all(err <= tol), f"softmax.V error {np.max(err) / tol:.3g} x tolerance"
     return float(np.max(err) / tol) if err.size else 0.0
+
+
+def check_nn(gpu_s, gpu_i, q, Pi, S, codebook, rec, norm, rnorm, d, bits, k):
+    """gpu_s/gpu_i: [nq, k] top-k scores and ids; q: [nq, d]; rec/norm/rnorm: the GPU's database
+    cache (already checked against the oracle's encoding). Returns the worst error / tolerance."""
+    gi, gs = otq.unpack(rec, d, bits, True)
+    ref = otq.logits(q, Pi, S, codebook, norm, rnorm, gi, gs)          # [nq, n_db] float64
+    n_db = ref.shape[1]
+    kk = min(k, n_db)
+    gpu_s = np.asarray(gpu_s, dtype=np.float64)
+    gpu_i = np.asarray(gpu_i)
+    assert np.all(gpu_i[:, kk:] == -1) and np.all(np.isneginf(gpu_s[:, kk:])), "padding entries"
+    worst = 0.0
+    qn = np.linalg.norm(np.asarray(q, dtype=np.float64), axis=1)
+    nmax = float(np.max(norm)) if n_db else 0.0
+    for a in range(gpu_s.shape[0]):
+        ids, sc = gpu_i[a, :kk], gpu_s[a, :kk]
+        assert np.all((ids >= 0) & (ids < n_db)), f"query {a}: ids out of range {ids}"
+        assert len(set(ids.tolist())) == kk, f"query {a}: repeated ids {ids}"
+        assert np.all(np.diff(sc) <= 0), f"query {a}: scores not sorted {sc}"
+        ties = np.nonzero(np.diff(sc) == 0)[0]
+        assert np.all(ids[ties] < ids[ties + 1]), f"query {a}: equal scores out of index order"
+        tol_j = LOGIT_TOL * qn[a] * np.asarray(norm)[ids] + 1e-30
+        err = np.abs(sc - ref[a, ids])
+        assert np.all(err <= tol_j), f"query {a}: score error {np.max(err / tol_j):.3g} x tolerance"
+        tol = LOGIT_TOL * qn[a] * nmax + 1e-30
+        order = np.sort(ref[a])[::-1][:kk]
+        oerr = np.abs(sc - order)
+        assert np.all(oerr <= tol), f"query {a}: rank error {np.max(oerr / tol):.3g} x tolerance"
+        worst = max(worst, float(np.max(err / tol_j)), float(np.max(oerr / tol)))
+    return worst

@@ -150,6 +150,33 @@ def test_decode_attend_argument_checks():
     assert lib.tq_decode_workspace_size(ctypes.byref(k), ctypes.byref(_desc(qjl=0, heads=4)), 2, nt) == 0
 
 
+def test_nn_search_argument_checks():
+    def call(db, nq=300, ndb=40, k=10, ws_bytes=1 << 26, q=FAKE, Pi=FAKE):
+        return lib.tq_nn_search(ctypes.byref(db), q, nq, ndb, Pi, FAKE, FAKE, k, FAKE, FAKE, FAKE, ws_bytes, None)
+    db = _desc(d=200, bits=1, heads=1)
+    assert call(_desc(d=200, bits=1, qjl=0, heads=1, rnorm=None)) == tqb.TQ_ERR_INVALID   # needs the sign field
+    assert call(_desc(d=200, bits=1, heads=2)) == tqb.TQ_ERR_INVALID                      # one stream
+    assert call(_desc(d=64, bits=1, heads=1)) == tqb.TQ_ERR_UNSUPPORTED
+    assert call(_desc(d=200, bits=4, heads=1)) == tqb.TQ_ERR_UNSUPPORTED
+    assert call(db, k=0) == tqb.TQ_ERR_INVALID
+    assert call(db, k=17) == tqb.TQ_ERR_INVALID
+    assert call(db, nq=-1) == tqb.TQ_ERR_INVALID
+    assert call(db, ndb=65) == tqb.TQ_ERR_CAPACITY
+    assert call(db, nq=0) == tqb.TQ_OK                                                    # nothing to do
+    assert call(db, q=None) == tqb.TQ_ERR_INVALID
+    assert call(db, Pi=FAKE + 4) == tqb.TQ_ERR_INVALID                                    # float4 rows
+    assert call(_desc(d=200, bits=1, heads=1, norm=FAKE + 4100)) == tqb.TQ_ERR_INVALID     # float4 norms
+    assert call(db, ws_bytes=1024) == tqb.TQ_ERR_WORKSPACE
+    assert call(db) == tqb.TQ_ERR_CUDA                                                    # passes -> injected
+    # status | fp16 query rows (padded K 448) | scales | (CTAs + blocks - 1) lists of 16 scores and ids
+    up = lambda v: (v + 255) // 256 * 256
+    nqb, tiles = 3, 1
+    slots = min(nqb * tiles, 256) + nqb - 1
+    want = 256 + up(nqb * 128 * 448 * 2) + up(nqb * 128 * 4) + 2 * up(slots * 128 * 16 * 4)
+    assert lib.tq_nn_workspace_size(ctypes.byref(db), 300, 40) == want
+    assert lib.tq_nn_workspace_size(ctypes.byref(db), 300, 0) == 256 + up(nqb * 128 * 448 * 2) + up(nqb * 128 * 4)
+
+
 def test_fault_injection_counts_down():
     tqb.tq_debug_inject(tqb.TQ_ERR_DEVICE, 2)
     assert _q(_desc(qjl=0)) == tqb.TQ_ERR_DEVICE

@@ -300,6 +300,85 @@ def test_decode_attend_parity(shape):
                              vn[s_, h, :T], d, vb)
 
 
+def test_decode_attend_caches_of_different_capacity():
+    # key and value caches sized differently (each indexed with its own capacity); the step equals
+    # the two calls on the same caches
+    d, B, H, T = 128, 2, 2, 1000
+    k = syn.gaussian((B, H, T, d), 71).to(torch.bfloat16).cuda()
+    v = syn.lognormal_sphere((B, H, T, d), 72, dtype=torch.bfloat16).cuda()
+    q = syn.gaussian((B, H, d), 73).cuda()
+    _, _, _, _, g = _setup(d, 2, 3)
+    kc = tqb.PackedCache.empty(d, 2, True, B, H, T + 37)
+    vc = tqb.PackedCache.empty(d, 3, False, B, H, T + 1029)
+    tqb.tq_quantize_append(kc, k, 0, g["Pi"], g["SPiT"], g["ck"])
+    tqb.tq_quantize_append(vc, v, 0, g["Pi"], None, g["cv"])
+    sc = 1.0 / math.sqrt(d)
+    lg = tqb.tq_logits(kc, q, T, g["Pi"], g["S"], g["ck"])
+    out2 = tqb.tq_attend_v(vc, lg, sc, T, g["Pi"], g["cv"])
+    ws = torch.empty(max(256, tqb.tq_decode_workspace_size(kc, vc, H, T)), dtype=torch.uint8, device="cuda")
+    out1 = tqb.tq_decode_attend(kc, vc, q, T, sc, g["Pi"], g["S"], g["ck"], g["cv"], workspace=ws)
+    torch.cuda.synchronize()
+    tqb.tq_workspace_status(ws)
+    assert torch.equal(out1, out2)
+
+
+# ---------------------------------------------------------------------------
+# nearest-neighbour search (top-k of the key estimator over one database stream)
+# ---------------------------------------------------------------------------
+
+def _nn_case(d, bits, n_db, n_q, k, capacity=None):
+    db, qs = syn.nn_inputs(n_db, n_q, d)
+    Pi, S, ck, _, g = _setup(d, bits, 1)
+    cache = tqb.PackedCache.empty(d, bits, True, 1, 1, capacity or max(n_db, 1))
+    if n_db:
+        tqb.tq_quantize_append(cache, db.reshape(1, 1, n_db, d).cuda(), 0, g["Pi"], g["SPiT"], g["ck"])
+    ws = torch.empty(max(256, tqb.tq_nn_workspace_size(cache, n_q, n_db)), dtype=torch.uint8, device="cuda")
+    sc, ids = tqb.tq_nn_search(cache, qs.cuda(), n_db, g["Pi"], g["S"], g["ck"], k, workspace=ws)
+    torch.cuda.synchronize()
+    tqb.tq_workspace_status(ws)
+    rec = par.as_u32(cache.records[0, 0, :n_db].cpu().numpy())
+    norm = cache.norm[0, 0, :n_db].cpu().numpy()
+    rnorm = cache.rnorm[0, 0, :n_db].cpu().numpy()
+    return db, qs, Pi, S, ck, rec, norm, rnorm, sc.cpu().numpy(), ids.cpu().numpy()
+
+
+@pytest.mark.parametrize("d,bits,n_db,n_q,k", [
+    (200, 1, 5000, 300, 10),     # 40 tiles (ragged 8), 3 query blocks (ragged 44): one unit per CTA
+    (200, 3, 5000, 300, 10),
+    (200, 1, 40000, 300, 10),    # 313 tiles x 3 blocks over the SMs: CTA ranges cross query blocks
+    (200, 3, 40000, 130, 16),
+    (200, 2, 20000, 257, 1),
+    (128, 2, 9000, 200, 7),
+    (128, 1, 3000, 1, 16),
+])
+def test_nn_search_parity(d, bits, n_db, n_q, k):
+    db, qs, Pi, S, ck, rec, norm, rnorm, sc, ids = _nn_case(d, bits, n_db, n_q, k)
+    par.check_encoding(db.numpy(), rec, norm, rnorm, Pi, S, ck, d, bits, True)
+    par.check_nn(sc, ids, qs.numpy(), Pi, S, ck, rec, norm, rnorm, d, bits, k)
+
+
+@pytest.mark.parametrize("n_db", [0, 1, 5])
+def test_nn_search_fewer_vectors_than_k(n_db):
+    db, qs, Pi, S, ck, rec, norm, rnorm, sc, ids = _nn_case(200, 1, n_db, 130, 10, capacity=64)
+    assert np.all(ids[:, n_db:] == -1) and np.all(np.isneginf(sc[:, n_db:]))
+    if n_db:
+        par.check_nn(sc, ids, qs.numpy(), Pi, S, ck, rec, norm, rnorm, 200, 1, 10)
+
+
+def test_nn_search_equal_vectors_rank_by_index():
+    # the same vector stored 300 times: every score ties, so the top-k are the k lowest indices
+    d, bits, n, k = 200, 1, 300, 16
+    _, qs = syn.nn_inputs(1, 40, d)
+    x = syn.nn_inputs(1, 1, d)[0].repeat(n, 1)
+    _, _, _, _, g = _setup(d, bits, 1)
+    cache = tqb.PackedCache.empty(d, bits, True, 1, 1, n)
+    tqb.tq_quantize_append(cache, x.reshape(1, 1, n, d).cuda(), 0, g["Pi"], g["SPiT"], g["ck"])
+    sc, ids = tqb.tq_nn_search(cache, qs.cuda(), n, g["Pi"], g["S"], g["ck"], k)
+    ids = ids.cpu().numpy()
+    assert np.all(ids == np.arange(k)[None, :]), ids[:3]
+    assert torch.all(sc == sc[:, :1]).item()
+
+
 def test_decode_attend_empty():
     d = 128
     _, _, _, _, g = _setup(d, 2, 3)
