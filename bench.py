@@ -67,7 +67,7 @@ def parse():
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--workload", default="llama",
                     choices=["llama"] + [f"sweep-b{b}{s}" for b in (2, 3, 4) for s in ("", "-s4")]
-                    + ["large-b3", "large-b4"])
+                    + ["large-b3", "large-b4", "nn-b2", "nn-b4"])
     ap.add_argument("--layers", type=int, default=80, help="layers streamed by the large-model workload")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -79,6 +79,13 @@ def parse():
 # ----------------------------------------------------------------------------
 
 def workload(name: str):
+    if name.startswith("nn"):
+        b = int(name.split("-")[1][1:])
+        return dict(kind="nn", name=f"nn-search-b{b}: 1,000,000 database vectors d=200 (unit-normalised anisotropic "
+                                    f"Gaussian, per-dimension std U[0.2, 2]), 10,000 queries of the same law, b={b} "
+                                    f"({b - 1}-bit codes + QJL), top-10 by the key estimator; a synthetic stand-in "
+                                    f"for the GloVe-200 benchmark",
+                    n_db=1_000_000, n_q=10_000, d=200, k_idx=b - 1, k=10)
     if name == "llama":
         return dict(name="llama3-8b-decode: B=1 Hq=32 Hkv=8 d=128 T=32768 bf16 K b=3 (2-bit codes+QJL) V b=3 MSE",
                     n_seq=1, hq=32, hkv=8, d=128, T=32768, k_idx=2, v_idx=3, dtype=torch.bfloat16,
@@ -513,6 +520,165 @@ def run_large(args, rank, world, local_rank):
     return result, w
 
 
+def nn_record_bytes(w) -> int:
+    return 4 * ((w["k_idx"] * w["d"] + 31) // 32 + (w["d"] + 31) // 32) + 8
+
+
+def run_nn(args, rank, world, local_rank):
+    """Nearest-neighbour search: per step, quantize the database into a packed key stream, flush
+    L2, then the top-10 search of every query (tq_nn_search). Recall@10 against the exact float64
+    inner products is measured after the timed region."""
+    import kv_cache_vector_quantize_b200 as tqb
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = workload(args.workload)
+    d, N, Q, k = w["d"], w["n_db"], w["n_q"], w["k"]
+    db, qs = syn.nn_inputs(N, Q, d, device=dev)
+    Pi = syn.rotation(d).to(dev)
+    S = syn.sketch(d).to(dev)
+    cb = tqb.tq_codebook_fit(d, w["k_idx"]).to(dev)
+    SPiT = tqb.tq_sketch_rotation(Pi, S)
+    cache = tqb.PackedCache.empty(d, w["k_idx"], True, 1, 1, N, device=dev)
+    x = db.reshape(1, 1, N, d)
+    scores = torch.empty((Q, k), dtype=torch.float32, device=dev)
+    ids = torch.empty((Q, k), dtype=torch.int64, device=dev)
+    ws = torch.empty(tqb.tq_nn_workspace_size(cache, Q, N), dtype=torch.uint8, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        tqb.tq_quantize_append(cache, x, 0, Pi, SPiT, cb)
+        if ev is not None:
+            ev[1].record(stream)
+        flush.fill_(1.0)
+        if ev is not None:
+            ev[2].record(stream)
+        tqb.tq_nn_search(cache, qs, N, Pi, S, cb, k, scores, ids, ws)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    tqb.tq_workspace_status(ws)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index)
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.mark_start()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.mark_end()
+    tqb.tq_workspace_status(ws)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    per = {n: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / len(evs)
+           for i, n in enumerate(("quantize", "l2_flush", "nn_search"))}
+    total_ms = t_start.elapsed_time(t_end)
+    total_ms, search_ms, quant_ms = max_over_ranks([total_ms, per["nn_search"], per["quantize"]], dev, world)
+
+    # recall@10 of the returned ids against the exact top-10 of the float64 inner products
+    hits = 0
+    dbd = db.double()
+    for a in range(0, Q, 500):
+        exact = (qs[a:a + 500].double() @ dbd.T).topk(k, dim=1).indices
+        hits += int((exact[:, :, None] == ids[a:a + 500, None, :]).any(dim=2).sum().item())
+    del dbd
+    recall = hits / (Q * k)
+
+    e2e = None
+    if args.e2e_steps > 0:
+        hx = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+        hq = torch.empty(qs.shape, dtype=qs.dtype, pin_memory=True)
+        hx.copy_(x)
+        hq.copy_(qs)
+        hs = torch.empty(scores.shape, dtype=scores.dtype, pin_memory=True)
+        hi = torch.empty(ids.shape, dtype=ids.dtype, pin_memory=True)
+
+        def step_e2e():
+            x.copy_(hx, non_blocking=True)
+            qs.copy_(hq, non_blocking=True)
+            tqb.tq_quantize_append(cache, x, 0, Pi, SPiT, cb)
+            tqb.tq_nn_search(cache, qs, N, Pi, S, cb, k, scores, ids, ws)
+            hs.copy_(scores, non_blocking=True)
+            hi.copy_(ids, non_blocking=True)
+
+        for _ in range(2):
+            step_e2e()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            step_e2e()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks([a.elapsed_time(b) / args.e2e_steps], dev, world)[0]
+        e2e = {"value": round(world * N * nn_record_bytes(w) / (e2e_ms * 1e-3) / 1e9, 3), "unit": UNIT,
+               "ms_per_step": round(e2e_ms, 4),
+               "h2d_bytes_per_step": hx.numel() * hx.element_size() + hq.numel() * hq.element_size(),
+               "d2h_bytes_per_step": hs.numel() * hs.element_size() + hi.numel() * hi.element_size(),
+               "note": "packed database bytes per end-to-end step (pinned H2D of the database and the queries, "
+                       "quantize, search, D2H of the top-10 scores and ids)"}
+
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    tf_burst = float(peaks["bf16_tflops"])
+    tf_sust = float(peaks.get("bf16_tflops_sustained", tf_burst))
+    src_txt = (f"bf16_tflops (burst; fp16 has the same nominal dense rate), {peak_src} (MEASURED_PEAKS.json)"
+               if peak_src == "measured" else "fallback")
+    nb = N * nn_record_bytes(w)
+    scan_gbs = nb / (search_ms * 1e-3) / 1e9
+    flops = 2.0 * Q * N * 2 * d
+    tfs = flops / (search_ms * 1e-3) / 1e12
+    kp = 64 * ((2 * d + 63) // 64)
+    padded = 2.0 * ((Q + 127) // 128 * 128) * ((N + 127) // 128 * 128) * kp
+    q_bytes, q_flops = N * (4 * d + nn_record_bytes(w)), N * 4 * d * d
+    q_gbs, q_tfs = q_bytes / (quant_ms * 1e-3) / 1e9, q_flops / (quant_ms * 1e-3) / 1e12
+    result = {
+        "metric": METRIC, "value": round(world * scan_gbs, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": w["name"], "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "flushed (2 x L2 write) between quantize and search inside every step",
+                   "value_definition": "packed database bytes (records + norms) per tq_nn_search call / its mean "
+                                       "device time; the call is bound by the tensor core (roofline)"},
+        "recall_at_10": round(recall, 4),
+        "quantize_tokens_per_s": round(world * N / (quant_ms * 1e-3), 1),
+        "per_kernel_ms": {n: round(v, 4) for n, v in per.items()},
+        "packed_bytes": {"database": nb},
+        "roofline": {"kernel": "tq_nn_search (query projection + nn_scan_kernel tensor-core scan + merge)",
+                     "bound": "tensor", "achieved": round(tfs, 1), "peak": tf_burst, "unit": "TFLOP/s",
+                     "frac": round(tfs / tf_burst, 4), "frac_vs_sustained": round(tfs / tf_sust, 4),
+                     "traffic": NCU_TRAFFIC.get(("nn_search", args.workload)), "peak_source": src_txt,
+                     "algorithmic": f"{4 * d} flop per (query, database vector) pair (two length-{d} dot "
+                                    f"products); the kernel issues {padded / flops:.3f}x that with the padding of "
+                                    f"K to {kp} and of queries and vectors to 128"},
+        "roofline_nn_scan_hbm": {"bound": "hbm", "achieved": round(scan_gbs, 2), "peak": hbm, "unit": "GB/s",
+                                 "frac": round(scan_gbs / hbm, 5)},
+        "roofline_quantize": {"kernel": "quantize_kernel (tq_quantize_append, d = 200 fp32 database)",
+                              "bound": "hbm" if q_bytes / hbm > q_flops / (tf_burst * 1e3) else "tensor",
+                              "achieved_gbs": round(q_gbs, 1), "hbm_frac": round(q_gbs / hbm, 4),
+                              "achieved_tflops": round(q_tfs, 2),
+                              "algorithmic": f"{4 * d + nn_record_bytes(w)} B and {4 * d * d} flop per vector"},
+        # per step: the quantize kernel; projection, scan and merge of the search
+        "gpu_launches": 4 * args.steps, "clocks": clk, "e2e": e2e,
+    }
+    return result, w
+
+
 # ----------------------------------------------------------------------------
 # the oracle on a bounded sample (cpu_baseline and the reference arm)
 # ----------------------------------------------------------------------------
@@ -546,7 +712,42 @@ def oracle_sample_step(w, state):
     vi, _ = otq.unpack(state["vrec"], d, w["v_idx"], False)
     otq.attend_v(lg, 1.0 / math.sqrt(d), state["vn"], vi, state["Pi"], state["cv"])
     rec = 4 * ((w["k_idx"] * d + 31) // 32 + (d + 31) // 32)
-    return state["krec"].shape[0] * (rec + 8), t2 - t1, t1 - t0, state["k_rows"].shape[0]
+    return state["krec"].shape[0] * (rec + 8), t2 - t1, t1 - t0, 2 * state["k_rows"].shape[0]
+
+
+def oracle_nn_step(w, state):
+    """One bounded sample of the search through the oracle: quantize 2048 database vectors;
+    unpack + estimator scores of 32 queries over 20000 packed vectors + top-10. Returns (the
+    workload's packed database bytes prorated to the (query, vector) pairs scored, scoring
+    seconds, quantize seconds, vectors quantized)."""
+    from oracle import turboquant as otq
+
+    d = w["d"]
+    t0 = time.perf_counter()
+    e = otq.quantize(state["rows"], state["Pi"], state["c"], state["S"])
+    otq.pack(e["idx"], e["sign"], d, w["k_idx"], True)
+    t1 = time.perf_counter()
+    gi, gs = otq.unpack(state["rec"], d, w["k_idx"], True)
+    lg = otq.logits(state["q"], state["Pi"], state["S"], state["c"], state["n"], state["r"], gi, gs)
+    otq.topk(lg, w["k"])
+    t2 = time.perf_counter()
+    pairs = state["q"].shape[0] * state["rec"].shape[0]
+    return nn_record_bytes(w) * pairs / w["n_q"], t2 - t1, t1 - t0, state["rows"].shape[0]
+
+
+def oracle_nn_state(w):
+    from oracle import codebook as ocb
+    from oracle import turboquant as otq
+
+    d = w["d"]
+    Pi = syn.rotation(d).double().numpy()
+    S = syn.sketch(d).double().numpy()
+    c = ocb.fit_codebook(d, w["k_idx"])[0]
+    db, qs = syn.nn_inputs(20000, 32, d)
+    dbn = db.double().numpy()
+    e = otq.quantize(dbn, Pi, c, S)
+    return {"Pi": Pi, "S": S, "c": c, "rows": dbn[:2048], "n": e["norm"], "r": e["rnorm"],
+            "rec": otq.pack(e["idx"], e["sign"], d, w["k_idx"], True), "q": qs.double().numpy()}
 
 
 def oracle_state(w):
@@ -576,19 +777,21 @@ def oracle_state(w):
 
 def run_oracle(w, n_steps, n_warmup, budget_s=None):
     """Returns (logit-scan GB/s, mean step seconds, steps, quantize head-vectors/s)."""
-    state = oracle_state(w)
+    nn = w.get("kind") == "nn"
+    state = oracle_nn_state(w) if nn else oracle_state(w)
+    sample_step = oracle_nn_step if nn else oracle_sample_step
     for _ in range(n_warmup):
-        oracle_sample_step(w, state)
+        sample_step(w, state)
     steps, lg_s, q_s, nbytes, nvec = [], 0.0, 0.0, 0, 0
     t_all = time.perf_counter()
     while True:
         t0 = time.perf_counter()
-        b, tl, tq_, nv = oracle_sample_step(w, state)
+        b, tl, tq_, nv = sample_step(w, state)
         steps.append(time.perf_counter() - t0)
         lg_s += tl
         q_s += tq_
         nbytes += b
-        nvec += 2 * nv
+        nvec += nv
         if budget_s is None:
             if len(steps) >= n_steps:
                 break
@@ -598,6 +801,11 @@ def run_oracle(w, n_steps, n_warmup, budget_s=None):
 
 
 def sample_text(w):
+    if w.get("kind") == "nn":
+        return (f"per step: oracle quantize of 2048 database vectors, unpack + estimator scores of 32 queries over "
+                f"20000 packed vectors + top-{w['k']}; value = the workload's packed database bytes x (pairs "
+                f"scored / {w['n_q']} queries x {w['n_db']} vectors) / oracle scoring time, i.e. the GB/s of one "
+                f"pass of all {w['n_q']} queries at the sampled rate")
     G = w["hq"] // w["hkv"]
     return (f"per step: oracle quantize of 2048 keys + 2048 values, unpack + logits of {G} query heads over one "
             f"KV head's {w['T']} packed keys, softmax.V over that head (1/{w['n_seq'] * w['hkv']} of the "
@@ -618,14 +826,15 @@ def main():
             return
         val, step_s, n, qvps = run_oracle(w, args.steps, args.warmup)
         cores = _threads()
-        line = {"metric": METRIC, "value": round(val, 6), "unit": UNIT, "n_gpus": args.gpus, "steps": n,
+        val = float(f"{val:.4g}")
+        line = {"metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus, "steps": n,
                 "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 2), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
                 "config": {"workload": w["name"], "parallelism": "single"},
                 "quantize_head_vectors_per_s": round(qvps, 1),
-                "cpu_baseline": {"value": round(val, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+                "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle",
                                  "sample": sample_text(w)},
-                "e2e": {"value": round(val, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+                "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
 
@@ -634,11 +843,13 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     if args.workload.startswith("large"):
         result, w = run_large(args, rank, world, local_rank)
+    elif args.workload.startswith("nn"):
+        result, w = run_nn(args, rank, world, local_rank)
     else:
         result, w = run_tq(args, rank, world, local_rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         val, step_s, n, qvps = run_oracle(w, 0, 1, budget_s=12.0)
-        result["cpu_baseline"] = {"value": round(val, 6), "unit": UNIT, "cores": _threads(), "kind": "oracle",
+        result["cpu_baseline"] = {"value": float(f"{val:.4g}"), "unit": UNIT, "cores": _threads(), "kind": "oracle",
                                   "quantize_head_vectors_per_s": round(qvps, 1),
                                   "sample": sample_text(w) + f"; {n} steps of {step_s:.2f} s"}
     if rank == 0:

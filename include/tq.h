@@ -187,8 +187,8 @@ size_t tq_nn_workspace_size(const tq_cache *db, int32_t n_queries, int64_t n_db)
  * the key estimator of tq_logits, in order of decreasing score (equal scores:
  * lower j first).
  *   db: key cache (qjl = 1) with n_seq = n_kv_heads = 1, d 128 or 200,
- *       idx_bits 1..3; its norm array 16-byte aligned. Fill it with
- *       tq_quantize_append.
+ *       idx_bits 1..3, filled by tq_quantize_append; its norm and rnorm
+ *       arrays 16-byte aligned (they are read by bulk copies).
  *   queries: [n_queries][d] float; Pi, S: [d][d] float, 16-byte aligned;
  *   codebook: 2^idx_bits floats.
  *   top_scores: [n_queries][k] float; top_ids: [n_queries][k] int64. A query

@@ -13,13 +13,16 @@
 //   score(q, j) = sigma_q n_j (A B^T)[q, j]
 // One persistent CTA per SM walks a contiguous range of (query block, database tile) units:
 //   * the 128 queries of the current block sit in tensor memory as the MMA's A operand;
-//   * eight decode warps turn each 128-vector tile's records into B, one 64-element K chunk
-//     at a time, in a ring of 128-byte-swizzled shared-memory chunks;
+//   * a copy warp streams each 128-vector tile's records and norms into shared memory;
+//   * eight decode warps turn them into B, one 64-element K chunk at a time, in a ring of
+//     128-byte-swizzled shared-memory chunks;
 //   * one thread issues tcgen05 MMAs (M = 128 queries, N = 128 vectors, K = 16) into one of
 //     two tensor-memory accumulators;
 //   * four epilogue warps (one per lane quadrant) keep a running top-k per query row in
 //     registers and write it to a per-CTA partial list when the query block changes.
 // A merge kernel then combines the partial lists of every CTA that covered a query block.
+#include <type_traits>
+
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -28,12 +31,14 @@ namespace {
 
 constexpr int kQB = 128;                 // queries per block: MMA M, one tensor-memory lane each
 constexpr int kNT = 128;                 // database vectors per tile: MMA N
-constexpr int kDecWarps = 8;             // two groups of four: even and odd K chunks
+constexpr int kDecWarps = 8;             // two groups of four (even and odd K chunks); a thread owns a row
 constexpr int kEpiWarps = 4;             // one per lane quadrant
-constexpr int kNnThreads = 32 * (1 + kDecWarps + kEpiWarps);
-constexpr int kSlots = 8;                // shared-memory ring of B chunks
+constexpr int kLists = kEpiWarps / 4;   // partial top-k lists per query row and CTA
+constexpr int kNnThreads = 32 * (2 + kDecWarps + kEpiWarps);   // + MMA warp + copy warp
+constexpr int kRStages = 4;              // ring of database tiles (records, norms, rnorms) in shared memory
 constexpr uint32_t kChunk = kNT * 128;   // one 64-element K block of a tile: 16 KB
 constexpr uint32_t kAcc0 = 256;          // first accumulator column; two buffers of kNT columns
+constexpr int kNrmRing = 4;              // tiles of database norms staged for the epilogue
 constexpr int kPrepQ = 16;               // queries per CTA of the projection kernel
 constexpr int kPrepThreads = 256;
 
@@ -63,12 +68,21 @@ struct NnRec {
   static_assert(RW % 2 == 0, "records are read as 8-byte pairs");
 };
 
-template <int BETA>
+template <int D, int BETA>
 struct NnSmem {
-  static constexpr uint32_t kBFull = 0, kBEmpty = 64, kDFull = 128, kDEmpty = 144, kAFull = 160, kTslot = 168;
+  static constexpr uint32_t kBFull = 0, kBEmpty = 96, kDFull = 192, kDEmpty = 208, kAFull = 224, kNFull = 232,
+                            kNEmpty = 264, kRFull = 296, kREmpty = 328, kTslot = 360;
+  static constexpr uint32_t kRecBytes = kNT * NnRec<D, BETA>::RW * 4;
+  static constexpr uint32_t kStage = kRecBytes + 2 * kNT * 4;   // records, norms, rnorms
+  static constexpr uint32_t kFixed = 1024 + NnLut<BETA>::BYTES + kNrmRing * kNT * 4 + kRStages * kStage;
+  // B chunks: as many as the opt-in shared memory (227 KB) leaves, at most 12
+  static constexpr int kSlots = (232448 - kFixed) / kChunk > 12 ? 12 : (int)((232448 - kFixed) / kChunk);
+  static_assert(kSlots >= 4, "B ring");
   static constexpr uint32_t kRing = 1024;   // 1024-byte aligned for the 128-byte swizzle
   static constexpr uint32_t kLut = kRing + kSlots * kChunk;
-  static constexpr uint32_t kBytes = kLut + NnLut<BETA>::BYTES;
+  static constexpr uint32_t kNrm = kLut + NnLut<BETA>::BYTES;   // [kNrmRing][kNT] database norms
+  static constexpr uint32_t kRec = kNrm + kNrmRing * kNT * 4;   // [kRStages] tile stages
+  static constexpr uint32_t kBytes = kRec + kRStages * kStage;
 };
 
 struct NnParams {
@@ -77,7 +91,7 @@ struct NnParams {
   const __half *qimg;     // [n_qb * 128][KP]
   const float *sigma;     // [n_qb * 128]
   const float *codebook;
-  float *part_s;          // [slots][128][kNnMaxK]
+  float *part_s;          // [slots][128][2][kNnMaxK] (the first kLists of each row used)
   int *part_i;
   uint32_t *status;
   int64_t n_db;
@@ -96,30 +110,30 @@ __device__ __forceinline__ uint2 lds64(uint32_t a) {
   return v;
 }
 
-// B values of 8 consecutive K elements (one 16-byte unit) of a database row. Units [0, D/8) hold
-// centroids c[idx] of coordinates 8 uk .. 8 uk + 7, units [D/8, D/4) the signed sketch weights
-// rho kappa (2 sign - 1), the rest zero padding. `nb` = fp16x2 of -rho kappa.
+// B values of 8 consecutive K elements (one 16-byte unit) of a database row whose record is held
+// in registers (`uk` a compile-time constant after unrolling, so every word index is too). Units
+// [0, D/8) hold centroids c[idx] of coordinates 8 uk .. 8 uk + 7 (one lookup of 8, or two of 4,
+// consecutive codes), units [D/8, D/4) the signed sketch weights rho kappa (2 sign - 1): half p of
+// word w takes sign bit 2 w + p into its own sign bit, the product placing bit 2w at bit 15 and bit
+// 2w + 1 at bit 31 without overlapping terms. The rest is zero padding. `nb` = fp16x2 of -rho kappa.
 template <int D, int BETA>
-__device__ __forceinline__ uint4 nn_unit(const uint32_t *rec, int uk, uint32_t lut, uint32_t nb) {
+__device__ __forceinline__ uint4 nn_unit_reg(const uint32_t *rec, int uk, uint32_t lut, uint32_t nb) {
   using R = NnRec<D, BETA>;
   constexpr int U8 = D / 8;
   if (uk < U8) {
     const int bit = 8 * BETA * uk, w = bit >> 5, sh = bit & 31;
     if constexpr (BETA == 1) {
-      const uint32_t e = (rec[w] >> sh) & 0xFFu;
-      return lds_u128(lut + 16u * e);
+      return lds_u128(lut + 16u * ((rec[w] >> sh) & 0xFFu));
     } else if constexpr (BETA == 2) {
       const uint32_t f = (rec[w] >> sh) & 0xFFFFu;
-      const uint2 lo = lds64(lut + 8u * (f & 0xFFu)), hi = lds64(lut + 8u * (f >> 8));
-      return make_uint4(lo.x, lo.y, hi.x, hi.y);
+      const uint2 a = lds64(lut + 8u * (f & 0xFFu)), b = lds64(lut + 8u * (f >> 8));
+      return make_uint4(a.x, a.y, b.x, b.y);
     } else {
-      const uint32_t f = (sh + 24 > 32 ? __funnelshift_r(rec[w], rec[w + 1], sh) : rec[w] >> sh) & 0xFFFFFFu;
-      const uint2 lo = lds64(lut + 8u * (f & 0xFFFu)), hi = lds64(lut + 8u * (f >> 12));
-      return make_uint4(lo.x, lo.y, hi.x, hi.y);
+      const uint32_t f = (sh > 8 ? __funnelshift_r(rec[w], rec[w + 1], sh) : rec[w] >> sh) & 0xFFFFFFu;
+      const uint2 a = lds64(lut + 8u * (f & 0xFFFu)), b = lds64(lut + 8u * (f >> 12));
+      return make_uint4(a.x, a.y, b.x, b.y);
     }
   } else if (uk < 2 * U8) {
-    // sign bits of coordinates 8 j .. 8 j + 7; half p of word w takes bit 2 w + p into its sign bit:
-    // the product places bit 2w at bit 15 and bit 2w + 1 at bit 31 without overlapping terms
     const int j = uk - U8;
     const uint32_t b = (rec[R::IW + (j >> 2)] >> (8 * (j & 3))) & 0xFFu;
     uint4 o;
@@ -153,9 +167,9 @@ template <int D, int BETA>
 __global__ void __launch_bounds__(kNnThreads, 1) nn_scan_kernel(const NnParams p) {
   using Dm = NnDim<D>;
   using R = NnRec<D, BETA>;
-  using L = NnSmem<BETA>;
+  using L = NnSmem<D, BETA>;
   using Lu = NnLut<BETA>;
-  constexpr int NCH = Dm::NCH, RW = R::RW;
+  constexpr int NCH = Dm::NCH, RW = R::RW, kSlots = L::kSlots;
   extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t sb = smem_u32(smem);
   auto b_full = [&](int s) { return sb + L::kBFull + 8u * s; };
@@ -163,7 +177,12 @@ __global__ void __launch_bounds__(kNnThreads, 1) nn_scan_kernel(const NnParams p
   auto d_full = [&](int b) { return sb + L::kDFull + 8u * b; };
   auto d_empty = [&](int b) { return sb + L::kDEmpty + 8u * b; };
   const uint32_t a_full = sb + L::kAFull;
-  const uint32_t ring = sb + L::kRing, lut = sb + L::kLut;
+  auto n_full = [&](int e) { return sb + L::kNFull + 8u * e; };
+  auto n_empty = [&](int e) { return sb + L::kNEmpty + 8u * e; };
+  auto r_full = [&](int e) { return sb + L::kRFull + 8u * e; };
+  auto r_empty = [&](int e) { return sb + L::kREmpty + 8u * e; };
+  const uint32_t ring = sb + L::kRing, lut = sb + L::kLut, stages = sb + L::kRec;
+  float *nrm_s = reinterpret_cast<float *>(smem + L::kNrm);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t u0 = p.units * blockIdx.x / gridDim.x, u1 = p.units * (blockIdx.x + 1) / gridDim.x;
@@ -171,7 +190,7 @@ __global__ void __launch_bounds__(kNnThreads, 1) nn_scan_kernel(const NnParams p
 
   if (tid == 0) {
     for (int s = 0; s < kSlots; ++s) {
-      mbar_init(b_full(s), 4);   // the four warps of the decode group that wrote the chunk
+      mbar_init(b_full(s), kDecWarps / 2);   // the decode group that wrote the chunk
       mbar_init(b_empty(s), 1);  // the MMAs' commit
     }
     for (int b = 0; b < 2; ++b) {
@@ -179,6 +198,14 @@ __global__ void __launch_bounds__(kNnThreads, 1) nn_scan_kernel(const NnParams p
       mbar_init(d_empty(b), kEpiWarps);
     }
     mbar_init(a_full, kEpiWarps);
+    for (int e = 0; e < kNrmRing; ++e) {
+      mbar_init(n_full(e), kDecWarps / 2);   // decode group 0 (all 128 rows)
+      mbar_init(n_empty(e), kEpiWarps);
+    }
+    for (int e = 0; e < kRStages; ++e) {
+      mbar_init(r_full(e), 1);   // the copy thread's expect_tx
+      mbar_init(r_empty(e), kDecWarps);
+    }
     mbar_fence_init();
   }
   if (warp == 0) {
@@ -243,58 +270,109 @@ __global__ void __launch_bounds__(kNnThreads, 1) nn_scan_kernel(const NnParams p
       // nothing may still write tensor memory when it is freed
       if (last >= 0) mbar_wait(d_full(last & 1), (last >> 1) & 1);
     }
-  } else if (warp <= kDecWarps) {
-    // -------------------------------- decode --------------------------------
-    const int dw = warp - 1, grp = dw >> 2, r = 32 * (dw & 3) + lane;
-    const uint32_t row_ofs = (uint32_t)r * 128u;
-    const int rsw = r & 7;
-    uint32_t cur[RW], nxt[RW];
-    float rho_c = 0.f, rho_n = 0.f;
-    auto load = [&](int i, uint32_t (&dst)[RW], float &rho) {
-      const int64_t t = (u0 + i) % p.n_tiles, j = t * kNT + r;
-      if (j < p.n_db) {
-        const uint2 *src = reinterpret_cast<const uint2 *>(p.records + (size_t)j * RW);
-#pragma unroll
-        for (int w = 0; w < RW / 2; ++w) {
-          const uint2 v = __ldg(src + w);
-          dst[2 * w] = v.x;
-          dst[2 * w + 1] = v.y;
-        }
-        rho = __ldg(p.rnorm + j);
-      } else {
-#pragma unroll
-        for (int w = 0; w < RW; ++w) dst[w] = 0u;
-        rho = 0.f;
-      }
-    };
-    if (n_my > 0) load(0, cur, rho_c);
-    for (int i = 0; i < n_my && ok; ++i) {
-      if (i + 1 < n_my) load(i + 1, nxt, rho_n);
-      const __half hn = __float2half_rn(-rho_c * p.kappa);
-      const uint32_t nb = (uint32_t)__half_as_ushort(hn) * 0x00010001u;
-#pragma unroll
-      for (int kc = 0; kc < NCH; ++kc) {
-        if ((kc & 1) != grp) continue;
-        const int g = NCH * i + kc, s = g % kSlots;
-        if (g >= kSlots && !mbar_wait(b_empty(s), ((g / kSlots) - 1) & 1)) {
+  } else if (warp == 1 + kDecWarps + kEpiWarps) {
+    // ------------------------------ tile copies ------------------------------
+    // records, norms and rnorms of each 128-vector tile; the bytes past the last 16-byte
+    // boundary of a ragged last tile are copied with plain loads before the stage is armed
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < n_my; ++i) {
+        const int e = i % kRStages;
+        if (i >= kRStages && !mbar_wait(r_empty(e), ((i / kRStages) - 1) & 1)) {
           ok = false;
           break;
         }
+        const int64_t j0 = ((u0 + i) % p.n_tiles) * kNT;
+        const uint32_t nv = (uint32_t)min((int64_t)kNT, p.n_db - j0);
+        const uint32_t st = stages + (uint32_t)e * L::kStage;
+        const uint32_t rb = nv * RW * 4, rb16 = rb & ~15u, nb = nv * 4, nb16 = nb & ~15u;
+        const uint32_t *rsrc = p.records + (size_t)j0 * RW;
+        for (uint32_t o = rb16; o < rb; o += 4) asm volatile("st.shared.u32 [%0], %1;" ::"r"(st + o), "r"(__ldg(rsrc + o / 4)) : "memory");
+        for (uint32_t o = nb16; o < nb; o += 4) {
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(st + L::kRecBytes + o), "f"(__ldg(p.norm + j0 + o / 4)) : "memory");
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(st + L::kRecBytes + kNT * 4 + o), "f"(__ldg(p.rnorm + j0 + o / 4))
+                       : "memory");
+        }
+        if (rb16 < rb || nb16 < nb) tc::fence_proxy_async();   // plain stores before later bulk writes here
+        mbar_arrive_expect_tx(r_full(e), rb16 + 2 * nb16);
+        if (rb16) bulk_g2s(st, rsrc, rb16, r_full(e));
+        if (nb16) {
+          bulk_g2s(st + L::kRecBytes, p.norm + j0, nb16, r_full(e));
+          bulk_g2s(st + L::kRecBytes + kNT * 4, p.rnorm + j0, nb16, r_full(e));
+        }
+        ++issued;
+      }
+      // no copy may still be landing when the CTA exits
+      for (int i = max(0, issued - kRStages); i < issued; ++i) mbar_wait(r_full(i % kRStages), (i / kRStages) & 1);
+      if (!ok) atomicOr(p.status, kDevTimeout);
+    }
+  } else if (warp <= kDecWarps) {
+    // -------------------------------- decode --------------------------------
+    // group 0 (warps 1-4) writes the even K chunks, group 1 the odd ones; a thread owns one row
+    // and holds its record in registers while it writes its group's chunks
+    const int dw = warp - 1, grp = dw >> 2, r = 32 * (dw & 3) + lane;
+    const uint32_t row_ofs = (uint32_t)r * 128u;
+    const int rsw = r & 7;
+    uint32_t rec[RW];
+    auto chunks = [&](auto G, int i, uint32_t nbh) {
+      constexpr int kc0 = decltype(G)::value;
+#pragma unroll
+      for (int kc = kc0; kc < NCH; kc += 2) {
+        const int g = NCH * i + kc, s = g % kSlots;
+        if (g >= kSlots && !mbar_wait(b_empty(s), ((g / kSlots) - 1) & 1)) {
+          ok = false;
+          return;
+        }
         const uint32_t dst = ring + (uint32_t)s * kChunk + row_ofs;
 #pragma unroll
-        for (int uu = 0; uu < 8; ++uu) sts128(dst + (uint32_t)((uu ^ rsw) << 4), nn_unit<D, BETA>(cur, 8 * kc + uu, lut, nb));
+        for (int uu = 0; uu < 8; ++uu)
+          sts128(dst + (uint32_t)((uu ^ rsw) << 4), nn_unit_reg<D, BETA>(rec, 8 * kc + uu, lut, nbh));
         tc::fence_proxy_async();   // generic stores -> tensor-core reads
         __syncwarp();
         if (lane == 0) mbar_arrive(b_full(s));
       }
+    };
+    for (int i = 0; i < n_my && ok; ++i) {
+      const int e = i % kRStages;
+      if (!mbar_wait(r_full(e), (i / kRStages) & 1)) {
+        ok = false;
+        break;
+      }
+      const uint32_t st = stages + (uint32_t)e * L::kStage;
+      const uint32_t rs = st + (uint32_t)r * RW * 4;
 #pragma unroll
-      for (int w = 0; w < RW; ++w) cur[w] = nxt[w];
-      rho_c = rho_n;
+      for (int w = 0; w < RW / 2; ++w) {
+        const uint2 v = lds64(rs + 8u * w);
+        rec[2 * w] = v.x;
+        rec[2 * w + 1] = v.y;
+      }
+      const bool valid = ((u0 + i) % p.n_tiles) * kNT + r < p.n_db;   // rows past the database: ignored columns
+      const float nrm = valid ? lds_f32(st + L::kRecBytes + 4u * r) : __int_as_float(0x7fc00000);
+      const float rho = valid ? lds_f32(st + L::kRecBytes + kNT * 4 + 4u * r) : 0.f;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(r_empty(e));   // the stage is in registers: the copy may refill it
+      if (grp == 0) {
+        // the tile's norms for the epilogue (its entry of the ring is free once tile i - 4 is scored)
+        const int ne = i % kNrmRing;
+        if (i >= kNrmRing && !mbar_wait(n_empty(ne), ((i / kNrmRing) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        nrm_s[ne * kNT + r] = nrm;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(n_full(ne));
+      }
+      const uint32_t nbh = (uint32_t)__half_as_ushort(__float2half_rn(-rho * p.kappa)) * 0x00010001u;
+      if (grp == 0)
+        chunks(std::integral_constant<int, 0>{}, i, nbh);
+      else
+        chunks(std::integral_constant<int, 1>{}, i, nbh);
     }
     if (!ok) atomicOr(p.status, kDevTimeout);
   } else {
     // ------------------------------- epilogue -------------------------------
-    const int q4 = warp & 3, r = 32 * q4 + lane;
+    const int ew = warp - 1 - kDecWarps, q4 = warp & 3, hh = ew >> 2, r = 32 * q4 + lane;
+    constexpr int kCols = kNT / kLists;   // columns of each tile this warp scores
     const uint32_t lane_ofs = (uint32_t)(32 * q4) << 16;
     float sv[kNnMaxK], sig = 1.f;
     int si[kNnMaxK];
@@ -306,13 +384,40 @@ __global__ void __launch_bounds__(kNnThreads, 1) nn_scan_kernel(const NnParams p
       }
     };
     auto flush = [&](int64_t qb) {
-      const size_t base = ((size_t)(blockIdx.x + qb) * kQB + r) * kNnMaxK;
+      const size_t base = (((size_t)(blockIdx.x + qb) * kQB + r) * 2 + hh) * kNnMaxK;
 #pragma unroll
       for (int j = 0; j < kNnMaxK; ++j)
         if (j >= kNnMaxK - p.k) {
           p.part_s[base + j - (kNnMaxK - p.k)] = sv[j] * sig;
           p.part_i[base + j - (kNnMaxK - p.k)] = si[j];
         }
+    };
+    // score 16 columns (accumulators in `acc`, norms from the staged tile) against the running list
+    auto score16 = [&](uint32_t (&acc)[16], const float4 *nr4, int jc) {
+      const float thr = sv[kNnMaxK - 1];
+      uint32_t hit = 0;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const float4 n4 = nr4[c4];   // same address in every lane: one broadcast
+        const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float v = __uint_as_float(acc[4 * c4 + c]) * nn[c];
+          acc[4 * c4 + c] = __float_as_uint(v);   // the score replaces the accumulator
+          hit |= (v > thr ? 1u : 0u) << (4 * c4 + c);
+        }
+      }
+      // columns above the running k-th score, inserted in column order
+      while (hit) {
+        const int c = __ffs(hit) - 1;
+        hit &= hit - 1;
+        uint32_t vb = acc[0];
+#pragma unroll
+        for (int m = 1; m < 16; ++m)
+          if (m == c) vb = acc[m];
+        const float v = __uint_as_float(vb);
+        if (v > sv[kNnMaxK - 1]) topk_insert(sv, si, v, jc + c);
+      }
     };
     reset();
     int64_t prev_qb = -1;
@@ -327,72 +432,49 @@ __global__ void __launch_bounds__(kNnThreads, 1) nn_scan_kernel(const NnParams p
         prev_qb = qb;
         const size_t row = (size_t)qb * kQB + r;
         sig = __ldg(p.sigma + row);
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.qimg + row * Dm::KP);
+        // this warp's share of the row: columns [hh ACOLS / kLists, (hh + 1) ACOLS / kLists)
+        constexpr int kAc = Dm::ACOLS / kLists;
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.qimg + row * Dm::KP + hh * 2 * kAc);
 #pragma unroll 2
-        for (int c = 0; c < Dm::ACOLS; c += 8) {
+        for (int c = 0; c < kAc; c += 8) {
           const uint4 a = __ldg(src + c / 4), b = __ldg(src + c / 4 + 1);
           const uint32_t v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-          tc::st8(tmem + lane_ofs + c, v);
+          tc::st8(tmem + lane_ofs + hh * kAc + c, v);
         }
         tc::wait_st();
         tc::fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(a_full);
       }
-      const int b = i & 1;
-      if (!mbar_wait(d_full(b), (i >> 1) & 1)) {
+      const int b = i & 1, ne = i % kNrmRing;
+      if (!mbar_wait(d_full(b), (i >> 1) & 1) || !mbar_wait(n_full(ne), (i / kNrmRing) & 1)) {
         ok = false;
         break;
       }
       tc::fence_after();
-      const int64_t j0 = t * kNT;
-      const uint32_t ta = tmem + lane_ofs + kAcc0 + kNT * b;
+      const int j0 = (int)(t * kNT) + kCols * hh;
+      const uint32_t ta = tmem + lane_ofs + kAcc0 + kNT * b + kCols * hh;
+      const float4 *nr4 = reinterpret_cast<const float4 *>(nrm_s + ne * kNT + kCols * hh);
+      // two 16-column groups per pass: the second is loaded from tensor memory while the first is scored
+      uint32_t acc0[16], acc1[16];
+      tc::ld16(ta, acc0);
+      tc::wait_ld();
 #pragma unroll 1
-      for (int g = 0; g < kNT / 16; ++g) {
-        const int c0 = 16 * g;
-        const int64_t jc = j0 + c0;
-        float nv[16];
-        if (jc + 16 <= p.n_db) {
-          const float4 *np4 = reinterpret_cast<const float4 *>(p.norm + jc);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const float4 v = __ldg(np4 + c);
-            nv[4 * c] = v.x;
-            nv[4 * c + 1] = v.y;
-            nv[4 * c + 2] = v.z;
-            nv[4 * c + 3] = v.w;
-          }
-        } else {
-          // past the database: NaN scores are never inserted
-#pragma unroll
-          for (int c = 0; c < 16; ++c) nv[c] = jc + c < p.n_db ? __ldg(p.norm + jc + c) : __int_as_float(0x7fc00000);
-        }
-        uint32_t acc[16];
+      for (int g = 0; g < kCols / 16; g += 2) {
+        tc::ld16(ta + 16 * (g + 1), acc1);
+        score16(acc0, nr4 + 4 * g, j0 + 16 * g);
         __syncwarp();
-        tc::ld16(ta + 16 * g, acc);
         tc::wait_ld();
-        if (g == kNT / 16 - 1) {
-          tc::fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(d_empty(b));   // the accumulator is in registers
-        }
-        // columns above the running k-th score, then inserted in column order (one insert site)
-        float vv[16];
-        uint32_t hit = 0;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          vv[c] = __uint_as_float(acc[c]) * nv[c];
-          hit |= (vv[c] > sv[kNnMaxK - 1] ? 1u : 0u) << c;
-        }
-        while (hit) {
-          const int c = __ffs(hit) - 1;
-          hit &= hit - 1;
-          float v = vv[0];
-#pragma unroll
-          for (int m = 1; m < 16; ++m)
-            if (m == c) v = vv[m];
-          if (v > sv[kNnMaxK - 1]) topk_insert(sv, si, v, (int)(jc + c));
-        }
+        if (g + 2 < kCols / 16) tc::ld16(ta + 16 * (g + 2), acc0);
+        score16(acc1, nr4 + 4 * (g + 1), j0 + 16 * (g + 1));
+        __syncwarp();
+        if (g + 2 < kCols / 16) tc::wait_ld();
+      }
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(d_empty(b));    // the accumulator has been read
+        mbar_arrive(n_empty(ne));   // and the norms
       }
     }
     if (ok && prev_qb >= 0) flush(prev_qb);
@@ -486,8 +568,8 @@ __global__ void __launch_bounds__(128) nn_merge_kernel(const float *__restrict__
     const int64_t c0 = units * c / grid, c1 = units * (c + 1) / grid;
     if (c0 >= hi) break;
     if (c1 <= lo || c0 == c1) continue;
-    {
-      const size_t base = ((size_t)(c + qb) * kQB + r) * kNnMaxK;
+    for (int hh = 0; hh < kLists; ++hh) {
+      const size_t base = (((size_t)(c + qb) * kQB + r) * 2 + hh) * kNnMaxK;
       for (int j = 0; j < k; ++j) {
         float v = part_s[base + j];
         int id = part_i[base + j];
@@ -517,7 +599,7 @@ __global__ void __launch_bounds__(128) nn_merge_kernel(const float *__restrict__
 template <int D, int BETA>
 cudaError_t launch_scan(const NnParams &p, int grid, cudaStream_t st) {
   auto kern = nn_scan_kernel<D, BETA>;
-  const size_t smem = NnSmem<BETA>::kBytes;
+  const size_t smem = NnSmem<D, BETA>::kBytes;
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
   return launch_after(kern, dim3((unsigned)grid), dim3(kNnThreads), smem, st, p);

@@ -556,7 +556,8 @@ tq_status tq_decode_attend(const tq_cache *k, const tq_cache *v, const float *q,
 }
 
 // Workspace of tq_nn_search: header | fp16 query rows | per-query scale | partial top-k lists
-// (one per (CTA, query block) pair a CTA's contiguous unit range touches: grid + blocks - 1).
+// (two per row for each (CTA, query block) pair a CTA's contiguous unit range touches:
+// grid + blocks - 1 pairs).
 struct NnWs {
   size_t qimg, sigma, part_s, part_i, total;
 };
@@ -570,8 +571,8 @@ NnWs nn_ws(int d, int n_queries, int64_t n_db) {
   w.qimg = kWsHeader;
   w.sigma = w.qimg + up((size_t)n_qb * 128 * nn_kp(d) * 2);
   w.part_s = w.sigma + up((size_t)n_qb * 128 * sizeof(float));
-  w.part_i = w.part_s + up((size_t)slots * 128 * kNnMaxK * sizeof(float));
-  w.total = w.part_i + up((size_t)slots * 128 * kNnMaxK * sizeof(int));
+  w.part_i = w.part_s + up((size_t)slots * 128 * 2 * kNnMaxK * sizeof(float));
+  w.total = w.part_i + up((size_t)slots * 128 * 2 * kNnMaxK * sizeof(int));
   return w;
 }
 
@@ -602,8 +603,8 @@ tq_status tq_nn_search(const tq_cache *db, const float *queries, int32_t n_queri
   if (n_queries == 0) return TQ_OK;
   if (!queries || !Pi || !S || !codebook || !top_scores || !top_ids)
     return fail(TQ_ERR_INVALID, "tq_nn_search: NULL tensor argument");
-  if (!aligned(Pi, 16) || !aligned(S, 16) || !aligned(db->norm, 16))
-    return fail(TQ_ERR_INVALID, "tq_nn_search: Pi, S and the database norms must be 16-byte aligned");
+  if (!aligned(Pi, 16) || !aligned(S, 16) || !aligned(db->norm, 16) || !aligned(db->rnorm, 16))
+    return fail(TQ_ERR_INVALID, "tq_nn_search: Pi, S and the database norm and rnorm arrays must be 16-byte aligned");
   const NnWs w = nn_ws(db->d, n_queries, n_db);
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.total)
     return fail(TQ_ERR_WORKSPACE, "tq_nn_search: workspace needs %zu bytes, 256-byte aligned (got %zu)", w.total,

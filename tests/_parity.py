@@ -101,11 +101,20 @@ def check_attend(gpu, lg, scale, Pi, codebook, rec, norm, d, bits):
     return float(np.max(err) / tol) if err.size else 0.0
 
 
+def nn_scores(q, Pi, S, codebook, rec, norm, rnorm, d, bits, rows=100_000):
+    """Oracle estimator scores [nq, n_db] of queries q over a packed database, unpacked in row blocks."""
+    n_db = rec.shape[0]
+    ref = np.empty((np.asarray(q).shape[0], n_db), dtype=np.float64)
+    for a in range(0, n_db, rows):
+        gi, gs = otq.unpack(rec[a:a + rows], d, bits, True)
+        ref[:, a:a + rows] = otq.logits(q, Pi, S, codebook, norm[a:a + rows], rnorm[a:a + rows], gi, gs)
+    return ref
+
+
 def check_nn(gpu_s, gpu_i, q, Pi, S, codebook, rec, norm, rnorm, d, bits, k):
     """gpu_s/gpu_i: [nq, k] top-k scores and ids; q: [nq, d]; rec/norm/rnorm: the GPU's database
     cache (already checked against the oracle's encoding). Returns the worst error / tolerance."""
-    gi, gs = otq.unpack(rec, d, bits, True)
-    ref = otq.logits(q, Pi, S, codebook, norm, rnorm, gi, gs)          # [nq, n_db] float64
+    ref = nn_scores(q, Pi, S, codebook, rec, norm, rnorm, d, bits)   # [nq, n_db] float64
     n_db = ref.shape[1]
     kk = min(k, n_db)
     gpu_s = np.asarray(gpu_s, dtype=np.float64)

@@ -165,14 +165,15 @@ def test_nn_search_argument_checks():
     assert call(db, nq=0) == tqb.TQ_OK                                                    # nothing to do
     assert call(db, q=None) == tqb.TQ_ERR_INVALID
     assert call(db, Pi=FAKE + 4) == tqb.TQ_ERR_INVALID                                    # float4 rows
-    assert call(_desc(d=200, bits=1, heads=1, norm=FAKE + 4100)) == tqb.TQ_ERR_INVALID     # float4 norms
+    assert call(_desc(d=200, bits=1, heads=1, norm=FAKE + 4100)) == tqb.TQ_ERR_INVALID     # bulk-copied norms
+    assert call(_desc(d=200, bits=1, heads=1, rnorm=FAKE + 8196)) == tqb.TQ_ERR_INVALID
     assert call(db, ws_bytes=1024) == tqb.TQ_ERR_WORKSPACE
     assert call(db) == tqb.TQ_ERR_CUDA                                                    # passes -> injected
-    # status | fp16 query rows (padded K 448) | scales | (CTAs + blocks - 1) lists of 16 scores and ids
+    # status | fp16 query rows (padded K 448) | scales | 2 lists of 16 scores and ids per row of (CTAs + blocks - 1)
     up = lambda v: (v + 255) // 256 * 256
     nqb, tiles = 3, 1
     slots = min(nqb * tiles, 256) + nqb - 1
-    want = 256 + up(nqb * 128 * 448 * 2) + up(nqb * 128 * 4) + 2 * up(slots * 128 * 16 * 4)
+    want = 256 + up(nqb * 128 * 448 * 2) + up(nqb * 128 * 4) + 2 * up(slots * 128 * 2 * 16 * 4)
     assert lib.tq_nn_workspace_size(ctypes.byref(db), 300, 40) == want
     assert lib.tq_nn_workspace_size(ctypes.byref(db), 300, 0) == 256 + up(nqb * 128 * 448 * 2) + up(nqb * 128 * 4)
 

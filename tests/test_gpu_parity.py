@@ -357,6 +357,29 @@ def test_nn_search_parity(d, bits, n_db, n_q, k):
     par.check_nn(sc, ids, qs.numpy(), Pi, S, ck, rec, norm, rnorm, d, bits, k)
 
 
+@pytest.mark.parametrize("bits", [1, 3])
+def test_nn_search_full_size_sampled(bits):
+    # the nearest-neighbour workload bench.py times (10^6 x d = 200 database, 10^4 queries, top-10):
+    # the encoding on 20000 sampled database rows, the top-10 of 12 sampled queries over all rows
+    d, N, Q, k = 200, 1_000_000, 10_000, 10
+    db, qs = syn.nn_inputs(N, Q, d, device="cuda")
+    Pi, S, ck, _, g = _setup(d, bits, 1)
+    cache = tqb.PackedCache.empty(d, bits, True, 1, 1, N)
+    tqb.tq_quantize_append(cache, db.reshape(1, 1, N, d), 0, g["Pi"], g["SPiT"], g["ck"])
+    ws = torch.empty(tqb.tq_nn_workspace_size(cache, Q, N), dtype=torch.uint8, device="cuda")
+    sc, ids = tqb.tq_nn_search(cache, qs, N, g["Pi"], g["S"], g["ck"], k, workspace=ws)
+    torch.cuda.synchronize()
+    tqb.tq_workspace_status(ws)
+    rec = par.as_u32(cache.records[0, 0].cpu().numpy())
+    norm = cache.norm[0, 0].cpu().numpy()
+    rnorm = cache.rnorm[0, 0].cpu().numpy()
+    rows = np.random.default_rng(3).choice(N, 20000, replace=False)
+    par.check_encoding(db[rows].cpu().numpy(), rec[rows], norm[rows], rnorm[rows], Pi, S, ck, d, bits, True)
+    qi = np.random.default_rng(4).choice(Q, 12, replace=False)
+    par.check_nn(sc[qi].cpu().numpy(), ids[qi].cpu().numpy(), qs[qi].cpu().numpy(), Pi, S, ck, rec, norm, rnorm,
+                 d, bits, k)
+
+
 @pytest.mark.parametrize("n_db", [0, 1, 5])
 def test_nn_search_fewer_vectors_than_k(n_db):
     db, qs, Pi, S, ck, rec, norm, rnorm, sc, ids = _nn_case(200, 1, n_db, 130, 10, capacity=64)
