@@ -395,7 +395,7 @@ __global__ void __launch_bounds__(kNnThreads, 1) nn_scan_kernel(const NnParams p
     // score 16 columns (accumulators in `acc`, norms from the staged tile) against the running list
     auto score16 = [&](uint32_t (&acc)[16], const float4 *nr4, int jc) {
       const float thr = sv[kNnMaxK - 1];
-      uint32_t hit = 0;
+      float mx = -INFINITY;
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
         const float4 n4 = nr4[c4];   // same address in every lane: one broadcast
@@ -404,9 +404,13 @@ __global__ void __launch_bounds__(kNnThreads, 1) nn_scan_kernel(const NnParams p
         for (int c = 0; c < 4; ++c) {
           const float v = __uint_as_float(acc[4 * c4 + c]) * nn[c];
           acc[4 * c4 + c] = __float_as_uint(v);   // the score replaces the accumulator
-          hit |= (v > thr ? 1u : 0u) << (4 * c4 + c);
+          mx = fmaxf(mx, v);                       // NaN (past the database) is dropped
         }
       }
+      if (!(mx > thr)) return;   // the common case once the list has filled
+      uint32_t hit = 0;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) hit |= (__uint_as_float(acc[c]) > thr ? 1u : 0u) << c;
       // columns above the running k-th score, inserted in column order
       while (hit) {
         const int c = __ffs(hit) - 1;
