@@ -56,6 +56,8 @@ NCU_TRAFFIC = {
     ("logits", "llama"): 15_756_288 + 0,               # logits_gqa_kernel<2, 4> (the scan; tables read from L2)
     ("attend_v", "llama"): 17_871_872 + 0,             # attend_fast_kernel<3, 4> (records, norms and logits)
     ("decode_attend", "sweep-b3"): 2 * (453_061_376 + 5_822_720),   # decode_fused_kernel<2, 3>, 4-sequence capture x 2
+    ("nn_search", "nn-b2-s"): 15_584_768 + 512,                    # nn_scan_kernel<200, 1> (the full size is not
+                                                                   # proportional: its database stays in L2)
 }
 
 
@@ -67,7 +69,7 @@ def parse():
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--workload", default="llama",
                     choices=["llama"] + [f"sweep-b{b}{s}" for b in (2, 3, 4) for s in ("", "-s4")]
-                    + ["large-b3", "large-b4", "nn-b2", "nn-b4"])
+                    + ["large-b3", "large-b4", "nn-b2", "nn-b4", "nn-b2-s", "nn-b4-s"])
     ap.add_argument("--layers", type=int, default=80, help="layers streamed by the large-model workload")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -80,12 +82,14 @@ def parse():
 
 def workload(name: str):
     if name.startswith("nn"):
+        # "nn-b2" is the full search; "nn-b2-s" keeps 10^5 of the 10^6 database vectors (a profiling size)
         b = int(name.split("-")[1][1:])
-        return dict(kind="nn", name=f"nn-search-b{b}: 1,000,000 database vectors d=200 (unit-normalised anisotropic "
+        n_db = 100_000 if name.endswith("-s") else 1_000_000
+        return dict(kind="nn", name=f"nn-search-b{b}: {n_db:,} database vectors d=200 (unit-normalised anisotropic "
                                     f"Gaussian, per-dimension std U[0.2, 2]), 10,000 queries of the same law, b={b} "
                                     f"({b - 1}-bit codes + QJL), top-10 by the key estimator; a synthetic stand-in "
                                     f"for the GloVe-200 benchmark",
-                    n_db=1_000_000, n_q=10_000, d=200, k_idx=b - 1, k=10)
+                    n_db=n_db, n_q=10_000, d=200, k_idx=b - 1, k=10)
     if name == "llama":
         return dict(name="llama3-8b-decode: B=1 Hq=32 Hkv=8 d=128 T=32768 bf16 K b=3 (2-bit codes+QJL) V b=3 MSE",
                     n_seq=1, hq=32, hkv=8, d=128, T=32768, k_idx=2, v_idx=3, dtype=torch.bfloat16,
