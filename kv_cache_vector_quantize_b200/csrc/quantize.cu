@@ -271,6 +271,7 @@ cudaError_t launch_quantize(const QuantParams &p, int bits, bool qjl, tq_dtype d
   if (p.d <= 32) return launch_q_dp<32>(p, bits, qjl, dtype, st);
   if (p.d <= 64) return launch_q_dp<64>(p, bits, qjl, dtype, st);
   if (p.d <= 128) return launch_q_dp<128>(p, bits, qjl, dtype, st);
+  if (p.d <= 224) return launch_q_dp<224>(p, bits, qjl, dtype, st);   // d = 200: 23% fewer products than 256
   return launch_q_dp<256>(p, bits, qjl, dtype, st);
 }
 

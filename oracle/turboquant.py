@@ -221,6 +221,31 @@ def attend_v(lg, scale, v_norm, v_idx, Pi, codebook_v):
     return acc @ Pi                                 # Pi^T acc, row by row
 
 
+def walsh_hadamard(x):
+    """Unnormalised fast Walsh-Hadamard transform over the last axis (length a power of two):
+    returns x H with H the Sylvester-Hadamard matrix, by log2(d) rounds of pairwise sums and
+    differences. The structured rotation the pages' "O(d) per vector" cost refers to
+    ([W] "1. PolarQuant"; a Hadamard product costs O(d log d)) is Pi = H diag(s) / sqrt(d)."""
+    y = np.array(x, dtype=np.float64, copy=True)
+    d = y.shape[-1]
+    if d < 1 or d & (d - 1):
+        raise ValueError(f"length {d} is not a power of two")
+    h = 1
+    while h < d:
+        y = y.reshape(y.shape[:-1] + (d // (2 * h), 2, h))
+        a, b = y[..., 0, :].copy(), y[..., 1, :].copy()
+        y[..., 0, :], y[..., 1, :] = a + b, a - b
+        y = y.reshape(y.shape[:-3] + (d,))
+        h *= 2
+    return y
+
+
+def structured_rotate(u, signs):
+    """Rows of u rotated by Pi = H diag(signs) / sqrt(d): (Pi u_row) = H (signs * u_row) / sqrt(d)."""
+    u = np.asarray(u, dtype=np.float64)
+    return walsh_hadamard(u * np.asarray(signs, dtype=np.float64)) / math.sqrt(u.shape[-1])
+
+
 def kv_head_of(q_head: int, n_q_heads: int, n_kv_heads: int) -> int:
     """Contiguous grouped-query mapping (reading; winningdata.io, "Limitacoes e trade-offs"
     leaves GQA open)."""

@@ -146,6 +146,27 @@ def test_shapes_parity(shape):
     _check_all(k, v, q, d, kb, vb, Pi, S, ck, cv, kc, vc, lg, out, sc)
 
 
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float32])
+def test_structured_rotation_full_path(dt):
+    # a randomized Hadamard rotation H diag(s) / sqrt(d) as the rotation input: quantize (tensor-core
+    # path for bf16, FP32 path for fp32), logits, softmax.V and the one-call decode step against the
+    # oracle on the same matrix
+    d, kb, vb, B, H, G, T = 128, 2, 3, 1, 2, 4, 777
+    k = syn.gaussian((B, H, T, d), 51).to(dt)
+    v = syn.lognormal_sphere((B, H, T, d), 52, dtype=dt)
+    q = syn.gaussian((B, H * G, d), 53)
+    Pi_t, S_t = syn.randomized_hadamard(d), syn.sketch(d)
+    ck, cv = _codebook(d, kb), _codebook(d, vb)
+    dev = torch.device("cuda")
+    g = dict(Pi=Pi_t.to(dev), S=S_t.to(dev), ck=torch.from_numpy(ck).to(dev), cv=torch.from_numpy(cv).to(dev))
+    g["SPiT"] = tqb.tq_sketch_rotation(g["Pi"], g["S"])
+    kc, vc, lg, out, sc = _run_path(k, v, q, d, kb, vb, g)
+    _check_all(k, v, q, d, kb, vb, Pi_t.numpy(), S_t.numpy(), ck, cv, kc, vc, lg, out, sc)
+    out_d = tqb.tq_decode_attend(kc, vc, q.cuda(), T, sc, g["Pi"], g["S"], g["ck"], g["cv"])
+    torch.cuda.synchronize()
+    assert torch.equal(out_d, out)
+
+
 def test_append_in_parts_equals_one_call():
     d, kb, T = 128, 2, 700
     k = syn.gaussian((2, 2, T, d), 41).to(torch.bfloat16).cuda()

@@ -37,6 +37,19 @@ def rotation(d: int, seed: int = SEED_PI) -> torch.Tensor:
     return q.to(torch.float32).contiguous()
 
 
+def randomized_hadamard(d: int, seed: int = SEED_PI) -> torch.Tensor:
+    """Structured orthogonal d x d matrix H diag(s) / sqrt(d): H the Sylvester-Hadamard matrix
+    (H_1 = [1], H_2m = [[H_m, H_m], [H_m, -H_m]]), s seeded random signs; d a power of two.
+    Float32 on the CPU; an alternative to `rotation` for the rotation input."""
+    if d < 1 or d & (d - 1):
+        raise ValueError(f"d={d} is not a power of two")
+    h = torch.ones(1, 1, dtype=torch.float64)
+    while h.shape[0] < d:
+        h = torch.cat([torch.cat([h, h], 1), torch.cat([h, -h], 1)], 0)
+    s = torch.where(torch.rand(d, generator=_gen(seed), dtype=torch.float64) < 0.5, -1.0, 1.0)
+    return (h * s[None, :] / d ** 0.5).to(torch.float32).contiguous()
+
+
 def sketch(d: int, seed: int = SEED_S) -> torch.Tensor:
     """d x d matrix with i.i.d. N(0, 1) entries, float32 on the CPU."""
     return torch.randn(d, d, generator=_gen(seed), dtype=torch.float32)
