@@ -56,8 +56,6 @@ NCU_TRAFFIC = {
     ("logits", "llama"): 15_756_288 + 0,               # logits_gqa_kernel<2, 4> (the scan; tables read from L2)
     ("attend_v", "llama"): 17_871_872 + 0,             # attend_fast_kernel<3, 4> (records, norms and logits)
     ("decode_attend", "sweep-b3"): 2 * (453_061_376 + 5_822_720),   # decode_fused_kernel<2, 3>, 4-sequence capture x 2
-    ("nn_search", "nn-b2-s"): 15_584_768 + 512,                    # nn_scan_kernel<200, 1> (the full size is not
-                                                                   # proportional: its database stays in L2)
 }
 
 

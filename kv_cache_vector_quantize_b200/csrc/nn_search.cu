@@ -57,7 +57,11 @@ struct NnLut {
   static constexpr int LB = BETA * CPL;           // code bits per lookup
   static constexpr int ENTRIES = 1 << LB;
   static constexpr int EB = 2 * CPL;              // bytes per entry (fp16 centroids)
-  static constexpr uint32_t BYTES = ENTRIES * EB;
+  // copies of each entry side by side, one per lane of a shared-memory phase (8 lanes of 16-byte
+  // loads, 16 lanes of 8-byte loads): lane l reads copy l mod REP, so a phase never conflicts
+  static constexpr int REP = BETA == 1 ? 8 : BETA == 2 ? 16 : 1;
+  static constexpr uint32_t STRIDE = REP * EB;    // bytes from one entry to the next
+  static constexpr uint32_t BYTES = ENTRIES * STRIDE;
 };
 
 template <int D, int BETA>
@@ -111,11 +115,13 @@ __device__ __forceinline__ uint2 lds64(uint32_t a) {
 }
 
 // B values of 8 consecutive K elements (one 16-byte unit) of a database row whose record is held
-// in registers (`uk` a compile-time constant after unrolling, so every word index is too). Units
-// [0, D/8) hold centroids c[idx] of coordinates 8 uk .. 8 uk + 7 (one lookup of 8, or two of 4,
-// consecutive codes), units [D/8, D/4) the signed sketch weights rho kappa (2 sign - 1): half p of
-// word w takes sign bit 2 w + p into its own sign bit, the product placing bit 2w at bit 15 and bit
-// 2w + 1 at bit 31 without overlapping terms. The rest is zero padding. `nb` = fp16x2 of -rho kappa.
+// in registers (`uk` a compile-time constant after unrolling, so every word index is too).
+//   * Units [0, D/8): centroids c[idx] of coordinates 8 uk .. 8 uk + 7, by one lookup of 8 or two
+//     of 4 consecutive codes (`lut` points at this lane's copy of the table).
+//   * Units [D/8, D/4): the signed sketch weights rho kappa (2 sign - 1). Half p of word w takes
+//     sign bit 2 w + p into its own sign bit: the product places bit 2w at bit 15 and bit 2w + 1 at
+//     bit 31 without overlapping terms; `nb` = fp16x2 of -rho kappa.
+//   * The rest: zero padding.
 template <int D, int BETA>
 __device__ __forceinline__ uint4 nn_unit_reg(const uint32_t *rec, int uk, uint32_t lut, uint32_t nb) {
   using R = NnRec<D, BETA>;
@@ -123,14 +129,14 @@ __device__ __forceinline__ uint4 nn_unit_reg(const uint32_t *rec, int uk, uint32
   if (uk < U8) {
     const int bit = 8 * BETA * uk, w = bit >> 5, sh = bit & 31;
     if constexpr (BETA == 1) {
-      return lds_u128(lut + 16u * ((rec[w] >> sh) & 0xFFu));
+      return lds_u128(lut + NnLut<1>::STRIDE * ((rec[w] >> sh) & 0xFFu));
     } else if constexpr (BETA == 2) {
       const uint32_t f = (rec[w] >> sh) & 0xFFFFu;
-      const uint2 a = lds64(lut + 8u * (f & 0xFFu)), b = lds64(lut + 8u * (f >> 8));
+      const uint2 a = lds64(lut + NnLut<2>::STRIDE * (f & 0xFFu)), b = lds64(lut + NnLut<2>::STRIDE * (f >> 8));
       return make_uint4(a.x, a.y, b.x, b.y);
     } else {
       const uint32_t f = (sh > 8 ? __funnelshift_r(rec[w], rec[w + 1], sh) : rec[w] >> sh) & 0xFFFFFFu;
-      const uint2 a = lds64(lut + 8u * (f & 0xFFFu)), b = lds64(lut + 8u * (f >> 12));
+      const uint2 a = lds64(lut + NnLut<3>::STRIDE * (f & 0xFFFu)), b = lds64(lut + NnLut<3>::STRIDE * (f >> 12));
       return make_uint4(a.x, a.y, b.x, b.y);
     }
   } else if (uk < 2 * U8) {
@@ -223,10 +229,13 @@ __global__ void __launch_bounds__(kNnThreads, 1) nn_scan_kernel(const NnParams p
       const float hi = __ldg(p.codebook + ((e >> (BETA * (2 * c2 + 1))) & ((1 << BETA) - 1)));
       wv[c2] = (uint32_t)__half_as_ushort(__float2half_rn(lo)) | ((uint32_t)__half_as_ushort(__float2half_rn(hi)) << 16);
     }
-    if constexpr (Lu::CPL == 8)
-      *reinterpret_cast<uint4 *>(smem + L::kLut + 16 * e) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-    else
-      *reinterpret_cast<uint2 *>(smem + L::kLut + 8 * e) = make_uint2(wv[0], wv[1]);
+#pragma unroll 1
+    for (int c = 0; c < Lu::REP; ++c) {
+      if constexpr (Lu::CPL == 8)
+        *reinterpret_cast<uint4 *>(smem + L::kLut + Lu::STRIDE * e + 16 * c) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      else
+        *reinterpret_cast<uint2 *>(smem + L::kLut + Lu::STRIDE * e + 8 * c) = make_uint2(wv[0], wv[1]);
+    }
   }
   tc::fence_before();
   __syncthreads();
@@ -313,6 +322,7 @@ __global__ void __launch_bounds__(kNnThreads, 1) nn_scan_kernel(const NnParams p
     const int dw = warp - 1, grp = dw >> 2, r = 32 * (dw & 3) + lane;
     const uint32_t row_ofs = (uint32_t)r * 128u;
     const int rsw = r & 7;
+    const uint32_t lut_l = lut + (uint32_t)(lane & (Lu::REP - 1)) * Lu::EB;   // this lane's copy of the table
     uint32_t rec[RW];
     auto chunks = [&](auto G, int i, uint32_t nbh) {
       constexpr int kc0 = decltype(G)::value;
@@ -326,7 +336,7 @@ __global__ void __launch_bounds__(kNnThreads, 1) nn_scan_kernel(const NnParams p
         const uint32_t dst = ring + (uint32_t)s * kChunk + row_ofs;
 #pragma unroll
         for (int uu = 0; uu < 8; ++uu)
-          sts128(dst + (uint32_t)((uu ^ rsw) << 4), nn_unit_reg<D, BETA>(rec, 8 * kc + uu, lut, nbh));
+          sts128(dst + (uint32_t)((uu ^ rsw) << 4), nn_unit_reg<D, BETA>(rec, 8 * kc + uu, lut_l, nbh));
         tc::fence_proxy_async();   // generic stores -> tensor-core reads
         __syncwarp();
         if (lane == 0) mbar_arrive(b_full(s));

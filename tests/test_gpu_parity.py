@@ -401,6 +401,25 @@ def test_nn_search_full_size_sampled(bits):
                  d, bits, k)
 
 
+def test_nn_search_query_scales_and_database_norms():
+    # queries of norm 1e-4 .. 1e4 and zero (the per-query power-of-two scaling of the fp16 operand),
+    # database rows with norms spread over two decades (the norm multiply of the epilogue)
+    d, bits, n_db, k = 200, 2, 3000, 10
+    db, qs = syn.nn_inputs(n_db, 8, d)
+    db = db * torch.exp(torch.linspace(-2.3, 2.3, n_db))[:, None]
+    qs = qs * torch.tensor([1e-4, 1e-2, 1.0, 1.0, 1e2, 1e4, 3e4, 0.0])[:, None]
+    Pi, S, ck, _, g = _setup(d, bits, 1)
+    cache = tqb.PackedCache.empty(d, bits, True, 1, 1, n_db)
+    tqb.tq_quantize_append(cache, db.reshape(1, 1, n_db, d).cuda(), 0, g["Pi"], g["SPiT"], g["ck"])
+    sc, ids = tqb.tq_nn_search(cache, qs.cuda(), n_db, g["Pi"], g["S"], g["ck"], k)
+    torch.cuda.synchronize()
+    rec = par.as_u32(cache.records[0, 0].cpu().numpy())
+    norm, rnorm = cache.norm[0, 0].cpu().numpy(), cache.rnorm[0, 0].cpu().numpy()
+    par.check_nn(sc.cpu().numpy(), ids.cpu().numpy(), qs.double().numpy(), Pi, S, ck, rec, norm, rnorm, d, bits, k)
+    # the zero query scores every vector 0: the k lowest indices, in order
+    assert np.array_equal(ids[7].cpu().numpy(), np.arange(k)) and torch.all(sc[7] == 0).item()
+
+
 @pytest.mark.parametrize("n_db", [0, 1, 5])
 def test_nn_search_fewer_vectors_than_k(n_db):
     db, qs, Pi, S, ck, rec, norm, rnorm, sc, ids = _nn_case(200, 1, n_db, 130, 10, capacity=64)
