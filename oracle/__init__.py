@@ -29,9 +29,11 @@ readings taken where they are silent are listed in the module docstrings and
 marked "reading:".
 
 Parity status: every function here is pinned by tests under ``tests/`` that
-use closed forms, textbook special cases, brute force or Monte Carlo -- except
-``nn_topk`` (top-k ordering convention only; pinned against a brute-force
-sort) -- see the individual docstrings.
+use closed forms, textbook special cases, an independently tabulated codebook
+and MSE table at finite d, brute force or Monte Carlo. ``turboquant.topk`` is an
+ordering convention (largest first, equal scores by lower index), pinned by a
+hand-worked case; ``turboquant.padding_is_zero`` is pinned by planting a stray
+bit at every unused position of a record.
 """
 
 from . import codebook, turboquant  # noqa: F401

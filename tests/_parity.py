@@ -1,9 +1,10 @@
 """Comparison of the CUDA path's packed cache, logits and outputs with the oracle.
 
 Tolerances (stated by the task for this method):
-  * codes and sign bits bit-exact, except a coordinate whose rotated value lies
-    within 1e-5 of a codebook threshold (|y_i - t_j| <= 1e-5 with ||u|| = 1 and
-    ||Pi_i|| = 1), or whose sketch value lies within 1e-5 ||S_i|| rho of zero;
+  * codes and sign bits bit-exact, except a code that moved exactly one cell across
+    the threshold t_j between its two cells while the rotated value lies within 1e-5
+    of that threshold (|y_i - t_j| <= 1e-5 with ||u|| = 1 and ||Pi_i|| = 1), or a sign
+    whose sketch value lies within 1e-5 ||S_i|| rho of zero;
     such excused flips must be at most 1e-4 of all coordinates;
   * norms (||x|| and rho) to 1e-5 relative;
   * logits to 2e-3 * ||q|| * n_t, with the oracle evaluated on the GPU's cache;
@@ -50,11 +51,17 @@ def check_encoding(x, rec, norm, rnorm, Pi, S, codebook, d, bits, qjl):
     assert not bad.any(), f"norm mismatch at rows {np.nonzero(bad)[0][:10]}: {norm[bad][:5]} vs {ref_n[bad][:5]}"
     gi, gs = otq.unpack(rec, d, bits, qjl)
     t = otq.thresholds_of(c)
-    dist = np.min(np.abs(enc["y"][:, :, None] - t[None, None, :]), axis=2)
-    idiff = gi != enc["idx"]
-    unexcused = idiff & (dist > FLIP_BAND)
+    oi = enc["idx"]
+    idiff = gi != oi
+    # An excused code moved exactly one cell, across the threshold between the two cells
+    # (t_j between cells j and j + 1), and y_i lies within the band of that threshold.
+    one_cell = np.abs(gi - oi) == 1
+    between = t[np.clip(np.minimum(gi, oi), 0, len(t) - 1)] if len(t) else np.zeros_like(enc["y"])
+    near = np.abs(enc["y"] - between) <= FLIP_BAND
+    unexcused = idiff & ~(one_cell & near)
     assert not unexcused.any(), (
-        f"{unexcused.sum()} code mismatches outside the threshold band; first at "
+        f"{unexcused.sum()} code mismatches that are not one-cell moves across a threshold within the band; "
+        f"first at "
         f"{np.argwhere(unexcused)[:5].tolist()} y={enc['y'][unexcused][:5]} gpu={gi[unexcused][:5]} "
         f"oracle={enc['idx'][unexcused][:5]}")
     out = {"coords": n * d, "index_flips": int(idiff.sum()), "sign_flips": 0}

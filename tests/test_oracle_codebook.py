@@ -175,3 +175,41 @@ def test_mse_monte_carlo_d128():
     err = np.sum((u - nearest) ** 2, axis=1)
     want = cb.mse_per_vector(d, c)
     assert abs(err.mean() - want) < 4 * err.std() / math.sqrt(n)
+
+
+def _read_finite_d():
+    cents, mses = {}, {}
+    with open(os.path.join(GOLDEN, "beta_lloyd_max_finite_d.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            kind, d, bits, vals = (p.strip() for p in line.split("|"))
+            key = (int(d), int(bits))
+            if kind == "centroids":
+                cents[key] = [float(v) for v in vals.split()]
+            else:
+                mses[key] = float(vals)
+    return cents, mses
+
+
+_CENTS, _MSES = _read_finite_d()
+
+
+@pytest.mark.parametrize("d,bits", sorted(_CENTS))
+def test_finite_d_centroids_match_independent_table(d, bits):
+    # Tabulated to 5 decimals: agreement within half a unit of the last printed place
+    # (plus 1e-6 for the table's own rounding of a value ending in 5).
+    c = cb.lloyd_max(d, bits)
+    pos = c[len(c) // 2:] * math.sqrt(d)
+    want = np.array(_CENTS[(d, bits)])
+    assert pos.shape == want.shape
+    assert np.all(np.abs(pos - want) <= 5e-6 + 1e-6), (pos, want)
+
+
+@pytest.mark.parametrize("d,bits", sorted(_MSES))
+def test_finite_d_mse_matches_independent_table(d, bits):
+    # Tabulated to 6 decimals; the oracle's integral of the fp32-rounded codebook (the one
+    # both quantizers use) and of the float64 fixed point must both round to the table.
+    want = _MSES[(d, bits)]
+    for c in (cb.lloyd_max(d, bits), cb.fit_codebook(d, bits)[0]):
+        assert abs(cb.mse_per_vector(d, c) - want) <= 5e-7 + 1e-9, (cb.mse_per_vector(d, c), want)

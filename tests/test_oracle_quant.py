@@ -257,3 +257,42 @@ def test_mse_only_reconstruction_error_matches_integral():
 def test_topk_orders_ties_by_index():
     s = np.array([[0.5, 0.9, 0.5, 0.9, 0.1]])
     assert tq.topk(s, 3).tolist() == [[1, 3, 0]]
+
+
+def _used_bit_mask(d, bits, qjl):
+    """Which bits of a record carry data, worked out from the layout's definition alone:
+    the index stream's first bits*d bits, then (keys) the sign field's first d bits."""
+    iw = (bits * d + 31) // 32
+    sw = (d + 31) // 32 if qjl else 0
+    used = np.zeros((iw + sw) * 32, dtype=bool)
+    used[:bits * d] = True
+    if qjl:
+        used[iw * 32:iw * 32 + d] = True
+    return used
+
+
+@pytest.mark.parametrize("d,bits,qjl", [(8, 1, True), (8, 3, True), (200, 1, True), (200, 3, True),
+                                        (8, 3, False), (200, 3, False)])
+def test_padding_check_rejects_every_single_stray_bit(d, bits, qjl):
+    # zubnet.ai news, paragraph 2: a record holds the indices and the sign bits and nothing
+    # else, so every other bit must be 0. Plant one stray bit at each unused position (in
+    # the index field's last word and in the sign field's last word) of an otherwise valid
+    # record: the check must fail every time, and pass on a record whose used bits are all 1.
+    rng = np.random.default_rng(d + 10 * bits + int(qjl))
+    idx = rng.integers(0, 1 << bits, size=(1, d))
+    sign = rng.integers(0, 2, size=(1, d)) if qjl else None
+    rec = tq.pack(idx, sign, d, bits, qjl)
+    assert tq.padding_is_zero(rec, d, bits, qjl)
+    used = _used_bit_mask(d, bits, qjl)
+    pad = np.nonzero(~used)[0]
+    assert len(pad) > 0
+    for pos in pad:
+        bad = rec.copy()
+        bad[0, pos // 32] |= np.uint32(1 << (pos % 32))
+        assert not tq.padding_is_zero(bad, d, bits, qjl), f"stray bit {pos} not caught"
+        # also as the second row of a batch (the check covers every row)
+        assert not tq.padding_is_zero(np.concatenate([rec, bad]), d, bits, qjl)
+    full = np.zeros_like(rec)
+    for pos in np.nonzero(used)[0]:
+        full[0, pos // 32] |= np.uint32(1 << (pos % 32))
+    assert tq.padding_is_zero(full, d, bits, qjl)
