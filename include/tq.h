@@ -24,7 +24,7 @@
  *     returns.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and is asynchronous: no entry point synchronises the stream,
- *     except tq_workspace_status, which says so.
+ *     except tq_workspace_status and tq_attend_v_noalloc_status, which say so.
  *   - Arguments are checked on the host before anything is launched; a failed
  *     check launches nothing and returns a status. Launch failures return
  *     TQ_ERR_CUDA. tq_last_error() gives a thread-local message for the last
@@ -136,7 +136,8 @@ tq_status tq_logits(const tq_cache *k, const float *q, int32_t n_q_heads, int64_
                     const float *Pi, const float *S, const float *codebook,
                     float *logits, void *workspace, size_t workspace_bytes, tq_stream stream);
 
-/* Workspace bytes tq_attend_v needs for this value cache, head count and length. */
+/* Workspace bytes tq_attend_v needs for this value cache, head count and length
+ * (SIZE_MAX if that product does not fit a size_t; tq_attend_v then refuses the shape). */
 size_t tq_attend_workspace_size(const tq_cache *v, int32_t n_q_heads, int64_t n_tokens);
 
 /* Softmax-weighted sum of the packed values (zubnet.ai, paragraph 1: the cache
@@ -144,7 +145,8 @@ size_t tq_attend_workspace_size(const tq_cache *v, int32_t n_q_heads, int64_t n_
  *   p = softmax_t(scale * logits[s][h][t]),
  *   out[s][h] = Pi^T sum_t p_t * norm_t * c[code_t]     (rotation undone once).
  *   logits: [n_seq][n_q_heads][n_tokens] float; out: [n_seq][n_q_heads][d] float.
- *   v->qjl must be 0. n_tokens == 0 writes zeros.
+ *   v->qjl must be 0. n_tokens == 0 writes zeros. Shapes with n_seq x n_kv_heads x
+ *   ceil(min(group, 4)-head blocks) above 65535 return TQ_ERR_UNSUPPORTED.
  * workspace: >= tq_attend_workspace_size bytes, 256-byte aligned. */
 tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale,
                       int32_t n_q_heads, int64_t n_tokens,
@@ -234,11 +236,17 @@ void tq_debug_inject(tq_status status, int32_t count);
  * Arguments and results are those of tq_attend_v; the scratch space comes from
  * a fixed array compiled into the library (TQ_ATTEND_NOALLOC_SCRATCH_BYTES).
  *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
- *   - The first call on a device looks up the array's device address (once per
- *     device, with that device current); make that first call before any
- *     stream capture.
- *   - Returns TQ_ERR_WORKSPACE, before any launch, when
+ *   - The array's device address is looked up (cudaGetSymbolAddress, with the
+ *     device current) by the first call in each CUDA context of a device, and
+ *     again after the context changes (a cudaDeviceReset loads the library's
+ *     device code anew). Make the first call on a device before any stream
+ *     capture.
+ *   - Arguments are checked exactly as tq_attend_v checks them, with the same
+ *     statuses; then TQ_ERR_WORKSPACE, before any launch, when
  *     tq_attend_workspace_size(v, n_q_heads, n_tokens) exceeds the array.
+ *   - The kernels' status word sits at the start of the array: read it with
+ *     tq_attend_v_noalloc_status, not tq_workspace_status (the caller does not
+ *     hold the array's address). The next call clears it.
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents: two calls whose work can overlap on the GPU (different
  *     streams, or different host threads) race and corrupt each other's
@@ -247,6 +255,13 @@ tq_status tq_attend_v_noalloc(const tq_cache *v, const float *logits, float scal
                               int32_t n_q_heads, int64_t n_tokens,
                               const float *Pi, const float *codebook, float *out,
                               tq_stream stream);
+
+/* tq_workspace_status for the built-in array of tq_attend_v_noalloc on the
+ * current device: synchronises `stream`, reads the status word that the kernels
+ * of the last tq_attend_v_noalloc call on this device wrote, and clears it.
+ * TQ_OK if no kernel reported a failure, TQ_ERR_DEVICE otherwise. Allocates
+ * nothing. (No counterpart in the pages.) */
+tq_status tq_attend_v_noalloc_status(tq_stream stream);
 
 #ifdef __cplusplus
 }

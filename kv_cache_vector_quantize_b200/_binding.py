@@ -57,6 +57,7 @@ def _load() -> ctypes.CDLL:
         "tq_attend_workspace_size": (SZ, [D, I32, I64]),
         "tq_attend_v": (I32, [D, P, F, I32, I64, P, P, P, P, SZ, P]),
         "tq_attend_v_noalloc": (I32, [D, P, F, I32, I64, P, P, P, P]),
+        "tq_attend_v_noalloc_status": (I32, [P]),
         "tq_decode_workspace_size": (SZ, [D, D, I32, I64]),
         "tq_decode_attend": (I32, [D, D, P, I32, I64, F, P, P, P, P, P, P, SZ, P]),
         "tq_nn_workspace_size": (SZ, [D, I32, I64]),

@@ -18,6 +18,8 @@
 #include <cstdio>
 #include <mutex>
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace tq {
@@ -293,33 +295,76 @@ namespace {
 // written by that same call).
 static __device__ __align__(256) unsigned char g_attend_scratch[TQ_ATTEND_NOALLOC_SCRATCH_BYTES];
 
+// The array's device address differs per CUDA context (a context created after
+// cudaDeviceReset loads the module again), so it is cached per (device, context
+// id). Context ids are unique for the life of the process, unlike context handles,
+// which a new context may reuse.
 constexpr int kScratchMaxDevices = 64;
-void *g_scratch_addr[kScratchMaxDevices] = {nullptr};
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  void *addr;
+};
+ScratchEntry g_scratch[kScratchMaxDevices] = {};
 std::mutex g_scratch_mutex;
 
-// Device address of g_attend_scratch on the current device (looked up once per
-// device; the host-side symbol is only a stand-in and must never reach a kernel).
-tq_status scratch_address(void **out) {
+typedef CUresult (*PfnCtxGetCurrent)(CUcontext *);
+typedef CUresult (*PfnCtxGetId)(CUcontext, unsigned long long *);
+
+// Id of the current context (after a runtime call made the primary context current).
+tq_status current_context_id(unsigned long long *id) {
+  static PfnCtxGetCurrent get_current = nullptr;
+  static PfnCtxGetId get_id = nullptr;
+  if (!get_current || !get_id) {
+    void *f1 = nullptr, *f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess || !f1 ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess || !f2)
+      return report_error(TQ_ERR_CUDA, "tq_attend_v_noalloc: driver entry points cuCtxGetCurrent/cuCtxGetId not found");
+    get_current = reinterpret_cast<PfnCtxGetCurrent>(f1);
+    get_id = reinterpret_cast<PfnCtxGetId>(f2);
+  }
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS)
+    return report_error(TQ_ERR_CUDA, "tq_attend_v_noalloc: cuCtxGetCurrent failed");
+  if (ctx == nullptr) {
+    // no context on this thread yet: since CUDA 12, cudaSetDevice initialises the device's
+    // primary context and makes it current (it allocates nothing)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess ||
+        get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+      return report_error(TQ_ERR_CUDA, "tq_attend_v_noalloc: no current CUDA context");
+  }
+  if (get_id(ctx, id) != CUDA_SUCCESS) return report_error(TQ_ERR_CUDA, "tq_attend_v_noalloc: cuCtxGetId failed");
+  return TQ_OK;
+}
+
+// Device address of g_attend_scratch in the current context. Looked up with the
+// device current, once per (device, context); the host-side symbol is only a
+// stand-in and must never reach a kernel.
+tq_status scratch_address(void **out, const char *what) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) {
     char msg[256];
-    snprintf(msg, sizeof msg, "tq_attend_v_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+    snprintf(msg, sizeof msg, "%s: cudaGetDevice: %s", what, cudaGetErrorString(e));
     return report_error(TQ_ERR_CUDA, msg);
   }
   if (dev < 0 || dev >= kScratchMaxDevices) return report_error(TQ_ERR_UNSUPPORTED, "tq_attend_v_noalloc: device index too large");
+  unsigned long long id = 0;
+  tq_status s = current_context_id(&id);
+  if (s != TQ_OK) return s;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (g_scratch[dev].addr == nullptr || g_scratch[dev].ctx_id != id) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_attend_scratch);
     if (e != cudaSuccess || p == nullptr) {
       char msg[256];
-      snprintf(msg, sizeof msg, "tq_attend_v_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+      snprintf(msg, sizeof msg, "%s: cudaGetSymbolAddress: %s", what, cudaGetErrorString(e));
       return report_error(TQ_ERR_CUDA, msg);
     }
-    g_scratch_addr[dev] = p;
+    g_scratch[dev] = ScratchEntry{id, p};
   }
-  *out = g_scratch_addr[dev];
+  *out = g_scratch[dev].addr;
   return TQ_OK;
 }
 
@@ -330,6 +375,11 @@ tq_status scratch_address(void **out) {
 extern "C" tq_status tq_attend_v_noalloc(const tq_cache *v, const float *logits, float scale, int32_t n_q_heads,
                                          int64_t n_tokens, const float *Pi, const float *codebook, float *out,
                                          tq_stream stream) {
+  tq::clear_error();
+  // the same argument checks as tq_attend_v first, so a bad argument gets the same status
+  tq_status s = tq::check_attend_args(v, logits, scale, n_q_heads, n_tokens, Pi, codebook, out,
+                                      "tq_attend_v_noalloc");
+  if (s != TQ_OK) return s;
   const size_t need = tq_attend_workspace_size(v, n_q_heads, n_tokens);
   if (need > TQ_ATTEND_NOALLOC_SCRATCH_BYTES) {
     char msg[256];
@@ -339,8 +389,16 @@ extern "C" tq_status tq_attend_v_noalloc(const tq_cache *v, const float *logits,
     return tq::report_error(TQ_ERR_WORKSPACE, msg);
   }
   void *scratch = nullptr;
-  tq_status s = tq::scratch_address(&scratch);
+  s = tq::scratch_address(&scratch, "tq_attend_v_noalloc");
   if (s != TQ_OK) return s;
   return tq_attend_v(v, logits, scale, n_q_heads, n_tokens, Pi, codebook, out, scratch,
                      TQ_ATTEND_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+extern "C" tq_status tq_attend_v_noalloc_status(tq_stream stream) {
+  tq::clear_error();
+  void *scratch = nullptr;
+  tq_status s = tq::scratch_address(&scratch, "tq_attend_v_noalloc_status");
+  if (s != TQ_OK) return s;
+  return tq_workspace_status(scratch, stream);
 }

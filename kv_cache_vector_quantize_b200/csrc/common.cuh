@@ -188,6 +188,11 @@ int device_sm_count();
 cudaError_t set_smem_once(const void *kernel, size_t bytes);
 size_t device_smem_optin();
 tq_status report_error(tq_status s, const char *msg);
+void clear_error();   // empties this thread's tq_last_error() text
+// The argument checks of tq_attend_v that do not involve the workspace (tq_api.cu).
+tq_status check_attend_args(const tq_cache *v, const float *logits, float scale, int32_t n_q_heads,
+                            int64_t n_tokens, const float *Pi, const float *codebook, const float *out,
+                            const char *what);
 
 }  // namespace tq
 

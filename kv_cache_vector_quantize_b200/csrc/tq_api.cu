@@ -171,6 +171,52 @@ tq_status report_error(tq_status s, const char *msg) { return fail(s, "%s", msg)
 
 }  // namespace tq
 
+namespace tq {
+
+// Bytes of the softmax.V chunk partials plus the header, or SIZE_MAX when the product overflows.
+size_t attend_ws_bytes(const tq_cache *v, int32_t n_q_heads, int64_t n_tokens) {
+  const int64_t n_chunks = (n_tokens + kAttendChunk - 1) / kAttendChunk;
+  size_t b = sizeof(float);
+  if (__builtin_mul_overflow(b, (size_t)v->n_seq, &b) || __builtin_mul_overflow(b, (size_t)n_q_heads, &b) ||
+      __builtin_mul_overflow(b, (size_t)n_chunks, &b) || __builtin_mul_overflow(b, (size_t)(v->d + 2), &b) ||
+      __builtin_add_overflow(b, kWsHeader, &b))
+    return SIZE_MAX;
+  return b;
+}
+
+void clear_error() { g_err[0] = 0; }
+
+// Every check of tq_attend_v that does not involve the workspace, in order; shared with
+// tq_attend_v_noalloc so that both report the same status for the same bad argument.
+tq_status check_attend_args(const tq_cache *v, const float *logits, float scale, int32_t n_q_heads,
+                            int64_t n_tokens, const float *Pi, const float *codebook, const float *out,
+                            const char *what) {
+  tq_status s = check_cache(v, what);
+  if (s != TQ_OK) return s;
+  if (v->qjl) return fail(TQ_ERR_INVALID, "%s: the cache is a key cache (qjl == 1)", what);
+  if (n_q_heads <= 0 || n_q_heads % v->n_kv_heads != 0)
+    return fail(TQ_ERR_INVALID, "%s: n_q_heads=%d is not a positive multiple of n_kv_heads=%d", what, n_q_heads,
+                v->n_kv_heads);
+  if (n_tokens < 0 || n_tokens > v->capacity)
+    return fail(TQ_ERR_CAPACITY, "%s: n_tokens=%lld outside [0, capacity=%lld]", what, (long long)n_tokens,
+                (long long)v->capacity);
+  if ((!logits && n_tokens > 0) || !Pi || !codebook || !out)
+    return fail(TQ_ERR_INVALID, "%s: NULL tensor argument", what);
+  if (!(scale == scale) || scale == INFINITY || scale == -INFINITY)
+    return fail(TQ_ERR_INVALID, "%s: scale is not finite", what);
+  const int group = n_q_heads / v->n_kv_heads;
+  const int q_per_cta = group < kAttendMaxQ ? group : kAttendMaxQ;
+  const int64_t grid_y = (int64_t)v->n_seq * v->n_kv_heads * ((group + q_per_cta - 1) / q_per_cta);
+  if (grid_y > 65535 || (int64_t)v->n_seq * n_q_heads > 0x7fffffffLL)
+    return fail(TQ_ERR_UNSUPPORTED, "%s: n_seq x n_kv_heads x query blocks = %lld exceeds 65535", what,
+                (long long)grid_y);
+  if (attend_ws_bytes(v, n_q_heads, n_tokens) == SIZE_MAX)
+    return fail(TQ_ERR_UNSUPPORTED, "%s: the chunk partials of this shape overflow a size_t", what);
+  return TQ_OK;
+}
+
+}  // namespace tq
+
 using namespace tq;
 
 extern "C" {
@@ -278,6 +324,9 @@ tq_status tq_logits(const tq_cache *k, const float *q, int32_t n_q_heads, int64_
   if (n_tokens < 0 || n_tokens > k->capacity)
     return fail(TQ_ERR_CAPACITY, "tq_logits: n_tokens=%lld outside [0, capacity=%lld]", (long long)n_tokens,
                 (long long)k->capacity);
+  if ((int64_t)k->n_seq * n_q_heads > 65535)
+    return fail(TQ_ERR_UNSUPPORTED, "tq_logits: n_seq x n_q_heads = %lld exceeds 65535",
+                (long long)k->n_seq * n_q_heads);
   if (n_tokens == 0) return TQ_OK;   // nothing to scan (logits may be an empty, NULL tensor)
   if (!q || !Pi || !S || !codebook || !logits) return fail(TQ_ERR_INVALID, "tq_logits: NULL tensor argument");
   const size_t need = tq_logits_workspace_size(k, n_q_heads);
@@ -351,26 +400,15 @@ tq_status tq_logits(const tq_cache *k, const float *q, int32_t n_q_heads, int64_
 
 size_t tq_attend_workspace_size(const tq_cache *v, int32_t n_q_heads, int64_t n_tokens) {
   if (!v || v->n_seq <= 0 || v->d <= 0 || n_q_heads <= 0 || n_tokens < 0) return 0;
-  const int64_t n_chunks = (n_tokens + kAttendChunk - 1) / kAttendChunk;
-  return kWsHeader + sizeof(float) * (size_t)v->n_seq * n_q_heads * (size_t)n_chunks * (v->d + 2);
+  return attend_ws_bytes(v, n_q_heads, n_tokens);
 }
 
 tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale, int32_t n_q_heads, int64_t n_tokens,
                       const float *Pi, const float *codebook, float *out, void *workspace, size_t workspace_bytes,
                       tq_stream stream) {
   g_err[0] = 0;
-  tq_status s = check_cache(v, "tq_attend_v");
+  tq_status s = check_attend_args(v, logits, scale, n_q_heads, n_tokens, Pi, codebook, out, "tq_attend_v");
   if (s != TQ_OK) return s;
-  if (v->qjl) return fail(TQ_ERR_INVALID, "tq_attend_v: the cache is a key cache (qjl == 1)");
-  if (n_q_heads <= 0 || n_q_heads % v->n_kv_heads != 0)
-    return fail(TQ_ERR_INVALID, "tq_attend_v: n_q_heads=%d is not a positive multiple of n_kv_heads=%d", n_q_heads,
-                v->n_kv_heads);
-  if (n_tokens < 0 || n_tokens > v->capacity)
-    return fail(TQ_ERR_CAPACITY, "tq_attend_v: n_tokens=%lld outside [0, capacity=%lld]", (long long)n_tokens,
-                (long long)v->capacity);
-  if ((!logits && n_tokens > 0) || !Pi || !codebook || !out)
-    return fail(TQ_ERR_INVALID, "tq_attend_v: NULL tensor argument");
-  if (!(scale == scale) || scale == INFINITY || scale == -INFINITY) return fail(TQ_ERR_INVALID, "tq_attend_v: scale is not finite");
   const size_t need = tq_attend_workspace_size(v, n_q_heads, n_tokens);
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < need)
     return fail(TQ_ERR_WORKSPACE, "tq_attend_v: workspace needs %zu bytes, 256-byte aligned (got %zu)", need,
@@ -488,6 +526,9 @@ tq_status tq_decode_attend(const tq_cache *k, const tq_cache *v, const float *q,
                 n_q_heads, k->n_kv_heads);
   if (n_tokens < 0 || n_tokens > k->capacity || n_tokens > v->capacity)
     return fail(TQ_ERR_CAPACITY, "tq_decode_attend: n_tokens=%lld outside [0, capacity]", (long long)n_tokens);
+  if ((int64_t)k->n_seq * n_q_heads > 65535)
+    return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attend: n_seq x n_q_heads = %lld exceeds 65535",
+                (long long)k->n_seq * n_q_heads);
   if (!q || !Pi || !S || !codebook_k || !codebook_v || !out)
     return fail(TQ_ERR_INVALID, "tq_decode_attend: NULL tensor argument");
   if (!(scale == scale) || scale == INFINITY || scale == -INFINITY)

@@ -184,3 +184,26 @@ def test_fault_injection_counts_down():
     assert _q(_desc(qjl=0)) == tqb.TQ_ERR_DEVICE
     assert "injected" in tqb.tq_last_error()
     tqb.tq_debug_inject(tqb.TQ_ERR_CUDA, 1000)
+
+
+def test_noalloc_checks_arguments_before_its_scratch_size():
+    # n_q_heads = 63 is not a multiple of 8 KV heads; the shape is also far beyond the
+    # built-in array. The argument error must win, with the same status as tq_attend_v.
+    desc = _desc(d=128, bits=3, qjl=0, n_seq=8, heads=8, cap=131072)
+    st = lib.tq_attend_v_noalloc(ctypes.byref(desc), FAKE, ctypes.c_float(0.1), 63, 131072, FAKE, FAKE, FAKE, None)
+    assert st == tqb.TQ_ERR_INVALID
+    assert "multiple" in tqb.tq_last_error()
+    st2 = lib.tq_attend_v(ctypes.byref(desc), FAKE, ctypes.c_float(0.1), 63, 131072, FAKE, FAKE, FAKE, FAKE, 1 << 30,
+                          None)
+    assert st2 == st
+
+
+def test_attend_workspace_size_does_not_wrap():
+    # a descriptor whose partials would overflow a size_t: the size query saturates and
+    # the call refuses the shape instead of writing past a small workspace
+    desc = _desc(d=256, bits=3, qjl=0, n_seq=2 ** 31 - 1, heads=1, cap=2 ** 62)
+    need = lib.tq_attend_workspace_size(ctypes.byref(desc), 2 ** 31 - 1, 2 ** 62)
+    assert need == 2 ** 64 - 1
+    st = lib.tq_attend_v(ctypes.byref(desc), FAKE, ctypes.c_float(0.1), 2 ** 31 - 1, 2 ** 62, FAKE, FAKE, FAKE, FAKE,
+                         1 << 30, None)
+    assert st == tqb.TQ_ERR_UNSUPPORTED

@@ -9,8 +9,11 @@ and outputs as tq_attend_v but uses a fixed array compiled into the library.
 These tests call it through the C ABI and compare its output with the regular
 tq_attend_v on the same inputs (with a caller workspace), for two calls in a
 row with different shapes, so that nothing left in the shared array by the
-first call can leak into the second. The file is named so that pytest collects
-it last.
+first call can leak into the second. Both paths run the same kernels on the same
+inputs, so the outputs must be bit-identical. After each call the array's status
+word is read with tq_attend_v_noalloc_status, the only way a caller can see a
+device-side failure of this entry point. The file is named so that pytest
+collects it last.
 """
 
 from __future__ import annotations
@@ -28,8 +31,6 @@ pytestmark = pytest.mark.gpu
 cuda_ok = torch.cuda.is_available()
 if cuda_ok:
     import kv_cache_vector_quantize_b200 as tqb
-
-OUT_TOL = 2e-3   # the softmax.V tolerance of the parity tests: 2e-3 * max_t n_t
 
 
 def _noalloc(vc, logits, scale, n_tokens, Pi, cb, out):
@@ -62,10 +63,11 @@ def test_noalloc_matches_workspace_path_on_two_calls():
         got = torch.full_like(want, float("nan"))
         status = _noalloc(vc, logits, scale, T, Pi, cb, got)
         assert status == tqb.TQ_OK, tqb.tq_last_error()
+        st = tqb.raw_lib().tq_attend_v_noalloc_status(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert st == tqb.TQ_OK, tqb.tq_last_error()
         torch.cuda.synchronize()
-        tol = OUT_TOL * float(vc.norm.max())
         assert torch.isfinite(got).all()
-        assert float((got - want).abs().max()) <= tol
+        assert torch.equal(got, want), float((got - want).abs().max())
 
 
 @pytest.mark.skipif(not cuda_ok, reason="needs a CUDA device")
