@@ -6,10 +6,16 @@ A step is one pass of the whole path over one batch of synthetic input:
   -> L2 flush (the decode reads a cache written long before, from HBM)
   -> tq_logits (query projection + logit scan) -> tq_attend_v (softmax.V).
 
-Default workload (N = 1): the Llama-3-8B-shaped decode -- 1 sequence, 32 query
-heads on 8 KV heads, d = 128, 32768 cached tokens, bf16 K/V with outlier
-channels, keys at 3 bits (2-bit codes + 1 QJL bit), values at 3 bits MSE-only.
-`--workload sweep-b{2,3,4}` runs the b-sweep caches (8 x 8 x 131072 tokens).
+Default workload (N = 1): the large-model cache -- 80 layers x 128 KV heads x
+d = 128 x 131072 tokens, fp16 K/V N(0,1) with outlier channels, keys at 3 bits
+(2-bit codes + 1 QJL bit), values at 3 bits MSE-only, one query head per KV
+head. It does not fit in HBM at once (687 GB of fp16), so it is streamed: one
+step is one layer, `--steps` layers are timed after `--warmup` warm-up layers,
+and the layer seeds cycle over the 80 layers. `--workload llama` runs the
+Llama-3-8B-shaped decode (32 query heads on 8 KV heads, 32768 tokens, bf16),
+`--workload sweep-b{2,3,4}` the b-sweep caches (8 x 8 x 131072 tokens),
+`--workload large-b4` the large-model cache at 4 bits and `--workload nn-b{2,4}`
+the nearest-neighbour search.
 
 Metric: packed-KV logit-scan GB/s = packed key bytes (records + norms) read
 by one tq_logits call / its device time; quantize tokens/s is reported beside
@@ -62,13 +68,12 @@ NCU_TRAFFIC = {
 def parse():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
-    ap.add_argument("--workload", default="llama",
+    ap.add_argument("--workload", default="large-b3",
                     choices=["llama"] + [f"sweep-b{b}{s}" for b in (2, 3, 4) for s in ("", "-s4")]
                     + ["large-b3", "large-b4", "nn-b2", "nn-b4", "nn-b2-s", "nn-b4-s"])
-    ap.add_argument("--layers", type=int, default=80, help="layers streamed by the large-model workload")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -409,15 +414,18 @@ def decode_roof(ms, two_call_ms, nbytes, w, hbm, src_txt, traffic=None):
 
 
 def run_large(args, rank, world, local_rank):
-    """Large-model cache streamed layer by layer: per layer, generate K and V on the device
-    (untimed), quantize both into the packed caches, flush L2, one decode step (logits and
-    softmax.V); the packed buffers are reused by every layer."""
+    """Large-model cache streamed layer by layer. A step is one layer: quantize its K and V
+    into the packed caches, flush L2, then one decode step on them (tq_logits, tq_attend_v).
+    The layer's fp16 inputs are generated on the device between steps (the 80 layers do not
+    fit in HBM at once: 687 GB), so every step starts with its inputs resident; steps cycle
+    through the 80 layer seeds. The packed buffers are reused by every layer."""
     import kv_cache_vector_quantize_b200 as tqb
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = workload(args.workload)
     d, H, T = w["d"], w["hkv"], w["T"]
+    n_layers = 80
     Pi = syn.rotation(d).to(dev)
     S = syn.sketch(d).to(dev)
     ck = tqb.tq_codebook_fit(d, w["k_idx"]).to(dev)
@@ -435,89 +443,182 @@ def run_large(args, rank, world, local_rank):
                         device=dev)
     stream = torch.cuda.current_stream(dev)
     scale = 1.0 / math.sqrt(d)
+    names = ("quantize_k", "quantize_v", "l2_flush", "logits", "attend_v")
 
     def path(k, v, q, ev=None):
+        calls = (lambda: tqb.tq_quantize_append(kc, k, 0, Pi, SPiT, ck),
+                 lambda: tqb.tq_quantize_append(vc, v, 0, Pi, None, cv),
+                 lambda: flush.fill_(1.0),
+                 lambda: tqb.tq_logits(kc, q, T, Pi, S, ck, logits=logits, workspace=ws_l),
+                 lambda: tqb.tq_attend_v(vc, logits, scale, T, Pi, cv, out=out, workspace=ws_a))
+        for i, call in enumerate(calls):
+            if ev is not None:
+                ev[i].record(stream)
+            call()
         if ev is not None:
-            ev[0].record(stream)
-        tqb.tq_quantize_append(kc, k, 0, Pi, SPiT, ck)
-        if ev is not None:
-            ev[1].record(stream)
-        tqb.tq_quantize_append(vc, v, 0, Pi, None, cv)
-        if ev is not None:
-            ev[2].record(stream)
-        flush.fill_(1.0)
-        if ev is not None:
-            ev[3].record(stream)
-        tqb.tq_logits(kc, q, T, Pi, S, ck, logits=logits, workspace=ws_l)
-        if ev is not None:
-            ev[4].record(stream)
-        tqb.tq_attend_v(vc, logits, scale, T, Pi, cv, out=out, workspace=ws_a)
-        if ev is not None:
-            ev[5].record(stream)
-        flush.fill_(1.0)   # the one-call decode step on the same caches, from HBM
-        if ev is not None:
-            ev[6].record(stream)
-        tqb.tq_decode_attend(kc, vc, q, T, scale, Pi, S, ck, cv, out=out_d, workspace=ws_d)
-        if ev is not None:
-            ev[7].record(stream)
+            ev[len(calls)].record(stream)
 
-    k, v, q = w["gen"](dev, rank_seed(rank))
-    for _ in range(args.warmup):
+    def layer_inputs(step):
+        return w["gen"](dev, step % n_layers + rank_seed(rank))
+
+    for i in range(args.warmup):
+        k, v, q = layer_inputs(i)
         path(k, v, q)
+        del k, v
     torch.cuda.synchronize(dev)
-    per = {n: 0.0 for n in ("quantize_k", "quantize_v", "l2_flush", "logits", "attend_v", "l2_flush_2",
-                            "decode_attend")}
+    tqb.tq_workspace_status(ws_l)
+    tqb.tq_workspace_status(ws_a)
+    per = {n: 0.0 for n in names}
     clocks = ClockSampler(dev.index)
-    if world > 1:
-        dist.barrier()
+    time.sleep(0.3)
     clocks.mark_start()
-    for layer in range(args.layers):
-        if layer > 0:
-            del k, v
-            k, v, q = w["gen"](dev, layer + rank_seed(rank))   # untimed input generation
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
+    for step in range(args.steps):
+        k, v, q = layer_inputs(step)   # generated on the device, outside the timed calls
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+        if world > 1:
+            dist.barrier()
         torch.cuda.synchronize(dev)
         path(k, v, q, ev)
         torch.cuda.synchronize(dev)
-        for i, n in enumerate(per):
+        for i, n in enumerate(names):
             per[n] += ev[i].elapsed_time(ev[i + 1])
+        if step + 1 < args.steps:
+            del k, v
     clocks.mark_end()
-    tqb.tq_workspace_status(ws_l)
+    tqb.tq_workspace_status(ws_l)   # raises if a kernel of the timed region reported a failure
     tqb.tq_workspace_status(ws_a)
-    tqb.tq_workspace_status(ws_d)
+    if world > 1:
+        dist.barrier()
     clk = clocks.stop()
-    logits_ms, quant_ms, total_ms, dec_ms = max_over_ranks(
-        [per["logits"], per["quantize_k"] + per["quantize_v"], sum(per.values()), per["decode_attend"]], dev, world)
-    L = args.layers
+    step_ms = {n: per[n] / args.steps for n in names}
+    path_ms = sum(step_ms[n] for n in names if n != "l2_flush")
+    logits_ms, quant_ms, path_ms, qk_ms, qv_ms, att_ms = max_over_ranks(
+        [step_ms["logits"], step_ms["quantize_k"] + step_ms["quantize_v"], path_ms, step_ms["quantize_k"],
+         step_ms["quantize_v"], step_ms["attend_v"]], dev, world)
+
+    # ---- the one-call decode step (tq_decode_attend) on the last layer's caches, L2 flushed before each ----
+    def decode_step():
+        tqb.tq_decode_attend(kc, vc, q, T, scale, Pi, S, ck, cv, out=out_d, workspace=ws_d)
+
+    for _ in range(3):
+        flush.fill_(1.0)
+        decode_step()
+    torch.cuda.synchronize(dev)
+    dec_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(10)]
+    for a, b in dec_evs:
+        flush.fill_(1.0)
+        a.record(stream)
+        decode_step()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    tqb.tq_workspace_status(ws_d)
+    dec_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in dec_evs) / len(dec_evs)], dev, world)[0]
+
+    # ---- end to end: one layer's pinned host K, V, q in, the path, out back, through the public API ----
+    e2e = None
+    if args.e2e_steps > 0:
+        hk = torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
+        hv = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+        hq_ = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        hk.copy_(k)
+        hv.copy_(v)
+        hq_.copy_(q)
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+
+        def step_e2e():
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            q.copy_(hq_, non_blocking=True)
+            path(k, v, q)
+            hout.copy_(out, non_blocking=True)
+
+        step_e2e()
+        torch.cuda.synchronize(dev)
+        n_e2e = min(args.e2e_steps, 5)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        a.record(stream)
+        for _ in range(n_e2e):
+            step_e2e()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks([a.elapsed_time(b) / n_e2e], dev, world)[0]
+        h2d = hk.numel() * hk.element_size() + hv.numel() * hv.element_size() + hq_.numel() * hq_.element_size()
+        e2e = {"value": round(world * key_bytes(w) / (e2e_ms * 1e-3) / 1e9, 3), "unit": UNIT,
+               "ms_per_step": round(e2e_ms, 4), "steps": n_e2e, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": hout.numel() * hout.element_size(),
+               "note": "packed key bytes scanned per end-to-end layer step (pinned H2D of the layer's fp16 K and V "
+                       "and its queries, quantize, flush, logits, softmax.V, D2H of out); bound by the H2D copy"}
+        del hk, hv
+
     kb, vb = key_bytes(w), value_bytes(w)
     fp16_bytes = 2 * H * T * d * 2
     peaks, peak_src = load_peaks()
     hbm = float(peaks["hbm_gbs"])
-    scan_gbs = L * kb / (logits_ms * 1e-3) / 1e9
-    qk_bytes = H * T * (2 * d) + kb
+    bf16 = float(peaks["bf16_tflops"])
+    src_txt = f"hbm_gbs / bf16_tflops, {peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    scan_gbs = kb / (logits_ms * 1e-3) / 1e9
+    hv_layer = H * T
+    qk_bytes, qv_bytes = hv_layer * 2 * d + kb, hv_layer * 2 * d + vb
+    qk_flops, qv_flops = hv_layer * 4 * d * d, hv_layer * 2 * d * d
+
+    def quant_roof(kernel, nbytes, nflops, ms, traffic):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        tfs = nflops / (ms * 1e-3) / 1e12
+        bound = "hbm" if nbytes / hbm > nflops / (bf16 * 1e3) else "tensor"
+        ach, peak, unit = (gbs, hbm, "GB/s") if bound == "hbm" else (tfs, bf16, "TFLOP/s")
+        return {"kernel": kernel, "bound": bound, "achieved": round(ach, 1), "peak": peak, "unit": unit,
+                "frac": round(ach / peak, 4), "traffic": traffic, "peak_source": src_txt,
+                "tensor_tflops": round(tfs, 1), "tensor_frac": round(tfs / bf16, 4), "ms": round(ms, 4),
+                "algorithmic": f"{nbytes // hv_layer} B and {nflops // hv_layer} flop per head-vector, "
+                               f"{hv_layer} head-vectors per launch"}
+
+    roofline = quant_roof("quantize_tc_kernel, key launch (tq_quantize_append on the layer's K cache)", qk_bytes,
+                          qk_flops, qk_ms, NCU_TRAFFIC.get(("quantize_k", args.workload)))
+    roof_qv = quant_roof("quantize_tc_kernel, value launch (tq_quantize_append on the layer's V cache)", qv_bytes,
+                         qv_flops, qv_ms, NCU_TRAFFIC.get(("quantize_v", args.workload)))
+    att_gbs = vb / (att_ms * 1e-3) / 1e9
     result = {
-        "metric": METRIC, "value": round(world * scan_gbs, 2), "unit": UNIT, "n_gpus": world, "steps": L,
-        "warmup": args.warmup, "ms_per_step": round(total_ms / L, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": w["name"].replace("L layers", f"{L} layers"), "parallelism": "single" if world == 1
-                   else f"replicas{world}", "step": "one layer (inputs generated on the device outside the timed "
-                   "calls)", "l2": "flushed (2 x L2 write) between quantize and decode in every layer"},
-        "quantize_tokens_per_s": round(world * L * T / (quant_ms * 1e-3), 1),
-        "quantize_head_vectors_per_s": round(world * L * H * T / (quant_ms * 1e-3), 1),
-        "per_kernel_ms_per_layer": {n: round(x / L, 5) for n, x in per.items()},
-        "compressed_bytes_total": L * (kb + vb), "uncompressed_fp16_bytes_total": L * fp16_bytes,
+        "metric": METRIC, "value": round(world * scan_gbs, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(path_ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": w["name"].replace("L layers", f"{n_layers} layers"),
+                   "parallelism": "single" if world == 1 else f"replicas{world}",
+                   "step": "one layer (layer seeds cycled over the 80 layers; its fp16 K/V generated on the device "
+                           "before the step, outside the timed calls): quantize K and V, L2 flush, tq_logits, "
+                           "tq_attend_v; ms_per_step = the four calls' device time, the flush excluded",
+                   "l2": "flushed (2 x L2 write) between quantize and the decode of every layer; every layer's "
+                         "inputs (8.6 GB) are also larger than L2",
+                   "value_definition": "packed K bytes of one layer per tq_logits call / its mean device time "
+                                       "(CUDA events), summed over ranks",
+                   "dtype_note": "narrowest arithmetic on the path: fp16 tensor-core products with split operands "
+                                 "and float32 accumulation in the quantizer; the single-head scan and softmax.V "
+                                 "accumulate in float32"},
+        "quantize_tokens_per_s": round(world * T / (quant_ms * 1e-3), 1),
+        "quantize_head_vectors_per_s": round(world * 2 * hv_layer / (quant_ms * 1e-3), 1),
+        "per_kernel_ms_per_layer": {n: round(x, 5) for n, x in step_ms.items()},
+        "compressed_bytes": {"per_layer": kb + vb, "timed_layers": args.steps * (kb + vb),
+                             "all_80_layers": n_layers * (kb + vb)},
+        "uncompressed_fp16_bytes": {"per_layer": fp16_bytes, "all_80_layers": n_layers * fp16_bytes},
         "compression_ratio_vs_fp16": round(fp16_bytes / (kb + vb), 4),
-        "roofline_logit_scan": {"kernel": "tq_logits", "bound": "hbm", "achieved": round(scan_gbs, 1), "peak": hbm,
-                                "unit": "GB/s", "frac": round(scan_gbs / hbm, 4), "traffic": None,
-                                "peak_source": peak_src},
-        "roofline_quantize_k": {"kernel": "quantize_tc_kernel (fp16 keys)", "bound": "hbm",
-                                "achieved": round(L * qk_bytes / (per["quantize_k"] * 1e-3) / 1e9, 1), "peak": hbm,
-                                "unit": "GB/s"},
-        "roofline_decode_attend": decode_roof(dec_ms / L, (per["logits"] + per["attend_v"]) / L, kb + vb, w, hbm,
-                                              peak_src),
-        # per layer: quantize K, V; projection + scan; V chunks + merge; and the one-call decode step
-        # (projection, fused pass, merge; or the two calls' four kernels and the status merge)
-        "gpu_launches": (6 + (3 if w["k_idx"] in (1, 2) else 5)) * L, "clocks": clk, "e2e": None,
+        "packed_bytes": {"keys": kb, "values": vb},
+        "roofline": roofline, "roofline_quantize_v": roof_qv,
+        "roofline_logit_scan": {"kernel": "tq_logits (query projection + logit scan)", "bound": "hbm",
+                                "achieved": round(scan_gbs, 1), "peak": hbm, "unit": "GB/s",
+                                "frac": round(scan_gbs / hbm, 4),
+                                "traffic": NCU_TRAFFIC.get(("logits", args.workload)), "peak_source": src_txt,
+                                "ms": round(logits_ms, 5),
+                                "algorithmic": f"{kb // hv_layer} B per key (record + norm + rnorm)"},
+        "roofline_attend_v": {"kernel": "tq_attend_v (chunk softmax.V + merge)", "bound": "hbm",
+                              "achieved": round(att_gbs, 1), "peak": hbm, "unit": "GB/s",
+                              "frac": round(att_gbs / hbm, 4),
+                              "traffic": NCU_TRAFFIC.get(("attend_v", args.workload)), "peak_source": src_txt,
+                              "ms": round(att_ms, 5), "algorithmic": f"{vb // hv_layer} B per value (record + norm)"},
+        "roofline_decode_attend": decode_roof(dec_ms, logits_ms + att_ms, kb + vb, w, hbm, src_txt,
+                                              NCU_TRAFFIC.get(("decode_attend", args.workload))),
+        # per step: quantize K, quantize V; projection + scan; V chunks + merge
+        "gpu_launches": 6 * args.steps, "clocks": clk, "e2e": e2e,
     }
     return result, w
 

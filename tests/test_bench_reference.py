@@ -23,9 +23,12 @@ def _run(args, env_extra=None):
     return r.stdout
 
 
-@pytest.mark.parametrize("workload,name", [("llama", "llama3-8b-decode"), ("nn-b2", "nn-search-b2")])
+@pytest.mark.parametrize("workload,name", [(None, "large-model-b3"), ("llama", "llama3-8b-decode"),
+                                           ("nn-b2", "nn-search-b2")])
 def test_reference_arm_line(workload, name):
-    out = _run(["--impl", "reference", "--workload", workload, "--steps", "1", "--warmup", "0"])
+    # workload None: bench.py's default (the large-model cache at 3 bits)
+    out = _run(["--impl", "reference", *(["--workload", workload] if workload else []), "--steps", "1",
+                "--warmup", "0"])
     lines = [ln for ln in out.splitlines() if ln.strip()]
     assert len(lines) == 1
     r = json.loads(lines[0])

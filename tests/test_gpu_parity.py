@@ -482,9 +482,23 @@ def test_llama_decode_full_size():
     assert np.isfinite(lg_np).all() and np.isfinite(out_np).all()
 
 
+def _decode_full_size(kc, vc, q, T, sc, g, out_two_calls):
+    """The one-call decode step on a full-size cache: equal bit for bit to tq_logits +
+    tq_attend_v (same tables, chunks and accumulation order), status clean."""
+    hq = q.shape[1]
+    ws = torch.empty(max(256, tqb.tq_decode_workspace_size(kc, vc, hq, T)), dtype=torch.uint8, device="cuda")
+    ws[:256].fill_(0xFF)   # the call must clear the status word itself
+    out1 = tqb.tq_decode_attend(kc, vc, q, T, sc, g["Pi"], g["S"], g["ck"], g["cv"], workspace=ws)
+    torch.cuda.synchronize()
+    tqb.tq_workspace_status(ws)
+    assert torch.equal(out1, out_two_calls), float((out1 - out_two_calls).abs().max())
+    return out1
+
+
 @pytest.mark.parametrize("bits", [2, 3, 4])
 def test_bsweep_full_size_sampled(bits):
-    # 8 x 8 KV heads x 131072 tokens x 128, bf16, lognormal norms; K at b bits (b-1 codes + QJL).
+    # 8 x 8 KV heads x 131072 tokens x 128, bf16, lognormal norms; K at b bits (b-1 codes + QJL),
+    # V at b bits (MSE only); the bench's launch shapes.
     B, H, T, d = 8, 8, 131072, 128
     k, v, q = syn.sweep_inputs(device="cuda")
     Pi, S, ck, cv, g = _setup(d, bits - 1, bits)
@@ -493,10 +507,14 @@ def test_bsweep_full_size_sampled(bits):
     tqb.tq_quantize_append(kc, k, 0, g["Pi"], g["SPiT"], g["ck"])
     tqb.tq_quantize_append(vc, v, 0, g["Pi"], None, g["cv"])
     ws = torch.empty(tqb.tq_logits_workspace_size(kc, H), dtype=torch.uint8, device="cuda")
+    ws_a = torch.empty(tqb.tq_attend_workspace_size(vc, H, T), dtype=torch.uint8, device="cuda")
     lg = tqb.tq_logits(kc, q, T, g["Pi"], g["S"], g["ck"], workspace=ws)
+    sc = 1.0 / math.sqrt(d)
+    out = tqb.tq_attend_v(vc, lg, sc, T, g["Pi"], g["cv"], workspace=ws_a)
     torch.cuda.synchronize()
     tqb.tq_workspace_status(ws)
-    del v
+    tqb.tq_workspace_status(ws_a)
+    out_d = _decode_full_size(kc, vc, q, T, sc, g, out)
     rng = np.random.default_rng(100 + bits)
     for _ in range(4):
         s, h = int(rng.integers(B)), int(rng.integers(H))
@@ -509,9 +527,17 @@ def test_bsweep_full_size_sampled(bits):
         par.check_encoding(kx, krec, kn, kr, Pi, S, ck, d, bits - 1, True)
         par.check_logits(lg[s, h].index_select(0, idx).cpu().numpy()[None, :],
                          q[s, h].cpu().numpy()[None, :].astype(np.float64), Pi, S, ck, krec, kn, kr, d, bits - 1)
-    # properties at full size: the packed norms are finite and positive, logits finite
-    assert torch.isfinite(lg).all()
-    assert bool((kc.norm > 0).all()) and bool(torch.isfinite(kc.rnorm).all())
+        vx = v[s, h].index_select(0, idx).float().cpu().numpy()
+        par.check_encoding(vx, par.as_u32(vc.records[s, h].index_select(0, idx).cpu().numpy()),
+                           vc.norm[s, h].index_select(0, idx).cpu().numpy(), None, Pi, None, cv, d, bits, False)
+        # softmax.V (two calls and the one-call step) over all of this head's tokens, oracle on the
+        # GPU's cache and logits
+        for o in (out, out_d):
+            par.check_attend(o[s, h:h + 1].cpu().numpy(), lg[s, h:h + 1].cpu().numpy().astype(np.float64), sc, Pi,
+                             cv, par.as_u32(vc.records[s, h].cpu().numpy()), vc.norm[s, h].cpu().numpy(), d, bits)
+    # properties at full size: the packed norms are finite and positive, logits and outputs finite
+    assert torch.isfinite(lg).all() and torch.isfinite(out).all()
+    assert bool((kc.norm > 0).all()) and bool(torch.isfinite(kc.rnorm).all()) and bool((vc.norm > 0).all())
 
 
 @pytest.mark.parametrize("bits", [3, 4])
@@ -533,6 +559,7 @@ def test_large_model_layer_sampled(bits):
     torch.cuda.synchronize()
     tqb.tq_workspace_status(ws_l)
     tqb.tq_workspace_status(ws_a)
+    out_d = _decode_full_size(kc, vc, q, T, sc, g, out)
     rng = np.random.default_rng(300 + bits)
     for h in [int(x) for x in rng.choice(H, size=3, replace=False)]:
         rows = np.sort(rng.choice(T, size=512, replace=False))
@@ -547,8 +574,10 @@ def test_large_model_layer_sampled(bits):
                            vc.norm[0, h].index_select(0, idx).cpu().numpy(), None, Pi, None, cv, d, bits, False)
         par.check_logits(lg[0, h].index_select(0, idx).cpu().numpy()[None, :],
                          q[0, h].cpu().numpy()[None, :].astype(np.float64), Pi, S, ck, krec, kn, kr, d, bits - 1)
-        # softmax.V over all of this head's tokens, oracle on the GPU's cache and logits
-        par.check_attend(out[0, h:h + 1].cpu().numpy(), lg[0, h:h + 1].cpu().numpy().astype(np.float64), sc, Pi, cv,
-                         par.as_u32(vc.records[0, h].cpu().numpy()), vc.norm[0, h].cpu().numpy(), d, bits)
+        # softmax.V (two calls and the one-call step) over all of this head's tokens, oracle on the
+        # GPU's cache and logits
+        for o in (out, out_d):
+            par.check_attend(o[0, h:h + 1].cpu().numpy(), lg[0, h:h + 1].cpu().numpy().astype(np.float64), sc, Pi,
+                             cv, par.as_u32(vc.records[0, h].cpu().numpy()), vc.norm[0, h].cpu().numpy(), d, bits)
     assert torch.isfinite(lg).all() and torch.isfinite(out).all()
     assert bool((kc.norm > 0).all()) and bool(torch.isfinite(kc.rnorm).all())
