@@ -24,6 +24,11 @@ What it computes, and the pages it follows:
   funciona" (1. PolarQuant: multiply by a random orthogonal matrix;
   2. QJL Residual: one extra bit per value removes the inner-product bias).
 
+* ``mixed_rate`` -- fractional bits per channel (the 3.5 and 2.5 bits per
+  channel of the zubnet.ai title and paragraph 2): the first m rotated
+  coordinates at one more code bit than the rest, each group with its own
+  Lloyd-Max codebook of the same law; encoder, packer, estimator, softmax.V.
+
 The pages print no estimator formula, codebook, QJL constant or layout; the
 readings taken where they are silent are listed in the module docstrings and
 marked "reading:".
@@ -36,4 +41,4 @@ hand-worked case; ``turboquant.padding_is_zero`` is pinned by planting a stray
 bit at every unused position of a record.
 """
 
-from . import codebook, turboquant  # noqa: F401
+from . import codebook, mixed_rate, turboquant  # noqa: F401
