@@ -72,7 +72,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--workload", default="large-b3",
-                    choices=["llama"] + [f"sweep-b{b}{s}" for b in (2, 3, 4) for s in ("", "-s4")]
+                    choices=["llama"] + [f"sweep-b{b}{s}" for b in (2, 3, 4, 2.5, 3.5) for s in ("", "-s4")]
                     + ["large-b3", "large-b4", "nn-b2", "nn-b4", "nn-b2-s", "nn-b4-s"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -104,22 +104,43 @@ def workload(name: str):
                     n_seq=1, hq=128, hkv=128, d=128, T=131072, k_idx=b - 1, v_idx=b, dtype=torch.float16,
                     gen=lambda dev, seed: syn.large_layer_inputs(seed, device=dev))
     # "sweep-b3" is the full b-sweep cache; "sweep-b3-s4" keeps 4 of its 8 sequences
-    # (a profiling size: still larger than L2, half the device memory)
-    b = int(name.split("-")[1][1:])
+    # (a profiling size: still larger than L2, half the device memory). "sweep-b3.5" and
+    # "sweep-b2.5": fractional bits per channel, half of the rotated coordinates at one more
+    # code bit (keys: b - 1 code bits on average + QJL; values: b code bits on average)
+    b = float(name.split("-")[1][1:])
     B = 4 if name.endswith("-s4") else 8
-    return dict(name=f"bsweep-b{b}: B={B} Hq=8 Hkv=8 d=128 T=131072 bf16 lognormal norms, K b={b} V b={b}",
-                n_seq=B, hq=8, hkv=8, d=128, T=131072, k_idx=b - 1, v_idx=b, dtype=torch.bfloat16,
-                gen=lambda dev, seed: syn.sweep_inputs(n_seq=B, device=dev, seed=seed))
+    d = 128
+    kb, vb = b - 1, b
+    k_idx, v_idx = int(math.floor(kb)), int(math.floor(vb))
+    k_nhi, v_nhi = int(round((kb - k_idx) * d)), int(round((vb - v_idx) * d))
+    btxt = f"{b:g}"
+    rate = (f" (keys: {k_idx + 1}-bit codes on {k_nhi} and {k_idx}-bit on {d - k_nhi} rotated coordinates + QJL; "
+            f"values: {v_idx + 1}-bit on {v_nhi} and {v_idx}-bit on {d - v_nhi})") if k_nhi or v_nhi else ""
+    return dict(name=f"bsweep-b{btxt}: B={B} Hq=8 Hkv=8 d=128 T=131072 bf16 lognormal norms, K b={btxt} V b={btxt}"
+                     + rate,
+                n_seq=B, hq=8, hkv=8, d=d, T=131072, k_idx=k_idx, v_idx=v_idx, k_nhi=k_nhi, v_nhi=v_nhi,
+                dtype=torch.bfloat16, gen=lambda dev, seed: syn.sweep_inputs(n_seq=B, device=dev, seed=seed))
+
+
+def _code_words(d, idx, n_hi) -> int:
+    return ((idx + 1) * n_hi + idx * (d - n_hi) + 31) // 32
 
 
 def key_bytes(w) -> int:
-    rec = 4 * ((w["k_idx"] * w["d"] + 31) // 32 + (w["d"] + 31) // 32)
+    rec = 4 * (_code_words(w["d"], w["k_idx"], w.get("k_nhi", 0)) + (w["d"] + 31) // 32)
     return w["n_seq"] * w["hkv"] * w["T"] * (rec + 8)
 
 
 def value_bytes(w) -> int:
-    rec = 4 * ((w["v_idx"] * w["d"] + 31) // 32)
+    rec = 4 * _code_words(w["d"], w["v_idx"], w.get("v_nhi", 0))
     return w["n_seq"] * w["hkv"] * w["T"] * (rec + 4)
+
+
+def fit_codebooks(tqb, d, idx, n_hi):
+    """The codebook argument of a cache: 2^idx centroids, followed for a mixed-rate cache by
+    the 2^(idx+1) centroids of its wider group (tq_codebook_fit, host setup)."""
+    c = tqb.tq_codebook_fit(d, idx)
+    return torch.cat([c, tqb.tq_codebook_fit(d, idx + 1)]) if n_hi else c
 
 
 def rank_seed(rank: int) -> int:
@@ -210,11 +231,12 @@ def run_tq(args, rank, world, local_rank):
     k, v, q = w["gen"](dev, rank_seed(rank))
     Pi = syn.rotation(d).to(dev)
     S = syn.sketch(d).to(dev)
-    ck = tqb.tq_codebook_fit(d, w["k_idx"]).to(dev)
-    cv = tqb.tq_codebook_fit(d, w["v_idx"]).to(dev)
+    ck = fit_codebooks(tqb, d, w["k_idx"], w.get("k_nhi", 0)).to(dev)
+    cv = fit_codebooks(tqb, d, w["v_idx"], w.get("v_nhi", 0)).to(dev)
     SPiT = tqb.tq_sketch_rotation(Pi, S)
-    kc = tqb.PackedCache.empty(d, w["k_idx"], True, w["n_seq"], w["hkv"], w["T"], device=dev)
-    vc = tqb.PackedCache.empty(d, w["v_idx"], False, w["n_seq"], w["hkv"], w["T"], device=dev)
+    kc = tqb.PackedCache.empty(d, w["k_idx"], True, w["n_seq"], w["hkv"], w["T"], device=dev, n_hi=w.get("k_nhi", 0))
+    vc = tqb.PackedCache.empty(d, w["v_idx"], False, w["n_seq"], w["hkv"], w["T"], device=dev,
+                               n_hi=w.get("v_nhi", 0))
     logits = torch.empty((w["n_seq"], w["hq"], w["T"]), dtype=torch.float32, device=dev)
     out = torch.empty((w["n_seq"], w["hq"], d), dtype=torch.float32, device=dev)
     ws_l = torch.empty(tqb.tq_logits_workspace_size(kc, w["hq"]), dtype=torch.uint8, device=dev)
@@ -404,7 +426,8 @@ def run_tq(args, rank, world, local_rank):
 
 def decode_roof(ms, two_call_ms, nbytes, w, hbm, src_txt, traffic=None):
     """The one-call decode step against HBM: packed key + value bytes per call / its time."""
-    one_pass = w["hq"] == w["hkv"] and w["d"] == 128 and w["k_idx"] in (1, 2)
+    one_pass = (w["hq"] == w["hkv"] and w["d"] == 128 and w["k_idx"] in (1, 2) and not w.get("k_nhi")
+                and not w.get("v_nhi"))
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"kernel": "tq_decode_attend (" + ("query projection + fused logits/softmax.V pass + merge" if one_pass
                                               else "tq_logits + tq_attend_v") + ")",
@@ -800,22 +823,20 @@ def oracle_sample_step(w, state):
     2048 values of one KV head; unpack + logits of that head's query group over
     all T keys of the head (pre-packed); softmax.V over the same head.
     Returns (packed key bytes scanned, logit seconds, quantize seconds, head-vectors quantized)."""
-    from oracle import turboquant as otq
-
     d = w["d"]
+    o = state["ops"]
     t0 = time.perf_counter()
-    ek = otq.quantize(state["k_rows"], state["Pi"], state["ck"], state["S"])
-    ev = otq.quantize(state["v_rows"], state["Pi"], state["cv"])
-    otq.pack(ek["idx"], ek["sign"], d, w["k_idx"], True)
-    otq.pack(ev["idx"], None, d, w["v_idx"], False)
+    ek = o["enc_k"](state["k_rows"])
+    ev = o["enc_v"](state["v_rows"])
+    o["pack_k"](ek)
+    o["pack_v"](ev)
     t1 = time.perf_counter()
-    gi, gs = otq.unpack(state["krec"], d, w["k_idx"], True)
-    lg = otq.logits(state["q"], state["Pi"], state["S"], state["ck"], state["kn"], state["kr"], gi, gs)
+    gi, gs = o["unpack_k"](state["krec"])
+    lg = o["logits"](state["q"], state["kn"], state["kr"], gi, gs)
     t2 = time.perf_counter()
-    vi, _ = otq.unpack(state["vrec"], d, w["v_idx"], False)
-    otq.attend_v(lg, 1.0 / math.sqrt(d), state["vn"], vi, state["Pi"], state["cv"])
-    rec = 4 * ((w["k_idx"] * d + 31) // 32 + (d + 31) // 32)
-    return state["krec"].shape[0] * (rec + 8), t2 - t1, t1 - t0, 2 * state["k_rows"].shape[0]
+    vi, _ = o["unpack_v"](state["vrec"])
+    o["attend"](lg, 1.0 / math.sqrt(d), state["vn"], vi)
+    return key_bytes(w) // (w["n_seq"] * w["hkv"]), t2 - t1, t1 - t0, 2 * state["k_rows"].shape[0]
 
 
 def oracle_nn_step(w, state):
@@ -863,18 +884,35 @@ def oracle_state(w):
     G = w["hq"] // w["hkv"]
     Pi = syn.rotation(d).double().numpy()
     S = syn.sketch(d).double().numpy()
-    ck = ocb.fit_codebook(d, w["k_idx"])[0]
-    cv = ocb.fit_codebook(d, w["v_idx"])[0]
+    from oracle import mixed_rate as omr
+
+    ki, vi, km, vm = w["k_idx"], w["v_idx"], w.get("k_nhi", 0), w.get("v_nhi", 0)
+    ck = ocb.fit_codebook(d, ki)[0]
+    cv = ocb.fit_codebook(d, vi)[0]
+    if km or vm:   # mixed rate: the codebooks of both widths
+        ckh, cvh = ocb.fit_codebook(d, ki + 1)[0], ocb.fit_codebook(d, vi + 1)[0]
+        ops = {"enc_k": lambda x: omr.quantize(x, Pi, ck, ckh, km, S), "enc_v": lambda x: omr.quantize(x, Pi, cv, cvh, vm),
+               "pack_k": lambda e: omr.pack(e["idx"], e["sign"], d, ki, km, True),
+               "pack_v": lambda e: omr.pack(e["idx"], None, d, vi, vm, False),
+               "unpack_k": lambda r: omr.unpack(r, d, ki, km, True), "unpack_v": lambda r: omr.unpack(r, d, vi, vm, False),
+               "logits": lambda q, n, r, i, sg: omr.logits(q, Pi, S, ck, ckh, km, n, r, i, sg),
+               "attend": lambda lg, sc, n, i: omr.attend_v(lg, sc, n, i, Pi, cv, cvh, vm)}
+    else:
+        ops = {"enc_k": lambda x: otq.quantize(x, Pi, ck, S), "enc_v": lambda x: otq.quantize(x, Pi, cv),
+               "pack_k": lambda e: otq.pack(e["idx"], e["sign"], d, ki, True),
+               "pack_v": lambda e: otq.pack(e["idx"], None, d, vi, False),
+               "unpack_k": lambda r: otq.unpack(r, d, ki, True), "unpack_v": lambda r: otq.unpack(r, d, vi, False),
+               "logits": lambda q, n, r, i, sg: otq.logits(q, Pi, S, ck, n, r, i, sg),
+               "attend": lambda lg, sc, n, i: otq.attend_v(lg, sc, n, i, Pi, cv)}
     g = torch.Generator().manual_seed(5)
     # one KV head of T keys/values of the workload's law, packed once by the oracle
     kfull = torch.randn(T, d, generator=g).to(w["dtype"]).double().numpy()
     vfull = torch.randn(T, d, generator=g).to(w["dtype"]).double().numpy()
-    ek = otq.quantize(kfull, Pi, ck, S)
-    ev = otq.quantize(vfull, Pi, cv)
-    return {"Pi": Pi, "S": S, "ck": ck, "cv": cv,
-            "k_rows": kfull[:2048], "v_rows": vfull[:2048],
-            "krec": otq.pack(ek["idx"], ek["sign"], d, w["k_idx"], True), "kn": ek["norm"], "kr": ek["rnorm"],
-            "vrec": otq.pack(ev["idx"], None, d, w["v_idx"], False), "vn": ev["norm"],
+    ek = ops["enc_k"](kfull)
+    ev = ops["enc_v"](vfull)
+    return {"Pi": Pi, "S": S, "ops": ops, "k_rows": kfull[:2048], "v_rows": vfull[:2048],
+            "krec": ops["pack_k"](ek), "kn": ek["norm"], "kr": ek["rnorm"],
+            "vrec": ops["pack_v"](ev), "vn": ev["norm"],
             "q": torch.randn(G, d, generator=g).double().numpy()}
 
 

@@ -43,6 +43,20 @@
  *   Records of one (sequence, head) are contiguous in token order; the array
  *   is [n_seq][n_kv_heads][capacity][R]. Norms are separate float arrays
  *   [n_seq][n_kv_heads][capacity].
+ *
+ * Fractional bits per channel (zubnet.ai, title and paragraph 2: 3.5 and 2.5
+ * bits per channel; the pages do not say how a fractional rate is reached).
+ * This library's reading: a cache with n_hi = m > 0 gives the first m rotated
+ * coordinates idx_bits + 1 code bits and the other d - m coordinates idx_bits,
+ * each group quantized with the Lloyd-Max codebook of the same coordinate law at
+ * its own width; the average rate is idx_bits + m/d code bits per coordinate
+ * (plus the sign bit for keys). Keys at 3.5 bits per channel: idx_bits 2,
+ * m = d/2; values at 3.5: idx_bits 3, m = d/2. The code of coordinate i < m sits
+ * at stream bits [(idx_bits+1) i, (idx_bits+1)(i+1)), the code of i >= m at
+ * [(idx_bits+1) m + idx_bits (i-m), ... + idx_bits); index_words =
+ * ceil(((idx_bits+1) m + idx_bits (d-m)) / 32); the sign field follows as above.
+ * Every entry point that takes a codebook then takes both: 2^idx_bits floats of
+ * the idx_bits codebook followed by 2^(idx_bits+1) floats of the wider one.
  */
 #ifndef TQ_H
 #define TQ_H
@@ -77,7 +91,9 @@ typedef struct {
   int32_t qjl;        /* 1: key cache (sign field + rnorm), 0: value cache (MSE only)  */
   int32_t n_seq;      /* sequences (batch)                                             */
   int32_t n_kv_heads; /* KV heads per sequence                                         */
-  int32_t reserved;   /* must be 0                                                     */
+  int32_t n_hi;       /* mixed rate: the first n_hi rotated coordinates carry idx_bits+1 */
+                      /* code bits, the others idx_bits (0 = integer rate; else a      */
+                      /* multiple of 32 below d, with idx_bits + 1 <= 4)               */
   int64_t capacity;   /* token slots per (sequence, head)                              */
   uint32_t *records;  /* [n_seq][n_kv_heads][capacity][tq_record_words(d,idx_bits,qjl)] */
   float *norm;        /* [n_seq][n_kv_heads][capacity]  ||x||                          */
@@ -86,6 +102,11 @@ typedef struct {
 
 /* Words per record for the layout above; -1 if (d, idx_bits) is unsupported. */
 int32_t tq_record_words(int32_t d, int32_t idx_bits, int32_t qjl);
+
+/* Words per record of a mixed-rate cache (n_hi coordinates at idx_bits + 1 code
+ * bits, see the layout above); n_hi = 0 gives tq_record_words. -1 if unsupported
+ * (n_hi not a multiple of 32 in [0, d), or idx_bits + 1 > 4 with n_hi > 0). */
+int32_t tq_record_words_mixed(int32_t d, int32_t idx_bits, int32_t n_hi, int32_t qjl);
 
 /* Lloyd-Max codebook for the coordinate law of a uniform point on the unit
  * sphere S^{d-1}, density proportional to (1 - y^2)^((d-3)/2) on [-1, 1]
@@ -110,7 +131,8 @@ tq_status tq_sketch_rotation(int32_t d, const float *Pi, const float *S, float *
  *   Pi:       [d][d] float rotation, y = Pi x / ||x||.
  *   SPiT:     [d][d] float, S Pi^T (see tq_sketch_rotation); ignored (may be NULL)
  *             for a value cache.
- *   codebook: 2^idx_bits ascending floats; code_i = #{j : y_i > (c_j + c_{j+1})/2}.
+ *   codebook: 2^idx_bits ascending floats; code_i = #{j : y_i > (c_j + c_{j+1})/2}
+ *             (mixed rate: the two codebooks, see the layout above).
  * For each vector: norm = ||x||; y = Pi x/||x||; codes; keys also store
  * rnorm = ||y - c[code]|| and sign bits of SPiT (y - c[code]). A zero vector
  * stores norm 0, rnorm 0, codes of y = 0 and all sign bits 1.
@@ -129,7 +151,8 @@ size_t tq_logits_workspace_size(const tq_cache *k, int32_t n_q_heads);
  * where q = q[s][h] and the key cache head is h / (n_q_heads / n_kv_heads).
  *   q:       [n_seq][n_q_heads][d] float.
  *   logits:  [n_seq][n_q_heads][n_tokens] float.
- *   Pi, S:   [d][d] float; codebook: 2^idx_bits floats (the key codebook).
+ *   Pi, S:   [d][d] float; codebook: 2^idx_bits floats (the key codebook; a
+ *            mixed-rate cache takes its two codebooks, see the layout above).
  * n_q_heads must be a positive multiple of k->n_kv_heads; k->qjl must be 1.
  * workspace: >= tq_logits_workspace_size bytes, 256-byte aligned. */
 tq_status tq_logits(const tq_cache *k, const float *q, int32_t n_q_heads, int64_t n_tokens,
@@ -145,6 +168,7 @@ size_t tq_attend_workspace_size(const tq_cache *v, int32_t n_q_heads, int64_t n_
  *   p = softmax_t(scale * logits[s][h][t]),
  *   out[s][h] = Pi^T sum_t p_t * norm_t * c[code_t]     (rotation undone once).
  *   logits: [n_seq][n_q_heads][n_tokens] float; out: [n_seq][n_q_heads][d] float.
+ *   codebook: the value codebook (two for a mixed-rate cache, see the layout above).
  *   v->qjl must be 0. n_tokens == 0 writes zeros. Shapes with n_seq x n_kv_heads x
  *   ceil(min(group, 4)-head blocks) above 65535 return TQ_ERR_UNSUPPORTED.
  * workspace: >= tq_attend_workspace_size bytes, 256-byte aligned. */
@@ -167,7 +191,9 @@ size_t tq_decode_workspace_size(const tq_cache *k, const tq_cache *v, int32_t n_
  * tq_logits and tq_attend_v inside the workspace and give the same results.
  *   k: key cache (qjl = 1); v: value cache (qjl = 0), same d, n_seq, n_kv_heads.
  *   q: [n_seq][n_q_heads][d] float; out: [n_seq][n_q_heads][d] float.
- *   Pi, S: [d][d] float; codebook_k / codebook_v: 2^idx_bits floats of each cache.
+ *   Pi, S: [d][d] float; codebook_k / codebook_v: 2^idx_bits floats of each cache
+ *   (both codebooks of a mixed-rate cache, see the layout above; mixed-rate caches
+ *   run the two calls).
  * n_q_heads must be a positive multiple of n_kv_heads; n_tokens <= both
  * capacities (n_tokens == 0 writes zeros); scale finite.
  * workspace: >= tq_decode_workspace_size bytes, 256-byte aligned; its status
@@ -188,7 +214,7 @@ size_t tq_nn_workspace_size(const tq_cache *db, int32_t n_queries, int64_t n_db)
  *   score(a, j) = norm_j * ( <Pi q_a, c[code_j]> + rnorm_j * sqrt(pi/2)/d * <S q_a, 2 sign_j - 1> ),
  * the key estimator of tq_logits, in order of decreasing score (equal scores:
  * lower j first).
- *   db: key cache (qjl = 1) with n_seq = n_kv_heads = 1, d 128 or 200,
+ *   db: key cache (qjl = 1, n_hi = 0) with n_seq = n_kv_heads = 1, d 128 or 200,
  *       idx_bits 1..3, filled by tq_quantize_append; its norm and rnorm
  *       arrays 16-byte aligned (they are read by bulk copies).
  *   queries: [n_queries][d] float; Pi, S: [d][d] float, 16-byte aligned;

@@ -6,7 +6,8 @@ cache), ``tq_logits`` (attention logits on the packed keys) and
 ``tq_attend_v`` (softmax-weighted packed values), ``tq_decode_attend`` (the
 three decode steps in one call, one pass over the tokens where the shapes allow),
 ``tq_nn_search`` (top-k inner-product search over a packed key stream),
-plus the setup helpers
+mixed-rate caches for fractional bits per channel (``PackedCache.empty(...,
+n_hi=...)``, ``tq_record_words_mixed``), plus the setup helpers
 ``tq_codebook_fit`` and ``tq_sketch_rotation``. All compute runs in the CUDA
 kernels of ``csrc/`` built for sm_100a.
 """
@@ -39,6 +40,7 @@ from ._binding import (  # noqa: F401
     tq_nn_workspace_size,
     tq_quantize_append,
     tq_record_words,
+    tq_record_words_mixed,
     tq_sketch_rotation,
     tq_workspace_status,
 )

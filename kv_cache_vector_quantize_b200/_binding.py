@@ -35,7 +35,7 @@ class TQError(RuntimeError):
 
 class TqCacheDesc(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("idx_bits", ctypes.c_int32), ("qjl", ctypes.c_int32),
-                ("n_seq", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("n_seq", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("n_hi", ctypes.c_int32),
                 ("capacity", ctypes.c_int64), ("records", ctypes.c_void_p), ("norm", ctypes.c_void_p),
                 ("rnorm", ctypes.c_void_p)]
 
@@ -49,6 +49,7 @@ def _load() -> ctypes.CDLL:
     D = ctypes.POINTER(TqCacheDesc)
     sig = {
         "tq_record_words": (I32, [I32, I32, I32]),
+        "tq_record_words_mixed": (I32, [I32, I32, I32, I32]),
         "tq_codebook_fit": (I32, [I32, I32, P]),
         "tq_sketch_rotation": (I32, [I32, P, P, P, P]),
         "tq_quantize_append": (I32, [D, P, I32, I64, I64, P, P, P, P]),
@@ -126,17 +127,23 @@ class PackedCache:
     records: torch.Tensor            # int32 view of the uint32 words [n_seq, n_kv_heads, capacity, R]
     norm: torch.Tensor               # float32 [n_seq, n_kv_heads, capacity]
     rnorm: torch.Tensor | None
+    n_hi: int = 0                    # mixed rate: leading coordinates at idx_bits + 1 code bits
 
     @classmethod
-    def empty(cls, d, idx_bits, qjl, n_seq, n_kv_heads, capacity, device="cuda"):
-        rw = tq_record_words(d, idx_bits, qjl)
+    def empty(cls, d, idx_bits, qjl, n_seq, n_kv_heads, capacity, device="cuda", n_hi=0):
+        rw = tq_record_words_mixed(d, idx_bits, n_hi, qjl)
         rec = torch.zeros((n_seq, n_kv_heads, capacity, rw), dtype=torch.int32, device=device)
         norm = torch.zeros((n_seq, n_kv_heads, capacity), dtype=torch.float32, device=device)
         rnorm = torch.zeros_like(norm) if qjl else None
-        return cls(d, idx_bits, bool(qjl), n_seq, n_kv_heads, capacity, rec, norm, rnorm)
+        return cls(d, idx_bits, bool(qjl), n_seq, n_kv_heads, capacity, rec, norm, rnorm, int(n_hi))
+
+    @property
+    def codebook_len(self) -> int:
+        """Floats of the codebook argument: 2^idx_bits, plus 2^(idx_bits+1) for a mixed-rate cache."""
+        return (1 << self.idx_bits) + ((2 << self.idx_bits) if self.n_hi else 0)
 
     def desc(self) -> TqCacheDesc:
-        return TqCacheDesc(self.d, self.idx_bits, int(self.qjl), self.n_seq, self.n_kv_heads, 0, self.capacity,
+        return TqCacheDesc(self.d, self.idx_bits, int(self.qjl), self.n_seq, self.n_kv_heads, self.n_hi, self.capacity,
                            self.records.data_ptr(), self.norm.data_ptr(),
                            self.rnorm.data_ptr() if self.rnorm is not None else None)
 
@@ -159,6 +166,13 @@ def tq_record_words(d: int, idx_bits: int, qjl) -> int:
     w = _lib.tq_record_words(d, idx_bits, int(qjl))
     if w < 0:
         raise TQError(TQ_ERR_UNSUPPORTED, f"unsupported d={d} idx_bits={idx_bits}")
+    return w
+
+
+def tq_record_words_mixed(d: int, idx_bits: int, n_hi: int, qjl) -> int:
+    w = _lib.tq_record_words_mixed(d, idx_bits, int(n_hi), int(qjl))
+    if w < 0:
+        raise TQError(TQ_ERR_UNSUPPORTED, f"unsupported d={d} idx_bits={idx_bits} n_hi={n_hi}")
     return w
 
 
@@ -189,7 +203,7 @@ def tq_quantize_append(cache: PackedCache, x: torch.Tensor, pos: int, Pi: torch.
     if x.dtype not in _DTYPE:
         raise ValueError(f"x dtype {x.dtype} unsupported")
     _need(Pi, "Pi", torch.float32, (cache.d, cache.d), cache.device)
-    _need(codebook, "codebook", torch.float32, (1 << cache.idx_bits,), cache.device)
+    _need(codebook, "codebook", torch.float32, (cache.codebook_len,), cache.device)
     if cache.qjl:
         _need(SPiT, "SPiT", torch.float32, (cache.d, cache.d), cache.device)
     desc = cache.desc()
@@ -212,7 +226,7 @@ def tq_logits(cache: PackedCache, q: torch.Tensor, n_tokens: int, Pi: torch.Tens
     _need(q, "q", torch.float32, device=cache.device)
     _need(Pi, "Pi", torch.float32, (cache.d, cache.d), cache.device)
     _need(S, "S", torch.float32, (cache.d, cache.d), cache.device)
-    _need(codebook, "codebook", torch.float32, (1 << cache.idx_bits,), cache.device)
+    _need(codebook, "codebook", torch.float32, (cache.codebook_len,), cache.device)
     if logits is None:
         logits = torch.empty((cache.n_seq, hq, n_tokens), dtype=torch.float32, device=cache.device)
     _need(logits, "logits", torch.float32, (cache.n_seq, hq, n_tokens), cache.device)
@@ -240,7 +254,7 @@ def tq_attend_v(cache: PackedCache, logits: torch.Tensor, scale: float, n_tokens
     hq = logits.shape[1]
     _need(logits, "logits", torch.float32, device=cache.device)
     _need(Pi, "Pi", torch.float32, (cache.d, cache.d), cache.device)
-    _need(codebook, "codebook", torch.float32, (1 << cache.idx_bits,), cache.device)
+    _need(codebook, "codebook", torch.float32, (cache.codebook_len,), cache.device)
     if out is None:
         out = torch.empty((cache.n_seq, hq, cache.d), dtype=torch.float32, device=cache.device)
     _need(out, "out", torch.float32, (cache.n_seq, hq, cache.d), cache.device)
@@ -270,8 +284,8 @@ def tq_decode_attend(kcache: PackedCache, vcache: PackedCache, q: torch.Tensor, 
     _need(q, "q", torch.float32, device=kcache.device)
     _need(Pi, "Pi", torch.float32, (kcache.d, kcache.d), kcache.device)
     _need(S, "S", torch.float32, (kcache.d, kcache.d), kcache.device)
-    _need(codebook_k, "codebook_k", torch.float32, (1 << kcache.idx_bits,), kcache.device)
-    _need(codebook_v, "codebook_v", torch.float32, (1 << vcache.idx_bits,), kcache.device)
+    _need(codebook_k, "codebook_k", torch.float32, (kcache.codebook_len,), kcache.device)
+    _need(codebook_v, "codebook_v", torch.float32, (vcache.codebook_len,), kcache.device)
     if out is None:
         out = torch.empty((kcache.n_seq, hq, kcache.d), dtype=torch.float32, device=kcache.device)
     _need(out, "out", torch.float32, (kcache.n_seq, hq, kcache.d), kcache.device)
@@ -301,7 +315,7 @@ def tq_nn_search(db: PackedCache, queries: torch.Tensor, n_db: int, Pi: torch.Te
     _need(queries, "queries", torch.float32, device=db.device)
     _need(Pi, "Pi", torch.float32, (db.d, db.d), db.device)
     _need(S, "S", torch.float32, (db.d, db.d), db.device)
-    _need(codebook, "codebook", torch.float32, (1 << db.idx_bits,), db.device)
+    _need(codebook, "codebook", torch.float32, (db.codebook_len,), db.device)
     if scores is None:
         scores = torch.empty((nq, k), dtype=torch.float32, device=db.device)
     if ids is None:

@@ -41,11 +41,10 @@ __device__ __forceinline__ float block_reduce(float v, float *red, bool is_max) 
 }
 
 // Shared memory of the chunk kernel: the chunk's records, the weights w[t][4],
-// the codebook, a reduction scratch and the per-phase accumulators.
-size_t chunk_smem(int d, int bits, int64_t chunk) {
-  const int rw = (bits * d + 31) / 32;
+// the codebooks, a reduction scratch and the per-phase accumulators.
+size_t chunk_smem(int d, int rw, int64_t chunk) {
   const int phases = kAThreads / (d / 4);
-  return (size_t)chunk * rw * 4 + (size_t)chunk * 4 * 4 + (16 + 32) * 4 + (size_t)phases * 4 * d * 4;
+  return (size_t)chunk * rw * 4 + (size_t)chunk * 4 * 4 + (32 + 32) * 4 + (size_t)phases * 4 * d * 4;
 }
 
 // One CTA per (token chunk, sequence, KV head, query block of <= 4 heads).
@@ -53,16 +52,18 @@ size_t chunk_smem(int d, int bits, int64_t chunk) {
 // coordinates of one token phase: per token it reads the code bits of its 4
 // coordinates once, looks up their centroids and updates 4 x (query heads)
 // accumulators with one 16-byte weight load. Phases are summed in a fixed
-// order (deterministic).
-template <int BITS>
+// order (deterministic). MIXED: a mixed-rate cache, whose first n_hi coordinates
+// carry BITS + 1 code bits (n_hi a multiple of 32, so a thread's 4 coordinates
+// are all in one group).
+template <int BITS, bool MIXED>
 __global__ void __launch_bounds__(kAThreads) attend_chunk_kernel(const AttendParams p) {
   constexpr int L = 1 << BITS;
   extern __shared__ __align__(16) float sm[];
   const int d = p.d, rw = p.rec_words;
   uint32_t *rec_s = reinterpret_cast<uint32_t *>(sm);          // [chunk][rw]
   float4 *w_s = reinterpret_cast<float4 *>(sm + p.chunk * rw);  // [chunk] (one lane per query head)
-  float *cbs = reinterpret_cast<float *>(w_s + p.chunk);         // [16]
-  float *red = cbs + 16;                                         // [32]
+  float *cbs = reinterpret_cast<float *>(w_s + p.chunk);         // [16] BITS codebook, [16] BITS + 1 codebook
+  float *red = cbs + 32;                                         // [32]
   float *accs = red + 32;                                        // [phases][4][d]
   const int tid = threadIdx.x;
   const int qb = blockIdx.y % p.qblocks;
@@ -76,6 +77,7 @@ __global__ void __launch_bounds__(kAThreads) attend_chunk_kernel(const AttendPar
   const size_t slot0 = (size_t)sk * p.capacity + t0;
 
   if (tid < L) cbs[tid] = p.codebook[tid];
+  if (MIXED && tid < 2 * L) cbs[16 + tid] = p.codebook[L + tid];
   // the chunk's records (contiguous in the cache) into shared memory
   const uint32_t *src = p.records + slot0 * rw;
   for (int e = tid; e < nt * rw; e += kAThreads) rec_s[e] = __ldg(src + e);
@@ -115,8 +117,21 @@ __global__ void __launch_bounds__(kAThreads) attend_chunk_kernel(const AttendPar
 #pragma unroll
     for (int qq = 0; qq < 4; ++qq) acc[a][qq] = 0.f;
   if (ph < phases) {
-    const int bit0 = BITS * i0, wd = bit0 >> 5, sh = bit0 & 31;
-    const bool two = sh + 4 * BITS > 32 && wd + 1 < rw;
+    // this thread's code width, first stream bit and codebook (compile-time unless MIXED)
+    int B = BITS, bit0 = BITS * i0;
+    const float *cbc = cbs;
+    if constexpr (MIXED) {
+      if (i0 < p.n_hi) {
+        B = BITS + 1;
+        bit0 = (BITS + 1) * i0;
+        cbc = cbs + 16;
+      } else {
+        bit0 = (BITS + 1) * p.n_hi + BITS * (i0 - p.n_hi);
+      }
+    }
+    const uint32_t msk = (1u << B) - 1u;
+    const int wd = bit0 >> 5, sh = bit0 & 31;
+    const bool two = sh + 4 * B > 32 && wd + 1 < rw;
     for (int t = ph; t < nt; t += phases) {
       const uint32_t *rec = rec_s + t * rw;
       const uint32_t lo = rec[wd], hi = two ? rec[wd + 1] : 0u;
@@ -124,7 +139,7 @@ __global__ void __launch_bounds__(kAThreads) attend_chunk_kernel(const AttendPar
       const float4 wt = w_s[t];
 #pragma unroll
       for (int a = 0; a < 4; ++a) {
-        const float cv = cbs[(bits >> (BITS * a)) & (L - 1)];
+        const float cv = cbc[(bits >> (B * a)) & msk];
         acc[a][0] = fmaf(wt.x, cv, acc[a][0]);
         acc[a][1] = fmaf(wt.y, cv, acc[a][1]);
         acc[a][2] = fmaf(wt.z, cv, acc[a][2]);
@@ -233,9 +248,9 @@ __global__ void __launch_bounds__(kCThreads) attend_combine_kernel(const float *
   }
 }
 
-template <int BITS>
+template <int BITS, bool MIXED>
 cudaError_t launch_a(const AttendParams &p, int n_seq, size_t smem, cudaStream_t st) {
-  auto kern = attend_chunk_kernel<BITS>;
+  auto kern = attend_chunk_kernel<BITS, MIXED>;
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.n_chunks, n_seq * p.n_kv_heads * p.qblocks);
@@ -246,11 +261,18 @@ cudaError_t launch_a(const AttendParams &p, int n_seq, size_t smem, cudaStream_t
 }  // namespace
 
 cudaError_t launch_attend(const AttendParams &p, int bits, int n_seq, size_t smem, cudaStream_t st) {
+  if (p.n_hi > 0) {
+    switch (bits) {
+      case 1: return launch_a<1, true>(p, n_seq, smem, st);
+      case 2: return launch_a<2, true>(p, n_seq, smem, st);
+      default: return launch_a<3, true>(p, n_seq, smem, st);
+    }
+  }
   switch (bits) {
-    case 1: return launch_a<1>(p, n_seq, smem, st);
-    case 2: return launch_a<2>(p, n_seq, smem, st);
-    case 3: return launch_a<3>(p, n_seq, smem, st);
-    default: return launch_a<4>(p, n_seq, smem, st);
+    case 1: return launch_a<1, false>(p, n_seq, smem, st);
+    case 2: return launch_a<2, false>(p, n_seq, smem, st);
+    case 3: return launch_a<3, false>(p, n_seq, smem, st);
+    default: return launch_a<4, false>(p, n_seq, smem, st);
   }
 }
 
@@ -276,7 +298,7 @@ cudaError_t launch_combine(const float *partial, int rows, int n_chunks, int d, 
   return cudaLaunchKernelEx(&cfg, attend_combine_kernel, partial, n_chunks, d, Pi, out, pi_in_smem);
 }
 
-size_t attend_chunk_smem(int d, int bits, int64_t chunk) { return chunk_smem(d, bits, chunk); }
+size_t attend_chunk_smem(int d, int rec_words, int64_t chunk) { return chunk_smem(d, rec_words, chunk); }
 
 }  // namespace tq
 

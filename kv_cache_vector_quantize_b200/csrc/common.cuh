@@ -63,6 +63,7 @@ struct QuantParams {
   int d;
   int rec_words;
   int idx_words;
+  int n_hi;                 // mixed rate: leading coordinates at bits + 1 code bits (0: integer rate)
 };
 
 struct LogitsParams {
@@ -85,6 +86,7 @@ struct LogitsParams {
   int group;                // n_q_heads / n_kv_heads
   int q_per_cta;            // query heads handled by one CTA
   int qblocks;              // ceil(group / q_per_cta)
+  int n_hi;                 // mixed rate: leading coordinates at bits + 1 code bits (0: integer rate)
 };
 
 // Lookup tables of the grouped-query scan (logits_gqa.cu).
@@ -117,6 +119,7 @@ struct AttendParams {
   int group;
   int q_per_cta;
   int qblocks;
+  int n_hi;                 // mixed rate: leading coordinates at bits + 1 code bits (0: integer rate)
 };
 
 // launchers (defined in the .cu files)
@@ -126,7 +129,7 @@ cudaError_t launch_quantize_tc(const QuantParams &p, int bits, bool qjl, bool f1
 cudaError_t launch_qprep(const float *q, int rows, int d, const float *Pi, const float *S,
                          float *qrot, float *qsk, uint32_t *status, cudaStream_t st);
 cudaError_t launch_logits(const LogitsParams &p, int bits, int n_seq, int n_chunks, size_t smem, cudaStream_t st);
-size_t logits_smem_per_query(int d, int bits);
+size_t logits_smem_per_query(int d, int bits, int n_hi = 0);
 int logits_fast_stages(int bits, int q, size_t limit);
 cudaError_t launch_logits_fast(const LogitsParams &p, int bits, int n_seq, size_t limit, cudaStream_t st);
 bool gqa_supported(int d, int bits, int group);
@@ -158,7 +161,7 @@ cudaError_t launch_status_or(uint32_t *dst, const uint32_t *a, const uint32_t *b
 bool attend_fast_supported(int d, int bits, int q_per_cta, const void *records);
 int64_t attend_fast_chunk(int64_t n_tokens, int units);
 cudaError_t launch_attend_fast(const AttendParams &p, int bits, int n_seq, cudaStream_t st);
-size_t attend_chunk_smem(int d, int bits, int64_t chunk);
+size_t attend_chunk_smem(int d, int rec_words, int64_t chunk);
 cudaError_t launch_combine(const float *partial, int rows, int n_chunks, int d, const float *Pi,
                            float *out, cudaStream_t st);
 // Nearest-neighbour search (nn_search.cu): running top-k of the key estimator over one packed

@@ -148,6 +148,100 @@ __global__ void __launch_bounds__(kLThreads) logits_kernel(const LogitsParams p)
   }
 }
 
+// Mixed-rate keys: the first n_hi coordinates carry BL + 1 code bits, the rest BL,
+// codes back to back in the stream (n_hi a multiple of 32, so both groups start on a
+// key boundary). The same estimator with one set of index tables per group: the
+// high group's keys of Keys<BL + 1> at stream bits KB_h j (coordinates G_h j ...),
+// the low group's keys of Keys<BL> at stream bits (BL + 1) n_hi + KB_l j
+// (coordinates n_hi + G_l j ...), and the sign tables as above.
+template <int BL>
+__global__ void __launch_bounds__(kLThreads) logits_mixed_kernel(const LogitsParams p) {
+  constexpr int BH = BL + 1;
+  using KH = Keys<BH>;
+  using KL = Keys<BL>;
+  constexpr int LL = 1 << BL, LH = 1 << BH;
+  extern __shared__ __align__(16) float tab[];
+  __shared__ float cbl[16], cbh[16];
+  const int tid = threadIdx.x;
+  const int qb = blockIdx.y % p.qblocks;
+  const int sk = blockIdx.y / p.qblocks;
+  const int seq = sk / p.n_kv_heads, kvh = sk - seq * p.n_kv_heads;
+  const int h0 = kvh * p.group + qb * p.q_per_cta;
+  const int nq = min(p.q_per_cta, p.group - qb * p.q_per_cta);
+  const int d = p.d, m = p.n_hi;
+  const int nkh = m / KH::G, nkl = (d - m) / KL::G, ns = d / 8;
+  const int lo_bit0 = BH * m;
+  const int per_q = nkh * KH::E + nkl * KL::E + ns * 256;
+  const float kappa = 1.2533141373155003f / (float)d;   // sqrt(pi/2) / d
+
+  if (tid < LL) cbl[tid] = p.codebook[tid];
+  if (tid < LH) cbh[tid] = p.codebook[LL + tid];
+  __syncthreads();
+  for (int qq = 0; qq < nq; ++qq) {
+    const size_t qrow = ((size_t)seq * p.n_q_heads + h0 + qq) * d;
+    const float *qr = p.qrot + qrow;
+    const float *qs = p.qsk + qrow;
+    float *th = tab + (size_t)qq * per_q;
+    for (int e = tid; e < nkh * KH::E; e += kLThreads) {
+      const int j = e / KH::E, key = e - j * KH::E;
+      float v = 0.f;
+#pragma unroll
+      for (int c = 0; c < KH::G; ++c) v = fmaf(__ldg(qr + j * KH::G + c), cbh[(key >> (BH * c)) & (LH - 1)], v);
+      th[e] = v;
+    }
+    float *tl = th + nkh * KH::E;
+    for (int e = tid; e < nkl * KL::E; e += kLThreads) {
+      const int j = e / KL::E, key = e - j * KL::E;
+      float v = 0.f;
+#pragma unroll
+      for (int c = 0; c < KL::G; ++c) v = fmaf(__ldg(qr + m + j * KL::G + c), cbl[(key >> (BL * c)) & (LL - 1)], v);
+      tl[e] = v;
+    }
+    float *ts = tl + nkl * KL::E;
+    for (int e = tid; e < ns * 256; e += kLThreads) {
+      const int j = e >> 8, b = e & 255;
+      float v = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float sv = __ldg(qs + 8 * j + c);
+        v += ((b >> c) & 1) ? sv : -sv;
+      }
+      ts[e] = kappa * v;
+    }
+  }
+  __syncthreads();
+
+  const int64_t t0 = (int64_t)blockIdx.x * p.chunk;
+  const int64_t t1 = min(p.n_tokens, t0 + p.chunk);
+  const int sw = (d + 31) / 32;
+  for (int64_t t = t0 + tid; t < t1; t += kLThreads) {
+    const size_t slot = (size_t)sk * p.capacity + t;
+    const uint32_t *rec = p.records + slot * p.rec_words;
+    const float n = __ldg(p.norm + slot), rho = __ldg(p.rnorm + slot);
+    for (int qq = 0; qq < nq; ++qq) {
+      const float *th = tab + (size_t)qq * per_q;
+      const float *tl = th + nkh * KH::E;
+      const float *ts = tl + nkl * KL::E;
+      float ai = 0.f, as = 0.f;
+      for (int j = 0; j < nkh; ++j) ai += th[j * KH::E + stream_bits(rec, KH::KB * j, KH::KB, p.idx_words)];
+      for (int j = 0; j < nkl; ++j)
+        ai += tl[j * KL::E + stream_bits(rec, lo_bit0 + KL::KB * j, KL::KB, p.idx_words)];
+      for (int j = 0; j < ns; ++j) as += ts[j * 256 + stream_bits(rec + p.idx_words, 8 * j, 8, sw)];
+      p.logits[((size_t)seq * p.n_q_heads + h0 + qq) * p.n_tokens + t] = n * fmaf(rho, as, ai);
+    }
+  }
+}
+
+template <int BL>
+cudaError_t launch_lm(const LogitsParams &p, int n_seq, int n_chunks, size_t smem, cudaStream_t st) {
+  auto kern = logits_mixed_kernel<BL>;
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(n_chunks, n_seq * p.n_kv_heads * p.qblocks);
+  kern<<<grid, kLThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
 template <int BITS>
 cudaError_t launch_l(const LogitsParams &p, int n_seq, int n_chunks, size_t smem, cudaStream_t st) {
   auto kern = logits_kernel<BITS>;
@@ -160,10 +254,12 @@ cudaError_t launch_l(const LogitsParams &p, int n_seq, int n_chunks, size_t smem
 
 }  // namespace
 
-size_t logits_smem_per_query(int d, int bits) {
-  int g = bits == 1 ? 8 : bits == 2 ? 4 : 2;
-  int kb = g * bits;
-  return ((size_t)(d / g) * ((size_t)1 << kb) + (size_t)(d / 8) * 256) * sizeof(float);
+size_t logits_smem_per_query(int d, int bits, int n_hi) {
+  auto tables = [](int coords, int b) {
+    const int g = b == 1 ? 8 : b == 2 ? 4 : 2;
+    return (size_t)(coords / g) * ((size_t)1 << (g * b));
+  };
+  return (tables(n_hi, bits + 1) + tables(d - n_hi, bits) + (size_t)(d / 8) * 256) * sizeof(float);
 }
 
 cudaError_t launch_qprep(const float *q, int rows, int d, const float *Pi, const float *S, float *qrot, float *qsk,
@@ -173,6 +269,13 @@ cudaError_t launch_qprep(const float *q, int rows, int d, const float *Pi, const
 }
 
 cudaError_t launch_logits(const LogitsParams &p, int bits, int n_seq, int n_chunks, size_t smem, cudaStream_t st) {
+  if (p.n_hi > 0) {
+    switch (bits) {
+      case 1: return launch_lm<1>(p, n_seq, n_chunks, smem, st);
+      case 2: return launch_lm<2>(p, n_seq, n_chunks, smem, st);
+      default: return launch_lm<3>(p, n_seq, n_chunks, smem, st);
+    }
+  }
   switch (bits) {
     case 1: return launch_l<1>(p, n_seq, n_chunks, smem, st);
     case 2: return launch_l<2>(p, n_seq, n_chunks, smem, st);

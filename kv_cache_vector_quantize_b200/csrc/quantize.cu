@@ -42,7 +42,7 @@ template <int DP, bool QJL>
 constexpr size_t quant_smem_bytes() {
   using Lay = QLayout<DP>;
   size_t f = (size_t)Lay::kMatFloats * ((QJL && Lay::kResident) ? 2 : 1)
-           + (size_t)kQTile * Lay::XS + 32;
+           + (size_t)kQTile * Lay::XS + 64;
   return f * sizeof(float) + (size_t)kQTile * kMaxRecWords * sizeof(uint32_t);
 }
 
@@ -108,14 +108,20 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_kernel(const QuantParam
   float *matP = smem;
   float *matM = (QJL && Lay::kResident) ? smem + Lay::kMatFloats : smem;
   float *xs = smem + Lay::kMatFloats * ((QJL && Lay::kResident) ? 2 : 1);
-  float *cb = xs + kQTile * Lay::XS;                         // [16] centroids, [16] thresholds
-  uint32_t *rs = reinterpret_cast<uint32_t *>(cb + 32);      // [kQTile][rec_words]
+  // [16] centroids and [16] thresholds of the `bits` codebook, then the same of the
+  // bits + 1 codebook of a mixed-rate cache (unused thresholds +huge)
+  float *cb = xs + kQTile * Lay::XS;
+  uint32_t *rs = reinterpret_cast<uint32_t *>(cb + 64);      // [kQTile][rec_words]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int d = p.d, L = 1 << bits, rw = p.rec_words, iw = p.idx_words;
+  const int LH = p.n_hi > 0 ? 2 * L : 0;                    // levels of the wider codebook
+  const int mhi = p.n_hi / 32;                              // 32-column groups at bits + 1 code bits
   if (tid < L) cb[tid] = p.codebook[tid];
+  if (tid < LH) cb[32 + tid] = p.codebook[L + tid];
   __syncthreads();
   if (tid < L - 1) cb[16 + tid] = 0.5f * (cb[tid] + cb[tid + 1]);
+  if (tid < 15) cb[48 + tid] = tid < LH - 1 ? 0.5f * (cb[32 + tid] + cb[32 + tid + 1]) : 3.0e38f;
   if constexpr (Lay::kResident) {
     load_matrix_chunk<DP>(matP, p.Pi, d, 0);
     if constexpr (QJL) load_matrix_chunk<DP>(matM, p.SPiT, d, 0);
@@ -164,21 +170,31 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_kernel(const QuantParam
         const int col = lane + 32 * m;
         const bool valid = col < d;
         const float y = acc[i][m] * inv;
+        // group m (32 columns) is at bits + 1 code bits when m < mhi (warp-uniform)
+        const bool ghi = m < mhi;
+        const int gb = ghi ? bits + 1 : bits;
+        const int gbase = ghi ? (bits + 1) * m : (bits + 1) * mhi + bits * (m - mhi);
+        const float *gcb = ghi ? cb + 32 : cb;
         uint32_t code = 0;
+        if (ghi) {
 #pragma unroll
-        for (int j = 0; j < 15; ++j) code += (y > th[j]) ? 1u : 0u;
+          for (int j = 0; j < 15; ++j) code += (y > cb[48 + j]) ? 1u : 0u;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 15; ++j) code += (y > th[j]) ? 1u : 0u;
+        }
         if (!valid) code = 0;
-        // code stream: the 32 columns of group m fill stream words [bits*m, bits*m + bits)
-        const int off = bits * lane, ww = off >> 5, sh = off & 31;
-        for (int w = 0; w < bits; ++w) {
+        // code stream: the 32 columns of group m fill stream words [gbase, gbase + gb)
+        const int off = gb * lane, ww = off >> 5, sh = off & 31;
+        for (int w = 0; w < gb; ++w) {
           uint32_t v = 0;
           if (ww == w) v = code << sh;
-          else if (ww + 1 == w && sh + bits > 32) v = code >> (32 - sh);
+          else if (ww + 1 == w && sh + gb > 32) v = code >> (32 - sh);
           const uint32_t word = __reduce_or_sync(0xffffffffu, v);
-          if (lane == 0 && bits * m + w < iw) rw_s[i * rw + bits * m + w] = word;
+          if (lane == 0 && gbase + w < iw) rw_s[i * rw + gbase + w] = word;
         }
         if constexpr (QJL) {
-          const float e = (valid && nrm[i] > 0.f) ? y - cb[code] : 0.f;
+          const float e = (valid && nrm[i] > 0.f) ? y - gcb[code] : 0.f;
           e2 = fmaf(e, e, e2);
           xw[i * Lay::XS + col] = e;    // residual replaces x (row private to this warp)
         }
@@ -264,7 +280,8 @@ __global__ void sketch_rotation_kernel(int d, const float *__restrict__ Pi, cons
 cudaError_t launch_quantize(const QuantParams &p, int bits, bool qjl, tq_dtype dtype, cudaStream_t st) {
   // bf16 / fp16 heads of 128 with 16-byte aligned rows and matrices take the tensor-core kernel (quantize_tc.cu)
   auto a16 = [](const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
-  if (p.d == 128 && (dtype == TQ_BF16 || dtype == TQ_FP16) && a16(p.x) && a16(p.Pi) && (!qjl || a16(p.SPiT))) {
+  if (p.d == 128 && p.n_hi == 0 && (dtype == TQ_BF16 || dtype == TQ_FP16) && a16(p.x) && a16(p.Pi) &&
+      (!qjl || a16(p.SPiT))) {
     const cudaError_t e = launch_quantize_tc(p, bits, qjl, dtype == TQ_FP16, st);
     if (e != cudaErrorNotSupported) return e;   // else (no tensor map for these rows): the FP32 kernel below
   }

@@ -60,9 +60,12 @@ tq_status check_cache(const tq_cache *c, const char *what) {
   if (c->idx_bits < 1 || c->idx_bits > kMaxBits)
     return fail(TQ_ERR_UNSUPPORTED, "%s: idx_bits=%d (need 1..%d)", what, c->idx_bits, kMaxBits);
   if (c->qjl != 0 && c->qjl != 1) return fail(TQ_ERR_INVALID, "%s: qjl=%d (need 0 or 1)", what, c->qjl);
-  if (c->n_seq <= 0 || c->n_kv_heads <= 0 || c->capacity < 0 || c->reserved != 0)
-    return fail(TQ_ERR_INVALID, "%s: n_seq=%d n_kv_heads=%d capacity=%lld reserved=%d", what, c->n_seq,
-                c->n_kv_heads, (long long)c->capacity, c->reserved);
+  if (c->n_seq <= 0 || c->n_kv_heads <= 0 || c->capacity < 0)
+    return fail(TQ_ERR_INVALID, "%s: n_seq=%d n_kv_heads=%d capacity=%lld", what, c->n_seq, c->n_kv_heads,
+                (long long)c->capacity);
+  if (c->n_hi != 0 && (c->n_hi < 0 || c->n_hi % 32 != 0 || c->n_hi >= c->d || c->idx_bits + 1 > kMaxBits))
+    return fail(TQ_ERR_UNSUPPORTED, "%s: n_hi=%d (need 0, or a multiple of 32 below d=%d with idx_bits + 1 <= %d)",
+                what, c->n_hi, c->d, kMaxBits);
   if (!c->records || !aligned(c->records, 16)) return fail(TQ_ERR_INVALID, "%s: records NULL or not 16-byte aligned", what);
   if (!c->norm || !aligned(c->norm, 4)) return fail(TQ_ERR_INVALID, "%s: norm NULL or misaligned", what);
   if (c->qjl && (!c->rnorm || !aligned(c->rnorm, 4))) return fail(TQ_ERR_INVALID, "%s: key cache needs rnorm", what);
@@ -70,8 +73,11 @@ tq_status check_cache(const tq_cache *c, const char *what) {
   return TQ_OK;
 }
 
-int idx_words_of(int d, int bits) { return (bits * d + 31) / 32; }
-int rec_words_of(int d, int bits, int qjl) { return idx_words_of(d, bits) + (qjl ? (d + 31) / 32 : 0); }
+// Code-stream words: n_hi coordinates at bits + 1 code bits, the others at bits (mixed rate).
+int idx_words_of(int d, int bits, int n_hi = 0) { return ((bits + 1) * n_hi + bits * (d - n_hi) + 31) / 32; }
+int rec_words_of(int d, int bits, int qjl, int n_hi = 0) {
+  return idx_words_of(d, bits, n_hi) + (qjl ? (d + 31) / 32 : 0);
+}
 
 struct LogitsPlan {
   int q_per_cta, qblocks, n_chunks;
@@ -82,7 +88,7 @@ struct LogitsPlan {
 LogitsPlan plan_logits(const tq_cache *k, int n_q_heads, int64_t n_tokens) {
   LogitsPlan pl{};
   const int group = n_q_heads / k->n_kv_heads;
-  const size_t per_q = logits_smem_per_query(k->d, k->idx_bits);
+  const size_t per_q = logits_smem_per_query(k->d, k->idx_bits, k->n_hi);
   const size_t budget = device_smem_optin() - 1024;
   int qpc = (int)(budget / per_q);
   if (qpc > group) qpc = group;
@@ -113,7 +119,7 @@ struct FastPlan {
 
 FastPlan plan_fast(const tq_cache *k, int n_q_heads) {
   FastPlan f{false, 0, 0};
-  if (k->d != 128 || k->idx_bits > 3 || !k->qjl) return f;
+  if (k->d != 128 || k->idx_bits > 3 || !k->qjl || k->n_hi != 0) return f;
   const int group = n_q_heads / k->n_kv_heads;
   const size_t limit = device_smem_optin() - 1024;
   int q = 0;
@@ -226,6 +232,12 @@ int32_t tq_record_words(int32_t d, int32_t idx_bits, int32_t qjl) {
   return rec_words_of(d, idx_bits, qjl);
 }
 
+int32_t tq_record_words_mixed(int32_t d, int32_t idx_bits, int32_t n_hi, int32_t qjl) {
+  if (tq_record_words(d, idx_bits, qjl) < 0) return -1;
+  if (n_hi != 0 && (n_hi < 0 || n_hi % 32 != 0 || n_hi >= d || idx_bits + 1 > kMaxBits)) return -1;
+  return rec_words_of(d, idx_bits, qjl, n_hi);
+}
+
 tq_status tq_codebook_fit(int32_t d, int32_t idx_bits, float *centroids_host) {
   g_err[0] = 0;
   if (d < 3 || d > 4096 || idx_bits < 1 || idx_bits > 8)
@@ -276,8 +288,9 @@ tq_status tq_quantize_append(const tq_cache *cache, const void *x, tq_dtype dtyp
   p.capacity = cache->capacity;
   p.pos = pos;
   p.d = cache->d;
-  p.rec_words = rec_words_of(cache->d, cache->idx_bits, cache->qjl);
-  p.idx_words = idx_words_of(cache->d, cache->idx_bits);
+  p.rec_words = rec_words_of(cache->d, cache->idx_bits, cache->qjl, cache->n_hi);
+  p.idx_words = idx_words_of(cache->d, cache->idx_bits, cache->n_hi);
+  p.n_hi = cache->n_hi;
   cudaError_t e = launch_quantize(p, cache->idx_bits, cache->qjl != 0, dtype, (cudaStream_t)stream);
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_quantize_append");
 }
@@ -296,7 +309,7 @@ LogitsWs logits_ws(const tq_cache *k, int32_t n_q_heads) {
   w.sigma = w.tables;
   w.total = w.tables;
   const int group = k->n_kv_heads > 0 ? n_q_heads / k->n_kv_heads : 0;
-  if (k->qjl && group * k->n_kv_heads == n_q_heads && gqa_supported(k->d, k->idx_bits, group)) {
+  if (k->qjl && k->n_hi == 0 && group * k->n_kv_heads == n_q_heads && gqa_supported(k->d, k->idx_bits, group)) {
     w.qh = group >= 4 ? 4 : 2;
     w.units = k->n_seq * k->n_kv_heads * (group / w.qh);
     w.sigma = w.tables + gqa_table_bytes(w.units);
@@ -362,8 +375,9 @@ tq_status tq_logits(const tq_cache *k, const float *q, int32_t n_q_heads, int64_
   p.capacity = k->capacity;
   p.chunk = pl.chunk;
   p.d = k->d;
-  p.rec_words = rec_words_of(k->d, k->idx_bits, 1);
-  p.idx_words = idx_words_of(k->d, k->idx_bits);
+  p.rec_words = rec_words_of(k->d, k->idx_bits, 1, k->n_hi);
+  p.idx_words = idx_words_of(k->d, k->idx_bits, k->n_hi);
+  p.n_hi = k->n_hi;
   p.n_kv_heads = k->n_kv_heads;
   p.n_q_heads = n_q_heads;
   p.group = n_q_heads / k->n_kv_heads;
@@ -438,7 +452,8 @@ tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale, int32
   p.n_chunks = (int)((n_tokens + kAttendChunk - 1) / kAttendChunk);
   p.scale = scale;
   p.d = v->d;
-  p.rec_words = rec_words_of(v->d, v->idx_bits, 0);
+  p.rec_words = rec_words_of(v->d, v->idx_bits, 0, v->n_hi);
+  p.n_hi = v->n_hi;
   p.n_kv_heads = v->n_kv_heads;
   p.n_q_heads = n_q_heads;
   p.group = group;
@@ -446,14 +461,14 @@ tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale, int32
   p.qblocks = (group + p.q_per_cta - 1) / p.q_per_cta;
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "tq_attend_v (status)");
-  if (attend_fast_supported(v->d, v->idx_bits, p.q_per_cta, v->records)) {
+  if (v->n_hi == 0 && attend_fast_supported(v->d, v->idx_bits, p.q_per_cta, v->records)) {
     // d = 128: tiles streamed by bulk copies, chunks sized to whole waves (never more chunks than
     // the 512-token split the workspace is sized for)
     p.chunk = attend_fast_chunk(n_tokens, v->n_seq * v->n_kv_heads * p.qblocks);
     p.n_chunks = (int)((n_tokens + p.chunk - 1) / p.chunk);
     e = launch_attend_fast(p, v->idx_bits, v->n_seq, (cudaStream_t)stream);
   } else {
-    e = launch_attend(p, v->idx_bits, v->n_seq, attend_chunk_smem(v->d, v->idx_bits, kAttendChunk),
+    e = launch_attend(p, v->idx_bits, v->n_seq, attend_chunk_smem(v->d, p.rec_words, kAttendChunk),
                       (cudaStream_t)stream);
   }
   if (e != cudaSuccess) return cuda_fail(e, "tq_attend_v (chunks)");
@@ -480,7 +495,8 @@ bool same_heads(const tq_cache *k, const tq_cache *v) {
 
 DecodeWs decode_ws(const tq_cache *k, const tq_cache *v, int n_q_heads, int64_t n_tokens) {
   DecodeWs w{};
-  w.fused = decode_fused_supported(k->d, k->idx_bits, v->idx_bits, n_q_heads, k->n_kv_heads, k->records,
+  w.fused = k->n_hi == 0 && v->n_hi == 0 &&
+            decode_fused_supported(k->d, k->idx_bits, v->idx_bits, n_q_heads, k->n_kv_heads, k->records,
                                    v->records, device_smem_optin() - 1024);
   const size_t rows = (size_t)k->n_seq * n_q_heads;
   if (w.fused) {
@@ -632,7 +648,7 @@ tq_status tq_nn_search(const tq_cache *db, const float *queries, int32_t n_queri
   if (db->n_seq != 1 || db->n_kv_heads != 1)
     return fail(TQ_ERR_INVALID, "tq_nn_search: the database is one stream (n_seq = n_kv_heads = 1), got %d x %d",
                 db->n_seq, db->n_kv_heads);
-  if (!nn_supported(db->d, db->idx_bits))
+  if (db->n_hi != 0 || !nn_supported(db->d, db->idx_bits))
     return fail(TQ_ERR_UNSUPPORTED, "tq_nn_search: d=%d idx_bits=%d (need d 128 or 200, idx_bits 1..3)", db->d,
                 db->idx_bits);
   if (k < 1 || k > kNnMaxK) return fail(TQ_ERR_INVALID, "tq_nn_search: k=%d (need 1..%d)", k, kNnMaxK);

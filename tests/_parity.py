@@ -146,3 +146,78 @@ def check_nn(gpu_s, gpu_i, q, Pi, S, codebook, rec, norm, rnorm, d, bits, k):
         assert np.all(oerr <= tol), f"query {a}: rank error {np.max(oerr / tol):.3g} x tolerance"
         worst = max(worst, float(np.max(err / tol_j)), float(np.max(oerr / tol)))
     return worst
+
+
+# ----------------------------------------------------------------------------
+# mixed rate (the first m coordinates at beta + 1 code bits): the same tolerances,
+# oracle/mixed_rate.py as the reference
+# ----------------------------------------------------------------------------
+
+def check_encoding_mixed(x, rec, norm, rnorm, Pi, S, c_lo, c_hi, d, beta, m, qjl):
+    from oracle import mixed_rate as omr
+
+    x = np.asarray(x, dtype=np.float64)
+    Pi = np.asarray(Pi, dtype=np.float64)
+    n = x.shape[0]
+    assert rec.shape == (n, omr.record_words(d, beta, m, qjl)), rec.shape
+    assert omr.padding_is_zero(rec, d, beta, m, qjl), "non-zero padding bits"
+    enc = omr.quantize(x, Pi, c_lo, c_hi, m, S if qjl else None)
+    ref_n = enc["norm"]
+    bad = np.abs(norm - ref_n) > NORM_RTOL * np.maximum(ref_n, 1e-30)
+    assert not bad.any(), f"norm mismatch at rows {np.nonzero(bad)[0][:10]}"
+    gi, gs = omr.unpack(rec, d, beta, m, qjl)
+    oi = enc["idx"]
+    idiff = gi != oi
+    t_lo = otq.thresholds_of(c_lo)
+    t_hi = otq.thresholds_of(c_hi)
+    lower = np.minimum(gi, oi)
+    between = np.empty(gi.shape)
+    between[:, :m] = t_hi[np.clip(lower[:, :m], 0, len(t_hi) - 1)]
+    between[:, m:] = t_lo[np.clip(lower[:, m:], 0, len(t_lo) - 1)]
+    near = np.abs(enc["y"] - between) <= FLIP_BAND
+    unexcused = idiff & ~((np.abs(gi - oi) == 1) & near)
+    assert not unexcused.any(), (
+        f"{unexcused.sum()} code mismatches that are not one-cell moves across a threshold within the band; "
+        f"first at {np.argwhere(unexcused)[:5].tolist()}")
+    out = {"coords": n * d, "index_flips": int(idiff.sum()), "sign_flips": 0}
+    if qjl:
+        S64 = np.asarray(S, dtype=np.float64)
+        nz = ref_n > 0
+        u = np.zeros_like(x)
+        u[nz] = x[nz] / ref_n[nz, None]
+        r = u - omr.centroids_per_coordinate(gi, c_lo, c_hi, m) @ Pi
+        r[~nz] = 0.0
+        rho = np.sqrt(np.sum(r * r, axis=1))
+        bad = np.abs(rnorm - rho) > NORM_RTOL * np.maximum(rho, 1e-30) + 1e-7 * (rho == 0)
+        assert not bad.any(), f"rnorm mismatch at rows {np.nonzero(bad)[0][:10]}"
+        s = r @ S64.T
+        sdiff = gs != (s >= 0).astype(np.int64)
+        band = FLIP_BAND * np.linalg.norm(S64, axis=1)[None, :] * rho[:, None]
+        unexcused = sdiff & (np.abs(s) > band)
+        assert not unexcused.any(), f"{unexcused.sum()} sign mismatches outside the zero band"
+        out["sign_flips"] = int(sdiff.sum())
+    for field in ("index_flips", "sign_flips"):
+        assert out[field] <= FLIP_RATE_MAX * n * d, f"excused {field} {out[field]} exceed 1e-4 of {n * d} coordinates"
+    return out
+
+
+def check_logits_mixed(gpu, q, Pi, S, c_lo, c_hi, rec, norm, rnorm, d, beta, m):
+    from oracle import mixed_rate as omr
+
+    gi, gs = omr.unpack(rec, d, beta, m, True)
+    ref = omr.logits(q, Pi, S, c_lo, c_hi, m, norm, rnorm, gi, gs)
+    tol = LOGIT_TOL * np.linalg.norm(np.asarray(q, dtype=np.float64), axis=1)[:, None] * np.asarray(norm)[None, :]
+    err = np.abs(np.asarray(gpu, dtype=np.float64) - ref)
+    assert np.all(err <= tol + 1e-30), f"logit error {np.max(err / (tol + 1e-30)):.3g} x tolerance"
+    return float(np.max(err / (tol + 1e-30))) if err.size else 0.0
+
+
+def check_attend_mixed(gpu, lg, scale, Pi, c_lo, c_hi, rec, norm, d, beta, m):
+    from oracle import mixed_rate as omr
+
+    gi, _ = omr.unpack(rec, d, beta, m, False)
+    ref = omr.attend_v(lg, scale, norm, gi, Pi, c_lo, c_hi, m)
+    tol = OUT_TOL * (float(np.max(norm)) if len(norm) else 1.0)
+    err = np.abs(np.asarray(gpu, dtype=np.float64) - ref)
+    assert np.all(err <= tol), f"softmax.V error {np.max(err) / tol:.3g} x tolerance"
+    return float(np.max(err) / tol) if err.size else 0.0

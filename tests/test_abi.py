@@ -207,3 +207,24 @@ def test_attend_workspace_size_does_not_wrap():
     st = lib.tq_attend_v(ctypes.byref(desc), FAKE, ctypes.c_float(0.1), 2 ** 31 - 1, 2 ** 62, FAKE, FAKE, FAKE, FAKE,
                          1 << 30, None)
     assert st == tqb.TQ_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("d,bits,n_hi,qjl", [(128, 2, 64, 1), (128, 3, 64, 0), (128, 1, 32, 1), (200, 2, 96, 1),
+                                             (64, 3, 32, 0), (256, 2, 224, 1)])
+def test_mixed_record_words_match_layout(d, bits, n_hi, qjl):
+    from oracle import mixed_rate as omr
+    assert tqb.tq_record_words_mixed(d, bits, n_hi, qjl) == omr.record_words(d, bits, n_hi, bool(qjl))
+    assert lib.tq_record_words_mixed(d, bits, 0, qjl) == lib.tq_record_words(d, bits, qjl)
+
+
+def test_mixed_rate_descriptors_checked():
+    for d, bits, n_hi in ((128, 2, 48), (128, 2, 128), (128, 2, -32), (128, 4, 32), (64, 2, 96)):
+        assert lib.tq_record_words_mixed(d, bits, n_hi, 1) == -1
+        desc = tqb.TqCacheDesc(d, bits, 1, 1, 2, n_hi, 64, FAKE, FAKE + 4096, FAKE + 8192)
+        st = lib.tq_quantize_append(ctypes.byref(desc), FAKE, 0, 0, 8, FAKE, FAKE, FAKE, None)   # dtype 0: bf16
+        assert st == tqb.TQ_ERR_UNSUPPORTED, (d, bits, n_hi)
+        assert "n_hi" in tqb.tq_last_error()
+    # the nearest-neighbour search takes integer-rate databases only
+    desc = tqb.TqCacheDesc(128, 2, 1, 1, 1, 64, 1000, FAKE, FAKE + 4096, FAKE + 8192)
+    st = lib.tq_nn_search(ctypes.byref(desc), FAKE, 10, 1000, FAKE, FAKE, FAKE, 10, FAKE, FAKE, FAKE, 1 << 30, None)
+    assert st == tqb.TQ_ERR_UNSUPPORTED
