@@ -177,6 +177,40 @@ tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale,
                       const float *Pi, const float *codebook, float *out,
                       void *workspace, size_t workspace_bytes, tq_stream stream);
 
+/* The softmax.V of tq_attend_v for a range of tokens, as a partial that
+ * tq_attend_merge combines with the partials of other ranges (for a cache whose
+ * tokens are split over GPUs; zubnet.ai, paragraph 1: keys and values).
+ * For every row r = (sequence, query head), partial[r] holds d + 2 floats
+ *   M = max_t scale * logits_t,  L = sum_t e^{scale * logits_t - M},
+ *   A = sum_t e^{scale * logits_t - M} * norm_t * c[code_t]   (rotated domain: no Pi^T).
+ * n_tokens == 0 gives (-inf, 0, 0 ... 0). Arguments, checks and workspace
+ * (tq_attend_workspace_size) as for tq_attend_v, without Pi.
+ *   partial: [n_seq * n_q_heads][d + 2] float. */
+tq_status tq_attend_v_partial(const tq_cache *v, const float *logits, float scale,
+                              int32_t n_q_heads, int64_t n_tokens, const float *codebook,
+                              float *partial, void *workspace, size_t workspace_bytes, tq_stream stream);
+
+/* Combines partials of tq_attend_v_partial: for each row r, with the parts
+ * p = 0 .. n_parts-1 of partials[r][p] = (M_p, L_p, A_p),
+ *   out[r] = Pi^T (sum_p e^{M_p - M} A_p) / (sum_p e^{M_p - M} L_p),  M = max_p M_p,
+ * the same result as tq_attend_v over all the ranges' tokens up to rounding;
+ * zeros when every part is empty.
+ *   partials: [rows][n_parts][d + 2] float; Pi: [d][d]; out: [rows][d] float.
+ * d: 8..256, multiple of 8; n_parts: 1..50000. */
+tq_status tq_attend_merge(const float *partials, int32_t n_parts, int32_t rows, int32_t d,
+                          const float *Pi, float *out, tq_stream stream);
+
+/* Top-k of several top-k lists per query (nearest-neighbour search over a
+ * database split into shards, one tq_nn_search per shard with its ids made
+ * global): for each query a, the k best entries of the n_parts lists
+ * part_scores / part_ids [n_parts][n_queries][k], each sorted by decreasing
+ * score (equal scores: lower id first) with id -1 (score -inf) only in places
+ * past its end; ordered the same way; (-inf, -1) where fewer than k exist.
+ * top_scores [n_queries][k] float, top_ids [n_queries][k] int64. k: 1..16. */
+tq_status tq_nn_merge(const float *part_scores, const int64_t *part_ids, int32_t n_parts,
+                      int32_t n_queries, int32_t k, float *top_scores, int64_t *top_ids,
+                      tq_stream stream);
+
 /* Workspace bytes tq_decode_attend needs for these caches, head count and length
  * (0 if the caches differ in d, n_seq or n_kv_heads). */
 size_t tq_decode_workspace_size(const tq_cache *k, const tq_cache *v, int32_t n_q_heads, int64_t n_tokens);
@@ -186,9 +220,12 @@ size_t tq_decode_workspace_size(const tq_cache *k, const tq_cache *v, int32_t n_
  * on the compressed cache; zubnet.ai, paragraph 1: keys and values):
  *   out[s][h] = Pi^T sum_t softmax_t(scale * l_t) * vnorm_t * cV[vcode_t],
  *   l_t = knorm_t * ( <Pi q, cK[kcode_t]> + krnorm_t * sqrt(pi/2)/d * <S q, 2 sign_t - 1> ).
- * With one query head per KV head, d = 128 and 1- or 2-bit key codes the whole
- * step is one pass over the tokens (the logits stay on chip); other shapes run
- * tq_logits and tq_attend_v inside the workspace and give the same results.
+ * With d = 128, 1- or 2-bit key codes and 1, 2, 4 or 8 query heads per KV head
+ * (value codes of 1..4 bits for one head, 1..3 bits for grouped heads, integer
+ * rates, Pi and S 16-byte aligned for grouped heads) the whole step is one pass
+ * over the tokens (the logits stay on chip); other shapes run tq_logits and
+ * tq_attend_v inside the workspace. Either way the result is bit-equal to
+ * tq_logits followed by tq_attend_v.
  *   k: key cache (qjl = 1); v: value cache (qjl = 0), same d, n_seq, n_kv_heads.
  *   q: [n_seq][n_q_heads][d] float; out: [n_seq][n_q_heads][d] float.
  *   Pi, S: [d][d] float; codebook_k / codebook_v: 2^idx_bits floats of each cache

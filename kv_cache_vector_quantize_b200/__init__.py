@@ -27,7 +27,9 @@ from ._binding import (  # noqa: F401
     TQError,
     declared_symbols,
     raw_lib,
+    tq_attend_merge,
     tq_attend_v,
+    tq_attend_v_partial,
     tq_attend_workspace_size,
     tq_codebook_fit,
     tq_debug_inject,
@@ -36,6 +38,7 @@ from ._binding import (  # noqa: F401
     tq_last_error,
     tq_logits,
     tq_logits_workspace_size,
+    tq_nn_merge,
     tq_nn_search,
     tq_nn_workspace_size,
     tq_quantize_append,

@@ -59,6 +59,9 @@ def _load() -> ctypes.CDLL:
         "tq_attend_v": (I32, [D, P, F, I32, I64, P, P, P, P, SZ, P]),
         "tq_attend_v_noalloc": (I32, [D, P, F, I32, I64, P, P, P, P]),
         "tq_attend_v_noalloc_status": (I32, [P]),
+        "tq_attend_v_partial": (I32, [D, P, F, I32, I64, P, P, P, SZ, P]),
+        "tq_attend_merge": (I32, [P, I32, I32, I32, P, P, P]),
+        "tq_nn_merge": (I32, [P, P, I32, I32, I32, P, P, P]),
         "tq_decode_workspace_size": (SZ, [D, D, I32, I64]),
         "tq_decode_attend": (I32, [D, D, P, I32, I64, F, P, P, P, P, P, P, SZ, P]),
         "tq_nn_workspace_size": (SZ, [D, I32, I64]),
@@ -266,6 +269,64 @@ def tq_attend_v(cache: PackedCache, logits: torch.Tensor, scale: float, n_tokens
                             _ptr(codebook), _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
                             _stream(stream)))
     return out
+
+
+def tq_attend_v_partial(cache: PackedCache, logits: torch.Tensor, scale: float, n_tokens: int, codebook: torch.Tensor,
+                        partial: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """logits [n_seq, H_q, n_tokens] -> the mergeable partial [n_seq * H_q, d + 2] (M, L, A) of these tokens."""
+    if logits.dim() != 3 or logits.shape[0] != cache.n_seq or logits.shape[2] != n_tokens:
+        raise ValueError(f"logits must be [{cache.n_seq}, H_q, {n_tokens}], got {tuple(logits.shape)}")
+    hq = logits.shape[1]
+    _need(logits, "logits", torch.float32, device=cache.device)
+    _need(codebook, "codebook", torch.float32, (cache.codebook_len,), cache.device)
+    if partial is None:
+        partial = torch.empty((cache.n_seq * hq, cache.d + 2), dtype=torch.float32, device=cache.device)
+    _need(partial, "partial", torch.float32, (cache.n_seq * hq, cache.d + 2), cache.device)
+    if workspace is None:
+        workspace = torch.empty(max(tq_attend_workspace_size(cache, hq, n_tokens), 256), dtype=torch.uint8,
+                                device=cache.device)
+    desc = cache.desc()
+    _check(_lib.tq_attend_v_partial(ctypes.byref(desc), _ptr(logits), float(scale), hq, int(n_tokens), _ptr(codebook),
+                                    _ptr(partial), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream(stream)))
+    return partial
+
+
+def tq_attend_merge(partials: torch.Tensor, Pi: torch.Tensor, out: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """partials [rows, n_parts, d + 2] (M, L, A of token ranges) -> out [rows, d]."""
+    if partials.dim() != 3:
+        raise ValueError(f"partials must be [rows, n_parts, d + 2], got {tuple(partials.shape)}")
+    rows, n_parts, d2 = partials.shape
+    d = d2 - 2
+    _need(partials, "partials", torch.float32)
+    _need(Pi, "Pi", torch.float32, (d, d), partials.device)
+    if out is None:
+        out = torch.empty((rows, d), dtype=torch.float32, device=partials.device)
+    _need(out, "out", torch.float32, (rows, d), partials.device)
+    _check(_lib.tq_attend_merge(_ptr(partials), n_parts, rows, d, _ptr(Pi), _ptr(out), _stream(stream)))
+    return out
+
+
+def tq_nn_merge(part_scores: torch.Tensor, part_ids: torch.Tensor, scores: torch.Tensor | None = None,
+                ids: torch.Tensor | None = None, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """part_scores / part_ids [n_parts, n_q, k] (sorted per-shard top-k lists, global ids) ->
+    the merged top-k (scores [n_q, k], ids [n_q, k])."""
+    if part_scores.dim() != 3 or part_ids.shape != part_scores.shape:
+        raise ValueError("part_scores and part_ids must both be [n_parts, n_q, k]")
+    n_parts, nq, k = part_scores.shape
+    _need(part_scores, "part_scores", torch.float32)
+    _need(part_ids, "part_ids", torch.int64, device=part_scores.device)
+    if scores is None:
+        scores = torch.empty((nq, k), dtype=torch.float32, device=part_scores.device)
+    if ids is None:
+        ids = torch.empty((nq, k), dtype=torch.int64, device=part_scores.device)
+    _need(scores, "scores", torch.float32, (nq, k), part_scores.device)
+    _need(ids, "ids", torch.int64, (nq, k), part_scores.device)
+    _check(_lib.tq_nn_merge(_ptr(part_scores), _ptr(part_ids), n_parts, nq, k, _ptr(scores), _ptr(ids),
+                            _stream(stream)))
+    return scores, ids
 
 
 def tq_decode_workspace_size(kcache: PackedCache, vcache: PackedCache, n_q_heads: int, n_tokens: int) -> int:

@@ -165,11 +165,14 @@ __global__ void __launch_bounds__(kAThreads) attend_chunk_kernel(const AttendPar
 // chunk sums split over all threads with independent loads in flight, then
 // out = Pi^T A / L, with Pi staged in shared memory when it fits. Launched as a
 // programmatic dependent of the chunk grid: it stages Pi while that grid's last
-// CTAs run and waits for the grid before reading any partial.
+// CTAs run and waits for the grid before reading any partial. With `merged`
+// given it writes the merged partial (M, L, A) there instead (Pi unused): the
+// part of a token range that another merge combines with other ranges.
 constexpr int kCThreads = 512;
 __global__ void __launch_bounds__(kCThreads) attend_combine_kernel(const float *__restrict__ partial, int n_chunks,
                                                                    int d, const float *__restrict__ Pi,
-                                                                   float *__restrict__ out, int pi_in_smem) {
+                                                                   float *__restrict__ out, int pi_in_smem,
+                                                                   float *__restrict__ merged) {
   extern __shared__ __align__(16) float cs[];          // [n_chunks] scale factors, then Pi (d x d) if staged
   __shared__ float a[kMaxD];
   __shared__ float part_sum[kCThreads];
@@ -187,7 +190,8 @@ __global__ void __launch_bounds__(kCThreads) attend_combine_kernel(const float *
   m = block_reduce(m, red, true);
   float l = 0.f;
   for (int c = tid; c < n_chunks; c += kCThreads) {
-    const float f = expf(part[(size_t)c * (d + 2)] - m);
+    // every part empty (merging token ranges that hold no tokens): nothing has weight
+    const float f = m == -INFINITY ? 0.f : expf(part[(size_t)c * (d + 2)] - m);
     cs[c] = f;
     l = fmaf(part[(size_t)c * (d + 2) + 1], f, l);
   }
@@ -212,10 +216,18 @@ __global__ void __launch_bounds__(kCThreads) attend_combine_kernel(const float *
     float v = 0.f;
     for (int q = 0; q < nsplit; ++q) v += part_sum[q * d + tid];
     a[tid] = v;
+    if (merged) merged[(size_t)row * (d + 2) + 2 + tid] = v;
+  }
+  if (merged) {
+    if (tid == 0) {
+      merged[(size_t)row * (d + 2)] = m;
+      merged[(size_t)row * (d + 2) + 1] = l;
+    }
+    return;
   }
   __syncthreads();
   // out_j = sum_i Pi[i][j] a_i / L, the i range split over the threads of column j
-  const float inv = 1.0f / l;
+  const float inv = l > 0.f ? 1.0f / l : 0.f;   // no weight anywhere: zeros
   const int j = tid % d, seg = tid / d, nseg = kCThreads / d;
   if (seg < nseg) {
     const int i0 = seg * ((d + nseg - 1) / nseg), i1 = min(d, i0 + (d + nseg - 1) / nseg);
@@ -277,10 +289,10 @@ cudaError_t launch_attend(const AttendParams &p, int bits, int n_seq, size_t sme
 }
 
 cudaError_t launch_combine(const float *partial, int rows, int n_chunks, int d, const float *Pi, float *out,
-                           cudaStream_t st) {
+                           cudaStream_t st, float *merged) {
   const size_t cs_bytes = (size_t)((n_chunks + 3) & ~3) * sizeof(float);
   const size_t pi_bytes = (size_t)d * d * sizeof(float);
-  const int pi_in_smem = (cs_bytes + pi_bytes <= 160 * 1024 && (reinterpret_cast<uintptr_t>(Pi) & 15) == 0 &&
+  const int pi_in_smem = (!merged && cs_bytes + pi_bytes <= 160 * 1024 && (reinterpret_cast<uintptr_t>(Pi) & 15) == 0 &&
                           (d * d) % 4 == 0) ? 1 : 0;
   const size_t smem = cs_bytes + (pi_in_smem ? pi_bytes : 0);
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(attend_combine_kernel), smem);
@@ -295,10 +307,25 @@ cudaError_t launch_combine(const float *partial, int rows, int n_chunks, int d, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attend_combine_kernel, partial, n_chunks, d, Pi, out, pi_in_smem);
+  return cudaLaunchKernelEx(&cfg, attend_combine_kernel, partial, n_chunks, d, Pi, out, pi_in_smem, merged);
 }
 
 size_t attend_chunk_smem(int d, int rec_words, int64_t chunk) { return chunk_smem(d, rec_words, chunk); }
+
+namespace {
+__global__ void empty_partial_kernel(float *partial, int rows, int d) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (int64_t)rows * (d + 2)) return;
+  partial[e] = (e % (d + 2)) == 0 ? -INFINITY : 0.f;
+}
+}  // namespace
+
+// The partial of a token range without tokens: (M, L, A) = (-inf, 0, 0) per row.
+cudaError_t launch_empty_partial(float *partial, int rows, int d, cudaStream_t st) {
+  const int64_t n = (int64_t)rows * (d + 2);
+  empty_partial_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(partial, rows, d);
+  return cudaGetLastError();
+}
 
 }  // namespace tq
 

@@ -18,10 +18,24 @@
 // merged once at the end. The logits and norms of the next tile are loaded
 // while the current one is accumulated. In the accumulation loop each
 // half-warp takes one token and a lane owns 8 consecutive coordinates: per
-// token it reads its code bits once (an 8 * BITS-bit field), the token's
-// weights for all query heads with one 16-byte load (two addresses per warp),
-// and one centroid per coordinate, shared by the query heads. Tokens past the
+// token it reads its code bits once (an 8 * BITS-bit field) and the token's
+// weights for all query heads (stored as (w, w) pairs), then looks up its 8
+// centroids two at a time in a table of centroid pairs indexed by two
+// consecutive codes (2 * BITS bits) and accumulates them with packed
+// two-lane float32 FMAs (fma.rn.f32x2: the same two round-to-nearest FMAs as
+// two scalar FMAs, in the same order). The pair table is stored once per lane
+// of a 16-lane shared-memory phase (entry (key, lane) at (16 key + lane) * 8
+// bytes), so the half-warp's random lookups never conflict. Tokens past the
 // end of a tile carry weight 0, so both half-warps run the same iterations.
+//
+// Mixed rate (MIXED, fractional bits per channel with the first 64 of the 128
+// coordinates at BITS + 1 code bits): lanes 0..7 of a half-warp hold
+// coordinates of the wider group (8 (BITS+1)-bit codes), lanes 8..15 of the
+// narrower one; each lane has its own field position and width and reads its
+// group's pair table (the wider group's first, then the narrower's), with the
+// same instruction count per pair. A mixed record is not a multiple of 16
+// bytes, so a tile with an odd number of tokens gets its last record by plain
+// loads from the producer before the bulk copy of the others.
 #include "common.cuh"
 
 namespace tq {
@@ -36,15 +50,20 @@ constexpr int kVStages = 4;
 constexpr int kVMaxQ = 4;
 constexpr uint32_t kVBarBytes = 128;           // full[kVStages], empty[kVStages], padded
 
-template <int BITS>
+template <int BITS, bool MIXED = false>
 struct VTile {
-  static constexpr int RW = BITS * kVD / 32;                    // record words (no sign field)
+  // record words (no sign field); mixed: 64 coordinates at BITS + 1 bits, 64 at BITS
+  static constexpr int RW = MIXED ? 2 * (2 * BITS + 1) : BITS * kVD / 32;
   static constexpr uint32_t kStageBytes = kVTile * RW * 4;      // 8 .. 32 KB
   static constexpr uint32_t kStages = kVStages * kStageBytes;
   static constexpr uint32_t kMerge = kVWarps * kVMaxQ * kVD * 4;   // 32 KB, aliases the stages
-  static constexpr uint32_t kScratch = kVWarps * 32 * 16;          // per-warp token weights (float4)
+  static constexpr uint32_t kScratch = kVWarps * 32 * kVMaxQ * 8;  // per-warp token weights ((w, w) per head)
+  // centroid-pair table entries, 16 lane copies (mixed: the wider group's table, then the narrower's)
+  static constexpr int kPairsHi = MIXED ? (1 << (2 * (BITS + 1))) * 16 : 0;
+  static constexpr int kPairs = kPairsHi + (1 << (2 * BITS)) * 16;
   static constexpr uint32_t kBytes = kVBarBytes + (kStages > kMerge ? kStages : kMerge) + kScratch;
-  static_assert((RW * 4) % 16 == 0, "bulk copies of whole records need 16-byte multiples");
+  static_assert(MIXED || (RW * 4) % 16 == 0, "bulk copies of whole records need 16-byte multiples");
+  static_assert(kStageBytes % 16 == 0, "stage slots 16-byte aligned");
   static_assert(kVBarBytes >= 2 * kVStages * 8, "barrier area");
 };
 
@@ -53,23 +72,26 @@ struct VFastParams {
   int tiles_per_chunk;
 };
 
-template <int BITS, int QMAX>
+template <int BITS, int QMAX, bool MIXED = false>
 __global__ void __launch_bounds__(kVThreads, 1) attend_fast_kernel(const VFastParams fp) {
-  using T = VTile<BITS>;
+  using T = VTile<BITS, MIXED>;
   constexpr int RW = T::RW;
   constexpr int L = 1 << BITS;
   constexpr int CPL = 8;          // coordinates per lane (16 lanes per token)
-  constexpr int FB = CPL * BITS;  // code bits of a lane's coordinates
+  constexpr int FB = CPL * BITS;  // code bits of a lane's coordinates (integer rate)
   const AttendParams &p = fp.p;
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ float cbs[16];
+  __shared__ float cbs[48];       // the BITS codebook at 0, the BITS + 1 codebook (mixed) at 16
   __shared__ float mst[kVWarps][kVMaxQ], lst[kVWarps][kVMaxQ];
+  // (c[k & (L-1)], c[k >> BITS]) at entry 16 k + lane copy; static, so a lookup's address is the
+  // byte offset plus an immediate
+  __shared__ __align__(128) uint64_t ptab[T::kPairs];
 
   const uint32_t sb = smem_u32(smem);
   auto full_bar = [&](int s) { return sb + 8u * s; };
   auto empty_bar = [&](int s) { return sb + 8u * (kVStages + s); };
   unsigned char *stages = smem + kVBarBytes;
-  float4 *wscr = reinterpret_cast<float4 *>(smem + T::kBytes - T::kScratch);   // [kVWarps][32]
+  uint64_t *wscr = reinterpret_cast<uint64_t *>(smem + T::kBytes - T::kScratch);   // [kVWarps][32][kVMaxQ]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int chunk = blockIdx.x, unit = blockIdx.y;
@@ -82,7 +104,6 @@ __global__ void __launch_bounds__(kVThreads, 1) attend_fast_kernel(const VFastPa
   const int n_tiles = t_begin < t_end ? (int)((t_end - t_begin + kVTile - 1) / kVTile) : 0;
   const size_t slot0 = (size_t)sk * p.capacity;
 
-  pdl_launch_dependents();   // the merge may become resident and stage its matrix meanwhile
   if (tid == 0) {
     for (int s = 0; s < kVStages; ++s) {
       mbar_init(full_bar(s), 1);
@@ -91,6 +112,17 @@ __global__ void __launch_bounds__(kVThreads, 1) attend_fast_kernel(const VFastPa
     mbar_fence_init();
   }
   if (tid < L) cbs[tid] = p.codebook[tid];
+  if (MIXED && tid < 2 * L) cbs[16 + tid] = p.codebook[L + tid];
+  __syncthreads();
+  for (int e = tid; e < T::kPairs; e += kVThreads) {
+    if (e < T::kPairsHi) {   // the wider group's pairs (mixed only)
+      const int key = e >> 4;
+      ptab[e] = f2_pack(cbs[16 + (key & (2 * L - 1))], cbs[16 + (key >> (BITS + 1))]);
+    } else {
+      const int key = (e - T::kPairsHi) >> 4;
+      ptab[e] = f2_pack(cbs[key & (L - 1)], cbs[key >> BITS]);
+    }
+  }
   __syncthreads();
 
   if (warp == kVWarps) {
@@ -104,9 +136,20 @@ __global__ void __launch_bounds__(kVThreads, 1) attend_fast_kernel(const VFastPa
           break;
         }
         const int64_t t0 = t_begin + (int64_t)i * kVTile;
-        const uint32_t bytes = (uint32_t)min((int64_t)kVTile, t_end - t0) * RW * 4;
+        int nrec = (int)min((int64_t)kVTile, t_end - t0);
+        if (MIXED && (nrec * RW * 4) % 16 != 0) {
+          // the last record by plain loads (before the arrival that releases the stage), the rest by copy
+          --nrec;
+          const uint32_t *src = p.records + (slot0 + t0 + nrec) * RW;
+          uint32_t *dst = reinterpret_cast<uint32_t *>(stages + (size_t)s * T::kStageBytes) + (size_t)nrec * RW;
+#pragma unroll
+          for (int w = 0; w < RW; ++w) dst[w] = __ldg(src + w);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // ordered with the copy engine's writes
+        }
+        const uint32_t bytes = (uint32_t)nrec * RW * 4;
         mbar_arrive_expect_tx(full_bar(s), bytes);
-        bulk_g2s(sb + kVBarBytes + (uint32_t)s * T::kStageBytes, p.records + (slot0 + t0) * RW, bytes, full_bar(s));
+        if (bytes > 0)
+          bulk_g2s(sb + kVBarBytes + (uint32_t)s * T::kStageBytes, p.records + (slot0 + t0) * RW, bytes, full_bar(s));
         ++issued;
       }
       // drain: every issued copy must land before the CTA exits
@@ -120,21 +163,31 @@ __global__ void __launch_bounds__(kVThreads, 1) attend_fast_kernel(const VFastPa
   }
 
   // -------------------------------- consumers --------------------------------
-  // running max (warp-uniform), this lane's share of l, coordinates 8 (lane mod 16) + a
-  float m[QMAX], l[QMAX], acc[CPL][QMAX];
+  // running max (warp-uniform), this lane's share of l, coordinates 8 (lane mod 16) + 2 pp + {0, 1}
+  float m[QMAX], l[QMAX];
+  uint64_t acc2[CPL / 2][QMAX];
 #pragma unroll
   for (int qq = 0; qq < QMAX; ++qq) {
     m[qq] = -INFINITY;
     l[qq] = 0.f;
 #pragma unroll
-    for (int a = 0; a < CPL; ++a) acc[a][qq] = 0.f;
+    for (int pp = 0; pp < CPL / 2; ++pp) acc2[pp][qq] = 0ull;   // (+0, +0)
   }
   const float *lrow[QMAX];
 #pragma unroll
   for (int qq = 0; qq < QMAX; ++qq) lrow[qq] = p.logits + ((size_t)seq * p.n_q_heads + h0 + min(qq, nq - 1)) * p.n_tokens;
   const int half = lane >> 4, sub = lane & 15;
-  const int bit0 = FB * sub, wd = bit0 >> 5, sh = bit0 & 31;
-  const bool two = sh + FB > 32;   // the field crosses into word wd + 1 (< RW)
+  // this lane's code field: integer rate FB bits at FB * sub; mixed: lanes 0..7 hold 8 codes of
+  // BITS + 1 bits at 8 (BITS+1) sub, lanes 8..15 8 codes of BITS bits after the 64 wider codes
+  const bool wide = MIXED && sub < 8;
+  const int lb = wide ? BITS + 1 : BITS;
+  const int bit0 = !MIXED ? FB * sub : wide ? 8 * (BITS + 1) * sub : 64 * (BITS + 1) + 8 * BITS * (sub - 8);
+  const int wd = bit0 >> 5, sh = bit0 & 31;
+  const bool two = sh + 8 * lb > 32;   // the field crosses into word wd + 1 (< RW)
+  // mixed: per lane, the pair key mask (shifted to byte offset 128 key) and the table base (the
+  // narrower group's table starts after the wider one's, a power of two of bytes)
+  const uint32_t kmask_l = 128u * ((1u << (2 * lb)) - 1u);
+  const uint32_t tbase_l = (MIXED && !wide ? 8u * (uint32_t)T::kPairsHi : 0u) | (8u * sub);
   const int tw = 32 * warp;        // this warp's first token in a tile
   const int k = tw + lane;         // this lane's token for the weights
   // logits (times scale) and norm of this lane's token in tile i
@@ -157,7 +210,6 @@ __global__ void __launch_bounds__(kVThreads, 1) attend_fast_kernel(const VFastPa
     for (int qq = 0; qq < QMAX; ++qq) z[qq] = zn[qq];
     const float nrm = nn;
     if (i + 1 < n_tiles) fetch(i + 1, zn, nn);   // in flight during this tile
-    float wq[QMAX];
 #pragma unroll
     for (int qq = 0; qq < QMAX; ++qq) {
       const float mx = fmaxf(m[qq], warp_max(z[qq]));
@@ -166,12 +218,12 @@ __global__ void __launch_bounds__(kVThreads, 1) attend_fast_kernel(const VFastPa
       const float e = mx == -INFINITY ? 0.f : expf(z[qq] - mx);
       m[qq] = mx;
       l[qq] = fmaf(l[qq], f, e);
+      const uint64_t f2 = f2_pack(f, f);
 #pragma unroll
-      for (int a = 0; a < CPL; ++a) acc[a][qq] *= f;
-      wq[qq] = e * nrm;   // 0 for a token past the end
+      for (int pp = 0; pp < CPL / 2; ++pp) acc2[pp][qq] = f2_mul(acc2[pp][qq], f2);
+      const float w = e * nrm;   // 0 for a token past the end
+      wscr[(tw + lane) * kVMaxQ + qq] = f2_pack(w, w);
     }
-    wscr[tw + lane] = make_float4(wq[0], QMAX > 1 ? wq[1 % QMAX] : 0.f, QMAX > 2 ? wq[2 % QMAX] : 0.f,
-                                  QMAX > 3 ? wq[3 % QMAX] : 0.f);
     __syncwarp();
     if (!mbar_wait(full_bar(s), (i / kVStages) & 1)) {
       atomicOr(p.status, kDevTimeout);
@@ -181,34 +233,58 @@ __global__ void __launch_bounds__(kVThreads, 1) attend_fast_kernel(const VFastPa
     // token tw + 2 j + half of the tile for this half-warp (records past n hold stale codes, weight 0)
     const uint32_t *rs = reinterpret_cast<const uint32_t *>(stages + (size_t)s * T::kStageBytes) + (size_t)(tw + half) * RW;
     const int np = (min(32, n - tw) + 1) >> 1;   // token pairs of this warp (warp-uniform, may be <= 0)
+    const uint32_t lane8 = 8u * sub;   // this lane's copy of the pair table
 #pragma unroll 2
     for (int j = 0; j < np; ++j) {
       const uint32_t *rec = rs + 2 * j * RW;
       const uint32_t lo = rec[wd];
       const uint32_t hi = two ? rec[wd + 1] : 0u;
       const uint32_t bits = __funnelshift_r(lo, hi, sh);
-      const float4 w4 = wscr[tw + 2 * j + half];
-      const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+      const uint64_t *wt = wscr + (tw + 2 * j + half) * kVMaxQ;
+      uint64_t w2[QMAX];
 #pragma unroll
-      for (int a = 0; a < CPL; ++a) {
-        // byte offset of code a in the centroid table: one shift and one mask
-        constexpr uint32_t kMask = 4u * (L - 1);
-        const int shr = BITS * a - 2;
-        const uint32_t off = (shr >= 0 ? bits >> (shr & 31) : bits << ((-shr) & 31)) & kMask;
-        const float cv = *reinterpret_cast<const float *>(reinterpret_cast<const unsigned char *>(cbs) + off);
+      for (int qq = 0; qq < QMAX; ++qq) w2[qq] = wt[qq];
+      if constexpr (!MIXED) {
 #pragma unroll
-        for (int qq = 0; qq < QMAX; ++qq) acc[a][qq] = fmaf(wv[qq], cv, acc[a][qq]);
+        for (int pp = 0; pp < CPL / 2; ++pp) {
+          // byte offset of the pair (codes 2 pp, 2 pp + 1) in the table: key * 128 (+ the lane copy)
+          constexpr uint32_t kMask = 128u * (L * L - 1);
+          const int shr = 2 * BITS * pp - 7;
+          const uint32_t off = ((shr >= 0 ? bits >> (shr & 31) : bits << ((-shr) & 31)) & kMask) | lane8;
+          const uint64_t cv = *reinterpret_cast<const uint64_t *>(reinterpret_cast<const unsigned char *>(ptab) + off);
+#pragma unroll
+          for (int qq = 0; qq < QMAX; ++qq) acc2[pp][qq] = f2_fma(w2[qq], cv, acc2[pp][qq]);
+        }
+      } else {
+        // bits << 7 as a 64-bit pair, so that a pair key of a runtime width is one funnel shift
+        const uint32_t lo7 = bits << 7, hi7 = bits >> 25;
+#pragma unroll
+        for (int pp = 0; pp < CPL / 2; ++pp) {
+          const uint32_t off = (__funnelshift_r(lo7, hi7, 2 * lb * pp) & kmask_l) | tbase_l;
+          const uint64_t cv = *reinterpret_cast<const uint64_t *>(reinterpret_cast<const unsigned char *>(ptab) + off);
+#pragma unroll
+          for (int qq = 0; qq < QMAX; ++qq) acc2[pp][qq] = f2_fma(w2[qq], cv, acc2[pp][qq]);
+        }
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_bar(s));   // this warp is done with the stage and its weights
   }
   // the two half-warps accumulated different tokens of the same coordinates
+  float acc[CPL][QMAX];
+#pragma unroll
+  for (int pp = 0; pp < CPL / 2; ++pp)
+#pragma unroll
+    for (int qq = 0; qq < QMAX; ++qq) f2_unpack(acc2[pp][qq], acc[2 * pp][qq], acc[2 * pp + 1][qq]);
 #pragma unroll
   for (int a = 0; a < CPL; ++a)
 #pragma unroll
     for (int qq = 0; qq < QMAX; ++qq) acc[a][qq] += __shfl_xor_sync(0xffffffffu, acc[a][qq], 16);
 
+  // Only now may the merge grid become resident (it stages its matrix while the last CTAs finish):
+  // its CTAs wait for this whole grid, and resident earlier they would hold registers and shared
+  // memory on SMs that this grid's later waves need.
+  pdl_launch_dependents();
   // ---- merge the warps: M = max_w m_w, each warp scaled by e^{m_w - M} ----
 #pragma unroll
   for (int qq = 0; qq < QMAX; ++qq) l[qq] = warp_sum(l[qq]);
@@ -253,37 +329,46 @@ __global__ void __launch_bounds__(kVThreads, 1) attend_fast_kernel(const VFastPa
   }
 }
 
-template <int BITS, int QMAX>
+template <int BITS, int QMAX, bool MIXED>
 cudaError_t launch_vf(const VFastParams &fp, int units, cudaStream_t st) {
-  auto kern = attend_fast_kernel<BITS, QMAX>;
-  const size_t smem = VTile<BITS>::kBytes;
+  auto kern = attend_fast_kernel<BITS, QMAX, MIXED>;
+  const size_t smem = VTile<BITS, MIXED>::kBytes;
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
   kern<<<dim3((unsigned)fp.p.n_chunks, (unsigned)units), kVThreads, smem, st>>>(fp);
   return cudaGetLastError();
 }
 
-template <int BITS>
+template <int BITS, bool MIXED = false>
 cudaError_t launch_vf_q(const VFastParams &fp, int units, cudaStream_t st) {
   switch (fp.p.q_per_cta) {
-    case 1: return launch_vf<BITS, 1>(fp, units, st);
-    case 2: return launch_vf<BITS, 2>(fp, units, st);
-    case 3: return launch_vf<BITS, 3>(fp, units, st);
-    default: return launch_vf<BITS, 4>(fp, units, st);
+    case 1: return launch_vf<BITS, 1, MIXED>(fp, units, st);
+    case 2: return launch_vf<BITS, 2, MIXED>(fp, units, st);
+    case 3: return launch_vf<BITS, 3, MIXED>(fp, units, st);
+    default: return launch_vf<BITS, 4, MIXED>(fp, units, st);
   }
 }
 
 }  // namespace
 
-bool attend_fast_supported(int d, int bits, int q_per_cta, const void *records) {
-  return d == kVD && bits >= 1 && bits <= 4 && q_per_cta >= 1 && q_per_cta <= kVMaxQ &&
-         (reinterpret_cast<uintptr_t>(records) & 15) == 0;
+bool attend_fast_supported(int d, int bits, int q_per_cta, const void *records, int n_hi, int64_t capacity) {
+  if (d != kVD || q_per_cta < 1 || q_per_cta > kVMaxQ || (reinterpret_cast<uintptr_t>(records) & 15) != 0)
+    return false;
+  if (n_hi == 0) return bits >= 1 && bits <= 4;
+  // mixed rate with the first 64 coordinates wider; the rows of every (sequence, head) must start on
+  // 16 bytes (a record is 40 or 56 bytes: an even capacity)
+  return n_hi == 64 && bits >= 1 && bits <= 3 && capacity % 2 == 0;
 }
 
 // Tokens per chunk (a multiple of the 512-token tile): the split of every
-// unit's tiles into equal chunks that minimises the busiest SM's tile count
-// (whole waves of one CTA per SM times tiles per chunk).
+// unit's tiles into equal chunks that minimises the busiest SM's time, counted
+// as whole waves of one CTA per SM times (tiles per chunk + a CTA's fixed cost:
+// set-up, the first copies' latency and the end-of-chunk merge, about two
+// tiles' time). Without the fixed cost, many units would be split into
+// one-tile chunks (16 384 CTAs on the 8 x 8 x 131072 cache), slower per token
+// and with 256 partials per query head to merge.
 int64_t attend_fast_chunk(int64_t n_tokens, int units) {
+  constexpr int64_t kCtaCost = 2;
   const int64_t tpu = (n_tokens + kVTile - 1) / kVTile;
   const int64_t slots = device_sm_count();
   int64_t best_tpc = tpu, best_cost = INT64_MAX;
@@ -291,7 +376,7 @@ int64_t attend_fast_chunk(int64_t n_tokens, int units) {
   for (int64_t nc = 1; nc <= max_nc; ++nc) {
     const int64_t tpc = (tpu + nc - 1) / nc;
     const int64_t ctas = (int64_t)units * ((tpu + tpc - 1) / tpc);
-    const int64_t cost = ((ctas + slots - 1) / slots) * tpc;
+    const int64_t cost = ((ctas + slots - 1) / slots) * (tpc + kCtaCost);
     if (cost < best_cost) {
       best_cost = cost;
       best_tpc = tpc;
@@ -305,6 +390,13 @@ cudaError_t launch_attend_fast(const AttendParams &p, int bits, int n_seq, cudaS
   fp.p = p;
   fp.tiles_per_chunk = (int)(p.chunk / kVTile);
   const int units = n_seq * p.n_kv_heads * p.qblocks;
+  if (p.n_hi == 64) {
+    switch (bits) {
+      case 1: return launch_vf_q<1, true>(fp, units, st);
+      case 2: return launch_vf_q<2, true>(fp, units, st);
+      default: return launch_vf_q<3, true>(fp, units, st);
+    }
+  }
   switch (bits) {
     case 1: return launch_vf_q<1>(fp, units, st);
     case 2: return launch_vf_q<2>(fp, units, st);

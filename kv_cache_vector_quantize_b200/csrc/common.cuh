@@ -23,6 +23,27 @@ __device__ __forceinline__ float to_float(float v) { return v; }
 __device__ __forceinline__ float to_float(__nv_bfloat16 v) { return __bfloat162float(v); }
 __device__ __forceinline__ float to_float(__half v) { return __half2float(v); }
 
+// Two float32 values in one 64-bit register (the lower coordinate in the low half) and the
+// packed two-lane float32 arithmetic of sm_100.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &a, float &b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -157,13 +178,38 @@ bool decode_fused_supported(int d, int kbits, int vbits, int n_q_heads, int n_kv
                             const void *vrec, size_t limit);
 cudaError_t launch_decode_fused(const DecodeFusedArgs &a, cudaStream_t st);
 cudaError_t launch_status_or(uint32_t *dst, const uint32_t *a, const uint32_t *b, cudaStream_t st);
+// Grouped-query tables alone (logits_gqa.cu): the four- or two-head float16 tables and scales of every unit.
+cudaError_t launch_gqa_tables(const GqaParams &g, int bits, int qh, int units, cudaStream_t st);
+// Fused decode for grouped queries (decode_gqa.cu): 2, 4 or 8 query heads per KV head, d = 128,
+// 1- or 2-bit key codes, 1..3-bit value codes; consumes the grouped-query tables and writes the
+// chunk partials of the softmax.V merge, bit-equal to tq_logits + tq_attend_v.
+struct DecodeGqaArgs {
+  const uint32_t *krec;
+  const float *knorm, *krnorm;
+  const uint32_t *vrec;
+  const float *vnorm;
+  const unsigned char *tables;
+  const float *sigma;
+  const float *cbv;
+  float *partial;
+  uint32_t *status;
+  int64_t n_tokens, cap_k, cap_v, chunk;
+  int n_seq, n_kv_heads, n_q_heads, qblocks, n_chunks, kbits, vbits;
+  float scale;
+  size_t smem_limit;
+};
+bool decode_gqa_supported(int d, int kbits, int vbits, int group, size_t limit);
+cudaError_t launch_decode_gqa(const DecodeGqaArgs &a, cudaStream_t st);
 // d = 128 softmax.V streamed by bulk copies (attend_fast.cu); p.chunk from attend_fast_chunk.
-bool attend_fast_supported(int d, int bits, int q_per_cta, const void *records);
+bool attend_fast_supported(int d, int bits, int q_per_cta, const void *records, int n_hi, int64_t capacity);
 int64_t attend_fast_chunk(int64_t n_tokens, int units);
 cudaError_t launch_attend_fast(const AttendParams &p, int bits, int n_seq, cudaStream_t st);
 size_t attend_chunk_smem(int d, int rec_words, int64_t chunk);
 cudaError_t launch_combine(const float *partial, int rows, int n_chunks, int d, const float *Pi,
-                           float *out, cudaStream_t st);
+                           float *out, cudaStream_t st, float *merged = nullptr);
+cudaError_t launch_empty_partial(float *partial, int rows, int d, cudaStream_t st);
+cudaError_t launch_nn_list_merge(const float *ps, const int64_t *pi, int n_parts, int n_q, int k, float *top_s,
+                                 int64_t *top_i, cudaStream_t st);
 // Nearest-neighbour search (nn_search.cu): running top-k of the key estimator over one packed
 // database stream for a batch of queries.
 struct NnArgs {
@@ -195,7 +241,7 @@ void clear_error();   // empties this thread's tq_last_error() text
 // The argument checks of tq_attend_v that do not involve the workspace (tq_api.cu).
 tq_status check_attend_args(const tq_cache *v, const float *logits, float scale, int32_t n_q_heads,
                             int64_t n_tokens, const float *Pi, const float *codebook, const float *out,
-                            const char *what);
+                            const char *what, bool need_pi = true);
 
 }  // namespace tq
 

@@ -132,7 +132,6 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(const Decode
                    (reinterpret_cast<uintptr_t>(p.krnorm + kslot0) % 16 == 0);
   const bool vnc = reinterpret_cast<uintptr_t>(p.vnorm + vslot0) % 16 == 0;
 
-  pdl_launch_dependents();   // the merge may become resident and stage its matrix meanwhile
   if (tid == 0) {
     for (int s = 0; s < kDMaxStages; ++s) {
       mbar_init(kfull(s), 1);
@@ -323,6 +322,10 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(const Decode
 #pragma unroll
   for (int a = 0; a < CPL; ++a) acc[a] += __shfl_xor_sync(0xffffffffu, acc[a], 16);
 
+  // Only now may the merge grid become resident (it stages its matrix while the last CTAs finish):
+  // its CTAs wait for this whole grid, and resident earlier they would hold registers and shared
+  // memory on SMs that this grid's later waves need.
+  pdl_launch_dependents();
   // ---- merge the warps: M = max_w m_w, each warp scaled by e^{m_w - M} ----
   lsum = warp_sum(lsum);
   if (lane == 0) {

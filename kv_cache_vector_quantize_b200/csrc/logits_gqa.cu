@@ -36,28 +36,26 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "gqa_core.cuh"
 
 namespace tq {
 
 namespace {
 
-constexpr int kGD = 128;                        // head dimension
+using namespace gqa;
+
 constexpr int kGConsumers = 16;
 constexpr int kGThreads = 32 * (kGConsumers + 1);
 constexpr int kGTile = 32 * kGConsumers;        // keys per stage
 constexpr int kGMaxStages = 6;
-constexpr uint32_t kGHalf = 65536;              // bytes of one table half in shared memory
 constexpr uint32_t kGBarBytes = 128;             // full[6], empty[6], table barrier; keeps the stage ring 16-byte aligned
 static_assert(kGBarBytes >= 8 * (2 * kGMaxStages + 1) && kGBarBytes % 16 == 0, "stage slots must start 16-byte aligned");
 
+// bytes of one scan stage: a tile's records, then its norms and residual norms
 template <int BETA>
-struct GKeys {
-  static constexpr int IW = BETA * kGD / 32;     // code-stream words
-  static constexpr int RW = IW + kGD / 32;       // record words
-  static constexpr int NI = BETA == 1 ? 16 : 32; // index bytes per record
-  static constexpr int G = 8 / BETA;             // coordinates per index byte
-  static constexpr uint32_t kStageBytes = kGTile * (RW + 2) * 4;
-  static_assert(kStageBytes % 16 == 0 && (kGTile * RW * 4) % 16 == 0, "bulk copies need 16-byte offsets");
+struct GStage {
+  static constexpr uint32_t kBytes = kGTile * (GKeys<BETA>::RW + 2) * 4;
+  static_assert(kBytes % 16 == 0 && (kGTile * GKeys<BETA>::RW * 4) % 16 == 0, "bulk copies need 16-byte offsets");
 };
 
 // ------------------------------------------------------------------------
@@ -195,69 +193,11 @@ struct GScan {
   uint32_t dyn_bytes;
 };
 
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ uint32_t lds32u(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ __half2 u2h2(uint32_t v) { return *reinterpret_cast<const __half2 *>(&v); }
-
-// Permute N words by XOR of their index with c (N a power of two, c < N).
-template <int N>
-__device__ __forceinline__ void xor_perm(uint32_t (&w)[N], int c) {
-#pragma unroll
-  for (int bit = 1; bit < N; bit <<= 1) {
-    uint32_t t[N];
-    const bool take = (c & bit) != 0;
-#pragma unroll
-    for (int j = 0; j < N; ++j) t[j] = take ? w[j ^ bit] : w[j];
-#pragma unroll
-    for (int j = 0; j < N; ++j) w[j] = t[j];
-  }
-}
-
-// NSTEP table reads at base offset OFF (0: index half, kGHalf: sign half),
-// summed per head into acc (float32), with float16 partial sums over 16 reads.
-template <int QH, int NSTEP, uint32_t OFF, int NW>
-__device__ __forceinline__ void gqa_sum(const uint32_t (&w)[NW], const uint32_t (&sel)[4], const uint32_t (&x)[16],
-                                        float (&acc)[QH]) {
-  constexpr int NP = QH / 2;   // head pairs
-  __half2 part[2][NP];
-#pragma unroll
-  for (int st = 0; st < NSTEP; ++st) {
-    if ((st & 15) == 0) {
-#pragma unroll
-      for (int k = 0; k < NP; ++k) part[0][k] = part[1][k] = __float2half2_rn(0.f);
-    }
-    const uint32_t addr = __byte_perm(w[st >> 2], x[st >> 1], sel[st & 3]) + OFF;
-    if constexpr (QH == 4) {
-      const uint2 v = lds64(addr);
-      part[st & 1][0] = __hadd2(part[st & 1][0], u2h2(v.x));
-      part[st & 1][1] = __hadd2(part[st & 1][1], u2h2(v.y));
-    } else {
-      part[st & 1][0] = __hadd2(part[st & 1][0], u2h2(lds32u(addr)));
-    }
-    if ((st & 15) == 15 || st == NSTEP - 1) {
-#pragma unroll
-      for (int k = 0; k < NP; ++k) {
-        const float2 a = __half22float2(part[0][k]), b = __half22float2(part[1][k]);
-        acc[2 * k] += a.x + b.x;
-        acc[2 * k + 1] += a.y + b.y;
-      }
-    }
-  }
-}
-
 template <int BETA, int QH>
 __global__ void __launch_bounds__(kGThreads, 1) logits_gqa_kernel(const GScan gs) {
   using K = GKeys<BETA>;
   constexpr int RW = K::RW, IW = K::IW;
-  constexpr uint32_t SB = K::kStageBytes;
+  constexpr uint32_t SB = GStage<BETA>::kBytes;
   constexpr uint32_t ESZ = 2 * QH;                 // bytes per table entry
   const LogitsParams &p = gs.p;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -460,12 +400,12 @@ cudaError_t launch_gqa_t(const LogitsParams &p, const GqaParams &g, int n_seq, s
   // dynamic shared memory: barriers, the 64 KB-aligned 128 KB table block, stage slots around it
   const uint32_t dyn0 = 1024;
   const uint32_t T0 = (dyn0 + kGBarBytes + kGHalf - 1) & ~(kGHalf - 1);
-  const uint32_t n_a = (T0 - dyn0 - kGBarBytes) / K::kStageBytes;
+  const uint32_t n_a = (T0 - dyn0 - kGBarBytes) / GStage<BETA>::kBytes;
   const uint32_t b0 = T0 + 2 * kGHalf;
   const uint32_t end = dyn0 + (uint32_t)limit;
-  uint32_t n_b = b0 < end ? (end - b0) / K::kStageBytes : 0;
+  uint32_t n_b = b0 < end ? (end - b0) / GStage<BETA>::kBytes : 0;
   if (n_a + n_b > (uint32_t)kGMaxStages) n_b = kGMaxStages > (int)n_a ? kGMaxStages - n_a : 0;
-  gs.dyn_bytes = (b0 + n_b * K::kStageBytes) - dyn0;
+  gs.dyn_bytes = (b0 + n_b * GStage<BETA>::kBytes) - dyn0;
   auto kern = logits_gqa_kernel<BETA, QH>;
   e = set_smem_once(reinterpret_cast<const void *>(kern), gs.dyn_bytes);
   if (e != cudaSuccess) return e;
@@ -494,6 +434,14 @@ bool gqa_supported(int d, int bits, int group) {
 }
 
 size_t gqa_table_bytes(int units) { return (size_t)units * 2 * kGHalf; }
+
+cudaError_t launch_gqa_tables(const GqaParams &g, int bits, int qh, int units, cudaStream_t st) {
+  const dim3 grid(units, 2, 4), block(256);
+  if (bits == 1) return qh == 4 ? launch_after(gqa_tables_kernel<1, 4>, grid, block, 0, st, g)
+                                : launch_after(gqa_tables_kernel<1, 2>, grid, block, 0, st, g);
+  return qh == 4 ? launch_after(gqa_tables_kernel<2, 4>, grid, block, 0, st, g)
+                 : launch_after(gqa_tables_kernel<2, 2>, grid, block, 0, st, g);
+}
 
 cudaError_t launch_logits_gqa(const LogitsParams &p, const GqaParams &g, int bits, int n_seq, size_t limit,
                               cudaStream_t st) {

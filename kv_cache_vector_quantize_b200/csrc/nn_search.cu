@@ -654,6 +654,53 @@ cudaError_t launch_d(const NnArgs &a, cudaStream_t st) {
 
 }  // namespace
 
+namespace {
+// Top-k of n_parts sorted lists per query (score descending, then id ascending; id -1 marks an
+// empty place, only at a list's end): the same insertion order as nn_merge_kernel.
+__global__ void __launch_bounds__(128) nn_list_merge_kernel(const float *__restrict__ ps, const int64_t *__restrict__ pi,
+                                                            int n_parts, int n_q, int k, float *top_s,
+                                                            int64_t *top_i) {
+  const int qi = blockIdx.x * blockDim.x + threadIdx.x;
+  if (qi >= n_q) return;
+  float sv[kNnMaxK];
+  int64_t si[kNnMaxK];
+#pragma unroll
+  for (int j = 0; j < kNnMaxK; ++j) {
+    sv[j] = -INFINITY;
+    si[j] = -1;
+  }
+  for (int c = 0; c < n_parts; ++c) {
+    const size_t base = ((size_t)c * n_q + qi) * k;
+    for (int j = 0; j < k; ++j) {
+      float v = ps[base + j];
+      int64_t id = pi[base + j];
+      if (id < 0) break;
+#pragma unroll
+      for (int m = 0; m < kNnMaxK; ++m) {
+        if (m < k && (v > sv[m] || (v == sv[m] && id < si[m]) || si[m] < 0)) {
+          const float tv = sv[m];
+          const int64_t ti = si[m];
+          sv[m] = v;
+          si[m] = id;
+          v = tv;
+          id = ti;
+        }
+      }
+    }
+  }
+  for (int j = 0; j < k; ++j) {
+    top_s[(size_t)qi * k + j] = sv[j];
+    top_i[(size_t)qi * k + j] = si[j];
+  }
+}
+}  // namespace
+
+cudaError_t launch_nn_list_merge(const float *ps, const int64_t *pi, int n_parts, int n_q, int k, float *top_s,
+                                 int64_t *top_i, cudaStream_t st) {
+  nn_list_merge_kernel<<<(n_q + 127) / 128, 128, 0, st>>>(ps, pi, n_parts, n_q, k, top_s, top_i);
+  return cudaGetLastError();
+}
+
 bool nn_supported(int d, int bits) { return (d == 128 || d == 200) && bits >= 1 && bits <= 3; }
 
 int nn_kp(int d) { return 64 * ((2 * d + 63) / 64); }

@@ -280,8 +280,8 @@ __global__ void sketch_rotation_kernel(int d, const float *__restrict__ Pi, cons
 cudaError_t launch_quantize(const QuantParams &p, int bits, bool qjl, tq_dtype dtype, cudaStream_t st) {
   // bf16 / fp16 heads of 128 with 16-byte aligned rows and matrices take the tensor-core kernel (quantize_tc.cu)
   auto a16 = [](const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
-  if (p.d == 128 && p.n_hi == 0 && (dtype == TQ_BF16 || dtype == TQ_FP16) && a16(p.x) && a16(p.Pi) &&
-      (!qjl || a16(p.SPiT))) {
+  if (p.d == 128 && (p.n_hi == 0 || (p.n_hi == 64 && bits <= 3)) && (dtype == TQ_BF16 || dtype == TQ_FP16) &&
+      a16(p.x) && a16(p.Pi) && (!qjl || a16(p.SPiT))) {
     const cudaError_t e = launch_quantize_tc(p, bits, qjl, dtype == TQ_FP16, st);
     if (e != cudaErrorNotSupported) return e;   // else (no tensor map for these rows): the FP32 kernel below
   }

@@ -35,8 +35,16 @@
 // role stops and the others time out behind it; no MMA is in flight when
 // tensor memory is freed).
 // Shared-memory operand tiles use the 128-byte swizzle K-major layout of tc.cuh (sw128_off).
+//
+// Mixed rate (MIXED: fractional bits per channel, the first 64 rotated
+// coordinates at BITS + 1 code bits): the epilogue thread of columns [0, 64)
+// searches the wider codebook and writes its 64 (BITS+1)-bit codes first, the
+// thread of columns [64, 128) the BITS-bit codebook and codes after them; the
+// products are the same.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "tc.cuh"
@@ -107,8 +115,8 @@ struct Ws {
   static constexpr uint32_t kX = QJL ? 4 * kTile : 2 * kTile;                // kNX A tiles
   static constexpr uint32_t kRho = kX + kNX * kTile;                         // float[3][128] (keys)
   static constexpr uint32_t kNrm = kRho + (QJL ? 3 * 128 * 4 : 0);           // float[kNormRing][128] ||x||
-  static constexpr uint32_t kCb = kNrm + kNormRing * 128 * 4;                // float[16] centroids
-  static constexpr uint32_t kBar = kCb + 64;
+  static constexpr uint32_t kCb = kNrm + kNormRing * 128 * 4;                // float[32] centroids (two codebooks if mixed)
+  static constexpr uint32_t kBar = kCb + 128;
   // barriers: x_full[4], x_empty[4], d1_full[2], d1_empty[2], e_full, d2_full, d2_empty, n_full[kNormRing]
   static constexpr int kBars = 4 + 4 + 2 + 2 + 1 + 1 + 1 + kNormRing;
   static constexpr uint32_t kTslot = kBar + 8 * kBars;
@@ -496,15 +504,16 @@ __device__ __forceinline__ void mma_tile(uint32_t d, uint32_t a, uint32_t b, uin
                  idesc, (accumulate_first || s) ? 1u : 0u);
 }
 
-template <bool QJL, int BITS, bool F16>
+template <bool QJL, int BITS, bool F16, bool MIXED = false>
 __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
     quantize_tc_kernel(const QuantParams p, const __grid_constant__ CUtensorMap xmap) {
   using L = Ws<QJL>;
   constexpr int CPT = 64;                         // columns per epilogue thread
-  constexpr int WPT = CPT * BITS / 32;            // code-stream words per epilogue thread
-  constexpr int IW = BITS * kTD / 32;             // code-stream words per record
+  constexpr int B0 = MIXED ? BITS + 1 : BITS;     // code bits of columns [0, 64) (the other half: BITS)
+  constexpr int IW = (B0 + BITS) * CPT / 32;      // code-stream words per record
   constexpr int RW = IW + (QJL ? kTD / 32 : 0);   // record words
   constexpr int NL = 1 << BITS;
+  constexpr int NLM = 1 << B0;                    // levels of the wider codebook
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_wait();   // launched as a dependent of the previous work: it must be finished first
@@ -518,7 +527,7 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
   // ---- set-up: split matrices, codebook, barriers, tensor memory ----
   load_split<L::kThreads, F16, !QJL>(smem + L::kPhi, smem + L::kPlo, p.Pi);
   if constexpr (QJL) load_split<L::kThreads, F16>(smem + L::kMhi, smem + L::kMlo, p.SPiT);
-  if (tid < NL) cb[tid] = p.codebook[tid];
+  if (tid < NL + (MIXED ? NLM : 0)) cb[tid] = p.codebook[tid];
   if (tid == 0) {
     for (int s = 0; s < L::kNX; ++s) {
       mbar_init(bar.x_full(s), 1);                         // the copy thread's expect_tx
@@ -642,15 +651,17 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
     // thread: token t = tensor-memory lane, columns [64 h, 64 h + 64)
     const int q = warp & 3, h = warp >> 2, t = 32 * q + lane;
     const uint32_t lane_ofs = (uint32_t)(32 * q) << 16;
-    // thresholds: midpoints of consecutive centroids; keys also keep the centroids
-    constexpr int NC = QJL ? NL : 1;
-    float th[NL - 1], cvk[NC];
+    // thresholds: midpoints of consecutive centroids of this half's codebook (mixed: the wider one
+    // for h = 0, stored after the narrower one); keys also keep the centroids
+    const bool wide = MIXED && h == 0;
+    const float *cbh = wide ? cb + NL : cb;
+    const int nlh = wide ? NLM : NL;
+    constexpr int NC = QJL ? NLM : 1;
+    float th[NLM - 1], cvk[NC];
 #pragma unroll
-    for (int j = 0; j < NL - 1; ++j) th[j] = 0.5f * (cb[j] + cb[j + 1]);
+    for (int j = 0; j < NLM - 1; ++j) th[j] = j < nlh - 1 ? 0.5f * (cbh[j] + cbh[j + 1]) : 0.f;
 #pragma unroll
-    for (int j = 0; j < NC; ++j) cvk[j] = QJL && j < NL ? cb[j] : 0.f;
-    FmaSearch<BITS> fs;
-    fs.init(th);
+    for (int j = 0; j < NC; ++j) cvk[j] = QJL && j < nlh ? cbh[j] : 0.f;
     float *rho = reinterpret_cast<float *>(smem + L::kRho);   // [3][128]: the h = 1 half's sum of e^2
     float e2prev = 0.f;
     int64_t slot_prev = 0;
@@ -702,55 +713,67 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
           tc::fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar.d1_empty(db));   // D1 may take the next tile's product
-          uint32_t wcur[WPT];
+          // the codes of this thread's 64 columns at CB bits (CB = B0 for h = 0, BITS for h = 1)
+          auto codes = [&](auto cbits) {
+            constexpr int CB = decltype(cbits)::value;
+            constexpr int WPT = CPT * CB / 32;           // code-stream words of this thread
+            const float(&thc)[(1 << CB) - 1] = *reinterpret_cast<const float(*)[(1 << CB) - 1]>(&th[0]);
+            uint32_t wcur[WPT];
 #pragma unroll
-          for (int w = 0; w < WPT; ++w) wcur[w] = 0u;
-          if constexpr (QJL) {
-            // keys: y = D1 / n, code, residual e = y - c[code] (0 for a zero vector), split into
-            // bf16 parts and stored to E[i & 1] (free: the sketch product of tile i - 2 is done)
-            const float inv = n > 0.f ? 1.0f / n : 0.f;
-            const float nz = n > 0.f ? 1.f : 0.f;
-            const uint32_t e_hi = tmem + lane_ofs + L::kE + 128 * (i & 1) + 32 * h;
+            for (int w = 0; w < WPT; ++w) wcur[w] = 0u;
+            if constexpr (QJL) {
+              // keys: y = D1 / n, code, residual e = y - c[code] (0 for a zero vector), split into
+              // bf16 parts and stored to E[i & 1] (free: the sketch product of tile i - 2 is done)
+              const float(&cvc)[1 << CB] = *reinterpret_cast<const float(*)[1 << CB]>(&cvk[0]);
+              const float inv = n > 0.f ? 1.0f / n : 0.f;
+              const float nz = n > 0.f ? 1.f : 0.f;
+              const uint32_t e_hi = tmem + lane_ofs + L::kE + 128 * (i & 1) + 32 * h;
 #pragma unroll
-            for (int g = 0; g < CPT / 8; ++g) {
-              float ev[8];
+              for (int g = 0; g < CPT / 8; ++g) {
+                float ev[8];
 #pragma unroll
-              for (int qq = 0; qq < 8; ++qq) {
-                const int j = 8 * g + qq;
-                const float y = __uint_as_float(r[j]) * inv;   // 0 for a zero vector
-                uint32_t m[BITS];
-                code_masks<BITS>(y, th, m);
-                put_code<BITS>(wcur, m, j);
-                ev[qq] = fmaf(-nz, centroid_of<BITS>(m, cvk), y);
-                e2 = fmaf(ev[qq], ev[qq], e2);
+                for (int qq = 0; qq < 8; ++qq) {
+                  const int j = 8 * g + qq;
+                  const float y = __uint_as_float(r[j]) * inv;   // 0 for a zero vector
+                  uint32_t m[CB];
+                  code_masks<CB>(y, thc, m);
+                  put_code<CB>(wcur, m, j);
+                  ev[qq] = fmaf(-nz, centroid_of<CB>(m, cvc), y);
+                  e2 = fmaf(ev[qq], ev[qq], e2);
+                }
+                uint32_t hp[4], lp[4];
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) H16<F16>::split2(ev[2 * qq], ev[2 * qq + 1], hp[qq], lp[qq]);
+                tmem_st4(e_hi + 4 * g, hp[0], hp[1], hp[2], hp[3]);
+                tmem_st4(e_hi + 64 + 4 * g, lp[0], lp[1], lp[2], lp[3]);
               }
-              uint32_t hp[4], lp[4];
+              tmem_wait_st();
+              tc::fence_before();
+              if (h == 1) rho[(i % 3) * 128 + t] = e2;
+              __syncwarp();
+              if (lane == 0) mbar_arrive(bar.e_full());
+            } else {
+              // values need only the codes (FMA-pipe search on y = D1 / n, 0 for a zero vector)
+              FmaSearch<CB> fs;
+              fs.init(thc);
+              const float inv = n > 0.f ? 1.0f / n : 0.f;
 #pragma unroll
-              for (int qq = 0; qq < 4; ++qq) H16<F16>::split2(ev[2 * qq], ev[2 * qq + 1], hp[qq], lp[qq]);
-              tmem_st4(e_hi + 4 * g, hp[0], hp[1], hp[2], hp[3]);
-              tmem_st4(e_hi + 64 + 4 * g, lp[0], lp[1], lp[2], lp[3]);
+              for (int j = 0; j < CPT; ++j) {
+                float f[CB];
+                fs.flags(__uint_as_float(r[j]) * inv, f);
+                put_code_f<CB>(wcur, f, j);
+              }
+              fix_words<CB>(wcur, CPT);
             }
-            tmem_wait_st();
-            tc::fence_before();
-            if (h == 1) rho[(i % 3) * 128 + t] = e2;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar.e_full());
-          } else {
-            // values need only the codes (FMA-pipe search on y = D1 / n, 0 for a zero vector)
-            const float inv = n > 0.f ? 1.0f / n : 0.f;
+            if (valid) {
+              // h = 1 writes after the CPT * B0 bits of the h = 0 half
+              uint32_t *rec = p.records + slot * RW + (CPT * B0 / 32) * h;
 #pragma unroll
-            for (int j = 0; j < CPT; ++j) {
-              float f[BITS];
-              fs.flags(__uint_as_float(r[j]) * inv, f);
-              put_code_f<BITS>(wcur, f, j);
+              for (int w = 0; w < WPT; w += 2) st_global_v2(rec + w, wcur[w], wcur[w + 1]);
             }
-            fix_words<BITS>(wcur, CPT);
-          }
-          if (valid) {
-            uint32_t *rec = p.records + slot * RW + WPT * h;
-#pragma unroll
-            for (int w = 0; w < WPT; w += 2) st_global_v2(rec + w, wcur[w], wcur[w + 1]);
-          }
+          };
+          if (wide) codes(std::integral_constant<int, B0>{});
+          else codes(std::integral_constant<int, BITS>{});
         }
       }
       if constexpr (QJL) {
@@ -816,11 +839,11 @@ bool make_x_map(CUtensorMap *map, const QuantParams &p, bool f16) {
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool QJL, int BITS, bool F16>
+template <bool QJL, int BITS, bool F16, bool MIXED = false>
 cudaError_t launch_tc(const QuantParams &p, cudaStream_t st) {
   CUtensorMap xmap;
   if (p.rows >= (int64_t)1 << 31 || !make_x_map(&xmap, p, F16)) return cudaErrorNotSupported;
-  auto kern = quantize_tc_kernel<QJL, BITS, F16>;
+  auto kern = quantize_tc_kernel<QJL, BITS, F16, MIXED>;
   constexpr size_t smem = Ws<QJL>::kBytes;
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
@@ -832,6 +855,15 @@ cudaError_t launch_tc(const QuantParams &p, cudaStream_t st) {
 
 template <bool F16>
 cudaError_t launch_tc_t(const QuantParams &p, int bits, bool qjl, cudaStream_t st) {
+  if (p.n_hi == 64) {   // mixed rate: columns [0, 64) one bit wider
+    switch (bits) {
+      case 1: return qjl ? launch_tc<true, 1, F16, true>(p, st) : launch_tc<false, 1, F16, true>(p, st);
+      case 2: return qjl ? launch_tc<true, 2, F16, true>(p, st) : launch_tc<false, 2, F16, true>(p, st);
+      case 3: return qjl ? launch_tc<true, 3, F16, true>(p, st) : launch_tc<false, 3, F16, true>(p, st);
+      default: return cudaErrorNotSupported;
+    }
+  }
+  if (p.n_hi != 0) return cudaErrorNotSupported;
   switch (bits) {
     case 1: return qjl ? launch_tc<true, 1, F16>(p, st) : launch_tc<false, 1, F16>(p, st);
     case 2: return qjl ? launch_tc<true, 2, F16>(p, st) : launch_tc<false, 2, F16>(p, st);

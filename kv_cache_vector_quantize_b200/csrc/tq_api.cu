@@ -196,7 +196,7 @@ void clear_error() { g_err[0] = 0; }
 // tq_attend_v_noalloc so that both report the same status for the same bad argument.
 tq_status check_attend_args(const tq_cache *v, const float *logits, float scale, int32_t n_q_heads,
                             int64_t n_tokens, const float *Pi, const float *codebook, const float *out,
-                            const char *what) {
+                            const char *what, bool need_pi) {
   tq_status s = check_cache(v, what);
   if (s != TQ_OK) return s;
   if (v->qjl) return fail(TQ_ERR_INVALID, "%s: the cache is a key cache (qjl == 1)", what);
@@ -206,7 +206,7 @@ tq_status check_attend_args(const tq_cache *v, const float *logits, float scale,
   if (n_tokens < 0 || n_tokens > v->capacity)
     return fail(TQ_ERR_CAPACITY, "%s: n_tokens=%lld outside [0, capacity=%lld]", what, (long long)n_tokens,
                 (long long)v->capacity);
-  if ((!logits && n_tokens > 0) || !Pi || !codebook || !out)
+  if ((!logits && n_tokens > 0) || (need_pi && !Pi) || !codebook || !out)
     return fail(TQ_ERR_INVALID, "%s: NULL tensor argument", what);
   if (!(scale == scale) || scale == INFINITY || scale == -INFINITY)
     return fail(TQ_ERR_INVALID, "%s: scale is not finite", what);
@@ -417,24 +417,27 @@ size_t tq_attend_workspace_size(const tq_cache *v, int32_t n_q_heads, int64_t n_
   return attend_ws_bytes(v, n_q_heads, n_tokens);
 }
 
-tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale, int32_t n_q_heads, int64_t n_tokens,
-                      const float *Pi, const float *codebook, float *out, void *workspace, size_t workspace_bytes,
-                      tq_stream stream) {
-  g_err[0] = 0;
-  tq_status s = check_attend_args(v, logits, scale, n_q_heads, n_tokens, Pi, codebook, out, "tq_attend_v");
+namespace {
+// tq_attend_v, or with `merged` the merged partial (M, L, A) of this token range (tq_attend_v_partial).
+tq_status attend_impl(const tq_cache *v, const float *logits, float scale, int32_t n_q_heads, int64_t n_tokens,
+                      const float *Pi, const float *codebook, float *out, float *merged, void *workspace,
+                      size_t workspace_bytes, tq_stream stream, const char *what) {
+  tq_status s = check_attend_args(v, logits, scale, n_q_heads, n_tokens, Pi, codebook, merged ? merged : out, what,
+                                  merged == nullptr);
   if (s != TQ_OK) return s;
   const size_t need = tq_attend_workspace_size(v, n_q_heads, n_tokens);
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < need)
-    return fail(TQ_ERR_WORKSPACE, "tq_attend_v: workspace needs %zu bytes, 256-byte aligned (got %zu)", need,
+    return fail(TQ_ERR_WORKSPACE, "%s: workspace needs %zu bytes, 256-byte aligned (got %zu)", what, need,
                 workspace_bytes);
   if (injected(&s)) return s;
   const size_t out_bytes = sizeof(float) * (size_t)v->n_seq * n_q_heads * v->d;
   if (n_tokens == 0) {
-    cudaError_t e = cudaMemsetAsync(out, 0, out_bytes, (cudaStream_t)stream);
-    return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_attend_v (empty)");
+    cudaError_t e = merged ? launch_empty_partial(merged, v->n_seq * n_q_heads, v->d, (cudaStream_t)stream)
+                           : cudaMemsetAsync(out, 0, out_bytes, (cudaStream_t)stream);
+    return e == cudaSuccess ? TQ_OK : cuda_fail(e, what);
   }
   if ((n_tokens + kAttendChunk - 1) / kAttendChunk > 50000)
-    return fail(TQ_ERR_UNSUPPORTED, "tq_attend_v: n_tokens=%lld exceeds the merge limit of %lld tokens",
+    return fail(TQ_ERR_UNSUPPORTED, "%s: n_tokens=%lld exceeds the merge limit of %lld tokens", what,
                 (long long)n_tokens, 50000LL * kAttendChunk);
   uint32_t *status = static_cast<uint32_t *>(workspace);
   float *partial = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWsHeader);
@@ -460,8 +463,8 @@ tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale, int32
   p.q_per_cta = group < kAttendMaxQ ? group : kAttendMaxQ;
   p.qblocks = (group + p.q_per_cta - 1) / p.q_per_cta;
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), (cudaStream_t)stream);
-  if (e != cudaSuccess) return cuda_fail(e, "tq_attend_v (status)");
-  if (v->n_hi == 0 && attend_fast_supported(v->d, v->idx_bits, p.q_per_cta, v->records)) {
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  if (attend_fast_supported(v->d, v->idx_bits, p.q_per_cta, v->records, v->n_hi, v->capacity)) {
     // d = 128: tiles streamed by bulk copies, chunks sized to whole waves (never more chunks than
     // the 512-token split the workspace is sized for)
     p.chunk = attend_fast_chunk(n_tokens, v->n_seq * v->n_kv_heads * p.qblocks);
@@ -471,9 +474,55 @@ tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale, int32
     e = launch_attend(p, v->idx_bits, v->n_seq, attend_chunk_smem(v->d, p.rec_words, kAttendChunk),
                       (cudaStream_t)stream);
   }
-  if (e != cudaSuccess) return cuda_fail(e, "tq_attend_v (chunks)");
-  e = launch_combine(partial, v->n_seq * n_q_heads, p.n_chunks, v->d, Pi, out, (cudaStream_t)stream);
-  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_attend_v (merge)");
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  e = launch_combine(partial, v->n_seq * n_q_heads, p.n_chunks, v->d, Pi, out, (cudaStream_t)stream, merged);
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, what);
+}
+}  // namespace
+
+tq_status tq_attend_v(const tq_cache *v, const float *logits, float scale, int32_t n_q_heads, int64_t n_tokens,
+                      const float *Pi, const float *codebook, float *out, void *workspace, size_t workspace_bytes,
+                      tq_stream stream) {
+  g_err[0] = 0;
+  return attend_impl(v, logits, scale, n_q_heads, n_tokens, Pi, codebook, out, nullptr, workspace, workspace_bytes,
+                     stream, "tq_attend_v");
+}
+
+tq_status tq_attend_v_partial(const tq_cache *v, const float *logits, float scale, int32_t n_q_heads,
+                              int64_t n_tokens, const float *codebook, float *partial, void *workspace,
+                              size_t workspace_bytes, tq_stream stream) {
+  g_err[0] = 0;
+  if (!partial) return fail(TQ_ERR_INVALID, "tq_attend_v_partial: partial is NULL");
+  return attend_impl(v, logits, scale, n_q_heads, n_tokens, nullptr, codebook, nullptr, partial, workspace,
+                     workspace_bytes, stream, "tq_attend_v_partial");
+}
+
+tq_status tq_attend_merge(const float *partials, int32_t n_parts, int32_t rows, int32_t d, const float *Pi, float *out,
+                          tq_stream stream) {
+  g_err[0] = 0;
+  if (d < 8 || d > kMaxD || d % 8 != 0) return fail(TQ_ERR_UNSUPPORTED, "tq_attend_merge: d=%d", d);
+  if (n_parts < 1 || n_parts > 50000 || rows < 0)
+    return fail(TQ_ERR_INVALID, "tq_attend_merge: n_parts=%d (need 1..50000) rows=%d", n_parts, rows);
+  if (rows == 0) return TQ_OK;
+  if (!partials || !Pi || !out) return fail(TQ_ERR_INVALID, "tq_attend_merge: NULL tensor argument");
+  tq_status s;
+  if (injected(&s)) return s;
+  cudaError_t e = launch_combine(partials, rows, n_parts, d, Pi, out, (cudaStream_t)stream);
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_attend_merge");
+}
+
+tq_status tq_nn_merge(const float *part_scores, const int64_t *part_ids, int32_t n_parts, int32_t n_queries,
+                      int32_t k, float *top_scores, int64_t *top_ids, tq_stream stream) {
+  g_err[0] = 0;
+  if (k < 1 || k > kNnMaxK) return fail(TQ_ERR_INVALID, "tq_nn_merge: k=%d (need 1..%d)", k, kNnMaxK);
+  if (n_parts < 1 || n_queries < 0) return fail(TQ_ERR_INVALID, "tq_nn_merge: n_parts=%d n_queries=%d", n_parts, n_queries);
+  if (n_queries == 0) return TQ_OK;
+  if (!part_scores || !part_ids || !top_scores || !top_ids) return fail(TQ_ERR_INVALID, "tq_nn_merge: NULL tensor argument");
+  tq_status s;
+  if (injected(&s)) return s;
+  cudaError_t e = launch_nn_list_merge(part_scores, part_ids, n_parts, n_queries, k, top_scores, top_ids,
+                                       (cudaStream_t)stream);
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_nn_merge");
 }
 
 // Workspace of tq_decode_attend. Fused path: status word | Pi q | S q | chunk partials.
@@ -483,8 +532,10 @@ namespace {
 size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 struct DecodeWs {
-  bool fused;
-  size_t qrot, qsk, partial;                  // fused
+  bool fused, gqa;
+  size_t qrot, qsk, partial;                  // fused (one query head per KV head); partial also grouped
+  size_t tables, sigma;                       // fused grouped queries
+  int qh;                                     // query heads per grouped-query unit
   size_t logits, ws_l, ws_l_bytes, ws_a, ws_a_bytes;   // two calls
   size_t total;
 };
@@ -499,6 +550,9 @@ DecodeWs decode_ws(const tq_cache *k, const tq_cache *v, int n_q_heads, int64_t 
             decode_fused_supported(k->d, k->idx_bits, v->idx_bits, n_q_heads, k->n_kv_heads, k->records,
                                    v->records, device_smem_optin() - 1024);
   const size_t rows = (size_t)k->n_seq * n_q_heads;
+  const int group = n_q_heads / k->n_kv_heads;
+  w.gqa = !w.fused && k->n_hi == 0 && v->n_hi == 0 && group * k->n_kv_heads == n_q_heads &&
+          decode_gqa_supported(k->d, k->idx_bits, v->idx_bits, group, device_smem_optin() - 1024);
   if (w.fused) {
     const int64_t n_chunks = (n_tokens + kAttendChunk - 1) / kAttendChunk;   // at least as many as the split uses
     w.qrot = kWsHeader;
@@ -512,6 +566,18 @@ DecodeWs decode_ws(const tq_cache *k, const tq_cache *v, int n_q_heads, int64_t 
     w.ws_a = w.ws_l + w.ws_l_bytes;
     w.ws_a_bytes = tq_attend_workspace_size(v, n_q_heads, n_tokens);
     w.total = w.ws_a + w.ws_a_bytes;
+    if (w.gqa) {
+      // status word | tables of every unit | per-head table scales | chunk partials; the two-call
+      // layout (used when the matrices are not 16-byte aligned) also has to fit
+      w.qh = group >= 4 ? 4 : 2;
+      const int units = k->n_seq * k->n_kv_heads * (group / w.qh);
+      const int64_t n_chunks = (n_tokens + kAttendChunk - 1) / kAttendChunk;   // at least as many as the split uses
+      w.tables = kWsHeader;
+      w.sigma = w.tables + align256(gqa_table_bytes(units));
+      w.partial = w.sigma + align256(sizeof(float) * rows);
+      const size_t total_gqa = w.partial + sizeof(float) * rows * (size_t)n_chunks * (k->d + 2);
+      if (total_gqa > w.total) w.total = total_gqa;
+    }
   }
   return w;
 }
@@ -565,6 +631,58 @@ tq_status tq_decode_attend(const tq_cache *k, const tq_cache *v, const float *q,
     e = cudaMemsetAsync(out, 0, out_bytes, (cudaStream_t)stream);
     if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, sizeof(uint32_t), (cudaStream_t)stream);
     return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_decode_attend (empty)");
+  }
+  if (w.gqa && aligned(Pi, 16) && aligned(S, 16)) {
+    // grouped queries: the grouped-query tables once per call (they also clear the status word),
+    // then one pass over keys and values per (chunk, unit), then the merge
+    const int group = n_q_heads / k->n_kv_heads;
+    const int qblocks = group / w.qh;
+    const int units = k->n_seq * k->n_kv_heads * qblocks;
+    unsigned char *tables = reinterpret_cast<unsigned char *>(ws + w.tables);
+    float *sigma = reinterpret_cast<float *>(ws + w.sigma);
+    float *partial = reinterpret_cast<float *>(ws + w.partial);
+    GqaParams g{};
+    g.q = q;
+    g.Pi = Pi;
+    g.S = S;
+    g.codebook = codebook_k;
+    g.tables = tables;
+    g.sigma = sigma;
+    g.status = status;
+    g.n_kv_heads = k->n_kv_heads;
+    g.n_q_heads = n_q_heads;
+    g.group = group;
+    g.qblocks = qblocks;
+    e = launch_gqa_tables(g, k->idx_bits, w.qh, units, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "tq_decode_attend (grouped-query tables)");
+    DecodeGqaArgs a{};
+    a.krec = k->records;
+    a.knorm = k->norm;
+    a.krnorm = k->rnorm;
+    a.vrec = v->records;
+    a.vnorm = v->norm;
+    a.tables = tables;
+    a.sigma = sigma;
+    a.cbv = codebook_v;
+    a.partial = partial;
+    a.status = status;
+    a.n_tokens = n_tokens;
+    a.cap_k = k->capacity;
+    a.cap_v = v->capacity;
+    a.chunk = attend_fast_chunk(n_tokens, units);   // the softmax.V kernel's split
+    a.n_seq = k->n_seq;
+    a.n_kv_heads = k->n_kv_heads;
+    a.n_q_heads = n_q_heads;
+    a.qblocks = qblocks;
+    a.n_chunks = (int)((n_tokens + a.chunk - 1) / a.chunk);
+    a.kbits = k->idx_bits;
+    a.vbits = v->idx_bits;
+    a.scale = scale;
+    a.smem_limit = device_smem_optin() - 1024;
+    e = launch_decode_gqa(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "tq_decode_attend (grouped-query pass)");
+    e = launch_combine(partial, k->n_seq * n_q_heads, a.n_chunks, k->d, Pi, out, (cudaStream_t)stream);
+    return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_decode_attend (merge)");
   }
   if (!w.fused) {
     // other head groupings and code widths: the two calls, their status words merged into this one

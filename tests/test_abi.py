@@ -228,3 +228,25 @@ def test_mixed_rate_descriptors_checked():
     desc = tqb.TqCacheDesc(128, 2, 1, 1, 1, 64, 1000, FAKE, FAKE + 4096, FAKE + 8192)
     st = lib.tq_nn_search(ctypes.byref(desc), FAKE, 10, 1000, FAKE, FAKE, FAKE, 10, FAKE, FAKE, FAKE, 1 << 30, None)
     assert st == tqb.TQ_ERR_UNSUPPORTED
+
+
+def test_merge_and_partial_entry_points_check_arguments():
+    # top-k merge: k outside 1..16, no parts, NULL outputs
+    assert lib.tq_nn_merge(FAKE, FAKE, 2, 10, 17, FAKE, FAKE, None) == tqb.TQ_ERR_INVALID
+    assert lib.tq_nn_merge(FAKE, FAKE, 0, 10, 5, FAKE, FAKE, None) == tqb.TQ_ERR_INVALID
+    assert lib.tq_nn_merge(FAKE, FAKE, 2, 10, 5, None, FAKE, None) == tqb.TQ_ERR_INVALID
+    assert lib.tq_nn_merge(FAKE, FAKE, 2, 0, 5, None, None, None) == tqb.TQ_OK      # nothing to merge
+    # softmax.V merge: unsupported d, no parts, NULL matrix
+    assert lib.tq_attend_merge(FAKE, 2, 4, 12, FAKE, FAKE, None) == tqb.TQ_ERR_UNSUPPORTED
+    assert lib.tq_attend_merge(FAKE, 0, 4, 128, FAKE, FAKE, None) == tqb.TQ_ERR_INVALID
+    assert lib.tq_attend_merge(FAKE, 2, 4, 128, None, FAKE, None) == tqb.TQ_ERR_INVALID
+    # partial: the checks of tq_attend_v (a key cache is refused; NULL output), without Pi
+    kdesc = _desc(qjl=1)
+    assert lib.tq_attend_v_partial(ctypes.byref(kdesc), FAKE, ctypes.c_float(0.1), 2, 8, FAKE, FAKE, FAKE, 1 << 20,
+                                   None) == tqb.TQ_ERR_INVALID
+    vdesc = _desc(qjl=0, bits=3)
+    assert lib.tq_attend_v_partial(ctypes.byref(vdesc), FAKE, ctypes.c_float(0.1), 2, 8, FAKE, None, FAKE, 1 << 20,
+                                   None) == tqb.TQ_ERR_INVALID
+    # valid arguments reach the (injected) launch failure
+    assert lib.tq_attend_v_partial(ctypes.byref(vdesc), FAKE, ctypes.c_float(0.1), 2, 8, FAKE, FAKE, FAKE, 1 << 20,
+                                   None) == tqb.TQ_ERR_CUDA

@@ -285,13 +285,21 @@ def test_logits_unaligned_query_and_matrices(kb, G):
 
 DECODE_SHAPES = [
     # k index bits, v bits, n_seq, kv heads, group, tokens: one query head per KV head takes the fused
-    # pass (1- or 2-bit key codes), every other shape the two calls inside the same entry point
+    # pass (1- or 2-bit key codes), 2 / 4 / 8 query heads per KV head the fused grouped-query pass
+    # (1- or 2-bit key codes, 1..3-bit value codes), every other shape the two calls inside the same
+    # entry point
     (2, 3, 2, 3, 1, 1537),
     (1, 2, 1, 2, 1, 777),
     (2, 4, 1, 1, 1, 4096),
     (2, 1, 3, 1, 1, 130),
     (3, 3, 1, 2, 1, 901),
     (2, 3, 1, 2, 4, 1100),
+    (1, 2, 2, 2, 2, 777),
+    (2, 3, 1, 2, 8, 1537),
+    (2, 1, 1, 3, 4, 130),
+    (2, 2, 2, 1, 4, 5000),
+    (1, 3, 1, 1, 2, 257),
+    (2, 4, 1, 1, 4, 600),
 ]
 
 
@@ -334,13 +342,16 @@ def test_decode_attend_caches_of_different_capacity():
     tqb.tq_quantize_append(kc, k, 0, g["Pi"], g["SPiT"], g["ck"])
     tqb.tq_quantize_append(vc, v, 0, g["Pi"], None, g["cv"])
     sc = 1.0 / math.sqrt(d)
-    lg = tqb.tq_logits(kc, q, T, g["Pi"], g["S"], g["ck"])
-    out2 = tqb.tq_attend_v(vc, lg, sc, T, g["Pi"], g["cv"])
-    ws = torch.empty(max(256, tqb.tq_decode_workspace_size(kc, vc, H, T)), dtype=torch.uint8, device="cuda")
-    out1 = tqb.tq_decode_attend(kc, vc, q, T, sc, g["Pi"], g["S"], g["ck"], g["cv"], workspace=ws)
-    torch.cuda.synchronize()
-    tqb.tq_workspace_status(ws)
-    assert torch.equal(out1, out2)
+    for G in (1, 4):   # the single-head and the grouped-query fused passes
+        qg = syn.gaussian((B, H * G, d), 74 + G).cuda()
+        lg = tqb.tq_logits(kc, qg, T, g["Pi"], g["S"], g["ck"])
+        out2 = tqb.tq_attend_v(vc, lg, sc, T, g["Pi"], g["cv"])
+        ws = torch.empty(max(256, tqb.tq_decode_workspace_size(kc, vc, H * G, T)), dtype=torch.uint8, device="cuda")
+        out1 = tqb.tq_decode_attend(kc, vc, qg, T, sc, g["Pi"], g["S"], g["ck"], g["cv"], workspace=ws)
+        torch.cuda.synchronize()
+        tqb.tq_workspace_status(ws)
+        assert torch.equal(out1, out2), G
+    del q
 
 
 # ---------------------------------------------------------------------------
@@ -464,6 +475,7 @@ def test_llama_decode_full_size():
     k, v, q = syn.llama_inputs(device="cuda")
     Pi, S, ck, cv, g = _setup(128, 2, 3)
     kc, vc, lg, out, sc = _run_path(k, v, q, 128, 2, 3, g)
+    _decode_full_size(kc, vc, q.cuda(), 32768, sc, g, out)   # the fused grouped-query pass, bit-equal
     rng = np.random.default_rng(17)
     rows = np.sort(rng.choice(32768, size=1024, replace=False))
     kx = k[0].float().cpu().numpy()
