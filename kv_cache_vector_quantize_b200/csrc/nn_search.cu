@@ -152,13 +152,17 @@ __device__ __forceinline__ uint4 nn_unit_reg(const uint32_t *rec, int uk, uint32
   return make_uint4(0u, 0u, 0u, 0u);
 }
 
-// Sorted (descending) top-k of one thread's stream in the last k of kNnMaxK slots; the first
-// kNnMaxK - k slots hold +inf and never move, so the k-th score is always the last slot. A new
-// score goes behind equal ones: within one stream the indices increase.
+// Sorted (descending score, then ascending index) top-k of one thread's stream in the last k of
+// kNnMaxK slots; the first kNnMaxK - k slots hold +inf and never move, so the k-th score is always
+// the last slot. A new score goes behind equal ones (within one stream the indices increase); an
+// entry that an insertion pushes down keeps its place ahead of equal scores with higher indices,
+// so an equal-scored entry of a higher index is the one that falls off the end.
 __device__ __forceinline__ void topk_insert(float (&sv)[kNnMaxK], int (&si)[kNnMaxK], float v, int id) {
+  bool moved = false;   // once the new entry is placed, the entries behind it shift down one slot each
 #pragma unroll
   for (int j = 0; j < kNnMaxK; ++j) {
-    if (v > sv[j]) {
+    if (moved || v > sv[j]) {
+      moved = true;
       const float tv = sv[j];
       const int ti = si[j];
       sv[j] = v;

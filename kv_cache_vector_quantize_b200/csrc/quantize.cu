@@ -100,8 +100,13 @@ __device__ __forceinline__ void project(const float *__restrict__ gmat, float *m
   }
 }
 
+// Blocks per SM: d > 128 streams the matrices in chunks between block barriers, so two CTAs per
+// SM let one CTA's barrier waits overlap the other's products.
+template <int DP>
+constexpr int q_blocks_per_sm() { return DP > 128 ? 2 : 1; }
+
 template <int DP, bool QJL, typename Tin>
-__global__ void __launch_bounds__(kQThreads, 1) quantize_kernel(const QuantParams p, const int bits) {
+__global__ void __launch_bounds__(kQThreads, q_blocks_per_sm<DP>()) quantize_kernel(const QuantParams p, const int bits) {
   using Lay = QLayout<DP>;
   constexpr int CPL = Lay::CPL;
   extern __shared__ __align__(16) float smem[];
@@ -246,7 +251,8 @@ cudaError_t launch_q(const QuantParams &p, int bits, cudaStream_t st) {
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
   const int64_t tiles = (p.rows + kQTile - 1) / kQTile;
-  const int grid = (int)(tiles < (int64_t)device_sm_count() ? tiles : device_sm_count());
+  const int64_t slots = (int64_t)device_sm_count() * q_blocks_per_sm<DP>();
+  const int grid = (int)(tiles < slots ? tiles : slots);
   kern<<<grid, kQThreads, smem, st>>>(p, bits);
   return cudaGetLastError();
 }

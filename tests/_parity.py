@@ -140,6 +140,13 @@ def check_nn(gpu_s, gpu_i, q, Pi, S, codebook, rec, norm, rnorm, d, bits, k):
         tol_j = LOGIT_TOL * qn[a] * np.asarray(norm)[ids] + 1e-30
         err = np.abs(sc - ref[a, ids])
         assert np.all(err <= tol_j), f"query {a}: score error {np.max(err / tol_j):.3g} x tolerance"
+        # a returned vector must not have an exactly equal oracle score with a lower index that was
+        # left out (identical records tie exactly; the lower index ranks first)
+        left_out = np.ones(n_db, dtype=bool)
+        left_out[ids] = False
+        for j in ids:
+            tied = np.nonzero(left_out[:j] & (ref[a, :j] == ref[a, j]))[0]
+            assert len(tied) == 0, f"query {a}: id {j} returned ahead of the equal-scored lower id {tied[0]}"
         tol = LOGIT_TOL * qn[a] * nmax + 1e-30
         order = np.sort(ref[a])[::-1][:kk]
         oerr = np.abs(sc - order)

@@ -453,6 +453,24 @@ def test_nn_search_equal_vectors_rank_by_index():
     assert torch.all(sc == sc[:, :1]).item()
 
 
+@pytest.mark.parametrize("k", [1, 3, 5, 10])
+def test_nn_search_duplicates_pushed_down_keep_index_order(k):
+    # vectors 0..119 stored again at 150..269: identical records tie exactly. When a later, higher
+    # score pushes a tied pair down the running list, the lower index must stay and the higher fall
+    # off (the case of a duplicate at the k-th place with a better vector after both)
+    d, bits, n = 128, 2, 300
+    db, qs = syn.nn_inputs(n, 200, d)
+    db[150:270] = db[0:120]
+    _, _, _, _, g = _setup(d, bits, 1)
+    Pi, S, ck = g["Pi"].cpu().numpy(), g["S"].cpu().numpy(), g["ck"].cpu().numpy()
+    cache = tqb.PackedCache.empty(d, bits, True, 1, 1, n)
+    tqb.tq_quantize_append(cache, db.reshape(1, 1, n, d).cuda(), 0, g["Pi"], g["SPiT"], g["ck"])
+    sc, ids = tqb.tq_nn_search(cache, qs.cuda(), n, g["Pi"], g["S"], g["ck"], k)
+    rec = par.as_u32(cache.records[0, 0].cpu().numpy())
+    par.check_nn(sc.cpu().numpy(), ids.cpu().numpy(), qs.numpy().astype(np.float64), Pi, S, ck, rec,
+                 cache.norm[0, 0].cpu().numpy(), cache.rnorm[0, 0].cpu().numpy(), d, bits, k)
+
+
 def test_decode_attend_empty():
     d = 128
     _, _, _, _, g = _setup(d, 2, 3)
