@@ -74,6 +74,9 @@ def parse():
     ap.add_argument("--workload", default="large-b3",
                     choices=["llama"] + [f"sweep-b{b}{s}" for b in (2, 3, 4, 2.5, 3.5) for s in ("", "-s4")]
                     + ["large-b3", "large-b4", "nn-b2", "nn-b4", "nn-b2-s", "nn-b4-s"])
+    ap.add_argument("--split", choices=["layers", "heads"], default="layers",
+                    help="large-model cache on N GPUs: every rank streams its own layers (weak scaling), or "
+                         "every layer's KV heads are split over the ranks (strong scaling); no exchange either way")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -141,6 +144,14 @@ def fit_codebooks(tqb, d, idx, n_hi):
     the 2^(idx+1) centroids of its wider group (tq_codebook_fit, host setup)."""
     c = tqb.tq_codebook_fit(d, idx)
     return torch.cat([c, tqb.tq_codebook_fit(d, idx + 1)]) if n_hi else c
+
+
+def head_split(n_heads: int, world: int, rank: int) -> tuple[int, int]:
+    """[first, end) of the KV heads rank owns when every layer's heads are split evenly over the ranks."""
+    if world < 1 or not 0 <= rank < world or n_heads % world:
+        raise ValueError(f"{n_heads} KV heads do not split evenly over {world} ranks")
+    per = n_heads // world
+    return rank * per, (rank + 1) * per
 
 
 def rank_seed(rank: int) -> int:
@@ -447,6 +458,11 @@ def run_large(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = workload(args.workload)
+    by_heads = args.split == "heads" and world > 1
+    if by_heads:
+        # this rank's slice of every layer: KV heads [h0, h1) and their query heads
+        h0, h1 = head_split(w["hkv"], world, rank)
+        w = dict(w, hkv=h1 - h0, hq=(h1 - h0) * (w["hq"] // w["hkv"]))
     d, H, T = w["d"], w["hkv"], w["T"]
     n_layers = 80
     Pi = syn.rotation(d).to(dev)
@@ -482,6 +498,8 @@ def run_large(args, rank, world, local_rank):
             ev[len(calls)].record(stream)
 
     def layer_inputs(step):
+        if by_heads:   # the same layer on every rank, each generating its own heads
+            return syn.large_layer_inputs(step % n_layers + 1000 * rank, n_heads=H, device=dev)
         return w["gen"](dev, step % n_layers + rank_seed(rank))
 
     for i in range(args.warmup):
@@ -577,6 +595,7 @@ def run_large(args, rank, world, local_rank):
 
     kb, vb = key_bytes(w), value_bytes(w)
     fp16_bytes = 2 * H * T * d * 2
+    lw = world if by_heads else 1   # ranks holding parts of one layer
     peaks, peak_src = load_peaks()
     hbm = float(peaks["hbm_gbs"])
     bf16 = float(peaks["bf16_tflops"])
@@ -604,10 +623,12 @@ def run_large(args, rank, world, local_rank):
     att_gbs = vb / (att_ms * 1e-3) / 1e9
     result = {
         "metric": METRIC, "value": round(world * scan_gbs, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(path_ms, 4), "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": round(path_ms, 4), "higher_is_better": True,
+        "scaling": "strong" if by_heads else "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
         "config": {"workload": w["name"].replace("L layers", f"{n_layers} layers"),
-                   "parallelism": "single" if world == 1 else f"replicas{world}",
+                   "parallelism": "single" if world == 1 else (f"heads{world}: {H} KV heads of every layer per rank"
+                                                               if by_heads else f"replicas{world}"),
                    "step": "one layer (layer seeds cycled over the 80 layers; its fp16 K/V generated on the device "
                            "before the step, outside the timed calls): quantize K and V, L2 flush, tq_logits, "
                            "tq_attend_v; ms_per_step = the four calls' device time, the flush excluded",
@@ -618,12 +639,13 @@ def run_large(args, rank, world, local_rank):
                    "dtype_note": "narrowest arithmetic on the path: fp16 tensor-core products with split operands "
                                  "and float32 accumulation in the quantizer; the single-head scan and softmax.V "
                                  "accumulate in float32"},
-        "quantize_tokens_per_s": round(world * T / (quant_ms * 1e-3), 1),
+        "quantize_tokens_per_s": round((1 if by_heads else world) * T / (quant_ms * 1e-3), 1),
         "quantize_head_vectors_per_s": round(world * 2 * hv_layer / (quant_ms * 1e-3), 1),
         "per_kernel_ms_per_layer": {n: round(x, 5) for n, x in step_ms.items()},
-        "compressed_bytes": {"per_layer": kb + vb, "timed_layers": args.steps * (kb + vb),
-                             "all_80_layers": n_layers * (kb + vb)},
-        "uncompressed_fp16_bytes": {"per_layer": fp16_bytes, "all_80_layers": n_layers * fp16_bytes},
+        # a whole layer (all ranks' heads when they are split)
+        "compressed_bytes": {"per_layer": lw * (kb + vb), "timed_layers": args.steps * lw * (kb + vb),
+                             "all_80_layers": n_layers * lw * (kb + vb)},
+        "uncompressed_fp16_bytes": {"per_layer": lw * fp16_bytes, "all_80_layers": n_layers * lw * fp16_bytes},
         "compression_ratio_vs_fp16": round(fp16_bytes / (kb + vb), 4),
         "packed_bytes": {"keys": kb, "values": vb},
         "roofline": roofline, "roofline_quantize_v": roof_qv,
