@@ -15,16 +15,19 @@
 // accumulates in float32 in tensor memory. The residual e (float32) is split
 // the same way, and (S Pi^T) e = E_hi M_hi^T + E_hi M_lo^T + E_lo M_hi^T
 // (three products; the dropped E_lo M_lo^T is below 2^-16 of the scale).
+// ||x|| is taken as ||Pi x|| (Pi orthogonal) from the same float32 product: the
+// split's error moves it by about 2^-17 / sqrt(d) of ||x||, far inside the 1e-5
+// tolerance, and no warp has to read the tile a second time.
 //
 // Warp roles (one persistent CTA per SM, 128-token tiles):
 //   - one copy thread: tensor-map copies of x straight into a ring of A tiles
 //     in shared memory (2 for keys, 4 for values), in the 128-byte swizzle layout;
-//   - 4 norm warps: ||x|| from each landed tile, written to the cache;
 //   - one MMA thread: for tile i, D1 = x Pi^T (two products); then, keys, the
 //     sketch product of tile i - 1, D2 = E M^T, with E (the split residual) read
 //     from tensor memory;
 //   - 8 epilogue warps, a warp pair per tensor-memory lane quarter splitting
-//     the 128 columns (one token per thread): D1 -> codes -> record words;
+//     the 128 columns (one token per thread): D1 -> ||x|| (the pair adds its two
+//     halves' squares through shared memory) -> codes -> record words;
 //     keys also write the residual parts into tensor memory (two E buffers, so
 //     tile i's residual never waits for tile i - 1's sketch product) and then
 //     turn D2 of tile i - 1 into sign words and ||e||.
@@ -57,7 +60,6 @@ constexpr int kTD = 128;                   // head dimension
 constexpr int kTT = 128;                   // tokens per tile (MMA M)
 constexpr uint32_t kTile = kTT * kTD * 2;  // bytes of one bf16 operand tile (32 KB)
 constexpr int kEpiWarps = 8;               // epilogue warps: 2 per lane quarter, 64 columns each
-constexpr int kNormRing = 8;               // ||x|| ring in shared memory (the norm warps run at most kNX + 1 tiles ahead)
 
 // The 16-bit operand type: bf16 (inputs in bf16) or f16 (inputs in fp16). A split
 // P = P_hi + P_lo rounds to nearest twice; RN pairs pack two values (lower index
@@ -100,10 +102,9 @@ struct H16 {
 
 template <bool QJL>
 struct Ws {
-  static constexpr int kNormWarps = 4;                  // ||x|| from the landed A tiles
-  static constexpr int kTmaWarp = kEpiWarps + kNormWarps;
+  static constexpr int kTmaWarp = kEpiWarps;
   static constexpr int kMmaWarp = kTmaWarp + 1;
-  static constexpr int kThreads = 32 * (kMmaWarp + 1);   // 448: at most 4 warps per SM sub-partition (128 registers)
+  static constexpr int kThreads = 32 * (kMmaWarp + 1);   // 320
   static constexpr int kNX = QJL ? 2 : 4;                // A-tile stages (tensor-map copies in flight)
   // values: Pi_hi and Pi_lo stacked as one 256-row B tile, so one N = 256 product per K step gives
   // both parts (summed by the epilogue), with two D1 buffers; keys: two N = 128 products into one D1
@@ -114,11 +115,11 @@ struct Ws {
   static constexpr uint32_t kMhi = 2 * kTile, kMlo = 3 * kTile;              // keys only
   static constexpr uint32_t kX = QJL ? 4 * kTile : 2 * kTile;                // kNX A tiles
   static constexpr uint32_t kRho = kX + kNX * kTile;                         // float[3][128] (keys)
-  static constexpr uint32_t kNrm = kRho + (QJL ? 3 * 128 * 4 : 0);           // float[kNormRing][128] ||x||
-  static constexpr uint32_t kCb = kNrm + kNormRing * 128 * 4;                // float[32] centroids (two codebooks if mixed)
+  static constexpr uint32_t kXch = kRho + (QJL ? 3 * 128 * 4 : 0);           // float2[2][2][128]: ||x|| halves
+  static constexpr uint32_t kCb = kXch + 2 * 2 * 128 * 8;                    // float[32] centroids (two codebooks if mixed)
   static constexpr uint32_t kBar = kCb + 128;
-  // barriers: x_full[4], x_empty[4], d1_full[2], d1_empty[2], e_full, d2_full, d2_empty, n_full[kNormRing]
-  static constexpr int kBars = 4 + 4 + 2 + 2 + 1 + 1 + 1 + kNormRing;
+  // barriers: x_full[4], x_empty[4], d1_full[2], d1_empty[2], e_full, d2_full, d2_empty
+  static constexpr int kBars = 4 + 4 + 2 + 2 + 1 + 1 + 1;
   static constexpr uint32_t kTslot = kBar + 8 * kBars;
   static constexpr uint32_t kBytes = kTslot + 16;
   static constexpr uint32_t kTmemCols = 512;   // keys: D1, D2, E[0], E[1]; values: D1[0], D1[1] (256 each)
@@ -137,7 +138,6 @@ struct Bars {
   __device__ uint32_t e_full() const { return base + 8u * 12; }
   __device__ uint32_t d2_full() const { return base + 8u * 13; }
   __device__ uint32_t d2_empty() const { return base + 8u * 14; }
-  __device__ uint32_t n_full(int k) const { return base + 8u * (15 + k); }
 };
 
 // Position of a CTA's current tile in the (sequence x head, token) grid, kept
@@ -375,12 +375,6 @@ __device__ __forceinline__ void put_code(uint32_t (&w)[NW], const uint32_t (&m)[
   }
 }
 
-// --------------------------------------------------------------------------
-// A tiles arrive by tensor-map copies (16 per tile, one per K chunk). The 4
-// norm warps then read them back: warp w owns tile rows [32 w, 32 w + 32);
-// lane l reads row 32 w + 8 g + (l & 7), 16-byte chunks 4 i + (l >> 3)
-// (g, i < 4), so each quarter-warp reads one contiguous 128-byte block.
-// --------------------------------------------------------------------------
 // One 2-D tensor-map copy: 64 columns (128 bytes) x 128 rows, landing as one K block of the
 // 128-byte swizzle layout (16 KB); completion counted on `bar`.
 __device__ __forceinline__ void tma_x_chunk(uint32_t dst, const CUtensorMap *map, int col, int row, uint32_t bar) {
@@ -390,81 +384,45 @@ __device__ __forceinline__ void tma_x_chunk(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
-// ||x|| of the four rows this lane holds; every lane of a row's quartet ends
-// with the full value. bf16 and fp16 squares are exact in float32, and a float32 sum of
-// 128 of them is within 128 * 2^-24 of ||x||^2 (half that on ||x||, inside the
-// 1e-5 tolerance); a row whose sum is outside [2^-100, 2^126) (an overflowed
-// or underflowed square, or a zero vector) is redone with rescaled values.
-// Each row's result depends on that row alone.
-template <bool F16>
-__device__ __forceinline__ void tile_norms(const unsigned char *xt, int w, int lane, float (&nrm)[4]) {
-  auto chunk = [&](int g, int i) {
-    return *reinterpret_cast<const uint4 *>(xt + tc::sw128_off(kTT, 32 * w + 8 * g + (lane & 7), 8 * (4 * i + (lane >> 3))));
-  };
-  uint4 v[4][4];   // all 16 chunks in flight before any arithmetic
+// ||x|| = ||Pi x|| of token t from its D1 row, whose 128 columns are split over
+// the pair of epilogue threads (h = 0, 1; warps q and q + 4). Each thread sums
+// its half's squares; a half whose sum leaves [2^-100, 2^125) (a zero half,
+// underflowed or overflowed squares) is summed again with its values scaled by
+// 2^-e, e the exponent of its largest magnitude, so that it stands for s * 4^e.
+// The pair swaps (s, e) through shared memory (xs: float2[2][128]) and both
+// threads combine the two halves in the same order, so they get the same n.
+// All 32 lanes of both warps must call it (named barrier 1 + q).
+template <int CPT>
+__device__ __forceinline__ float pair_norm(const uint32_t (&r)[CPT], float2 *xs, int h, int t, int q) {
+  float s = 0.f;
 #pragma unroll
-  for (int g = 0; g < 4; ++g)
+  for (int j = 0; j < CPT; ++j) s = fmaf(__uint_as_float(r[j]), __uint_as_float(r[j]), s);
+  int e = 0;
+  if (!(s >= 0x1p-100f && s < 0x1p125f)) {
+    uint32_t mx = 0;   // largest magnitude as a bit pattern (ordered like the magnitudes)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[g][i] = chunk(g, i);
-  float sf[4];
-  bool bad[4], any = false;
+    for (int j = 0; j < CPT; ++j) mx = max(mx, r[j] & 0x7FFFFFFFu);
+    if (mx == 0) {
+      s = 0.f;
+      e = -512;   // an all-zero half: never the larger exponent, and its share underflows to 0
+    } else {
+      e = max(-126, min(126, (int)(mx >> 23) - 127));
+      const float sc = __uint_as_float((uint32_t)(127 - e) << 23);   // 2^-e, a normal number
+      s = 0.f;
 #pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    float part[4];   // one accumulator per chunk: four short chains instead of one long one
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t wv[4] = {v[g][i].x, v[g][i].y, v[g][i].z, v[g][i].w};
-      float s = 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float a = H16<F16>::lo(wv[q]), b = H16<F16>::hi(wv[q]);
-        s = fmaf(a, a, fmaf(b, b, s));
+      for (int j = 0; j < CPT; ++j) {
+        const float v = __uint_as_float(r[j]) * sc;
+        s = fmaf(v, v, s);
       }
-      part[i] = s;
-    }
-    float s = (part[0] + part[1]) + (part[2] + part[3]);
-    s += __shfl_xor_sync(0xffffffffu, s, 8);
-    s += __shfl_xor_sync(0xffffffffu, s, 16);
-    sf[g] = s;
-    bad[g] = !(s >= 0x1p-100f && s < 0x1p126f);
-    any |= bad[g];
-    nrm[g] = sqrtf(s);
-  }
-  // fp16 values are below 2^16 and at least 2^-24, so their sums of squares never leave float32's
-  // range (a zero vector sums to exactly 0); for bf16 a row out of range is summed again with its
-  // values scaled by a power of two taken from its largest magnitude (exact scaling; squares more
-  // than 2^-100 below the largest one are negligible)
-  if (!F16 && __any_sync(0xffffffffu, any)) {   // the whole warp takes part in the shuffles
-#pragma unroll 1
-    for (int g = 0; g < 4; ++g) {
-      uint32_t mx = 0;   // largest |x| as a bit pattern (ordered like the magnitudes)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 v = chunk(g, i);
-        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) mx = max(mx, max((wv[q] << 16) & 0x7FFFFFFFu, wv[q] & 0x7FFF0000u));
-      }
-      mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-      mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      const int e = (int)(mx >> 23) - 127;            // exponent of the largest magnitude
-      const float sc = __uint_as_float((uint32_t)(127 - e) << 23);   // 2^-e (e in [-127, 127])
-      float s = 0.f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 v = chunk(g, i);
-        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float a = H16<F16>::lo(wv[q]) * sc, b = H16<F16>::hi(wv[q]) * sc;
-          s = fmaf(a, a, fmaf(b, b, s));
-        }
-      }
-      s += __shfl_xor_sync(0xffffffffu, s, 8);
-      s += __shfl_xor_sync(0xffffffffu, s, 16);
-      if (bad[g]) nrm[g] = mx == 0 ? 0.f : ldexpf(sqrtf(s), e);
     }
   }
+  xs[h * 128 + t] = make_float2(s, __int_as_float(e));
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+  const float2 a0 = xs[t], a1 = xs[128 + t];
+  const int e0 = __float_as_int(a0.y), e1 = __float_as_int(a1.y);
+  if ((e0 | e1) == 0) return sqrtf(a0.x + a1.x);
+  const int E = max(e0, e1);
+  return ldexpf(sqrtf(ldexpf(a0.x, 2 * (e0 - E)) + ldexpf(a1.x, 2 * (e1 - E))), E);
 }
 
 // D[tmem] (+)= A[tmem] * B[smem]^T, A in tensor memory (row m = lane m, two bf16
@@ -531,7 +489,7 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < L::kNX; ++s) {
       mbar_init(bar.x_full(s), 1);                         // the copy thread's expect_tx
-      mbar_init(bar.x_empty(s), 1 + 32 * L::kNormWarps);   // the first product's commit + the norm threads
+      mbar_init(bar.x_empty(s), 1);   // the first product's commit
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar.d1_full(b), 1);
@@ -540,7 +498,6 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
     mbar_init(bar.e_full(), kEpiWarps);
     mbar_init(bar.d2_full(), 1);
     mbar_init(bar.d2_empty(), kEpiWarps);
-    for (int k = 0; k < kNormRing; ++k) mbar_init(bar.n_full(k), 32 * L::kNormWarps);
     mbar_fence_init();
   }
   if (warp == 0) {
@@ -561,7 +518,7 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
       int issued = 0;
       for (int i = 0; i < n_my; ++i) {
         const int s = i % L::kNX;
-        // A tile s is free once tile i - kNX's first product is done and its norms are read
+        // A tile s is free once tile i - kNX's first product is done
         if (i >= L::kNX && !mbar_wait(bar.x_empty(s), ((i / L::kNX) - 1) & 1)) break;
         mbar_arrive_expect_tx(bar.x_full(s), kTile);
         const uint32_t dst = sbase + L::kX + s * kTile;
@@ -572,33 +529,6 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
       }
       // no copy may still be landing when the CTA exits
       for (int i = max(0, issued - L::kNX); i < issued; ++i) mbar_wait(bar.x_full(i % L::kNX), (i / L::kNX) & 1);
-    }
-  } else if (warp >= kEpiWarps && warp < L::kTmaWarp) {
-    // ------------------------------- norms -------------------------------
-    const int w = warp - kEpiWarps;
-    TileCursor cur;
-    cur.init(p);
-    for (int i = 0; i < n_my; ++i) {
-      const int s = i % L::kNX;
-      if (!mbar_wait(bar.x_full(s), (i / L::kNX) & 1)) {
-        ok = false;
-        break;
-      }
-      const int64_t row0 = row0_of(i);
-      float nrm[4];
-      tile_norms<F16>(smem + L::kX + s * kTile, w, lane, nrm);
-      mbar_arrive(bar.x_empty(s));   // this thread is done reading the tile
-      if ((lane >> 3) == 0) {
-        float *ring = reinterpret_cast<float *>(smem + L::kNrm) + (i & (kNormRing - 1)) * 128;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int r = 32 * w + 8 * g + lane;
-          ring[r] = nrm[g];
-          if (row0 + r < p.rows) p.norm[cur.slot(p, r)] = nrm[g];
-        }
-      }
-      cur.advance(p);
-      mbar_arrive(bar.n_full(i & (kNormRing - 1)));   // releases this lane's ring entries
     }
   } else if (warp == L::kMmaWarp) {
     // ----------------------------- MMA issuer ------------------------------
@@ -666,7 +596,7 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
     float e2prev = 0.f;
     int64_t slot_prev = 0;
     bool vprev = false;
-    const float *nrm_ring = reinterpret_cast<const float *>(smem + L::kNrm);
+    float2 *xch = reinterpret_cast<float2 *>(smem + L::kXch);   // [2][2][128]: ||x|| halves, by tile parity
     TileCursor cur;
     cur.init(p);
 
@@ -676,25 +606,17 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
       float e2 = 0.f;
       int64_t slot = 0;
       bool valid = false;
-      if (i < n_my && ok) {
-        // ---- first epilogue of tile i: codes (and, keys, the residual into E[i & 1]) ----
-        // ||x|| of this token from the norm warps' ring (read before D1 is released, which keeps
-        // the ring slot from being overwritten: see kNormRing)
-        float n = 0.f;
-        if (!mbar_wait(bar.n_full(i & (kNormRing - 1)), (i / kNormRing) & 1)) {
-          ok = false;
-        } else {
-          n = nrm_ring[(i & (kNormRing - 1)) * 128 + t];
-          valid = row0_of(i) + t < p.rows;
-          slot = valid ? cur.slot(p, t) : 0;
-          cur.advance(p);
-        }
+      if (i < n_my) {
+        // ---- first epilogue of tile i: ||x||, codes (and, keys, the residual into E[i & 1]) ----
+        valid = row0_of(i) + t < p.rows;
+        slot = valid ? cur.slot(p, t) : 0;
+        cur.advance(p);
         const int db = i % L::kND1;
-        if (!ok || !mbar_wait(bar.d1_full(db), (i / L::kND1) & 1)) {
-          ok = false;
-        } else {
+        uint32_t r[CPT];
+        // the tensor-memory loads are warp-wide: the whole warp loads or none of it does
+        const bool have = __all_sync(0xffffffffu, ok && mbar_wait(bar.d1_full(db), (i / L::kND1) & 1));
+        if (have) {
           tc::fence_after();
-          uint32_t r[CPT];
           const uint32_t d1 = tmem + lane_ofs + 256 * db + CPT * h;
           tc::ld32(d1, *reinterpret_cast<uint32_t (*)[32]>(r));
           tc::ld32(d1 + 32, *reinterpret_cast<uint32_t (*)[32]>(r + 32));
@@ -713,6 +635,15 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
           tc::fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar.d1_empty(db));   // D1 may take the next tile's product
+        } else {
+          ok = false;
+#pragma unroll
+          for (int j = 0; j < CPT; ++j) r[j] = 0u;
+        }
+        // both threads of the pair meet here every tile, whether or not their loads ran
+        const float n = pair_norm<CPT>(r, xch + (i & 1) * 256, h, t, q);
+        if (have) {
+          if (valid && h == 0) p.norm[slot] = n;
           // the codes of this thread's 64 columns at CB bits (CB = B0 for h = 0, BITS for h = 1)
           auto codes = [&](auto cbits) {
             constexpr int CB = decltype(cbits)::value;
@@ -781,7 +712,7 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
           // ---- second epilogue of tile i - 1: sign words and ||e|| ----
           const int j = i - 1;
           uint32_t sw[2] = {0u, 0u};
-          if (ok && mbar_wait(bar.d2_full(), j & 1)) {
+          if (__all_sync(0xffffffffu, ok && mbar_wait(bar.d2_full(), j & 1))) {
             tc::fence_after();
             uint32_t r[CPT];
             tc::ld32(tmem + lane_ofs + L::kD2 + CPT * h, *reinterpret_cast<uint32_t (*)[32]>(r));
