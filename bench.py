@@ -154,6 +154,16 @@ def head_split(n_heads: int, world: int, rank: int) -> tuple[int, int]:
     return rank * per, (rank + 1) * per
 
 
+def tensor_executed(products: int, d: int, head_vectors: int, ms: float, bf16: float) -> dict:
+    """Tensor work the d = 128 quantizer actually issues: its d x d products run on split 16-bit
+    operands (keys: Pi x as hi + lo, and the sketch as three split products; values: hi + lo),
+    `products` of them per head-vector at 2 d^2 flop each, against the dense bf16 peak."""
+    flop = products * 2 * d * d
+    tfs = flop * head_vectors / (ms * 1e-3) / 1e12
+    return {"products_per_head_vector": products, "flop_per_head_vector": flop, "tflops": round(tfs, 1),
+            "frac": round(tfs / bf16, 4)}
+
+
 def rank_seed(rank: int) -> int:
     """Seed of a rank's replica of the workload (ranks draw different data)."""
     return syn.SEED_DATA + 7919 * rank
@@ -402,6 +412,9 @@ def run_tq(args, rank, world, local_rank):
                           mean["quantize_k"], NCU_TRAFFIC.get(("quantize_k", args.workload)))
     roof_qv = quant_roof("quantize_tc_kernel, value launch (tq_quantize_append on the V cache)", qv_bytes, qv_flops,
                          mean["quantize_v"], NCU_TRAFFIC.get(("quantize_v", args.workload)))
+    if w["d"] == 128:
+        roofline["tensor_executed"] = tensor_executed(5, w["d"], head_vectors, mean["quantize_k"], bf16)
+        roof_qv["tensor_executed"] = tensor_executed(2, w["d"], head_vectors, mean["quantize_v"], bf16)
     roof_scan = {"kernel": "tq_logits (query projection + logit scan)", "bound": "hbm",
                  "achieved": round(scan_gbs_rank, 1), "peak": hbm, "unit": "GB/s",
                  "frac": round(scan_gbs_rank / hbm, 4), "traffic": NCU_TRAFFIC.get(("logits", args.workload)),
@@ -620,6 +633,8 @@ def run_large(args, rank, world, local_rank):
                           qk_flops, qk_ms, NCU_TRAFFIC.get(("quantize_k", args.workload)))
     roof_qv = quant_roof("quantize_tc_kernel, value launch (tq_quantize_append on the layer's V cache)", qv_bytes,
                          qv_flops, qv_ms, NCU_TRAFFIC.get(("quantize_v", args.workload)))
+    roofline["tensor_executed"] = tensor_executed(5, d, hv_layer, qk_ms, bf16)
+    roof_qv["tensor_executed"] = tensor_executed(2, d, hv_layer, qv_ms, bf16)
     att_gbs = vb / (att_ms * 1e-3) / 1e9
     result = {
         "metric": METRIC, "value": round(world * scan_gbs, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,

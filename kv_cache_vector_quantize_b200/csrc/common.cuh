@@ -151,7 +151,7 @@ cudaError_t launch_qprep(const float *q, int rows, int d, const float *Pi, const
                          float *qrot, float *qsk, uint32_t *status, cudaStream_t st);
 cudaError_t launch_logits(const LogitsParams &p, int bits, int n_seq, int n_chunks, size_t smem, cudaStream_t st);
 size_t logits_smem_per_query(int d, int bits, int n_hi = 0);
-int logits_fast_stages(int bits, int q, size_t limit);
+int logits_fast_stages(int bits, int q, size_t limit, int n_hi = 0);
 cudaError_t launch_logits_fast(const LogitsParams &p, int bits, int n_seq, size_t limit, cudaStream_t st);
 bool gqa_supported(int d, int bits, int group);
 size_t gqa_table_bytes(int units);

@@ -36,9 +36,12 @@ constexpr int kFMaxStages = 8;
 constexpr uint32_t kBarBytes = 2 * kFMaxStages * 8;
 constexpr uint32_t kQStage = 2048;                     // shared bytes for the staged Pi q and S q of 2 query heads
 
-template <int BETA>
-struct FastKeys : scan::FastKeys<BETA> {
-  static constexpr uint32_t kStageBytes = kFTile * (scan::FastKeys<BETA>::RW + 2) * 4;
+// Record words and stage bytes; MIXED: the mixed-rate record (scan::MixedKeys), whose 40 or 56 bytes
+// are not a multiple of 16: a tile with an odd number of keys gets its last record by plain loads.
+template <int BETA, bool MIXED = false>
+struct FastKeys {
+  static constexpr int RW = MIXED ? scan::MixedKeys<BETA>::RW : scan::FastKeys<BETA>::RW;
+  static constexpr uint32_t kStageBytes = kFTile * (RW + 2) * 4;
 };
 
 struct FastParams {
@@ -50,14 +53,14 @@ struct FastParams {
 };
 
 
-template <int BETA, int QMAX>
+template <int BETA, int QMAX, bool MIXED>
 __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastParams fp) {
-  using K = FastKeys<BETA>;
+  using K = FastKeys<BETA, MIXED>;
   constexpr int RW = K::RW;
   constexpr uint32_t SB = K::kStageBytes;
   const LogitsParams &p = fp.p;
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ float cbs[8];
+  __shared__ float cbs[24];   // the codebook (mixed: the narrow one, then the wide one)
 
   // ---- layout in the shared window ----
   const uint32_t dyn0 = smem_u32(smem);
@@ -105,7 +108,7 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
     }
     mbar_fence_init();
   }
-  if (tid < (1 << BETA)) cbs[tid] = p.codebook[tid];
+  if (tid < (1 << BETA) + (MIXED ? 2 << BETA : 0)) cbs[tid] = p.codebook[tid];
   __syncthreads();
 
   auto norms_by_copy = [&](size_t first, int n) {
@@ -127,11 +130,21 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
         const int64_t t0 = (int64_t)tile * kFTile;
         const int n = (int)min((int64_t)kFTile, p.n_tokens - t0);
         const size_t first = unit_first + t0;
-        const uint32_t rec_bytes = (uint32_t)n * RW * 4;
+        const uint32_t st = slot(s);
+        int ncopy = n;
+        if (MIXED && (n & 1)) {
+          // the last record by plain loads (before the arrival that completes the stage), the rest by copy
+          --ncopy;
+          const uint32_t *src = p.records + (first + ncopy) * RW;
+          uint32_t *dst = reinterpret_cast<uint32_t *>(smem + (st - dyn0)) + (size_t)ncopy * RW;
+#pragma unroll
+          for (int w = 0; w < RW; ++w) dst[w] = __ldg(src + w);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // ordered with the copy engine's writes
+        }
+        const uint32_t rec_bytes = (uint32_t)ncopy * RW * 4;
         const bool nc = norms_by_copy(first, n);
         mbar_arrive_expect_tx(full_bar(s), rec_bytes + (nc ? 8u * n : 0u));
-        const uint32_t st = slot(s);
-        bulk_g2s(st, p.records + first * RW, rec_bytes, full_bar(s));
+        if (rec_bytes > 0) bulk_g2s(st, p.records + first * RW, rec_bytes, full_bar(s));
         if (nc) {
           bulk_g2s(st + kFTile * RW * 4, p.norm + first, 4u * n, full_bar(s));
           bulk_g2s(st + kFTile * RW * 4 + kFTile * 4, p.rnorm + first, 4u * n, full_bar(s));
@@ -198,7 +211,11 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
       asm volatile("bar.sync 1, %0;" ::"n"(32 * kFConsumers) : "memory");
       for (int qq = 0; qq < nq; ++qq) {
         const float *qr = qv + qq * 2 * kFD;
-        scan::build_tables<BETA, kFTile>(qr, qr + kFD, tables + (size_t)qq * (kTabStride / 4), cbs, tid, kappa);
+        if constexpr (MIXED)
+          scan::build_tables_mixed<BETA, kFTile>(qr, qr + kFD, tables + (size_t)qq * (kTabStride / 4), cbs,
+                                                 cbs + (1 << BETA), tid, kappa);
+        else
+          scan::build_tables<BETA, kFTile>(qr, qr + kFD, tables + (size_t)qq * (kTabStride / 4), cbs, tid, kappa);
       }
       asm volatile("bar.sync 1, %0;" ::"n"(32 * kFConsumers) : "memory");
     }
@@ -214,7 +231,7 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
     // this lane's record, read whether or not the key exists: slots past n hold stale words whose
     // logits are never stored, so the load needs no branch
     uint32_t w[RW];
-    {
+    if constexpr (RW % 4 == 0) {
       const uint4 *src = reinterpret_cast<const uint4 *>(st + (size_t)k * RW * 4);
 #pragma unroll
       for (int j = 0; j < RW / 4; ++j) {
@@ -223,6 +240,14 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
         w[4 * j + 1] = v.y;
         w[4 * j + 2] = v.z;
         w[4 * j + 3] = v.w;
+      }
+    } else {   // mixed records: 8-byte aligned
+      const uint2 *src = reinterpret_cast<const uint2 *>(st + (size_t)k * RW * 4);
+#pragma unroll
+      for (int j = 0; j < RW / 2; ++j) {
+        const uint2 v = src[j];
+        w[2 * j] = v.x;
+        w[2 * j + 1] = v.y;
       }
     }
     float nrm, rho;
@@ -241,7 +266,8 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
     }
 
     float out[QMAX];
-    scan::key_logits<BETA, QMAX>(w, lane, T0, nq, nrm, rho, out);
+    if constexpr (MIXED) scan::key_logits_mixed<BETA, QMAX>(w, lane, T0, nq, nrm, rho, out);
+    else scan::key_logits<BETA, QMAX>(w, lane, T0, nq, nrm, rho, out);
     if (valid) {
 #pragma unroll
       for (int qq = 0; qq < QMAX; ++qq)
@@ -257,9 +283,9 @@ __global__ void __launch_bounds__(kFThreads, 1) logits_fast_kernel(const FastPar
 // Dynamic shared memory for QMAX query heads' tables with dynamic smem starting
 // at `dyn0` (the reserved region below it): the aligned table block plus as many
 // stage slots as fit, capped by the opt-in limit.
-template <int BETA>
+template <int BETA, bool MIXED = false>
 uint32_t fast_dyn_bytes(int qmax, uint32_t limit, int *stages_out) {
-  using K = FastKeys<BETA>;
+  using K = FastKeys<BETA, MIXED>;
   const uint32_t dyn0 = 1024;   // reserved shared memory below the dynamic window on sm_100
   const uint32_t T0 = (dyn0 + kBarBytes + kTabStride - 1) & ~(kTabStride - 1);
   const uint32_t n_a = (T0 - kQStage - dyn0 - kBarBytes) / K::kStageBytes;
@@ -275,15 +301,15 @@ uint32_t fast_dyn_bytes(int qmax, uint32_t limit, int *stages_out) {
   return end - dyn0;
 }
 
-template <int BETA, int QMAX>
+template <int BETA, int QMAX, bool MIXED = false>
 cudaError_t launch_fast(const LogitsParams &p, int n_seq, uint32_t limit, cudaStream_t st) {
   FastParams fp{};
   fp.p = p;
   fp.tiles_per_unit = (int)((p.n_tokens + kFTile - 1) / kFTile);
   fp.total_tiles = (int64_t)n_seq * p.n_kv_heads * p.qblocks * fp.tiles_per_unit;
   int stages = 0;
-  fp.dyn_bytes = fast_dyn_bytes<BETA>(QMAX, limit, &stages);
-  auto kern = logits_fast_kernel<BETA, QMAX>;
+  fp.dyn_bytes = fast_dyn_bytes<BETA, MIXED>(QMAX, limit, &stages);
+  auto kern = logits_fast_kernel<BETA, QMAX, MIXED>;
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), fp.dyn_bytes);
   if (e != cudaSuccess) return e;
   // Two splits over one CTA per SM, costed in tiles of the busiest CTA, a table
@@ -326,14 +352,20 @@ cudaError_t launch_fast(const LogitsParams &p, int n_seq, uint32_t limit, cudaSt
 }  // namespace
 
 // Stage slots the d = 128 scan gets for `q` query heads per CTA within `limit`
-// bytes of dynamic shared memory (0 if the tables do not fit).
-int logits_fast_stages(int bits, int q, size_t limit) {
+// bytes of dynamic shared memory (0 if the tables do not fit); n_hi = 64: the
+// mixed-rate records (bits 1 or 2).
+int logits_fast_stages(int bits, int q, size_t limit, int n_hi) {
   int stages = 0;
   const uint32_t lim = (uint32_t)limit;
-  switch (bits) {
-    case 1: fast_dyn_bytes<1>(q, lim, &stages); break;
-    case 2: fast_dyn_bytes<2>(q, lim, &stages); break;
-    default: fast_dyn_bytes<3>(q, lim, &stages); break;
+  if (n_hi == 64) {
+    if (bits == 1) fast_dyn_bytes<1, true>(q, lim, &stages);
+    else fast_dyn_bytes<2, true>(q, lim, &stages);
+  } else {
+    switch (bits) {
+      case 1: fast_dyn_bytes<1>(q, lim, &stages); break;
+      case 2: fast_dyn_bytes<2>(q, lim, &stages); break;
+      default: fast_dyn_bytes<3>(q, lim, &stages); break;
+    }
   }
   const uint32_t need = 65536 * (uint32_t)(q + 1);   // aligned table block inside the window
   return need <= lim + 1024 ? stages : 0;
@@ -342,6 +374,10 @@ int logits_fast_stages(int bits, int q, size_t limit) {
 cudaError_t launch_logits_fast(const LogitsParams &p, int bits, int n_seq, size_t limit, cudaStream_t st) {
   const int q = p.q_per_cta;
   const uint32_t lim = (uint32_t)limit;
+  if (p.n_hi == 64) {
+    if (bits == 1) return q == 1 ? launch_fast<1, 1, true>(p, n_seq, lim, st) : launch_fast<1, 2, true>(p, n_seq, lim, st);
+    return q == 1 ? launch_fast<2, 1, true>(p, n_seq, lim, st) : launch_fast<2, 2, true>(p, n_seq, lim, st);
+  }
   switch (bits) {
     case 1: return q == 1 ? launch_fast<1, 1>(p, n_seq, lim, st) : launch_fast<1, 2>(p, n_seq, lim, st);
     case 2: return q == 1 ? launch_fast<2, 1>(p, n_seq, lim, st) : launch_fast<2, 2>(p, n_seq, lim, st);

@@ -25,9 +25,10 @@
 //   - one MMA thread: for tile i, D1 = x Pi^T (two products); then, keys, the
 //     sketch product of tile i - 1, D2 = E M^T, with E (the split residual) read
 //     from tensor memory;
-//   - 8 epilogue warps, a warp pair per tensor-memory lane quarter splitting
-//     the 128 columns (one token per thread): D1 -> ||x|| (the pair adds its two
-//     halves' squares through shared memory) -> codes -> record words;
+//   - 8 epilogue warps (mixed rate: 16), NP = 2 (4) per tensor-memory lane
+//     quarter, splitting the 128 columns into NP parts (NP threads per token):
+//     D1 -> ||x|| (the token's threads add their parts' squares through shared
+//     memory) -> codes -> record words;
 //     keys also write the residual parts into tensor memory (two E buffers, so
 //     tile i's residual never waits for tile i - 1's sketch product) and then
 //     turn D2 of tile i - 1 into sign words and ||e||.
@@ -59,7 +60,6 @@ namespace {
 constexpr int kTD = 128;                   // head dimension
 constexpr int kTT = 128;                   // tokens per tile (MMA M)
 constexpr uint32_t kTile = kTT * kTD * 2;  // bytes of one bf16 operand tile (32 KB)
-constexpr int kEpiWarps = 8;               // epilogue warps: 2 per lane quarter, 64 columns each
 
 // The 16-bit operand type: bf16 (inputs in bf16) or f16 (inputs in fp16). A split
 // P = P_hi + P_lo rounds to nearest twice; RN pairs pack two values (lower index
@@ -100,11 +100,18 @@ struct H16 {
   }
 };
 
-template <bool QJL>
+// Epilogue threads per token (NP parts of kTD / NP columns): 2 for the integer rates, 4 for the
+// mixed rate, whose wider half has more code-search work per column (measured best for each).
+template <bool MIXED>
+constexpr int epi_parts() { return MIXED ? 4 : 2; }
+
+template <bool QJL, int NP>
 struct Ws {
+  static constexpr int kParts = NP;                      // epilogue threads per token
+  static constexpr int kEpiWarps = 4 * NP;               // NP warps per tensor-memory lane quarter
   static constexpr int kTmaWarp = kEpiWarps;
   static constexpr int kMmaWarp = kTmaWarp + 1;
-  static constexpr int kThreads = 32 * (kMmaWarp + 1);   // 320
+  static constexpr int kThreads = 32 * (kMmaWarp + 1);   // 320 (168 registers a thread) or 576 (96)
   static constexpr int kNX = QJL ? 2 : 4;                // A-tile stages (tensor-map copies in flight)
   // values: Pi_hi and Pi_lo stacked as one 256-row B tile, so one N = 256 product per K step gives
   // both parts (summed by the epilogue), with two D1 buffers; keys: two N = 128 products into one D1
@@ -114,9 +121,9 @@ struct Ws {
   static constexpr uint32_t kPhi = 0, kPlo = kTile;
   static constexpr uint32_t kMhi = 2 * kTile, kMlo = 3 * kTile;              // keys only
   static constexpr uint32_t kX = QJL ? 4 * kTile : 2 * kTile;                // kNX A tiles
-  static constexpr uint32_t kRho = kX + kNX * kTile;                         // float[3][128] (keys)
-  static constexpr uint32_t kXch = kRho + (QJL ? 3 * 128 * 4 : 0);           // float2[2][2][128]: ||x|| halves
-  static constexpr uint32_t kCb = kXch + 2 * 2 * 128 * 8;                    // float[32] centroids (two codebooks if mixed)
+  static constexpr uint32_t kRho = kX + kNX * kTile;                         // float[3][kParts][128] (keys)
+  static constexpr uint32_t kXch = kRho + (QJL ? 3 * kParts * 128 * 4 : 0);  // float2[2][kParts][128]: ||x|| parts
+  static constexpr uint32_t kCb = kXch + 2 * kParts * 128 * 8;               // float[32] centroids (two codebooks if mixed)
   static constexpr uint32_t kBar = kCb + 128;
   // barriers: x_full[4], x_empty[4], d1_full[2], d1_empty[2], e_full, d2_full, d2_empty
   static constexpr int kBars = 4 + 4 + 2 + 2 + 1 + 1 + 1;
@@ -385,15 +392,15 @@ __device__ __forceinline__ void tma_x_chunk(uint32_t dst, const CUtensorMap *map
 }
 
 // ||x|| = ||Pi x|| of token t from its D1 row, whose 128 columns are split over
-// the pair of epilogue threads (h = 0, 1; warps q and q + 4). Each thread sums
-// its half's squares; a half whose sum leaves [2^-100, 2^125) (a zero half,
+// the NP epilogue threads of the token (part h; warps q + 4 h). Each thread sums
+// its part's squares; a part whose sum leaves [2^-100, 2^125) (a zero part,
 // underflowed or overflowed squares) is summed again with its values scaled by
 // 2^-e, e the exponent of its largest magnitude, so that it stands for s * 4^e.
-// The pair swaps (s, e) through shared memory (xs: float2[2][128]) and both
-// threads combine the two halves in the same order, so they get the same n.
-// All 32 lanes of both warps must call it (named barrier 1 + q).
-template <int CPT>
-__device__ __forceinline__ float pair_norm(const uint32_t (&r)[CPT], float2 *xs, int h, int t, int q) {
+// The threads swap (s, e) through shared memory (xs: float2[NP][128]) and each
+// combines the NP parts in the same order, so all get the same n. All 32 lanes
+// of the NP warps must call it (named barrier 1 + q).
+template <int CPT, int NP>
+__device__ __forceinline__ float part_norm(const uint32_t (&r)[CPT], float2 *xs, int h, int t, int q) {
   float s = 0.f;
 #pragma unroll
   for (int j = 0; j < CPT; ++j) s = fmaf(__uint_as_float(r[j]), __uint_as_float(r[j]), s);
@@ -404,7 +411,7 @@ __device__ __forceinline__ float pair_norm(const uint32_t (&r)[CPT], float2 *xs,
     for (int j = 0; j < CPT; ++j) mx = max(mx, r[j] & 0x7FFFFFFFu);
     if (mx == 0) {
       s = 0.f;
-      e = -512;   // an all-zero half: never the larger exponent, and its share underflows to 0
+      e = -512;   // an all-zero part: never the larger exponent, and its share underflows to 0
     } else {
       e = max(-126, min(126, (int)(mx >> 23) - 127));
       const float sc = __uint_as_float((uint32_t)(127 - e) << 23);   // 2^-e, a normal number
@@ -417,12 +424,25 @@ __device__ __forceinline__ float pair_norm(const uint32_t (&r)[CPT], float2 *xs,
     }
   }
   xs[h * 128 + t] = make_float2(s, __int_as_float(e));
-  asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
-  const float2 a0 = xs[t], a1 = xs[128 + t];
-  const int e0 = __float_as_int(a0.y), e1 = __float_as_int(a1.y);
-  if ((e0 | e1) == 0) return sqrtf(a0.x + a1.x);
-  const int E = max(e0, e1);
-  return ldexpf(sqrtf(ldexpf(a0.x, 2 * (e0 - E)) + ldexpf(a1.x, 2 * (e1 - E))), E);
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "n"(32 * NP) : "memory");
+  float2 a[NP];
+  int any = 0, E = -512;
+#pragma unroll
+  for (int k = 0; k < NP; ++k) {
+    a[k] = xs[k * 128 + t];
+    any |= __float_as_int(a[k].y);
+    E = max(E, __float_as_int(a[k].y));
+  }
+  if (any == 0) {   // no part rescaled: the plain sum (fewer than 2^126 in total)
+    float tot = a[0].x;
+#pragma unroll
+    for (int k = 1; k < NP; ++k) tot += a[k].x;
+    return sqrtf(tot);
+  }
+  float tot = 0.f;
+#pragma unroll
+  for (int k = 0; k < NP; ++k) tot += ldexpf(a[k].x, 2 * (__float_as_int(a[k].y) - E));
+  return ldexpf(sqrtf(tot), E);
 }
 
 // D[tmem] (+)= A[tmem] * B[smem]^T, A in tensor memory (row m = lane m, two bf16
@@ -463,12 +483,14 @@ __device__ __forceinline__ void mma_tile(uint32_t d, uint32_t a, uint32_t b, uin
 }
 
 template <bool QJL, int BITS, bool F16, bool MIXED = false>
-__global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
+__global__ void __launch_bounds__(Ws<QJL, epi_parts<MIXED>()>::kThreads, 1)
     quantize_tc_kernel(const QuantParams p, const __grid_constant__ CUtensorMap xmap) {
-  using L = Ws<QJL>;
-  constexpr int CPT = 64;                         // columns per epilogue thread
+  using L = Ws<QJL, epi_parts<MIXED>()>;
+  constexpr int kParts = L::kParts;
+  constexpr int kEpiWarps = L::kEpiWarps;
+  constexpr int CPT = kTD / kParts;               // columns per epilogue thread
   constexpr int B0 = MIXED ? BITS + 1 : BITS;     // code bits of columns [0, 64) (the other half: BITS)
-  constexpr int IW = (B0 + BITS) * CPT / 32;      // code-stream words per record
+  constexpr int IW = (B0 + BITS) * (kTD / 2) / 32;   // code-stream words per record
   constexpr int RW = IW + (QJL ? kTD / 32 : 0);   // record words
   constexpr int NL = 1 << BITS;
   constexpr int NLM = 1 << B0;                    // levels of the wider codebook
@@ -578,12 +600,15 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
     }
   } else {
     // ------------------------------- epilogue -------------------------------
-    // thread: token t = tensor-memory lane, columns [64 h, 64 h + 64)
+    // thread: token t = tensor-memory lane, columns [CPT h, CPT h + CPT)
     const int q = warp & 3, h = warp >> 2, t = 32 * q + lane;
     const uint32_t lane_ofs = (uint32_t)(32 * q) << 16;
-    // thresholds: midpoints of consecutive centroids of this half's codebook (mixed: the wider one
-    // for h = 0, stored after the narrower one); keys also keep the centroids
-    const bool wide = MIXED && h == 0;
+    // thresholds: midpoints of consecutive centroids of this part's codebook (mixed: the wider one
+    // for columns [0, 64), stored after the narrower one); keys also keep the centroids
+    const bool wide = MIXED && h < kParts / 2;
+    // this part's first code-stream word: mixed, the wider parts come first
+    const int woff = !MIXED ? h * (CPT * BITS / 32)
+                            : (wide ? h * (CPT * B0 / 32) : (kParts / 2) * (CPT * B0 / 32) + (h - kParts / 2) * (CPT * BITS / 32));
     const float *cbh = wide ? cb + NL : cb;
     const int nlh = wide ? NLM : NL;
     constexpr int NC = QJL ? NLM : 1;
@@ -592,16 +617,15 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
     for (int j = 0; j < NLM - 1; ++j) th[j] = j < nlh - 1 ? 0.5f * (cbh[j] + cbh[j + 1]) : 0.f;
 #pragma unroll
     for (int j = 0; j < NC; ++j) cvk[j] = QJL && j < nlh ? cbh[j] : 0.f;
-    float *rho = reinterpret_cast<float *>(smem + L::kRho);   // [3][128]: the h = 1 half's sum of e^2
-    float e2prev = 0.f;
+    float *rho = reinterpret_cast<float *>(smem + L::kRho);   // [3][kParts][128]: each part's sum of e^2
     int64_t slot_prev = 0;
     bool vprev = false;
-    float2 *xch = reinterpret_cast<float2 *>(smem + L::kXch);   // [2][2][128]: ||x|| halves, by tile parity
+    float2 *xch = reinterpret_cast<float2 *>(smem + L::kXch);   // [2][kParts][128]: ||x|| parts, by tile parity
     TileCursor cur;
     cur.init(p);
 
     // Every epilogue thread runs all n_my + 1 iterations (after a failed wait it
-    // skips the work but still meets the pair barrier of each iteration).
+    // skips the work but still meets the token's barriers of each iteration).
     for (int i = 0; i <= n_my; ++i) {
       float e2 = 0.f;
       int64_t slot = 0;
@@ -618,8 +642,8 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
         if (have) {
           tc::fence_after();
           const uint32_t d1 = tmem + lane_ofs + 256 * db + CPT * h;
-          tc::ld32(d1, *reinterpret_cast<uint32_t (*)[32]>(r));
-          tc::ld32(d1 + 32, *reinterpret_cast<uint32_t (*)[32]>(r + 32));
+#pragma unroll
+          for (int c = 0; c < CPT / 32; ++c) tc::ld32(d1 + 32 * c, *reinterpret_cast<uint32_t (*)[32]>(r + 32 * c));
           tc::wait_ld();
           if constexpr (L::kPW == 256) {
             // the lo-part product sits 128 columns to the right: D1 = x Pi_hi^T + x Pi_lo^T
@@ -640,11 +664,11 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
 #pragma unroll
           for (int j = 0; j < CPT; ++j) r[j] = 0u;
         }
-        // both threads of the pair meet here every tile, whether or not their loads ran
-        const float n = pair_norm<CPT>(r, xch + (i & 1) * 256, h, t, q);
+        // the token's threads meet here every tile, whether or not their loads ran
+        const float n = part_norm<CPT, kParts>(r, xch + (i & 1) * (kParts * 128), h, t, q);
         if (have) {
           if (valid && h == 0) p.norm[slot] = n;
-          // the codes of this thread's 64 columns at CB bits (CB = B0 for h = 0, BITS for h = 1)
+          // the codes of this thread's CPT columns at CB bits (B0 for the wider parts, else BITS)
           auto codes = [&](auto cbits) {
             constexpr int CB = decltype(cbits)::value;
             constexpr int WPT = CPT * CB / 32;           // code-stream words of this thread
@@ -658,7 +682,7 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
               const float(&cvc)[1 << CB] = *reinterpret_cast<const float(*)[1 << CB]>(&cvk[0]);
               const float inv = n > 0.f ? 1.0f / n : 0.f;
               const float nz = n > 0.f ? 1.f : 0.f;
-              const uint32_t e_hi = tmem + lane_ofs + L::kE + 128 * (i & 1) + 32 * h;
+              const uint32_t e_hi = tmem + lane_ofs + L::kE + 128 * (i & 1) + (CPT / 2) * h;
 #pragma unroll
               for (int g = 0; g < CPT / 8; ++g) {
                 float ev[8];
@@ -680,7 +704,7 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
               }
               tmem_wait_st();
               tc::fence_before();
-              if (h == 1) rho[(i % 3) * 128 + t] = e2;
+              rho[((i % 3) * kParts + h) * 128 + t] = e2;
               __syncwarp();
               if (lane == 0) mbar_arrive(bar.e_full());
             } else {
@@ -697,10 +721,14 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
               fix_words<CB>(wcur, CPT);
             }
             if (valid) {
-              // h = 1 writes after the CPT * B0 bits of the h = 0 half
-              uint32_t *rec = p.records + slot * RW + (CPT * B0 / 32) * h;
+              uint32_t *rec = p.records + slot * RW + woff;
+              if (WPT % 2 == 0 && (woff & 1) == 0) {
 #pragma unroll
-              for (int w = 0; w < WPT; w += 2) st_global_v2(rec + w, wcur[w], wcur[w + 1]);
+                for (int w = 0; w < WPT; w += 2) st_global_v2(rec + w, wcur[w], wcur[(w + 1) % WPT]);
+              } else {
+#pragma unroll
+                for (int w = 0; w < WPT; ++w) rec[w] = wcur[w];
+              }
             }
           };
           if (wide) codes(std::integral_constant<int, B0>{});
@@ -711,31 +739,40 @@ __global__ void __launch_bounds__(Ws<QJL>::kThreads, 1)
         if (i >= 1) {
           // ---- second epilogue of tile i - 1: sign words and ||e|| ----
           const int j = i - 1;
-          uint32_t sw[2] = {0u, 0u};
+          uint32_t sw[CPT / 32];
+#pragma unroll
+          for (int c = 0; c < CPT / 32; ++c) sw[c] = 0u;
           if (__all_sync(0xffffffffu, ok && mbar_wait(bar.d2_full(), j & 1))) {
             tc::fence_after();
             uint32_t r[CPT];
-            tc::ld32(tmem + lane_ofs + L::kD2 + CPT * h, *reinterpret_cast<uint32_t (*)[32]>(r));
-            tc::ld32(tmem + lane_ofs + L::kD2 + CPT * h + 32, *reinterpret_cast<uint32_t (*)[32]>(r + 32));
+#pragma unroll
+            for (int c = 0; c < CPT / 32; ++c)
+              tc::ld32(tmem + lane_ofs + L::kD2 + CPT * h + 32 * c, *reinterpret_cast<uint32_t (*)[32]>(r + 32 * c));
             tc::wait_ld();
             tc::fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar.d2_empty());
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
+            for (int c = 0; c < CPT / 32; ++c)
 #pragma unroll
               for (int qq = 0; qq < 32; ++qq) put_bit(sw[c], ge0(__uint_as_float(r[32 * c + qq])), qq);
           } else {
             ok = false;
           }
-          // pair barrier (warps q and q + 4): the h = 1 partner's sum of e^2 for tile j is visible
-          asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+          // the token's barrier (warps q + 4 h): every part's sum of e^2 for tile j is visible
+          asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "n"(32 * kParts) : "memory");
           if (ok && vprev) {
-            st_global_v2(p.records + slot_prev * RW + IW + 2 * h, sw[0], sw[1]);
-            if (h == 0) p.rnorm[slot_prev] = sqrtf(e2prev + rho[(j % 3) * 128 + t]);
+            uint32_t *sdst = p.records + slot_prev * RW + IW + (CPT / 32) * h;
+            if constexpr (CPT == 64) st_global_v2(sdst, sw[0], sw[CPT / 32 - 1]);
+            else sdst[0] = sw[0];
+            if (h == 0) {
+              float e2s = 0.f;
+#pragma unroll
+              for (int k = 0; k < kParts; ++k) e2s += rho[((j % 3) * kParts + k) * 128 + t];
+              p.rnorm[slot_prev] = sqrtf(e2s);
+            }
           }
         }
-        e2prev = e2;
         slot_prev = slot;
         vprev = valid;
       }
@@ -775,13 +812,14 @@ cudaError_t launch_tc(const QuantParams &p, cudaStream_t st) {
   CUtensorMap xmap;
   if (p.rows >= (int64_t)1 << 31 || !make_x_map(&xmap, p, F16)) return cudaErrorNotSupported;
   auto kern = quantize_tc_kernel<QJL, BITS, F16, MIXED>;
-  constexpr size_t smem = Ws<QJL>::kBytes;
+  using L = Ws<QJL, epi_parts<MIXED>()>;
+  constexpr size_t smem = L::kBytes;
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
   const int64_t tiles = (p.rows + kTT - 1) / kTT;
   const int64_t slots = (int64_t)device_sm_count();
   const int grid = (int)(tiles < slots ? tiles : slots);
-  return launch_after(kern, dim3(grid), dim3(Ws<QJL>::kThreads), smem, st, p, xmap);
+  return launch_after(kern, dim3(grid), dim3(L::kThreads), smem, st, p, xmap);
 }
 
 template <bool F16>

@@ -309,5 +309,123 @@ __device__ __forceinline__ void build_tables(const float *qr, const float *qs, f
   }
 }
 
+// ---------------------------------------------------------------------------
+// Mixed rate (fractional bits per channel): the first 64 rotated coordinates at
+// BETA + 1 code bits, the other 64 at BETA (BETA = 1: 2.5 bits per channel with
+// the sign bit, BETA = 2: 3.5). The record holds the 64 wide codes, the 64
+// narrow codes and the 16 sign bytes back to back. Keys are taken two wide
+// coordinates at a time (32 keys of 2 (BETA + 1) bits) and 8 / BETA narrow bits
+// at a time (4-bit keys: 32 of them for BETA = 2, 16 for BETA = 1), plus the 16
+// sign bytes; every table has rows of 32 words (a key shifted to bit 7) and one
+// column per key position, read at position (s + l) mod 32 after the lane's
+// streams are rotated, as for the 6-bit keys above. Sets of 16 positions sit
+// twice (p and p + 16). Per query head: wide tables at +0 (2^(2 BETA + 2) rows),
+// narrow at +8 KB (16 rows), signs at +32 KB (256 rows).
+template <int BETA>
+struct MixedKeys {
+  static constexpr int WW = 2 * (BETA + 1);      // wide code words (64 codes of BETA + 1 bits)
+  static constexpr int NW = 2 * BETA;            // narrow code words
+  static constexpr int IW = WW + NW;
+  static constexpr int RW = IW + kFD / 32;       // + the sign words
+  static constexpr int KW = 2 * (BETA + 1);      // wide key bits (two coordinates)
+  static constexpr int NKN = BETA == 2 ? 32 : 16;   // narrow 4-bit keys
+  static constexpr int CN = 4 / BETA;            // coordinates per narrow key
+  static constexpr uint32_t kNarrow = 8192, kSign = 32768;   // byte offsets in a query head's tables
+};
+
+template <int BETA, int QQ>
+__device__ __forceinline__ float scan_mixed(const uint32_t (&wr)[MixedKeys<BETA>::WW],
+                                            const uint32_t (&nr)[MixedKeys<BETA>::NW], const uint32_t (&rs)[4],
+                                            const uint32_t (&bank)[32], float nrm, float rho) {
+  using M = MixedKeys<BETA>;
+  float a[4], b[2];   // each chain starts at its first lookup
+#pragma unroll
+  for (int st = 0; st < 32; ++st) {
+    const float v = lds_at<QQ * kTabStride>(key_addr7<M::KW>(wr, M::KW * st, bank[st]));
+    a[st & 1] = st < 2 ? v : a[st & 1] + v;
+  }
+#pragma unroll
+  for (int st = 0; st < M::NKN; ++st) {
+    const float v = lds_at<QQ * kTabStride + M::kNarrow>(key_addr7<4>(nr, 4 * st, bank[st]));
+    a[2 + (st & 1)] = st < 2 ? v : a[2 + (st & 1)] + v;
+  }
+#pragma unroll
+  for (int st = 0; st < 16; ++st) {
+    const float v = lds_at<QQ * kTabStride + M::kSign>(key_addr7<8>(rs, 8 * st, bank[st]));
+    b[st & 1] = st < 2 ? v : b[st & 1] + v;
+  }
+  const float a0 = a[0], a1 = a[1], a2 = a[2], a3 = a[3], b0 = b[0], b1 = b[1];
+  return nrm * fmaf(rho, b0 + b1, (a0 + a1) + (a2 + a3));
+}
+
+// The logits of one mixed-rate key record for QMAX query heads (as key_logits).
+template <int BETA, int QMAX>
+__device__ __forceinline__ void key_logits_mixed(const uint32_t (&w)[MixedKeys<BETA>::RW], int lane, uint32_t T0,
+                                                 int nq, float nrm, float rho, float (&out)[QMAX]) {
+  using M = MixedKeys<BETA>;
+#pragma unroll
+  for (int qq = 0; qq < QMAX; ++qq) out[qq] = 0.f;
+  uint32_t bank[32];
+#pragma unroll
+  for (int s2 = 0; s2 < 32; ++s2) bank[s2] = T0 | (uint32_t)(((s2 + lane) & 31) << 2);
+  uint32_t wr[M::WW], nr[M::NW], rs[4];
+#pragma unroll
+  for (int j = 0; j < M::WW; ++j) wr[j] = w[j];
+#pragma unroll
+  for (int j = 0; j < M::NW; ++j) nr[j] = w[M::WW + j];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) rs[j] = w[M::IW + j];
+  rotate_stream<M::WW>(wr, M::KW * lane);
+  rotate_stream<M::NW>(nr, 4 * (lane & (M::NKN - 1)));
+  rotate_stream<4>(rs, 8 * (lane & 15));
+  out[0] = scan_mixed<BETA, 0>(wr, nr, rs, bank, nrm, rho);
+  if constexpr (QMAX > 1)
+    if (nq > 1) out[1] = scan_mixed<BETA, 1>(wr, nr, rs, bank, nrm, rho);
+}
+
+// The mixed-rate tables of one query head at tq_, from qr = Pi q and qs = S q;
+// cbn / cbw: the narrow (2^BETA) and wide (2^(BETA+1)) codebooks. Each thread
+// keeps one table position and walks the key values with a stride of NTHR / 32,
+// so a warp shares one key: codebook reads broadcast and stores hit 32 banks.
+template <int BETA, int NTHR>
+__device__ __forceinline__ void build_tables_mixed(const float *qr, const float *qs, float *tq_, const float *cbn,
+                                                   const float *cbw, int tid, float kappa) {
+  using M = MixedKeys<BETA>;
+  constexpr int LW = 1 << (BETA + 1), LN = 1 << BETA;
+  const int pos = tid & 31, k0 = tid >> 5;
+  constexpr int KS = NTHR / 32;
+  {   // wide: position pos = coordinates 2 pos, 2 pos + 1
+    const float q0 = qr[2 * pos], q1 = qr[2 * pos + 1];
+    for (int key = k0; key < (1 << M::KW); key += KS)
+      tq_[key * 32 + pos] = fmaf(q1, cbw[key >> (BETA + 1)], q0 * cbw[key & (LW - 1)]);
+  }
+  {   // narrow: position pos (mod the key count) = coordinates 64 + CN p .. 64 + CN p + CN - 1
+    const int pn = pos & (M::NKN - 1);
+    float qn[M::CN];
+#pragma unroll
+    for (int c = 0; c < M::CN; ++c) qn[c] = qr[64 + M::CN * pn + c];
+    float *tn = tq_ + M::kNarrow / 4;
+    for (int key = k0; key < 16; key += KS) {
+      float v = qn[0] * cbn[key & (LN - 1)];
+#pragma unroll
+      for (int c = 1; c < M::CN; ++c) v = fmaf(qn[c], cbn[(key >> (BETA * c)) & (LN - 1)], v);
+      tn[key * 32 + pos] = v;
+    }
+  }
+  {   // signs: position pos (mod 16) = 8 sign bits, +-kappa (S q)_i
+    const int t = pos & 15;
+    float sv[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) sv[c] = kappa * qs[8 * t + c];
+    float *ts = tq_ + M::kSign / 4;
+    for (int key = k0; key < 256; key += KS) {
+      float v = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) v += ((key >> c) & 1) ? sv[c] : -sv[c];
+      ts[key * 32 + pos] = v;
+    }
+  }
+}
+
 }  // namespace scan
 }  // namespace tq

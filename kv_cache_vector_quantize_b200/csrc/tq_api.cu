@@ -119,12 +119,15 @@ struct FastPlan {
 
 FastPlan plan_fast(const tq_cache *k, int n_q_heads) {
   FastPlan f{false, 0, 0};
-  if (k->d != 128 || k->idx_bits > 3 || !k->qjl || k->n_hi != 0) return f;
+  if (k->d != 128 || k->idx_bits > 3 || !k->qjl) return f;
+  // mixed rate: the first 64 coordinates one bit wider, 2.5 or 3.5 bits per channel; the rows of
+  // every (sequence, head) start on 16 bytes (a record is 40 or 56 bytes: an even capacity)
+  if (k->n_hi != 0 && !(k->n_hi == 64 && k->idx_bits <= 2 && k->capacity % 2 == 0)) return f;
   const int group = n_q_heads / k->n_kv_heads;
   const size_t limit = device_smem_optin() - 1024;
   int q = 0;
-  if (group >= 2 && logits_fast_stages(k->idx_bits, 2, limit) >= 3) q = 2;
-  else if (logits_fast_stages(k->idx_bits, 1, limit) >= 2) q = 1;
+  if (group >= 2 && logits_fast_stages(k->idx_bits, 2, limit, k->n_hi) >= 3) q = 2;
+  else if (logits_fast_stages(k->idx_bits, 1, limit, k->n_hi) >= 2) q = 1;
   if (q == 0) return f;
   f = FastPlan{true, q, limit};
   return f;

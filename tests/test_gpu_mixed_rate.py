@@ -46,6 +46,8 @@ SHAPES = [
     (64, 1, 32, 3, 32, 1, 2, 2, 513, torch.float32),
     (200, 2, 96, 2, 32, 1, 1, 3, 300, torch.float32),
     (128, 3, 32, 3, 96, 1, 1, 1, 130, torch.bfloat16),    # keys with 4-bit high-group codes
+    (128, 2, 64, 2, 64, 1, 2, 2, 513, torch.bfloat16),    # 3.5 / 2.5 bits: a last tile of one record
+    (128, 2, 64, 2, 64, 1, 1, 2, 300, torch.bfloat16),    # odd capacity: rows not 16-byte aligned
 ]
 
 
