@@ -31,7 +31,10 @@
 //     memory) -> codes -> record words;
 //     keys also write the residual parts into tensor memory (two E buffers, so
 //     tile i's residual never waits for tile i - 1's sketch product) and then
-//     turn D2 of tile i - 1 into sign words and ||e||.
+//     turn D2 of tile i - 1 into sign words and ||e||;
+//   - integer-rate keys with 2- or more-bit codes: that last step runs on 4
+//     sign warps of its own (a whole token per thread), so the epilogue warps
+//     never wait for the sketch product.
 // Tensor memory (keys): D1 [0, 128), D2 [128, 256), E[b] at 256 + 128 b
 // (E_hi: 64 columns of bf16 pairs, E_lo: the next 64). D1 and D2 are read
 // into registers and released at once, so one buffer of each suffices.
@@ -104,14 +107,22 @@ struct H16 {
 // mixed rate, whose wider half has more code-search work per column (measured best for each).
 template <bool MIXED>
 constexpr int epi_parts() { return MIXED ? 4 : 2; }
+// Keys with 2- and 3-bit codes: 4 sign warps (one per lane quarter, a whole token per thread) turn D2
+// into sign words and rho, so the epilogue warps run only the first epilogue (measured: 3-bit codes
+// 16% faster, 2-bit codes 1-2%, 1-bit codes 3% slower, so those keep one epilogue loop); the mixed
+// rate's 16 epilogue warps do both (no registers left for more warps).
+template <bool QJL, int BITS, bool MIXED>
+constexpr bool epi_split() { return QJL && !MIXED && BITS >= 2; }
 
-template <bool QJL, int NP>
+template <bool QJL, int NP, bool SPLIT>
 struct Ws {
   static constexpr int kParts = NP;                      // epilogue threads per token
   static constexpr int kEpiWarps = 4 * NP;               // NP warps per tensor-memory lane quarter
-  static constexpr int kTmaWarp = kEpiWarps;
+  static constexpr bool kSplit = SPLIT;
+  static constexpr int kSignWarps = kSplit ? 4 : 0;
+  static constexpr int kTmaWarp = kEpiWarps + kSignWarps;
   static constexpr int kMmaWarp = kTmaWarp + 1;
-  static constexpr int kThreads = 32 * (kMmaWarp + 1);   // 320 (168 registers a thread) or 576 (96)
+  static constexpr int kThreads = 32 * (kMmaWarp + 1);   // 320 (168 registers), 448 (128) or 576 (96)
   static constexpr int kNX = QJL ? 2 : 4;                // A-tile stages (tensor-map copies in flight)
   // values: Pi_hi and Pi_lo stacked as one 256-row B tile, so one N = 256 product per K step gives
   // both parts (summed by the epilogue), with two D1 buffers; keys: two N = 128 products into one D1
@@ -125,8 +136,8 @@ struct Ws {
   static constexpr uint32_t kXch = kRho + (QJL ? 3 * kParts * 128 * 4 : 0);  // float2[2][kParts][128]: ||x|| parts
   static constexpr uint32_t kCb = kXch + 2 * kParts * 128 * 8;               // float[32] centroids (two codebooks if mixed)
   static constexpr uint32_t kBar = kCb + 128;
-  // barriers: x_full[4], x_empty[4], d1_full[2], d1_empty[2], e_full, d2_full, d2_empty
-  static constexpr int kBars = 4 + 4 + 2 + 2 + 1 + 1 + 1;
+  // barriers: x_full[4], x_empty[4], d1_full[2], d1_empty[2], e_full, d2_full, d2_empty, rho_full[3]
+  static constexpr int kBars = 4 + 4 + 2 + 2 + 1 + 1 + 1 + 3;
   static constexpr uint32_t kTslot = kBar + 8 * kBars;
   static constexpr uint32_t kBytes = kTslot + 16;
   static constexpr uint32_t kTmemCols = 512;   // keys: D1, D2, E[0], E[1]; values: D1[0], D1[1] (256 each)
@@ -145,6 +156,7 @@ struct Bars {
   __device__ uint32_t e_full() const { return base + 8u * 12; }
   __device__ uint32_t d2_full() const { return base + 8u * 13; }
   __device__ uint32_t d2_empty() const { return base + 8u * 14; }
+  __device__ uint32_t rho_full(int k) const { return base + 8u * (15 + k); }   // rho of tile i in slot i % 3
 };
 
 // Position of a CTA's current tile in the (sequence x head, token) grid, kept
@@ -483,9 +495,9 @@ __device__ __forceinline__ void mma_tile(uint32_t d, uint32_t a, uint32_t b, uin
 }
 
 template <bool QJL, int BITS, bool F16, bool MIXED = false>
-__global__ void __launch_bounds__(Ws<QJL, epi_parts<MIXED>()>::kThreads, 1)
+__global__ void __launch_bounds__(Ws<QJL, epi_parts<MIXED>(), epi_split<QJL, BITS, MIXED>()>::kThreads, 1)
     quantize_tc_kernel(const QuantParams p, const __grid_constant__ CUtensorMap xmap) {
-  using L = Ws<QJL, epi_parts<MIXED>()>;
+  using L = Ws<QJL, epi_parts<MIXED>(), epi_split<QJL, BITS, MIXED>()>;
   constexpr int kParts = L::kParts;
   constexpr int kEpiWarps = L::kEpiWarps;
   constexpr int CPT = kTD / kParts;               // columns per epilogue thread
@@ -519,7 +531,8 @@ __global__ void __launch_bounds__(Ws<QJL, epi_parts<MIXED>()>::kThreads, 1)
     }
     mbar_init(bar.e_full(), kEpiWarps);
     mbar_init(bar.d2_full(), 1);
-    mbar_init(bar.d2_empty(), kEpiWarps);
+    mbar_init(bar.d2_empty(), L::kSplit ? L::kSignWarps : kEpiWarps);
+    for (int k = 0; k < 3; ++k) mbar_init(bar.rho_full(k), kEpiWarps);
     mbar_fence_init();
   }
   if (warp == 0) {
@@ -551,6 +564,52 @@ __global__ void __launch_bounds__(Ws<QJL, epi_parts<MIXED>()>::kThreads, 1)
       }
       // no copy may still be landing when the CTA exits
       for (int i = max(0, issued - L::kNX); i < issued; ++i) mbar_wait(bar.x_full(i % L::kNX), (i / L::kNX) & 1);
+    }
+  } else if (L::kSplit && warp >= kEpiWarps && warp < L::kTmaWarp) {
+    // ------------------------------- sign warps -------------------------------
+    // thread: token t = tensor-memory lane, all 128 sketch columns. Tile j: wait for the epilogue's
+    // sums of e^2 (rho_full) and the sketch product (d2_full), read both, release D2, store.
+    const int q = warp & 3, t = 32 * q + lane;
+    const uint32_t lane_ofs = (uint32_t)(32 * q) << 16;
+    const float *rho = reinterpret_cast<const float *>(smem + L::kRho);   // [3][kParts][128]
+    TileCursor cur;
+    cur.init(p);
+    for (int j = 0; j < n_my; ++j) {
+      const bool valid = row0_of(j) + t < p.rows;
+      const int64_t slot = valid ? cur.slot(p, t) : 0;
+      cur.advance(p);
+      // the tensor-memory loads are warp-wide: the whole warp loads or none of it does
+      if (!__all_sync(0xffffffffu, mbar_wait(bar.rho_full(j % 3), (j / 3) & 1) && mbar_wait(bar.d2_full(), j & 1)))
+        break;
+      tc::fence_after();
+      uint32_t sw[4];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r[64];
+        tc::ld32(tmem + lane_ofs + L::kD2 + 64 * hh, *reinterpret_cast<uint32_t (*)[32]>(r));
+        tc::ld32(tmem + lane_ofs + L::kD2 + 64 * hh + 32, *reinterpret_cast<uint32_t (*)[32]>(r + 32));
+        tc::wait_ld();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          sw[2 * hh + c] = 0u;
+#pragma unroll
+          for (int qq = 0; qq < 32; ++qq) put_bit(sw[2 * hh + c], ge0(__uint_as_float(r[32 * c + qq])), qq);
+        }
+      }
+      // rho of tile j is read before D2 is released: the epilogue cannot reuse its slot until the sketch
+      // of tile j + 1, which waits for that release, has been issued
+      float e2s = 0.f;
+#pragma unroll
+      for (int k = 0; k < L::kParts; ++k) e2s += rho[((j % 3) * L::kParts + k) * 128 + t];
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar.d2_empty());   // D2 may take the next tile's sketch
+      if (valid) {
+        uint32_t *sdst = p.records + slot * RW + IW;
+        st_global_v2(sdst, sw[0], sw[1]);
+        st_global_v2(sdst + 2, sw[2], sw[3]);
+        p.rnorm[slot] = sqrtf(e2s);
+      }
     }
   } else if (warp == L::kMmaWarp) {
     // ----------------------------- MMA issuer ------------------------------
@@ -706,7 +765,10 @@ __global__ void __launch_bounds__(Ws<QJL, epi_parts<MIXED>()>::kThreads, 1)
               tc::fence_before();
               rho[((i % 3) * kParts + h) * 128 + t] = e2;
               __syncwarp();
-              if (lane == 0) mbar_arrive(bar.e_full());
+              if (lane == 0) {
+                mbar_arrive(bar.e_full());
+                if constexpr (L::kSplit) mbar_arrive(bar.rho_full(i % 3));   // for the sign warps
+              }
             } else {
               // values need only the codes (FMA-pipe search on y = D1 / n, 0 for a zero vector)
               FmaSearch<CB> fs;
@@ -735,7 +797,7 @@ __global__ void __launch_bounds__(Ws<QJL, epi_parts<MIXED>()>::kThreads, 1)
           else codes(std::integral_constant<int, BITS>{});
         }
       }
-      if constexpr (QJL) {
+      if constexpr (QJL && !L::kSplit) {
         if (i >= 1) {
           // ---- second epilogue of tile i - 1: sign words and ||e|| ----
           const int j = i - 1;
@@ -812,7 +874,7 @@ cudaError_t launch_tc(const QuantParams &p, cudaStream_t st) {
   CUtensorMap xmap;
   if (p.rows >= (int64_t)1 << 31 || !make_x_map(&xmap, p, F16)) return cudaErrorNotSupported;
   auto kern = quantize_tc_kernel<QJL, BITS, F16, MIXED>;
-  using L = Ws<QJL, epi_parts<MIXED>()>;
+  using L = Ws<QJL, epi_parts<MIXED>(), epi_split<QJL, BITS, MIXED>()>;
   constexpr size_t smem = L::kBytes;
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
