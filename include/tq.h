@@ -142,6 +142,25 @@ tq_status tq_quantize_append(const tq_cache *cache, const void *x, tq_dtype dtyp
                              const float *Pi, const float *SPiT, const float *codebook,
                              tq_stream stream);
 
+/* tq_quantize_append with the structured rotation Pi = H diag(signs) / sqrt(d),
+ * H the d x d Sylvester-Hadamard matrix in natural order (H_ij = (-1)^popcount(i & j)):
+ * y = H (signs * x) / (sqrt(d) ||x||) by a fast Walsh-Hadamard transform, log2(d)
+ * rounds of pairwise sums and differences, O(d log d) per vector instead of the
+ * dense product's O(d^2) (winningdata.io, "1. PolarQuant", the rotation's cost per
+ * vector). Everything else, the record layout included, is tq_quantize_append's,
+ * so tq_logits / tq_attend_v / tq_decode_attend read the cache with the dense Pi of
+ * the same rotation.
+ *   signs: [d] device floats, each +1 or -1.
+ *   SPiT:  [d][d] float, S Pi^T for that Pi (tq_sketch_rotation of the dense Pi);
+ *          ignored (may be NULL) for a value cache.
+ * d must be a power of two in [32, 256] (TQ_ERR_UNSUPPORTED otherwise); x of any
+ * dtype; mixed-rate caches are accepted. Runs on the FP32 cores. Other errors as
+ * tq_quantize_append. */
+tq_status tq_quantize_append_hadamard(const tq_cache *cache, const void *x, tq_dtype dtype,
+                                      int64_t pos, int64_t n_tokens,
+                                      const float *signs, const float *SPiT, const float *codebook,
+                                      tq_stream stream);
+
 /* Workspace bytes tq_logits needs for this key cache and query-head count. */
 size_t tq_logits_workspace_size(const tq_cache *k, int32_t n_q_heads);
 

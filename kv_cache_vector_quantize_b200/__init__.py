@@ -42,6 +42,7 @@ from ._binding import (  # noqa: F401
     tq_nn_search,
     tq_nn_workspace_size,
     tq_quantize_append,
+    tq_quantize_append_hadamard,
     tq_record_words,
     tq_record_words_mixed,
     tq_sketch_rotation,

@@ -53,6 +53,7 @@ def _load() -> ctypes.CDLL:
         "tq_codebook_fit": (I32, [I32, I32, P]),
         "tq_sketch_rotation": (I32, [I32, P, P, P, P]),
         "tq_quantize_append": (I32, [D, P, I32, I64, I64, P, P, P, P]),
+        "tq_quantize_append_hadamard": (I32, [D, P, I32, I64, I64, P, P, P, P]),
         "tq_logits_workspace_size": (SZ, [D, I32]),
         "tq_logits": (I32, [D, P, I32, I64, P, P, P, P, P, SZ, P]),
         "tq_attend_workspace_size": (SZ, [D, I32, I64]),
@@ -212,6 +213,24 @@ def tq_quantize_append(cache: PackedCache, x: torch.Tensor, pos: int, Pi: torch.
     desc = cache.desc()
     _check(_lib.tq_quantize_append(ctypes.byref(desc), _ptr(x), _DTYPE[x.dtype], int(pos), int(x.shape[2]),
                                    _ptr(Pi), _ptr(SPiT), _ptr(codebook), _stream(stream)))
+
+
+def tq_quantize_append_hadamard(cache: PackedCache, x: torch.Tensor, pos: int, signs: torch.Tensor,
+                                SPiT: torch.Tensor | None, codebook: torch.Tensor, stream=None) -> None:
+    """tq_quantize_append with Pi = H diag(signs) / sqrt(d) applied by a fast Walsh-Hadamard transform;
+    signs: [d] float32 of +-1, d a power of two in [32, 256]."""
+    if x.dim() != 4 or x.shape[0] != cache.n_seq or x.shape[1] != cache.n_kv_heads or x.shape[3] != cache.d:
+        raise ValueError(f"x must be [{cache.n_seq}, {cache.n_kv_heads}, T, {cache.d}], got {tuple(x.shape)}")
+    _need(x, "x", device=cache.device)
+    if x.dtype not in _DTYPE:
+        raise ValueError(f"x dtype {x.dtype} unsupported")
+    _need(signs, "signs", torch.float32, (cache.d,), cache.device)
+    _need(codebook, "codebook", torch.float32, (cache.codebook_len,), cache.device)
+    if cache.qjl:
+        _need(SPiT, "SPiT", torch.float32, (cache.d, cache.d), cache.device)
+    desc = cache.desc()
+    _check(_lib.tq_quantize_append_hadamard(ctypes.byref(desc), _ptr(x), _DTYPE[x.dtype], int(pos), int(x.shape[2]),
+                                            _ptr(signs), _ptr(SPiT), _ptr(codebook), _stream(stream)))
 
 
 def tq_logits_workspace_size(cache: PackedCache, n_q_heads: int) -> int:

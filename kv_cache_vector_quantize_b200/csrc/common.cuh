@@ -85,6 +85,7 @@ struct QuantParams {
   int rec_words;
   int idx_words;
   int n_hi;                 // mixed rate: leading coordinates at bits + 1 code bits (0: integer rate)
+  const float *signs;       // structured rotation Pi = H diag(signs) / sqrt(d) (then Pi is unused), or NULL
 };
 
 struct LogitsParams {
@@ -146,6 +147,9 @@ struct AttendParams {
 // launchers (defined in the .cu files)
 cudaError_t launch_sketch_rotation(int d, const float *Pi, const float *S, float *SPiT, cudaStream_t st);
 cudaError_t launch_quantize(const QuantParams &p, int bits, bool qjl, tq_dtype dtype, cudaStream_t st);
+// The FP32-core quantizer with y = H (signs * x) / (sqrt(d) ||x||) by a fast Walsh-Hadamard transform
+// (d a power of two, 32..256); keys still project the residual with the dense S Pi^T.
+cudaError_t launch_quantize_hadamard(const QuantParams &p, int bits, bool qjl, tq_dtype dtype, cudaStream_t st);
 cudaError_t launch_quantize_tc(const QuantParams &p, int bits, bool qjl, bool f16, cudaStream_t st);
 cudaError_t launch_qprep(const float *q, int rows, int d, const float *Pi, const float *S,
                          float *qrot, float *qsk, uint32_t *status, cudaStream_t st);

@@ -100,12 +100,54 @@ __device__ __forceinline__ void project(const float *__restrict__ gmat, float *m
   }
 }
 
+// y = H (s * x) / sqrt(d) for the kQTpw rows of a warp (structured rotation, winningdata.io
+// "1. PolarQuant": the rotation's cost per vector; a Hadamard product is O(d log d)). H is the
+// Sylvester-Hadamard matrix in natural order, so log2(d) rounds of pairs (i, i + h), i & h = 0,
+// become (a + b, a - b). Lane l holds coordinates l + 32 m: rounds h < 32 pair lanes (one
+// shuffle), rounds h >= 32 pair registers m and m + h / 32. DP = d, a power of two.
+template <int DP>
+__device__ __forceinline__ void fwht_rows(const float *xw, const float *__restrict__ signs, int lane,
+                                          float (&acc)[kQTpw][QLayout<DP>::CPL]) {
+  using Lay = QLayout<DP>;
+  constexpr int CPL = Lay::CPL;
+  float sg[CPL];
+#pragma unroll
+  for (int m = 0; m < CPL; ++m) sg[m] = __ldg(signs + lane + 32 * m);
+  const float scale = 1.0f / sqrtf((float)DP);
+#pragma unroll
+  for (int i = 0; i < kQTpw; ++i) {
+    float v[CPL];
+#pragma unroll
+    for (int m = 0; m < CPL; ++m) v[m] = xw[i * Lay::XS + lane + 32 * m] * sg[m];
+#pragma unroll
+    for (int h = 1; h < 32 && h < DP; h <<= 1) {
+      const bool hi = (lane & h) != 0;
+#pragma unroll
+      for (int m = 0; m < CPL; ++m) {
+        const float o = __shfl_xor_sync(0xffffffffu, v[m], h);
+        v[m] = hi ? o - v[m] : v[m] + o;
+      }
+    }
+#pragma unroll
+    for (int hm = 1; hm < CPL; hm <<= 1)
+#pragma unroll
+      for (int m = 0; m < CPL; ++m)
+        if ((m & hm) == 0) {
+          const float a = v[m], b = v[m + hm];
+          v[m] = a + b;
+          v[m + hm] = a - b;
+        }
+#pragma unroll
+    for (int m = 0; m < CPL; ++m) acc[i][m] = v[m] * scale;
+  }
+}
+
 // Blocks per SM: d > 128 streams the matrices in chunks between block barriers, so two CTAs per
 // SM let one CTA's barrier waits overlap the other's products.
 template <int DP>
 constexpr int q_blocks_per_sm() { return DP > 128 ? 2 : 1; }
 
-template <int DP, bool QJL, typename Tin>
+template <int DP, bool QJL, typename Tin, bool HAD = false>
 __global__ void __launch_bounds__(kQThreads, q_blocks_per_sm<DP>()) quantize_kernel(const QuantParams p, const int bits) {
   using Lay = QLayout<DP>;
   constexpr int CPL = Lay::CPL;
@@ -128,7 +170,7 @@ __global__ void __launch_bounds__(kQThreads, q_blocks_per_sm<DP>()) quantize_ker
   if (tid < L - 1) cb[16 + tid] = 0.5f * (cb[tid] + cb[tid + 1]);
   if (tid < 15) cb[48 + tid] = tid < LH - 1 ? 0.5f * (cb[32 + tid] + cb[32 + tid + 1]) : 3.0e38f;
   if constexpr (Lay::kResident) {
-    load_matrix_chunk<DP>(matP, p.Pi, d, 0);
+    if constexpr (!HAD) load_matrix_chunk<DP>(matP, p.Pi, d, 0);
     if constexpr (QJL) load_matrix_chunk<DP>(matM, p.SPiT, d, 0);
   }
   __syncthreads();
@@ -164,7 +206,8 @@ __global__ void __launch_bounds__(kQThreads, q_blocks_per_sm<DP>()) quantize_ker
     }
     // ---- y = Pi x / n ----
     float acc[kQTpw][CPL];
-    project<DP>(p.Pi, matP, xw, d, lane, acc);
+    if constexpr (HAD) fwht_rows<DP>(xw, p.signs, lane, acc);
+    else project<DP>(p.Pi, matP, xw, d, lane, acc);
     __syncwarp();
 #pragma unroll
     for (int i = 0; i < kQTpw; ++i) {
@@ -244,9 +287,9 @@ __global__ void __launch_bounds__(kQThreads, q_blocks_per_sm<DP>()) quantize_ker
   }
 }
 
-template <int DP, bool QJL, typename Tin>
+template <int DP, bool QJL, typename Tin, bool HAD = false>
 cudaError_t launch_q(const QuantParams &p, int bits, cudaStream_t st) {
-  auto kern = quantize_kernel<DP, QJL, Tin>;
+  auto kern = quantize_kernel<DP, QJL, Tin, HAD>;
   constexpr size_t smem = quant_smem_bytes<DP, QJL>();
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
@@ -257,18 +300,18 @@ cudaError_t launch_q(const QuantParams &p, int bits, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int DP, bool QJL>
+template <int DP, bool QJL, bool HAD = false>
 cudaError_t launch_q_dtype(const QuantParams &p, int bits, tq_dtype dt, cudaStream_t st) {
   switch (dt) {
-    case TQ_BF16: return launch_q<DP, QJL, __nv_bfloat16>(p, bits, st);
-    case TQ_FP16: return launch_q<DP, QJL, __half>(p, bits, st);
-    default: return launch_q<DP, QJL, float>(p, bits, st);
+    case TQ_BF16: return launch_q<DP, QJL, __nv_bfloat16, HAD>(p, bits, st);
+    case TQ_FP16: return launch_q<DP, QJL, __half, HAD>(p, bits, st);
+    default: return launch_q<DP, QJL, float, HAD>(p, bits, st);
   }
 }
 
-template <int DP>
+template <int DP, bool HAD = false>
 cudaError_t launch_q_dp(const QuantParams &p, int bits, bool qjl, tq_dtype dt, cudaStream_t st) {
-  return qjl ? launch_q_dtype<DP, true>(p, bits, dt, st) : launch_q_dtype<DP, false>(p, bits, dt, st);
+  return qjl ? launch_q_dtype<DP, true, HAD>(p, bits, dt, st) : launch_q_dtype<DP, false, HAD>(p, bits, dt, st);
 }
 
 // SPiT[i][j] = sum_k S[i][k] Pi[j][k], accumulated in double.
@@ -296,6 +339,16 @@ cudaError_t launch_quantize(const QuantParams &p, int bits, bool qjl, tq_dtype d
   if (p.d <= 128) return launch_q_dp<128>(p, bits, qjl, dtype, st);
   if (p.d <= 224) return launch_q_dp<224>(p, bits, qjl, dtype, st);   // d = 200: 23% fewer products than 256
   return launch_q_dp<256>(p, bits, qjl, dtype, st);
+}
+
+cudaError_t launch_quantize_hadamard(const QuantParams &p, int bits, bool qjl, tq_dtype dtype, cudaStream_t st) {
+  switch (p.d) {
+    case 32: return launch_q_dp<32, true>(p, bits, qjl, dtype, st);
+    case 64: return launch_q_dp<64, true>(p, bits, qjl, dtype, st);
+    case 128: return launch_q_dp<128, true>(p, bits, qjl, dtype, st);
+    case 256: return launch_q_dp<256, true>(p, bits, qjl, dtype, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_sketch_rotation(int d, const float *Pi, const float *S, float *SPiT, cudaStream_t st) {

@@ -298,6 +298,50 @@ tq_status tq_quantize_append(const tq_cache *cache, const void *x, tq_dtype dtyp
   return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_quantize_append");
 }
 
+tq_status tq_quantize_append_hadamard(const tq_cache *cache, const void *x, tq_dtype dtype, int64_t pos,
+                                      int64_t n_tokens, const float *signs, const float *SPiT,
+                                      const float *codebook, tq_stream stream) {
+  g_err[0] = 0;
+  tq_status s = check_cache(cache, "tq_quantize_append_hadamard");
+  if (s != TQ_OK) return s;
+  const int d = cache->d;
+  if (d < 32 || d > 256 || (d & (d - 1)) != 0)
+    return fail(TQ_ERR_UNSUPPORTED, "tq_quantize_append_hadamard: d=%d is not a power of two in [32, 256]", d);
+  if (dtype != TQ_BF16 && dtype != TQ_FP16 && dtype != TQ_FP32)
+    return fail(TQ_ERR_INVALID, "tq_quantize_append_hadamard: dtype=%d", (int)dtype);
+  if (pos < 0 || n_tokens < 0)
+    return fail(TQ_ERR_INVALID, "tq_quantize_append_hadamard: pos=%lld n_tokens=%lld", (long long)pos,
+                (long long)n_tokens);
+  if (pos + n_tokens > cache->capacity)
+    return fail(TQ_ERR_CAPACITY, "tq_quantize_append_hadamard: pos %lld + n_tokens %lld > capacity %lld",
+                (long long)pos, (long long)n_tokens, (long long)cache->capacity);
+  if (n_tokens == 0) return TQ_OK;
+  const size_t esz = dtype == TQ_FP32 ? 4 : 2;
+  if (!x || !aligned(x, esz)) return fail(TQ_ERR_INVALID, "tq_quantize_append_hadamard: x NULL or misaligned");
+  if (!signs || !aligned(signs, 4) || !codebook)
+    return fail(TQ_ERR_INVALID, "tq_quantize_append_hadamard: signs or codebook NULL or misaligned");
+  if (cache->qjl && !SPiT) return fail(TQ_ERR_INVALID, "tq_quantize_append_hadamard: key cache needs SPiT");
+  if (injected(&s)) return s;
+  QuantParams p{};
+  p.x = x;
+  p.records = cache->records;
+  p.norm = cache->norm;
+  p.rnorm = cache->rnorm;
+  p.signs = signs;
+  p.SPiT = SPiT;
+  p.codebook = codebook;
+  p.rows = (int64_t)cache->n_seq * cache->n_kv_heads * n_tokens;
+  p.n_tokens = n_tokens;
+  p.capacity = cache->capacity;
+  p.pos = pos;
+  p.d = d;
+  p.rec_words = rec_words_of(d, cache->idx_bits, cache->qjl, cache->n_hi);
+  p.idx_words = idx_words_of(d, cache->idx_bits, cache->n_hi);
+  p.n_hi = cache->n_hi;
+  cudaError_t e = launch_quantize_hadamard(p, cache->idx_bits, cache->qjl != 0, dtype, (cudaStream_t)stream);
+  return e == cudaSuccess ? TQ_OK : cuda_fail(e, "tq_quantize_append_hadamard");
+}
+
 // Workspace of tq_logits: status word | Pi q | S q, and for the grouped-query
 // path a 256-byte aligned table block per unit and one scale per query head.
 namespace {

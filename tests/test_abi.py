@@ -74,6 +74,26 @@ def _q(desc, x=FAKE, pos=0, n=8, Pi=FAKE, SPiT=FAKE, cb=FAKE, dtype=0):
     return lib.tq_quantize_append(ctypes.byref(desc) if desc is not None else None, x, dtype, pos, n, Pi, SPiT, cb, None)
 
 
+def test_quantize_hadamard_argument_checks():
+    def qh(desc, x=FAKE, pos=0, n=8, signs=FAKE, SPiT=FAKE, cb=FAKE, dtype=0):
+        return lib.tq_quantize_append_hadamard(ctypes.byref(desc) if desc is not None else None, x, dtype, pos, n,
+                                               signs, SPiT, cb, None)
+    assert qh(None) == tqb.TQ_ERR_INVALID
+    for d in (8, 16, 96, 200, 512):          # not a power of two in [32, 256] (or an invalid cache)
+        assert qh(_desc(d=d)) in (tqb.TQ_ERR_UNSUPPORTED, tqb.TQ_ERR_INVALID), d
+    assert qh(_desc(d=200)) == tqb.TQ_ERR_UNSUPPORTED
+    assert qh(_desc(), dtype=7) == tqb.TQ_ERR_INVALID
+    assert qh(_desc(), pos=-1) == tqb.TQ_ERR_INVALID
+    assert qh(_desc(cap=16), pos=10, n=8) == tqb.TQ_ERR_CAPACITY
+    assert qh(_desc(), n=0) == tqb.TQ_OK                     # no-op, nothing launched
+    assert qh(_desc(), signs=None) == tqb.TQ_ERR_INVALID
+    assert qh(_desc(), cb=None) == tqb.TQ_ERR_INVALID
+    assert qh(_desc(qjl=1), SPiT=None) == tqb.TQ_ERR_INVALID
+    assert qh(_desc(qjl=0), SPiT=None) == tqb.TQ_ERR_CUDA    # values need no SPiT: checks pass, injected error
+    for d in (32, 64, 128, 256):
+        assert qh(_desc(d=d)) == tqb.TQ_ERR_CUDA            # every check passes: the injected launch error
+
+
 def test_quantize_argument_checks():
     assert _q(None) == tqb.TQ_ERR_INVALID
     assert _q(_desc(d=12)) == tqb.TQ_ERR_UNSUPPORTED

@@ -37,16 +37,21 @@ def rotation(d: int, seed: int = SEED_PI) -> torch.Tensor:
     return q.to(torch.float32).contiguous()
 
 
-def randomized_hadamard(d: int, seed: int = SEED_PI) -> torch.Tensor:
-    """Structured orthogonal d x d matrix H diag(s) / sqrt(d): H the Sylvester-Hadamard matrix
-    (H_1 = [1], H_2m = [[H_m, H_m], [H_m, -H_m]]), s seeded random signs; d a power of two.
-    Float32 on the CPU; an alternative to `rotation` for the rotation input."""
+def hadamard_signs(d: int, seed: int = SEED_PI) -> torch.Tensor:
+    """The seeded random signs s (+-1, float32, CPU) of `randomized_hadamard(d, seed)`."""
     if d < 1 or d & (d - 1):
         raise ValueError(f"d={d} is not a power of two")
+    return torch.where(torch.rand(d, generator=_gen(seed), dtype=torch.float64) < 0.5, -1.0, 1.0).to(torch.float32)
+
+
+def randomized_hadamard(d: int, seed: int = SEED_PI) -> torch.Tensor:
+    """Structured orthogonal d x d matrix H diag(s) / sqrt(d): H the Sylvester-Hadamard matrix
+    (H_1 = [1], H_2m = [[H_m, H_m], [H_m, -H_m]]), s = `hadamard_signs(d, seed)`; d a power of two.
+    Float32 on the CPU; an alternative to `rotation` for the rotation input."""
+    s = hadamard_signs(d, seed).to(torch.float64)
     h = torch.ones(1, 1, dtype=torch.float64)
     while h.shape[0] < d:
         h = torch.cat([torch.cat([h, h], 1), torch.cat([h, -h], 1)], 0)
-    s = torch.where(torch.rand(d, generator=_gen(seed), dtype=torch.float64) < 0.5, -1.0, 1.0)
     return (h * s[None, :] / d ** 0.5).to(torch.float32).contiguous()
 
 
