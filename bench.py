@@ -55,13 +55,19 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0
 # stands (profiles/), keyed by (kernel, workload); a key is removed when its
 # kernel changes, and the bench then reports traffic as null.
 NCU_TRAFFIC = {
-    ("quantize_k", "llama"): 67_326_976 + 2_125_824,   # quantize_tc_kernel<1, 2, 0>
-    ("quantize_v", "llama"): 67_240_704 + 2_118_144,   # quantize_tc_kernel<0, 3, 0>
+    ("quantize_k", "llama"): 67_329_280 + 1_720_064,   # quantize_tc_kernel<1, 2, 0, 0> (with sign warps)
+    ("quantize_v", "llama"): 67_229_696 + 2_305_536,   # quantize_tc_kernel<0, 3, 0, 0>
+    # the large-model layer's launches, too large to capture: the Llama capture scaled by the head-vectors
+    # processed (16 777 216 / 262 144 = 64; the traffic is the 256 B input and the record per head-vector)
+    ("quantize_k", "large-b3"): 64 * (67_329_280 + 1_720_064),
+    ("quantize_v", "large-b3"): 64 * (67_229_696 + 2_305_536),
     ("logits", "sweep-b3"): 2 * (234_967_296 + 16_118_528),   # logits_fast_kernel<2, 1>, 4-sequence capture x 2
-    ("attend_v", "sweep-b3"): 2 * (234_927_616 + 3_965_184),  # attend_fast_kernel<3, 1>, 4-sequence capture x 2
+    ("attend_v", "sweep-b3"): 2 * (234_913_280 + 5_718_528),  # attend_fast_kernel<3, 1, 0>, 4-sequence capture x 2
+    # the large-model layer's scan and softmax.V: the 4-sequence b-sweep captures (4 194 304 keys, one query
+    # head per KV head, the same kernels) scaled by the keys processed (x 4)
+    ("logits", "large-b3"): 4 * (234_967_296 + 16_118_528),
+    ("attend_v", "large-b3"): 4 * (234_913_280 + 5_718_528),
     ("logits", "llama"): 15_756_288 + 0,               # logits_gqa_kernel<2, 4> (the scan; tables read from L2)
-    ("attend_v", "llama"): 17_871_872 + 0,             # attend_fast_kernel<3, 4> (records, norms and logits)
-    ("decode_attend", "sweep-b3"): 2 * (453_061_376 + 5_822_720),   # decode_fused_kernel<2, 3>, 4-sequence capture x 2
 }
 
 
@@ -73,6 +79,7 @@ def parse():
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--workload", default="large-b3",
                     choices=["llama"] + [f"sweep-b{b}{s}" for b in (2, 3, 4, 2.5, 3.5) for s in ("", "-s4")]
+                    + ["sweep-b3-had"]
                     + ["large-b3", "large-b4", "nn-b2", "nn-b4", "nn-b2-s", "nn-b4-s"])
     ap.add_argument("--split", choices=["layers", "heads"], default="layers",
                     help="large-model cache on N GPUs: every rank streams its own layers (weak scaling), or "
@@ -106,6 +113,12 @@ def workload(name: str):
                          f"channels, streamed layer by layer, K b={b} V b={b}, one query head per KV head",
                     n_seq=1, hq=128, hkv=128, d=128, T=131072, k_idx=b - 1, v_idx=b, dtype=torch.float16,
                     gen=lambda dev, seed: syn.large_layer_inputs(seed, device=dev))
+    # "sweep-b3-had": the b-sweep at b = 3 with the structured rotation Pi = H diag(s) / sqrt(d), the
+    # quantizer applying it by the fast Walsh-Hadamard transform (tq_quantize_append_hadamard)
+    if name == "sweep-b3-had":
+        w = workload("sweep-b3")
+        w.update(name=w["name"] + "; rotation H diag(s)/sqrt(d) by the fast Walsh-Hadamard transform", hadamard=True)
+        return w
     # "sweep-b3" is the full b-sweep cache; "sweep-b3-s4" keeps 4 of its 8 sequences
     # (a profiling size: still larger than L2, half the device memory). "sweep-b3.5" and
     # "sweep-b2.5": fractional bits per channel, half of the rotated coordinates at one more
@@ -250,7 +263,9 @@ def run_tq(args, rank, world, local_rank):
     w = workload(args.workload)
     d = w["d"]
     k, v, q = w["gen"](dev, rank_seed(rank))
-    Pi = syn.rotation(d).to(dev)
+    had = w.get("hadamard", False)
+    Pi = (syn.randomized_hadamard(d) if had else syn.rotation(d)).to(dev)
+    signs = syn.hadamard_signs(d).to(dev) if had else None
     S = syn.sketch(d).to(dev)
     ck = fit_codebooks(tqb, d, w["k_idx"], w.get("k_nhi", 0)).to(dev)
     cv = fit_codebooks(tqb, d, w["v_idx"], w.get("v_nhi", 0)).to(dev)
@@ -267,13 +282,19 @@ def run_tq(args, rank, world, local_rank):
     scale = 1.0 / math.sqrt(d)
     stream = torch.cuda.current_stream(dev)
 
+    def quantize(cache, x, spit, cb):
+        if had:
+            tqb.tq_quantize_append_hadamard(cache, x, 0, signs, spit, cb)
+        else:
+            tqb.tq_quantize_append(cache, x, 0, Pi, spit, cb)
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        tqb.tq_quantize_append(kc, k, 0, Pi, SPiT, ck)
+        quantize(kc, k, SPiT, ck)
         if ev is not None:
             ev[1].record(stream)
-        tqb.tq_quantize_append(vc, v, 0, Pi, None, cv)
+        quantize(vc, v, None, cv)
         if ev is not None:
             ev[2].record(stream)
         flush.fill_(1.0)
@@ -331,6 +352,69 @@ def run_tq(args, rank, world, local_rank):
     value = world * scan_gbs_rank
     head_vectors = w["n_seq"] * w["hkv"] * w["T"]
     quant_tps = world * w["n_seq"] * w["T"] / (quant_ms * 1e-3)
+
+    # ---- structured rotation: the dense-Pi quantizers on the same rotation and inputs, for comparison ----
+    dense = None
+    if had:
+        dk = tqb.PackedCache.empty(d, w["k_idx"], True, w["n_seq"], w["hkv"], w["T"], device=dev)
+        dv = tqb.PackedCache.empty(d, w["v_idx"], False, w["n_seq"], w["hkv"], w["T"], device=dev)
+        kf, vf = k.float(), v.float()   # fp32 inputs take the FP32-core kernel on both rotations
+        calls = {
+            "tensor_core_dense_bf16": (lambda: tqb.tq_quantize_append(dk, k, 0, Pi, SPiT, ck),
+                                       lambda: tqb.tq_quantize_append(dv, v, 0, Pi, None, cv)),
+            "fp32_cores_dense_fp32": (lambda: tqb.tq_quantize_append(dk, kf, 0, Pi, SPiT, ck),
+                                      lambda: tqb.tq_quantize_append(dv, vf, 0, Pi, None, cv)),
+            "fp32_cores_hadamard_fp32": (lambda: tqb.tq_quantize_append_hadamard(dk, kf, 0, signs, SPiT, ck),
+                                         lambda: tqb.tq_quantize_append_hadamard(dv, vf, 0, signs, None, cv)),
+        }
+        dense = {"note": "ms per call on the same rotation and inputs: the dense Pi on the tensor cores (bf16 "
+                         "inputs, the step's default), and on the FP32 cores with fp32 inputs against the fast "
+                         "Walsh-Hadamard transform on the FP32 cores (per_kernel_ms: the transform on bf16 inputs)"}
+        for label, (fk, fv) in calls.items():
+            tk = tv = 0.0
+            for rep_ in range(2 + args.steps):
+                for which, fn in (("k", fk), ("v", fv)):
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    fn()
+                    b.record(stream)
+                    torch.cuda.synchronize(dev)
+                    if rep_ >= 2:
+                        if which == "k":
+                            tk += a.elapsed_time(b) / args.steps
+                        else:
+                            tv += a.elapsed_time(b) / args.steps
+            dense[label] = {"quantize_k_ms": round(tk, 5), "quantize_v_ms": round(tv, 5)}
+        del dk, dv, kf, vf
+        # d = 256 (fp32, 1 x 8 heads x 131072 tokens): where the transform's d log d against d^2 matters more
+        d2 = 256
+        x2 = syn.gaussian((1, 8, w["T"], d2), 91, device=dev)
+        Pi2, s2 = syn.randomized_hadamard(d2).to(dev), syn.hadamard_signs(d2).to(dev)
+        SPiT2 = tqb.tq_sketch_rotation(Pi2, syn.sketch(d2).to(dev))
+        ck2, cv2 = tqb.tq_codebook_fit(d2, w["k_idx"]).to(dev), tqb.tq_codebook_fit(d2, w["v_idx"]).to(dev)
+        dk2 = tqb.PackedCache.empty(d2, w["k_idx"], True, 1, 8, w["T"], device=dev)
+        dv2 = tqb.PackedCache.empty(d2, w["v_idx"], False, 1, 8, w["T"], device=dev)
+        for label, fk, fv in (("d256_fp32_cores_dense_fp32", lambda: tqb.tq_quantize_append(dk2, x2, 0, Pi2, SPiT2, ck2),
+                               lambda: tqb.tq_quantize_append(dv2, x2, 0, Pi2, None, cv2)),
+                              ("d256_fp32_cores_hadamard_fp32",
+                               lambda: tqb.tq_quantize_append_hadamard(dk2, x2, 0, s2, SPiT2, ck2),
+                               lambda: tqb.tq_quantize_append_hadamard(dv2, x2, 0, s2, None, cv2))):
+            tk = tv = 0.0
+            for rep_ in range(2 + args.steps):
+                for which, fn in (("k", fk), ("v", fv)):
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    fn()
+                    b.record(stream)
+                    torch.cuda.synchronize(dev)
+                    if rep_ >= 2:
+                        if which == "k":
+                            tk += a.elapsed_time(b) / args.steps
+                        else:
+                            tv += a.elapsed_time(b) / args.steps
+            dense[label] = {"quantize_k_ms": round(tk, 5), "quantize_v_ms": round(tv, 5),
+                            "head_vectors": 8 * w["T"]}
+        del x2, dk2, dv2
 
     # ---- the one-call decode step (tq_decode_attend) on the same caches, L2 flushed before each ----
     ws_d = torch.empty(max(256, tqb.tq_decode_workspace_size(kc, vc, w["hq"], w["T"])), dtype=torch.uint8, device=dev)
@@ -437,6 +521,7 @@ def run_tq(args, rank, world, local_rank):
         "quantize_tokens_per_s": round(quant_tps, 1),
         "quantize_head_vectors_per_s": round(world * head_vectors / (quant_ms * 1e-3), 1),
         "per_kernel_ms": {kk: round(vv, 5) for kk, vv in mean.items()},
+        **({"dense_rotation_quantize": dense} if dense is not None else {}),
         "packed_bytes": {"keys": kb, "values": vb},
         "roofline": roofline, "roofline_logit_scan": roof_scan, "roofline_quantize_v": roof_qv,
         "roofline_attend_v": roof_att,
@@ -919,7 +1004,7 @@ def oracle_state(w):
     d = w["d"]
     T = w["T"]
     G = w["hq"] // w["hkv"]
-    Pi = syn.rotation(d).double().numpy()
+    Pi = (syn.randomized_hadamard(d) if w.get("hadamard") else syn.rotation(d)).double().numpy()
     S = syn.sketch(d).double().numpy()
     from oracle import mixed_rate as omr
 

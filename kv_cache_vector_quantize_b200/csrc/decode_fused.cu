@@ -25,10 +25,15 @@
 // warp accumulates the values of the same 32 tokens (a half-warp per token,
 // 8 coordinates per lane), so no logit or weight crosses warps. The 16 warps'
 // (m, l, acc) merge once at the end. Every wait is bounded and reports a
-// timeout through the workspace status word.
+// timeout through the workspace status word. Value codes of 1-3 bits are read
+// two coordinates at a time from a table of centroid pairs stored once per
+// lane of a 16-lane phase and accumulated with packed two-lane FMAs
+// (fma.rn.f32x2), as the softmax.V kernel does, so the sums are bit-equal to
+// its; 4-bit codes (a 32 KB pair table would cost a value stage) take one
+// centroid and one FMA per coordinate, the same operations.
 //
 // Shared memory: barriers | key stages (below the 64 KB-aligned table base) |
-// staged Pi q, S q | tables (64 KB) | value stages | token weights.
+// staged Pi q, S q | tables (64 KB) | value stages | token weights | pair table.
 #include "scan_core.cuh"
 
 namespace tq {
@@ -50,6 +55,9 @@ template <int BETA, int VBITS>
 struct DLayout {
   static constexpr int KRW = scan::FastKeys<BETA>::RW;         // key record words
   static constexpr int VRW = VBITS * kFD / 32;                  // value record words
+  // centroid pairs (c[k & (2^VBITS - 1)], c[k >> VBITS]) at entry 16 k + lane copy, 1-3-bit codes
+  static constexpr int kPairs = VBITS <= 3 ? (1 << (2 * VBITS)) * 16 : 0;
+  static constexpr uint32_t kPairBytes = kPairs * 8;
   static constexpr uint32_t kKStage = kDTile * (KRW + 2) * 4;   // records, norm, rnorm
   static constexpr uint32_t kVStage = kDTile * (VRW + 1) * 4;   // records, norm
   static constexpr uint32_t kMerge = kDWarps * kFD * 4;         // warp accumulators at the end
@@ -75,7 +83,7 @@ struct DecodeParams {
 // Shared-memory plan of a launch with dynamic memory starting at dyn0.
 template <int BETA, int VBITS>
 struct DPlan {
-  uint32_t T0, ka, vb, nk, nv, wscr, end;
+  uint32_t T0, ka, vb, nk, nv, wscr, ptab, end;
   __host__ __device__ DPlan(uint32_t dyn0, uint32_t limit) {
     using L = DLayout<BETA, VBITS>;
     T0 = (dyn0 + kDBarBytes + kTabStride - 1) & ~(kTabStride - 1);
@@ -85,13 +93,15 @@ struct DPlan {
     if (nk > (uint32_t)kDMaxStages) nk = kDMaxStages;
     vb = T0 + kTabStride;
     const uint32_t dyn_end = dyn0 + limit;
-    const uint32_t above = dyn_end > vb + kDScratch ? dyn_end - vb - kDScratch : 0;
+    const uint32_t tail = kDScratch + L::kPairBytes;
+    const uint32_t above = dyn_end > vb + tail ? dyn_end - vb - tail : 0;
     nv = above / L::kVStage;
     if (nv > (uint32_t)kDMaxStages) nv = kDMaxStages;
     uint32_t vend = vb + nv * L::kVStage;
     if (vend < vb + L::kMerge) vend = vb + L::kMerge;   // the merge reuses the value stages
     wscr = vend;
-    end = wscr + kDScratch;
+    ptab = wscr + kDScratch;
+    end = ptab + L::kPairBytes;
   }
 };
 
@@ -222,11 +232,20 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(const Decode
     qv[e] = e < kFD ? p.qrot[(size_t)sk * kFD + e] : p.qsk[(size_t)sk * kFD + e - kFD];
   asm volatile("bar.sync 1, %0;" ::"n"(32 * kDWarps) : "memory");
   scan::build_tables<BETA, 32 * kDWarps>(qv, qv + kFD, tables, cbk, tid, kappa);
+  uint64_t *ptab = reinterpret_cast<uint64_t *>(smem + (plan.ptab - dyn0));
+  for (int e2 = tid; e2 < L::kPairs; e2 += 32 * kDWarps) {
+    const int key = e2 >> 4;
+    ptab[e2] = f2_pack(cbv[key & (LV - 1)], cbv[key >> VBITS]);
+  }
   asm volatile("bar.sync 1, %0;" ::"n"(32 * kDWarps) : "memory");
 
   float m = -INFINITY, lsum = 0.f, acc[CPL];   // running max (warp-uniform), this lane's share of l
+  uint64_t acc2[CPL / 2];                       // coordinate pairs (2 pp, 2 pp + 1), the 1-3-bit codes
 #pragma unroll
   for (int a = 0; a < CPL; ++a) acc[a] = 0.f;
+#pragma unroll
+  for (int pp = 0; pp < CPL / 2; ++pp) acc2[pp] = 0ull;   // (+0, +0)
+  const uint32_t lane8 = 8u * (uint32_t)(lane & 15);     // this lane's copy of the pair table
   float *wscr = reinterpret_cast<float *>(smem + (plan.wscr - dyn0));   // [kDWarps][32]
   const int half = lane >> 4, sub = lane & 15;
   const int bit0 = FB * sub, wd = bit0 >> 5, sh = bit0 & 31;
@@ -286,8 +305,14 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(const Decode
     const float e = mx == -INFINITY ? 0.f : expf(z - mx);
     m = mx;
     lsum = fmaf(lsum, f, e);
+    if constexpr (L::kPairs > 0) {
+      const uint64_t f2 = f2_pack(f, f);
 #pragma unroll
-    for (int a = 0; a < CPL; ++a) acc[a] *= f;
+      for (int pp = 0; pp < CPL / 2; ++pp) acc2[pp] = f2_mul(acc2[pp], f2);
+    } else {
+#pragma unroll
+      for (int a = 0; a < CPL; ++a) acc[a] *= f;
+    }
     // ---- values of the warp's 32 tokens ----
     if (!mbar_wait(vfull(sv), vph)) {
       atomicOr(p.status, kDevTimeout);
@@ -308,8 +333,21 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(const Decode
       const uint32_t hi = two ? rec[wd + 1] : 0u;
       const uint32_t bits = __funnelshift_r(lo, hi, sh);
       const float wt = wscr[tw + 2 * j + half];
+      if constexpr (L::kPairs > 0) {
+        const uint64_t w2 = f2_pack(wt, wt);
 #pragma unroll
-      for (int a = 0; a < CPL; ++a) acc[a] = fmaf(wt, cbv[(bits >> (VBITS * a)) & (LV - 1)], acc[a]);
+        for (int pp = 0; pp < CPL / 2; ++pp) {
+          // byte offset of the pair (codes 2 pp, 2 pp + 1) in the table: key * 128 (+ the lane copy)
+          constexpr uint32_t kMask = 128u * (LV * LV - 1);
+          const int shr = 2 * VBITS * pp - 7;
+          const uint32_t off = ((shr >= 0 ? bits >> (shr & 31) : bits << ((-shr) & 31)) & kMask) | lane8;
+          const uint64_t cv = *reinterpret_cast<const uint64_t *>(reinterpret_cast<const unsigned char *>(ptab) + off);
+          acc2[pp] = f2_fma(w2, cv, acc2[pp]);
+        }
+      } else {
+#pragma unroll
+        for (int a = 0; a < CPL; ++a) acc[a] = fmaf(wt, cbv[(bits >> (VBITS * a)) & (LV - 1)], acc[a]);
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(vempty(sv));   // this warp is done with the value stage and its weights
@@ -317,6 +355,10 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(const Decode
       sv = 0;
       vph ^= 1u;
     }
+  }
+  if constexpr (L::kPairs > 0) {
+#pragma unroll
+    for (int pp = 0; pp < CPL / 2; ++pp) f2_unpack(acc2[pp], acc[2 * pp], acc[2 * pp + 1]);
   }
   // the two half-warps accumulated different tokens of the same coordinates
 #pragma unroll
