@@ -68,6 +68,8 @@ NCU_TRAFFIC = {
     ("logits", "large-b3"): 4 * (234_967_296 + 16_118_528),
     ("attend_v", "large-b3"): 4 * (234_913_280 + 5_718_528),
     ("logits", "llama"): 15_756_288 + 0,               # logits_gqa_kernel<2, 4> (the scan; tables read from L2)
+    ("decode_attend", "sweep-b3"): 2 * (453_062_656 + 5_392_640),   # decode_fused_kernel<2, 3>, 4-sequence capture x 2
+    ("decode_attend", "large-b3"): 4 * (453_062_656 + 5_392_640),   # the same capture scaled by the tokens (x 4)
 }
 
 
