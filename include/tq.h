@@ -303,6 +303,17 @@ const char *tq_last_error(void);
  * work return `status` instead, before any launch. count = 0 disarms. */
 void tq_debug_inject(tq_status status, int32_t count);
 
+/* Failure detection test hook: with tries > 0, the d = 128 softmax.V kernel of
+ * the following tq_attend_v / tq_attend_v_partial / tq_decode_attend (two-call
+ * path) calls has its consumer warps wait on an mbarrier that nothing completes,
+ * for `tries` attempts, so that the wait runs out. The kernel then records a
+ * timeout in the call's status word (tq_workspace_status returns TQ_ERR_DEVICE),
+ * its copy thread gives up on the stages the consumers never release after as
+ * many tries, every copy in flight still lands before the CTA exits, and the
+ * context stays usable; the output is undefined. tries = 0 (the default)
+ * restores normal operation. Not thread-safe against concurrent calls. */
+void tq_debug_stall_consumers(uint32_t tries);
+
 /* Size of the library's built-in scratch array used by tq_attend_v_noalloc:
  * 4 MiB of device memory, held on every GPU that loads this library until the
  * process exits. */

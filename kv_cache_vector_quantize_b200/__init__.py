@@ -33,6 +33,7 @@ from ._binding import (  # noqa: F401
     tq_attend_workspace_size,
     tq_codebook_fit,
     tq_debug_inject,
+    tq_debug_stall_consumers,
     tq_decode_attend,
     tq_decode_workspace_size,
     tq_last_error,

@@ -70,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "tq_workspace_status": (I32, [P, P]),
         "tq_last_error": (ctypes.c_char_p, []),
         "tq_debug_inject": (None, [I32, I32]),
+        "tq_debug_stall_consumers": (None, [ctypes.c_uint32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -421,6 +422,11 @@ def tq_last_error() -> str:
 
 def tq_debug_inject(status: int, count: int) -> None:
     _lib.tq_debug_inject(int(status), int(count))
+
+
+def tq_debug_stall_consumers(tries: int) -> None:
+    """Test hook: softmax.V consumers wait `tries` times on a barrier nothing completes (0 disarms)."""
+    _lib.tq_debug_stall_consumers(int(tries))
 
 
 def raw_lib() -> ctypes.CDLL:

@@ -142,7 +142,14 @@ struct AttendParams {
   int q_per_cta;
   int qblocks;
   int n_hi;                 // mixed rate: leading coordinates at bits + 1 code bits (0: integer rate)
+  // failure-detection test hook (tq_debug_stall_consumers): > 0 makes the d = 128 softmax.V kernel's
+  // consumers wait on a barrier that nothing completes, for this many tries, and its copy thread give up
+  // on the stages they never release after as many; 0 in normal use
+  uint32_t stall_tries;
 };
+
+// Tries of the stalled consumer wait the next tq_attend_v call's kernel is launched with (0: none).
+uint32_t debug_stall_tries();
 
 // launchers (defined in the .cu files)
 cudaError_t launch_sketch_rotation(int d, const float *Pi, const float *S, float *SPiT, cudaStream_t st);
@@ -305,9 +312,9 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
-// Waits for the phase with the given parity to complete; false after kSpinLimit tries.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  for (uint32_t it = 0; it < kSpinLimit; ++it) {
+// Waits for the phase with the given parity to complete; false after `limit` tries.
+__device__ __forceinline__ bool mbar_wait_n(uint32_t bar, uint32_t parity, uint32_t limit) {
+  for (uint32_t it = 0; it < limit; ++it) {
     uint32_t done;
     asm volatile(
         "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
@@ -318,6 +325,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   }
   return false;
 }
+
+// Waits for the phase with the given parity to complete; false after kSpinLimit tries.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) { return mbar_wait_n(bar, parity, kSpinLimit); }
 
 // 1-D bulk copy global -> shared, completion counted on `bar` (bytes % 16 == 0,
 // both addresses 16-byte aligned).

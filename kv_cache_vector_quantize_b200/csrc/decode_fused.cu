@@ -326,8 +326,8 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(const Decode
     __syncwarp();
     const uint32_t *rs = reinterpret_cast<const uint32_t *>(vst) + (size_t)(tw + half) * VRW;
     const int np = (min(32, n - tw) + 1) >> 1;   // token pairs of this warp (warp-uniform, may be <= 0)
-#pragma unroll 2
-    for (int j = 0; j < np; ++j) {
+    // token pair j of this warp: two tokens, one per half-warp
+    auto pair_step = [&](int j) {
       const uint32_t *rec = rs + 2 * j * VRW;
       const uint32_t lo = rec[wd];
       const uint32_t hi = two ? rec[wd + 1] : 0u;
@@ -348,6 +348,14 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_fused_kernel(const Decode
 #pragma unroll
         for (int a = 0; a < CPL; ++a) acc[a] = fmaf(wt, cbv[(bits >> (VBITS * a)) & (LV - 1)], acc[a]);
       }
+    };
+    if (np == 16) {
+      // a whole warp's 32 tokens: fully unrolled (immediate addresses, no loop counter)
+#pragma unroll
+      for (int j = 0; j < 16; ++j) pair_step(j);
+    } else {
+#pragma unroll 2
+      for (int j = 0; j < np; ++j) pair_step(j);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(vempty(sv));   // this warp is done with the value stage and its weights

@@ -16,6 +16,7 @@ namespace {
 thread_local char g_err[512] = "";
 std::atomic<int> g_inject_count{0};
 std::atomic<int> g_inject_status{0};
+std::atomic<uint32_t> g_stall_tries{0};   // tq_debug_stall_consumers
 
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices] = {0};
@@ -137,6 +138,8 @@ constexpr int64_t kAttendChunk = 512;
 constexpr int kAttendMaxQ = 4;
 
 }  // namespace
+
+uint32_t debug_stall_tries() { return g_stall_tries.load(); }
 
 int device_sm_count() {
   const int dev = current_device();
@@ -504,6 +507,7 @@ tq_status attend_impl(const tq_cache *v, const float *logits, float scale, int32
   p.d = v->d;
   p.rec_words = rec_words_of(v->d, v->idx_bits, 0, v->n_hi);
   p.n_hi = v->n_hi;
+  p.stall_tries = debug_stall_tries();
   p.n_kv_heads = v->n_kv_heads;
   p.n_q_heads = n_q_heads;
   p.group = group;
@@ -889,5 +893,7 @@ void tq_debug_inject(tq_status status, int32_t count) {
   g_inject_status.store((int)status);
   g_inject_count.store(count > 0 ? count : 0);
 }
+
+void tq_debug_stall_consumers(uint32_t tries) { g_stall_tries.store(tries); }
 
 }  // extern "C"
