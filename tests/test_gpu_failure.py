@@ -44,8 +44,9 @@ def test_consumer_wait_runs_out_and_is_reported():
     tqb.tq_quantize_append(vc, v, 0, Pig, None, cvg)
     lg = 3.0 * syn.gaussian((1, H, T), 96, device=dev)
     sc = 1.0 / math.sqrt(d)
-    ws = torch.empty(max(256, tqb.tq_attend_workspace_size(vc, H, T)), dtype=torch.uint8, device=dev)
-    tqb.tq_workspace_status(ws)                       # clean before
+    ws = torch.zeros(max(256, tqb.tq_attend_workspace_size(vc, H, T)), dtype=torch.uint8, device=dev)
+    tqb.tq_attend_v(vc, lg, sc, T, Pig, cvg, workspace=ws)
+    tqb.tq_workspace_status(ws)                       # a normal call: clean
     tqb.tq_debug_stall_consumers(64)
     try:
         tqb.tq_attend_v(vc, lg, sc, T, Pig, cvg, workspace=ws)
