@@ -124,10 +124,12 @@ struct Ws {
   static constexpr int kMmaWarp = kTmaWarp + 1;
   static constexpr int kThreads = 32 * (kMmaWarp + 1);   // 320 (168 registers), 448 (128) or 576 (96)
   static constexpr int kNX = QJL ? 2 : 4;                // A-tile stages (tensor-map copies in flight)
-  // values: Pi_hi and Pi_lo stacked as one 256-row B tile, so one N = 256 product per K step gives
-  // both parts (summed by the epilogue), with two D1 buffers; keys: two N = 128 products into one D1
+  // values at the integer rates: Pi_hi and Pi_lo stacked as one 256-row B tile, so one N = 256 product
+  // per K step gives both parts (summed by the epilogue), with two D1 buffers; keys, and the mixed
+  // rate's values (NP = 4, whose 16 epilogue warps then skip that sum: 21% faster there, 5-20% slower
+  // for the integer rates): two N = 128 products accumulated into one D1 (two buffers for values)
   static constexpr int kND1 = QJL ? 1 : 2;
-  static constexpr int kPW = QJL ? 128 : 256;
+  static constexpr int kPW = (QJL || NP == 4) ? 128 : 256;
   // dynamic shared memory, byte offsets
   static constexpr uint32_t kPhi = 0, kPlo = kTile;
   static constexpr uint32_t kMhi = 2 * kTile, kMlo = 3 * kTile;              // keys only
@@ -140,7 +142,7 @@ struct Ws {
   static constexpr int kBars = 4 + 4 + 2 + 2 + 1 + 1 + 1 + 3;
   static constexpr uint32_t kTslot = kBar + 8 * kBars;
   static constexpr uint32_t kBytes = kTslot + 16;
-  static constexpr uint32_t kTmemCols = 512;   // keys: D1, D2, E[0], E[1]; values: D1[0], D1[1] (256 each)
+  static constexpr uint32_t kTmemCols = 512;   // keys: D1, D2, E[0], E[1]; values: D1[0], D1[1] (kPW each)
   static constexpr uint32_t kD2 = 128, kE = 256;   // tensor-memory column offsets (keys)
   static_assert(kBytes <= 232448, "shared memory over the per-CTA limit");
 };
@@ -517,7 +519,7 @@ __global__ void __launch_bounds__(Ws<QJL, epi_parts<MIXED>(), epi_split<QJL, BIT
   auto row0_of = [&](int i) -> int64_t { return ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * kTT; };
 
   // ---- set-up: split matrices, codebook, barriers, tensor memory ----
-  load_split<L::kThreads, F16, !QJL>(smem + L::kPhi, smem + L::kPlo, p.Pi);
+  load_split<L::kThreads, F16, L::kPW == 256>(smem + L::kPhi, smem + L::kPlo, p.Pi);
   if constexpr (QJL) load_split<L::kThreads, F16>(smem + L::kMhi, smem + L::kMlo, p.SPiT);
   if (tid < NL + (MIXED ? NLM : 0)) cb[tid] = p.codebook[tid];
   if (tid == 0) {
@@ -642,8 +644,8 @@ __global__ void __launch_bounds__(Ws<QJL, epi_parts<MIXED>(), epi_split<QJL, BIT
         if constexpr (L::kPW == 256) {
           mma_tile(tmem + 256 * db, xa, sbase + L::kPhi, idesc_w, false, 2 * kTT);
         } else {
-          mma_tile(tmem, xa, sbase + L::kPhi, idesc, false);
-          mma_tile(tmem, xa, sbase + L::kPlo, idesc, true);
+          mma_tile(tmem + 128 * db, xa, sbase + L::kPhi, idesc, false);
+          mma_tile(tmem + 128 * db, xa, sbase + L::kPlo, idesc, true);
         }
         tc::commit(bar.x_empty(xs));
         tc::commit(bar.d1_full(db));
@@ -700,7 +702,7 @@ __global__ void __launch_bounds__(Ws<QJL, epi_parts<MIXED>(), epi_split<QJL, BIT
         const bool have = __all_sync(0xffffffffu, ok && mbar_wait(bar.d1_full(db), (i / L::kND1) & 1));
         if (have) {
           tc::fence_after();
-          const uint32_t d1 = tmem + lane_ofs + 256 * db + CPT * h;
+          const uint32_t d1 = tmem + lane_ofs + (L::kPW == 256 ? 256 : 128) * db + CPT * h;
 #pragma unroll
           for (int c = 0; c < CPT / 32; ++c) tc::ld32(d1 + 32 * c, *reinterpret_cast<uint32_t (*)[32]>(r + 32 * c));
           tc::wait_ld();
