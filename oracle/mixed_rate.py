@@ -8,8 +8,8 @@ per channel with no measurable quality loss, and 2.5 bits per channel loses a
 little. The pages do not say how a fractional number of bits per channel is
 reached with a per-coordinate scalar quantizer.
 
-Reading taken here (the plainest one the rest of the pages supports, and the one
-listed in DESIGN.md): "b bits per channel" is the average over the d coordinates
+Reading taken here (the plainest one the rest of the pages supports): "b bits per
+channel" is the average over the d coordinates
 of the bits stored per coordinate. After the random rotation every coordinate of
 y = Pi u has the same law f_d, so which coordinates get the extra bit does not
 matter for the error; the first m rotated coordinates get beta + 1 code bits and

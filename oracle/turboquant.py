@@ -23,7 +23,7 @@ L = 2**bits centroids c (ascending), thresholds t_j = (c_j + c_{j+1})/2,
 idx_i = #{j : y_i > t_j}, yhat_i = c[idx_i], r = u - Pi^T yhat, rho = ||r||,
 s = S r, sign bit_i = [s_i >= 0].
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
   * keys carry bits-1 index bits + 1 sign bit per coordinate; values carry
     `bits` index bits and no sketch (MSE only).
   * keys store both n and rho; values store n only.
