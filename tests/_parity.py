@@ -1,6 +1,6 @@
 """Comparison of the CUDA path's packed cache, logits and outputs with the oracle.
 
-Tolerances (stated by the task for this method):
+Tolerances (the method's parity bounds):
   * codes and sign bits bit-exact, except a code that moved exactly one cell across
     the threshold t_j between its two cells while the rotated value lies within 1e-5
     of that threshold (|y_i - t_j| <= 1e-5 with ||u|| = 1 and ||Pi_i|| = 1), or a sign

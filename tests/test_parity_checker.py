@@ -4,8 +4,8 @@ reject planted mistakes.
 Records that stand in for the GPU's output are built by the oracle on the CPU and then
 altered by hand: a code moved one cell across the threshold it lies next to (excused), a
 code moved two cells, a code moved one cell across the other threshold of its cell, a
-stray padding bit, a sign flipped far from zero. Tolerances follow the benchmark spec
-for this method: codes bit-exact except within 1e-5 of a threshold, norms to 1e-5.
+stray padding bit, a sign flipped far from zero. The tolerances are the method's parity
+bounds: codes bit-exact except within 1e-5 of a threshold, norms to 1e-5.
 """
 
 import numpy as np
