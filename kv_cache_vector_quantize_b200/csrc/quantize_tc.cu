@@ -103,10 +103,11 @@ struct H16 {
   }
 };
 
-// Epilogue threads per token (NP parts of kTD / NP columns): 2 for the integer rates, 4 for the
-// mixed rate, whose wider half has more code-search work per column (measured best for each).
-template <bool MIXED>
-constexpr int epi_parts() { return MIXED ? 4 : 2; }
+// Epilogue threads per token (NP parts of kTD / NP columns): 4 for the mixed rate and for values with
+// 4-bit codes, whose code search is longest (values at b = 4: 10% faster), 2 otherwise (4 measured up to
+// 26% slower for 2-bit value codes and for keys).
+template <bool QJL, int BITS, bool MIXED>
+constexpr int epi_parts() { return (MIXED || (!QJL && BITS >= 4)) ? 4 : 2; }
 // Keys with 2- and 3-bit codes: 4 sign warps (one per lane quarter, a whole token per thread) turn D2
 // into sign words and rho, so the epilogue warps run only the first epilogue (measured: 3-bit codes
 // 16% faster, 2-bit codes 1-2%, 1-bit codes 3% slower, so those keep one epilogue loop); the mixed
@@ -124,10 +125,11 @@ struct Ws {
   static constexpr int kMmaWarp = kTmaWarp + 1;
   static constexpr int kThreads = 32 * (kMmaWarp + 1);   // 320 (168 registers), 448 (128) or 576 (96)
   static constexpr int kNX = QJL ? 2 : 4;                // A-tile stages (tensor-map copies in flight)
-  // values at the integer rates: Pi_hi and Pi_lo stacked as one 256-row B tile, so one N = 256 product
-  // per K step gives both parts (summed by the epilogue), with two D1 buffers; keys, and the mixed
-  // rate's values (NP = 4, whose 16 epilogue warps then skip that sum: 21% faster there, 5-20% slower
-  // for the integer rates): two N = 128 products accumulated into one D1 (two buffers for values)
+  // values with two threads per token: Pi_hi and Pi_lo stacked as one 256-row B tile, so one N = 256
+  // product per K step gives both parts (summed by the epilogue), with two D1 buffers; keys, and values
+  // with four threads per token (NP = 4: the mixed rate, 4-bit codes; their 16 epilogue warps then skip
+  // that sum, 21% faster at 3.5 bits, slower for 2-bit codes): two N = 128 products accumulated into one
+  // D1 (two buffers for values)
   static constexpr int kND1 = QJL ? 1 : 2;
   static constexpr int kPW = (QJL || NP == 4) ? 128 : 256;
   // dynamic shared memory, byte offsets
@@ -497,9 +499,9 @@ __device__ __forceinline__ void mma_tile(uint32_t d, uint32_t a, uint32_t b, uin
 }
 
 template <bool QJL, int BITS, bool F16, bool MIXED = false>
-__global__ void __launch_bounds__(Ws<QJL, epi_parts<MIXED>(), epi_split<QJL, BITS, MIXED>()>::kThreads, 1)
+__global__ void __launch_bounds__(Ws<QJL, epi_parts<QJL, BITS, MIXED>(), epi_split<QJL, BITS, MIXED>()>::kThreads, 1)
     quantize_tc_kernel(const QuantParams p, const __grid_constant__ CUtensorMap xmap) {
-  using L = Ws<QJL, epi_parts<MIXED>(), epi_split<QJL, BITS, MIXED>()>;
+  using L = Ws<QJL, epi_parts<QJL, BITS, MIXED>(), epi_split<QJL, BITS, MIXED>()>;
   constexpr int kParts = L::kParts;
   constexpr int kEpiWarps = L::kEpiWarps;
   constexpr int CPT = kTD / kParts;               // columns per epilogue thread
@@ -876,7 +878,7 @@ cudaError_t launch_tc(const QuantParams &p, cudaStream_t st) {
   CUtensorMap xmap;
   if (p.rows >= (int64_t)1 << 31 || !make_x_map(&xmap, p, F16)) return cudaErrorNotSupported;
   auto kern = quantize_tc_kernel<QJL, BITS, F16, MIXED>;
-  using L = Ws<QJL, epi_parts<MIXED>(), epi_split<QJL, BITS, MIXED>()>;
+  using L = Ws<QJL, epi_parts<QJL, BITS, MIXED>(), epi_split<QJL, BITS, MIXED>()>;
   constexpr size_t smem = L::kBytes;
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
