@@ -62,11 +62,11 @@ NCU_TRAFFIC = {
     ("quantize_k", "large-b3"): 64 * (67_329_280 + 1_720_064),
     ("quantize_v", "large-b3"): 64 * (67_229_696 + 2_305_536),
     ("logits", "sweep-b3"): 2 * (234_967_296 + 16_118_528),   # logits_fast_kernel<2, 1>, 4-sequence capture x 2
-    ("attend_v", "sweep-b3"): 2 * (234_913_280 + 5_718_528),  # attend_fast_kernel<3, 1, 0>, 4-sequence capture x 2
+    ("attend_v", "sweep-b3"): 2 * (234_991_616 + 3_727_616),  # attend_fast_kernel<3, 1, 0>, 4-sequence capture x 2
     # the large-model layer's scan and softmax.V: the 4-sequence b-sweep captures (4 194 304 keys, one query
     # head per KV head, the same kernels) scaled by the keys processed (x 4)
     ("logits", "large-b3"): 4 * (234_967_296 + 16_118_528),
-    ("attend_v", "large-b3"): 4 * (234_913_280 + 5_718_528),
+    ("attend_v", "large-b3"): 4 * (234_991_616 + 3_727_616),
     ("logits", "llama"): 15_756_288 + 0,               # logits_gqa_kernel<2, 4> (the scan; tables read from L2)
     ("decode_attend", "sweep-b3"): 2 * (453_062_656 + 5_392_640),   # decode_fused_kernel<2, 3>, 4-sequence capture x 2
     ("decode_attend", "large-b3"): 4 * (453_062_656 + 5_392_640),   # the same capture scaled by the tokens (x 4)
