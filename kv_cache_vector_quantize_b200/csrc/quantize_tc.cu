@@ -25,8 +25,8 @@
 //   - one MMA thread: for tile i, D1 = x Pi^T (two products); then, keys, the
 //     sketch product of tile i - 1, D2 = E M^T, with E (the split residual) read
 //     from tensor memory;
-//   - 8 epilogue warps (mixed rate: 16), NP = 2 (4) per tensor-memory lane
-//     quarter, splitting the 128 columns into NP parts (NP threads per token):
+//   - 16 epilogue warps, 4 per tensor-memory lane quarter, splitting the 128
+//     columns into 4 parts of 32 (4 threads per token):
 //     D1 -> ||x|| (the token's threads add their parts' squares through shared
 //     memory) -> codes -> record words;
 //     keys also write the residual parts into tensor memory (two E buffers, so
@@ -44,9 +44,9 @@
 // Shared-memory operand tiles use the 128-byte swizzle K-major layout of tc.cuh (sw128_off).
 //
 // Mixed rate (MIXED: fractional bits per channel, the first 64 rotated
-// coordinates at BITS + 1 code bits): the epilogue thread of columns [0, 64)
-// searches the wider codebook and writes its 64 (BITS+1)-bit codes first, the
-// thread of columns [64, 128) the BITS-bit codebook and codes after them; the
+// coordinates at BITS + 1 code bits): the epilogue threads of columns [0, 64)
+// search the wider codebook and write their 64 (BITS+1)-bit codes first, the
+// threads of columns [64, 128) the BITS-bit codebook and codes after them; the
 // products are the same.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -103,35 +103,33 @@ struct H16 {
   }
 };
 
-// Epilogue threads per token (NP parts of kTD / NP columns): 4 for the mixed rate and for values with
-// 4-bit codes, whose code search is longest (values at b = 4: 10% faster), 2 otherwise (4 measured up to
-// 26% slower for 2-bit value codes and for keys).
-template <bool QJL, int BITS, bool MIXED>
-constexpr int epi_parts() { return (MIXED || (!QJL && BITS >= 4)) ? 4 : 2; }
-// Keys with 2- and 3-bit codes: 4 sign warps (one per lane quarter, a whole token per thread) turn D2
-// into sign words and rho, so the epilogue warps run only the first epilogue (measured: 3-bit codes
-// 16% faster, 2-bit codes 1-2%, 1-bit codes 3% slower, so those keep one epilogue loop); the mixed
-// rate's 16 epilogue warps do both (no registers left for more warps).
+// Keys with 2- and 3-bit codes at the integer rate: 4 sign warps (one per lane quarter, a whole token per
+// thread) turn D2 into sign words and rho, so the epilogue warps run only the first epilogue (measured:
+// 3-bit codes 16% faster, 2-bit codes 1-2%, 1-bit codes 3% slower, so those keep one epilogue loop); the
+// mixed rate's epilogue warps do both (measured 6% faster than with sign warps at 2 + 3 bits).
 template <bool QJL, int BITS, bool MIXED>
 constexpr bool epi_split() { return QJL && !MIXED && BITS >= 2; }
+// The 2-bit mixed-rate keys issue each K step's descriptors afresh, one step at a time: measured 4.10 ms
+// per 16.8 M keys against 4.46 ms with the precomputed descriptors of the other widths.
+template <bool QJL, int BITS, bool MIXED>
+constexpr bool mma_paced() { return QJL && MIXED && BITS >= 2; }
 
-template <bool QJL, int NP, bool SPLIT>
+// Four epilogue threads per token (parts of kTD / 4 columns), four warps per tensor-memory lane quarter:
+// measured against two threads per token, keys 15-20% faster (the residual's tensor-memory stores and
+// its split wait less), values 3% (2-bit codes) to 10% (4-bit codes).
+template <bool QJL, bool SPLIT>
 struct Ws {
-  static constexpr int kParts = NP;                      // epilogue threads per token
-  static constexpr int kEpiWarps = 4 * NP;               // NP warps per tensor-memory lane quarter
+  static constexpr int kParts = 4;                       // epilogue threads per token
+  static constexpr int kEpiWarps = 4 * kParts;
   static constexpr bool kSplit = SPLIT;
   static constexpr int kSignWarps = kSplit ? 4 : 0;
   static constexpr int kTmaWarp = kEpiWarps + kSignWarps;
   static constexpr int kMmaWarp = kTmaWarp + 1;
-  static constexpr int kThreads = 32 * (kMmaWarp + 1);   // 320 (168 registers), 448 (128) or 576 (96)
+  static constexpr int kThreads = 32 * (kMmaWarp + 1);   // 576 (96 registers) or, with sign warps, 704 (80)
   static constexpr int kNX = QJL ? 2 : 4;                // A-tile stages (tensor-map copies in flight)
-  // values with two threads per token: Pi_hi and Pi_lo stacked as one 256-row B tile, so one N = 256
-  // product per K step gives both parts (summed by the epilogue), with two D1 buffers; keys, and values
-  // with four threads per token (NP = 4: the mixed rate, 4-bit codes; their 16 epilogue warps then skip
-  // that sum, 21% faster at 3.5 bits, slower for 2-bit codes): two N = 128 products accumulated into one
-  // D1 (two buffers for values)
+  // D1 = x Pi_hi^T + x Pi_lo^T: two N = 128 products accumulated into one buffer (keys: one buffer,
+  // values: two, so a tile's products run while the epilogue reads the previous one)
   static constexpr int kND1 = QJL ? 1 : 2;
-  static constexpr int kPW = (QJL || NP == 4) ? 128 : 256;
   // dynamic shared memory, byte offsets
   static constexpr uint32_t kPhi = 0, kPlo = kTile;
   static constexpr uint32_t kMhi = 2 * kTile, kMlo = 3 * kTile;              // keys only
@@ -144,7 +142,7 @@ struct Ws {
   static constexpr int kBars = 4 + 4 + 2 + 2 + 1 + 1 + 1 + 3;
   static constexpr uint32_t kTslot = kBar + 8 * kBars;
   static constexpr uint32_t kBytes = kTslot + 16;
-  static constexpr uint32_t kTmemCols = 512;   // keys: D1, D2, E[0], E[1]; values: D1[0], D1[1] (kPW each)
+  static constexpr uint32_t kTmemCols = QJL ? 512 : 256;   // keys: D1, D2, E[0], E[1]; values: D1[0], D1[1]
   static constexpr uint32_t kD2 = 128, kE = 256;   // tensor-memory column offsets (keys)
   static_assert(kBytes <= 232448, "shared memory over the per-CTA limit");
 };
@@ -204,7 +202,7 @@ struct TileCursor {
 // contiguous 128-byte block); every thread issues all of its loads before
 // converting, so the L2 round trips overlap instead of serialising.
 // src must be 16-byte aligned.
-template <int NTHREADS, bool F16, bool STACKED = false>
+template <int NTHREADS, bool F16>
 __device__ __forceinline__ void load_split(unsigned char *hi, unsigned char *lo, const float *__restrict__ src) {
   constexpr int kChunks = kTD * kTD / 8;                       // 2048
   constexpr int kPer = (kChunks + NTHREADS - 1) / NTHREADS;
@@ -227,11 +225,9 @@ __device__ __forceinline__ void load_split(unsigned char *hi, unsigned char *lo,
 #pragma unroll
       for (int qq = 0; qq < 4; ++qq) H16<F16>::split2(f[2 * qq], f[2 * qq + 1], hw[qq], lw[qq]);
       const int n = e & 127, k = 8 * (e >> 7);
-      // STACKED: one 256-row tile at `hi`, rows [0, 128) the hi parts, [128, 256) the lo parts
-      const uint32_t oh = STACKED ? tc::sw128_off(2 * kTT, n, k) : tc::sw128_off(kTT, n, k);
-      const uint32_t ol = STACKED ? tc::sw128_off(2 * kTT, n + kTT, k) : tc::sw128_off(kTT, n, k);
-      *reinterpret_cast<uint4 *>(hi + oh) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4 *>((STACKED ? hi : lo) + ol) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      const uint32_t o = tc::sw128_off(kTT, n, k);
+      *reinterpret_cast<uint4 *>(hi + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4 *>(lo + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
   }
 }
@@ -480,28 +476,51 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b,
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// The MMA thread builds each operand's shared-memory descriptor once per product and steps it along K by
+// adding the step's byte offset / 16 to the start-address field (the field cannot carry: shared
+// addresses stay below 256 KB), so a K step costs one add instead of a descriptor build. PACED: the
+// descriptors are built at each step, a loop of one step per iteration.
+
 // The 8 K-steps of one split product D (+)= A B^T with A in tensor memory (64 columns).
+template <bool PACED>
 __device__ __forceinline__ void mma_tile_ts(uint32_t d, uint32_t a_tmem, uint32_t b, uint32_t idesc,
                                             bool accumulate_first) {
+  if constexpr (PACED) {
 #pragma unroll 1
-  for (int s = 0; s < 8; ++s)
-    mma_bf16_ts(d, a_tmem + 8 * s, tc::smem_desc_sw128(tc::sw128_kstep(b, kTT, s)), idesc,
-                (accumulate_first || s) ? 1u : 0u);
+    for (int s = 0; s < 8; ++s)
+      mma_bf16_ts(d, a_tmem + 8 * s, tc::smem_desc_sw128(tc::sw128_kstep(b, kTT, s)), idesc,
+                  (accumulate_first || s) ? 1u : 0u);
+  } else {
+    const uint64_t db = tc::smem_desc_sw128(b);
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+      mma_bf16_ts(d, a_tmem + 8 * s, db + (tc::sw128_kstep(0, kTT, s) >> 4), idesc,
+                  (accumulate_first || s) ? 1u : 0u);
+  }
 }
 
 // Issue the 8 K-steps of one split product D (+)= A B^T (A, B: 128 x 128 bf16 tiles).
-__device__ __forceinline__ void mma_tile(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc, bool accumulate_first,
-                                         int rows_b = kTT) {
+template <bool PACED>
+__device__ __forceinline__ void mma_tile(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc, bool accumulate_first) {
+  if constexpr (PACED) {
 #pragma unroll 1
-  for (int s = 0; s < 8; ++s)
-    tc::mma_bf16(d, tc::smem_desc_sw128(tc::sw128_kstep(a, kTT, s)), tc::smem_desc_sw128(tc::sw128_kstep(b, rows_b, s)),
-                 idesc, (accumulate_first || s) ? 1u : 0u);
+    for (int s = 0; s < 8; ++s)
+      tc::mma_bf16(d, tc::smem_desc_sw128(tc::sw128_kstep(a, kTT, s)), tc::smem_desc_sw128(tc::sw128_kstep(b, kTT, s)),
+                   idesc, (accumulate_first || s) ? 1u : 0u);
+  } else {
+    const uint64_t da = tc::smem_desc_sw128(a), db = tc::smem_desc_sw128(b);
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+      tc::mma_bf16(d, da + (tc::sw128_kstep(0, kTT, s) >> 4), db + (tc::sw128_kstep(0, kTT, s) >> 4), idesc,
+                   (accumulate_first || s) ? 1u : 0u);
+  }
 }
 
 template <bool QJL, int BITS, bool F16, bool MIXED = false>
-__global__ void __launch_bounds__(Ws<QJL, epi_parts<QJL, BITS, MIXED>(), epi_split<QJL, BITS, MIXED>()>::kThreads, 1)
+__global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThreads, 1)
     quantize_tc_kernel(const QuantParams p, const __grid_constant__ CUtensorMap xmap) {
-  using L = Ws<QJL, epi_parts<QJL, BITS, MIXED>(), epi_split<QJL, BITS, MIXED>()>;
+  using L = Ws<QJL, epi_split<QJL, BITS, MIXED>()>;
+  constexpr bool kPaced = mma_paced<QJL, BITS, MIXED>();
   constexpr int kParts = L::kParts;
   constexpr int kEpiWarps = L::kEpiWarps;
   constexpr int CPT = kTD / kParts;               // columns per epilogue thread
@@ -521,7 +540,7 @@ __global__ void __launch_bounds__(Ws<QJL, epi_parts<QJL, BITS, MIXED>(), epi_spl
   auto row0_of = [&](int i) -> int64_t { return ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * kTT; };
 
   // ---- set-up: split matrices, codebook, barriers, tensor memory ----
-  load_split<L::kThreads, F16, L::kPW == 256>(smem + L::kPhi, smem + L::kPlo, p.Pi);
+  load_split<L::kThreads, F16>(smem + L::kPhi, smem + L::kPlo, p.Pi);
   if constexpr (QJL) load_split<L::kThreads, F16>(smem + L::kMhi, smem + L::kMlo, p.SPiT);
   if (tid < NL + (MIXED ? NLM : 0)) cb[tid] = p.codebook[tid];
   if (tid == 0) {
@@ -619,16 +638,15 @@ __global__ void __launch_bounds__(Ws<QJL, epi_parts<QJL, BITS, MIXED>(), epi_spl
     // ----------------------------- MMA issuer ------------------------------
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16(kTT, kTD, !F16);
-      const uint32_t idesc_w = tc::idesc_bf16(kTT, L::kPW, !F16);
       int last_pi = -1, last_sk = -1;
       auto sketch = [&](int j) -> bool {   // D2 = E_hi M_hi^T + E_hi M_lo^T + E_lo M_hi^T
         if (!mbar_wait(bar.e_full(), j & 1)) return false;
         if (j >= 1 && !mbar_wait(bar.d2_empty(), (j - 1) & 1)) return false;
         tc::fence_after();
         const uint32_t d2 = tmem + L::kD2, e = tmem + L::kE + 128 * (j & 1);
-        mma_tile_ts(d2, e, sbase + L::kMhi, idesc, false);
-        mma_tile_ts(d2, e, sbase + L::kMlo, idesc, true);
-        mma_tile_ts(d2, e + 64, sbase + L::kMhi, idesc, true);
+        mma_tile_ts<kPaced>(d2, e, sbase + L::kMhi, idesc, false);
+        mma_tile_ts<kPaced>(d2, e, sbase + L::kMlo, idesc, true);
+        mma_tile_ts<kPaced>(d2, e + 64, sbase + L::kMhi, idesc, true);
         tc::commit(bar.d2_full());
         last_sk = j;
         return true;
@@ -643,12 +661,8 @@ __global__ void __launch_bounds__(Ws<QJL, epi_parts<QJL, BITS, MIXED>(), epi_spl
         }
         tc::fence_after();
         const uint32_t xa = sbase + L::kX + xs * kTile;
-        if constexpr (L::kPW == 256) {
-          mma_tile(tmem + 256 * db, xa, sbase + L::kPhi, idesc_w, false, 2 * kTT);
-        } else {
-          mma_tile(tmem + 128 * db, xa, sbase + L::kPhi, idesc, false);
-          mma_tile(tmem + 128 * db, xa, sbase + L::kPlo, idesc, true);
-        }
+        mma_tile<kPaced>(tmem + 128 * db, xa, sbase + L::kPhi, idesc, false);
+        mma_tile<kPaced>(tmem + 128 * db, xa, sbase + L::kPlo, idesc, true);
         tc::commit(bar.x_empty(xs));
         tc::commit(bar.d1_full(db));
         last_pi = i;
@@ -704,21 +718,10 @@ __global__ void __launch_bounds__(Ws<QJL, epi_parts<QJL, BITS, MIXED>(), epi_spl
         const bool have = __all_sync(0xffffffffu, ok && mbar_wait(bar.d1_full(db), (i / L::kND1) & 1));
         if (have) {
           tc::fence_after();
-          const uint32_t d1 = tmem + lane_ofs + (L::kPW == 256 ? 256 : 128) * db + CPT * h;
+          const uint32_t d1 = tmem + lane_ofs + 128 * db + CPT * h;
 #pragma unroll
           for (int c = 0; c < CPT / 32; ++c) tc::ld32(d1 + 32 * c, *reinterpret_cast<uint32_t (*)[32]>(r + 32 * c));
           tc::wait_ld();
-          if constexpr (L::kPW == 256) {
-            // the lo-part product sits 128 columns to the right: D1 = x Pi_hi^T + x Pi_lo^T
-#pragma unroll
-            for (int c = 0; c < CPT / 32; ++c) {
-              uint32_t lo[32];
-              tc::ld32(d1 + 128 + 32 * c, lo);
-              tc::wait_ld();
-#pragma unroll
-              for (int q = 0; q < 32; ++q) r[32 * c + q] = __float_as_uint(__uint_as_float(r[32 * c + q]) + __uint_as_float(lo[q]));
-            }
-          }
           tc::fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar.d1_empty(db));   // D1 may take the next tile's product
@@ -878,7 +881,7 @@ cudaError_t launch_tc(const QuantParams &p, cudaStream_t st) {
   CUtensorMap xmap;
   if (p.rows >= (int64_t)1 << 31 || !make_x_map(&xmap, p, F16)) return cudaErrorNotSupported;
   auto kern = quantize_tc_kernel<QJL, BITS, F16, MIXED>;
-  using L = Ws<QJL, epi_parts<QJL, BITS, MIXED>(), epi_split<QJL, BITS, MIXED>()>;
+  using L = Ws<QJL, epi_split<QJL, BITS, MIXED>()>;
   constexpr size_t smem = L::kBytes;
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), smem);
   if (e != cudaSuccess) return e;
