@@ -329,6 +329,25 @@ __device__ __forceinline__ bool mbar_wait_n(uint32_t bar, uint32_t parity, uint3
 // Waits for the phase with the given parity to complete; false after kSpinLimit tries.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) { return mbar_wait_n(bar, parity, kSpinLimit); }
 
+// As mbar_wait, for waits that overlap other warps' work: each try may suspend the thread for up to
+// kSleepHintNs (it resumes as soon as the phase completes), so a waiting warp takes few issue slots
+// from the warps that share its scheduler. Bounded by kSleepLimit tries: at most about 2 s when every
+// try sleeps its full hint, at least 2^21 tries when the hardware resumes earlier.
+constexpr uint32_t kSleepHintNs = 1000;
+constexpr uint32_t kSleepLimit = 1u << 21;
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kSleepLimit; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity), "n"(kSleepHintNs)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
 // 1-D bulk copy global -> shared, completion counted on `bar` (bytes % 16 == 0,
 // both addresses 16-byte aligned).
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {

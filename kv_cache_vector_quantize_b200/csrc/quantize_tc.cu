@@ -258,6 +258,19 @@ __device__ __forceinline__ float bsel(uint32_t m, float a, float b) {
 // word |= bit at `pos` when m is all ones (the bit is known to be clear)
 __device__ __forceinline__ void put_bit(uint32_t &word, uint32_t m, int pos) { word += m * (0u - (1u << pos)); }
 
+// Sign word of the 32 sketch values v[o, o + 32): bit k = (v[o + k] >= 0). The values' sign bits are
+// shifted in from the top, one funnel shift each, and the word inverted: that is v >= 0 for every value
+// but -0.0, which it reads as negative. The product gives an exact zero only for a zero residual (a
+// zero vector); the caller sets that token's words to all ones, as the sign of 0 is +1.
+template <int O, int N>
+__device__ __forceinline__ uint32_t sign_word(const uint32_t (&v)[N]) {
+  static_assert(O + 32 <= N, "32 values from offset O");
+  uint32_t w = 0u;
+#pragma unroll
+  for (int k = 31; k >= 0; --k) w = __funnelshift_l(v[O + k], w, 1);
+  return ~w;
+}
+
 // m[k] = all ones iff bit k of code = #{j : y > th[j]} is set (ascending
 // thresholds th[0 .. 2^BITS - 2]): a binary search, top bit first.
 template <int BITS>
@@ -602,7 +615,8 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
       const int64_t slot = valid ? cur.slot(p, t) : 0;
       cur.advance(p);
       // the tensor-memory loads are warp-wide: the whole warp loads or none of it does
-      if (!__all_sync(0xffffffffu, mbar_wait(bar.rho_full(j % 3), (j / 3) & 1) && mbar_wait(bar.d2_full(), j & 1)))
+      if (!__all_sync(0xffffffffu, mbar_wait_sleep(bar.rho_full(j % 3), (j / 3) & 1) &&
+                                       mbar_wait_sleep(bar.d2_full(), j & 1)))
         break;
       tc::fence_after();
       uint32_t sw[4];
@@ -612,6 +626,7 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
         tc::ld32(tmem + lane_ofs + L::kD2 + 64 * hh, *reinterpret_cast<uint32_t (*)[32]>(r));
         tc::ld32(tmem + lane_ofs + L::kD2 + 64 * hh + 32, *reinterpret_cast<uint32_t (*)[32]>(r + 32));
         tc::wait_ld();
+        // (the sign words by compare and multiply-add: sign_word's shift chain spills here at 80 registers)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           sw[2 * hh + c] = 0u;
@@ -715,7 +730,7 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
         const int db = i % L::kND1;
         uint32_t r[CPT];
         // the tensor-memory loads are warp-wide: the whole warp loads or none of it does
-        const bool have = __all_sync(0xffffffffu, ok && mbar_wait(bar.d1_full(db), (i / L::kND1) & 1));
+        const bool have = __all_sync(0xffffffffu, ok && mbar_wait_sleep(bar.d1_full(db), (i / L::kND1) & 1));
         if (have) {
           tc::fence_after();
           const uint32_t d1 = tmem + lane_ofs + 128 * db + CPT * h;
@@ -808,10 +823,9 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
         if (i >= 1) {
           // ---- second epilogue of tile i - 1: sign words and ||e|| ----
           const int j = i - 1;
-          uint32_t sw[CPT / 32];
-#pragma unroll
-          for (int c = 0; c < CPT / 32; ++c) sw[c] = 0u;
-          if (__all_sync(0xffffffffu, ok && mbar_wait(bar.d2_full(), j & 1))) {
+          static_assert(CPT == 32, "one sign word per epilogue thread");
+          uint32_t sw[1] = {0u};
+          if (__all_sync(0xffffffffu, ok && mbar_wait_sleep(bar.d2_full(), j & 1))) {
             tc::fence_after();
             uint32_t r[CPT];
 #pragma unroll
@@ -821,25 +835,19 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
             tc::fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar.d2_empty());
-#pragma unroll
-            for (int c = 0; c < CPT / 32; ++c)
-#pragma unroll
-              for (int qq = 0; qq < 32; ++qq) put_bit(sw[c], ge0(__uint_as_float(r[32 * c + qq])), qq);
+            sw[0] = sign_word<0>(r);
           } else {
             ok = false;
           }
           // the token's barrier (warps q + 4 h): every part's sum of e^2 for tile j is visible
           asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "n"(32 * kParts) : "memory");
           if (ok && vprev) {
-            uint32_t *sdst = p.records + slot_prev * RW + IW + (CPT / 32) * h;
-            if constexpr (CPT == 64) st_global_v2(sdst, sw[0], sw[CPT / 32 - 1]);
-            else sdst[0] = sw[0];
-            if (h == 0) {
-              float e2s = 0.f;
+            float e2s = 0.f;
 #pragma unroll
-              for (int k = 0; k < kParts; ++k) e2s += rho[((j % 3) * kParts + k) * 128 + t];
-              p.rnorm[slot_prev] = sqrtf(e2s);
-            }
+            for (int k = 0; k < kParts; ++k) e2s += rho[((j % 3) * kParts + k) * 128 + t];
+            if (e2s == 0.f) sw[0] = ~0u;   // a zero residual: every sign +1
+            p.records[slot_prev * RW + IW + h] = sw[0];
+            if (h == 0) p.rnorm[slot_prev] = sqrtf(e2s);
           }
         }
         slot_prev = slot;
