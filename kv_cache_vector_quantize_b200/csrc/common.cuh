@@ -86,6 +86,7 @@ struct QuantParams {
   int idx_words;
   int n_hi;                 // mixed rate: leading coordinates at bits + 1 code bits (0: integer rate)
   const float *signs;       // structured rotation Pi = H diag(signs) / sqrt(d) (then Pi is unused), or NULL
+  uint32_t *tiles;          // tensor-core quantizer: [2] zeroed tile-schedule counters (NULL: a fixed tile order)
 };
 
 struct LogitsParams {
@@ -244,6 +245,8 @@ bool nn_supported(int d, int bits);
 int nn_kp(int d);                   // padded K of a query row (fp16 elements)
 cudaError_t launch_nn_search(const NnArgs &a, cudaStream_t st);
 int device_sm_count();
+// A pair of zeroed tile-schedule counters for a quantizer launch on `st` (tq_api.cu), or NULL.
+uint32_t *tile_counters(cudaStream_t st);
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device).
 cudaError_t set_smem_once(const void *kernel, size_t bytes);
 size_t device_smem_optin();

@@ -19,8 +19,10 @@
 // split's error moves it by about 2^-17 / sqrt(d) of ||x||, far inside the 1e-5
 // tolerance, and no warp has to read the tile a second time.
 //
-// Warp roles (one persistent CTA per SM, 128-token tiles):
-//   - one copy thread: tensor-map copies of x straight into a ring of A tiles
+// Warp roles (one persistent CTA per SM, 128-token tiles taken from a
+// per-launch counter, so that a CTA on a slower SM takes fewer of them):
+//   - one copy thread: takes the next tile, publishes it to the other roles
+//     and copies its x rows by tensor map straight into a ring of A tiles
 //     in shared memory (2 for keys, 4 for values), in the 128-byte swizzle layout;
 //   - one MMA thread: for tile i, D1 = x Pi^T (two products); then, keys, the
 //     sketch product of tile i - 1, D2 = E M^T, with E (the split residual) read
@@ -103,6 +105,18 @@ struct H16 {
   }
 };
 
+// Tile schedule. The copy thread takes the CTA's tiles one at a time, from a per-launch counter when
+// QuantParams::tiles is set (dynamic: a CTA on a slower SM simply takes fewer tiles) or else as
+// blockIdx.x + i gridDim.x, and publishes each as entry i of a ring in shared memory: the tile's first row
+// and its position in the (sequence x head, token) grid, row0 = sh n_tokens + tt with 0 <= tt < n_tokens,
+// or row0 = -1 after the last tile. The other roles read entry i when they start tile i. The ring has
+// kRingN entries: no role is more than 6 tiles behind the copy thread (the input stages, the D1 and D2
+// hand-offs and the two E buffers bound the lead), so an entry is never overwritten before all have read it.
+constexpr int kRingN = 16;
+struct TileSlot {
+  int64_t row0, sh, tt;
+};
+
 // Keys with 2- and 3-bit codes at the integer rate: 4 sign warps (one per lane quarter, a whole token per
 // thread) turn D2 into sign words and rho, so the epilogue warps run only the first epilogue (measured:
 // 3-bit codes 16% faster, 2-bit codes 1-2%, 1-bit codes 3% slower, so those keep one epilogue loop); the
@@ -137,9 +151,10 @@ struct Ws {
   static constexpr uint32_t kRho = kX + kNX * kTile;                         // float[3][kParts][128] (keys)
   static constexpr uint32_t kXch = kRho + (QJL ? 3 * kParts * 128 * 4 : 0);  // float2[2][kParts][128]: ||x|| parts
   static constexpr uint32_t kCb = kXch + 2 * kParts * 128 * 8;               // float[32] centroids (two codebooks if mixed)
-  static constexpr uint32_t kBar = kCb + 128;
-  // barriers: x_full[4], x_empty[4], d1_full[2], d1_empty[2], e_full, d2_full, d2_empty, rho_full[3]
-  static constexpr int kBars = 4 + 4 + 2 + 2 + 1 + 1 + 1 + 3;
+  static constexpr uint32_t kRing = kCb + 128;                               // TileSlot[kRingN]: the tile schedule
+  static constexpr uint32_t kBar = kRing + kRingN * sizeof(TileSlot);
+  // barriers: x_full[4], x_empty[4], d1_full[2], d1_empty[2], e_full, d2_full, d2_empty, rho_full[3], slot_full[kRingN]
+  static constexpr int kBars = 4 + 4 + 2 + 2 + 1 + 1 + 1 + 3 + kRingN;
   static constexpr uint32_t kTslot = kBar + 8 * kBars;
   static constexpr uint32_t kBytes = kTslot + 16;
   static constexpr uint32_t kTmemCols = QJL ? 512 : 256;   // keys: D1, D2, E[0], E[1]; values: D1[0], D1[1]
@@ -159,42 +174,18 @@ struct Bars {
   __device__ uint32_t d2_full() const { return base + 8u * 13; }
   __device__ uint32_t d2_empty() const { return base + 8u * 14; }
   __device__ uint32_t rho_full(int k) const { return base + 8u * (15 + k); }   // rho of tile i in slot i % 3
+  __device__ uint32_t slot_full(int k) const { return base + 8u * (18 + k); }  // schedule entry i in slot i % kRingN
 };
 
-// Position of a CTA's current tile in the (sequence x head, token) grid, kept
-// incrementally so that the tile loop needs no 64-bit division: row0 =
-// sh * n_tokens + tt with 0 <= tt < n_tokens; the persistent CTA advances by
-// gridDim.x tiles = step_q * n_tokens + step_r rows.
-struct TileCursor {
-  int64_t sh, tt, step_q, step_r, base;   // base = slot of the tile's first row
-  __device__ void init(const QuantParams &p) {
-    const int64_t row0 = (int64_t)blockIdx.x * 128, step = (int64_t)gridDim.x * 128;
-    sh = row0 / p.n_tokens;
-    tt = row0 - sh * p.n_tokens;
-    step_q = step / p.n_tokens;
-    step_r = step - step_q * p.n_tokens;
-    base = sh * p.capacity + p.pos + tt;
+// Cache slot of row r of a tile whose first row is (sh, tt).
+__device__ __forceinline__ int64_t tile_row_slot(const QuantParams &p, const TileSlot &ts, int r) {
+  int64_t t2 = ts.tt + r, s2 = ts.sh;
+  while (t2 >= p.n_tokens) {
+    t2 -= p.n_tokens;
+    ++s2;
   }
-  __device__ void advance(const QuantParams &p) {
-    tt += step_r;
-    sh += step_q;
-    if (tt >= p.n_tokens) {
-      tt -= p.n_tokens;
-      ++sh;
-    }
-    base = sh * p.capacity + p.pos + tt;
-  }
-  // cache slot of tile row r
-  __device__ int64_t slot(const QuantParams &p, int r) const {
-    if (tt + r < p.n_tokens) return base + r;   // the row is in the tile's first (sequence, head)
-    int64_t t2 = tt + r, s2 = sh;
-    while (t2 >= p.n_tokens) {
-      t2 -= p.n_tokens;
-      ++s2;
-    }
-    return s2 * p.capacity + p.pos + t2;
-  }
-};
+  return s2 * p.capacity + p.pos + t2;
+}
 
 // Split float32 matrix rows into hi/lo bf16 operand tiles (rows = output coordinates).
 // A work item is one 16-byte row chunk (8 consecutive k of one row;
@@ -549,8 +540,18 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
   const Bars<QJL> bar{sbase + L::kBar};
   float *cb = reinterpret_cast<float *>(smem + L::kCb);
   const int64_t n_tiles = (p.rows + kTT - 1) / kTT;
-  const int n_my = n_tiles > blockIdx.x ? (int)((n_tiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
-  auto row0_of = [&](int i) -> int64_t { return ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * kTT; };
+  TileSlot *ring = reinterpret_cast<TileSlot *>(smem + L::kRing);
+  // schedule entry i (row0 = -1: no more tiles, also after a failed wait)
+  auto take = [&](int i) -> TileSlot {
+    TileSlot ts{-1, 0, 0};
+    if (mbar_wait(bar.slot_full(i % kRingN), (i / kRingN) & 1)) {
+      const volatile TileSlot *e = ring + i % kRingN;
+      ts.row0 = e->row0;
+      ts.sh = e->sh;
+      ts.tt = e->tt;
+    }
+    return ts;
+  };
 
   // ---- set-up: split matrices, codebook, barriers, tensor memory ----
   load_split<L::kThreads, F16>(smem + L::kPhi, smem + L::kPlo, p.Pi);
@@ -569,6 +570,7 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
     mbar_init(bar.d2_full(), 1);
     mbar_init(bar.d2_empty(), L::kSplit ? L::kSignWarps : kEpiWarps);
     for (int k = 0; k < 3; ++k) mbar_init(bar.rho_full(k), kEpiWarps);
+    for (int k = 0; k < kRingN; ++k) mbar_init(bar.slot_full(k), 1);   // the copy thread's arrive
     mbar_fence_init();
   }
   if (warp == 0) {
@@ -587,15 +589,29 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
       int issued = 0;
-      for (int i = 0; i < n_my; ++i) {
+      // the next tile's ticket is drawn one tile ahead, so the atomic's round trip overlaps the copies
+      int64_t ticket = p.tiles ? (int64_t)atomicAdd(p.tiles, 1u) : (int64_t)blockIdx.x;
+      for (int i = 0;; ++i) {
+        const int64_t tile = ticket < n_tiles ? ticket : -1;
         const int s = i % L::kNX;
         // A tile s is free once tile i - kNX's first product is done
-        if (i >= L::kNX && !mbar_wait(bar.x_empty(s), ((i / L::kNX) - 1) & 1)) break;
+        const bool go = tile >= 0 && (i < L::kNX || mbar_wait(bar.x_empty(s), ((i / L::kNX) - 1) & 1));
+        TileSlot *e = ring + i % kRingN;
+        if (go) {
+          const int64_t row0 = tile * kTT, sh = row0 / p.n_tokens;
+          e->row0 = row0;
+          e->sh = sh;
+          e->tt = row0 - sh * p.n_tokens;
+          ticket = p.tiles ? (int64_t)atomicAdd(p.tiles, 1u) : ticket + gridDim.x;
+        } else {
+          e->row0 = -1;
+        }
+        mbar_arrive(bar.slot_full(i % kRingN));   // release: the entry is visible to whoever waits on it
+        if (!go) break;
         mbar_arrive_expect_tx(bar.x_full(s), kTile);
         const uint32_t dst = sbase + L::kX + s * kTile;
-        const int row0 = (int)row0_of(i);
 #pragma unroll 1
-        for (int kb = 0; kb < 2; ++kb) tma_x_chunk(dst + kb * (kTile / 2), &xmap, 64 * kb, row0, bar.x_full(s));
+        for (int kb = 0; kb < 2; ++kb) tma_x_chunk(dst + kb * (kTile / 2), &xmap, 64 * kb, (int)e->row0, bar.x_full(s));
         ++issued;
       }
       // no copy may still be landing when the CTA exits
@@ -608,12 +624,11 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
     const int q = warp & 3, t = 32 * q + lane;
     const uint32_t lane_ofs = (uint32_t)(32 * q) << 16;
     const float *rho = reinterpret_cast<const float *>(smem + L::kRho);   // [3][kParts][128]
-    TileCursor cur;
-    cur.init(p);
-    for (int j = 0; j < n_my; ++j) {
-      const bool valid = row0_of(j) + t < p.rows;
-      const int64_t slot = valid ? cur.slot(p, t) : 0;
-      cur.advance(p);
+    for (int j = 0;; ++j) {
+      const TileSlot ts = take(j);   // the same entry for the whole warp (a failed wait: row0 = -1 for all)
+      if (!__all_sync(0xffffffffu, ts.row0 >= 0)) break;
+      const bool valid = ts.row0 + t < p.rows;
+      const int64_t slot = valid ? tile_row_slot(p, ts, t) : 0;
       // the tensor-memory loads are warp-wide: the whole warp loads or none of it does
       if (!__all_sync(0xffffffffu, mbar_wait_sleep(bar.rho_full(j % 3), (j / 3) & 1) &&
                                        mbar_wait_sleep(bar.d2_full(), j & 1)))
@@ -666,7 +681,9 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
         last_sk = j;
         return true;
       };
-      for (int i = 0; i < n_my && ok; ++i) {
+      int n_my = 0;
+      for (int i = 0; ok; ++i) {
+        if (take(i).row0 < 0) break;
         const int xs = i % L::kNX;
         const int db = i % L::kND1;
         if (!mbar_wait(bar.x_full(xs), (i / L::kNX) & 1) ||
@@ -681,6 +698,7 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
         tc::commit(bar.x_empty(xs));
         tc::commit(bar.d1_full(db));
         last_pi = i;
+        n_my = i + 1;
         if constexpr (QJL)
           if (i >= 1) ok = sketch(i - 1);
       }
@@ -713,20 +731,21 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
     int64_t slot_prev = 0;
     bool vprev = false;
     float2 *xch = reinterpret_cast<float2 *>(smem + L::kXch);   // [2][kParts][128]: ||x|| parts, by tile parity
-    TileCursor cur;
-    cur.init(p);
-
-    // Every epilogue thread runs all n_my + 1 iterations (after a failed wait it
-    // skips the work but still meets the token's barriers of each iteration).
-    for (int i = 0; i <= n_my; ++i) {
+    // The token's threads (warps q + 4 h) run the same iterations: whether tile i exists is agreed on
+    // at their named barrier (an AND over the group, so a failed wait in one warp ends the loop for all),
+    // and after a failed D1 wait a thread skips the work but still meets the token's barriers.
+    for (int i = 0;; ++i) {
       float e2 = 0.f;
       int64_t slot = 0;
       bool valid = false;
-      if (i < n_my) {
+      const TileSlot ts = take(i);
+      uint32_t more;
+      asm volatile("{\n .reg .pred p, r;\n setp.ge.s64 p, %1, 0;\n bar.red.and.pred r, %2, %3, p;\n selp.u32 %0, 1, 0, r;\n}"
+                   : "=r"(more) : "l"(ts.row0), "r"(1 + q), "n"(32 * kParts) : "memory");
+      if (more) {
         // ---- first epilogue of tile i: ||x||, codes (and, keys, the residual into E[i & 1]) ----
-        valid = row0_of(i) + t < p.rows;
-        slot = valid ? cur.slot(p, t) : 0;
-        cur.advance(p);
+        valid = ts.row0 + t < p.rows;
+        slot = valid ? tile_row_slot(p, ts, t) : 0;
         const int db = i % L::kND1;
         uint32_t r[CPT];
         // the tensor-memory loads are warp-wide: the whole warp loads or none of it does
@@ -853,6 +872,7 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
         slot_prev = slot;
         vprev = valid;
       }
+      if (!more) break;
     }
   }
 
@@ -860,6 +880,15 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
   tc::fence_before();
   __syncthreads();
   if (warp == 0) tc::dealloc(tmem, L::kTmemCols);
+  // every ticket of this CTA was drawn before the barrier above; the last CTA to finish zeroes the counter
+  // for the next launch on the stream
+  if (p.tiles && tid == 0) {
+    __threadfence();
+    if (atomicAdd(p.tiles + 1, 1u) == gridDim.x - 1) {
+      atomicExch(p.tiles, 0u);
+      atomicExch(p.tiles + 1, 0u);
+    }
+  }
 }
 
 // The x rows as a 2-D tensor map: 128 16-bit elements per row, `rows` rows of 256 bytes; a
@@ -896,7 +925,9 @@ cudaError_t launch_tc(const QuantParams &p, cudaStream_t st) {
   const int64_t tiles = (p.rows + kTT - 1) / kTT;
   const int64_t slots = (int64_t)device_sm_count();
   const int grid = (int)(tiles < slots ? tiles : slots);
-  return launch_after(kern, dim3(grid), dim3(L::kThreads), smem, st, p, xmap);
+  QuantParams q = p;
+  q.tiles = tiles > grid ? tile_counters(st) : nullptr;   // one tile per CTA needs no schedule
+  return launch_after(kern, dim3(grid), dim3(L::kThreads), smem, st, q, xmap);
 }
 
 template <bool F16>

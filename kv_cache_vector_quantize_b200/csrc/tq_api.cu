@@ -5,6 +5,8 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
+#include <unordered_map>
 
 #include "common.cuh"
 
@@ -140,6 +142,61 @@ constexpr int kAttendMaxQ = 4;
 }  // namespace
 
 uint32_t debug_stall_tries() { return g_stall_tries.load(); }
+
+// Tile-schedule counters of the tensor-core quantizer. Per device a pool of counter pairs: one pair per
+// stream (keyed by the stream's unique id, so launches that share a pair are stream-ordered) and a pair
+// of its own for every launch recorded into a graph. A pair is zeroed by a stream-ordered memset when
+// it is handed out, and the launch's last CTA zeroes it again. NULL (the kernel then takes its tiles in
+// a fixed order) when the pool is used up, or when a graph is being recorded before the pool exists.
+namespace {
+constexpr int kTilePairs = 1024;
+struct TilePool {
+  uint32_t *base = nullptr;
+  int used = 0;
+  std::unordered_map<unsigned long long, int> by_stream;
+};
+TilePool g_tile_pool[kMaxDevices];
+std::mutex g_tile_mu;
+}  // namespace
+
+uint32_t *tile_counters(cudaStream_t st) {
+  const int dev = current_device();
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  const bool capturing = cs != cudaStreamCaptureStatusNone;
+  std::lock_guard<std::mutex> lock(g_tile_mu);
+  TilePool &tp = g_tile_pool[dev];
+  if (!tp.base) {
+    if (capturing) return nullptr;
+    void *b = nullptr;
+    if (cudaMalloc(&b, kTilePairs * 2 * sizeof(uint32_t)) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    tp.base = static_cast<uint32_t *>(b);
+  }
+  unsigned long long id = 0;
+  if (!capturing) {
+    if (cudaStreamGetId(st, &id) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    auto it = tp.by_stream.find(id);
+    if (it != tp.by_stream.end()) return tp.base + 2 * it->second;
+  }
+  if (tp.used == kTilePairs) return nullptr;
+  uint32_t *c = tp.base + 2 * tp.used;
+  if (cudaMemsetAsync(c, 0, 2 * sizeof(uint32_t), st) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (!capturing) tp.by_stream.emplace(id, tp.used);
+  ++tp.used;
+  return c;
+}
 
 int device_sm_count() {
   const int dev = current_device();
