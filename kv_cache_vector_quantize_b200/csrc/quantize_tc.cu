@@ -19,9 +19,9 @@
 // split's error moves it by about 2^-17 / sqrt(d) of ||x||, far inside the 1e-5
 // tolerance, and no warp has to read the tile a second time.
 //
-// Warp roles (one persistent CTA per SM, 128-token tiles taken from a
-// per-launch counter, so that a CTA on a slower SM takes fewer of them):
-//   - one copy thread: takes the next tile, publishes it to the other roles
+// Warp roles (one persistent CTA per SM, 128-token tiles; keys take them from
+// a per-launch counter, so that a CTA on a slower SM takes fewer of them):
+//   - one copy thread: takes the next tile (keys: publishes it to the other roles)
 //     and copies its x rows by tensor map straight into a ring of A tiles
 //     in shared memory (2 for keys, 4 for values), in the 128-byte swizzle layout;
 //   - one MMA thread: for tile i, D1 = x Pi^T (two products); then, keys, the
@@ -105,13 +105,15 @@ struct H16 {
   }
 };
 
-// Tile schedule. The copy thread takes the CTA's tiles one at a time, from a per-launch counter when
-// QuantParams::tiles is set (dynamic: a CTA on a slower SM simply takes fewer tiles) or else as
+// Tile schedule of the keys. The copy thread takes the CTA's tiles one at a time, from a per-launch counter
+// when QuantParams::tiles is set (dynamic: a CTA on a slower SM simply takes fewer tiles) or else as
 // blockIdx.x + i gridDim.x, and publishes each as entry i of a ring in shared memory: the tile's first row
 // and its position in the (sequence x head, token) grid, row0 = sh n_tokens + tt with 0 <= tt < n_tokens,
 // or row0 = -1 after the last tile. The other roles read entry i when they start tile i. The ring has
 // kRingN entries: no role is more than 6 tiles behind the copy thread (the input stages, the D1 and D2
 // hand-offs and the two E buffers bound the lead), so an entry is never overwritten before all have read it.
+// Measured on the large-model layer's fresh inputs: keys 2.92 -> 2.80 ms; values, whose per-CTA times
+// hardly differ, 1.78 -> 1.83 ms, so they keep the fixed order (blockIdx.x + i gridDim.x) and no ring.
 constexpr int kRingN = 16;
 struct TileSlot {
   int64_t row0, sh, tt;
@@ -175,6 +177,40 @@ struct Bars {
   __device__ uint32_t d2_empty() const { return base + 8u * 14; }
   __device__ uint32_t rho_full(int k) const { return base + 8u * (15 + k); }   // rho of tile i in slot i % 3
   __device__ uint32_t slot_full(int k) const { return base + 8u * (18 + k); }  // schedule entry i in slot i % kRingN
+};
+
+// Position of a CTA's current tile in the fixed order (values), kept incrementally so that the tile loop
+// needs no 64-bit division: row0 = sh * n_tokens + tt with 0 <= tt < n_tokens; the persistent CTA
+// advances by gridDim.x tiles = step_q * n_tokens + step_r rows.
+struct TileCursor {
+  int64_t sh, tt, step_q, step_r, base;   // base = slot of the tile's first row
+  __device__ void init(const QuantParams &p) {
+    const int64_t row0 = (int64_t)blockIdx.x * 128, step = (int64_t)gridDim.x * 128;
+    sh = row0 / p.n_tokens;
+    tt = row0 - sh * p.n_tokens;
+    step_q = step / p.n_tokens;
+    step_r = step - step_q * p.n_tokens;
+    base = sh * p.capacity + p.pos + tt;
+  }
+  __device__ void advance(const QuantParams &p) {
+    tt += step_r;
+    sh += step_q;
+    if (tt >= p.n_tokens) {
+      tt -= p.n_tokens;
+      ++sh;
+    }
+    base = sh * p.capacity + p.pos + tt;
+  }
+  // cache slot of tile row r
+  __device__ int64_t slot(const QuantParams &p, int r) const {
+    if (tt + r < p.n_tokens) return base + r;   // the row is in the tile's first (sequence, head)
+    int64_t t2 = tt + r, s2 = sh;
+    while (t2 >= p.n_tokens) {
+      t2 -= p.n_tokens;
+      ++s2;
+    }
+    return s2 * p.capacity + p.pos + t2;
+  }
 };
 
 // Cache slot of row r of a tile whose first row is (sh, tt).
@@ -540,6 +576,9 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
   const Bars<QJL> bar{sbase + L::kBar};
   float *cb = reinterpret_cast<float *>(smem + L::kCb);
   const int64_t n_tiles = (p.rows + kTT - 1) / kTT;
+  constexpr bool kSched = QJL;   // keys: the tile schedule through the ring; values: the fixed order
+  const int n_fixed = n_tiles > blockIdx.x ? (int)((n_tiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+  auto row0_of = [&](int i) -> int64_t { return ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * kTT; };
   TileSlot *ring = reinterpret_cast<TileSlot *>(smem + L::kRing);
   // schedule entry i (row0 = -1: no more tiles, also after a failed wait)
   auto take = [&](int i) -> TileSlot {
@@ -589,30 +628,44 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
       int issued = 0;
-      // the next tile's ticket is drawn one tile ahead, so the atomic's round trip overlaps the copies
-      int64_t ticket = p.tiles ? (int64_t)atomicAdd(p.tiles, 1u) : (int64_t)blockIdx.x;
-      for (int i = 0;; ++i) {
-        const int64_t tile = ticket < n_tiles ? ticket : -1;
-        const int s = i % L::kNX;
-        // A tile s is free once tile i - kNX's first product is done
-        const bool go = tile >= 0 && (i < L::kNX || mbar_wait(bar.x_empty(s), ((i / L::kNX) - 1) & 1));
-        TileSlot *e = ring + i % kRingN;
-        if (go) {
-          const int64_t row0 = tile * kTT, sh = row0 / p.n_tokens;
-          e->row0 = row0;
-          e->sh = sh;
-          e->tt = row0 - sh * p.n_tokens;
-          ticket = p.tiles ? (int64_t)atomicAdd(p.tiles, 1u) : ticket + gridDim.x;
-        } else {
-          e->row0 = -1;
-        }
-        mbar_arrive(bar.slot_full(i % kRingN));   // release: the entry is visible to whoever waits on it
-        if (!go) break;
-        mbar_arrive_expect_tx(bar.x_full(s), kTile);
-        const uint32_t dst = sbase + L::kX + s * kTile;
+      if constexpr (kSched) {
+        // the next tile's ticket is drawn one tile ahead, so the atomic's round trip overlaps the copies
+        int64_t ticket = p.tiles ? (int64_t)atomicAdd(p.tiles, 1u) : (int64_t)blockIdx.x;
+        for (int i = 0;; ++i) {
+          const int64_t tile = ticket < n_tiles ? ticket : -1;
+          const int s = i % L::kNX;
+          // A tile s is free once tile i - kNX's first product is done
+          const bool go = tile >= 0 && (i < L::kNX || mbar_wait(bar.x_empty(s), ((i / L::kNX) - 1) & 1));
+          TileSlot *e = ring + i % kRingN;
+          if (go) {
+            const int64_t row0 = tile * kTT, sh = row0 / p.n_tokens;
+            e->row0 = row0;
+            e->sh = sh;
+            e->tt = row0 - sh * p.n_tokens;
+            ticket = p.tiles ? (int64_t)atomicAdd(p.tiles, 1u) : ticket + gridDim.x;
+          } else {
+            e->row0 = -1;
+          }
+          mbar_arrive(bar.slot_full(i % kRingN));   // release: the entry is visible to whoever waits on it
+          if (!go) break;
+          mbar_arrive_expect_tx(bar.x_full(s), kTile);
+          const uint32_t dst = sbase + L::kX + s * kTile;
 #pragma unroll 1
-        for (int kb = 0; kb < 2; ++kb) tma_x_chunk(dst + kb * (kTile / 2), &xmap, 64 * kb, (int)e->row0, bar.x_full(s));
-        ++issued;
+          for (int kb = 0; kb < 2; ++kb) tma_x_chunk(dst + kb * (kTile / 2), &xmap, 64 * kb, (int)e->row0, bar.x_full(s));
+          ++issued;
+        }
+      } else {
+        for (int i = 0; i < n_fixed; ++i) {
+          const int s = i % L::kNX;
+          // A tile s is free once tile i - kNX's first product is done
+          if (i >= L::kNX && !mbar_wait(bar.x_empty(s), ((i / L::kNX) - 1) & 1)) break;
+          mbar_arrive_expect_tx(bar.x_full(s), kTile);
+          const uint32_t dst = sbase + L::kX + s * kTile;
+          const int row0 = (int)row0_of(i);
+#pragma unroll 1
+          for (int kb = 0; kb < 2; ++kb) tma_x_chunk(dst + kb * (kTile / 2), &xmap, 64 * kb, row0, bar.x_full(s));
+          ++issued;
+        }
       }
       // no copy may still be landing when the CTA exits
       for (int i = max(0, issued - L::kNX); i < issued; ++i) mbar_wait(bar.x_full(i % L::kNX), (i / L::kNX) & 1);
@@ -683,7 +736,11 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
       };
       int n_my = 0;
       for (int i = 0; ok; ++i) {
-        if (take(i).row0 < 0) break;
+        if constexpr (kSched) {
+          if (take(i).row0 < 0) break;
+        } else {
+          if (i >= n_fixed) break;
+        }
         const int xs = i % L::kNX;
         const int db = i % L::kND1;
         if (!mbar_wait(bar.x_full(xs), (i / L::kNX) & 1) ||
@@ -731,21 +788,34 @@ __global__ void __launch_bounds__(Ws<QJL, epi_split<QJL, BITS, MIXED>()>::kThrea
     int64_t slot_prev = 0;
     bool vprev = false;
     float2 *xch = reinterpret_cast<float2 *>(smem + L::kXch);   // [2][kParts][128]: ||x|| parts, by tile parity
-    // The token's threads (warps q + 4 h) run the same iterations: whether tile i exists is agreed on
-    // at their named barrier (an AND over the group, so a failed wait in one warp ends the loop for all),
-    // and after a failed D1 wait a thread skips the work but still meets the token's barriers.
+    TileCursor cur;   // the fixed order (values)
+    if constexpr (!kSched) cur.init(p);
+    // The token's threads (warps q + 4 h) run the same iterations: keys agree on whether tile i exists at
+    // their named barrier (an AND over the group, so a failed wait in one warp ends the loop for all), values
+    // run n_fixed + 1; after a failed D1 wait a thread skips the work but still meets the token's barriers.
     for (int i = 0;; ++i) {
       float e2 = 0.f;
       int64_t slot = 0;
       bool valid = false;
-      const TileSlot ts = take(i);
       uint32_t more;
-      asm volatile("{\n .reg .pred p, r;\n setp.ge.s64 p, %1, 0;\n bar.red.and.pred r, %2, %3, p;\n selp.u32 %0, 1, 0, r;\n}"
-                   : "=r"(more) : "l"(ts.row0), "r"(1 + q), "n"(32 * kParts) : "memory");
+      TileSlot ts{-1, 0, 0};
+      if constexpr (kSched) {
+        ts = take(i);
+        asm volatile("{\n .reg .pred p, r;\n setp.ge.s64 p, %1, 0;\n bar.red.and.pred r, %2, %3, p;\n selp.u32 %0, 1, 0, r;\n}"
+                     : "=r"(more) : "l"(ts.row0), "r"(1 + q), "n"(32 * kParts) : "memory");
+      } else {
+        more = i < n_fixed;
+      }
       if (more) {
         // ---- first epilogue of tile i: ||x||, codes (and, keys, the residual into E[i & 1]) ----
-        valid = ts.row0 + t < p.rows;
-        slot = valid ? tile_row_slot(p, ts, t) : 0;
+        if constexpr (kSched) {
+          valid = ts.row0 + t < p.rows;
+          slot = valid ? tile_row_slot(p, ts, t) : 0;
+        } else {
+          valid = row0_of(i) + t < p.rows;
+          slot = valid ? cur.slot(p, t) : 0;
+          cur.advance(p);
+        }
         const int db = i % L::kND1;
         uint32_t r[CPT];
         // the tensor-memory loads are warp-wide: the whole warp loads or none of it does
@@ -926,7 +996,7 @@ cudaError_t launch_tc(const QuantParams &p, cudaStream_t st) {
   const int64_t slots = (int64_t)device_sm_count();
   const int grid = (int)(tiles < slots ? tiles : slots);
   QuantParams q = p;
-  q.tiles = tiles > grid ? tile_counters(st) : nullptr;   // one tile per CTA needs no schedule
+  q.tiles = QJL && tiles > grid ? tile_counters(st) : nullptr;   // keys only; one tile per CTA needs no schedule
   return launch_after(kern, dim3(grid), dim3(L::kThreads), smem, st, q, xmap);
 }
 

@@ -1,11 +1,12 @@
-"""The tensor-core quantizer's dynamic tile schedule: streams, repeats and graphs.
+"""The tensor-core quantizer's tile schedule: streams, repeats and graphs.
 
-Its CTAs take 128-token tiles from a counter that the library hands out per stream (and per
-launch recorded into a graph), and the launch's last CTA zeroes it again. Which CTA encodes a
-tile does not change the encoding, so every launch must give the records, norms and rnorms of
-the first one bit for bit: back-to-back launches on one stream (the counter is reset between
-them), launches on four streams at once (each with its own counter) and a graph's replays.
-The first launch is checked against the float64 oracle on sampled tokens.
+For keys its CTAs take 128-token tiles from a counter that the library hands out per stream
+(and per launch recorded into a graph), and the launch's last CTA zeroes it again; values take
+their tiles in a fixed order. Which CTA encodes a tile does not change the encoding, so every
+launch must give the records, norms and rnorms of the first one bit for bit: back-to-back
+launches on one stream (the counter is reset between them), launches on four streams at once
+(each with its own counter) and a graph's replays. The first launch is checked against the
+float64 oracle on sampled tokens.
 """
 
 from __future__ import annotations
