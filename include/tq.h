@@ -19,9 +19,14 @@
  *
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller unless the
- *     comment says "host". The library never allocates device memory; scratch
- *     space is a caller-provided workspace whose size a *_workspace_size call
- *     returns.
+ *     comment says "host". Scratch space is a caller-provided workspace whose
+ *     size a *_workspace_size call returns. The library's one allocation is
+ *     8 KB of tile-schedule counters per device and CUDA context, made by the
+ *     first tq_quantize_append of keys that runs on the tensor cores (a
+ *     cudaMalloc: make that call before recording graphs; a call recorded
+ *     before it takes its tiles in a fixed order instead, with the same
+ *     result). A stream's first such call, and each such call recorded into a
+ *     graph, enqueues an 8-byte memset on the stream.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and is asynchronous: no entry point synchronises the stream,
  *     except tq_workspace_status and tq_attend_v_noalloc_status, which say so.

@@ -1,6 +1,8 @@
 // C ABI entry points (include/tq.h): host-side argument checks, workspace
 // carving, launch configuration and status reporting. Every compute step runs
 // in the kernels of quantize.cu, logits.cu and attend.cu.
+#include <cuda.h>
+
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -143,20 +145,46 @@ constexpr int kAttendMaxQ = 4;
 
 uint32_t debug_stall_tries() { return g_stall_tries.load(); }
 
-// Tile-schedule counters of the tensor-core quantizer. Per device a pool of counter pairs: one pair per
+// Tile-schedule counters of the tensor-core key quantizer. Per device and CUDA context a pool of counter
+// pairs (8 KB, allocated by the first call that needs it; the library's one allocation): one pair per
 // stream (keyed by the stream's unique id, so launches that share a pair are stream-ordered) and a pair
 // of its own for every launch recorded into a graph. A pair is zeroed by a stream-ordered memset when
 // it is handed out, and the launch's last CTA zeroes it again. NULL (the kernel then takes its tiles in
-// a fixed order) when the pool is used up, or when a graph is being recorded before the pool exists.
+// a fixed order) when the pool is used up, when a graph is being recorded before the pool exists, or when
+// the context cannot be identified. A new context (after cudaDeviceReset) gets a new pool: the old
+// pool's memory went with the old context.
 namespace {
 constexpr int kTilePairs = 1024;
 struct TilePool {
+  unsigned long long ctx_id = 0;
   uint32_t *base = nullptr;
   int used = 0;
   std::unordered_map<unsigned long long, int> by_stream;
 };
 TilePool g_tile_pool[kMaxDevices];
 std::mutex g_tile_mu;
+
+typedef CUresult (*PfnCtxGetCurrent)(CUcontext *);
+typedef CUresult (*PfnCtxGetId)(CUcontext, unsigned long long *);
+
+// Id of the calling thread's current context (unique for the life of the process, unlike the handle).
+bool current_ctx_id(unsigned long long *id) {
+  static PfnCtxGetCurrent get_current = nullptr;
+  static PfnCtxGetId get_id = nullptr;
+  if (!get_current || !get_id) {
+    void *f1 = nullptr, *f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess || !f1 ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess || !f2) {
+      cudaGetLastError();
+      return false;
+    }
+    get_current = reinterpret_cast<PfnCtxGetCurrent>(f1);
+    get_id = reinterpret_cast<PfnCtxGetId>(f2);
+  }
+  CUcontext ctx = nullptr;
+  return get_current(&ctx) == CUDA_SUCCESS && ctx != nullptr && get_id(ctx, id) == CUDA_SUCCESS;
+}
 }  // namespace
 
 uint32_t *tile_counters(cudaStream_t st) {
@@ -167,15 +195,19 @@ uint32_t *tile_counters(cudaStream_t st) {
     return nullptr;
   }
   const bool capturing = cs != cudaStreamCaptureStatusNone;
+  unsigned long long ctx_id = 0;
+  if (!current_ctx_id(&ctx_id)) return nullptr;
   std::lock_guard<std::mutex> lock(g_tile_mu);
   TilePool &tp = g_tile_pool[dev];
-  if (!tp.base) {
+  if (!tp.base || tp.ctx_id != ctx_id) {
     if (capturing) return nullptr;
     void *b = nullptr;
     if (cudaMalloc(&b, kTilePairs * 2 * sizeof(uint32_t)) != cudaSuccess) {
       cudaGetLastError();
       return nullptr;
     }
+    tp = TilePool{};
+    tp.ctx_id = ctx_id;
     tp.base = static_cast<uint32_t *>(b);
   }
   unsigned long long id = 0;

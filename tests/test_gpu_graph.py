@@ -1,9 +1,10 @@
 """The path replayed from CUDA graphs: every call is stream-ordered and capturable.
 
 A serving loop captures its per-token work once and replays it; the library's calls make no host
-synchronisation and allocate nothing, and their kernels' programmatic-dependent launches are captured
-as graph edges. Captured once after a warm-up call (which also sets the kernels' shared-memory
-attributes), each graph is replayed several times and must give the eager call's result bit for bit:
+synchronisation and, after the first key quantize call, allocate nothing, and their kernels'
+programmatic-dependent launches are captured as graph edges. Captured once after a warm-up call
+(which also sets the kernels' shared-memory attributes), each graph is replayed several times and
+must give the eager call's result bit for bit:
 the one-call decode step for one and for four query heads per KV head, and quantize-append + logits +
 softmax.V as one graph.
 """
